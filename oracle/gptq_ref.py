@@ -1,0 +1,340 @@
+"""Plain float64 CPU oracle for GPTQ's per-layer solve (test infrastructure).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke`` and the
+benchmark's CPU-baseline leg may import this module.  It shares no code, table
+or helper with the CUDA library; the two meet only at the seeded inputs of the
+``synth`` package.
+
+Every step follows the description on the source pages, cited by page title
+and section:
+
+* [Tutorial]  "GPTQ：一键量化大模型压缩" (aiqz.cc) -- sections 二阶信息 (Hessian
+  H = 2 sum x x^T), 逐层量化 (layer objective ||W X - W^ X||_F^2), 误差补偿
+  (OBS compensation delta_F = (q - w_q)/[H^-1]_qq [H^-1]_{F,q}), 分组方案
+  (scale = (max - min)/(2^b - 1), zero = -min/scale, group-wise parameters).
+* [Survey]    "LLM 量化技术" blog (astro-blog, llm-quantization-techniques) --
+  §1.2 量化原理 (x_q = round(x/s + z), dequantised s(x_q - z)), §2.2 OBQ
+  (the OBS update of the remaining weights), §2.3 items 1-3 (fixed column
+  order, blocks of B = 128 columns, Cholesky for the needed rows of H^-1).
+* [Card]      "GPTQ: Accurate Post-Training Quantization for Generative
+  Pre-trained Transformers" reading card -- section 方法适配 (any fixed order,
+  lazy batch of B = 128 columns with the global update deferred to the end of
+  the block, Cholesky reformulation with mild damping).
+* [Explainer] "一文读懂GPTQ" (mcipr.com) -- section 三 (int32 packing of 3/4-bit
+  codes, group_size, desc_act).
+
+Readings where the pages are silent or garbled (each one is listed in the
+design notes):
+
+* q in the compensation equation is the quantised value, so the remaining
+  columns move by -(w_j - w^_j)/U_jj * U[j, j+1:] with U the upper Cholesky
+  factor of H^-1 (the sign of the [Survey] §2.2 update).
+* The error form "tr(dW^T H^-1 dW)" printed on two pages is garbled; the
+  objective is ||(W - W^) X^T||_F^2 = 1/2 tr(dW H dW^T) with H = 2 X^T X.
+* Damping adds lambda = damp * mean(diag H) to the diagonal.
+* Quantiser: integer zero point.  xmin = min(0, min x), xmax = max(0, max x),
+  s = (xmax - xmin)/(2^b - 1) (s = 1 when xmax == xmin), z = rint(-xmin/s),
+  q = clip(rint(w/s) + z, 0, 2^b - 1), w^ = s (q - z).  rint rounds half to
+  even.
+* Group parameters are taken from the current (compensated) W when the sweep
+  reaches a group's first column; with group = -1 they come from the original
+  row.
+* Act-order: stable argsort of -diag(H) (ties keep the lower index); groups
+  are formed over permuted positions and g_idx maps original columns to them.
+* Packing: per row, codes form an LSB-first bit stream along the input
+  dimension, 32 bits per int32 word; 3-bit codes straddle words.
+
+Parity status: every function here is pinned by tests under ``tests/``
+(closed forms, invariants, special cases and brute force); none is unpinned.
+"""
+
+from __future__ import annotations
+
+import itertools
+
+import numpy as np
+
+F64 = np.float64
+
+
+# ---------------------------------------------------------------------------
+# Hessian  ([Tutorial] §二阶信息: H = 2 * sum_i x_i x_i^T)
+# ---------------------------------------------------------------------------
+
+def hessian(X: np.ndarray, chunk: int = 8192) -> np.ndarray:
+    """H = 2 * sum_t x_t x_t^T in float64 for X [n x d] (rows are tokens).
+
+    fp16 inputs are exact in float64; the sum over tokens is taken in chunks of
+    ``chunk`` rows with a float64 matrix product per chunk.
+    """
+    X = np.asarray(X)
+    n, d = X.shape
+    H = np.zeros((d, d), dtype=F64)
+    for t0 in range(0, n, chunk):
+        Xc = X[t0:t0 + chunk].astype(F64)
+        H += Xc.T @ Xc
+    return 2.0 * H
+
+
+def hessian_rows(X: np.ndarray, rows: np.ndarray, chunk: int = 8192) -> np.ndarray:
+    """Rows ``rows`` of H = 2 X^T X in float64, without forming all of H."""
+    X = np.asarray(X)
+    n, d = X.shape
+    rows = np.asarray(rows, dtype=np.int64)
+    out = np.zeros((rows.size, d), dtype=F64)
+    for t0 in range(0, n, chunk):
+        Xc = X[t0:t0 + chunk].astype(F64)
+        out += Xc[:, rows].T @ Xc
+    return 2.0 * out
+
+
+# ---------------------------------------------------------------------------
+# Damping, act-order, inverse-Hessian factor  ([Card] 方法适配; [Survey] §2.3)
+# ---------------------------------------------------------------------------
+
+def dampen(H: np.ndarray, damp: float) -> tuple[np.ndarray, float]:
+    """H_d = H + lambda I with lambda = damp * mean(diag H)."""
+    H = np.asarray(H, dtype=F64)
+    lam = float(damp) * float(np.mean(np.diag(H)))
+    Hd = H.copy()
+    Hd[np.diag_indices_from(Hd)] += lam
+    return Hd, lam
+
+
+def act_order_perm(H: np.ndarray) -> np.ndarray:
+    """Quantisation order: columns by descending diag(H), ties by lower index."""
+    return np.argsort(-np.diag(np.asarray(H, dtype=F64)), kind="stable")
+
+
+def inverse_upper_cholesky(Hd: np.ndarray) -> np.ndarray:
+    """U upper triangular with positive diagonal and U^T U = Hd^-1.
+
+    Plain definition: invert, then take the Cholesky factor of the inverse
+    (numpy returns the lower factor L with Hd^-1 = L L^T; U = L^T).
+    """
+    Hinv = np.linalg.inv(np.asarray(Hd, dtype=F64))
+    L = np.linalg.cholesky(Hinv)
+    return np.ascontiguousarray(L.T)
+
+
+# ---------------------------------------------------------------------------
+# Asymmetric min-max quantiser  ([Tutorial] §分组方案; [Survey] §1.2)
+# ---------------------------------------------------------------------------
+
+def quant_params(x: np.ndarray, bits: int) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row (scale, zero) of x [rows x cols] (float64 in, float64 out)."""
+    x = np.asarray(x, dtype=F64)
+    maxq = (1 << bits) - 1
+    xmin = np.minimum(x.min(axis=1), 0.0)
+    xmax = np.maximum(x.max(axis=1), 0.0)
+    flat = xmax == xmin
+    s = np.where(flat, 1.0, (xmax - xmin) / maxq)
+    z = np.rint(-xmin / s)
+    return s, z
+
+
+def quantize(w: np.ndarray, s: np.ndarray, z: np.ndarray, bits: int) -> np.ndarray:
+    """Integer code clip(rint(w/s) + z, 0, 2^b - 1) (float64 holding integers)."""
+    maxq = (1 << bits) - 1
+    return np.clip(np.rint(np.asarray(w, dtype=F64) / s) + z, 0, maxq)
+
+
+def dequantize(q: np.ndarray, s: np.ndarray, z: np.ndarray) -> np.ndarray:
+    """w^ = s (q - z)."""
+    return s * (q - z)
+
+
+def rtn(W: np.ndarray, bits: int, group: int) -> tuple[np.ndarray, np.ndarray]:
+    """Round-to-nearest baseline: same quantiser, parameters from W, no compensation.
+
+    Returns (codes int64 [r x d], W^ float64 [r x d]).
+    """
+    W = np.asarray(W, dtype=F64)
+    r, d = W.shape
+    g = d if group == -1 else group
+    codes = np.zeros((r, d), dtype=np.int64)
+    What = np.zeros((r, d), dtype=F64)
+    for c0 in range(0, d, g):
+        blk = W[:, c0:c0 + g]
+        s, z = quant_params(blk, bits)
+        q = quantize(blk, s[:, None], z[:, None], bits)
+        codes[:, c0:c0 + g] = q.astype(np.int64)
+        What[:, c0:c0 + g] = dequantize(q, s[:, None], z[:, None])
+    return codes, What
+
+
+# ---------------------------------------------------------------------------
+# Column sweep with OBS compensation and lazy batches
+# ([Tutorial] §误差补偿; [Survey] §2.2, §2.3; [Card] 方法适配)
+# ---------------------------------------------------------------------------
+
+def _check_groups(d: int, group: int, block: int) -> None:
+    if group == -1:
+        return
+    if group <= 0 or d % group:
+        raise ValueError("group must be -1 or a positive divisor of d")
+    if block < d and not (block % group == 0 or group % block == 0):
+        # A group that straddles a block end would read columns whose deferred
+        # update has not been applied yet; the lazy form is then not exact.
+        raise ValueError("lazy batches need block % group == 0 or group % block == 0")
+
+
+def gptq_sweep(W: np.ndarray, U: np.ndarray, bits: int, group: int, block: int):
+    """Quantise W [r x d] column by column in fixed order.
+
+    At column j: q = quantize(w_j), e_j = (w_j - w^_j)/U_jj, and the columns
+    after j move by -e_j * U[j, j+1:].  Inside a block of ``block`` columns the
+    move is applied at once; the move of the columns after the block is
+    deferred to the block's end as one product E_blk @ U[blk, end:] (the lazy
+    batch).  ``block >= d`` is the plain unblocked loop.
+
+    Returns (codes int64, scales, zeros (float64 holding integers), W^ float64,
+    E float64 [r x d] with E[:, j] = e_j).
+    """
+    W = np.array(W, dtype=F64, copy=True)
+    U = np.asarray(U, dtype=F64)
+    r, d = W.shape
+    _check_groups(d, group, block)
+    G = 1 if group == -1 else d // group
+    codes = np.zeros((r, d), dtype=np.int64)
+    scales = np.zeros((r, G), dtype=F64)
+    zeros = np.zeros((r, G), dtype=F64)
+    E = np.zeros((r, d), dtype=F64)
+    if group == -1:
+        s, z = quant_params(W, bits)
+        scales[:, 0], zeros[:, 0] = s, z
+    for b0 in range(0, d, block):
+        b1 = min(d, b0 + block)
+        for j in range(b0, b1):
+            if group != -1 and j % group == 0:
+                s, z = quant_params(W[:, j:j + group], bits)
+                scales[:, j // group], zeros[:, j // group] = s, z
+            w = W[:, j]
+            q = quantize(w, s, z, bits)
+            wq = dequantize(q, s, z)
+            e = (w - wq) / U[j, j]
+            codes[:, j] = q.astype(np.int64)
+            E[:, j] = e
+            W[:, j] = wq
+            if j + 1 < b1:
+                W[:, j + 1:b1] -= np.outer(e, U[j, j + 1:b1])
+        if b1 < d:
+            W[:, b1:] -= E[:, b0:b1] @ U[b0:b1, b1:]
+    return codes, scales, zeros, W, E
+
+
+# ---------------------------------------------------------------------------
+# Layer objective  ([Tutorial] §逐层量化)
+# ---------------------------------------------------------------------------
+
+def layer_loss(W: np.ndarray, What: np.ndarray, H: np.ndarray) -> float:
+    """||(W - W^) X^T||_F^2 written through H = 2 X^T X: 1/2 tr(D H D^T)."""
+    D = np.asarray(W, dtype=F64) - np.asarray(What, dtype=F64)
+    return 0.5 * float(np.sum((D @ np.asarray(H, dtype=F64)) * D))
+
+
+def layer_loss_direct(W: np.ndarray, What: np.ndarray, X: np.ndarray) -> float:
+    """||W X^T - W^ X^T||_F^2 straight from the activations (X [n x d])."""
+    D = np.asarray(W, dtype=F64) - np.asarray(What, dtype=F64)
+    Y = D @ np.asarray(X, dtype=F64).T
+    return float(np.sum(Y * Y))
+
+
+# ---------------------------------------------------------------------------
+# The whole layer
+# ---------------------------------------------------------------------------
+
+def gptq_quantize_layer(W: np.ndarray, H: np.ndarray, *, bits: int, group: int,
+                        block: int = 128, damp: float = 0.01,
+                        act_order: bool = False, rows: np.ndarray | None = None) -> dict:
+    """Damp, order, factor, sweep, score and unpermute one layer.
+
+    ``rows`` restricts the sweep to a subset of output rows (rows are
+    independent once U is fixed), for checks at full layer width.
+    """
+    W = np.asarray(W, dtype=F64)
+    H = np.asarray(H, dtype=F64)
+    if rows is not None:
+        W = W[np.asarray(rows)]
+    r, d = W.shape
+    Hd, lam = dampen(H, damp)
+    perm = act_order_perm(H) if act_order else np.arange(d)
+    inv = np.argsort(perm)
+    U = inverse_upper_cholesky(Hd[np.ix_(perm, perm)])
+    codes_p, scales, zeros, What_p, E = gptq_sweep(W[:, perm], U, bits, group, block)
+    codes = codes_p[:, inv]
+    What = What_p[:, inv]
+    g_idx = (inv // group) if group != -1 else np.zeros(d, dtype=np.int64)
+    return {
+        "codes": codes,
+        "scales": scales,
+        "zeros": zeros.astype(np.int64),
+        "g_idx": g_idx.astype(np.int64),
+        "What": What,
+        "loss": layer_loss(W, What, H),
+        "obs_sum": 0.5 * float(np.sum(E * E)),
+        "lambda": lam,
+        "perm": perm,
+        "U": U,
+        "E": E,
+    }
+
+
+# ---------------------------------------------------------------------------
+# Brute force for tiny rows (the grid is fixed by the row's own min/max)
+# ---------------------------------------------------------------------------
+
+def brute_force_min_loss(w: np.ndarray, H: np.ndarray, bits: int) -> float:
+    """min over every code vector of 1/2 (w - w^) H (w - w^)^T for one row.
+
+    The row's (s, z) come from its original values (group = -1), as in the
+    sweep, so every candidate lies on the same grid.  Only for tiny d.
+    """
+    w = np.asarray(w, dtype=F64).reshape(1, -1)
+    d = w.shape[1]
+    s, z = quant_params(w, bits)
+    levels = np.arange(1 << bits, dtype=F64)
+    cand = np.array(list(itertools.product(levels, repeat=d)), dtype=F64)
+    D = w - dequantize(cand, s[0], z[0])
+    return 0.5 * float(np.min(np.einsum("ij,jk,ik->i", D, np.asarray(H, dtype=F64), D)))
+
+
+# ---------------------------------------------------------------------------
+# int32 packing  ([Explainer] §三: 3/4-bit codes stored in 32-bit integers)
+# ---------------------------------------------------------------------------
+
+def pack_rows(codes: np.ndarray, bits: int) -> np.ndarray:
+    """Pack codes [r x d] into int32 [r x d*bits/32]: LSB-first bit stream per row.
+
+    Code c of a row occupies stream bits [c*bits, (c+1)*bits); stream bit k
+    is bit (k mod 32) of word k // 32.
+    """
+    codes = np.asarray(codes)
+    r, d = codes.shape
+    if (d * bits) % 32:
+        raise ValueError("d * bits must be a multiple of 32")
+    words = np.zeros((r, d * bits // 32), dtype=np.uint64)
+    for c in range(d):
+        pos = c * bits
+        wi, off = divmod(pos, 32)
+        v = codes[:, c].astype(np.uint64) << np.uint64(off)
+        words[:, wi] |= v & np.uint64(0xFFFFFFFF)
+        if off + bits > 32:
+            words[:, wi + 1] |= v >> np.uint64(32)
+    return words.astype(np.uint32).view(np.int32)
+
+
+def unpack_rows(words: np.ndarray, bits: int, d: int) -> np.ndarray:
+    """Inverse of ``pack_rows``: int32 [r x d*bits/32] -> codes int64 [r x d]."""
+    w = np.asarray(words).view(np.uint32).astype(np.uint64)
+    r = w.shape[0]
+    mask = np.uint64((1 << bits) - 1)
+    out = np.zeros((r, d), dtype=np.int64)
+    for c in range(d):
+        pos = c * bits
+        wi, off = divmod(pos, 32)
+        v = w[:, wi] >> np.uint64(off)
+        if off + bits > 32:
+            v |= w[:, wi + 1] << np.uint64(32 - off)
+        out[:, c] = (v & mask).astype(np.int64)
+    return out

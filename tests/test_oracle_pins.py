@@ -1,0 +1,334 @@
+"""Pins of the float64 oracle against facts other than itself.
+
+Each test checks the oracle against a closed form, an invariant of the
+mathematics, a special case that reduces to a textbook result, hand-worked
+fixtures under tests/golden/, or brute force on tiny inputs.  The sources are
+the GPTQ pages: "GPTQ：一键量化大模型压缩" (§二阶信息, §逐层量化, §误差补偿,
+§分组方案), the "LLM 量化技术" blog (§1.2, §2.2, §2.3), the GPTQ reading card
+(方法适配) and "一文读懂GPTQ" (§三, packing).
+"""
+
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from synth import make_problem
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- Hessian ---
+
+def test_hessian_identity_input_gives_2I():
+    # X = I: each token is one unit vector, so H = 2 * sum e_i e_i^T = 2 I.
+    d = 24
+    X = np.eye(d, dtype=np.float16)
+    np.testing.assert_array_equal(oracle.hessian(X), 2.0 * np.eye(d))
+
+
+def test_hessian_integer_brute_force():
+    # Tiny integer activations: every product and sum is an exact integer, so a
+    # Python-int triple loop gives the exact H to compare bit for bit.
+    rng = _rng(1)
+    n, d = 9, 5
+    Xi = rng.integers(-8, 9, size=(n, d))
+    exact = [[2 * sum(int(Xi[t, i]) * int(Xi[t, j]) for t in range(n)) for j in range(d)]
+             for i in range(d)]
+    np.testing.assert_array_equal(oracle.hessian(Xi.astype(np.float16)),
+                                  np.array(exact, dtype=np.float64))
+
+
+def test_hessian_quadratic_form_identity():
+    # ||X v||^2 = 1/2 v^T H v: fixes the factor 2 and which side is transposed.
+    X, _ = make_problem(4, 32, 300, seed=3)
+    H = oracle.hessian(X)
+    v = _rng(2).standard_normal(32)
+    lhs = float(np.sum((X.astype(np.float64) @ v) ** 2))
+    assert lhs == pytest.approx(0.5 * v @ H @ v, rel=1e-12)
+
+
+def test_hessian_chunking_and_rows():
+    X, _ = make_problem(4, 64, 20000, seed=4)
+    H = oracle.hessian(X, chunk=8192)
+    H1 = oracle.hessian(X, chunk=10 ** 9)
+    np.testing.assert_allclose(H, H1, rtol=1e-13, atol=1e-9)
+    rows = np.array([0, 7, 63])
+    np.testing.assert_allclose(oracle.hessian_rows(X, rows), H[rows], rtol=1e-13, atol=1e-9)
+    # symmetric positive semi-definite
+    np.testing.assert_array_equal(H, H.T)
+    assert np.linalg.eigvalsh(H).min() > -1e-9 * np.abs(H).max()
+
+
+# ------------------------------------------------- damping, order, factor ---
+
+def test_damping_trace_closed_form():
+    X, _ = make_problem(4, 48, 500, seed=5)
+    H = oracle.hessian(X)
+    Hd, lam = oracle.dampen(H, 0.01)
+    assert lam == pytest.approx(0.01 * np.trace(H) / 48, rel=1e-14)
+    assert np.trace(Hd) == pytest.approx(1.01 * np.trace(H), rel=1e-13)
+    off = ~np.eye(48, dtype=bool)
+    np.testing.assert_array_equal(Hd[off], H[off])
+
+
+def test_act_order_descending_stable():
+    H = np.diag([1.0, 3.0, 3.0, 2.0, 3.0])
+    np.testing.assert_array_equal(oracle.act_order_perm(H), [1, 2, 4, 3, 0])
+
+
+def test_inverse_upper_cholesky_2x2_closed_form():
+    # H = [[a, b], [b, c]]: H^-1 = [[c, -b], [-b, a]]/det, and the upper factor
+    # with U^T U = H^-1 is U11 = sqrt(c/det), U12 = -b/sqrt(c det), U22 = 1/sqrt(c).
+    a, b, c = 5.0, 2.0, 3.0
+    det = a * c - b * b
+    U = oracle.inverse_upper_cholesky(np.array([[a, b], [b, c]]))
+    expect = np.array([[np.sqrt(c / det), -b / np.sqrt(c * det)], [0.0, 1.0 / np.sqrt(c)]])
+    np.testing.assert_allclose(U, expect, rtol=1e-14)
+
+
+def test_inverse_upper_cholesky_diagonal_and_residual():
+    h = np.array([4.0, 9.0, 0.25, 16.0])
+    np.testing.assert_allclose(oracle.inverse_upper_cholesky(np.diag(h)),
+                               np.diag(1.0 / np.sqrt(h)), rtol=1e-15)
+    X, _ = make_problem(4, 96, 2000, seed=6)
+    Hd, _ = oracle.dampen(oracle.hessian(X), 0.01)
+    U = oracle.inverse_upper_cholesky(Hd)
+    assert np.all(np.tril(U, -1) == 0)
+    assert np.all(np.diag(U) > 0)
+    res = U.T @ U @ Hd - np.eye(96)
+    assert np.abs(res).max() < 1e-10
+
+
+# -------------------------------------------------------------- quantiser ---
+
+def _golden_quantizer():
+    cases = []
+    with open(os.path.join(GOLDEN, "quantizer_cases.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            bits, xs, s, z, q, wq = [p.strip() for p in line.split(";")]
+            cases.append((int(bits), np.array(xs.split(), float), float(s), float(z),
+                          np.array(q.split(), float), np.array(wq.split(), float)))
+    return cases
+
+
+@pytest.mark.parametrize("case", _golden_quantizer())
+def test_quantizer_golden(case):
+    bits, x, s_exp, z_exp, q_exp, wq_exp = case
+    s, z = oracle.quant_params(x[None, :], bits)
+    assert s[0] == s_exp and z[0] == z_exp
+    q = oracle.quantize(x, s[0], z[0], bits)
+    np.testing.assert_array_equal(q, q_exp)
+    np.testing.assert_array_equal(oracle.dequantize(q, s[0], z[0]), wq_exp)
+
+
+def test_quantizer_error_bound():
+    # Unclipped codes are within s/2 of the value (plain rounding); the rounding
+    # of z shifts the grid by at most s/2, so a clipped end is within s.
+    rng = _rng(7)
+    for bits in (2, 3, 4, 8):
+        x = rng.standard_normal((50, 64))
+        s, z = oracle.quant_params(x, bits)
+        s2, z2 = s[:, None], z[:, None]
+        q = oracle.quantize(x, s2, z2, bits)
+        err = np.abs(oracle.dequantize(q, s2, z2) - x)
+        raw = np.rint(x / s2) + z2
+        inside = (raw >= 0) & (raw <= (1 << bits) - 1)
+        assert np.all(err[inside] <= np.broadcast_to(s2, x.shape)[inside] * (0.5 + 1e-12))
+        assert np.all(err <= s2 * (1 + 1e-12))
+        assert q.min() >= 0 and q.max() <= (1 << bits) - 1
+
+
+# ------------------------------------------------------------ column sweep ---
+
+@pytest.mark.parametrize("group", [-1, 32])
+@pytest.mark.parametrize("bits", [3, 4])
+def test_identity_hessian_reduces_to_rtn(bits, group):
+    # With H proportional to I the factor U is diagonal: no column compensates
+    # another, so GPTQ is round-to-nearest exactly (for any damping).
+    _, W = make_problem(16, 128, 1, seed=8)
+    for scale in (1.0, 37.5):
+        out = oracle.gptq_quantize_layer(W, scale * np.eye(128), bits=bits, group=group)
+        codes, What = oracle.rtn(W, bits, group)
+        np.testing.assert_array_equal(out["codes"], codes)
+        np.testing.assert_allclose(out["What"], What, rtol=0, atol=0)
+
+
+def test_loss_identity_with_activations():
+    # ||(W - W^) X^T||_F^2 = 1/2 tr(D H D^T) with H = 2 X^T X ([Tutorial] §逐层量化).
+    X, W = make_problem(12, 64, 700, seed=9)
+    H = oracle.hessian(X)
+    out = oracle.gptq_quantize_layer(W, H, bits=4, group=32)
+    assert out["loss"] == pytest.approx(oracle.layer_loss_direct(W, out["What"], X), rel=1e-10)
+
+
+def test_obs_sum_identity():
+    # Sum of 1/2 e_j^2 equals 1/2 tr(D H_d D^T): each step leaves (D H_d)_F = 0 on
+    # the unquantised columns F, so the squared errors add up exactly.
+    X, W = make_problem(10, 96, 900, seed=10)
+    H = oracle.hessian(X)
+    out = oracle.gptq_quantize_layer(W, H, bits=3, group=-1)
+    D = W.astype(np.float64) - out["What"]
+    assert out["obs_sum"] == pytest.approx(out["loss"] + 0.5 * out["lambda"] * np.sum(D * D),
+                                           rel=1e-10)
+
+
+def test_each_step_is_the_obs_optimum():
+    # Before column j is rounded, its value (and every later column's) is the
+    # minimiser of the damped objective with columns < j fixed at their
+    # quantised values: w_F - (H_d)_FF^-1 (H_d)_FQ (w^_Q - w_Q).  This is the OBS
+    # update of [Survey] §2.2 / [Tutorial] §误差补偿 applied recursively,
+    # computed from H_d directly (no Cholesky factor involved).
+    X, W = make_problem(6, 12, 200, seed=11)
+    H = oracle.hessian(X)
+    Hd, _ = oracle.dampen(H, 0.01)
+    out = oracle.gptq_quantize_layer(W, H, bits=2, group=-1, block=5)
+    U, E, What = out["U"], out["E"], out["What"]
+    W64 = W.astype(np.float64)
+    pre = What + E * np.diag(U)[None, :]    # value of column j just before rounding
+    for j in range(1, 12):
+        Q, F = np.arange(j), np.arange(j, 12)
+        corr = np.linalg.solve(Hd[np.ix_(F, F)], Hd[np.ix_(F, Q)] @ (What[:, Q] - W64[:, Q]).T).T
+        np.testing.assert_allclose(pre[:, j], (W64[:, F] - corr)[:, 0], rtol=1e-9, atol=1e-12)
+
+
+def test_single_column_update_matches_paper_form():
+    # delta_F = (q - w_q)/[H^-1]_qq * [H^-1]_{F,q} for the first column.
+    X, W = make_problem(5, 6, 100, seed=12)
+    H = oracle.hessian(X)
+    Hd, _ = oracle.dampen(H, 0.01)
+    Hinv = np.linalg.inv(Hd)
+    out = oracle.gptq_quantize_layer(W, H, bits=3, group=-1)
+    W64 = W.astype(np.float64)
+    pre1 = out["What"][:, 1] + out["E"][:, 1] * out["U"][1, 1]
+    expect = W64[:, 1] + (out["What"][:, 0] - W64[:, 0]) / Hinv[0, 0] * Hinv[1, 0]
+    np.testing.assert_allclose(pre1, expect, rtol=1e-10)
+
+
+@pytest.mark.parametrize("group", [-1, 32])
+def test_lazy_batches_are_exact(group):
+    # [Card] 方法适配: deferring the global update to the block end does not change
+    # the result.  Block sizes 1, 32, 128 and d must agree.
+    X, W = make_problem(20, 256, 1500, seed=13)
+    H = oracle.hessian(X)
+    ref = oracle.gptq_quantize_layer(W, H, bits=4, group=group, block=256)
+    for block in (1, 32, 128) if group == -1 else (32, 128):
+        out = oracle.gptq_quantize_layer(W, H, bits=4, group=group, block=block)
+        np.testing.assert_array_equal(out["codes"], ref["codes"])
+        np.testing.assert_allclose(out["What"], ref["What"], rtol=0, atol=1e-12)
+        assert out["loss"] == pytest.approx(ref["loss"], rel=1e-12)
+
+
+def test_scale_invariance():
+    # lambda is relative to mean(diag H), so scaling H leaves every code alone.
+    X, W = make_problem(16, 128, 800, seed=14)
+    H = oracle.hessian(X)
+    ref = oracle.gptq_quantize_layer(W, H, bits=4, group=64)
+    for c in (1e-3, 7.25):
+        out = oracle.gptq_quantize_layer(W, c * H, bits=4, group=64)
+        np.testing.assert_array_equal(out["codes"], ref["codes"])
+
+
+def test_act_order_is_permutation_equivariant():
+    X, W = make_problem(16, 128, 900, seed=15)
+    H = oracle.hessian(X)
+    out = oracle.gptq_quantize_layer(W, H, bits=4, group=32, act_order=True)
+    p = out["perm"]
+    assert np.all(np.diff(np.diag(H)[p]) <= 0)
+    ref = oracle.gptq_quantize_layer(W[:, p], H[np.ix_(p, p)], bits=4, group=32)
+    inv = np.argsort(p)
+    np.testing.assert_array_equal(out["codes"], ref["codes"][:, inv])
+    # lambda's mean(diag) is summed in another order, so allow the last ulp
+    np.testing.assert_allclose(out["scales"], ref["scales"], rtol=1e-12)
+    np.testing.assert_array_equal(out["g_idx"], inv // 32)
+    assert out["loss"] == pytest.approx(ref["loss"], rel=1e-12)
+
+
+def test_dequantised_output_is_on_the_grid():
+    X, W = make_problem(8, 128, 600, seed=16)
+    out = oracle.gptq_quantize_layer(W, oracle.hessian(X), bits=3, group=32)
+    s = np.repeat(out["scales"], 32, axis=1)
+    z = np.repeat(out["zeros"], 32, axis=1)
+    np.testing.assert_array_equal(out["What"], s * (out["codes"] - z))
+    assert out["codes"].min() >= 0 and out["codes"].max() <= 7
+    assert out["zeros"].min() >= 0 and out["zeros"].max() <= 7
+
+
+def test_brute_force_bounds_tiny_rows():
+    # 2 rows x 6 columns at 2 bits: all 4^6 code vectors on the row's grid.
+    # GPTQ can never beat the exhaustive minimum of the damped objective it
+    # optimises.  It is greedy, so it does not always beat round-to-nearest on
+    # the undamped objective, but it should on most rows and on average
+    # ([Card] 证据: RTN loses far more than GPTQ).  On these 1000 fixed seeds
+    # it wins 929 times.
+    wins, g_total, r_total = 0, 0.0, 0.0
+    seeds = range(1000)
+    for seed in seeds:
+        rng = _rng(10_000 + seed)
+        X = (rng.standard_normal((16, 6)) * rng.lognormal(0, 1, 6)).astype(np.float16)
+        W = rng.standard_normal((2, 6)) * 0.02
+        H = oracle.hessian(X)
+        Hd, _ = oracle.dampen(H, 0.01)
+        out = oracle.gptq_quantize_layer(W, H, bits=2, group=-1)
+        _, What_rtn = oracle.rtn(W, 2, -1)
+        for i in range(2):
+            D = W[i] - out["What"][i]
+            g_damped = 0.5 * D @ Hd @ D
+            assert g_damped >= oracle.brute_force_min_loss(W[i], Hd, 2) * (1 - 1e-9)
+        g = out["loss"]
+        rl = oracle.layer_loss(W, What_rtn, H)
+        wins += g <= rl * (1 + 1e-12)
+        g_total += g
+        r_total += rl
+    assert wins >= 0.90 * len(seeds)
+    assert g_total < r_total
+
+
+# ------------------------------------------------------------------ pack ---
+
+def _golden_pack():
+    cases = []
+    with open(os.path.join(GOLDEN, "pack_words.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            bits, codes, words = [p.strip() for p in line.split(";")]
+            cases.append((int(bits), [int(c) for c in codes.split()],
+                          [int(w, 16) for w in words.split()]))
+    return cases
+
+
+@pytest.mark.parametrize("case", _golden_pack())
+def test_pack_golden_words(case):
+    bits, codes, words = case
+    got = oracle.pack_rows(np.array([codes]), bits).view(np.uint32)[0]
+    assert [int(w) for w in got] == words
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_pack_matches_big_integer_stream(bits):
+    # Independent route: the whole row as one Python integer, sum c_k << (b k).
+    rng = _rng(20 + bits)
+    d = 96
+    codes = rng.integers(0, 1 << bits, size=(3, d))
+    got = oracle.pack_rows(codes, bits).view(np.uint32)
+    for i in range(3):
+        stream = sum(int(c) << (bits * k) for k, c in enumerate(codes[i]))
+        expect = [(stream >> (32 * w)) & 0xFFFFFFFF for w in range(d * bits // 32)]
+        assert [int(x) for x in got[i]] == expect
+    np.testing.assert_array_equal(oracle.unpack_rows(oracle.pack_rows(codes, bits), bits, d),
+                                  codes)
+
+
+def test_pack_rejects_partial_words():
+    with pytest.raises(ValueError):
+        oracle.pack_rows(np.zeros((1, 5), dtype=np.int64), 3)
