@@ -1,0 +1,201 @@
+/*
+ * gptq.h -- C ABI of the B200 (sm_100a) GPTQ per-layer solve.
+ *
+ * The operations follow the GPTQ descriptions on these pages:
+ *   [Tutorial]  "GPTQ：一键量化大模型压缩": §二阶信息 (H = 2 sum x x^T),
+ *               §逐层量化 (layer objective ||W X - W^ X||_F^2), §误差补偿 (OBS
+ *               compensation), §分组方案 (min-max scale/zero, groups).
+ *   [Survey]    "LLM 量化技术" blog: §1.2 (x_q = round(x/s + z), s(x_q - z)),
+ *               §2.3 (fixed column order, blocks of B = 128, Cholesky rows of H^-1).
+ *   [Card]      "GPTQ: Accurate Post-Training Quantization for Generative
+ *               Pre-trained Transformers" reading card, 方法适配 (lazy batch
+ *               updates, Cholesky reformulation with mild damping).
+ *   [Explainer] "一文读懂GPTQ" §三 (codes packed into int32 arrays; bits,
+ *               group_size, desc_act).
+ *
+ * Conventions for every entry point
+ *   - Matrices are row-major.  Device pointers are CUDA global memory owned by
+ *     the caller; the library keeps no pointer after a call returns and
+ *     allocates no device memory (scratch comes from the caller's workspace).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued on it; what a call synchronises is stated per call.
+ *   - Arguments are validated on the host before anything is enqueued; a bad
+ *     argument returns GPTQ_ERR_INVALID_ARG and touches no memory.
+ *   - No kernel traps.  Every wait inside a kernel is bounded (about one
+ *     second); a wait that runs out records GPTQ_ERR_TIMEOUT in a device status
+ *     word that the synchronising calls (and gptq_check_device_status) report.
+ *   - Return value: a gptq_status (int).
+ */
+#ifndef GPTQ_B200_GPTQ_H
+#define GPTQ_B200_GPTQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st *gptq_stream_t;
+
+typedef enum {
+  GPTQ_OK = 0,
+  GPTQ_ERR_INVALID_ARG = 1, /* an argument failed validation; nothing was enqueued  */
+  GPTQ_ERR_NOT_PD = 2,      /* damped H has a non-positive pivot (not positive definite) */
+  GPTQ_ERR_CUDA = 3,        /* a CUDA runtime call failed                           */
+  GPTQ_ERR_NO_MEMORY = 4,   /* workspace smaller than the size query returned       */
+  GPTQ_ERR_TIMEOUT = 5      /* a bounded in-kernel wait ran out                     */
+} gptq_status;
+
+/* Static English text for a status code (never NULL). */
+const char *gptq_status_string(int status);
+
+/*
+ * gptq_hessian_accumulate -- H += 2 X^T X   ([Tutorial] §二阶信息, H = 2 sum_i x_i x_i^T)
+ *
+ *   X    device, fp16 (IEEE binary16 bits), [n x d] row-major with leading
+ *        dimension ldx (elements): row t is the activation vector of token t.
+ *        16-byte aligned; ldx >= d and ldx % 8 == 0.
+ *   n    number of tokens, n >= 0 (n == 0 enqueues nothing).
+ *   d    input features, d > 0 and d % 32 == 0.
+ *   H    device, fp32 [d x d] row-major (leading dimension d), 16-byte aligned.
+ *        On return (stream order) H = sym(upper(H_in) + 2 X^T X): the upper
+ *        triangle accumulates, and the lower triangle is written with the
+ *        mirror of the new upper triangle.  Pass H = 0 for a fresh Hessian;
+ *        calling repeatedly over token chunks sums them.
+ *   Products of fp16 values are exact in fp32; the fp32 sums are folded out of
+ *   the tensor-core accumulator every 512 tokens to bound rounding growth.
+ *   Asynchronous: returns after enqueueing one kernel.
+ */
+int gptq_hessian_accumulate(const void *X, int64_t n, int64_t d, int64_t ldx, float *H,
+                            gptq_stream_t stream);
+
+/*
+ * gptq_quantize_workspace_bytes -- device workspace needed by gptq_quantize_layer
+ * for these arguments (0 if the arguments are invalid).  The workspace must be
+ * 256-byte aligned.
+ */
+size_t gptq_quantize_workspace_bytes(int64_t r, int64_t d, int bits, int group, int block,
+                                     int act_order);
+
+/*
+ * gptq_quantize_layer -- GPTQ solve of one linear layer
+ *   ([Card] 方法适配; [Survey] §2.3; [Tutorial] §误差补偿, §分组方案)
+ *
+ * Steps, all on the GPU in stream order:
+ *   1. lambda = damp * mean(diag H); H_d = H + lambda I.
+ *   2. act_order != 0: perm = stable argsort of -diag(H) (ties keep the lower
+ *      index); columns of W and rows/columns of H_d are taken in that order.
+ *   3. U = upper Cholesky factor of H_d^-1 (U^T U = H_d^-1), computed as the
+ *      "reverse" Cholesky H_d = R R^T (R upper) and U = R^-1.
+ *   4. For j = 0..d-1 in blocks of `block` columns: at a group start, per-row
+ *      s = (xmax - xmin)/(2^bits - 1) and z = rint(-xmin/s) over the current
+ *      group columns (xmin <= 0 <= xmax; s = 1 if the range is empty); for
+ *      group = -1 once per row from the original W.  q = clamp(rint(w_j/s) + z,
+ *      0, 2^bits - 1), w^_j = s (q - z), e_j = (w_j - w^_j)/U_jj, and the
+ *      later columns of the block move by -e_j U[j, j+1:].  Later blocks are
+ *      moved once per block (lazy batch) or once per 1024 columns, an exact
+ *      reordering of the same updates.
+ *   5. loss = ||(W - W^) X^T||_F^2 = 1/2 tr(D H D^T) with D = W - W^ and the
+ *      undamped H, evaluated as sum_j 1/2 e_j^2 - lambda/2 ||D||_F^2.
+ *   6. Codes are returned in the original column order and packed.
+ *
+ *   W         device fp32 [r x d], read only.
+ *   r, d      r >= 0 (r == 0: returns GPTQ_OK with *loss = 0, enqueues nothing),
+ *             d > 0, d % 32 == 0.
+ *   H         device fp32 [d x d], full symmetric (as written by
+ *             gptq_hessian_accumulate).  CONSUMED: overwritten with the
+ *             factorisation (U in the upper triangle when act_order == 0; the
+ *             contents are unspecified when act_order != 0).
+ *   bits      2, 3, 4 or 8.
+ *   group     -1 (one scale/zero per row) or a multiple of 32 that divides d
+ *             with block % group == 0 or group % block == 0.
+ *   block     32, 64 or 128 (the lazy-batch width B; the pages use 128).
+ *   damp      relative damping >= 0 (the pages' "mild damping"; 0.01 typical).
+ *   act_order 0 or 1.
+ *   W_hat     device fp32 [r x d] or NULL: dequantised weights s(q - z) in the
+ *             original column order.  May alias W.
+ *   qweight   device int32 [r x d*bits/32]: per row, the codes of columns
+ *             0..d-1 as an LSB-first bit stream (code c at stream bits
+ *             [c*bits, (c+1)*bits), stream bit k = bit k%32 of word k/32).
+ *   scales    device fp32 [r x G], G = d/group (G = 1 for group = -1).
+ *             Column k belongs to quantisation group k (permuted positions
+ *             [k*group, (k+1)*group) under act-order).
+ *   zeros     device int32 [r x G], integer zero points in [0, 2^bits - 1].
+ *   g_idx     device int32 [d] or NULL: group of each original column.
+ *   codes     device uint8 [r x d] or NULL: unpacked codes, original order.
+ *   loss      host double or NULL: the layer loss of step 5.
+ *   workspace device scratch of at least gptq_quantize_workspace_bytes(...)
+ *             bytes, 256-byte aligned; contents on entry are ignored.
+ *   Synchronises `stream` once, at the end, to read the status and the loss.
+ *   Returns GPTQ_ERR_NOT_PD if the damped H is not positive definite (outputs
+ *   are then unspecified), GPTQ_ERR_NO_MEMORY if workspace_bytes is too small.
+ */
+int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int group,
+                        int block, float damp, int act_order, float *W_hat, int32_t *qweight,
+                        float *scales, int32_t *zeros, int32_t *g_idx, uint8_t *codes,
+                        double *loss, void *workspace, size_t workspace_bytes,
+                        gptq_stream_t stream);
+
+/*
+ * gptq_pack -- pack codes into int32 words   ([Explainer] §三, int32 storage of 3/4-bit codes)
+ *
+ *   codes   device uint8 [r x d], values < 2^bits (higher bits are masked off).
+ *   d       d > 0, d % 32 == 0.   bits: 2, 3, 4 or 8.
+ *   qweight device int32 [r x d*bits/32], layout as in gptq_quantize_layer.
+ *   Asynchronous.
+ */
+int gptq_pack(const uint8_t *codes, int64_t r, int64_t d, int bits, int32_t *qweight,
+              gptq_stream_t stream);
+
+/*
+ * gptq_layer_host_workspace_bytes / gptq_solve_layer_host -- the whole layer
+ * from HOST buffers: copy X and W to the device, H = 2 X^T X, quantise, pack,
+ * and copy qweight, scales, zeros, g_idx and the loss back.
+ *
+ *   X_host   host fp16 bits [n x d] (pinned memory gives full copy bandwidth).
+ *   W_host   host fp32 [r x d].
+ *   outputs  host buffers with the shapes of gptq_quantize_layer (g_idx_host
+ *            may be NULL).
+ *   dev_workspace  device scratch of gptq_layer_host_workspace_bytes(...) bytes,
+ *            256-byte aligned; it holds the device copies of X, W, H and the
+ *            outputs plus the quantiser's workspace.
+ *   Synchronous: returns when the outputs are in the host buffers.
+ */
+size_t gptq_layer_host_workspace_bytes(int64_t r, int64_t d, int64_t n, int bits, int group,
+                                       int block, int act_order);
+int gptq_solve_layer_host(const uint16_t *X_host, int64_t n, const float *W_host, int64_t r,
+                          int64_t d, int bits, int group, int block, float damp, int act_order,
+                          int32_t *qweight_host, float *scales_host, int32_t *zeros_host,
+                          int32_t *g_idx_host, double *loss, void *dev_workspace,
+                          size_t dev_workspace_bytes, gptq_stream_t stream);
+
+/*
+ * gptq_check_device_status -- synchronise `stream`, then return and clear the
+ * library's device status word (GPTQ_ERR_TIMEOUT if an asynchronous kernel,
+ * such as the Hessian, gave up on a bounded wait; GPTQ_OK otherwise).
+ */
+int gptq_check_device_status(gptq_stream_t stream);
+
+/* Number of kernels this library has launched in this process (all devices). */
+uint64_t gptq_launch_count(void);
+
+/*
+ * Phase timing for gptq_quantize_layer (off by default, process-wide, not
+ * thread-safe).  When on, each call records CUDA events on its stream between
+ * phases; gptq_last_phase_ms writes up to `n` durations in ms of the last call:
+ *   [0] damping + act-order permutation + working copy of W
+ *   [1] Cholesky factor and triangular inverse (U)
+ *   [2] column sweep (in-block kernels and trailing-update GEMMs)
+ *   [3] unpermute, loss and packing
+ * and returns the number written.
+ */
+int gptq_set_phase_timing(int enable);
+int gptq_last_phase_ms(float *ms, int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_GPTQ_H */

@@ -1,0 +1,22 @@
+"""B200-native (sm_100a) GPTQ per-layer solve behind a C ABI.
+
+The compute lives in libgptq_b200.so (hand-written CUDA kernels: tcgen05/TMA
+Hessian, fp64-leaf recursive Cholesky with its inverse, warp-per-row column
+sweep with lazy trailing updates, fused unpermute/pack).  This package holds
+the nvcc build step, a ctypes view of include/gptq.h and a thin torch binding
+with the same entry-point names.
+"""
+
+from .gptq import (  # noqa: F401
+    GPTQError,
+    gptq_check_device_status,
+    gptq_hessian_accumulate,
+    gptq_last_phase_ms,
+    gptq_launch_count,
+    gptq_layer_host_workspace_bytes,
+    gptq_pack,
+    gptq_quantize_layer,
+    gptq_quantize_workspace_bytes,
+    gptq_set_phase_timing,
+    gptq_solve_layer_host,
+)

@@ -1,0 +1,350 @@
+// C-ABI entry points of the layer solve: validation, workspace layout, and the
+// stream-ordered sequence of kernels (see include/gptq.h for the contract).
+#include <string.h>
+
+#include "gptq_internal.h"
+
+namespace gptq {
+
+std::atomic<uint64_t> g_launches{0};
+
+namespace {
+
+constexpr int kSuperblock = 1024;  // columns per global (deferred) trailing update
+
+bool valid_bits(int b) { return b == 2 || b == 3 || b == 4 || b == 8; }
+
+bool valid_layer(int64_t r, int64_t d, int bits, int group, int block) {
+  if (r < 0 || r > (int64_t)INT32_MAX / 2) return false;
+  if (d <= 0 || d % 32 != 0 || d > 65536) return false;
+  if (!valid_bits(bits)) return false;
+  if (block != 32 && block != 64 && block != 128) return false;
+  if (group != -1) {
+    if (group < 32 || group % 32 != 0 || d % group != 0) return false;
+    if (!(block % group == 0 || group % block == 0)) return false;
+  }
+  return true;
+}
+
+// Columns between global trailing updates: a multiple of the block, and
+// aligned so that no quantisation group straddles a superblock end unless it
+// also starts at a superblock start (then every column it reads is current).
+int superblock(int64_t d, int group, int block) {
+  int S = kSuperblock;
+  if (group > block && S % group != 0 && group % S != 0) S = group;
+  const int64_t dr = (d + block - 1) / block * block;
+  if (S > dr) S = (int)dr;
+  return S;
+}
+
+struct Layout {
+  size_t Wk, ErrS, codes_p, perm, inv, Hp, T1, loss_rows, dsq_rows, out, lambda, status, total;
+};
+
+Layout layout(int64_t r, int64_t d, int group, int block, int act_order) {
+  Layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  const int S = superblock(d, group, block);
+  L.Wk = take((size_t)r * d * 4);
+  L.ErrS = take((size_t)r * S * 4);
+  L.codes_p = take((size_t)r * d);
+  L.perm = take((size_t)d * 4);
+  L.inv = take((size_t)d * 4);
+  L.Hp = take(act_order ? (size_t)d * d * 4 : 0);
+  L.T1 = take(factor_scratch_floats(d) * 4);
+  L.loss_rows = take((size_t)r * 8);
+  L.dsq_rows = take((size_t)r * 8);
+  L.out = take(4 * 8);
+  L.lambda = take(4);
+  L.status = take(16);
+  L.total = off;
+  return L;
+}
+
+// Phase timing (optional).
+bool g_timing = false;
+float g_phase_ms[4] = {0, 0, 0, 0};
+cudaEvent_t g_ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+
+int record(int i, cudaStream_t s) {
+  if (!g_timing) return GPTQ_OK;
+  if (!g_ev[i]) GPTQ_CUDA_TRY(cudaEventCreate(&g_ev[i]));
+  GPTQ_CUDA_TRY(cudaEventRecord(g_ev[i], s));
+  return GPTQ_OK;
+}
+
+#define GPTQ_TRY(expr)                      \
+  do {                                      \
+    const int rc_ = (expr);                 \
+    if (rc_ != GPTQ_OK) return rc_;         \
+  } while (0)
+
+}  // namespace
+}  // namespace gptq
+
+using namespace gptq;
+
+extern "C" const char *gptq_status_string(int status) {
+  switch (status) {
+    case GPTQ_OK: return "ok";
+    case GPTQ_ERR_INVALID_ARG: return "invalid argument";
+    case GPTQ_ERR_NOT_PD: return "damped Hessian is not positive definite";
+    case GPTQ_ERR_CUDA: return "CUDA runtime error";
+    case GPTQ_ERR_NO_MEMORY: return "workspace too small";
+    case GPTQ_ERR_TIMEOUT: return "bounded in-kernel wait timed out";
+    default: return "unknown status";
+  }
+}
+
+extern "C" uint64_t gptq_launch_count(void) { return g_launches.load(); }
+
+extern "C" int gptq_set_phase_timing(int enable) {
+  g_timing = enable != 0;
+  return GPTQ_OK;
+}
+
+extern "C" int gptq_last_phase_ms(float *ms, int n) {
+  if (!ms || n < 0) return 0;
+  const int k = n < 4 ? n : 4;
+  for (int i = 0; i < k; ++i) ms[i] = g_phase_ms[i];
+  return k;
+}
+
+extern "C" int gptq_check_device_status(gptq_stream_t stream) {
+  GPTQ_CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
+  int *w = device_status_word();
+  if (!w) return GPTQ_ERR_CUDA;
+  int v = 0;
+  GPTQ_CUDA_TRY(cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost));
+  if (v != 0) {
+    const int zero = 0;
+    GPTQ_CUDA_TRY(cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice));
+  }
+  return v;
+}
+
+extern "C" size_t gptq_quantize_workspace_bytes(int64_t r, int64_t d, int bits, int group,
+                                                int block, int act_order) {
+  if (!valid_layer(r, d, bits, group, block)) return 0;
+  return layout(r, d, group, block, act_order).total;
+}
+
+extern "C" int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits,
+                                   int group, int block, float damp, int act_order, float *W_hat,
+                                   int32_t *qweight, float *scales, int32_t *zeros,
+                                   int32_t *g_idx, uint8_t *codes, double *loss, void *workspace,
+                                   size_t workspace_bytes, gptq_stream_t stream) {
+  if (!valid_layer(r, d, bits, group, block)) return GPTQ_ERR_INVALID_ARG;
+  if (!(damp >= 0.f) || damp > 1e30f) return GPTQ_ERR_INVALID_ARG;
+  if (act_order != 0 && act_order != 1) return GPTQ_ERR_INVALID_ARG;
+  if (r == 0) {
+    if (loss) *loss = 0.0;
+    return GPTQ_OK;
+  }
+  if (!W || !H || !qweight || !scales || !zeros || !workspace) return GPTQ_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(W) % 16 || reinterpret_cast<uintptr_t>(H) % 16 ||
+      reinterpret_cast<uintptr_t>(workspace) % 256 ||
+      (W_hat && reinterpret_cast<uintptr_t>(W_hat) % 16) ||
+      reinterpret_cast<uintptr_t>(qweight) % 4 || reinterpret_cast<uintptr_t>(scales) % 4 ||
+      reinterpret_cast<uintptr_t>(zeros) % 4 || (g_idx && reinterpret_cast<uintptr_t>(g_idx) % 4))
+    return GPTQ_ERR_INVALID_ARG;
+  const Layout L = layout(r, d, group, block, act_order);
+  if (workspace_bytes < L.total) return GPTQ_ERR_NO_MEMORY;
+
+  cudaStream_t st = (cudaStream_t)stream;
+  char *ws = static_cast<char *>(workspace);
+  float *Wk = reinterpret_cast<float *>(ws + L.Wk);
+  float *ErrS = reinterpret_cast<float *>(ws + L.ErrS);
+  uint8_t *codes_p = reinterpret_cast<uint8_t *>(ws + L.codes_p);
+  int *perm = reinterpret_cast<int *>(ws + L.perm);
+  int *inv = reinterpret_cast<int *>(ws + L.inv);
+  float *Hp = reinterpret_cast<float *>(ws + L.Hp);
+  float *T1 = reinterpret_cast<float *>(ws + L.T1);
+  double *loss_rows = reinterpret_cast<double *>(ws + L.loss_rows);
+  double *dsq_rows = reinterpret_cast<double *>(ws + L.dsq_rows);
+  double *out = reinterpret_cast<double *>(ws + L.out);
+  float *lambda = reinterpret_cast<float *>(ws + L.lambda);
+  int *status = reinterpret_cast<int *>(ws + L.status);
+  const int ri = (int)r, di = (int)d;
+  const int G = group < 0 ? 1 : di / group;
+  const int S = superblock(d, group, block);
+
+  GPTQ_TRY(record(0, st));
+  GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 16, st));
+  GPTQ_CUDA_TRY(cudaMemsetAsync(loss_rows, 0, (size_t)r * 8, st));
+
+  // Phase 0: damping, act-order, working copy of W.
+  float *Hf = H;
+  if (act_order) {
+    GPTQ_TRY(launch_damp(H, d, di, damp, false, lambda, st));
+    GPTQ_TRY(launch_act_order(H, d, di, perm, inv, lambda, Hp, st));
+    Hf = Hp;
+  } else {
+    GPTQ_TRY(launch_damp(H, d, di, damp, true, lambda, st));
+  }
+  GPTQ_TRY(launch_gather_w(W, ri, di, act_order ? perm : nullptr, Wk, status, st));
+  GPTQ_TRY(record(1, st));
+
+  // Phase 1: U = upper Cholesky factor of H_d^-1, in place.
+  GPTQ_TRY(launch_factor(Hf, d, T1, status, st));
+  GPTQ_TRY(record(2, st));
+
+  // Phase 2: column sweep in blocks, lazy trailing updates.
+  if (group < 0) GPTQ_TRY(launch_row_params(Wk, ri, di, bits, scales, zeros, status, st));
+  for (int s0 = 0; s0 < di; s0 += S) {
+    const int sEnd = s0 + S < di ? s0 + S : di;
+    for (int j0 = s0; j0 < sEnd; j0 += block) {
+      const int j1 = j0 + block < sEnd ? j0 + block : sEnd;
+      SweepArgs a{};
+      a.Wk = Wk;
+      a.ldw = d;
+      a.U = Hf;
+      a.ldu = d;
+      a.r = ri;
+      a.j0 = j0;
+      a.ncols = j1 - j0;
+      a.bits = bits;
+      a.group = group;
+      a.scales = scales;
+      a.zeros = zeros;
+      a.G = G;
+      a.codes = codes_p;
+      a.ldc = d;
+      a.err = ErrS + (j0 - s0);
+      a.lde = S;
+      a.loss_rows = loss_rows;
+      a.status = status;
+      GPTQ_TRY(launch_sweep_block(a, block, st));
+      if (j1 < sEnd) {
+        // Rest of this superblock: W[:, j1:sEnd] -= E_blk U[j0:j1, j1:sEnd]
+        GemmArgs g{ri, sEnd - j1, j1 - j0, ErrS + (j0 - s0), S, Hf + (size_t)j0 * d + j1, d,
+                   Wk + j1, d, -1.f, 1.f, 0, status};
+        GPTQ_TRY(launch_gemm(g, false, st));
+      }
+    }
+    if (sEnd < di) {
+      // Deferred global update: W[:, sEnd:] -= E_S U[s0:sEnd, sEnd:]
+      GemmArgs g{ri, di - sEnd, sEnd - s0, ErrS, S, Hf + (size_t)s0 * d + sEnd, d, Wk + sEnd, d,
+                 -1.f, 1.f, 0, status};
+      GPTQ_TRY(launch_gemm(g, false, st));
+    }
+  }
+  GPTQ_TRY(record(3, st));
+
+  // Phase 3: unpermute, loss, packing.
+  FinalizeArgs f{};
+  f.W = W;
+  f.Wk = Wk;
+  f.codes_p = codes_p;
+  f.inv = act_order ? inv : nullptr;
+  f.r = ri;
+  f.d = di;
+  f.bits = bits;
+  f.group = group;
+  f.W_hat = W_hat;
+  f.codes = codes;
+  f.qweight = qweight;
+  f.g_idx = g_idx;
+  f.dsq_rows = dsq_rows;
+  f.status = status;
+  GPTQ_TRY(launch_finalize(f, st));
+  GPTQ_TRY(launch_loss_reduce(loss_rows, dsq_rows, ri, lambda, out, status, st));
+  GPTQ_TRY(record(4, st));
+
+  double host_out[3] = {0, 0, 0};
+  int host_status = 0;
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(host_out, out, sizeof(host_out), cudaMemcpyDeviceToHost, st));
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(&host_status, status, sizeof(int), cudaMemcpyDeviceToHost, st));
+  GPTQ_CUDA_TRY(cudaStreamSynchronize(st));
+  if (g_timing)
+    for (int i = 0; i < 4; ++i) cudaEventElapsedTime(&g_phase_ms[i], g_ev[i], g_ev[i + 1]);
+  if (host_status != 0) return host_status;
+  if (loss) *loss = host_out[0];
+  return GPTQ_OK;
+}
+
+namespace {
+
+struct HostLayout {
+  size_t X, H, W, qw, sc, zr, gi, qws, total;
+};
+
+HostLayout host_layout(int64_t r, int64_t d, int64_t n, int bits, int group, int block,
+                       int act_order) {
+  HostLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  const int64_t G = group < 0 ? 1 : d / group;
+  L.X = take((size_t)n * d * 2);
+  L.H = take((size_t)d * d * 4);
+  L.W = take((size_t)r * d * 4);
+  L.qw = take((size_t)r * (d * bits / 32) * 4);
+  L.sc = take((size_t)r * G * 4);
+  L.zr = take((size_t)r * G * 4);
+  L.gi = take((size_t)d * 4);
+  L.qws = take(layout(r, d, group, block, act_order).total);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" size_t gptq_layer_host_workspace_bytes(int64_t r, int64_t d, int64_t n, int bits,
+                                                  int group, int block, int act_order) {
+  if (!valid_layer(r, d, bits, group, block) || n < 0 || n > (int64_t)INT32_MAX) return 0;
+  return host_layout(r, d, n, bits, group, block, act_order).total;
+}
+
+extern "C" int gptq_solve_layer_host(const uint16_t *X_host, int64_t n, const float *W_host,
+                                     int64_t r, int64_t d, int bits, int group, int block,
+                                     float damp, int act_order, int32_t *qweight_host,
+                                     float *scales_host, int32_t *zeros_host,
+                                     int32_t *g_idx_host, double *loss, void *dev_workspace,
+                                     size_t dev_workspace_bytes, gptq_stream_t stream) {
+  if (!valid_layer(r, d, bits, group, block) || n < 0 || n > (int64_t)INT32_MAX)
+    return GPTQ_ERR_INVALID_ARG;
+  if ((n > 0 && !X_host) || !W_host || !qweight_host || !scales_host || !zeros_host ||
+      !dev_workspace || reinterpret_cast<uintptr_t>(dev_workspace) % 256)
+    return GPTQ_ERR_INVALID_ARG;
+  if (r == 0) {
+    if (loss) *loss = 0.0;
+    return GPTQ_OK;
+  }
+  const HostLayout L = host_layout(r, d, n, bits, group, block, act_order);
+  if (dev_workspace_bytes < L.total) return GPTQ_ERR_NO_MEMORY;
+  cudaStream_t st = (cudaStream_t)stream;
+  char *ws = static_cast<char *>(dev_workspace);
+  uint16_t *X = reinterpret_cast<uint16_t *>(ws + L.X);
+  float *H = reinterpret_cast<float *>(ws + L.H);
+  float *W = reinterpret_cast<float *>(ws + L.W);
+  int32_t *qw = reinterpret_cast<int32_t *>(ws + L.qw);
+  float *sc = reinterpret_cast<float *>(ws + L.sc);
+  int32_t *zr = reinterpret_cast<int32_t *>(ws + L.zr);
+  int32_t *gi = reinterpret_cast<int32_t *>(ws + L.gi);
+  const int64_t G = group < 0 ? 1 : d / group;
+
+  if (n > 0)
+    GPTQ_CUDA_TRY(cudaMemcpyAsync(X, X_host, (size_t)n * d * 2, cudaMemcpyHostToDevice, st));
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(W, W_host, (size_t)r * d * 4, cudaMemcpyHostToDevice, st));
+  GPTQ_CUDA_TRY(cudaMemsetAsync(H, 0, (size_t)d * d * 4, st));
+  GPTQ_TRY(gptq_hessian_accumulate(X, n, d, d, H, stream));
+  GPTQ_TRY(gptq_quantize_layer(W, r, d, H, bits, group, block, damp, act_order, nullptr, qw, sc,
+                               zr, gi, nullptr, loss, ws + L.qws, L.total - L.qws, stream));
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(qweight_host, qw, (size_t)r * (d * bits / 32) * 4,
+                                cudaMemcpyDeviceToHost, st));
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(scales_host, sc, (size_t)r * G * 4, cudaMemcpyDeviceToHost, st));
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(zeros_host, zr, (size_t)r * G * 4, cudaMemcpyDeviceToHost, st));
+  if (g_idx_host)
+    GPTQ_CUDA_TRY(cudaMemcpyAsync(g_idx_host, gi, (size_t)d * 4, cudaMemcpyDeviceToHost, st));
+  GPTQ_CUDA_TRY(cudaStreamSynchronize(st));
+  return GPTQ_OK;
+}

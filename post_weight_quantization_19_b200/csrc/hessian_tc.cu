@@ -1,0 +1,339 @@
+// H += 2 X^T X on the sm_100a tensor cores (tcgen05 + TMEM, operands by TMA).
+//
+// Source: "GPTQ：一键量化大模型压缩" §二阶信息 -- the layer Hessian is
+// H = 2 sum_i x_i x_i^T over the calibration activations; with X [n x d]
+// (tokens x features) that is 2 X^T X.
+//
+// Design (B200):
+//  * H is symmetric, so only 128 x 256 output tiles that touch the upper
+//    triangle are computed (tile (I, J) with J >= floor(I/2)); the epilogue
+//    writes each upper element and its mirror exactly once.
+//  * X is token-major, so both UMMA operands are MN-major: a TMA box of
+//    64 features x 64 tokens (128-byte rows, 128-byte swizzle) is one swizzle
+//    atom column; A = X[:, i0:i0+128]^T takes two boxes, B = X[:, j0:j0+256]
+//    four.  One tcgen05.mma of M=128, N=256, K=16 consumes 16 tokens.
+//  * Warp roles: warp 0 issues TMA into a 4-stage ring, warp 1 issues UMMA
+//    into one of two 256-column TMEM accumulators, warps 2..9 drain TMEM.
+//  * Accuracy: the tensor core's fp32 accumulation is not guaranteed to round
+//    to nearest, so each TMEM accumulation chain is limited to 512 tokens and
+//    then folded into fp32 registers of the epilogue warps (double-buffered
+//    TMEM, so the tensor core keeps running while a chain is folded).
+//  * Persistent grid of one CTA per SM walking the tile list; all CTAs sweep
+//    the tokens at the same pace, so the current X slab is shared through L2.
+#include <mutex>
+
+#include "gptq_common.cuh"
+
+namespace gptq {
+
+__device__ int g_device_status;
+
+int *device_status_word() {
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+  return static_cast<int *>(p);
+}
+
+int num_sms() {
+  int dev = 0, v = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+  return v > 0 ? v : 1;
+}
+
+namespace {
+
+constexpr int HM = 128;                          // tile rows  (UMMA M)
+constexpr int HN = 256;                          // tile cols  (UMMA N)
+constexpr int HK = 64;                           // tokens per pipeline stage
+constexpr int STAGES = 4;
+constexpr int FOLD = 8;                          // stages per TMEM chain (512 tokens)
+constexpr int BOXF = 64;                         // features per TMA box (128 bytes)
+constexpr int BOX_BYTES = BOXF * HK * 2;         // 8 KB
+constexpr int A_BYTES = HM * HK * 2;             // 16 KB
+constexpr int B_BYTES = HN * HK * 2;             // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 48 KB
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int THREADS = 32 * (2 + NUM_EPI_WARPS);
+constexpr uint32_t TMEM_COLS = 512;              // two 256-column accumulators
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024;
+
+struct HessShared {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t accf[2];
+  uint64_t acce[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void tile_coords(int t, int nI, int nJ, int &I, int &J) {
+  for (I = 0; I < nI; ++I) {
+    const int cnt = nJ - I / 2;
+    if (t < cnt) {
+      J = I / 2 + t;
+      return;
+    }
+    t -= cnt;
+  }
+  I = nI - 1;
+  J = nJ - 1;
+}
+
+__device__ __forceinline__ void record_timeout(int *status, HessShared &sh) {
+  atomicCAS(status, 0, (int)GPTQ_ERR_TIMEOUT);
+  *(volatile int *)&sh.abort = 1;
+}
+
+__global__ void __maxnreg__(200)
+    hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, int64_t n, int d,
+                      float *__restrict__ H, int *__restrict__ status) {
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ HessShared sh;
+  uint8_t *smem =
+      reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nI = (d + HM - 1) / HM;
+  const int nJ = (d + HN - 1) / HN;
+  int T = 0;
+  for (int I = 0; I < nI; ++I) T += nJ - I / 2;
+  const int nsteps = (int)((n + HK - 1) / HK);
+  const int nchunks = (nsteps + FOLD - 1) / FOLD;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh.accf[b], 1);
+      mbar_init(&sh.acce[b], NUM_EPI_WARPS);
+    }
+    mbar_init(&sh.drain, 1);
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tmap);
+  if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t issued = 0, issued_par = 0;  // bit s: stage s has a load in flight / its parity
+      bool ok = true;
+      for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
+        int I, J;
+        tile_coords(t, nI, nJ, I, J);
+        const int i0 = I * HM, j0 = J * HN;
+        for (int ks = 0; ks < nsteps; ++ks) {
+          if (*(volatile int *)&sh.abort) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1)) {
+            record_timeout(status, sh);
+            ok = false;
+            break;
+          }
+          uint8_t *sA = smem + (size_t)stage * STAGE_BYTES;
+          uint8_t *sB = sA + A_BYTES;
+          const int y = ks * HK;
+          mbar_arrive_expect_tx(&sh.full[stage], STAGE_BYTES);
+          tma_load_2d(sA, &tmap, i0, y, &sh.full[stage]);
+          tma_load_2d(sA + BOX_BYTES, &tmap, i0 + BOXF, y, &sh.full[stage]);
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            tma_load_2d(sB + m * BOX_BYTES, &tmap, j0 + m * BOXF, y, &sh.full[stage]);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Let every load this thread started land before the CTA can exit.
+      for (int s = 0; s < STAGES; ++s)
+        if (issued & (1u << s)) (void)mbar_wait_bounded(&sh.full[s], (issued_par >> s) & 1u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc(0, 0, 1, 1, HM, HN);
+      uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
+        for (int c = 0; c < nchunks && ok; ++c) {
+          if (!mbar_wait_bounded(&sh.acce[abuf], aphase ^ 1)) {
+            record_timeout(status, sh);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t dt = tmem + abuf * HN;
+          const int s0 = c * FOLD;
+          const int s1 = min(nsteps, s0 + FOLD);
+          for (int ks = s0; ks < s1; ++ks) {
+            if (!mbar_wait_bounded(&sh.full[stage], phase)) {
+              record_timeout(status, sh);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(smem + (size_t)stage * STAGE_BYTES);
+            const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < HK / 16; ++kk) {
+              // 16 tokens = two 8-row groups of the 128-byte swizzle atom.
+              const uint64_t ad = smem_desc(a0 + kk * 2048, BOX_BYTES, 1024, 2);
+              const uint64_t bd = smem_desc(b0 + kk * 2048, BOX_BYTES, 1024, 2);
+              umma_f16_ss(dt, ad, bd, idesc, (ks > s0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&sh.empty[stage]);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+          if (!ok) break;
+          umma_commit(&sh.accf[abuf]);
+          abuf ^= 1;
+          if (abuf == 0) aphase ^= 1;
+        }
+      }
+      // Every MMA this thread issued has completed once the drain barrier fires.
+      umma_commit(&sh.drain);
+      (void)mbar_wait_bounded(&sh.drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int quarter = warp & 3;       // TMEM lanes this warp may access
+    const int half = ew >> 2;           // which 128 of the 256 tile columns
+    uint32_t abuf = 0, aphase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
+      int I, J;
+      tile_coords(t, nI, nJ, I, J);
+      const int i0 = I * HM, j0 = J * HN;
+      float acc[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      for (int c = 0; c < nchunks; ++c) {
+        if (!mbar_wait_bounded(&sh.accf[abuf], aphase)) {
+          if (lane == 0) record_timeout(status, sh);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + abuf * HN + half * 128;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          float v[32];
+          tmem_ld_32x32b_x32(base + p * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[p * 32 + i] += v[i];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.acce[abuf]);
+        abuf ^= 1;
+        if (abuf == 0) aphase ^= 1;
+      }
+      if (!ok) break;
+      const int row = i0 + quarter * 32 + lane;
+      const int cb = j0 + half * 128;
+      if (row < d) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const int col = cb + i;
+          if (col < d && col >= row) {
+            const float v = 2.f * acc[i];
+            H[(size_t)row * d + col] += v;
+            if (col > row) H[(size_t)col * d + row] += v;
+          }
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+}  // namespace gptq
+
+using namespace gptq;
+
+extern "C" int gptq_hessian_accumulate(const void *X, int64_t n, int64_t d, int64_t ldx, float *H,
+                                       gptq_stream_t stream) {
+  if (!X || !H) return GPTQ_ERR_INVALID_ARG;
+  if (n < 0 || n > (int64_t)INT32_MAX) return GPTQ_ERR_INVALID_ARG;
+  if (d <= 0 || d % 32 != 0 || d > 65536) return GPTQ_ERR_INVALID_ARG;
+  if (ldx < d || ldx % 8 != 0) return GPTQ_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(X) % 16 != 0 || reinterpret_cast<uintptr_t>(H) % 16 != 0)
+    return GPTQ_ERR_INVALID_ARG;
+  if (n == 0) return GPTQ_OK;
+
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return GPTQ_ERR_CUDA;
+  CUtensorMap tmap;
+  const cuuint64_t gdim[2] = {(cuuint64_t)d, (cuuint64_t)n};
+  const cuuint64_t gstride[1] = {(cuuint64_t)ldx * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BOXF, (cuuint32_t)HK};
+  const cuuint32_t estride[2] = {1, 1};
+  if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(X), gdim, gstride, box,
+          estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return GPTQ_ERR_CUDA;
+
+  int *status = device_status_word();
+  if (!status) return GPTQ_ERR_CUDA;
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(hessian_tc_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES));
+  const int nI = (int)((d + HM - 1) / HM), nJ = (int)((d + HN - 1) / HN);
+  int T = 0;
+  for (int I = 0; I < nI; ++I) T += nJ - I / 2;
+  const int grid = T < num_sms() ? T : num_sms();
+  hessian_tc_kernel<<<grid, THREADS, SMEM_BYTES, (cudaStream_t)stream>>>(tmap, n, (int)d, H,
+                                                                         status);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}

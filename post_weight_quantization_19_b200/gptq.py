@@ -1,0 +1,167 @@
+"""Python binding of the C ABI: the same entry points, taking torch CUDA tensors.
+
+Argument marshalling only -- dtype/shape/device checks and pointer extraction.
+Every step of the solve runs in the CUDA kernels of libgptq_b200.so; there is
+no CPU path.  PyTorch provides device memory and streams.
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi
+
+
+class GPTQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = _abi.load()
+        msg = lib.gptq_status_string(status).decode()
+        super().__init__(f"{where}: {_abi.STATUS.get(status, status)} ({msg})")
+        self.status = status
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise GPTQError(status, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None, dtype: torch.dtype | None = None, name: str = "") -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def gptq_hessian_accumulate(X: torch.Tensor, H: torch.Tensor, stream=None) -> None:
+    """H += 2 X^T X on the GPU (X fp16 [n, d] row-major, H fp32 [d, d])."""
+    lib = _abi.load()
+    n, d = X.shape
+    if H.shape != (d, d):
+        raise ValueError("H must be [d, d]")
+    _check(lib.gptq_hessian_accumulate(_ptr(X, torch.float16, "X"), n, d, d,
+                                       _ptr(H, torch.float32, "H"), _stream(stream)),
+           "gptq_hessian_accumulate")
+
+
+def gptq_quantize_workspace_bytes(r: int, d: int, bits: int, group: int, block: int = 128,
+                                  act_order: bool = False) -> int:
+    return int(_abi.load().gptq_quantize_workspace_bytes(r, d, bits, group, block,
+                                                         int(act_order)))
+
+
+def gptq_quantize_layer(W: torch.Tensor, H: torch.Tensor, *, bits: int, group: int,
+                        block: int = 128, damp: float = 0.01, act_order: bool = False,
+                        W_hat: torch.Tensor | None = None, codes: torch.Tensor | None = None,
+                        g_idx: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                        outputs: dict | None = None, stream=None) -> dict:
+    """GPTQ solve of one layer.  H is consumed.  Returns qweight/scales/zeros/loss (+ optional).
+
+    ``outputs`` may hold preallocated ``qweight``, ``scales`` and ``zeros`` tensors.
+    """
+    lib = _abi.load()
+    r, d = W.shape
+    G = 1 if group == -1 else d // max(group, 1)
+    dev = W.device
+    out = dict(outputs or {})
+    qweight = out.get("qweight")
+    if qweight is None:
+        qweight = torch.empty((r, d * bits // 32), dtype=torch.int32, device=dev)
+    scales = out.get("scales")
+    if scales is None:
+        scales = torch.empty((r, G), dtype=torch.float32, device=dev)
+    zeros = out.get("zeros")
+    if zeros is None:
+        zeros = torch.empty((r, G), dtype=torch.int32, device=dev)
+    need = lib.gptq_quantize_workspace_bytes(r, d, bits, group, block, int(act_order))
+    if need == 0 and r > 0:
+        raise GPTQError(1, "gptq_quantize_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    loss = ctypes.c_double(0.0)
+    _check(lib.gptq_quantize_layer(
+        _ptr(W, torch.float32, "W"), r, d, _ptr(H, torch.float32, "H"), bits, group, block,
+        float(damp), int(act_order), _ptr(W_hat, torch.float32, "W_hat"),
+        _ptr(qweight, torch.int32, "qweight"), _ptr(scales, torch.float32, "scales"),
+        _ptr(zeros, torch.int32, "zeros"), _ptr(g_idx, torch.int32, "g_idx"),
+        _ptr(codes, torch.uint8, "codes"), ctypes.byref(loss), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "gptq_quantize_layer")
+    res = {"qweight": qweight, "scales": scales, "zeros": zeros, "loss": loss.value}
+    if W_hat is not None:
+        res["W_hat"] = W_hat
+    if codes is not None:
+        res["codes"] = codes
+    if g_idx is not None:
+        res["g_idx"] = g_idx
+    return res
+
+
+def gptq_pack(codes: torch.Tensor, bits: int, qweight: torch.Tensor | None = None,
+              stream=None) -> torch.Tensor:
+    lib = _abi.load()
+    r, d = codes.shape
+    if qweight is None:
+        qweight = torch.empty((r, d * bits // 32), dtype=torch.int32, device=codes.device)
+    _check(lib.gptq_pack(_ptr(codes, torch.uint8, "codes"), r, d, bits,
+                         _ptr(qweight, torch.int32, "qweight"), _stream(stream)), "gptq_pack")
+    return qweight
+
+
+def gptq_layer_host_workspace_bytes(r: int, d: int, n: int, bits: int, group: int,
+                                    block: int = 128, act_order: bool = False) -> int:
+    return int(_abi.load().gptq_layer_host_workspace_bytes(r, d, n, bits, group, block,
+                                                           int(act_order)))
+
+
+def gptq_solve_layer_host(X: torch.Tensor, W: torch.Tensor, *, bits: int, group: int,
+                          block: int = 128, damp: float = 0.01, act_order: bool = False,
+                          dev_workspace: torch.Tensor, outputs: dict, stream=None) -> float:
+    """Whole layer from host (CPU, ideally pinned) tensors; fills ``outputs`` host tensors."""
+    lib = _abi.load()
+    n, d = X.shape
+    r = W.shape[0]
+    for t, name in ((X, "X"), (W, "W")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor")
+    if X.dtype != torch.float16 or W.dtype != torch.float32:
+        raise ValueError("X must be float16 and W float32")
+    loss = ctypes.c_double(0.0)
+    gi = outputs.get("g_idx")
+    _check(lib.gptq_solve_layer_host(
+        X.data_ptr(), n, W.data_ptr(), r, d, bits, group, block, float(damp), int(act_order),
+        outputs["qweight"].data_ptr(), outputs["scales"].data_ptr(), outputs["zeros"].data_ptr(),
+        gi.data_ptr() if gi is not None else None, ctypes.byref(loss),
+        _ptr(dev_workspace, None, "dev_workspace"),
+        dev_workspace.numel() * dev_workspace.element_size(), _stream(stream)),
+        "gptq_solve_layer_host")
+    return loss.value
+
+
+def gptq_check_device_status(stream=None) -> int:
+    return int(_abi.load().gptq_check_device_status(_stream(stream)))
+
+
+def gptq_launch_count() -> int:
+    return int(_abi.load().gptq_launch_count())
+
+
+def gptq_set_phase_timing(enable: bool) -> None:
+    _abi.load().gptq_set_phase_timing(int(enable))
+
+
+def gptq_last_phase_ms() -> list[float]:
+    buf = (ctypes.c_float * 4)()
+    n = _abi.load().gptq_last_phase_ms(buf, 4)
+    return [float(buf[i]) for i in range(n)]

@@ -1,0 +1,98 @@
+"""The C-ABI library loads on a machine without a GPU and exports the header.
+
+Only host-side logic is exercised here: symbol presence, status strings,
+workspace size queries and argument validation (which returns before any CUDA
+call).  Compute is covered by the GPU tests.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from post_weight_quantization_19_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    with open(os.path.join(ROOT, "include", "gptq.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gptq_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _header_functions()
+    assert len(names) >= 11
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(_abi.SIGNATURES) == names
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.gptq_status_string(code)
+    assert lib.gptq_status_string(999) == b"unknown status"
+
+
+def test_workspace_query(lib):
+    ws = lib.gptq_quantize_workspace_bytes
+    base = ws(4096, 4096, 4, 128, 128, 0)
+    # working copy of W, superblock errors, codes, and the recursion scratch
+    assert base >= 4096 * 4096 * 4 + 4096 * 1024 * 4 + 4096 * 4096 + 2048 * 2048 * 4
+    assert ws(4096, 4096, 4, 128, 128, 1) >= base + 4096 * 4096 * 4   # permuted H
+    assert base % 256 == 0
+    for bad in [(16, 100, 4, -1, 128, 0),      # d % 32
+                (16, 256, 5, -1, 128, 0),      # bits
+                (16, 256, 4, 48, 128, 0),      # group not a divisor of the block
+                (16, 256, 4, 96, 128, 0),
+                (16, 256, 4, -1, 96, 0),       # block
+                (-1, 256, 4, -1, 128, 0)]:
+        assert ws(*bad) == 0, bad
+    hw = lib.gptq_layer_host_workspace_bytes(128, 256, 2048, 4, -1, 128, 0)
+    assert hw >= 2048 * 256 * 2 + 256 * 256 * 4 + 128 * 256 * 4
+
+
+def test_validation_returns_before_cuda(lib):
+    p = ctypes.c_void_p(4096)   # never dereferenced: validation fails first
+    loss = ctypes.c_double(-1)
+    q = lib.gptq_quantize_layer
+    # bits
+    assert q(p, 8, 256, p, 5, -1, 128, 0.01, 0, None, p, p, p, None, None,
+             ctypes.byref(loss), p, 1 << 30, None) == 1
+    # damp negative / NaN
+    assert q(p, 8, 256, p, 4, -1, 128, -1.0, 0, None, p, p, p, None, None,
+             ctypes.byref(loss), p, 1 << 30, None) == 1
+    assert q(p, 8, 256, p, 4, -1, 128, float("nan"), 0, None, p, p, p, None, None,
+             ctypes.byref(loss), p, 1 << 30, None) == 1
+    # missing output pointer
+    assert q(p, 8, 256, p, 4, -1, 128, 0.01, 0, None, None, p, p, None, None,
+             ctypes.byref(loss), p, 1 << 30, None) == 1
+    # workspace too small
+    ws = ctypes.c_void_p(1 << 20)
+    assert q(p, 8, 256, p, 4, -1, 128, 0.01, 0, None, p, p, p, None, None,
+             ctypes.byref(loss), ws, 1024, None) == 4
+    # empty layer: OK, loss 0, nothing enqueued
+    assert q(p, 0, 256, p, 4, -1, 128, 0.01, 0, None, p, p, p, None, None,
+             ctypes.byref(loss), p, 0, None) == 0
+    assert loss.value == 0.0
+    h = lib.gptq_hessian_accumulate
+    assert h(p, 10, 100, 100, p, None) == 1          # d % 32
+    assert h(p, 10, 128, 100, p, None) == 1          # ldx < d
+    assert h(ctypes.c_void_p(4098), 10, 128, 128, p, None) == 1   # X not 16-byte aligned
+    assert h(p, -1, 128, 128, p, None) == 1
+    assert h(p, 0, 128, 128, p, None) == 0           # no tokens: nothing to do
+    assert lib.gptq_pack(p, 4, 100, 4, p, None) == 1
+    assert lib.gptq_pack(p, 4, 128, 6, p, None) == 1
+
+
+def test_no_kernels_launched_on_cpu(lib):
+    assert lib.gptq_launch_count() == 0
+
+
+def test_library_is_in_tree():
+    path = _abi.library_path()
+    assert path.startswith(os.path.join(ROOT, "post_weight_quantization_19_b200"))
+    assert os.path.exists(path)

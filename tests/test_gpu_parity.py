@@ -1,0 +1,221 @@
+"""CUDA path vs the float64 oracle on seeded inputs (needs a B200).
+
+Every call goes through the C ABI (via the thin torch binding).  Sizes span
+several tiles with ragged tails; full-size layers are compared on sampled rows.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from parity_util import (H_REL_FRO, assert_codes_close, check_against_oracle, gpu_layer,
+                         rel_fro)
+from synth import make_activations, make_problem, make_weights, workload, workload_inputs
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import post_weight_quantization_19_b200 as g
+    yield g
+    assert g.gptq_check_device_status() == 0
+
+
+def _hessian_gpu(X):
+    import post_weight_quantization_19_b200 as g
+    d = X.shape[1]
+    H = torch.zeros((d, d), dtype=torch.float32, device="cuda")
+    g.gptq_hessian_accumulate(torch.from_numpy(X).cuda(), H)
+    torch.cuda.synchronize()
+    return H.cpu().numpy()
+
+
+# ------------------------------------------------------------------ Hessian
+
+@pytest.mark.parametrize("n,d", [(2048, 256), (1000, 160), (777, 96), (20000, 640), (64, 32),
+                                 (5000, 416)])
+def test_hessian_matches_oracle(n, d):
+    X = make_activations(n, d, sigma=1.0, outlier_frac=0.001, outlier_mult=50.0, seed=n + d)
+    H = _hessian_gpu(X)
+    assert rel_fro(H, oracle.hessian(X)) <= H_REL_FRO
+    np.testing.assert_array_equal(H, H.T)
+
+
+def test_hessian_small_integers_are_exact():
+    # Integer activations: products and partial sums are exact in fp32, so the
+    # tensor-core result must equal the exact Hessian bit for bit.
+    rng = np.random.default_rng(5)
+    X = rng.integers(-6, 7, size=(3000, 288)).astype(np.float16)
+    np.testing.assert_array_equal(_hessian_gpu(X), oracle.hessian(X))
+
+
+def test_hessian_accumulates_over_calls():
+    import post_weight_quantization_19_b200 as g
+    X = make_activations(4000, 256, seed=3)
+    H0 = oracle.hessian(make_activations(50, 256, seed=4)).astype(np.float32)
+    H = torch.from_numpy(H0.copy()).cuda()
+    Xd = torch.from_numpy(X).cuda()
+    g.gptq_hessian_accumulate(Xd[:1500], H)
+    g.gptq_hessian_accumulate(Xd[1500:], H)
+    torch.cuda.synchronize()
+    assert rel_fro(H.cpu().numpy(), H0.astype(np.float64) + oracle.hessian(X)) <= H_REL_FRO
+
+
+def test_hessian_no_tokens_is_a_no_op():
+    import post_weight_quantization_19_b200 as g
+    H = torch.full((64, 64), 3.0, device="cuda")
+    g.gptq_hessian_accumulate(torch.zeros((0, 64), dtype=torch.float16, device="cuda"), H)
+    torch.cuda.synchronize()
+    assert bool((H == 3.0).all())
+
+
+# ------------------------------------------------------------------ the solve
+
+SOLVE_CASES = [
+    # r, d, n, bits, group, block, act_order
+    (128, 256, 2048, 4, -1, 128, False),
+    (64, 512, 4096, 4, 128, 128, False),
+    (37, 384, 3000, 3, 128, 128, False),
+    (50, 256, 2048, 4, 32, 128, False),
+    (40, 256, 2048, 4, 64, 64, False),
+    (33, 512, 4096, 3, 256, 128, False),
+    (64, 256, 2048, 2, -1, 32, False),
+    (64, 256, 2048, 8, 128, 128, False),
+    (48, 384, 3000, 4, 128, 128, True),
+    (48, 256, 2048, 3, -1, 128, True),
+    (16, 160, 1500, 4, 32, 128, False),      # ragged last block
+    (1, 96, 500, 4, -1, 64, False),           # single row, ragged
+    (200, 2176, 8192, 4, 128, 128, False),    # several superblocks + a ragged one
+]
+
+
+@pytest.mark.parametrize("case", SOLVE_CASES, ids=lambda c: "r{}_d{}_b{}_g{}_B{}_a{}".format(
+    c[0], c[1], c[3], c[4], c[5], int(c[6])))
+def test_solve_matches_oracle_given_same_H(case):
+    # The solve alone: both sides start from the same fp32 Hessian values.
+    r, d, n, bits, group, block, act = case
+    X, W = make_problem(r, d, n, seed=r * 7 + d)
+    H32 = oracle.hessian(X).astype(np.float32)
+    got = gpu_layer(None, W, bits=bits, group=group, block=block, act_order=act, H32=H32)
+    ref = oracle.gptq_quantize_layer(W, H32.astype(np.float64), bits=bits, group=group,
+                                     block=block, act_order=act)
+    check_against_oracle(got, ref, W, bits=bits, group=group)
+
+
+@pytest.mark.parametrize("case", SOLVE_CASES[:4] + SOLVE_CASES[8:9],
+                         ids=lambda c: "r{}_d{}_g{}_a{}".format(c[0], c[1], c[4], int(c[6])))
+def test_full_path_matches_oracle(case):
+    # Hessian + solve on the GPU against Hessian + solve in float64.
+    r, d, n, bits, group, block, act = case
+    X, W = make_problem(r, d, n, seed=r * 11 + d)
+    got = gpu_layer(X, W, bits=bits, group=group, block=block, act_order=act)
+    H = oracle.hessian(X)
+    assert rel_fro(got["H"], H) <= H_REL_FRO
+    ref = oracle.gptq_quantize_layer(W, H, bits=bits, group=group, block=block, act_order=act)
+    check_against_oracle(got, ref, W, bits=bits, group=group)
+
+
+def test_tiny_workload_end_to_end():
+    wl = workload("tiny_128x256")
+    X, W = workload_inputs(wl)
+    got = gpu_layer(X, W, bits=wl.bits, group=wl.group, block=wl.block, damp=wl.damp,
+                    act_order=wl.act_order)
+    H = oracle.hessian(X)
+    assert rel_fro(got["H"], H) <= H_REL_FRO
+    ref = oracle.gptq_quantize_layer(W, H, bits=wl.bits, group=wl.group, block=wl.block,
+                                     damp=wl.damp, act_order=wl.act_order)
+    stats = check_against_oracle(got, ref, W, bits=wl.bits, group=wl.group)
+    # the reported loss is the layer objective of the GPU's own output
+    assert got["loss"] == pytest.approx(oracle.layer_loss(W, got["W_hat"], H), rel=1e-4)
+    assert stats["code_match"] >= 0.999
+
+
+def test_identity_hessian_gives_rtn_on_gpu():
+    # H proportional to I: no compensation, codes are round-to-nearest.
+    _, W = make_problem(64, 256, 1, seed=9)
+    got = gpu_layer(None, W, bits=4, group=64, H32=np.eye(256, dtype=np.float32) * 3.0)
+    codes, _ = oracle.rtn(W, 4, 64)
+    assert_codes_close(got["codes"], codes, frac=0.9999)
+
+
+def test_deterministic():
+    X, W = make_problem(64, 512, 4096, seed=21)
+    a = gpu_layer(X, W, bits=4, group=128)
+    b = gpu_layer(X, W, bits=4, group=128)
+    for k in ("H", "codes", "qweight", "scales", "zeros", "W_hat"):
+        np.testing.assert_array_equal(a[k], b[k])
+    assert a["loss"] == b["loss"]
+
+
+# ------------------------------------------------------------------ pack
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("r,d", [(1, 32), (7, 96), (64, 4096)])
+def test_pack_bit_exact(bits, r, d):
+    import post_weight_quantization_19_b200 as g
+    codes = np.random.default_rng(bits * 100 + r).integers(0, 1 << bits, size=(r, d),
+                                                           dtype=np.uint8)
+    q = g.gptq_pack(torch.from_numpy(codes).cuda(), bits)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(q.cpu().numpy(), oracle.pack_rows(codes, bits))
+
+
+# ------------------------------------------------------------------ errors and edges
+
+def test_not_positive_definite_is_reported():
+    import post_weight_quantization_19_b200 as g
+    W = torch.zeros((8, 64), device="cuda")
+    for H in (-torch.eye(64, device="cuda"), torch.zeros((64, 64), device="cuda")):
+        with pytest.raises(g.GPTQError) as e:
+            g.gptq_quantize_layer(W, H, bits=4, group=-1, damp=0.0)
+        assert e.value.status == 2
+
+
+def test_empty_layer_and_single_row():
+    import post_weight_quantization_19_b200 as g
+    H = torch.eye(64, device="cuda")
+    res = g.gptq_quantize_layer(torch.zeros((0, 64), device="cuda"), H, bits=4, group=-1)
+    assert res["loss"] == 0.0
+    W = make_weights(1, 64, seed=1)
+    got = gpu_layer(None, W, bits=4, group=32, H32=np.eye(64, dtype=np.float32))
+    codes, _ = oracle.rtn(W, 4, 32)
+    np.testing.assert_array_equal(got["codes"], codes)
+
+
+def test_host_buffer_entry_point_matches_device_path():
+    import post_weight_quantization_19_b200 as g
+    wl = workload("tiny_128x256")
+    X, W = workload_inputs(wl)
+    dev = gpu_layer(X, W, bits=wl.bits, group=wl.group)
+    r, d = W.shape
+    n = X.shape[0]
+    ws = torch.empty(g.gptq_layer_host_workspace_bytes(r, d, n, wl.bits, wl.group),
+                     dtype=torch.uint8, device="cuda")
+    out = {"qweight": torch.empty((r, d * wl.bits // 32), dtype=torch.int32).pin_memory(),
+           "scales": torch.empty((r, 1), dtype=torch.float32).pin_memory(),
+           "zeros": torch.empty((r, 1), dtype=torch.int32).pin_memory()}
+    loss = g.gptq_solve_layer_host(torch.from_numpy(X).pin_memory(),
+                                   torch.from_numpy(W).pin_memory(), bits=wl.bits,
+                                   group=wl.group, dev_workspace=ws, outputs=out)
+    np.testing.assert_array_equal(out["qweight"].numpy(), dev["qweight"])
+    np.testing.assert_array_equal(out["scales"].numpy(), dev["scales"])
+    np.testing.assert_array_equal(out["zeros"].numpy(), dev["zeros"])
+    assert loss == dev["loss"]
+
+
+def test_workspace_too_small_is_reported():
+    import post_weight_quantization_19_b200 as g
+    W = torch.zeros((8, 64), device="cuda")
+    with pytest.raises(g.GPTQError) as e:
+        g.gptq_quantize_layer(W, torch.eye(64, device="cuda"), bits=4, group=-1,
+                              workspace=torch.empty(1024, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == 4
+
+
+def test_kernels_were_launched():
+    import post_weight_quantization_19_b200 as g
+    assert g.gptq_launch_count() > 0
