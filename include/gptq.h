@@ -57,7 +57,7 @@ const char *gptq_status_string(int status);
  *   X    device, fp16 (IEEE binary16 bits), [n x d] row-major with leading
  *        dimension ldx (elements): row t is the activation vector of token t.
  *        16-byte aligned; ldx >= d and ldx % 8 == 0.
- *   n    number of tokens, n >= 0 (n == 0 enqueues nothing).
+ *   n    number of tokens, n >= 0 (n == 0 enqueues nothing; X may then be NULL).
  *   d    input features, d > 0 and d % 32 == 0.
  *   H    device, fp32 [d x d] row-major (leading dimension d), 16-byte aligned.
  *        On return (stream order) H = sym(upper(H_in) + 2 X^T X): the upper
@@ -177,6 +177,13 @@ int gptq_solve_layer_host(const uint16_t *X_host, int64_t n, const float *W_host
  * such as the Hessian, gave up on a bounded wait; GPTQ_OK otherwise).
  */
 int gptq_check_device_status(gptq_stream_t stream);
+
+/*
+ * Text describing the last CUDA failure seen by this thread ("" if none):
+ * source location, the failing call and the CUDA error name.  Valid until the
+ * next failure on the same thread.
+ */
+const char *gptq_last_error(void);
 
 /* Number of kernels this library has launched in this process (all devices). */
 uint64_t gptq_launch_count(void);

@@ -37,6 +37,7 @@ SIGNATURES = {
                                       c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "gptq_check_device_status": (c_int, [c_void_p]),
     "gptq_launch_count": (ctypes.c_uint64, []),
+    "gptq_last_error": (ctypes.c_char_p, []),
     "gptq_set_phase_timing": (c_int, [c_int]),
     "gptq_last_phase_ms": (c_int, [c_void_p, c_int]),
 }

@@ -1,5 +1,6 @@
 // C-ABI entry points of the layer solve: validation, workspace layout, and the
 // stream-ordered sequence of kernels (see include/gptq.h for the contract).
+#include <stdio.h>
 #include <string.h>
 
 #include "gptq_internal.h"
@@ -7,6 +8,21 @@
 namespace gptq {
 
 std::atomic<uint64_t> g_launches{0};
+
+namespace {
+thread_local char g_last_error[512] = "";
+}
+
+void set_last_error(const char *file, int line, const char *what, cudaError_t e) {
+  const char *base = strrchr(file, '/');
+  snprintf(g_last_error, sizeof(g_last_error), "%s:%d %s: %s (%s)", base ? base + 1 : file, line,
+           what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+void set_last_error_msg(const char *file, int line, const char *msg) {
+  const char *base = strrchr(file, '/');
+  snprintf(g_last_error, sizeof(g_last_error), "%s:%d %s", base ? base + 1 : file, line, msg);
+}
 
 namespace {
 
@@ -102,6 +118,8 @@ extern "C" const char *gptq_status_string(int status) {
 }
 
 extern "C" uint64_t gptq_launch_count(void) { return g_launches.load(); }
+
+extern "C" const char *gptq_last_error(void) { return g_last_error; }
 
 extern "C" int gptq_set_phase_timing(int enable) {
   g_timing = enable != 0;

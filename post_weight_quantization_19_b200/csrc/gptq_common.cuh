@@ -19,19 +19,28 @@ extern std::atomic<uint64_t> g_launches;
 
 inline void count_launch(uint64_t k = 1) { g_launches.fetch_add(k, std::memory_order_relaxed); }
 
-#define GPTQ_CUDA_TRY(expr)                         \
-  do {                                              \
-    cudaError_t e_ = (expr);                        \
-    if (e_ != cudaSuccess) return GPTQ_ERR_CUDA;    \
+// Remember which CUDA call failed (file:line, error name) for gptq_last_error().
+void set_last_error(const char *file, int line, const char *what, cudaError_t e);
+void set_last_error_msg(const char *file, int line, const char *msg);
+
+#define GPTQ_CUDA_TRY(expr)                                          \
+  do {                                                               \
+    cudaError_t e_ = (expr);                                         \
+    if (e_ != cudaSuccess) {                                         \
+      ::gptq::set_last_error(__FILE__, __LINE__, #expr, e_);         \
+      return GPTQ_ERR_CUDA;                                          \
+    }                                                                \
   } while (0)
 
-#define GPTQ_LAUNCH_CHECK()                                 \
-  do {                                                      \
-    ::gptq::count_launch();                                 \
-    if (cudaPeekAtLastError() != cudaSuccess) {             \
-      (void)cudaGetLastError();                             \
-      return GPTQ_ERR_CUDA;                                 \
-    }                                                       \
+#define GPTQ_LAUNCH_CHECK()                                          \
+  do {                                                               \
+    ::gptq::count_launch();                                          \
+    cudaError_t e_ = cudaPeekAtLastError();                          \
+    if (e_ != cudaSuccess) {                                         \
+      (void)cudaGetLastError();                                      \
+      ::gptq::set_last_error(__FILE__, __LINE__, "kernel launch", e_); \
+      return GPTQ_ERR_CUDA;                                          \
+    }                                                                \
   } while (0)
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -180,6 +189,19 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32
         "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]), "=r"(u[19]),
         "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]), "=r"(u[25]),
         "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// 32 lanes x 16 columns of 32-bit TMEM -> 16 registers per thread.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, float (&v)[16]) {
+  uint32_t *u = reinterpret_cast<uint32_t *>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+        "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]),
+        "=r"(u[14]), "=r"(u[15])
       : "r"(taddr)
       : "memory");
 }

@@ -86,7 +86,7 @@ __device__ __forceinline__ void record_timeout(int *status, HessShared &sh) {
   *(volatile int *)&sh.abort = 1;
 }
 
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(THREADS, 1)
     hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, int64_t n, int d,
                       float *__restrict__ H, int *__restrict__ status) {
   extern __shared__ uint8_t dyn_smem[];
@@ -239,12 +239,12 @@ __global__ void __maxnreg__(200)
         tc_fence_after();
         const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + abuf * HN + half * 128;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          float v[32];
-          tmem_ld_32x32b_x32(base + p * 32, v);
+        for (int p = 0; p < 8; ++p) {
+          float v[16];
+          tmem_ld_32x32b_x16(base + p * 16, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[p * 32 + i] += v[i];
+          for (int i = 0; i < 16; ++i) acc[p * 16 + i] += v[i];
         }
         tc_fence_before();
         __syncwarp();
@@ -304,16 +304,19 @@ using namespace gptq;
 
 extern "C" int gptq_hessian_accumulate(const void *X, int64_t n, int64_t d, int64_t ldx, float *H,
                                        gptq_stream_t stream) {
-  if (!X || !H) return GPTQ_ERR_INVALID_ARG;
   if (n < 0 || n > (int64_t)INT32_MAX) return GPTQ_ERR_INVALID_ARG;
   if (d <= 0 || d % 32 != 0 || d > 65536) return GPTQ_ERR_INVALID_ARG;
   if (ldx < d || ldx % 8 != 0) return GPTQ_ERR_INVALID_ARG;
+  if (n == 0) return GPTQ_OK;  // nothing to add; X may be NULL
+  if (!X || !H) return GPTQ_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(X) % 16 != 0 || reinterpret_cast<uintptr_t>(H) % 16 != 0)
     return GPTQ_ERR_INVALID_ARG;
-  if (n == 0) return GPTQ_OK;
 
   EncodeTiledFn enc = encode_fn();
-  if (!enc) return GPTQ_ERR_CUDA;
+  if (!enc) {
+    set_last_error_msg(__FILE__, __LINE__, "cuTensorMapEncodeTiled entry point not available");
+    return GPTQ_ERR_CUDA;
+  }
   CUtensorMap tmap;
   const cuuint64_t gdim[2] = {(cuuint64_t)d, (cuuint64_t)n};
   const cuuint64_t gstride[1] = {(cuuint64_t)ldx * 2};
@@ -321,11 +324,16 @@ extern "C" int gptq_hessian_accumulate(const void *X, int64_t n, int64_t d, int6
   const cuuint32_t estride[2] = {1, 1};
   if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(X), gdim, gstride, box,
           estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+    set_last_error_msg(__FILE__, __LINE__, "cuTensorMapEncodeTiled rejected the X descriptor");
     return GPTQ_ERR_CUDA;
+  }
 
   int *status = device_status_word();
-  if (!status) return GPTQ_ERR_CUDA;
+  if (!status) {
+    set_last_error_msg(__FILE__, __LINE__, "cudaGetSymbolAddress of the status word failed");
+    return GPTQ_ERR_CUDA;
+  }
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(hessian_tc_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES));
   const int nI = (int)((d + HM - 1) / HM), nJ = (int)((d + HN - 1) / HN);

@@ -18,7 +18,9 @@ class GPTQError(RuntimeError):
     def __init__(self, status: int, where: str):
         lib = _abi.load()
         msg = lib.gptq_status_string(status).decode()
-        super().__init__(f"{where}: {_abi.STATUS.get(status, status)} ({msg})")
+        detail = lib.gptq_last_error().decode() if status == 3 else ""
+        super().__init__(f"{where}: {_abi.STATUS.get(status, status)} ({msg})"
+                         + (f": {detail}" if detail else ""))
         self.status = status
 
 
