@@ -150,6 +150,37 @@ int gptq_pack(const uint8_t *codes, int64_t r, int64_t d, int bits, int32_t *qwe
               gptq_stream_t stream);
 
 /*
+ * gptq_quantize_layer_noalloc -- gptq_quantize_layer for callers that cannot
+ * allocate device memory.  (The GPTQ pages have no counterpart: this is a
+ * deployment convenience of this library, not a step of the method.)
+ *
+ * Some callers cannot call cudaMalloc -- they run inside a memory pool that
+ * forbids side allocations, or their runtime has reserved the whole device in
+ * advance, or they can hand over only inputs and outputs.  This entry point
+ * takes its scratch from a fixed array of GPTQ_NOALLOC_SCRATCH_BYTES bytes in
+ * the library's own device memory instead of a workspace argument; every GPU
+ * that loads the library holds that array until the process exits.  It calls
+ * no allocator of any kind.
+ *
+ *   Arguments, results and synchronisation are those of gptq_quantize_layer
+ *   without the workspace pair.
+ *   Limit: returns GPTQ_ERR_NO_MEMORY (nothing enqueued) when
+ *   gptq_quantize_workspace_bytes(r, d, bits, group, block, act_order) exceeds
+ *   GPTQ_NOALLOC_SCRATCH_BYTES -- e.g. r = d = 2048 fits, r = d = 4096 does not.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.  All calls share the one array, and each call leaves its contents
+ *   behind; the next call clears what it needs cleared.  Calls whose work may
+ *   overlap on the GPU (different streams or threads without ordering) race on
+ *   the array: serialise them.
+ */
+#define GPTQ_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+int gptq_quantize_layer_noalloc(const float *W, int64_t r, int64_t d, float *H, int bits,
+                                int group, int block, float damp, int act_order, float *W_hat,
+                                int32_t *qweight, float *scales, int32_t *zeros, int32_t *g_idx,
+                                uint8_t *codes, double *loss, gptq_stream_t stream);
+
+/*
  * gptq_layer_host_workspace_bytes / gptq_solve_layer_host -- the whole layer
  * from HOST buffers: copy X and W to the device, H = 2 X^T X, quantise, pack,
  * and copy qweight, scales, zeros, g_idx and the loss back.

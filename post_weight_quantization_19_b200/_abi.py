@@ -30,6 +30,9 @@ SIGNATURES = {
                                     c_float, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "gptq_pack": (c_int, [c_void_p, c_int64, c_int64, c_int, c_void_p, c_void_p]),
+    "gptq_quantize_layer_noalloc": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int, c_int,
+                                            c_int, c_float, c_int, c_void_p, c_void_p, c_void_p,
+                                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "gptq_layer_host_workspace_bytes": (c_size_t, [c_int64, c_int64, c_int64, c_int, c_int, c_int,
                                                    c_int]),
     "gptq_solve_layer_host": (c_int, [c_void_p, c_int64, c_void_p, c_int64, c_int64, c_int, c_int,

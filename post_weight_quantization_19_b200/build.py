@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgptq_b200.so")
-SOURCES = ["hessian_tc.cu", "factor.cu", "sweep.cu", "pack.cu", "api.cu"]
+SOURCES = ["hessian_tc.cu", "factor.cu", "sweep.cu", "pack.cu", "api.cu", "noalloc.cu"]
 
 
 def nvcc() -> str:
