@@ -101,7 +101,8 @@ size_t gptq_quantize_workspace_bytes(int64_t r, int64_t d, int bits, int group, 
  *      undamped H, evaluated as sum_j 1/2 e_j^2 - lambda/2 ||D||_F^2.
  *   6. Codes are returned in the original column order and packed.
  *
- *   W         device fp32 [r x d], read only.
+ *   W         device fp32 [r x d], read only.  W, H, W_hat and g_idx must be
+ *             16-byte aligned; codes, qweight, scales and zeros 4-byte aligned.
  *   r, d      r >= 0 (r == 0: returns GPTQ_OK with *loss = 0, enqueues nothing),
  *             d > 0, d % 32 == 0.
  *   H         device fp32 [d x d], full symmetric (as written by

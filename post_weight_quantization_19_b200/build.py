@@ -15,7 +15,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgptq_b200.so")
-SOURCES = ["hessian_tc.cu", "factor.cu", "sweep.cu", "pack.cu", "api.cu", "noalloc.cu"]
+SOURCES = ["hessian_tc.cu", "gemm_tc.cu", "factor.cu", "leaf.cu", "sweep.cu", "pack.cu", "api.cu",
+           "noalloc.cu"]
 
 
 def nvcc() -> str:

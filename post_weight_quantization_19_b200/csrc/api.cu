@@ -169,7 +169,8 @@ extern "C" int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *
       reinterpret_cast<uintptr_t>(workspace) % 256 ||
       (W_hat && reinterpret_cast<uintptr_t>(W_hat) % 16) ||
       reinterpret_cast<uintptr_t>(qweight) % 4 || reinterpret_cast<uintptr_t>(scales) % 4 ||
-      reinterpret_cast<uintptr_t>(zeros) % 4 || (g_idx && reinterpret_cast<uintptr_t>(g_idx) % 4))
+      reinterpret_cast<uintptr_t>(zeros) % 4 || (g_idx && reinterpret_cast<uintptr_t>(g_idx) % 16) ||
+      (codes && reinterpret_cast<uintptr_t>(codes) % 4))
     return GPTQ_ERR_INVALID_ARG;
   const Layout L = layout(r, d, group, block, act_order);
   if (workspace_bytes < L.total) return GPTQ_ERR_NO_MEMORY;

@@ -1,0 +1,341 @@
+// fp32 GEMM on the sm_100a tensor cores with error-compensated TF32 (3xTF32).
+//
+//   C = alpha * A * op(B) + beta * C     (row-major fp32; op(B) = B or B^T)
+//
+// Used by the trailing (lazy-batch) updates of the column sweep and by the
+// block recursion that forms U -- the dense contractions of the layer solve
+// (GPTQ reading card, 方法适配: the deferred global update is a matrix product).
+//
+// Each fp32 operand x is split as hi = tf32(x) (round to nearest) and
+// lo = tf32(x - hi); the product is hi*hi + hi*lo + lo*hi, three
+// tcgen05.mma.kind::tf32 per K step accumulating in TMEM, which keeps about
+// 21 bits of each operand (the dropped lo*lo term is ~2^-22 relative).
+//
+// Tile 128 x 128 x 32 per stage, 3-stage TMA ring.  A (and B^T) are K-major
+// with a 128-byte swizzle; a row-major B is consumed MN-major with the
+// 128-byte swizzle of 32-byte atoms (the only MN-major layout for tf32).  Warp 0 issues
+// TMA, warp 1 issues UMMA, warps 2..5 split each landed stage into hi/lo in
+// shared memory and afterwards drain the TMEM accumulator into C.
+#include <mutex>
+
+#include "gptq_internal.h"
+
+namespace gptq {
+namespace {
+
+constexpr int TM = 128, TN = 128, TK = 32;
+constexpr int STAGES = 3;
+constexpr int TILE_BYTES = 128 * TK * 4;   // 16 KB: 128 rows x 32 fp32
+constexpr int STAGE_BYTES = 4 * TILE_BYTES; // A, B, A_lo, B_lo
+constexpr int THREADS = 32 * 6;
+constexpr int CONV_THREADS = 128;
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024;
+
+struct TcShared {
+  uint64_t full[STAGES];
+  uint64_t conv[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t accf;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct TcArgs {
+  int M, N, K;
+  float *C;
+  int64_t ldc;
+  float alpha, beta;
+  int flags;
+  int trans_b;
+  const int *status;
+  int *dev_status;
+};
+
+__device__ __forceinline__ uint32_t tf32_rn(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void fail_timeout(TcShared &sh, int *dev_status) {
+  if (dev_status) atomicCAS(dev_status, 0, (int)GPTQ_ERR_TIMEOUT);
+  *(volatile int *)&sh.abort = 1;
+}
+
+// hi/lo split of one 16 KB tile in place: x -> tf32(x), lo <- tf32(x - tf32(x)).
+__device__ __forceinline__ void split_tile(uint8_t *tile, uint8_t *lo, int t) {
+  float4 *p = reinterpret_cast<float4 *>(tile);
+  float4 *q = reinterpret_cast<float4 *>(lo);
+#pragma unroll 4
+  for (int i = t; i < TILE_BYTES / 16; i += CONV_THREADS) {
+    float4 v = p[i];
+    float4 h, l;
+    h.x = __uint_as_float(tf32_rn(v.x));
+    h.y = __uint_as_float(tf32_rn(v.y));
+    h.z = __uint_as_float(tf32_rn(v.z));
+    h.w = __uint_as_float(tf32_rn(v.w));
+    l.x = __uint_as_float(tf32_rn(v.x - h.x));
+    l.y = __uint_as_float(tf32_rn(v.y - h.y));
+    l.z = __uint_as_float(tf32_rn(v.z - h.z));
+    l.w = __uint_as_float(tf32_rn(v.w - h.w));
+    p[i] = h;
+    q[i] = l;
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   TcArgs g) {
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ TcShared sh;
+  if (g.status && *(volatile const int *)g.status) return;
+  const int bn = blockIdx.x, bm = blockIdx.y;
+  if ((g.flags & GEMM_UPPER_C) && bn < bm) return;
+  const int m0 = bm * TM, n0 = bn * TN;
+  int klo = 0, khi = g.K;
+  if (g.flags & GEMM_KMIN_ROW) klo = max(klo, m0);
+  if (g.flags & GEMM_KMIN_COL) klo = max(klo, n0);
+  if (g.flags & GEMM_KMAX_COL) khi = min(khi, n0 + TN);
+  const int nk = khi > klo ? (khi - klo) / TK : 0;
+
+  uint8_t *smem =
+      reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.conv[s], CONV_THREADS / 32);
+      mbar_init(&sh.empty[s], 1);
+    }
+    mbar_init(&sh.accf, 1);
+    mbar_init(&sh.drain, 1);
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, TN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t issued = 0, issued_par = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (kb / STAGES) & 1;
+        if (*(volatile int *)&sh.abort) break;
+        if (!mbar_wait_bounded(&sh.empty[s], ph ^ 1)) {
+          fail_timeout(sh, g.dev_status);
+          break;
+        }
+        uint8_t *st = smem + (size_t)s * STAGE_BYTES;
+        const int k0 = klo + kb * TK;
+        mbar_arrive_expect_tx(&sh.full[s], 2 * TILE_BYTES);
+        tma_load_2d(st, &tmA, k0, m0, &sh.full[s]);
+        if (g.trans_b) {
+          tma_load_2d(st + TILE_BYTES, &tmB, k0, n0, &sh.full[s]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < TN / 32; ++c)
+            tma_load_2d(st + TILE_BYTES + c * (TK * 128), &tmB, n0 + 32 * c, k0, &sh.full[s]);
+        }
+        issued |= 1u << s;
+        issued_par = (issued_par & ~(1u << s)) | (ph << s);
+      }
+      for (int s = 0; s < STAGES; ++s)
+        if (issued & (1u << s)) (void)mbar_wait_bounded(&sh.full[s], (issued_par >> s) & 1u);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = instr_desc(2, 2, 0, g.trans_b ? 0u : 1u, TM, TN);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (kb / STAGES) & 1;
+        if (!mbar_wait_bounded(&sh.conv[s], ph)) {
+          fail_timeout(sh, g.dev_status);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a = smem_u32(smem + (size_t)s * STAGE_BYTES);
+        const uint32_t b = a + TILE_BYTES, al = a + 2 * TILE_BYTES, bl = a + 3 * TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < TK / 8; ++kk) {
+          // A, B^T: K-major, 8 tf32 = 32 bytes per K step inside the swizzle atom.
+          // B row-major: MN-major, 8 K rows (1024 bytes) per K step.
+          const uint64_t ad = smem_desc(a + kk * 32, 16, 1024, 2);
+          const uint64_t ald = smem_desc(al + kk * 32, 16, 1024, 2);
+          uint64_t bd, bld;
+          if (g.trans_b) {
+            bd = smem_desc(b + kk * 32, 16, 1024, 2);
+            bld = smem_desc(bl + kk * 32, 16, 1024, 2);
+          } else {
+            // MN-major tf32 uses the 128-byte swizzle with 32-byte atoms: 4-row K
+            // groups 512 bytes apart, 32-column boxes 4 KB apart.
+            bd = smem_desc(b + kk * 1024, TK * 128, 512, 1);
+            bld = smem_desc(bl + kk * 1024, TK * 128, 512, 1);
+          }
+          const uint32_t acc0 = (kb > 0 || kk > 0) ? 1u : 0u;
+          umma_tf32_ss(tmem, ad, bd, idesc, acc0);
+          umma_tf32_ss(tmem, ad, bld, idesc, 1u);
+          umma_tf32_ss(tmem, ald, bd, idesc, 1u);
+        }
+        umma_commit(&sh.empty[s]);
+      }
+      umma_commit(&sh.accf);
+      umma_commit(&sh.drain);
+      (void)mbar_wait_bounded(&sh.drain, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- split + epilogue
+    const int t = threadIdx.x - 64;
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % STAGES;
+      const uint32_t ph = (kb / STAGES) & 1;
+      if (!mbar_wait_bounded(&sh.full[s], ph)) {
+        if (lane == 0) fail_timeout(sh, g.dev_status);
+        ok = false;
+        break;
+      }
+      uint8_t *st = smem + (size_t)s * STAGE_BYTES;
+      split_tile(st, st + 2 * TILE_BYTES, t);
+      split_tile(st + TILE_BYTES, st + 3 * TILE_BYTES, t);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.conv[s]);
+    }
+    const int quarter = warp & 3;
+    const int row = m0 + quarter * 32 + lane;
+    if (ok && nk > 0) {
+      if (!mbar_wait_bounded(&sh.accf, 0)) {
+        if (lane == 0) fail_timeout(sh, g.dev_status);
+        ok = false;
+      }
+      tc_fence_after();
+    }
+    if (ok) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < TN; c0 += 32) {
+        float v[32];
+        if (nk > 0) {
+          tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + c0, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        }
+        if (row < g.M) {
+          float *cp = g.C + (size_t)row * g.ldc + n0 + c0;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            if (n0 + c0 + i < g.N) {
+              float4 o;
+              if (g.beta != 0.f) {
+                const float4 c = *reinterpret_cast<const float4 *>(cp + i);
+                o.x = fmaf(g.alpha, v[i + 0], g.beta * c.x);
+                o.y = fmaf(g.alpha, v[i + 1], g.beta * c.y);
+                o.z = fmaf(g.alpha, v[i + 2], g.beta * c.z);
+                o.w = fmaf(g.alpha, v[i + 3], g.beta * c.w);
+              } else {
+                o = make_float4(g.alpha * v[i], g.alpha * v[i + 1], g.alpha * v[i + 2],
+                                g.alpha * v[i + 3]);
+              }
+              *reinterpret_cast<float4 *>(cp + i) = o;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TN);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// fp32 row-major view [rows x cols] with leading dimension ld, box {32, box_rows}.
+bool make_map(CUtensorMap *m, const float *base, int64_t rows, int64_t cols, int64_t ld,
+              int box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t gstride[1] = {(cuuint64_t)ld * 4};
+  const cuuint32_t box[2] = {32u, (cuuint32_t)box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), gdim, gstride, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+}  // namespace
+
+int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return GPTQ_OK;
+  if (g.K % TK != 0 || g.lda % 4 || g.ldb % 4 || g.ldc % 4 ||
+      reinterpret_cast<uintptr_t>(g.A) % 16 || reinterpret_cast<uintptr_t>(g.B) % 16 ||
+      reinterpret_cast<uintptr_t>(g.C) % 16) {
+    set_last_error_msg(__FILE__, __LINE__, "GEMM operands not 16-byte aligned / K % 32 != 0");
+    return GPTQ_ERR_INVALID_ARG;
+  }
+  CUtensorMap ta, tb;
+  const CUtensorMapSwizzle kmaj = CU_TENSOR_MAP_SWIZZLE_128B;
+  const CUtensorMapSwizzle mnmaj = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
+  if (!make_map(&ta, g.A, g.M, g.K, g.lda, TM, kmaj) ||
+      !(trans_b ? make_map(&tb, g.B, g.N, g.K, g.ldb, TN, kmaj)
+                : make_map(&tb, g.B, g.K, g.N, g.ldb, TK, mnmaj))) {
+    set_last_error_msg(__FILE__, __LINE__, "cuTensorMapEncodeTiled rejected a GEMM operand");
+    return GPTQ_ERR_CUDA;
+  }
+  static bool attr = false;
+  if (!attr) {
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SMEM_BYTES));
+    attr = true;
+  }
+  TcArgs a{g.M, g.N, g.K, g.C, g.ldc, g.alpha, g.beta, g.flags, trans_b ? 1 : 0, g.status,
+           device_status_word()};
+  dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM);
+  if (grid.y > 65535) return GPTQ_ERR_INVALID_ARG;
+  gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, a);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+}  // namespace gptq

@@ -38,6 +38,8 @@ int launch_damp(float *H, int64_t ld, int d, float damp, bool add_in_place, floa
 int launch_act_order(const float *H, int64_t ld, int d, int *perm, int *inv, const float *lambda,
                      float *Hp, cudaStream_t stream);
 size_t factor_scratch_floats(int64_t d);
+// One diagonal block (nb <= 128, nb % 32 == 0) of H_d -> U in place (full block, zeros below).
+int launch_leaf(float *A, int64_t ld, int nb, int *status, cudaStream_t stream);
 int launch_factor(float *A, int64_t d, float *T1, int *status, cudaStream_t stream);
 
 struct SweepArgs {

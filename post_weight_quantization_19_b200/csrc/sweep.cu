@@ -23,7 +23,7 @@
 namespace gptq {
 namespace {
 
-constexpr int SWEEP_THREADS = 256;
+constexpr int SWEEP_THREADS = 512;
 constexpr int SWEEP_WARPS = SWEEP_THREADS / 32;
 
 __device__ __forceinline__ float warp_min(float v) {
@@ -44,6 +44,10 @@ __device__ __forceinline__ void minmax_params(float lo, float hi, float maxq, fl
   s = (xmax == xmin) ? 1.f : __fdiv_rn(xmax - xmin, maxq);
   z = rintf(__fdiv_rn(-xmin, s));
 }
+
+// 1/s rounded to nearest; w * (1/s) is within about one ulp of w / s, which
+// moves a code only when w/s sits within that distance of a rounding tie.
+__device__ __forceinline__ float recip(float s) { return __frcp_rn(s); }
 
 __global__ void gather_w_kernel(const float *__restrict__ W, int64_t total, int d,
                                 const int *__restrict__ perm, float *__restrict__ Wk,
@@ -92,12 +96,27 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nc = a.ncols;
-  for (int idx = tid; idx < B * B; idx += SWEEP_THREADS) {
-    const int j = idx / B, c = idx - j * B;
-    sU[idx] = (j < nc && c < nc && c > j) ? a.U[(size_t)(a.j0 + j) * a.ldu + a.j0 + c] : 0.f;
+  // U block -> shared memory with 16-byte loads (rows of U are contiguous and
+  // the block starts on a multiple of 32 columns); entries on or below the
+  // diagonal are zeroed, the diagonal is kept as 1/U_jj.
+  constexpr int Q = B / 4;   // float4 per row
+#pragma unroll 4
+  for (int idx = tid; idx < B * Q; idx += SWEEP_THREADS) {
+    const int j = idx / Q, c4 = (idx - j * Q) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < nc && c4 < nc)
+      v = *reinterpret_cast<const float4 *>(a.U + (size_t)(a.j0 + j) * a.ldu + a.j0 + c4);
+    if (j < nc && j >= c4 && j < c4 + 4) {
+      const float dj = j == c4 ? v.x : j == c4 + 1 ? v.y : j == c4 + 2 ? v.z : v.w;
+      sDinv[j] = 1.f / dj;
+    }
+    v.x = c4 + 0 > j ? v.x : 0.f;
+    v.y = c4 + 1 > j ? v.y : 0.f;
+    v.z = c4 + 2 > j ? v.z : 0.f;
+    v.w = c4 + 3 > j ? v.w : 0.f;
+    *reinterpret_cast<float4 *>(sU + idx * 4) = v;
   }
-  for (int j = tid; j < B; j += SWEEP_THREADS)
-    sDinv[j] = j < nc ? 1.f / a.U[(size_t)(a.j0 + j) * a.ldu + a.j0 + j] : 0.f;
+  for (int j = nc + tid; j < B; j += SWEEP_THREADS) sDinv[j] = 0.f;
   __syncthreads();
 
   const float maxq = (float)((1 << a.bits) - 1);
@@ -119,10 +138,11 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
       code[v] = 0;
       eo[v] = 0.f;
     }
-    float s = 1.f, z = 0.f;
+    float s = 1.f, z = 0.f, si = 1.f;
     if (inherit) {
       s = a.scales[(size_t)row * a.G + gi0];
       z = (float)a.zeros[(size_t)row * a.G + gi0];
+      si = recip(s);
     }
     float esq = 0.f;
     // Column j = jj*V + v lives in register v of lane jj.  nc is a multiple of
@@ -156,6 +176,7 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
           lo = warp_min(lo);
           hi = warp_max(hi);
           minmax_params(lo, hi, maxq, s, z);
+          si = recip(s);
           if (lane == 0) {
             const int gi = (a.j0 + j) / g;
             a.scales[(size_t)row * a.G + gi] = s;
@@ -163,7 +184,7 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
           }
         }
         const float wj = __shfl_sync(0xffffffffu, w[v], jj);
-        float q = rintf(__fdiv_rn(wj, s)) + z;
+        float q = rintf(wj * si) + z;
         q = fminf(fmaxf(q, 0.f), maxq);
         const float wq = s * (q - z);
         const float e = (wj - wq) * sDinv[j];
@@ -192,44 +213,75 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
 }
 
 // Unpermute, dequantised output, ||W - W^||^2 per row, codes and packing.
-// One CTA per row; each thread handles groups of 32 columns.
+// One CTA per row, in chunks of 1024 columns: each thread handles 4
+// consecutive columns (16-byte loads and stores of W, W^), the chunk's codes
+// are staged in shared memory, then 32 threads pack them (32 codes -> BITS
+// words each).
 template <int BITS>
 __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
+  constexpr int CH = 1024;
+  __shared__ uint8_t sc[CH];
+  __shared__ double red[8];
   if (*(volatile const int *)a.status) return;
   const int row = blockIdx.x;
-  const int ngroups = a.d >> 5;
-  const float *w = a.W + (size_t)row * a.d;
-  const float *wk = a.Wk + (size_t)row * a.d;
-  const uint8_t *cp = a.codes_p + (size_t)row * a.d;
+  const size_t rb = (size_t)row * a.d;
+  const float *w = a.W + rb;
+  const float *wk = a.Wk + rb;
+  const uint8_t *cp = a.codes_p + rb;
+  uint32_t *qrow = reinterpret_cast<uint32_t *>(a.qweight) + (size_t)row * (a.d / 32) * BITS;
   double dsq = 0.0;
-  for (int gq = threadIdx.x; gq < ngroups; gq += blockDim.x) {
-    uint32_t c32[32];
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const int c = gq * 32 + k;
-      const int p = a.inv ? a.inv[c] : c;
-      const float wq = wk[p];
-      const float df = w[c] - wq;
-      dsq += (double)df * (double)df;
-      c32[k] = cp[p];
-      if (a.W_hat) a.W_hat[(size_t)row * a.d + c] = wq;
-      if (a.codes) a.codes[(size_t)row * a.d + c] = (uint8_t)c32[k];
-      if (row == 0 && a.g_idx) a.g_idx[c] = a.group < 0 ? 0 : p / a.group;
+  for (int c0 = 0; c0 < a.d; c0 += CH) {
+    const int c = c0 + threadIdx.x * 4;
+    if (c < a.d) {
+      const float4 wo = *reinterpret_cast<const float4 *>(w + c);
+      float4 wq;
+      uchar4 q;
+      if (a.inv) {
+        const int4 p = *reinterpret_cast<const int4 *>(a.inv + c);
+        wq = make_float4(wk[p.x], wk[p.y], wk[p.z], wk[p.w]);
+        q = make_uchar4(cp[p.x], cp[p.y], cp[p.z], cp[p.w]);
+        if (row == 0 && a.g_idx) {
+          const int g = a.group;
+          *reinterpret_cast<int4 *>(a.g_idx + c) =
+              g < 0 ? make_int4(0, 0, 0, 0) : make_int4(p.x / g, p.y / g, p.z / g, p.w / g);
+        }
+      } else {
+        wq = *reinterpret_cast<const float4 *>(wk + c);
+        q = *reinterpret_cast<const uchar4 *>(cp + c);
+        if (row == 0 && a.g_idx) {
+          const int g = a.group;
+          *reinterpret_cast<int4 *>(a.g_idx + c) =
+              g < 0 ? make_int4(0, 0, 0, 0)
+                    : make_int4(c / g, (c + 1) / g, (c + 2) / g, (c + 3) / g);
+        }
+      }
+      const double dx = (double)wo.x - wq.x, dy = (double)wo.y - wq.y;
+      const double dz = (double)wo.z - wq.z, dw = (double)wo.w - wq.w;
+      dsq += dx * dx + dy * dy + dz * dz + dw * dw;
+      if (a.W_hat) *reinterpret_cast<float4 *>(a.W_hat + rb + c) = wq;
+      if (a.codes) *reinterpret_cast<uchar4 *>(a.codes + rb + c) = q;
+      *reinterpret_cast<uchar4 *>(sc + threadIdx.x * 4) = q;
     }
-    uint32_t words[BITS];
-    pack32<BITS>(c32, words);
-    uint32_t *qw = reinterpret_cast<uint32_t *>(a.qweight) + (size_t)row * ngroups * BITS +
-                   (size_t)gq * BITS;
+    __syncthreads();
+    const int ng = min(CH, a.d - c0) / 32;
+    if (threadIdx.x < ng) {
+      uint32_t c32[32];
 #pragma unroll
-    for (int k = 0; k < BITS; ++k) qw[k] = words[k];
+      for (int k = 0; k < 32; ++k) c32[k] = sc[threadIdx.x * 32 + k];
+      uint32_t words[BITS];
+      pack32<BITS>(c32, words);
+      uint32_t *qw = qrow + (size_t)(c0 / 32 + threadIdx.x) * BITS;
+#pragma unroll
+      for (int k = 0; k < BITS; ++k) qw[k] = words[k];
+    }
+    __syncthreads();
   }
-  __shared__ double red[8];
   for (int o = 16; o > 0; o >>= 1) dsq += __shfl_xor_sync(0xffffffffu, dsq, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = dsq;
   __syncthreads();
   if (threadIdx.x == 0) {
     double t = 0.0;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
+    for (int i = 0; i < 8; ++i) t += red[i];
     a.dsq_rows[row] = t;
   }
 }
@@ -294,8 +346,10 @@ static int sweep_launch(const SweepArgs &a, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     attr = true;
   }
+  // One resident warp per row when the SMs can hold them all (2 CTAs of 16
+  // warps per SM), so no CTA runs a sparse second round.
   const int want = (a.r + SWEEP_WARPS - 1) / SWEEP_WARPS;
-  const int cap = num_sms() * 3;
+  const int cap = num_sms() * 2;
   const int grid = want < cap ? want : cap;
   sweep_block_kernel<V><<<grid, SWEEP_THREADS, smem, stream>>>(a);
   GPTQ_LAUNCH_CHECK();
