@@ -27,39 +27,44 @@ constexpr int LLD = LB + 1;        // shared-memory leading dimension
 constexpr int LT = 256;            // threads (255 registers each for the warp factor)
 constexpr size_t LEAF_SMEM = ((size_t)LB * LLD + 64 * 64) * sizeof(real);
 
-// C[M x N] = alpha * A[M x K] * op(B) + beta * C for M, N, K <= 64 in shared
-// memory; op(B) = B (K x N) or B^T (B stored N x K).  Each thread owns a 4 x 4
-// tile of C.  upper: only entries with column >= row are written (C is a
-// diagonal block).  Ends with a CTA barrier.
-__device__ __noinline__ void smem_gemm(real *C, int ldc, const real *A, int lda, const real *B, int ldb,
-                          int M, int N, int K, real alpha, real beta, bool transB, bool upper) {
-  const int tiles_n = N / 4;
-  const int ntiles = (M / 4) * tiles_n;
-  for (int tile = threadIdx.x; tile < ntiles; tile += LT) {
-    const int i0 = (tile / tiles_n) * 4, j0 = (tile % tiles_n) * 4;
-    if (upper && j0 + 3 < i0) continue;
-    real acc[4][4];
+// C[M x N] = alpha * A[M x K] * op(B) + beta * C in shared memory, all shapes
+// and strides known at compile time; op(B) = B (K x N) or B^T (B stored N x K).
+// The M x N outputs are spread over all threads in RM x RN register tiles.
+// UPPER: only entries with column >= row are written (C is a diagonal block).
+// Ends with a CTA barrier.
+template <int M, int N, int K, int LDA, int LDB, int LDC, bool TB, bool UPPER>
+__device__ __forceinline__ void smem_gemm(real *C, const real *A, const real *B, real alpha,
+                                          real beta) {
+  constexpr int RM = (M * N >= 16 * LT) ? 4 : 2;
+  constexpr int RN = (M * N >= 8 * LT) ? 4 : 2;
+  constexpr int TN = N / RN;
+  constexpr int NT = (M / RM) * TN;
+  for (int tile = threadIdx.x; tile < NT; tile += LT) {
+    const int i0 = (tile / TN) * RM, j0 = (tile % TN) * RN;
+    if (UPPER && j0 + RN - 1 < i0) continue;
+    real acc[RM][RN];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+    for (int r = 0; r < RM; ++r)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+      for (int c = 0; c < RN; ++c) acc[r][c] = 0.f;
+#pragma unroll 16
     for (int k = 0; k < K; ++k) {
-      real a[4], b[4];
+      real a[RM], b[RN];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) a[r] = A[(i0 + r) * lda + k];
+      for (int r = 0; r < RM; ++r) a[r] = A[(i0 + r) * LDA + k];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) b[c] = transB ? B[(j0 + c) * ldb + k] : B[k * ldb + j0 + c];
+      for (int c = 0; c < RN; ++c) b[c] = TB ? B[(j0 + c) * LDB + k] : B[k * LDB + j0 + c];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int r = 0; r < RM; ++r)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+        for (int c = 0; c < RN; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+    for (int r = 0; r < RM; ++r)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (upper && j0 + c < i0 + r) continue;
-        real *p = C + (i0 + r) * ldc + j0 + c;
+      for (int c = 0; c < RN; ++c) {
+        if (UPPER && j0 + c < i0 + r) continue;
+        real *p = C + (i0 + r) * LDC + j0 + c;
         *p = alpha * acc[r][c] + (beta != 0.f ? beta * *p : 0.f);
       }
   }
@@ -73,7 +78,10 @@ __device__ __noinline__ void smem_gemm(real *C, int ldc, const real *A, int lda,
 //                                                              (i < k <= c)
 //   row k             S[k][c]  = (c == k ? 1 : S[k][c]) / sqrt(p)   (c >= k)
 // Returns false (for every lane) on a non-positive pivot.
-__device__ __forceinline__ bool warp_factor32(real *S, int ld) {
+__device__ __noinline__ bool warp_factor32(real *S, int ld) {
+  // The caller's tile loops may leave the warp split into divergent groups; a
+  // split warp would run every shuffle below once per group.
+  __syncwarp();
   const int i = threadIdx.x & 31;
   real d[32];
 #pragma unroll
@@ -88,8 +96,9 @@ __device__ __forceinline__ bool warp_factor32(real *S, int ld) {
     ri = ri * fmaf(-0.5f * p * ri, ri, 1.5f);   // one Newton step
     const real ri2 = ri * ri;
     const real ck = d[k];
+    // Descending j: the next pivot (row k-1, column k-1) is updated first.
 #pragma unroll
-    for (int j = 0; j < k; ++j) {
+    for (int j = k - 1; j >= 0; --j) {
       const real cj = __shfl_sync(0xffffffffu, d[k], j);
       if (i <= j) d[j] = fmaf(-ck * ri2, cj, d[j]);
     }
@@ -126,11 +135,11 @@ __device__ __forceinline__ bool node_factor(real *S, real *T, int off, bool *fai
     real *A11 = S + off * LLD + off;
     real *A12 = S + off * LLD + off + h;
     const real *U22 = S + (off + h) * LLD + off + h;
-    smem_gemm(T, m, A12, LLD, U22, LLD, h, m, m, 1.f, 0.f, true, false);    // R12 = A12 U22^T
-    smem_gemm(A11, LLD, T, m, T, m, h, h, m, -1.f, 1.f, true, true);        // A11 -= R12 R12^T
-    smem_gemm(A12, LLD, T, m, U22, LLD, h, m, m, 1.f, 0.f, false, false);   // A12 = R12 U22
+    smem_gemm<h, m, m, LLD, LLD, m, true, false>(T, A12, U22, 1.f, 0.f);      // R12 = A12 U22^T
+    smem_gemm<h, h, m, m, m, LLD, true, true>(A11, T, T, -1.f, 1.f);          // A11 -= R12 R12^T
+    smem_gemm<h, m, m, m, LLD, LLD, false, false>(A12, T, U22, 1.f, 0.f);     // A12 = R12 U22
     if (!node_factor<h>(S, T, off, fail)) return false;
-    smem_gemm(T, m, A11, LLD, A12, LLD, h, m, h, -1.f, 0.f, false, false);  // T = -U11 A12
+    smem_gemm<h, m, h, LLD, LLD, m, false, false>(T, A11, A12, -1.f, 0.f);    // T = -U11 A12
     for (int idx = threadIdx.x; idx < h * m; idx += LT) {
       const int r = idx / m, c = idx - r * m;
       A12[r * LLD + c] = T[r * m + c];
