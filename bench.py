@@ -225,7 +225,8 @@ def run_ours(args, wl, rank: int, world: int, dist):
             "scales": torch.empty((r, G), dtype=torch.float32, device=dev),
             "zeros": torch.empty((r, G), dtype=torch.int32, device=dev)}
     g_idx = torch.empty((d,), dtype=torch.int32, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    stream = torch.cuda.Stream(dev)   # a capturable stream: the solve replays as a CUDA graph
+    torch.cuda.set_stream(stream)
     h_start = torch.cuda.Event(enable_timing=True)
     h_end = torch.cuda.Event(enable_timing=True)
 

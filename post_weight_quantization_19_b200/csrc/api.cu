@@ -3,6 +3,9 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+#include <vector>
+
 #include "gptq_internal.h"
 
 namespace gptq {
@@ -91,6 +94,91 @@ int record(int i, cudaStream_t s) {
   if (!g_timing) return GPTQ_OK;
   if (!g_ev[i]) GPTQ_CUDA_TRY(cudaEventCreate(&g_ev[i]));
   GPTQ_CUDA_TRY(cudaEventRecord(g_ev[i], s));
+  return GPTQ_OK;
+}
+
+// ---------------------------------------------------------------- graph cache
+
+struct GraphKey {
+  const void *W, *H, *W_hat, *qweight, *scales, *zeros, *g_idx, *codes, *ws;
+  size_t ws_bytes;
+  cudaStream_t stream;
+  int64_t r, d;
+  int bits, group, block;
+  float damp;
+  int act_order;
+  int device = -1;
+  bool operator==(const GraphKey &o) const {
+    return W == o.W && H == o.H && W_hat == o.W_hat && qweight == o.qweight &&
+           scales == o.scales && zeros == o.zeros && g_idx == o.g_idx && codes == o.codes &&
+           ws == o.ws && ws_bytes == o.ws_bytes && stream == o.stream && r == o.r &&
+           d == o.d && bits == o.bits && group == o.group && block == o.block &&
+           memcmp(&damp, &o.damp, sizeof(float)) == 0 && act_order == o.act_order &&
+           device == o.device;
+  }
+};
+
+struct GraphEntry {
+  GraphKey key;
+  int seen = 0;
+  cudaGraphExec_t exec = nullptr;
+  uint64_t kernels = 0;
+  uint64_t last_use = 0;
+};
+
+std::mutex g_graph_mu;
+std::vector<GraphEntry> g_graphs;
+uint64_t g_graph_clock = 0;
+constexpr size_t kMaxGraphs = 16;
+
+template <class F>
+int run_graph_cached(GraphKey key, cudaStream_t st, F &&enqueue) {
+  GPTQ_CUDA_TRY(cudaGetDevice(&key.device));
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (st == nullptr || cudaStreamIsCapturing(st, &cs) != cudaSuccess ||
+      cs != cudaStreamCaptureStatusNone)
+    return enqueue();
+  std::lock_guard<std::mutex> lock(g_graph_mu);
+  GraphEntry *e = nullptr;
+  for (auto &x : g_graphs)
+    if (x.key == key) e = &x;
+  if (!e) {
+    if (g_graphs.size() >= kMaxGraphs) {
+      auto victim = g_graphs.begin();
+      for (auto it = g_graphs.begin(); it != g_graphs.end(); ++it)
+        if (it->last_use < victim->last_use) victim = it;
+      if (victim->exec) cudaGraphExecDestroy(victim->exec);
+      g_graphs.erase(victim);
+    }
+    g_graphs.push_back(GraphEntry{key});
+    e = &g_graphs.back();
+  }
+  e->last_use = ++g_graph_clock;
+  if (!e->exec && e->seen++ == 0) return enqueue();   // first sighting: run directly
+  if (!e->exec) {
+    const uint64_t before = g_launches.load();
+    GPTQ_CUDA_TRY(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+    const int rc = enqueue();
+    cudaGraph_t graph = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(st, &graph);
+    const uint64_t captured = g_launches.load() - before;
+    g_launches.fetch_sub(captured);
+    if (rc != GPTQ_OK || ce != cudaSuccess) {
+      if (graph) cudaGraphDestroy(graph);
+      (void)cudaGetLastError();
+      return rc != GPTQ_OK ? rc : GPTQ_ERR_CUDA;
+    }
+    const cudaError_t ie = cudaGraphInstantiate(&e->exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (ie != cudaSuccess) {
+      e->exec = nullptr;
+      set_last_error(__FILE__, __LINE__, "cudaGraphInstantiate", ie);
+      return GPTQ_ERR_CUDA;
+    }
+    e->kernels = captured;
+  }
+  GPTQ_CUDA_TRY(cudaGraphLaunch(e->exec, st));
+  count_launch(e->kernels);
   return GPTQ_OK;
 }
 
@@ -193,87 +281,105 @@ extern "C" int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *
   const int G = group < 0 ? 1 : di / group;
   const int S = superblock(d, group, block);
 
-  GPTQ_TRY(record(0, st));
-  GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 16, st));
-  GPTQ_CUDA_TRY(cudaMemsetAsync(loss_rows, 0, (size_t)r * 8, st));
+  auto enqueue = [&]() -> int {
+    GPTQ_TRY(record(0, st));
+    GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 16, st));
+    GPTQ_CUDA_TRY(cudaMemsetAsync(loss_rows, 0, (size_t)r * 8, st));
 
-  // Phase 0: damping, act-order, working copy of W.
-  float *Hf = H;
-  if (act_order) {
-    GPTQ_TRY(launch_damp(H, d, di, damp, false, lambda, st));
-    GPTQ_TRY(launch_act_order(H, d, di, perm, inv, lambda, Hp, st));
-    Hf = Hp;
-  } else {
-    GPTQ_TRY(launch_damp(H, d, di, damp, true, lambda, st));
-  }
-  GPTQ_TRY(launch_gather_w(W, ri, di, act_order ? perm : nullptr, Wk, status, st));
-  GPTQ_TRY(record(1, st));
+    // Phase 0: damping, act-order, working copy of W.
+    float *Hf = H;
+    if (act_order) {
+      GPTQ_TRY(launch_damp(H, d, di, damp, false, lambda, st));
+      GPTQ_TRY(launch_act_order(H, d, di, perm, inv, lambda, Hp, st));
+      Hf = Hp;
+    } else {
+      GPTQ_TRY(launch_damp(H, d, di, damp, true, lambda, st));
+    }
+    GPTQ_TRY(launch_gather_w(W, ri, di, act_order ? perm : nullptr, Wk, status, st));
+    GPTQ_TRY(record(1, st));
 
-  // Phase 1: U = upper Cholesky factor of H_d^-1, in place.
-  GPTQ_TRY(launch_factor(Hf, d, T1, status, st));
-  GPTQ_TRY(record(2, st));
+    // Phase 1: U = upper Cholesky factor of H_d^-1, in place.
+    GPTQ_TRY(launch_factor(Hf, d, T1, status, st));
+    GPTQ_TRY(record(2, st));
 
-  // Phase 2: column sweep in blocks, lazy trailing updates.
-  if (group < 0) GPTQ_TRY(launch_row_params(Wk, ri, di, bits, scales, zeros, status, st));
-  for (int s0 = 0; s0 < di; s0 += S) {
-    const int sEnd = s0 + S < di ? s0 + S : di;
-    for (int j0 = s0; j0 < sEnd; j0 += block) {
-      const int j1 = j0 + block < sEnd ? j0 + block : sEnd;
-      SweepArgs a{};
-      a.Wk = Wk;
-      a.ldw = d;
-      a.U = Hf;
-      a.ldu = d;
-      a.r = ri;
-      a.j0 = j0;
-      a.ncols = j1 - j0;
-      a.bits = bits;
-      a.group = group;
-      a.scales = scales;
-      a.zeros = zeros;
-      a.G = G;
-      a.codes = codes_p;
-      a.ldc = d;
-      a.err = ErrS + (j0 - s0);
-      a.lde = S;
-      a.loss_rows = loss_rows;
-      a.status = status;
-      GPTQ_TRY(launch_sweep_block(a, block, st));
-      if (j1 < sEnd) {
-        // Rest of this superblock: W[:, j1:sEnd] -= E_blk U[j0:j1, j1:sEnd]
-        GemmArgs g{ri, sEnd - j1, j1 - j0, ErrS + (j0 - s0), S, Hf + (size_t)j0 * d + j1, d,
-                   Wk + j1, d, -1.f, 1.f, 0, status};
+    // Phase 2: column sweep in blocks, lazy trailing updates.
+    if (group < 0) GPTQ_TRY(launch_row_params(Wk, ri, di, bits, scales, zeros, status, st));
+    for (int s0 = 0; s0 < di; s0 += S) {
+      const int sEnd = s0 + S < di ? s0 + S : di;
+      for (int j0 = s0; j0 < sEnd; j0 += block) {
+        const int j1 = j0 + block < sEnd ? j0 + block : sEnd;
+        SweepArgs a{};
+        a.Wk = Wk;
+        a.ldw = d;
+        a.U = Hf;
+        a.ldu = d;
+        a.r = ri;
+        a.j0 = j0;
+        a.ncols = j1 - j0;
+        a.bits = bits;
+        a.group = group;
+        a.scales = scales;
+        a.zeros = zeros;
+        a.G = G;
+        a.codes = codes_p;
+        a.ldc = d;
+        a.err = ErrS + (j0 - s0);
+        a.lde = S;
+        a.loss_rows = loss_rows;
+        a.status = status;
+        GPTQ_TRY(launch_sweep_block(a, block, st));
+        if (j1 < sEnd) {
+          // Rest of this superblock: W[:, j1:sEnd] -= E_blk U[j0:j1, j1:sEnd]
+          GemmArgs g{ri, sEnd - j1, j1 - j0, ErrS + (j0 - s0), S, Hf + (size_t)j0 * d + j1, d,
+                     Wk + j1, d, -1.f, 1.f, 0, status};
+          GPTQ_TRY(launch_gemm(g, false, st));
+        }
+      }
+      if (sEnd < di) {
+        // Deferred global update: W[:, sEnd:] -= E_S U[s0:sEnd, sEnd:]
+        GemmArgs g{ri, di - sEnd, sEnd - s0, ErrS, S, Hf + (size_t)s0 * d + sEnd, d, Wk + sEnd, d,
+                   -1.f, 1.f, 0, status};
         GPTQ_TRY(launch_gemm(g, false, st));
       }
     }
-    if (sEnd < di) {
-      // Deferred global update: W[:, sEnd:] -= E_S U[s0:sEnd, sEnd:]
-      GemmArgs g{ri, di - sEnd, sEnd - s0, ErrS, S, Hf + (size_t)s0 * d + sEnd, d, Wk + sEnd, d,
-                 -1.f, 1.f, 0, status};
-      GPTQ_TRY(launch_gemm(g, false, st));
-    }
-  }
-  GPTQ_TRY(record(3, st));
+    GPTQ_TRY(record(3, st));
 
-  // Phase 3: unpermute, loss, packing.
-  FinalizeArgs f{};
-  f.W = W;
-  f.Wk = Wk;
-  f.codes_p = codes_p;
-  f.inv = act_order ? inv : nullptr;
-  f.r = ri;
-  f.d = di;
-  f.bits = bits;
-  f.group = group;
-  f.W_hat = W_hat;
-  f.codes = codes;
-  f.qweight = qweight;
-  f.g_idx = g_idx;
-  f.dsq_rows = dsq_rows;
-  f.status = status;
-  GPTQ_TRY(launch_finalize(f, st));
-  GPTQ_TRY(launch_loss_reduce(loss_rows, dsq_rows, ri, lambda, out, status, st));
-  GPTQ_TRY(record(4, st));
+    // Phase 3: unpermute, loss, packing.
+    FinalizeArgs f{};
+    f.W = W;
+    f.Wk = Wk;
+    f.codes_p = codes_p;
+    f.inv = act_order ? inv : nullptr;
+    f.r = ri;
+    f.d = di;
+    f.bits = bits;
+    f.group = group;
+    f.W_hat = W_hat;
+    f.codes = codes;
+    f.qweight = qweight;
+    f.g_idx = g_idx;
+    f.dsq_rows = dsq_rows;
+    f.status = status;
+    GPTQ_TRY(launch_finalize(f, st));
+    GPTQ_TRY(launch_loss_reduce(loss_rows, dsq_rows, ri, lambda, out, status, st));
+    GPTQ_TRY(record(4, st));
+    return GPTQ_OK;
+  };
+
+  // Replay the whole kernel sequence as a CUDA graph when the same call
+  // (pointers, sizes, settings, stream) repeats: the sequence holds a few
+  // hundred short kernels whose launch cost would otherwise pace the GPU.  The
+  // first call of a configuration runs directly, the second is captured, later
+  // ones replay.  Streams that cannot be captured run directly.
+  const GraphKey key{W, H, W_hat, qweight, scales, zeros, g_idx, codes, workspace,
+                     workspace_bytes, st, r, d, bits, group, block, damp, act_order};
+  int rc = GPTQ_OK;
+  if (g_timing) {
+    rc = enqueue();
+  } else {
+    rc = run_graph_cached(key, st, enqueue);
+  }
+  if (rc != GPTQ_OK) return rc;
 
   double host_out[3] = {0, 0, 0};
   int host_status = 0;

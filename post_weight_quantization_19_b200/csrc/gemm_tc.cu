@@ -6,16 +6,18 @@
 // block recursion that forms U -- the dense contractions of the layer solve
 // (GPTQ reading card, 方法适配: the deferred global update is a matrix product).
 //
-// Each fp32 operand x is split as hi = tf32(x) (round to nearest) and
-// lo = tf32(x - hi); the product is hi*hi + hi*lo + lo*hi, three
+// Each fp32 operand x is split as hi = tf32(x) (rounded) and lo = tf32(x - hi)
+// (truncated), with integer operations; the product is hi*hi + hi*lo + lo*hi, three
 // tcgen05.mma.kind::tf32 per K step accumulating in TMEM, which keeps about
 // 21 bits of each operand (the dropped lo*lo term is ~2^-22 relative).
 //
-// Tile 128 x 128 x 32 per stage, 3-stage TMA ring.  A (and B^T) are K-major
+// Tile 128 x 128 x 32 per stage: a 4-deep TMA ring of raw A/B tiles (the hi
+// parts are written back in place) and a 3-deep ring of lo tiles.  A (and B^T) are K-major
 // with a 128-byte swizzle; a row-major B is consumed MN-major with the
 // 128-byte swizzle of 32-byte atoms (the only MN-major layout for tf32).  Warp 0 issues
-// TMA, warp 1 issues UMMA, warps 2..5 split each landed stage into hi/lo in
-// shared memory and afterwards drain the TMEM accumulator into C.
+// TMA, warp 1 issues UMMA, warps 2..9 split each landed stage into hi/lo in
+// shared memory and afterwards drain the TMEM accumulator into C (two warps
+// per TMEM lane quarter, 64 columns each).
 #include <mutex>
 
 #include "gptq_internal.h"
@@ -24,17 +26,19 @@ namespace gptq {
 namespace {
 
 constexpr int TM = 128, TN = 128, TK = 32;
-constexpr int STAGES = 3;
-constexpr int TILE_BYTES = 128 * TK * 4;   // 16 KB: 128 rows x 32 fp32
-constexpr int STAGE_BYTES = 4 * TILE_BYTES; // A, B, A_lo, B_lo
-constexpr int THREADS = 32 * 6;
-constexpr int CONV_THREADS = 128;
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024;
+constexpr int RS = 4;                       // TMA ring: raw A, B tiles (hi in place)
+constexpr int LS = 3;                       // lo ring: A_lo, B_lo tiles
+constexpr int TILE_BYTES = 128 * TK * 4;    // 16 KB: 128 rows x 32 fp32
+constexpr int PAIR_BYTES = 2 * TILE_BYTES;  // A and B
+constexpr int THREADS = 32 * 10;
+constexpr int CONV_THREADS = 256;
+constexpr size_t SMEM_BYTES = (size_t)(RS + LS) * PAIR_BYTES + 1024;
 
 struct TcShared {
-  uint64_t full[STAGES];
-  uint64_t conv[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[RS];
+  uint64_t empty[RS];
+  uint64_t conv[LS];
+  uint64_t lofree[LS];
   uint64_t accf;
   uint64_t drain;
   uint32_t tmem_base;
@@ -52,10 +56,15 @@ struct TcArgs {
   int *dev_status;
 };
 
-__device__ __forceinline__ uint32_t tf32_rn(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
+// tf32 split with integer operations (full ALU rate, unlike conversions):
+// hi = x rounded to 10 mantissa bits (ties away from zero; a carry into the
+// exponent rounds up to the next binade), lo = x - hi exactly, then lo with
+// its low 13 bits cleared.  |x - hi - lo| <= 2^-21 |x|.
+__device__ __forceinline__ float tf32_hi(float x) {
+  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+}
+__device__ __forceinline__ float tf32_trunc(float x) {
+  return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -67,7 +76,7 @@ __device__ __forceinline__ void fail_timeout(TcShared &sh, int *dev_status) {
   *(volatile int *)&sh.abort = 1;
 }
 
-// hi/lo split of one 16 KB tile in place: x -> tf32(x), lo <- tf32(x - tf32(x)).
+// hi/lo split of one 16 KB tile in place: x -> hi, lo buffer <- lo.
 __device__ __forceinline__ void split_tile(uint8_t *tile, uint8_t *lo, int t) {
   float4 *p = reinterpret_cast<float4 *>(tile);
   float4 *q = reinterpret_cast<float4 *>(lo);
@@ -75,14 +84,14 @@ __device__ __forceinline__ void split_tile(uint8_t *tile, uint8_t *lo, int t) {
   for (int i = t; i < TILE_BYTES / 16; i += CONV_THREADS) {
     float4 v = p[i];
     float4 h, l;
-    h.x = __uint_as_float(tf32_rn(v.x));
-    h.y = __uint_as_float(tf32_rn(v.y));
-    h.z = __uint_as_float(tf32_rn(v.z));
-    h.w = __uint_as_float(tf32_rn(v.w));
-    l.x = __uint_as_float(tf32_rn(v.x - h.x));
-    l.y = __uint_as_float(tf32_rn(v.y - h.y));
-    l.z = __uint_as_float(tf32_rn(v.z - h.z));
-    l.w = __uint_as_float(tf32_rn(v.w - h.w));
+    h.x = tf32_hi(v.x);
+    h.y = tf32_hi(v.y);
+    h.z = tf32_hi(v.z);
+    h.w = tf32_hi(v.w);
+    l.x = tf32_trunc(v.x - h.x);
+    l.y = tf32_trunc(v.y - h.y);
+    l.z = tf32_trunc(v.z - h.z);
+    l.w = tf32_trunc(v.w - h.w);
     p[i] = h;
     q[i] = l;
   }
@@ -108,10 +117,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < RS; ++s) {
       mbar_init(&sh.full[s], 1);
-      mbar_init(&sh.conv[s], CONV_THREADS / 32);
       mbar_init(&sh.empty[s], 1);
+    }
+    for (int t = 0; t < LS; ++t) {
+      mbar_init(&sh.conv[t], CONV_THREADS / 32);
+      mbar_init(&sh.lofree[t], 1);
     }
     mbar_init(&sh.accf, 1);
     mbar_init(&sh.drain, 1);
@@ -135,14 +147,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       uint32_t issued = 0, issued_par = 0;
       for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
+        const int s = kb % RS;
+        const uint32_t ph = (kb / RS) & 1;
         if (*(volatile int *)&sh.abort) break;
         if (!mbar_wait_bounded(&sh.empty[s], ph ^ 1)) {
           fail_timeout(sh, g.dev_status);
           break;
         }
-        uint8_t *st = smem + (size_t)s * STAGE_BYTES;
+        uint8_t *st = smem + (size_t)s * PAIR_BYTES;
         const int k0 = klo + kb * TK;
         mbar_arrive_expect_tx(&sh.full[s], 2 * TILE_BYTES);
         tma_load_2d(st, &tmA, k0, m0, &sh.full[s]);
@@ -156,22 +168,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         issued |= 1u << s;
         issued_par = (issued_par & ~(1u << s)) | (ph << s);
       }
-      for (int s = 0; s < STAGES; ++s)
+      for (int s = 0; s < RS; ++s)
         if (issued & (1u << s)) (void)mbar_wait_bounded(&sh.full[s], (issued_par >> s) & 1u);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = instr_desc(2, 2, 0, g.trans_b ? 0u : 1u, TM, TN);
       for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        if (!mbar_wait_bounded(&sh.conv[s], ph)) {
+        const int s = kb % RS, t = kb % LS;
+        if (!mbar_wait_bounded(&sh.conv[t], (kb / LS) & 1)) {
           fail_timeout(sh, g.dev_status);
           break;
         }
         tc_fence_after();
-        const uint32_t a = smem_u32(smem + (size_t)s * STAGE_BYTES);
-        const uint32_t b = a + TILE_BYTES, al = a + 2 * TILE_BYTES, bl = a + 3 * TILE_BYTES;
+        const uint32_t a = smem_u32(smem + (size_t)s * PAIR_BYTES);
+        const uint32_t b = a + TILE_BYTES;
+        const uint32_t al = smem_u32(smem + (size_t)(RS + t) * PAIR_BYTES);
+        const uint32_t bl = al + TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < TK / 8; ++kk) {
           // A, B^T: K-major, 8 tf32 = 32 bytes per K step inside the swizzle atom.
@@ -194,6 +207,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           umma_tf32_ss(tmem, ald, bd, idesc, 1u);
         }
         umma_commit(&sh.empty[s]);
+        umma_commit(&sh.lofree[t]);
       }
       umma_commit(&sh.accf);
       umma_commit(&sh.drain);
@@ -201,24 +215,26 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------------- split + epilogue
-    const int t = threadIdx.x - 64;
+    const int tt = threadIdx.x - 64;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if (!mbar_wait_bounded(&sh.full[s], ph)) {
+      const int s = kb % RS, t = kb % LS;
+      if (!mbar_wait_bounded(&sh.full[s], (kb / RS) & 1) ||
+          !mbar_wait_bounded(&sh.lofree[t], ((kb / LS) & 1) ^ 1)) {
         if (lane == 0) fail_timeout(sh, g.dev_status);
         ok = false;
         break;
       }
-      uint8_t *st = smem + (size_t)s * STAGE_BYTES;
-      split_tile(st, st + 2 * TILE_BYTES, t);
-      split_tile(st + TILE_BYTES, st + 3 * TILE_BYTES, t);
+      uint8_t *st = smem + (size_t)s * PAIR_BYTES;
+      uint8_t *lo = smem + (size_t)(RS + t) * PAIR_BYTES;
+      split_tile(st, lo, tt);
+      split_tile(st + TILE_BYTES, lo + TILE_BYTES, tt);
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.conv[s]);
+      if (lane == 0) mbar_arrive(&sh.conv[t]);
     }
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;   // which 64 of the 128 columns
     const int row = m0 + quarter * 32 + lane;
     if (ok && nk > 0) {
       if (!mbar_wait_bounded(&sh.accf, 0)) {
@@ -229,7 +245,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (ok) {
 #pragma unroll 1
-      for (int c0 = 0; c0 < TN; c0 += 32) {
+      for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
         float v[32];
         if (nk > 0) {
           tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + c0, v);

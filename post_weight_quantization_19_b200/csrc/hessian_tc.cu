@@ -28,17 +28,31 @@ namespace gptq {
 
 __device__ int g_device_status;
 
+// Per-device lookups are cached so that no runtime query runs inside a
+// stream capture of the solve.
 int *device_status_word() {
-  void *p = nullptr;
-  if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-  return static_cast<int *>(p);
+  static int *cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cache[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<int *>(p);
+  }
+  return cache[dev];
 }
 
 int num_sms() {
-  int dev = 0, v = 0;
+  static int cache[64] = {};
+  int dev = 0;
   cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-  return v > 0 ? v : 1;
+  if (dev < 0 || dev >= 64) return 1;
+  if (!cache[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = v > 0 ? v : 1;
+  }
+  return cache[dev];
 }
 
 namespace {

@@ -1,8 +1,12 @@
-"""Full-size layers on the GPU, checked on sampled rows against the float64 oracle.
+"""Full-size layers on the GPU, checked against the float64 oracle (needs a B200).
 
-The GPU runs the whole layer in the launch configuration the benchmark times;
-the oracle computes the full float64 Hessian and U (rows are independent once
-U is fixed) and sweeps a seeded sample of rows.
+The GPU runs the whole layer in the launch configuration the benchmark times.
+Where the float64 Hessian fits on the host, the oracle computes H and U in
+full (rows are independent once U is fixed) and sweeps a seeded sample of rows.
+The OPT-175B fc2 layer (d = 49152: a float64 H alone is 19 GB) is checked
+through properties that hold at any size: sampled rows of H, the
+dequantisation and packing identities, and GPTQ's layer objective against
+round-to-nearest on sampled rows, both evaluated from X directly.
 """
 
 import numpy as np
@@ -28,6 +32,7 @@ def _check_sampled(name: str, nrows: int = 64):
     got = gpu_layer(X, W, bits=wl.bits, group=wl.group, block=wl.block, damp=wl.damp,
                     act_order=wl.act_order)
     H = oracle.hessian(X)
+    del X
     err = rel_fro(got["H"], H)
     assert err <= H_REL_FRO, err
     rows = np.sort(np.random.default_rng(wl.seed).choice(wl.r, nrows, replace=False))
@@ -38,11 +43,76 @@ def _check_sampled(name: str, nrows: int = 64):
     assert abs(gl - ref["loss"]) <= LOSS_REL * ref["loss"], (gl, ref["loss"])
     total = oracle.layer_loss(W, got["W_hat"], H)
     assert abs(got["loss"] - total) <= LOSS_REL * total, (got["loss"], total)
-    np.testing.assert_array_equal(got["qweight"][rows], oracle.pack_rows(got["codes"][rows],
-                                                                         wl.bits))
+    np.testing.assert_array_equal(got["qweight"][rows],
+                                  oracle.pack_rows(got["codes"][rows], wl.bits))
+    if wl.act_order:
+        np.testing.assert_array_equal(got["g_idx"], ref["g_idx"])
     print(f"{name}: H rel {err:.2e}, codes {match:.6f}, sampled loss rel "
           f"{abs(gl - ref['loss']) / ref['loss']:.2e}")
 
 
 def test_llama7b_q_proj_4096x4096():
     _check_sampled("llama7b_q_proj_4096x4096")
+
+
+@pytest.mark.parametrize("name", ["llama7b_up_proj_11008x4096",
+                                  "llama7b_up_proj_11008x4096_actorder"])
+def test_llama7b_up_proj(name):
+    _check_sampled(name)
+
+
+@pytest.mark.parametrize("name", ["llama7b_down_proj_4096x11008",
+                                  "llama7b_down_proj_4096x11008_actorder"])
+def test_llama7b_down_proj(name):
+    _check_sampled(name, nrows=32)
+
+
+@pytest.mark.parametrize("name", ["w3_8192x8192_perrow", "w3_8192x8192_g128"])
+def test_w3_8192(name):
+    _check_sampled(name, nrows=32)
+
+
+def test_opt175b_fc2_properties():
+    wl = workload("opt175b_fc2_12288x49152")
+    X, W = workload_inputs(wl)
+    r, d = W.shape
+    import post_weight_quantization_19_b200 as g
+
+    dev = torch.device("cuda")
+    Xd = torch.from_numpy(X).to(dev)
+    H = torch.zeros((d, d), dtype=torch.float32, device=dev)
+    g.gptq_hessian_accumulate(Xd, H)
+    del Xd
+    hrows = np.array([0, 777, d // 2, d - 1])
+    Hs = H[torch.from_numpy(hrows).to(dev)].cpu().numpy()
+    Href = oracle.hessian_rows(X, hrows)
+    assert rel_fro(Hs, Href) <= H_REL_FRO
+    Wd = torch.from_numpy(W).to(dev)
+    W_hat = torch.empty_like(Wd)
+    codes = torch.empty((r, d), dtype=torch.uint8, device=dev)
+    g_idx = torch.empty((d,), dtype=torch.int32, device=dev)
+    res = g.gptq_quantize_layer(Wd, H, bits=wl.bits, group=wl.group, block=wl.block,
+                                damp=wl.damp, W_hat=W_hat, codes=codes, g_idx=g_idx)
+    torch.cuda.synchronize()
+    del H
+    rows = np.sort(np.random.default_rng(wl.seed).choice(r, 8, replace=False))
+    rt = torch.from_numpy(rows).to(dev)
+    c = codes[rt].cpu().numpy()
+    wh = W_hat[rt].cpu().numpy()
+    sc = res["scales"][rt].cpu().numpy()
+    zr = res["zeros"][rt].cpu().numpy()
+    q = res["qweight"][rt].cpu().numpy()
+    gi = np.arange(d) // wl.group
+    np.testing.assert_array_equal(g_idx.cpu().numpy(), gi)
+    assert c.max() <= (1 << wl.bits) - 1 and zr.min() >= 0 and zr.max() <= (1 << wl.bits) - 1
+    np.testing.assert_array_equal(wh, sc[:, gi] * (c.astype(np.float32) - zr[:, gi]))
+    np.testing.assert_array_equal(q, oracle.pack_rows(c, wl.bits))
+    # GPTQ's objective on the sampled rows against round-to-nearest, both from X
+    _, rtn_hat = oracle.rtn(W[rows], wl.bits, wl.group)
+    # ||D X^T||^2 is a sum over tokens, so it is taken over 4096-token chunks
+    lg = sum(oracle.layer_loss_direct(W[rows], wh, X[t:t + 4096]) for t in range(0, wl.n, 4096))
+    lr = sum(oracle.layer_loss_direct(W[rows], rtn_hat, X[t:t + 4096])
+             for t in range(0, wl.n, 4096))
+    assert lg < lr, (lg, lr)
+    assert np.isfinite(res["loss"]) and res["loss"] > 0
+    print(f"opt175b fc2: sampled-row objective GPTQ {lg:.4g} vs RTN {lr:.4g}")

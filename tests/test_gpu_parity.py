@@ -216,6 +216,37 @@ def test_workspace_too_small_is_reported():
     assert e.value.status == 4
 
 
-def test_kernels_were_launched():
+def test_zz_kernels_were_launched():
     import post_weight_quantization_19_b200 as g
     assert g.gptq_launch_count() > 0
+
+
+def test_graph_replay_matches_direct_launch():
+    # On a non-default stream a repeated call is captured once and then replayed
+    # as a CUDA graph; every call must give the same result as the first
+    # (direct) one, with fresh inputs each time.
+    import post_weight_quantization_19_b200 as g
+    X, W = make_problem(48, 384, 3000, seed=41)
+    s = torch.cuda.Stream()
+    Wd = torch.from_numpy(W).cuda()
+    Xd = torch.from_numpy(X).cuda()
+    r, d = W.shape
+    ws = torch.empty(g.gptq_quantize_workspace_bytes(r, d, 4, 128), dtype=torch.uint8,
+                     device="cuda")
+    H = torch.empty((d, d), device="cuda")
+    outs = {"qweight": torch.empty((r, d // 8), dtype=torch.int32, device="cuda"),
+            "scales": torch.empty((r, 3), device="cuda"),
+            "zeros": torch.empty((r, 3), dtype=torch.int32, device="cuda")}
+    results = []
+    with torch.cuda.stream(s):
+        for call in range(4):
+            H.zero_()
+            g.gptq_hessian_accumulate(Xd, H, stream=s)
+            launches = g.gptq_launch_count()
+            res = g.gptq_quantize_layer(Wd, H, bits=4, group=128, workspace=ws, outputs=outs,
+                                        stream=s)
+            assert g.gptq_launch_count() > launches
+            results.append((res["loss"], outs["qweight"].cpu().numpy().copy()))
+    for loss, q in results[1:]:
+        assert loss == results[0][0]
+        np.testing.assert_array_equal(q, results[0][1])
