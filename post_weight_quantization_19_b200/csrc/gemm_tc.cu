@@ -6,18 +6,19 @@
 // block recursion that forms U -- the dense contractions of the layer solve
 // (GPTQ reading card, 方法适配: the deferred global update is a matrix product).
 //
-// Each fp32 operand x is split as hi = tf32(x) (rounded) and lo = tf32(x - hi)
-// (truncated), with integer operations; the product is hi*hi + hi*lo + lo*hi, three
-// tcgen05.mma.kind::tf32 per K step accumulating in TMEM, which keeps about
-// 21 bits of each operand (the dropped lo*lo term is ~2^-22 relative).
+// Each fp32 operand x is split as hi = tf32(x) and lo = tf32(x - hi), both
+// truncations; hi is the raw operand as the tensor core reads it.  The product
+// is hi*hi + hi*lo + lo*hi: three tcgen05.mma.kind::tf32 per K step
+// accumulating in TMEM, which keeps about 20 bits of each operand (the
+// dropped lo*lo term is ~2^-20 relative).
 //
-// Tile 128 x 128 x 32 per stage: a 4-deep TMA ring of raw A/B tiles (the hi
-// parts are written back in place) and a 3-deep ring of lo tiles.  A (and B^T) are K-major
-// with a 128-byte swizzle; a row-major B is consumed MN-major with the
-// 128-byte swizzle of 32-byte atoms (the only MN-major layout for tf32).  Warp 0 issues
-// TMA, warp 1 issues UMMA, warps 2..9 split each landed stage into hi/lo in
-// shared memory and afterwards drain the TMEM accumulator into C (two warps
-// per TMEM lane quarter, 64 columns each).
+// Tile 128 x 128 x 32 per stage: a 4-deep TMA ring of raw A/B tiles (read
+// directly as the hi parts) and a 3-deep ring of lo tiles.  A (and B^T) are
+// K-major with a 128-byte swizzle; a row-major B is consumed MN-major with the
+// 128-byte swizzle of 32-byte atoms (the only MN-major layout for tf32).
+// Warp 0 issues TMA, warp 1 issues UMMA, warps 2..9 write each landed stage's
+// lo tiles and afterwards drain the TMEM accumulator into C (two warps per
+// TMEM lane quarter, 64 columns each).
 #include <mutex>
 
 #include "gptq_internal.h"
@@ -56,13 +57,10 @@ struct TcArgs {
   int *dev_status;
 };
 
-// tf32 split with integer operations (full ALU rate, unlike conversions):
-// hi = x rounded to 10 mantissa bits (ties away from zero; a carry into the
-// exponent rounds up to the next binade), lo = x - hi exactly, then lo with
-// its low 13 bits cleared.  |x - hi - lo| <= 2^-21 |x|.
-__device__ __forceinline__ float tf32_hi(float x) {
-  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
-}
+// The tensor core reads an fp32 operand in kind::tf32 as its top 19 bits
+// (sign, exponent, 10 mantissa bits): the raw tile already is hi = trunc(x).
+// The split only has to produce lo = trunc(x - trunc(x)), with integer masks
+// (full ALU rate): |x - hi - lo| <= 2^-20 |x|.
 __device__ __forceinline__ float tf32_trunc(float x) {
   return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
 }
@@ -76,23 +74,18 @@ __device__ __forceinline__ void fail_timeout(TcShared &sh, int *dev_status) {
   *(volatile int *)&sh.abort = 1;
 }
 
-// hi/lo split of one 16 KB tile in place: x -> hi, lo buffer <- lo.
-__device__ __forceinline__ void split_tile(uint8_t *tile, uint8_t *lo, int t) {
-  float4 *p = reinterpret_cast<float4 *>(tile);
+// lo part of one 16 KB tile: lo = trunc(x - trunc(x)), same (swizzled) layout.
+__device__ __forceinline__ void split_tile(const uint8_t *tile, uint8_t *lo, int t) {
+  const float4 *p = reinterpret_cast<const float4 *>(tile);
   float4 *q = reinterpret_cast<float4 *>(lo);
 #pragma unroll 4
   for (int i = t; i < TILE_BYTES / 16; i += CONV_THREADS) {
-    float4 v = p[i];
-    float4 h, l;
-    h.x = tf32_hi(v.x);
-    h.y = tf32_hi(v.y);
-    h.z = tf32_hi(v.z);
-    h.w = tf32_hi(v.w);
-    l.x = tf32_trunc(v.x - h.x);
-    l.y = tf32_trunc(v.y - h.y);
-    l.z = tf32_trunc(v.z - h.z);
-    l.w = tf32_trunc(v.w - h.w);
-    p[i] = h;
+    const float4 v = p[i];
+    float4 l;
+    l.x = tf32_trunc(v.x - tf32_trunc(v.x));
+    l.y = tf32_trunc(v.y - tf32_trunc(v.y));
+    l.z = tf32_trunc(v.z - tf32_trunc(v.z));
+    l.w = tf32_trunc(v.w - tf32_trunc(v.w));
     q[i] = l;
   }
 }

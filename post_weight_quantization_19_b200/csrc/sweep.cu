@@ -129,13 +129,13 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
   for (int row = blockIdx.x * SWEEP_WARPS + warp; row < a.r; row += gridDim.x * SWEEP_WARPS) {
     float *wrow = a.Wk + (size_t)row * a.ldw + a.j0;
     float w[V];
-    uint32_t code[V];
+    float code[V];   // converted to bytes once, at the store
     float eo[V];
 #pragma unroll
     for (int v = 0; v < V; ++v) {
       const int c = lane * V + v;
       w[v] = c < nc ? wrow[c] : 0.f;
-      code[v] = 0;
+      code[v] = 0.f;
       eo[v] = 0.f;
     }
     float s = 1.f, z = 0.f, si = 1.f;
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
         const float e = (wj - wq) * sDinv[j];
         if (lane == jj) {
           w[v] = wq;
-          code[v] = (uint32_t)q;
+          code[v] = q;
           eo[v] = e;
         }
         esq = fmaf(e, e, esq);
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
       const int c = lane * V + v;
       if (c < nc) {
         wrow[c] = w[v];
-        a.codes[(size_t)row * a.ldc + a.j0 + c] = (uint8_t)code[v];
+        a.codes[(size_t)row * a.ldc + a.j0 + c] = (uint8_t)(int)code[v];
         a.err[(size_t)row * a.lde + c] = eo[v];
       }
     }

@@ -105,7 +105,7 @@ def test_opt175b_fc2_properties():
     gi = np.arange(d) // wl.group
     np.testing.assert_array_equal(g_idx.cpu().numpy(), gi)
     assert c.max() <= (1 << wl.bits) - 1 and zr.min() >= 0 and zr.max() <= (1 << wl.bits) - 1
-    np.testing.assert_array_equal(wh, sc[:, gi] * (c.astype(np.float32) - zr[:, gi]))
+    np.testing.assert_array_equal(wh, sc[:, gi] * (c.astype(np.float32) - zr[:, gi].astype(np.float32)))
     np.testing.assert_array_equal(q, oracle.pack_rows(c, wl.bits))
     # GPTQ's objective on the sampled rows against round-to-nearest, both from X
     _, rtn_hat = oracle.rtn(W[rows], wl.bits, wl.group)
