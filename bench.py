@@ -63,6 +63,33 @@ def _config(wl) -> dict:
     }
 
 
+# DRAM bytes (read + write) of one full-size launch of the dominant kernel, from a one-pass
+# ncu capture (profiles/hessian_tc_kernel_traffic.md).  Valid only for the kernel source it
+# was taken on: reported as null as soon as the sources hash differently.
+KERNEL_TRAFFIC = {
+    "llama7b_q_proj_4096x4096": {
+        "kernel": "hessian_tc_kernel",
+        "sources": ["post_weight_quantization_19_b200/csrc/hessian_tc.cu",
+                    "post_weight_quantization_19_b200/csrc/gptq_common.cuh"],
+        "sha256": "c460715a14acb797348c8504e4476aaed7dda78cc09441861821a5dc7a1c7085",
+        "bytes": 3705183232 + 41523712,
+    },
+}
+
+
+def _traffic(wl) -> float | None:
+    import hashlib
+
+    rec = KERNEL_TRAFFIC.get(wl.name)
+    if not rec or rec["bytes"] is None or rec["sha256"] is None:
+        return None
+    h = hashlib.sha256()
+    for rel in rec["sources"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return float(rec["bytes"]) if h.hexdigest() == rec["sha256"] else None
+
+
 def _peaks() -> dict:
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -176,8 +203,8 @@ def cpu_baseline(wl, X, W, n_s: int, r_s: int) -> dict:
 def run_reference(args, wl, rank: int, world: int):
     if rank != 0:
         return
-    X, W = workload_inputs(wl, n=min(wl.n, 4096))
-    n_s, r_s = min(wl.n, 2048), min(wl.r, 8)
+    n_s, r_s = min(wl.n, 8192), min(wl.r, 32)
+    X, W = workload_inputs(wl, n=n_s)
     for _ in range(args.warmup):
         _oracle_sample(wl, X, W, n_s, r_s)
     vals, wall = [], 0.0
@@ -343,7 +370,7 @@ def run_ours(args, wl, rank: int, world: int, dist):
         "config": _config(wl),
         "roofline": {"bound": "tensor", "kernel": "hessian_tc_kernel",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": _traffic(wl),
                      "peak_source": peak_src + " bf16 cuBLAS peak; fp16 runs at the same rate",
                      "flops_per_launch": flops, "avg_launch_ms": round(h_avg, 4)},
         "phases_ms": {"hessian": round(phase_h, 4), "damp_perm_copy": round(phases[0], 4),
