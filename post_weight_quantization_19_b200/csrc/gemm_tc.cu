@@ -12,13 +12,16 @@
 // accumulating in TMEM, which keeps about 20 bits of each operand (the
 // dropped lo*lo term is ~2^-20 relative).
 //
-// Tile 128 x 128 x 32 per stage: a 4-deep TMA ring of raw A/B tiles (read
-// directly as the hi parts) and a 3-deep ring of lo tiles.  A (and B^T) are
+// Tile 128 x 128 x 32 per stage: a 3-deep TMA ring of raw A/B tiles (read
+// directly as the hi parts) and a 2-deep ring of lo tiles.  A (and B^T) are
 // K-major with a 128-byte swizzle; a row-major B is consumed MN-major with the
 // 128-byte swizzle of 32-byte atoms (the only MN-major layout for tf32).
 // Warp 0 issues TMA, warp 1 issues UMMA, warps 2..9 write each landed stage's
-// lo tiles and afterwards drain the TMEM accumulator into C (two warps per
-// TMEM lane quarter, 64 columns each).
+// lo tiles and afterwards drain the TMEM accumulator (two warps per TMEM lane
+// quarter, 64 columns each).  The C tile travels by TMA both ways: it is
+// loaded into shared memory while the main loop runs (when beta != 0), updated
+// there in place by the epilogue warps, and stored with four bulk tensor
+// stores, so every global access of the epilogue is a full 128-byte line.
 #include <mutex>
 
 #include "gptq_internal.h"
@@ -27,13 +30,15 @@ namespace gptq {
 namespace {
 
 constexpr int TM = 128, TN = 128, TK = 32;
-constexpr int RS = 4;                       // TMA ring: raw A, B tiles (hi in place)
-constexpr int LS = 3;                       // lo ring: A_lo, B_lo tiles
+constexpr int RS = 3;                       // TMA ring: raw A, B tiles (hi in place)
+constexpr int LS = 2;                       // lo ring: A_lo, B_lo tiles
 constexpr int TILE_BYTES = 128 * TK * 4;    // 16 KB: 128 rows x 32 fp32
 constexpr int PAIR_BYTES = 2 * TILE_BYTES;  // A and B
 constexpr int THREADS = 32 * 10;
 constexpr int CONV_THREADS = 256;
-constexpr size_t SMEM_BYTES = (size_t)(RS + LS) * PAIR_BYTES + 1024;
+constexpr int C_BOX_BYTES = 128 * 32 * 4;  // one 32-column box of the C tile
+constexpr int C_BYTES = 4 * C_BOX_BYTES;    // 64 KB: the 128 x 128 C tile
+constexpr size_t SMEM_BYTES = (size_t)(RS + LS) * PAIR_BYTES + C_BYTES + 1024;
 
 struct TcShared {
   uint64_t full[RS];
@@ -42,6 +47,7 @@ struct TcShared {
   uint64_t lofree[LS];
   uint64_t accf;
   uint64_t drain;
+  uint64_t cfull;
   uint32_t tmem_base;
   int abort;
 };
@@ -69,6 +75,26 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// 2-D tiled TMA store shared -> global (bulk-group completion).  Elements of
+// the box outside the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *tmap, const void *smem_src, int x,
+                                             int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(x), "r"(y), "r"(smem_u32(smem_src))
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_and_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Epilogue warps only (warps 2..9).
+__device__ __forceinline__ void epilogue_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(CONV_THREADS) : "memory");
+}
+
 __device__ __forceinline__ void fail_timeout(TcShared &sh, int *dev_status) {
   if (dev_status) atomicCAS(dev_status, 0, (int)GPTQ_ERR_TIMEOUT);
   *(volatile int *)&sh.abort = 1;
@@ -92,7 +118,7 @@ __device__ __forceinline__ void split_tile(const uint8_t *tile, uint8_t *lo, int
 
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   TcArgs g) {
+                   const __grid_constant__ CUtensorMap tmC, TcArgs g) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ TcShared sh;
   if (g.status && *(volatile const int *)g.status) return;
@@ -120,13 +146,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(&sh.accf, 1);
     mbar_init(&sh.drain, 1);
+    mbar_init(&sh.cfull, 1);
     sh.abort = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmC);
   }
+  uint8_t *ctile = smem + (size_t)(RS + LS) * PAIR_BYTES;
+  const bool load_c = g.beta != 0.f;
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, TN);
     tmem_relinquish();
@@ -139,6 +169,17 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       uint32_t issued = 0, issued_par = 0;
+      // C is needed only by the epilogue: request it once the first ring
+      // fill (the main loop's critical path) is on its way.
+      const int c_after = min(nk, RS) - 1;
+      bool c_issued = false;
+      auto issue_c = [&]() {
+        mbar_arrive_expect_tx(&sh.cfull, C_BYTES);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_load_2d(ctile + b * C_BOX_BYTES, &tmC, n0 + 32 * b, m0, &sh.cfull);
+        c_issued = true;
+      };
+      if (load_c && c_after < 0) issue_c();
       for (int kb = 0; kb < nk; ++kb) {
         const int s = kb % RS;
         const uint32_t ph = (kb / RS) & 1;
@@ -160,9 +201,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         issued |= 1u << s;
         issued_par = (issued_par & ~(1u << s)) | (ph << s);
+        if (load_c && kb == c_after) issue_c();
       }
       for (int s = 0; s < RS; ++s)
         if (issued & (1u << s)) (void)mbar_wait_bounded(&sh.full[s], (issued_par >> s) & 1u);
+      if (c_issued) (void)mbar_wait_bounded(&sh.cfull, 0);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -228,7 +271,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;   // which 64 of the 128 columns
-    const int row = m0 + quarter * 32 + lane;
+    const int row = quarter * 32 + lane;  // row of the tile = TMEM lane
     if (ok && nk > 0) {
       if (!mbar_wait_bounded(&sh.accf, 0)) {
         if (lane == 0) fail_timeout(sh, g.dev_status);
@@ -236,38 +279,54 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_after();
     }
+    if (ok && load_c && !mbar_wait_bounded(&sh.cfull, 0)) {
+      if (lane == 0) fail_timeout(sh, g.dev_status);
+      ok = false;
+    }
     if (ok) {
+      // The C tile sits in shared memory as four 128-byte-swizzled boxes of
+      // 128 rows x 32 columns: 16-byte chunk c of a row is stored at chunk
+      // position c ^ (row & 7), so the 8 rows of each quarter-warp phase hit
+      // distinct banks.
 #pragma unroll 1
-      for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+      for (int j = 0; j < 2; ++j) {
+        const int box = 2 * half + j;
         float v[32];
         if (nk > 0) {
-          tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + c0, v);
+          tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + box * 32, v);
           tmem_wait_ld();
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = 0.f;
         }
-        if (row < g.M) {
-          float *cp = g.C + (size_t)row * g.ldc + n0 + c0;
+        uint8_t *rp = ctile + box * C_BOX_BYTES + row * 128;
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            if (n0 + c0 + i < g.N) {
-              float4 o;
-              if (g.beta != 0.f) {
-                const float4 c = *reinterpret_cast<const float4 *>(cp + i);
-                o.x = fmaf(g.alpha, v[i + 0], g.beta * c.x);
-                o.y = fmaf(g.alpha, v[i + 1], g.beta * c.y);
-                o.z = fmaf(g.alpha, v[i + 2], g.beta * c.z);
-                o.w = fmaf(g.alpha, v[i + 3], g.beta * c.w);
-              } else {
-                o = make_float4(g.alpha * v[i], g.alpha * v[i + 1], g.alpha * v[i + 2],
-                                g.alpha * v[i + 3]);
-              }
-              *reinterpret_cast<float4 *>(cp + i) = o;
-            }
+        for (int c = 0; c < 8; ++c) {
+          float4 *q = reinterpret_cast<float4 *>(rp + ((c ^ (row & 7)) << 4));
+          float4 o;
+          if (load_c) {
+            const float4 cv = *q;
+            o.x = fmaf(g.alpha, v[4 * c + 0], g.beta * cv.x);
+            o.y = fmaf(g.alpha, v[4 * c + 1], g.beta * cv.y);
+            o.z = fmaf(g.alpha, v[4 * c + 2], g.beta * cv.z);
+            o.w = fmaf(g.alpha, v[4 * c + 3], g.beta * cv.w);
+          } else {
+            o = make_float4(g.alpha * v[4 * c], g.alpha * v[4 * c + 1], g.alpha * v[4 * c + 2],
+                            g.alpha * v[4 * c + 3]);
           }
+          *q = o;
         }
       }
+      fence_async_smem();
+    }
+    // ok is the same in every epilogue warp unless a wait timed out; the
+    // barrier is passed by all of them either way.
+    epilogue_bar();
+    if (ok && tt == 0 && !*(volatile int *)&sh.abort) {
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        if (n0 + 32 * b < g.N) tma_store_2d(&tmC, ctile + b * C_BOX_BYTES, n0 + 32 * b, m0);
+      bulk_commit_and_wait_read();
     }
   }
 
@@ -323,12 +382,13 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
     set_last_error_msg(__FILE__, __LINE__, "GEMM operands not 16-byte aligned / K % 32 != 0");
     return GPTQ_ERR_INVALID_ARG;
   }
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
   const CUtensorMapSwizzle kmaj = CU_TENSOR_MAP_SWIZZLE_128B;
   const CUtensorMapSwizzle mnmaj = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
   if (!make_map(&ta, g.A, g.M, g.K, g.lda, TM, kmaj) ||
       !(trans_b ? make_map(&tb, g.B, g.N, g.K, g.ldb, TN, kmaj)
-                : make_map(&tb, g.B, g.K, g.N, g.ldb, TK, mnmaj))) {
+                : make_map(&tb, g.B, g.K, g.N, g.ldb, TK, mnmaj)) ||
+      !make_map(&tc, g.C, g.M, g.N, g.ldc, TM, kmaj)) {
     set_last_error_msg(__FILE__, __LINE__, "cuTensorMapEncodeTiled rejected a GEMM operand");
     return GPTQ_ERR_CUDA;
   }
@@ -342,7 +402,7 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
            device_status_word()};
   dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM);
   if (grid.y > 65535) return GPTQ_ERR_INVALID_ARG;
-  gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, a);
+  gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, tc, a);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }

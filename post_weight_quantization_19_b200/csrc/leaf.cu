@@ -7,15 +7,14 @@
 // come from a Cholesky kernel; the "LLM 量化技术" blog §2.3 item 3.
 //
 // The block lives in shared memory (fp32, like the rest of the solve) and is
-// processed by the same 2 x 2
-// block recursion as the full matrix,
+// processed by the same 2 x 2 block recursion as the full matrix,
 //     A22 -> U22;  T = A12 U22^T;  A11 -= T T^T;  A12 = T U22;
 //     A11 -> U11;  A12 = -U11 A12,
-// with register-tiled shared-memory products run by all 256 threads, down to
-// 32 x 32 blocks that a single warp factors and inverts in registers (one row
-// per lane, every index static, shuffles instead of CTA barriers).  The lower
-// triangle is kept at zero throughout, so the triangular operands can be used
-// as dense ones.
+// with register-tiled shared-memory products run by all LT threads, down to
+// blocks of at most BASE columns that the whole CTA factors and inverts one
+// column at a time (each thread keeps a small tile in registers; one barrier
+// per column).  The lower triangle is kept at zero between steps, so the
+// triangular operands can be used as dense ones.
 #include "gptq_internal.h"
 
 namespace gptq {
@@ -24,7 +23,9 @@ namespace {
 typedef float real;                // leaf arithmetic
 constexpr int LB = 128;            // largest block
 constexpr int LLD = LB + 1;        // shared-memory leading dimension
-constexpr int LT = 256;            // threads (255 registers each for the warp factor)
+constexpr int LT = 256;            // threads
+constexpr int GC = 16;             // column-factor thread grid: (LT / GC) x GC tiles
+constexpr int BASE = 32;           // blocks up to this size go to the column factor
 constexpr size_t LEAF_SMEM = ((size_t)LB * LLD + 64 * 64) * sizeof(real);
 
 // C[M x N] = alpha * A[M x K] * op(B) + beta * C in shared memory, all shapes
@@ -71,49 +72,87 @@ __device__ __forceinline__ void smem_gemm(real *C, const real *A, const real *B,
   __syncthreads();
 }
 
-// One warp: 32 x 32 block S (upper triangle, zeros below) -> U = R^-1.
-// Lane i holds row i.  Step k = 31..0 with p = S[k][k]:
-//   Cholesky update   S[i][j] -= S[i][k] S[j][k] / p          (i <= j < k)
-//   right-hand sides  S[i][c]  = (c == k ? 0 : S[i][c]) - S[i][k] (c == k ? 1 : S[k][c]) / p
-//                                                              (i < k <= c)
-//   row k             S[k][c]  = (c == k ? 1 : S[k][c]) / sqrt(p)   (c >= k)
-// Returns false (for every lane) on a non-positive pivot.
-__device__ __noinline__ bool warp_factor32(real *S, int ld) {
-  // The caller's tile loops may leave the warp split into divergent groups; a
-  // split warp would run every shuffle below once per group.
-  __syncwarp();
-  const int i = threadIdx.x & 31;
-  real d[32];
+// Column factor of an N x N block at S (leading dimension LLD, N = 32 or 64)
+// by all LT threads: H_d = R R^T with R upper, overwritten by U = R^-1.
+// Thread (gr, gc) of a (LT / GC) x GC grid keeps the TR x TC tile at rows
+// gr * TR, columns gc * TC in registers.  Step k = N-1 .. 0 reads a vector v
+// that holds column k above the diagonal (v_j = S[j][k], j < k), the pivot
+// p = S[k][k] at index k and row k right of the diagonal (v_j = S[k][j],
+// j > k).  With v_k taken as 1,
+//   rows i < k:  S[i][j] <- (j == k ? 0 : S[i][j]) - S[i][k] v_j / p
+//   row  k:      S[k][j] <- v_j / sqrt(p)
+// i.e. the Cholesky update of the leading block together with the
+// substitution that turns the finished rows into rows of R^-1.  Rows below k
+// are final; entries below the diagonal may pick up junk on the way and are
+// zeroed when the tile is written back.  The owners of column k-1 and row k-1
+// publish the next vector into the other half of a double buffer, so a step
+// costs one CTA barrier.  Returns false (in every thread) on a non-positive
+// pivot.
+template <int N>
+__device__ __forceinline__ bool col_factor(real *S, real *vbuf) {
+  constexpr int GR = LT / GC;
+  constexpr int TR = N / GR, TC = N / GC;
+  static_assert(TR >= 1 && TC >= 1 && TR * GR == N && TC * GC == N, "tile grid");
+  const int gr = threadIdx.x / GC, gc = threadIdx.x % GC;
+  const int i0 = gr * TR, j0 = gc * TC;
+  const bool owner = j0 + TC - 1 >= i0;   // the tile reaches the upper triangle
+  real t[TR][TC];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) d[j] = j >= i ? S[i * ld + j] : 0.f;
+  for (int r = 0; r < TR; ++r)
+#pragma unroll
+    for (int q = 0; q < TC; ++q) t[r][q] = owner ? S[(i0 + r) * LLD + j0 + q] : 0.f;
+  if (owner && j0 + TC == N) {
+#pragma unroll
+    for (int r = 0; r < TR; ++r) vbuf[((N - 1) & 1) * N + i0 + r] = t[r][TC - 1];
+  }
+  __syncthreads();
   bool bad = false;
-#pragma unroll
-  for (int k = 31; k >= 0; --k) {
-    real p = __shfl_sync(0xffffffffu, d[k], k);
+  for (int k = N - 1; k >= 0; --k) {
+    const real *vb = vbuf + (k & 1) * N;
+    real p = vb[k];
     bad |= !(p > 0.f);
     p = bad ? 1.f : p;
     real ri = rsqrtf(p);
     ri = ri * fmaf(-0.5f * p * ri, ri, 1.5f);   // one Newton step
-    const real ri2 = ri * ri;
-    const real ck = d[k];
-    // Descending j: the next pivot (row k-1, column k-1) is updated first.
+    if (owner && i0 <= k) {
+      const real mip = -ri * ri;
+      real c[TR], v[TC];
 #pragma unroll
-    for (int j = k - 1; j >= 0; --j) {
-      const real cj = __shfl_sync(0xffffffffu, d[k], j);
-      if (i <= j) d[j] = fmaf(-ck * ri2, cj, d[j]);
-    }
+      for (int r = 0; r < TR; ++r) c[r] = i0 + r < k ? vb[i0 + r] * mip : 0.f;
 #pragma unroll
-    for (int c = k; c < 32; ++c) {
-      const real rc = __shfl_sync(0xffffffffu, d[c], k);
-      if (i < k) {
-        d[c] = fmaf(-ck * ri2, c == k ? 1.f : rc, c == k ? 0.f : d[c]);
-      } else if (i == k) {
-        d[c] = (c == k ? 1.f : rc) * ri;
+      for (int q = 0; q < TC; ++q) v[q] = j0 + q == k ? 1.f : vb[j0 + q];
+#pragma unroll
+      for (int r = 0; r < TR; ++r)
+#pragma unroll
+        for (int q = 0; q < TC; ++q) t[r][q] = fmaf(c[r], v[q], j0 + q == k ? 0.f : t[r][q]);
+#pragma unroll
+      for (int r = 0; r < TR; ++r)
+        if (i0 + r == k) {
+#pragma unroll
+          for (int q = 0; q < TC; ++q) t[r][q] = v[q] * ri;
+        }
+      const int kn = k - 1;
+      if (kn >= 0) {
+        real *nb = vbuf + (kn & 1) * N;
+#pragma unroll
+        for (int r = 0; r < TR; ++r)
+#pragma unroll
+          for (int q = 0; q < TC; ++q) {
+            if (j0 + q == kn && i0 + r <= kn) nb[i0 + r] = t[r][q];
+            if (i0 + r == kn && j0 + q > kn) nb[j0 + q] = t[r][q];
+          }
       }
     }
+    __syncthreads();
   }
+  if (owner) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) S[i * ld + j] = d[j];
+    for (int r = 0; r < TR; ++r)
+#pragma unroll
+      for (int q = 0; q < TC; ++q)
+        S[(i0 + r) * LLD + j0 + q] = j0 + q >= i0 + r ? t[r][q] : 0.f;
+  }
+  __syncthreads();
   return !bad;
 }
 
@@ -121,24 +160,19 @@ __device__ __noinline__ bool warp_factor32(real *S, int ld) {
 // (32, 64, 96 or 128), so the recursion unfolds at compile time and uses no
 // call stack.
 template <int N>
-__device__ __forceinline__ bool node_factor(real *S, real *T, int off, bool *fail) {
-  if constexpr (N == 32) {
-    if (threadIdx.x < 32) {
-      const bool ok = warp_factor32(S + off * LLD + off, LLD);
-      if (threadIdx.x == 0 && !ok) *fail = true;
-    }
-    __syncthreads();
-    return !*fail;
+__device__ __forceinline__ bool node_factor(real *S, real *T, real *vbuf, int off) {
+  if constexpr (N <= BASE) {
+    return col_factor<N>(S + off * LLD + off, vbuf);
   } else {
     constexpr int h = 32 * ((N / 32) / 2), m = N - h;
-    if (!node_factor<m>(S, T, off + h, fail)) return false;
+    if (!node_factor<m>(S, T, vbuf, off + h)) return false;
     real *A11 = S + off * LLD + off;
     real *A12 = S + off * LLD + off + h;
     const real *U22 = S + (off + h) * LLD + off + h;
     smem_gemm<h, m, m, LLD, LLD, m, true, false>(T, A12, U22, 1.f, 0.f);      // R12 = A12 U22^T
     smem_gemm<h, h, m, m, m, LLD, true, true>(A11, T, T, -1.f, 1.f);          // A11 -= R12 R12^T
     smem_gemm<h, m, m, m, LLD, LLD, false, false>(A12, T, U22, 1.f, 0.f);     // A12 = R12 U22
-    if (!node_factor<h>(S, T, off, fail)) return false;
+    if (!node_factor<h>(S, T, vbuf, off)) return false;
     smem_gemm<h, m, h, LLD, LLD, m, false, false>(T, A11, A12, -1.f, 0.f);    // T = -U11 A12
     for (int idx = threadIdx.x; idx < h * m; idx += LT) {
       const int r = idx / m, c = idx - r * m;
@@ -151,7 +185,7 @@ __device__ __forceinline__ bool node_factor(real *S, real *T, int off, bool *fai
 
 __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb, int *status) {
   extern __shared__ real lsm[];
-  __shared__ bool fail;
+  __shared__ real vbuf[2 * BASE];
   if (*(volatile int *)status) return;
   real *S = lsm;
   real *T = lsm + LB * LLD;
@@ -168,14 +202,13 @@ __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb,
       s[3] = j + 3 >= i ? v.w : 0.f;
     }
   }
-  if (threadIdx.x == 0) fail = false;
   __syncthreads();
   bool ok;
   switch (nb) {
-    case 32: ok = node_factor<32>(S, T, 0, &fail); break;
-    case 64: ok = node_factor<64>(S, T, 0, &fail); break;
-    case 96: ok = node_factor<96>(S, T, 0, &fail); break;
-    default: ok = node_factor<128>(S, T, 0, &fail); break;
+    case 32: ok = node_factor<32>(S, T, vbuf, 0); break;
+    case 64: ok = node_factor<64>(S, T, vbuf, 0); break;
+    case 96: ok = node_factor<96>(S, T, vbuf, 0); break;
+    default: ok = node_factor<128>(S, T, vbuf, 0); break;
   }
   if (!ok) {
     if (threadIdx.x == 0) atomicCAS(status, 0, (int)GPTQ_ERR_NOT_PD);
