@@ -11,10 +11,12 @@
 // With U the upper Cholesky factor of H_d^-1, column j of every row does
 //   q = clamp(rint(w_j / s) + z, 0, 2^b - 1),  w^_j = s (q - z),
 //   e_j = (w_j - w^_j) / U_jj,  w_{j+1..} -= e_j U[j, j+1..].
-// Rows are independent, so one warp owns one row of the current block: lane l
-// holds columns l*V .. l*V+V-1 (V = B/32) in registers, the block of U sits in
-// shared memory, and each step is one shuffle (broadcast w_j), the quantiser,
-// and V fused multiply-adds per lane.  No inter-warp synchronisation at all.
+// Rows are independent.  One row of the current block belongs to L = B/32
+// neighbouring lanes of a warp, each holding 32 consecutive columns in
+// registers; the block of U sits in shared memory.  Column j is broadcast
+// from its lane by one shuffle, every lane of the row runs the quantiser on
+// it (the same value, so no divergence) and updates its 32 columns with
+// fused multiply-adds.  No inter-warp synchronisation at all.
 #include <float.h>
 
 #include "gptq_internal.h"
@@ -23,8 +25,9 @@
 namespace gptq {
 namespace {
 
-constexpr int SWEEP_THREADS = 512;
-constexpr int SWEEP_WARPS = SWEEP_THREADS / 32;
+constexpr int SWEEP_WARPS = 4;
+constexpr int SWEEP_THREADS = 32 * SWEEP_WARPS;
+constexpr int SWEEP_CW = 16;    // columns of a 128-column block held by one lane
 
 __device__ __forceinline__ float warp_min(float v) {
 #pragma unroll
@@ -34,6 +37,19 @@ __device__ __forceinline__ float warp_min(float v) {
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+// Over the L lanes of one row (xor offsets below L stay inside the row's lanes).
+template <int L>
+__device__ __forceinline__ float row_min(float v) {
+#pragma unroll
+  for (int o = L / 2; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+template <int L>
+__device__ __forceinline__ float row_max(float v) {
+#pragma unroll
+  for (int o = L / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
 
@@ -87,128 +103,197 @@ __global__ void row_params_kernel(const float *__restrict__ Wk, int r, int d, in
   }
 }
 
-template <int V>
+// Round to nearest even through the float adder: exact for |x| < 2^22.
+__device__ __forceinline__ float round_even(float x) {
+  const float m = 12582912.f;   // 1.5 * 2^23
+  return __fsub_rn(__fadd_rn(x, m), m);
+}
+
+// 16-byte global -> shared copy that does not wait (all of a thread's copies
+// are in flight together).
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// B = CW * L columns per block: each row is held by L lanes with CW columns each.
+template <int CW, int L>
 __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a) {
-  constexpr int B = 32 * V;
-  extern __shared__ __align__(16) float sU[];  // B x B: U[j0+j][j0+c] for c > j, else 0
+  constexpr int B = CW * L;
+  constexpr int CHUNK = CW + 4;        // stride of one lane's part of a U row in shared
+                                       // memory: the L parts start in different banks
+  constexpr int RSTRIDE = CHUNK * L;   // floats per U row in shared memory
+  constexpr int RPW = 32 / L;          // rows per warp
+  // U[j0+j][j0+c] for c > j, else 0; element (j, c) at j * RSTRIDE + (c / CW) * CHUNK + c % CW
+  extern __shared__ __align__(16) float sU[];
   __shared__ float sDinv[B];
   if (*(volatile const int *)a.status) return;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nc = a.ncols;
-  // U block -> shared memory with 16-byte loads (rows of U are contiguous and
-  // the block starts on a multiple of 32 columns); entries on or below the
-  // diagonal are zeroed, the diagonal is kept as 1/U_jj.
-  constexpr int Q = B / 4;   // float4 per row
-#pragma unroll 4
+  // U block -> shared memory with 16-byte asynchronous copies, all in flight
+  // at once (rows of U are contiguous and the block starts on a multiple of 32
+  // columns); then entries on or below the diagonal are zeroed and the
+  // diagonal is kept as 1/U_jj.
+  constexpr int Q = B / 4;   // 16-byte pieces per row
   for (int idx = tid; idx < B * Q; idx += SWEEP_THREADS) {
     const int j = idx / Q, c4 = (idx - j * Q) * 4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (j < nc && c4 < nc)
-      v = *reinterpret_cast<const float4 *>(a.U + (size_t)(a.j0 + j) * a.ldu + a.j0 + c4);
-    if (j < nc && j >= c4 && j < c4 + 4) {
-      const float dj = j == c4 ? v.x : j == c4 + 1 ? v.y : j == c4 + 2 ? v.z : v.w;
-      sDinv[j] = 1.f / dj;
-    }
-    v.x = c4 + 0 > j ? v.x : 0.f;
-    v.y = c4 + 1 > j ? v.y : 0.f;
-    v.z = c4 + 2 > j ? v.z : 0.f;
-    v.w = c4 + 3 > j ? v.w : 0.f;
-    *reinterpret_cast<float4 *>(sU + idx * 4) = v;
+    float *dst = sU + j * RSTRIDE + (c4 / CW) * CHUNK + c4 % CW;
+    if (j < nc && c4 < nc && c4 + 3 >= j)   // pieces wholly below the diagonal stay zero
+      cp_async16(dst, a.U + (size_t)(a.j0 + j) * a.ldu + a.j0 + c4);
+    else
+      *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  for (int j = nc + tid; j < B; j += SWEEP_THREADS) sDinv[j] = 0.f;
+  cp_async_wait_all();
+  __syncthreads();
+  // The piece holding the diagonal: keep 1/U_jj, zero the entries up to it.
+  for (int j = tid; j < B; j += SWEEP_THREADS) {
+    const int c4 = j & ~3;
+    float *piece = sU + j * RSTRIDE + (c4 / CW) * CHUNK + c4 % CW;
+    sDinv[j] = j < nc ? 1.f / piece[j - c4] : 0.f;
+    for (int c = c4; c <= j; ++c) piece[c - c4] = 0.f;
+  }
   __syncthreads();
 
   const float maxq = (float)((1 << a.bits) - 1);
-  const int g = a.group;
-  const int gmask = (g > 0 && g <= B) ? g - 1 : -1;         // group starts inside the block
+  const int g = a.group;   // -1 or a multiple of 32
+  const int gmask = (g > 0 && g <= B) ? g - 1 : -1;         // groups start inside the block
   const bool start_here = g > B && (a.j0 % g) == 0;         // a long group starts at column 0
   const bool inherit = g < 0 || (g > B && !start_here);     // parameters set before this block
   const int gi0 = g < 0 ? 0 : a.j0 / (g > 0 ? g : 1);
+  const int ql = lane % L;        // this lane holds columns ql*32 .. ql*32+31 of the block
+  const int base = lane - ql;     // first lane of the row
+  const int nsub = nc / CW;       // 32-column parts present in this block
+  const bool mine = ql < nsub;
 
-  for (int row = blockIdx.x * SWEEP_WARPS + warp; row < a.r; row += gridDim.x * SWEEP_WARPS) {
-    float *wrow = a.Wk + (size_t)row * a.ldw + a.j0;
-    float w[V];
-    float code[V];   // converted to bytes once, at the store
-    float eo[V];
+  for (int row0 = (blockIdx.x * SWEEP_WARPS + warp) * RPW; row0 < a.r;
+       row0 += gridDim.x * SWEEP_WARPS * RPW) {
+    // Lanes of rows past the end keep going (zeros) so the shuffles stay whole.
+    const int row = row0 + lane / L;
+    const bool valid = row < a.r;
+    float *wrow = a.Wk + (size_t)(valid ? row : 0) * a.ldw + a.j0;
+    float w[CW];
+    float code[CW];   // converted to bytes once, at the store
+    float eo[CW];
 #pragma unroll
-    for (int v = 0; v < V; ++v) {
-      const int c = lane * V + v;
-      w[v] = c < nc ? wrow[c] : 0.f;
-      code[v] = 0.f;
-      eo[v] = 0.f;
+    for (int c = 0; c < CW; c += 4) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (valid && mine) v = *reinterpret_cast<const float4 *>(wrow + ql * CW + c);
+      w[c] = v.x;
+      w[c + 1] = v.y;
+      w[c + 2] = v.z;
+      w[c + 3] = v.w;
     }
+#pragma unroll
+    for (int c = 0; c < CW; ++c) {
+      code[c] = 0.f;
+      eo[c] = 0.f;
+    }
+    const double loss0 = (ql == 0 && valid) ? a.loss_rows[row] : 0.0;   // needed at the end
     float s = 1.f, z = 0.f, si = 1.f;
-    if (inherit) {
+    if (inherit && valid) {
       s = a.scales[(size_t)row * a.G + gi0];
       z = (float)a.zeros[(size_t)row * a.G + gi0];
       si = recip(s);
     }
     float esq = 0.f;
-    // Column j = jj*V + v lives in register v of lane jj.  nc is a multiple of
-    // 32, so every lane group of V columns is either whole or absent.
-    const int njj = nc / V;
-    for (int jj = 0; jj < njj; ++jj) {
+    for (int sb = 0; sb < nsub; ++sb) {
+      const int jb = sb * CW;
+      // Groups are multiples of 32 columns, so they start only at a part's first column.
+      if ((gmask >= 0 && (jb & gmask) == 0) || (jb == 0 && start_here)) {
+        float lo = FLT_MAX, hi = -FLT_MAX;
+        const int jend = gmask >= 0 ? jb + g : B;
+        if (mine && ql >= sb && ql * CW < jend) {
 #pragma unroll
-      for (int v = 0; v < V; ++v) {
-        const int j = jj * V + v;
-        if ((gmask >= 0 && (j & gmask) == 0) || (j == 0 && start_here)) {
-          float lo = FLT_MAX, hi = -FLT_MAX;
-          const int jend = gmask >= 0 ? j + g : B;
-#pragma unroll
-          for (int u = 0; u < V; ++u) {
-            const int c = lane * V + u;
-            if (c >= j && c < jend && c < nc) {
-              lo = fminf(lo, w[u]);
-              hi = fmaxf(hi, w[u]);
-            }
-          }
-          if (gmask < 0) {
-            // A group longer than the block: its remaining columns are already
-            // up to date in global memory (every earlier column's update has
-            // landed there).
-            for (int c = B + lane; c < g; c += 32) {
-              const float x = wrow[c];
-              lo = fminf(lo, x);
-              hi = fmaxf(hi, x);
-            }
-          }
-          lo = warp_min(lo);
-          hi = warp_max(hi);
-          minmax_params(lo, hi, maxq, s, z);
-          si = recip(s);
-          if (lane == 0) {
-            const int gi = (a.j0 + j) / g;
-            a.scales[(size_t)row * a.G + gi] = s;
-            a.zeros[(size_t)row * a.G + gi] = (int32_t)z;
+          for (int c = 0; c < CW; ++c) {
+            lo = fminf(lo, w[c]);
+            hi = fmaxf(hi, w[c]);
           }
         }
-        const float wj = __shfl_sync(0xffffffffu, w[v], jj);
-        float q = rintf(wj * si) + z;
-        q = fminf(fmaxf(q, 0.f), maxq);
-        const float wq = s * (q - z);
-        const float e = (wj - wq) * sDinv[j];
-        if (lane == jj) {
-          w[v] = wq;
-          code[v] = q;
-          eo[v] = e;
+        if (gmask < 0 && valid) {
+          // A group longer than the block: its remaining columns are already
+          // up to date in global memory (every earlier column's update has
+          // landed there).
+          for (int c = B + ql; c < g; c += L) {
+            const float x = wrow[c];
+            lo = fminf(lo, x);
+            hi = fmaxf(hi, x);
+          }
+        }
+        lo = row_min<L>(lo);
+        hi = row_max<L>(hi);
+        minmax_params(lo, hi, maxq, s, z);
+        si = recip(s);
+        if (ql == 0 && valid) {
+          const int gi = (a.j0 + jb) / g;
+          a.scales[(size_t)row * a.G + gi] = s;
+          a.zeros[(size_t)row * a.G + gi] = (int32_t)z;
+        }
+      }
+      const float *ub = sU + jb * RSTRIDE + ql * CHUNK;
+      const float *dv = sDinv + jb;
+      // clamp(rint(x) + z, 0, maxq) - z == clamp(rint(x), -z, maxq - z) exactly
+      // (z is a small integer), which takes two operations off the chain.
+      // rint(x) is taken as (x + 1.5 * 2^23) - 1.5 * 2^23 in round-to-nearest-
+      // even: exact for |x| < 2^22, and for larger |x| both forms clamp to the
+      // same end of [-z, maxq - z].
+      const float tlo = -z, thi = maxq - z;
+      float wj = __shfl_sync(0xffffffffu, w[0], base + sb);
+#pragma unroll
+      for (int i = 0; i < CW; ++i) {
+        const float t = fminf(fmaxf(round_even(wj * si), tlo), thi);
+        const float wq = s * t;
+        const float e = (wj - wq) * dv[i];
+        if (ql == sb) {
+          w[i] = wq;
+          code[i] = t + z;
+          eo[i] = e;
         }
         esq = fmaf(e, e, esq);
-        const float *urow = sU + j * B + lane * V;
+        float u[CW];
+        const float4 *u4 = reinterpret_cast<const float4 *>(ub + i * RSTRIDE);
 #pragma unroll
-        for (int u = 0; u < V; ++u) w[u] = fmaf(-e, urow[u], w[u]);
+        for (int c = 0; c < CW; c += 4) {
+          const float4 v = u4[c / 4];
+          u[c] = v.x;
+          u[c + 1] = v.y;
+          u[c + 2] = v.z;
+          u[c + 3] = v.w;
+        }
+        // The next column first: its broadcast is the next step's critical path.
+        if (i + 1 < CW) {
+          w[i + 1] = fmaf(-e, u[i + 1], w[i + 1]);
+          wj = __shfl_sync(0xffffffffu, w[i + 1], base + sb);
+        }
+#pragma unroll
+        for (int c = 0; c < CW; ++c)
+          if (c != i + 1) w[c] = fmaf(-e, u[c], w[c]);
       }
     }
+    if (valid && mine) {
+      float *wp = wrow + ql * CW;
+      float *ep = a.err + (size_t)row * a.lde + ql * CW;
+      uint8_t *cp = a.codes + (size_t)row * a.ldc + a.j0 + ql * CW;
 #pragma unroll
-    for (int v = 0; v < V; ++v) {
-      const int c = lane * V + v;
-      if (c < nc) {
-        wrow[c] = w[v];
-        a.codes[(size_t)row * a.ldc + a.j0 + c] = (uint8_t)(int)code[v];
-        a.err[(size_t)row * a.lde + c] = eo[v];
+      for (int c = 0; c < CW; c += 4) {
+        *reinterpret_cast<float4 *>(wp + c) = make_float4(w[c], w[c + 1], w[c + 2], w[c + 3]);
+        *reinterpret_cast<float4 *>(ep + c) = make_float4(eo[c], eo[c + 1], eo[c + 2], eo[c + 3]);
+      }
+#pragma unroll
+      for (int c = 0; c < CW; c += 16) {
+        uint32_t wd[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          wd[k] = (uint32_t)(int)code[c + 4 * k] | ((uint32_t)(int)code[c + 4 * k + 1] << 8) |
+                  ((uint32_t)(int)code[c + 4 * k + 2] << 16) |
+                  ((uint32_t)(int)code[c + 4 * k + 3] << 24);
+        *reinterpret_cast<uint4 *>(cp + c) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
       }
     }
-    if (lane == 0) a.loss_rows[row] += 0.5 * (double)esq;
+    if (ql == 0 && valid) a.loss_rows[row] = loss0 + 0.5 * (double)esq;
   }
 }
 
@@ -336,31 +421,32 @@ int launch_row_params(const float *Wk, int r, int d, int bits, float *scales, in
   return GPTQ_OK;
 }
 
-template <int V>
+template <int CW, int L>
 static int sweep_launch(const SweepArgs &a, cudaStream_t stream) {
-  constexpr int B = 32 * V;
-  const size_t smem = (size_t)B * B * sizeof(float);
+  constexpr int B = CW * L;
+  const size_t smem = (size_t)B * (CW + 4) * L * sizeof(float);
   static bool attr = false;
   if (!attr) {
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(sweep_block_kernel<V>,
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(sweep_block_kernel<CW, L>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     attr = true;
   }
-  // One resident warp per row when the SMs can hold them all (2 CTAs of 16
-  // warps per SM), so no CTA runs a sparse second round.
-  const int want = (a.r + SWEEP_WARPS - 1) / SWEEP_WARPS;
+  // Every row gets its lanes in one wave when the SMs can hold them (two CTAs
+  // per SM: about 180 registers per thread).
+  const int rows_per_cta = SWEEP_WARPS * (32 / L);
+  const int want = (a.r + rows_per_cta - 1) / rows_per_cta;
   const int cap = num_sms() * 2;
   const int grid = want < cap ? want : cap;
-  sweep_block_kernel<V><<<grid, SWEEP_THREADS, smem, stream>>>(a);
+  sweep_block_kernel<CW, L><<<grid, SWEEP_THREADS, smem, stream>>>(a);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }
 
 int launch_sweep_block(const SweepArgs &a, int block, cudaStream_t stream) {
   switch (block) {
-    case 32: return sweep_launch<1>(a, stream);
-    case 64: return sweep_launch<2>(a, stream);
-    case 128: return sweep_launch<4>(a, stream);
+    case 32: return sweep_launch<32, 1>(a, stream);
+    case 64: return sweep_launch<32, 2>(a, stream);
+    case 128: return sweep_launch<SWEEP_CW, 128 / SWEEP_CW>(a, stream);
     default: return GPTQ_ERR_INVALID_ARG;
   }
 }
