@@ -373,7 +373,7 @@ def run_ours(args, wl, rank: int, world: int, dist):
                      "frac": round(achieved / peak, 4), "traffic": _traffic(wl),
                      "peak_source": peak_src + " bf16 cuBLAS peak; fp16 runs at the same rate",
                      "flops_per_launch": flops, "avg_launch_ms": round(h_avg, 4)},
-        "phases_ms": {"hessian": round(phase_h, 4), "damp_perm_copy": round(phases[0], 4),
+        "phases_ms": {"hessian": round(phase_h, 4), "damp_perm": round(phases[0], 4),
                       "factor_U": round(phases[1], 4), "sweep": round(phases[2], 4),
                       "finalize_pack": round(phases[3], 4)},
         "loss": loss,

@@ -224,9 +224,10 @@ uint64_t gptq_launch_count(void);
  * Phase timing for gptq_quantize_layer (off by default, process-wide, not
  * thread-safe).  When on, each call records CUDA events on its stream between
  * phases; gptq_last_phase_ms writes up to `n` durations in ms of the last call:
- *   [0] damping + act-order permutation + working copy of W
+ *   [0] damping + act-order permutation
  *   [1] Cholesky factor and triangular inverse (U)
- *   [2] column sweep (in-block kernels and trailing-update GEMMs)
+ *   [2] working copy of W and column sweep (in-block kernels and
+ *       trailing-update GEMMs)
  *   [3] unpermute, loss and packing
  * and returns the number written.
  */

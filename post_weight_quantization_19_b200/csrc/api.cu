@@ -286,7 +286,7 @@ extern "C" int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *
     GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 16, st));
     GPTQ_CUDA_TRY(cudaMemsetAsync(loss_rows, 0, (size_t)r * 8, st));
 
-    // Phase 0: damping, act-order, working copy of W.
+    // Phase 0: damping and act-order.
     float *Hf = H;
     if (act_order) {
       GPTQ_TRY(launch_damp(H, d, di, damp, false, lambda, st));
@@ -295,14 +295,17 @@ extern "C" int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *
     } else {
       GPTQ_TRY(launch_damp(H, d, di, damp, true, lambda, st));
     }
-    GPTQ_TRY(launch_gather_w(W, ri, di, act_order ? perm : nullptr, Wk, status, st));
     GPTQ_TRY(record(1, st));
 
     // Phase 1: U = upper Cholesky factor of H_d^-1, in place.
     GPTQ_TRY(launch_factor(Hf, d, T1, status, st));
     GPTQ_TRY(record(2, st));
 
-    // Phase 2: column sweep in blocks, lazy trailing updates.
+    // Phase 2: working copy of W, column sweep in blocks, lazy trailing
+    // updates.  The sweep kernels read their U block before waiting for their
+    // predecessor, so the kernel just before each of them must not write U:
+    // the copy of W separates the factorisation from the first block.
+    GPTQ_TRY(launch_gather_w(W, ri, di, act_order ? perm : nullptr, Wk, status, st));
     if (group < 0) GPTQ_TRY(launch_row_params(Wk, ri, di, bits, scales, zeros, status, st));
     for (int s0 = 0; s0 < di; s0 += S) {
       const int sEnd = s0 + S < di ? s0 + S : di;

@@ -30,6 +30,7 @@ constexpr int64_t kLeaf = 128;   // diagonal block handled by one CTA (leaf.cu)
 __global__ void __launch_bounds__(1024) damp_kernel(float *H, int64_t ld, int d, float damp,
                                                     int add_in_place, float *lambda_out) {
   __shared__ double red[32];
+  pdl_wait_then_release();
   double s = 0.0;
   for (int i = threadIdx.x; i < d; i += blockDim.x) s += (double)H[(size_t)i * ld + i];
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -55,6 +56,7 @@ __global__ void __launch_bounds__(1024) damp_kernel(float *H, int64_t ld, int d,
 __global__ void __launch_bounds__(256) rank_kernel(const float *H, int64_t ld, int d, int *perm,
                                                    int *inv) {
   __shared__ float tile[1024];
+  pdl_wait_then_release();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   const float hi = i < d ? H[(size_t)i * ld + i] : 0.f;
   int rank = 0;
@@ -79,6 +81,7 @@ __global__ void __launch_bounds__(256) rank_kernel(const float *H, int64_t ld, i
 // Hp[a][b] = H[perm[a]][perm[b]] (+ lambda on the diagonal).
 __global__ void permute_sym_kernel(const float *H, int64_t ld, int d, const int *perm,
                                    const float *lambda, float *Hp) {
+  pdl_wait_then_release();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   const int a = blockIdx.y;
   if (b >= d) return;
@@ -88,24 +91,39 @@ __global__ void permute_sym_kernel(const float *H, int64_t ld, int d, const int 
   Hp[(size_t)a * d + b] = v;
 }
 
+// dst[i][j] = src[i][j] for a rows x cols block (cols a multiple of 4, rows
+// 16-byte aligned).
+__global__ void copy_block_kernel(float *dst, int64_t ldd, const float *src, int64_t lds, int rows,
+                                  int cols, const int *status) {
+  pdl_wait_then_release();
+  if (*(volatile const int *)status) return;
+  const int q = cols / 4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)rows * q;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / q;
+    const int c = (int)(i - r * q) * 4;
+    *reinterpret_cast<float4 *>(dst + r * ldd + c) =
+        *reinterpret_cast<const float4 *>(src + r * lds + c);
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- host drivers
 
 int launch_damp(float *H, int64_t ld, int d, float damp, bool add_in_place, float *lambda,
                 cudaStream_t stream) {
-  damp_kernel<<<1, 1024, 0, stream>>>(H, ld, d, damp, add_in_place ? 1 : 0, lambda);
-  GPTQ_LAUNCH_CHECK();
+  GPTQ_LAUNCH_PDL(damp_kernel, dim3(1), dim3(1024), 0, stream, H, ld, d, damp,
+                  add_in_place ? 1 : 0, lambda);
   return GPTQ_OK;
 }
 
 int launch_act_order(const float *H, int64_t ld, int d, int *perm, int *inv, const float *lambda,
                      float *Hp, cudaStream_t stream) {
-  rank_kernel<<<(d + 255) / 256, 256, 0, stream>>>(H, ld, d, perm, inv);
-  GPTQ_LAUNCH_CHECK();
+  GPTQ_LAUNCH_PDL(rank_kernel, dim3((d + 255) / 256), dim3(256), 0, stream, H, ld, d, perm, inv);
   dim3 grid((d + 255) / 256, d);
-  permute_sym_kernel<<<grid, 256, 0, stream>>>(H, ld, d, perm, lambda, Hp);
-  GPTQ_LAUNCH_CHECK();
+  GPTQ_LAUNCH_PDL(permute_sym_kernel, grid, dim3(256), 0, stream, H, ld, d, (const int *)perm,
+                  lambda, Hp);
   return GPTQ_OK;
 }
 
@@ -145,8 +163,13 @@ int potrf_inv(float *A, int64_t ld, int64_t off, int64_t n, float *T1, int *stat
   // T1 = -U11 (R12 U22)   (U11 upper: k >= m)
   g = GemmArgs{(int)h, (int)m, (int)h, A11, ld, A12, ld, T1, m, -1.f, 0.f, GEMM_KMIN_ROW, status};
   if ((rc = launch_gemm(g, false, stream)) != GPTQ_OK) return rc;
-  GPTQ_CUDA_TRY(cudaMemcpy2DAsync(A12, ld * sizeof(float), T1, m * sizeof(float),
-                                  m * sizeof(float), h, cudaMemcpyDeviceToDevice, stream));
+  {
+    const int64_t pieces = h * (m / 4);
+    const int64_t cap = (int64_t)num_sms() * 8;
+    const int blocks = (int)((pieces + 255) / 256 < cap ? (pieces + 255) / 256 : cap);
+    GPTQ_LAUNCH_PDL(copy_block_kernel, dim3(blocks), dim3(256), 0, stream, A12, ld,
+                    (const float *)T1, m, (int)h, (int)m, (const int *)status);
+  }
   return GPTQ_OK;
 }
 

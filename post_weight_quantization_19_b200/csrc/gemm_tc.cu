@@ -121,7 +121,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                    const __grid_constant__ CUtensorMap tmC, TcArgs g) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ TcShared sh;
-  if (g.status && *(volatile const int *)g.status) return;
   const int bn = blockIdx.x, bm = blockIdx.y;
   if ((g.flags & GEMM_UPPER_C) && bn < bm) return;
   const int m0 = bm * TM, n0 = bn * TN;
@@ -155,6 +154,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmC);
   }
+  // Operands and C come from earlier kernels of the sequence.
+  pdl_wait_then_release();
+  if (threadIdx.x == 0) sh.abort = g.status ? *(volatile const int *)g.status : 0;
+  __syncthreads();
+  if (sh.abort) return;   // an earlier step failed: the same value in every thread
   uint8_t *ctile = smem + (size_t)(RS + LS) * PAIR_BYTES;
   const bool load_c = g.beta != 0.f;
   if (warp == 1) {
@@ -402,8 +406,7 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
            device_status_word()};
   dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM);
   if (grid.y > 65535) return GPTQ_ERR_INVALID_ARG;
-  gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, tc, a);
-  GPTQ_LAUNCH_CHECK();
+  GPTQ_LAUNCH_PDL(gemm_tc_kernel, grid, dim3(THREADS), SMEM_BYTES, stream, ta, tb, tc, a);
   return GPTQ_OK;
 }
 

@@ -1,9 +1,54 @@
 // Internal launch interfaces between the translation units of the library.
 #pragma once
 
+#include <utility>
+
 #include "gptq_common.cuh"
 
 namespace gptq {
+
+// ---- programmatic dependent launch ----
+// The kernels of the layer sequence are launched with programmatic stream
+// serialisation: a kernel may start while its predecessor is still running,
+// does only set-up that needs nothing from its predecessor (barriers,
+// descriptor prefetch, reads of data its predecessor does not write), then
+// waits for the predecessor grid to complete and only after that lets its own
+// successor launch.  So when a kernel starts, every grid before its
+// predecessor has completed, and at most two grids of the sequence are in
+// flight.
+__device__ __forceinline__ void pdl_wait_then_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args &&...args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// launch_pdl with the library's launch accounting and error reporting; a
+// template kernel name goes in parentheses.
+#define GPTQ_LAUNCH_PDL(kernel, grid, block, smem, stream, ...)                          \
+  do {                                                                                  \
+    ::gptq::count_launch();                                                             \
+    cudaError_t e_ = ::gptq::launch_pdl(kernel, grid, block, smem, stream, __VA_ARGS__); \
+    if (e_ != cudaSuccess) {                                                            \
+      (void)cudaGetLastError();                                                         \
+      ::gptq::set_last_error(__FILE__, __LINE__, "kernel launch", e_);                  \
+      return GPTQ_ERR_CUDA;                                                             \
+    }                                                                                   \
+  } while (0)
 
 // Tile-granular triangular structure for launch_gemm (tiles are 128 x 128 and
 // a triangular operand must hold zeros below the diagonal inside the tiles on

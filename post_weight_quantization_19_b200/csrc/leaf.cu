@@ -186,6 +186,7 @@ __device__ __forceinline__ bool node_factor(real *S, real *T, real *vbuf, int of
 __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb, int *status) {
   extern __shared__ real lsm[];
   __shared__ real vbuf[2 * BASE];
+  pdl_wait_then_release();
   if (*(volatile int *)status) return;
   real *S = lsm;
   real *T = lsm + LB * LLD;
@@ -234,8 +235,7 @@ int launch_leaf(float *A, int64_t ld, int nb, int *status, cudaStream_t stream) 
                                        (int)LEAF_SMEM));
     attr = true;
   }
-  leaf_kernel<<<1, LT, LEAF_SMEM, stream>>>(A, ld, nb, status);
-  GPTQ_LAUNCH_CHECK();
+  GPTQ_LAUNCH_PDL(leaf_kernel, dim3(1), dim3(LT), LEAF_SMEM, stream, A, ld, nb, status);
   return GPTQ_OK;
 }
 

@@ -68,6 +68,7 @@ __device__ __forceinline__ float recip(float s) { return __frcp_rn(s); }
 __global__ void gather_w_kernel(const float *__restrict__ W, int64_t total, int d,
                                 const int *__restrict__ perm, float *__restrict__ Wk,
                                 const int *status) {
+  pdl_wait_then_release();
   if (*(volatile const int *)status) return;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -82,6 +83,7 @@ __global__ void gather_w_kernel(const float *__restrict__ W, int64_t total, int 
 __global__ void row_params_kernel(const float *__restrict__ Wk, int r, int d, int bits,
                                   float *__restrict__ scales, int32_t *__restrict__ zeros,
                                   const int *status) {
+  pdl_wait_then_release();
   if (*(volatile const int *)status) return;
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -130,7 +132,6 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
   // U[j0+j][j0+c] for c > j, else 0; element (j, c) at j * RSTRIDE + (c / CW) * CHUNK + c % CW
   extern __shared__ __align__(16) float sU[];
   __shared__ float sDinv[B];
-  if (*(volatile const int *)a.status) return;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nc = a.ncols;
@@ -157,6 +158,10 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
     for (int c = c4; c <= j; ++c) piece[c - c4] = 0.f;
   }
   __syncthreads();
+  // U was finished by the factorisation, before this kernel's predecessor
+  // began; W, the parameters and the outputs belong to the sequence.
+  pdl_wait_then_release();
+  if (*(volatile const int *)a.status) return;
 
   const float maxq = (float)((1 << a.bits) - 1);
   const int g = a.group;   // -1 or a multiple of 32
@@ -307,6 +312,7 @@ __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
   constexpr int CH = 1024;
   __shared__ uint8_t sc[CH];
   __shared__ double red[8];
+  pdl_wait_then_release();
   if (*(volatile const int *)a.status) return;
   const int row = blockIdx.x;
   const size_t rb = (size_t)row * a.d;
@@ -373,6 +379,7 @@ __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
 
 __global__ void loss_reduce_kernel(const double *loss_rows, const double *dsq_rows, int r,
                                    const float *lambda, double *out, const int *status) {
+  pdl_wait_then_release();
   if (*(volatile const int *)status) return;
   __shared__ double ra[32], rb[32];
   double sa = 0.0, sb = 0.0;
@@ -409,15 +416,15 @@ int launch_gather_w(const float *W, int r, int d, const int *perm, float *Wk, co
   int64_t blocks = (total + 255) / 256;
   const int64_t cap = (int64_t)num_sms() * 16;
   if (blocks > cap) blocks = cap;
-  gather_w_kernel<<<(unsigned)blocks, 256, 0, stream>>>(W, total, d, perm, Wk, status);
-  GPTQ_LAUNCH_CHECK();
+  GPTQ_LAUNCH_PDL(gather_w_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, W, total, d, perm,
+                  Wk, status);
   return GPTQ_OK;
 }
 
 int launch_row_params(const float *Wk, int r, int d, int bits, float *scales, int32_t *zeros,
                       const int *status, cudaStream_t stream) {
-  row_params_kernel<<<(r + 7) / 8, 256, 0, stream>>>(Wk, r, d, bits, scales, zeros, status);
-  GPTQ_LAUNCH_CHECK();
+  GPTQ_LAUNCH_PDL(row_params_kernel, dim3((r + 7) / 8), dim3(256), 0, stream, Wk, r, d, bits, scales,
+                  zeros, status);
   return GPTQ_OK;
 }
 
@@ -437,8 +444,7 @@ static int sweep_launch(const SweepArgs &a, cudaStream_t stream) {
   const int want = (a.r + rows_per_cta - 1) / rows_per_cta;
   const int cap = num_sms() * 2;
   const int grid = want < cap ? want : cap;
-  sweep_block_kernel<CW, L><<<grid, SWEEP_THREADS, smem, stream>>>(a);
-  GPTQ_LAUNCH_CHECK();
+  GPTQ_LAUNCH_PDL((sweep_block_kernel<CW, L>), dim3(grid), dim3(SWEEP_THREADS), smem, stream, a);
   return GPTQ_OK;
 }
 
@@ -453,21 +459,20 @@ int launch_sweep_block(const SweepArgs &a, int block, cudaStream_t stream) {
 
 int launch_finalize(const FinalizeArgs &a, cudaStream_t stream) {
   switch (a.bits) {
-    case 2: finalize_kernel<2><<<a.r, 256, 0, stream>>>(a); break;
-    case 3: finalize_kernel<3><<<a.r, 256, 0, stream>>>(a); break;
-    case 4: finalize_kernel<4><<<a.r, 256, 0, stream>>>(a); break;
-    case 8: finalize_kernel<8><<<a.r, 256, 0, stream>>>(a); break;
+    case 2: GPTQ_LAUNCH_PDL(finalize_kernel<2>, dim3(a.r), dim3(256), 0, stream, a); break;
+    case 3: GPTQ_LAUNCH_PDL(finalize_kernel<3>, dim3(a.r), dim3(256), 0, stream, a); break;
+    case 4: GPTQ_LAUNCH_PDL(finalize_kernel<4>, dim3(a.r), dim3(256), 0, stream, a); break;
+    case 8: GPTQ_LAUNCH_PDL(finalize_kernel<8>, dim3(a.r), dim3(256), 0, stream, a); break;
     default: return GPTQ_ERR_INVALID_ARG;
   }
-  GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }
 
 int launch_loss_reduce(const double *loss_rows, const double *dsq_rows, int r,
                        const float *lambda, double *out, const int *status,
                        cudaStream_t stream) {
-  loss_reduce_kernel<<<1, 1024, 0, stream>>>(loss_rows, dsq_rows, r, lambda, out, status);
-  GPTQ_LAUNCH_CHECK();
+  GPTQ_LAUNCH_PDL(loss_reduce_kernel, dim3(1), dim3(1024), 0, stream, loss_rows, dsq_rows, r, lambda,
+                  out, status);
   return GPTQ_OK;
 }
 
