@@ -240,11 +240,12 @@ extern "C" size_t gptq_quantize_workspace_bytes(int64_t r, int64_t d, int bits, 
   return layout(r, d, group, block, act_order).total;
 }
 
-extern "C" int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits,
-                                   int group, int block, float damp, int act_order, float *W_hat,
-                                   int32_t *qweight, float *scales, int32_t *zeros,
-                                   int32_t *g_idx, uint8_t *codes, double *loss, void *workspace,
-                                   size_t workspace_bytes, gptq_stream_t stream) {
+namespace gptq {
+
+int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int group, int block,
+                   float damp, int act_order, float *W_hat, int32_t *qweight, float *scales,
+                   int32_t *zeros, int32_t *g_idx, uint8_t *codes, double *loss, void *workspace,
+                   size_t workspace_bytes, gptq_stream_t stream, bool plain) {
   if (!valid_layer(r, d, bits, group, block)) return GPTQ_ERR_INVALID_ARG;
   if (!(damp >= 0.f) || damp > 1e30f) return GPTQ_ERR_INVALID_ARG;
   if (act_order != 0 && act_order != 1) return GPTQ_ERR_INVALID_ARG;
@@ -298,7 +299,7 @@ extern "C" int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *
     GPTQ_TRY(record(1, st));
 
     // Phase 1: U = upper Cholesky factor of H_d^-1, in place.
-    GPTQ_TRY(launch_factor(Hf, d, T1, status, st));
+    GPTQ_TRY(launch_factor(Hf, d, T1, status, st, !plain));
     GPTQ_TRY(record(2, st));
 
     // Phase 2: working copy of W, column sweep in blocks, lazy trailing
@@ -377,7 +378,7 @@ extern "C" int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *
   const GraphKey key{W, H, W_hat, qweight, scales, zeros, g_idx, codes, workspace,
                      workspace_bytes, st, r, d, bits, group, block, damp, act_order};
   int rc = GPTQ_OK;
-  if (g_timing) {
+  if (g_timing || plain) {
     rc = enqueue();
   } else {
     rc = run_graph_cached(key, st, enqueue);
@@ -394,6 +395,18 @@ extern "C" int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *
   if (host_status != 0) return host_status;
   if (loss) *loss = host_out[0];
   return GPTQ_OK;
+}
+
+}  // namespace gptq
+
+extern "C" int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits,
+                                   int group, int block, float damp, int act_order, float *W_hat,
+                                   int32_t *qweight, float *scales, int32_t *zeros,
+                                   int32_t *g_idx, uint8_t *codes, double *loss, void *workspace,
+                                   size_t workspace_bytes, gptq_stream_t stream) {
+  return gptq::quantize_layer(W, r, d, H, bits, group, block, damp, act_order, W_hat, qweight,
+                              scales, zeros, g_idx, codes, loss, workspace, workspace_bytes,
+                              stream, false);
 }
 
 namespace {

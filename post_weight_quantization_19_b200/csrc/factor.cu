@@ -15,6 +15,9 @@
 // whose work is dense GEMMs with triangular operands (tensor cores, 3xTF32,
 // gemm_tc.cu), down to 128 x 128 leaves that one CTA factors and inverts in
 // registers (fp64).
+#include <mutex>
+#include <vector>
+
 #include "gptq_common.cuh"
 #include "gptq_internal.h"
 
@@ -127,56 +130,159 @@ int launch_act_order(const float *H, int64_t ld, int d, int *perm, int *inv, con
   return GPTQ_OK;
 }
 
-size_t factor_scratch_floats(int64_t d) {
-  const int64_t nblk = (d + kLeaf - 1) / kLeaf;
-  if (nblk <= 1) return 0;
-  const int64_t h = kLeaf * (nblk / 2);
-  return (size_t)h * (size_t)(d - h);
+int launch_priority(bool background) {
+  static int least = 0, greatest = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) least = greatest = 0;
+  });
+  return background ? least : greatest;
 }
 
 namespace {
 
-// Node [off, off+n) of the matrix A (leading dimension ld) -> U in place.
-int potrf_inv(float *A, int64_t ld, int64_t off, int64_t n, float *T1, int *status,
-              cudaStream_t stream) {
+// Node sizes of the recursion: a node of n columns (nblk = ceil(n/128)
+// blocks) splits into h = 128 * floor(nblk/2) leading and m = n - h trailing
+// columns.  The largest node of each depth is the trailing child of the
+// largest node of the depth above.
+void split(int64_t n, int64_t *h, int64_t *m) {
   const int64_t nblk = (n + kLeaf - 1) / kLeaf;
-  if (nblk <= 1) return launch_leaf(A + off * ld + off, ld, (int)n, status, stream);
-  const int64_t h = kLeaf * (nblk / 2);
-  const int64_t m = n - h;
+  *h = kLeaf * (nblk / 2);
+  *m = n - *h;
+}
+
+}  // namespace
+
+size_t factor_scratch_floats(int64_t d) {
+  size_t total = 0;
+  for (int64_t n = d; (n + kLeaf - 1) / kLeaf > 1;) {
+    int64_t h, m;
+    split(n, &h, &m);
+    total += (size_t)h * (size_t)m;
+    n = m;
+  }
+  return total;
+}
+
+namespace {
+
+// Per-device stream for the background products, and events to fork and
+// join it (two per recursion node).
+struct SideStream {
+  cudaStream_t s = nullptr;
+  std::vector<cudaEvent_t> ev;
+};
+
+int side_stream(int64_t d, SideStream **out) {
+  static SideStream side[64];
+  static std::mutex mu;
+  int dev = 0;
+  GPTQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return GPTQ_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(mu);
+  SideStream &ss = side[dev];
+  if (!ss.s) GPTQ_CUDA_TRY(cudaStreamCreateWithPriority(&ss.s, cudaStreamNonBlocking,
+                                                        launch_priority(true)));
+  const size_t need = 2 * (size_t)((d + kLeaf - 1) / kLeaf);
+  while (ss.ev.size() < need) {
+    cudaEvent_t e;
+    GPTQ_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    ss.ev.push_back(e);
+  }
+  *out = &ss;
+  return GPTQ_OK;
+}
+
+struct FactorRun {
+  float *A;
+  int64_t ld;
+  float *scratch;                  // factor_scratch_floats(d) floats
+  std::vector<size_t> depth_off;   // offset of each depth's product in scratch
+  int *status;
+  cudaStream_t stream;
+  SideStream *side;
+  size_t next_ev;
+};
+
+// Node [off, off+n) of A -> U in place.
+//   A22 -> U22 (recursively);  T = A12 U22^T;  A11 -= T T^T;  P = T U22;
+//   A11 -> U11 (recursively);  A12 = -U11 P.
+// P does not depend on U11, so when the node is square (h == m) it is formed
+// on the side stream, at the least priority, while A11 is factored, and it is
+// stored in the node's strictly lower block A21 (h x m there, scratch), so
+// the last product writes A12 directly.  T lives in its depth's scratch,
+// which the A11 subtree (one depth down) does not touch.
+int potrf_inv(FactorRun &fr, int64_t off, int64_t n, int depth) {
+  const int64_t nblk = (n + kLeaf - 1) / kLeaf;
+  float *A = fr.A;
+  const int64_t ld = fr.ld;
+  if (nblk <= 1) return launch_leaf(A + off * ld + off, ld, (int)n, fr.status, fr.stream);
+  int64_t h, m;
+  split(n, &h, &m);
   float *A11 = A + off * ld + off;
   float *A12 = A + off * ld + (off + h);
+  float *A21 = A + (off + h) * ld + off;
   float *A22 = A + (off + h) * ld + (off + h);
+  float *T = fr.scratch + fr.depth_off[depth];
+  int *status = fr.status;
+  cudaStream_t st = fr.stream;
   int rc;
-  if ((rc = potrf_inv(A, ld, off + h, m, T1, status, stream)) != GPTQ_OK) return rc;
-  GemmArgs g{};
-  g.status = status;
-  // R12 = A12 U22^T   (U22^T is lower: k >= n)
-  g = GemmArgs{(int)h, (int)m, (int)m, A12, ld, A22, ld, T1, m, 1.f, 0.f, GEMM_KMIN_COL, status};
-  if ((rc = launch_gemm(g, true, stream)) != GPTQ_OK) return rc;
-  // A11 -= R12 R12^T  (upper tiles)
-  g = GemmArgs{(int)h, (int)h, (int)m, T1, m, T1, m, A11, ld, -1.f, 1.f, GEMM_UPPER_C, status};
-  if ((rc = launch_gemm(g, true, stream)) != GPTQ_OK) return rc;
-  // A12 <- R12 U22    (U22 upper: k <= n)
-  g = GemmArgs{(int)h, (int)m, (int)m, T1, m, A22, ld, A12, ld, 1.f, 0.f, GEMM_KMAX_COL, status};
-  if ((rc = launch_gemm(g, false, stream)) != GPTQ_OK) return rc;
-  if ((rc = potrf_inv(A, ld, off, h, T1, status, stream)) != GPTQ_OK) return rc;
-  // T1 = -U11 (R12 U22)   (U11 upper: k >= m)
-  g = GemmArgs{(int)h, (int)m, (int)h, A11, ld, A12, ld, T1, m, -1.f, 0.f, GEMM_KMIN_ROW, status};
-  if ((rc = launch_gemm(g, false, stream)) != GPTQ_OK) return rc;
-  {
-    const int64_t pieces = h * (m / 4);
-    const int64_t cap = (int64_t)num_sms() * 8;
-    const int blocks = (int)((pieces + 255) / 256 < cap ? (pieces + 255) / 256 : cap);
-    GPTQ_LAUNCH_PDL(copy_block_kernel, dim3(blocks), dim3(256), 0, stream, A12, ld,
-                    (const float *)T1, m, (int)h, (int)m, (const int *)status);
+  if ((rc = potrf_inv(fr, off + h, m, depth + 1)) != GPTQ_OK) return rc;
+  // T = A12 U22^T   (U22^T is lower: k >= n)
+  GemmArgs g{(int)h, (int)m, (int)m, A12, ld, A22, ld, T, m, 1.f, 0.f, GEMM_KMIN_COL, status};
+  if ((rc = launch_gemm(g, true, st)) != GPTQ_OK) return rc;
+  // A11 -= T T^T  (upper tiles)
+  g = GemmArgs{(int)h, (int)h, (int)m, T, m, T, m, A11, ld, -1.f, 1.f, GEMM_UPPER_C, status};
+  if ((rc = launch_gemm(g, true, st)) != GPTQ_OK) return rc;
+  if (h == m && fr.side) {
+    cudaEvent_t fork = fr.side->ev[fr.next_ev++], join = fr.side->ev[fr.next_ev++];
+    GPTQ_CUDA_TRY(cudaEventRecord(fork, st));
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(fr.side->s, fork, 0));
+    // P = T U22 into A21   (U22 upper: k <= n)
+    g = GemmArgs{(int)h, (int)m, (int)m, T, m, A22, ld, A21, ld, 1.f, 0.f, GEMM_KMAX_COL, status,
+                 true};
+    if ((rc = launch_gemm(g, false, fr.side->s)) != GPTQ_OK) return rc;
+    GPTQ_CUDA_TRY(cudaEventRecord(join, fr.side->s));
+    if ((rc = potrf_inv(fr, off, h, depth + 1)) != GPTQ_OK) return rc;
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(st, join, 0));
+    // A12 = -U11 P   (U11 upper: k >= m)
+    g = GemmArgs{(int)h, (int)m, (int)h, A11, ld, A21, ld, A12, ld, -1.f, 0.f, GEMM_KMIN_ROW,
+                 status};
+    return launch_gemm(g, false, st);
   }
+  // A12 <- T U22
+  g = GemmArgs{(int)h, (int)m, (int)m, T, m, A22, ld, A12, ld, 1.f, 0.f, GEMM_KMAX_COL, status};
+  if ((rc = launch_gemm(g, false, st)) != GPTQ_OK) return rc;
+  if ((rc = potrf_inv(fr, off, h, depth + 1)) != GPTQ_OK) return rc;
+  // T = -U11 A12, then A12 <- T
+  g = GemmArgs{(int)h, (int)m, (int)h, A11, ld, A12, ld, T, m, -1.f, 0.f, GEMM_KMIN_ROW, status};
+  if ((rc = launch_gemm(g, false, st)) != GPTQ_OK) return rc;
+  const int64_t pieces = h * (m / 4);
+  const int64_t cap = (int64_t)num_sms() * 8;
+  const int blocks = (int)((pieces + 255) / 256 < cap ? (pieces + 255) / 256 : cap);
+  GPTQ_LAUNCH_PDL(copy_block_kernel, dim3(blocks), dim3(256), 0, st, A12, ld, (const float *)T, m,
+                  (int)h, (int)m, (const int *)status);
   return GPTQ_OK;
 }
 
 }  // namespace
 
-int launch_factor(float *A, int64_t d, float *T1, int *status, cudaStream_t stream) {
-  return potrf_inv(A, d, 0, d, T1, status, stream);
+int launch_factor(float *A, int64_t d, float *T1, int *status, cudaStream_t stream,
+                  bool use_side) {
+  FactorRun fr{A, d, T1, {}, status, stream, nullptr, 0};
+  size_t off = 0;
+  for (int64_t n = d; (n + kLeaf - 1) / kLeaf > 1;) {
+    int64_t h, m;
+    split(n, &h, &m);
+    fr.depth_off.push_back(off);
+    off += (size_t)h * (size_t)m;
+    n = m;
+  }
+  if (use_side && !fr.depth_off.empty()) {
+    const int rc = side_stream(d, &fr.side);
+    if (rc != GPTQ_OK) return rc;
+  }
+  return potrf_inv(fr, 0, d, 0);
 }
 
 }  // namespace gptq

@@ -406,7 +406,14 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
            device_status_word()};
   dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM);
   if (grid.y > 65535) return GPTQ_ERR_INVALID_ARG;
-  GPTQ_LAUNCH_PDL(gemm_tc_kernel, grid, dim3(THREADS), SMEM_BYTES, stream, ta, tb, tc, a);
+  count_launch();
+  const cudaError_t e = launch_pdl_prio(g.background, gemm_tc_kernel, grid, dim3(THREADS),
+                                        SMEM_BYTES, stream, ta, tb, tc, a);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    set_last_error(__FILE__, __LINE__, "kernel launch", e);
+    return GPTQ_ERR_CUDA;
+  }
   return GPTQ_OK;
 }
 

@@ -21,20 +21,34 @@ __device__ __forceinline__ void pdl_wait_then_release() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Scheduling priority of a launch: the layer sequence runs at the device's
+// greatest priority; work taken off its critical path (the background
+// products of the factorisation) at the least, so the SMs it frees go to the
+// critical path first.
+int launch_priority(bool background);
+
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t stream, Args &&...args) {
-  cudaLaunchAttribute attr[1];
+cudaError_t launch_pdl_prio(bool background, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                            size_t smem, cudaStream_t stream, Args &&...args) {
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributePriority;
+  attr[1].val.priority = launch_priority(background);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args &&...args) {
+  return launch_pdl_prio(false, kernel, grid, block, smem, stream, std::forward<Args>(args)...);
 }
 
 // launch_pdl with the library's launch accounting and error reporting; a
@@ -74,6 +88,7 @@ struct GemmArgs {
   float alpha, beta;
   int flags;
   const int *status;  // skip the launch's work if *status != 0 (may be NULL)
+  bool background = false;   // off the critical path: least launch priority
 };
 
 int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream);
@@ -82,10 +97,21 @@ int launch_damp(float *H, int64_t ld, int d, float damp, bool add_in_place, floa
                 cudaStream_t stream);
 int launch_act_order(const float *H, int64_t ld, int d, int *perm, int *inv, const float *lambda,
                      float *Hp, cudaStream_t stream);
+// Scratch of the factorisation: one h x m product per recursion depth.
 size_t factor_scratch_floats(int64_t d);
 // One diagonal block (nb <= 128, nb % 32 == 0) of H_d -> U in place (full block, zeros below).
 int launch_leaf(float *A, int64_t ld, int nb, int *status, cudaStream_t stream);
-int launch_factor(float *A, int64_t d, float *T1, int *status, cudaStream_t stream);
+// use_side: form the background products on a second stream (created once
+// per device, with its events); false keeps everything on `stream`.
+int launch_factor(float *A, int64_t d, float *T1, int *status, cudaStream_t stream,
+                  bool use_side);
+
+// gptq_quantize_layer; plain = true creates nothing (no CUDA graph, no second
+// stream or events) and launches every kernel directly on `stream`.
+int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int group, int block,
+                   float damp, int act_order, float *W_hat, int32_t *qweight, float *scales,
+                   int32_t *zeros, int32_t *g_idx, uint8_t *codes, double *loss, void *workspace,
+                   size_t workspace_bytes, gptq_stream_t stream, bool plain);
 
 struct SweepArgs {
   float *Wk;          // working weights r x d (sweep order), row stride ldw

@@ -72,7 +72,9 @@ extern "C" int gptq_quantize_layer_noalloc(const float *W, int64_t r, int64_t d,
   if (rc != GPTQ_OK) return rc;
   // The solve clears every part of its workspace that must start at zero, so
   // whatever an earlier call left in the array does not leak into this one.
-  return gptq_quantize_layer(W, r, d, H, bits, group, block, damp, act_order, W_hat, qweight,
-                             scales, zeros, g_idx, codes, loss, scratch, gptq::kScratchBytes,
-                             stream);
+  // The plain form launches the kernels directly: no CUDA graph and no second
+  // stream are created on this path.
+  return gptq::quantize_layer(W, r, d, H, bits, group, block, damp, act_order, W_hat, qweight,
+                              scales, zeros, g_idx, codes, loss, scratch, gptq::kScratchBytes,
+                              stream, true);
 }
