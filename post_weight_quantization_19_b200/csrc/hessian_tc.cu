@@ -5,21 +5,29 @@
 // (tokens x features) that is 2 X^T X.
 //
 // Design (B200):
-//  * H is symmetric, so only 128 x 256 output tiles that touch the upper
-//    triangle are computed (tile (I, J) with J >= floor(I/2)); the epilogue
-//    writes each upper element and its mirror exactly once.
+//  * H is symmetric, so only output tiles that touch the upper triangle are
+//    computed; the epilogue writes each upper element and its mirror once.
+//  * CTA pairs (clusters of 2) share each 256 x 256 output tile through one
+//    tcgen05.mma.cta_group::2 of M = 256, N = 256, K = 16: each CTA loads its
+//    own 128 rows of A and half (128 columns) of B, and the pair's MMA reads
+//    both halves of B from both CTAs' shared memory.  Per SM that is 32 KB of
+//    X per 64-token stage for a 128 x 256 share of the product (48 KB for a
+//    lone CTA), which matters because the operand stream from L2 is what
+//    bounds this kernel.  No TMA load is multicast.
 //  * X is token-major, so both UMMA operands are MN-major: a TMA box of
 //    64 features x 64 tokens (128-byte rows, 128-byte swizzle) is one swizzle
-//    atom column; A = X[:, i0:i0+128]^T takes two boxes, B = X[:, j0:j0+256]
-//    four.  One tcgen05.mma of M=128, N=256, K=16 consumes 16 tokens.
-//  * Warp roles: warp 0 issues TMA into a 4-stage ring, warp 1 issues UMMA
-//    into one of two 256-column TMEM accumulators, warps 2..9 drain TMEM.
+//    atom column; each CTA's A and B halves take two boxes each.
+//  * Warp roles: warp 0 issues TMA into a 6-stage ring (both CTAs; the
+//    loads complete on the leader CTA's barrier), warp 1 of the leader issues
+//    the pair's UMMAs into one of two 256-column TMEM accumulators and
+//    commits to barriers in both CTAs, warps 2..9 of each CTA drain its TMEM.
 //  * Accuracy: the tensor core's fp32 accumulation is not guaranteed to round
 //    to nearest, so each TMEM accumulation chain is limited to 512 tokens and
 //    then folded into fp32 registers of the epilogue warps (double-buffered
 //    TMEM, so the tensor core keeps running while a chain is folded).
-//  * Persistent grid of one CTA per SM walking the tile list; all CTAs sweep
-//    the tokens at the same pace, so the current X slab is shared through L2.
+//  * Persistent grid of one cluster per SM pair walking the tile list; all
+//    clusters sweep the tokens at the same pace, so the current X slab is
+//    shared through L2.
 #include <mutex>
 
 #include "gptq_common.cuh"
@@ -57,41 +65,124 @@ int num_sms() {
 
 namespace {
 
-constexpr int HM = 128;                          // tile rows  (UMMA M)
+constexpr int HM = 128;                          // tile rows per CTA (UMMA M = 256 per pair)
 constexpr int HN = 256;                          // tile cols  (UMMA N)
 constexpr int HK = 64;                           // tokens per pipeline stage
-constexpr int STAGES = 4;
+constexpr int STAGES = 6;
 constexpr int FOLD = 8;                          // stages per TMEM chain (512 tokens)
 constexpr int BOXF = 64;                         // features per TMA box (128 bytes)
 constexpr int BOX_BYTES = BOXF * HK * 2;         // 8 KB
-constexpr int A_BYTES = HM * HK * 2;             // 16 KB
-constexpr int B_BYTES = HN * HK * 2;             // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 48 KB
+constexpr int A_BYTES = HM * HK * 2;             // 16 KB: this CTA's 128 rows
+constexpr int B_BYTES = (HN / 2) * HK * 2;       // 16 KB: this CTA's half of the columns
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 32 KB
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int THREADS = 32 * (2 + NUM_EPI_WARPS);
 constexpr uint32_t TMEM_COLS = 512;              // two 256-column accumulators
 constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024;
 
 struct HessShared {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
-  uint64_t accf[2];
-  uint64_t acce[2];
-  uint64_t drain;
+  uint64_t full[STAGES];   // leader: both CTAs' loads of a stage have landed
+  uint64_t empty[STAGES];  // each CTA: the pair's MMAs are done reading its stage
+  uint64_t accf[2];        // each CTA: an accumulator buffer is complete
+  uint64_t acce[2];        // leader: both CTAs have folded an accumulator buffer
+  uint64_t drain;          // leader: every MMA issued has completed
   uint32_t tmem_base;
   int abort;
 };
 
-__device__ __forceinline__ void tile_coords(int t, int nI, int nJ, int &I, int &J) {
-  for (I = 0; I < nI; ++I) {
-    const int cnt = nJ - I / 2;
+// ---- CTA-pair primitives (cluster of two CTAs) ----
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of this CTA's shared variable `p` as seen in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr)
+               : "memory");
+}
+
+// 2-D TMA load into this CTA's shared memory whose completion is counted on an
+// mbarrier that may live in the other CTA of the pair.
+__device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorMap *tmap, int x,
+                                                 int y, uint32_t bar_addr) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar_addr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// The pair's MMA: D (both CTAs' TMEM) (+)= A (both CTAs) * B (both halves).
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on the barrier at this offset in both CTAs when the pair's
+// earlier MMAs have completed.
+__device__ __forceinline__ void umma_commit_both(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
+// Arrive on this CTA's barrier only.
+__device__ __forceinline__ void umma_commit_pair_local(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// Pair tile t -> (P, J): the 256 x 256 output block with rows 256 P .. and
+// columns 256 J .., J >= P.
+__device__ __forceinline__ void tile_coords(int t, int nP, int nJ, int &P, int &J) {
+  for (P = 0; P < nP; ++P) {
+    const int cnt = nJ - P;
     if (t < cnt) {
-      J = I / 2 + t;
+      J = P + t;
       return;
     }
     t -= cnt;
   }
-  I = nI - 1;
+  P = nP - 1;
   J = nJ - 1;
 }
 
@@ -100,7 +191,7 @@ __device__ __forceinline__ void record_timeout(int *status, HessShared &sh) {
   *(volatile int *)&sh.abort = 1;
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, int64_t n, int d,
                       float *__restrict__ H, int *__restrict__ status) {
   extern __shared__ uint8_t dyn_smem[];
@@ -110,10 +201,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int nI = (d + HM - 1) / HM;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int nJ = (d + HN - 1) / HN;
+  const int nP = nJ;   // row blocks of 256 (two CTAs of 128)
   int T = 0;
-  for (int I = 0; I < nI; ++I) T += nJ - I / 2;
+  for (int P = 0; P < nP; ++P) T += nJ - P;
   const int nsteps = (int)((n + HK - 1) / HK);
   const int nchunks = (nsteps + FOLD - 1) / FOLD;
 
@@ -124,7 +218,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.accf[b], 1);
-      mbar_init(&sh.acce[b], NUM_EPI_WARPS);
+      mbar_init(&sh.acce[b], 2 * NUM_EPI_WARPS);
     }
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -132,25 +226,30 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   if (warp == 0 && lane == 0) prefetch_tmap(&tmap);
   if (warp == 1) {
-    tmem_alloc(&sh.tmem_base, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(&sh.tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
   }
+  // Both CTAs' barriers are initialised and the pair's TMEM is allocated
+  // before either CTA signals the other.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
+      const uint32_t full0 = cluster_addr(&sh.full[0], 0);   // the leader's barriers
       uint32_t stage = 0, phase = 0;
-      uint32_t issued = 0, issued_par = 0;  // bit s: stage s has a load in flight / its parity
+      uint32_t issued = 0, issued_par = 0;  // leader: bit s = stage s armed / its parity
       bool ok = true;
-      for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
-        int I, J;
-        tile_coords(t, nI, nJ, I, J);
-        const int i0 = I * HM, j0 = J * HN;
+      for (int t = pair; t < T && ok; t += npairs) {
+        int P, J;
+        tile_coords(t, nP, nJ, P, J);
+        const int i0 = P * 2 * HM + (int)rank * HM;      // this CTA's rows
+        const int j0 = J * HN + (int)rank * (HN / 2);    // this CTA's half of the columns
         for (int ks = 0; ks < nsteps; ++ks) {
+          // A failure in the other CTA surfaces here as a bounded wait running out.
           if (*(volatile int *)&sh.abort) {
             ok = false;
             break;
@@ -163,31 +262,34 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint8_t *sA = smem + (size_t)stage * STAGE_BYTES;
           uint8_t *sB = sA + A_BYTES;
           const int y = ks * HK;
-          mbar_arrive_expect_tx(&sh.full[stage], STAGE_BYTES);
-          tma_load_2d(sA, &tmap, i0, y, &sh.full[stage]);
-          tma_load_2d(sA + BOX_BYTES, &tmap, i0 + BOXF, y, &sh.full[stage]);
-#pragma unroll
-          for (int m = 0; m < 4; ++m)
-            tma_load_2d(sB + m * BOX_BYTES, &tmap, j0 + m * BOXF, y, &sh.full[stage]);
-          issued |= 1u << stage;
-          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          const uint32_t fb = full0 + stage * (uint32_t)sizeof(uint64_t);
+          if (leader) {
+            mbar_arrive_expect_tx(&sh.full[stage], 2 * STAGE_BYTES);
+            issued |= 1u << stage;
+            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          }
+          tma_load_2d_pair(sA, &tmap, i0, y, fb);
+          tma_load_2d_pair(sA + BOX_BYTES, &tmap, i0 + BOXF, y, fb);
+          tma_load_2d_pair(sB, &tmap, j0, y, fb);
+          tma_load_2d_pair(sB + BOX_BYTES, &tmap, j0 + BOXF, y, fb);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
-      // Let every load this thread started land before the CTA can exit.
-      for (int s = 0; s < STAGES; ++s)
-        if (issued & (1u << s)) (void)mbar_wait_bounded(&sh.full[s], (issued_par >> s) & 1u);
+      // Let every armed stage land (both CTAs' loads) before the pair can exit.
+      if (leader)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) (void)mbar_wait_bounded(&sh.full[s], (issued_par >> s) & 1u);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = instr_desc(0, 0, 1, 1, HM, HN);
+    // ------------------------------------------------------------ UMMA issuer (leader)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = instr_desc(0, 0, 1, 1, 2 * HM, HN);
       uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
+      for (int t = pair; t < T && ok; t += npairs) {
         for (int c = 0; c < nchunks && ok; ++c) {
           if (!mbar_wait_bounded(&sh.acce[abuf], aphase ^ 1)) {
             record_timeout(status, sh);
@@ -212,35 +314,35 @@ __global__ void __launch_bounds__(THREADS, 1)
               // 16 tokens = two 8-row groups of the 128-byte swizzle atom.
               const uint64_t ad = smem_desc(a0 + kk * 2048, BOX_BYTES, 1024, 2);
               const uint64_t bd = smem_desc(b0 + kk * 2048, BOX_BYTES, 1024, 2);
-              umma_f16_ss(dt, ad, bd, idesc, (ks > s0 || kk > 0) ? 1u : 0u);
+              umma_f16_pair(dt, ad, bd, idesc, (ks > s0 || kk > 0) ? 1u : 0u);
             }
-            umma_commit(&sh.empty[stage]);
+            umma_commit_both(&sh.empty[stage]);
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1;
             }
           }
           if (!ok) break;
-          umma_commit(&sh.accf[abuf]);
+          umma_commit_both(&sh.accf[abuf]);
           abuf ^= 1;
           if (abuf == 0) aphase ^= 1;
         }
       }
       // Every MMA this thread issued has completed once the drain barrier fires.
-      umma_commit(&sh.drain);
+      umma_commit_pair_local(&sh.drain);
       (void)mbar_wait_bounded(&sh.drain, 0);
     }
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (both CTAs)
     const int ew = warp - 2;
     const int quarter = warp & 3;       // TMEM lanes this warp may access
     const int half = ew >> 2;           // which 128 of the 256 tile columns
     uint32_t abuf = 0, aphase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
-      int I, J;
-      tile_coords(t, nI, nJ, I, J);
-      const int i0 = I * HM, j0 = J * HN;
+    for (int t = pair; t < T && ok; t += npairs) {
+      int P, J;
+      tile_coords(t, nP, nJ, P, J);
+      const int i0 = P * 2 * HM + (int)rank * HM, j0 = J * HN;
       float acc[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.f;
@@ -262,7 +364,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.acce[abuf]);
+        if (lane == 0) mbar_arrive_cluster(cluster_addr(&sh.acce[abuf], 0));   // the leader's
         abuf ^= 1;
         if (abuf == 0) aphase ^= 1;
       }
@@ -283,11 +385,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
 
-  __syncthreads();
+  // Neither CTA leaves (or frees the pair's TMEM) while the other may still
+  // touch its shared memory, barriers or TMEM.
+  tc_fence_before();
+  cluster_sync();
   if (warp == 1) {
-    __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 
@@ -350,12 +454,13 @@ extern "C" int gptq_hessian_accumulate(const void *X, int64_t n, int64_t d, int6
   }
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(hessian_tc_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES));
-  const int nI = (int)((d + HM - 1) / HM), nJ = (int)((d + HN - 1) / HN);
+  const int nJ = (int)((d + HN - 1) / HN);
   int T = 0;
-  for (int I = 0; I < nI; ++I) T += nJ - I / 2;
-  const int grid = T < num_sms() ? T : num_sms();
-  hessian_tc_kernel<<<grid, THREADS, SMEM_BYTES, (cudaStream_t)stream>>>(tmap, n, (int)d, H,
-                                                                         status);
+  for (int P = 0; P < nJ; ++P) T += nJ - P;
+  const int max_pairs = num_sms() / 2 > 0 ? num_sms() / 2 : 1;
+  const int pairs = T < max_pairs ? T : max_pairs;
+  hessian_tc_kernel<<<2 * pairs, THREADS, SMEM_BYTES, (cudaStream_t)stream>>>(tmap, n, (int)d, H,
+                                                                              status);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }
