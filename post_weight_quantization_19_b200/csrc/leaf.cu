@@ -26,7 +26,7 @@ constexpr int LLD = LB + 1;        // shared-memory leading dimension
 constexpr int LT = 256;            // threads
 constexpr int GC = 16;             // column-factor thread grid: (LT / GC) x GC tiles
 constexpr int BASE = 32;           // blocks up to this size go to the column factor
-constexpr size_t LEAF_SMEM = ((size_t)LB * LLD + 64 * 64) * sizeof(real);
+constexpr size_t LEAF_SMEM = ((size_t)LB * LLD + 64 * 65) * sizeof(real);
 
 // C[M x N] = alpha * A[M x K] * op(B) + beta * C in shared memory, all shapes
 // and strides known at compile time; op(B) = B (K x N) or B^T (B stored N x K).
@@ -169,14 +169,17 @@ __device__ __forceinline__ bool node_factor(real *S, real *T, real *vbuf, int of
     real *A11 = S + off * LLD + off;
     real *A12 = S + off * LLD + off + h;
     const real *U22 = S + (off + h) * LLD + off + h;
-    smem_gemm<h, m, m, LLD, LLD, m, true, false>(T, A12, U22, 1.f, 0.f);      // R12 = A12 U22^T
-    smem_gemm<h, h, m, m, m, LLD, true, true>(A11, T, T, -1.f, 1.f);          // A11 -= R12 R12^T
-    smem_gemm<h, m, m, m, LLD, LLD, false, false>(A12, T, U22, 1.f, 0.f);     // A12 = R12 U22
+    // T (h x m) has an odd leading dimension so that reading it transposed
+    // (the B operand of the rank-m update) spreads over the banks.
+    constexpr int LT_ = m + 1;
+    smem_gemm<h, m, m, LLD, LLD, LT_, true, false>(T, A12, U22, 1.f, 0.f);    // R12 = A12 U22^T
+    smem_gemm<h, h, m, LT_, LT_, LLD, true, true>(A11, T, T, -1.f, 1.f);      // A11 -= R12 R12^T
+    smem_gemm<h, m, m, LT_, LLD, LLD, false, false>(A12, T, U22, 1.f, 0.f);   // A12 = R12 U22
     if (!node_factor<h>(S, T, vbuf, off)) return false;
-    smem_gemm<h, m, h, LLD, LLD, m, false, false>(T, A11, A12, -1.f, 0.f);    // T = -U11 A12
+    smem_gemm<h, m, h, LLD, LLD, LT_, false, false>(T, A11, A12, -1.f, 0.f);  // T = -U11 A12
     for (int idx = threadIdx.x; idx < h * m; idx += LT) {
       const int r = idx / m, c = idx - r * m;
-      A12[r * LLD + c] = T[r * m + c];
+      A12[r * LLD + c] = T[r * LT_ + c];
     }
     __syncthreads();
     return true;
