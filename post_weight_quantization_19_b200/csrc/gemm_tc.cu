@@ -12,13 +12,16 @@
 // accumulating in TMEM, which keeps about 20 bits of each operand (the
 // dropped lo*lo term is ~2^-20 relative).
 //
-// Tile 128 x 128 x 32 per stage: a 3-deep TMA ring of raw A/B tiles (read
-// directly as the hi parts) and a 2-deep ring of lo tiles.  A (and B^T) are
-// K-major with a 128-byte swizzle; a row-major B is consumed MN-major with the
-// 128-byte swizzle of 32-byte atoms (the only MN-major layout for tf32).
-// Warp 0 issues TMA, warp 1 issues UMMA, warps 2..9 write each landed stage's
-// lo tiles and afterwards drain the TMEM accumulator (two warps per TMEM lane
-// quarter, 64 columns each).  The C tile travels by TMA both ways: it is
+// Tile 128 x 128 x 32 per stage: a 3-deep TMA ring of raw A/B tiles and a
+// 3-deep ring of converted operands.  A (and B^T) are K-major with a 128-byte
+// swizzle; a row-major B is consumed MN-major with the 128-byte swizzle of
+// 32-byte atoms (the only MN-major layout for tf32).  The converter warps put
+// A's hi and lo parts into tensor memory (tcgen05.st; the MMAs take A from
+// TMEM) and B's lo part into shared memory (B's hi part is the raw tile), so
+// the three MMAs of a K step read only B from shared memory -- shared-memory
+// bandwidth is what bounds this three-pass product.  Warp 0 issues TMA, warp 1
+// issues UMMA, warps 2..9 convert each landed stage and afterwards drain the
+// TMEM accumulator (two warps per TMEM lane quarter, 64 columns each).  The C tile travels by TMA both ways: it is
 // loaded into shared memory while the main loop runs (when beta != 0), updated
 // there in place by the epilogue warps, and stored with four bulk tensor
 // stores, so every global access of the epilogue is a full 128-byte line.
@@ -30,15 +33,22 @@ namespace gptq {
 namespace {
 
 constexpr int TM = 128, TN = 128, TK = 32;
-constexpr int RS = 3;                       // TMA ring: raw A, B tiles (hi in place)
-constexpr int LS = 2;                       // lo ring: A_lo, B_lo tiles
+constexpr int RS = 3;                       // TMA ring: raw A, B tiles
+constexpr int LS = 3;                       // converted operands: B_lo (shared), A hi/lo (TMEM)
 constexpr int TILE_BYTES = 128 * TK * 4;    // 16 KB: 128 rows x 32 fp32
 constexpr int PAIR_BYTES = 2 * TILE_BYTES;  // A and B
 constexpr int THREADS = 32 * 10;
 constexpr int CONV_THREADS = 256;
 constexpr int C_BOX_BYTES = 128 * 32 * 4;  // one 32-column box of the C tile
 constexpr int C_BYTES = 4 * C_BOX_BYTES;    // 64 KB: the 128 x 128 C tile
-constexpr size_t SMEM_BYTES = (size_t)(RS + LS) * PAIR_BYTES + C_BYTES + 1024;
+constexpr size_t SMEM_BYTES = (size_t)RS * PAIR_BYTES + (size_t)LS * TILE_BYTES + C_BYTES + 1024;
+// TMEM columns: the 128 x 128 accumulator, then per converted stage t the A
+// hi part (32 columns, one K value each) and the A lo part (32 columns).
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_A0 = TN;
+__host__ __device__ constexpr uint32_t tmem_a_hi(int t) { return TMEM_A0 + (uint32_t)t * 2 * TK; }
+__host__ __device__ constexpr uint32_t tmem_a_lo(int t) { return tmem_a_hi(t) + TK; }
+static_assert(TMEM_A0 + LS * 2 * TK <= TMEM_COLS, "TMEM budget");
 
 struct TcShared {
   uint64_t full[RS];
@@ -88,6 +98,33 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *tmap, const void
 __device__ __forceinline__ void bulk_commit_and_wait_read() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// 32 lanes x 16 columns of 32-bit TMEM <- 16 registers per thread (thread t <-> lane t).
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const float (&v)[16]) {
+  const uint32_t *u = reinterpret_cast<const uint32_t *>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]),
+      "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]),
+      "r"(u[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem], kind::tf32.
+__device__ __forceinline__ void umma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // Epilogue warps only (warps 2..9).
@@ -159,10 +196,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) sh.abort = g.status ? *(volatile const int *)g.status : 0;
   __syncthreads();
   if (sh.abort) return;   // an earlier step failed: the same value in every thread
-  uint8_t *ctile = smem + (size_t)(RS + LS) * PAIR_BYTES;
+  uint8_t *loring = smem + (size_t)RS * PAIR_BYTES;       // B lo tiles
+  uint8_t *ctile = loring + (size_t)LS * TILE_BYTES;
   const bool load_c = g.beta != 0.f;
   if (warp == 1) {
-    tmem_alloc(&sh.tmem_base, TN);
+    tmem_alloc(&sh.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -221,16 +259,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t a = smem_u32(smem + (size_t)s * PAIR_BYTES);
-        const uint32_t b = a + TILE_BYTES;
-        const uint32_t al = smem_u32(smem + (size_t)(RS + t) * PAIR_BYTES);
-        const uint32_t bl = al + TILE_BYTES;
+        const uint32_t b = smem_u32(smem + (size_t)s * PAIR_BYTES) + TILE_BYTES;
+        const uint32_t bl = smem_u32(loring + (size_t)t * TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < TK / 8; ++kk) {
-          // A, B^T: K-major, 8 tf32 = 32 bytes per K step inside the swizzle atom.
+          // A from TMEM: 8 K values = 8 columns per K step.
+          // B^T: K-major, 8 tf32 = 32 bytes per K step inside the swizzle atom.
           // B row-major: MN-major, 8 K rows (1024 bytes) per K step.
-          const uint64_t ad = smem_desc(a + kk * 32, 16, 1024, 2);
-          const uint64_t ald = smem_desc(al + kk * 32, 16, 1024, 2);
+          const uint32_t ah = tmem + tmem_a_hi(t) + kk * 8;
+          const uint32_t al = tmem + tmem_a_lo(t) + kk * 8;
           uint64_t bd, bld;
           if (g.trans_b) {
             bd = smem_desc(b + kk * 32, 16, 1024, 2);
@@ -242,9 +279,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             bld = smem_desc(bl + kk * 1024, TK * 128, 512, 1);
           }
           const uint32_t acc0 = (kb > 0 || kk > 0) ? 1u : 0u;
-          umma_tf32_ss(tmem, ad, bd, idesc, acc0);
-          umma_tf32_ss(tmem, ad, bld, idesc, 1u);
-          umma_tf32_ss(tmem, ald, bd, idesc, 1u);
+          umma_tf32_ts(tmem, ah, bd, idesc, acc0);
+          umma_tf32_ts(tmem, ah, bld, idesc, 1u);
+          umma_tf32_ts(tmem, al, bd, idesc, 1u);
         }
         umma_commit(&sh.empty[s]);
         umma_commit(&sh.lofree[t]);
@@ -266,10 +303,33 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       uint8_t *st = smem + (size_t)s * PAIR_BYTES;
-      uint8_t *lo = smem + (size_t)(RS + t) * PAIR_BYTES;
-      split_tile(st, lo, tt);
-      split_tile(st + TILE_BYTES, lo + TILE_BYTES, tt);
+      split_tile(st + TILE_BYTES, loring + (size_t)t * TILE_BYTES, tt);
+      {
+        // A: this thread's row (TMEM lane) and 16 of the 32 K values; the raw
+        // tile is K-major with the 128-byte swizzle (16-byte chunk c of row r
+        // at chunk position c ^ (r & 7)).
+        const int q = warp & 3, hf = (warp - 2) >> 2;
+        const int r = q * 32 + lane;
+        const uint8_t *rowp = st + r * 128;
+        float hi[16], lo[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float4 v =
+              *reinterpret_cast<const float4 *>(rowp + (((hf * 4 + c) ^ (r & 7)) << 4));
+          hi[4 * c + 0] = v.x;
+          hi[4 * c + 1] = v.y;
+          hi[4 * c + 2] = v.z;
+          hi[4 * c + 3] = v.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) lo[i] = tf32_trunc(hi[i] - tf32_trunc(hi[i]));
+        const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + hf * 16;
+        tmem_st_32x32b_x16(lane_base + tmem_a_hi(t), hi);
+        tmem_st_32x32b_x16(lane_base + tmem_a_lo(t), lo);
+        tmem_wait_st();
+      }
       fence_async_smem();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.conv[t]);
     }
@@ -339,7 +399,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, TN);
+    tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
