@@ -71,8 +71,8 @@ KERNEL_TRAFFIC = {
         "kernel": "hessian_tc_kernel",
         "sources": ["post_weight_quantization_19_b200/csrc/hessian_tc.cu",
                     "post_weight_quantization_19_b200/csrc/gptq_common.cuh"],
-        "sha256": "c460715a14acb797348c8504e4476aaed7dda78cc09441861821a5dc7a1c7085",
-        "bytes": 3705183232 + 41523712,
+        "sha256": "53c32a78488a3a1be69bbb69f51edb36d0ae8754eef01037ae5f30d86b1c4e17",
+        "bytes": 7386331136 + 51261184,
     },
 }
 
