@@ -11,7 +11,7 @@
 //     A22 -> U22;  T = A12 U22^T;  A11 -= T T^T;  A12 = T U22;
 //     A11 -> U11;  A12 = -U11 A12,
 // with register-tiled shared-memory products run by all LT threads, down to
-// blocks of at most BASE columns that the whole CTA factors and inverts one
+// blocks of at most BASE columns that CF_THREADS threads factor and invert one
 // column at a time (each thread keeps a small tile in registers; one barrier
 // per column).  The lower triangle is kept at zero between steps, so the
 // triangular operands can be used as dense ones.
@@ -22,59 +22,108 @@ namespace {
 
 typedef float real;                // leaf arithmetic
 constexpr int LB = 128;            // largest block
-constexpr int LLD = LB + 1;        // shared-memory leading dimension
+constexpr int LLD = LB + 4;        // shared-memory leading dimension (16-byte rows)
 constexpr int LT = 256;            // threads
-constexpr int GC = 16;             // column-factor thread grid: (LT / GC) x GC tiles
+constexpr int GC = 16;             // column-factor thread grid: (CF_THREADS / GC) x GC tiles
+constexpr int CF_THREADS = LT;     // threads of the column factor
 constexpr int BASE = 32;           // blocks up to this size go to the column factor
-constexpr size_t LEAF_SMEM = ((size_t)LB * LLD + 64 * 65) * sizeof(real);
+constexpr size_t LEAF_SMEM = ((size_t)LB * LLD + 64 * 68) * sizeof(real);
 
 // C[M x N] = alpha * A[M x K] * op(B) + beta * C in shared memory, all shapes
 // and strides known at compile time; op(B) = B (K x N) or B^T (B stored N x K).
-// The M x N outputs are spread over all threads in RM x RN register tiles.
-// UPPER: only entries with column >= row are written (C is a diagonal block).
-// Ends with a CTA barrier.
+// The M x N outputs are spread over all threads in RM x RN register tiles; A
+// (and B^T) are read 4 k values at a time with 16-byte loads.  A thread's
+// columns are interleaved (jt + TN c) when B is read transposed, so the B rows
+// of neighbouring threads fall in different banks, and contiguous otherwise,
+// for 16-byte loads of a B row.  UPPER: only entries with column >= row are
+// written (C is a diagonal block).  Ends with a CTA barrier.
 template <int M, int N, int K, int LDA, int LDB, int LDC, bool TB, bool UPPER>
 __device__ __forceinline__ void smem_gemm(real *C, const real *A, const real *B, real alpha,
                                           real beta) {
+  static_assert(K % 4 == 0 && LDA % 4 == 0 && LDB % 4 == 0 && LDC % 4 == 0, "16-byte rows");
   constexpr int RM = (M * N >= 16 * LT) ? 4 : 2;
   constexpr int RN = (M * N >= 8 * LT) ? 4 : 2;
   constexpr int TN = N / RN;
   constexpr int NT = (M / RM) * TN;
   for (int tile = threadIdx.x; tile < NT; tile += LT) {
-    const int i0 = (tile / TN) * RM, j0 = (tile % TN) * RN;
-    if (UPPER && j0 + RN - 1 < i0) continue;
+    const int i0 = (tile / TN) * RM, jt = tile % TN;
+    auto col = [&](int c) { return TB ? jt + TN * c : jt * RN + c; };
+    if (UPPER && col(RN - 1) < i0) continue;
     real acc[RM][RN];
 #pragma unroll
     for (int r = 0; r < RM; ++r)
 #pragma unroll
       for (int c = 0; c < RN; ++c) acc[r][c] = 0.f;
-#pragma unroll 16
-    for (int k = 0; k < K; ++k) {
-      real a[RM], b[RN];
+#pragma unroll 4
+    for (int k = 0; k < K; k += 4) {
+      float4 a4[RM];
 #pragma unroll
-      for (int r = 0; r < RM; ++r) a[r] = A[(i0 + r) * LDA + k];
+      for (int r = 0; r < RM; ++r) a4[r] = *reinterpret_cast<const float4 *>(A + (i0 + r) * LDA + k);
+      real a[RM][4];
 #pragma unroll
-      for (int c = 0; c < RN; ++c) b[c] = TB ? B[(j0 + c) * LDB + k] : B[k * LDB + j0 + c];
+      for (int r = 0; r < RM; ++r) {
+        a[r][0] = a4[r].x;
+        a[r][1] = a4[r].y;
+        a[r][2] = a4[r].z;
+        a[r][3] = a4[r].w;
+      }
+      real b[4][RN];
+      if (TB) {
 #pragma unroll
-      for (int r = 0; r < RM; ++r)
+        for (int c = 0; c < RN; ++c) {
+          const float4 v = *reinterpret_cast<const float4 *>(B + col(c) * LDB + k);
+          b[0][c] = v.x;
+          b[1][c] = v.y;
+          b[2][c] = v.z;
+          b[3][c] = v.w;
+        }
+      } else {
 #pragma unroll
-        for (int c = 0; c < RN; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+        for (int kk = 0; kk < 4; ++kk) {
+          const real *br = B + (k + kk) * LDB + jt * RN;
+          if constexpr (RN == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(br);
+            b[kk][0] = v.x;
+            b[kk][1] = v.y;
+            b[kk][2] = v.z;
+            b[kk][3] = v.w;
+          } else {
+            const float2 v = *reinterpret_cast<const float2 *>(br);
+            b[kk][0] = v.x;
+            b[kk][1] = v.y;
+          }
+        }
+      }
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int r = 0; r < RM; ++r)
+#pragma unroll
+          for (int c = 0; c < RN; ++c) acc[r][c] = fmaf(a[r][kk], b[kk][c], acc[r][c]);
     }
 #pragma unroll
     for (int r = 0; r < RM; ++r)
 #pragma unroll
       for (int c = 0; c < RN; ++c) {
-        if (UPPER && j0 + c < i0 + r) continue;
-        real *p = C + (i0 + r) * LDC + j0 + c;
+        if (UPPER && col(c) < i0 + r) continue;
+        real *p = C + (i0 + r) * LDC + col(c);
         *p = alpha * acc[r][c] + (beta != 0.f ? beta * *p : 0.f);
       }
   }
   __syncthreads();
 }
 
+// Barrier of the column factor's threads only (warps 0 .. CF_THREADS/32 - 1).
+__device__ __forceinline__ void cf_barrier() {
+  if constexpr (CF_THREADS == LT)
+    __syncthreads();
+  else
+    asm volatile("bar.sync 1, %0;" ::"n"(CF_THREADS) : "memory");
+}
+
 // Column factor of an N x N block at S (leading dimension LLD, N = 32 or 64)
-// by all LT threads: H_d = R R^T with R upper, overwritten by U = R^-1.
-// Thread (gr, gc) of a (LT / GC) x GC grid keeps the TR x TC tile at rows
+// by CF_THREADS threads: H_d = R R^T with R upper, overwritten by U = R^-1.
+// Thread (gr, gc) of a (CF_THREADS / GC) x GC grid keeps the TR x TC tile at rows
 // gr * TR, columns gc * TC in registers.  Step k = N-1 .. 0 reads a vector v
 // that holds column k above the diagonal (v_j = S[j][k], j < k), the pivot
 // p = S[k][k] at index k and row k right of the diagonal (v_j = S[k][j],
@@ -90,7 +139,12 @@ __device__ __forceinline__ void smem_gemm(real *C, const real *A, const real *B,
 // pivot.
 template <int N>
 __device__ __forceinline__ bool col_factor(real *S, real *vbuf) {
-  constexpr int GR = LT / GC;
+  __shared__ int cf_ok;
+  if (threadIdx.x >= CF_THREADS) {   // the other warps wait at the closing barrier
+    __syncthreads();
+    return cf_ok != 0;
+  }
+  constexpr int GR = CF_THREADS / GC;
   constexpr int TR = N / GR, TC = N / GC;
   static_assert(TR >= 1 && TC >= 1 && TR * GR == N && TC * GC == N, "tile grid");
   const int gr = threadIdx.x / GC, gc = threadIdx.x % GC;
@@ -105,8 +159,10 @@ __device__ __forceinline__ bool col_factor(real *S, real *vbuf) {
 #pragma unroll
     for (int r = 0; r < TR; ++r) vbuf[((N - 1) & 1) * N + i0 + r] = t[r][TC - 1];
   }
-  __syncthreads();
+  cf_barrier();
   bool bad = false;
+  // Fully unrolled: every comparison with k below becomes static.
+#pragma unroll
   for (int k = N - 1; k >= 0; --k) {
     const real *vb = vbuf + (k & 1) * N;
     real p = vb[k];
@@ -143,7 +199,7 @@ __device__ __forceinline__ bool col_factor(real *S, real *vbuf) {
           }
       }
     }
-    __syncthreads();
+    cf_barrier();
   }
   if (owner) {
 #pragma unroll
@@ -152,6 +208,7 @@ __device__ __forceinline__ bool col_factor(real *S, real *vbuf) {
       for (int q = 0; q < TC; ++q)
         S[(i0 + r) * LLD + j0 + q] = j0 + q >= i0 + r ? t[r][q] : 0.f;
   }
+  if (threadIdx.x == 0) cf_ok = !bad;
   __syncthreads();
   return !bad;
 }
@@ -169,9 +226,9 @@ __device__ __forceinline__ bool node_factor(real *S, real *T, real *vbuf, int of
     real *A11 = S + off * LLD + off;
     real *A12 = S + off * LLD + off + h;
     const real *U22 = S + (off + h) * LLD + off + h;
-    // T (h x m) has an odd leading dimension so that reading it transposed
-    // (the B operand of the rank-m update) spreads over the banks.
-    constexpr int LT_ = m + 1;
+    // T (h x m): leading dimension m + 4, so rows stay 16-byte aligned and
+    // the rows that neighbouring threads read transposed fall in different banks.
+    constexpr int LT_ = m + 4;
     smem_gemm<h, m, m, LLD, LLD, LT_, true, false>(T, A12, U22, 1.f, 0.f);    // R12 = A12 U22^T
     smem_gemm<h, h, m, LT_, LT_, LLD, true, true>(A11, T, T, -1.f, 1.f);      // A11 -= R12 R12^T
     smem_gemm<h, m, m, LT_, LLD, LLD, false, false>(A12, T, U22, 1.f, 0.f);   // A12 = R12 U22
@@ -199,11 +256,9 @@ __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb,
     const int i = idx >> 5, j = (idx & 31) * 4;
     if (i < nb && j < nb) {
       const float4 v = *reinterpret_cast<const float4 *>(A + (size_t)i * lda + j);
-      real *s = S + i * LLD + j;
-      s[0] = j + 0 >= i ? v.x : 0.f;
-      s[1] = j + 1 >= i ? v.y : 0.f;
-      s[2] = j + 2 >= i ? v.z : 0.f;
-      s[3] = j + 3 >= i ? v.w : 0.f;
+      *reinterpret_cast<float4 *>(S + i * LLD + j) =
+          make_float4(j + 0 >= i ? v.x : 0.f, j + 1 >= i ? v.y : 0.f, j + 2 >= i ? v.z : 0.f,
+                      j + 3 >= i ? v.w : 0.f);
     }
   }
   __syncthreads();
@@ -221,10 +276,9 @@ __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb,
 #pragma unroll 4
   for (int idx = threadIdx.x; idx < LB * (LB / 4); idx += LT) {
     const int i = idx >> 5, j = (idx & 31) * 4;
-    if (i < nb && j < nb) {
-      const real *s = S + i * LLD + j;
-      *reinterpret_cast<float4 *>(A + (size_t)i * lda + j) = make_float4(s[0], s[1], s[2], s[3]);
-    }
+    if (i < nb && j < nb)
+      *reinterpret_cast<float4 *>(A + (size_t)i * lda + j) =
+          *reinterpret_cast<const float4 *>(S + i * LLD + j);
   }
 }
 
