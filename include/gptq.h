@@ -193,6 +193,10 @@ int gptq_quantize_layer_noalloc(const float *W, int64_t r, int64_t d, float *H, 
  *   dev_workspace  device scratch of gptq_layer_host_workspace_bytes(...) bytes,
  *            256-byte aligned; it holds the device copies of X, W, H and the
  *            outputs plus the quantiser's workspace.
+ *   X is copied in chunks of max(32768, ceil(n/64)) tokens on a second stream
+ *   (created once per device) and H is accumulated chunk by chunk as the chunks
+ *   land -- the same H as gptq_hessian_accumulate called once per chunk -- so
+ *   the Hessian overlaps the upload.
  *   Synchronous: returns when the outputs are in the host buffers.
  */
 size_t gptq_layer_host_workspace_bytes(int64_t r, int64_t d, int64_t n, int bits, int group,

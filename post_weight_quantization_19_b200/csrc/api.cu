@@ -415,6 +415,37 @@ struct HostLayout {
   size_t X, H, W, qw, sc, zr, gi, qws, total;
 };
 
+// Per-device stream for the host-to-device copies of the end-to-end entry
+// point, and events to hand each copied chunk to the computing stream.
+struct CopyStream {
+  cudaStream_t s = nullptr;
+  std::vector<cudaEvent_t> ev;
+};
+
+int copy_stream(size_t events, CopyStream **out) {
+  static CopyStream cs[64];
+  static std::mutex mu;
+  int dev = 0;
+  GPTQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return GPTQ_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(mu);
+  CopyStream &c = cs[dev];
+  if (!c.s) GPTQ_CUDA_TRY(cudaStreamCreateWithFlags(&c.s, cudaStreamNonBlocking));
+  while (c.ev.size() < events) {
+    cudaEvent_t e;
+    GPTQ_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    c.ev.push_back(e);
+  }
+  *out = &c;
+  return GPTQ_OK;
+}
+
+// Tokens per copied chunk of X: at least 32768, at most 64 chunks.
+int64_t x_chunk_tokens(int64_t n) {
+  const int64_t c = (n + 63) / 64;
+  return c > 32768 ? c : 32768;
+}
+
 HostLayout host_layout(int64_t r, int64_t d, int64_t n, int bits, int group, int block,
                        int act_order) {
   HostLayout L{};
@@ -473,11 +504,27 @@ extern "C" int gptq_solve_layer_host(const uint16_t *X_host, int64_t n, const fl
   int32_t *gi = reinterpret_cast<int32_t *>(ws + L.gi);
   const int64_t G = group < 0 ? 1 : d / group;
 
-  if (n > 0)
-    GPTQ_CUDA_TRY(cudaMemcpyAsync(X, X_host, (size_t)n * d * 2, cudaMemcpyHostToDevice, st));
-  GPTQ_CUDA_TRY(cudaMemcpyAsync(W, W_host, (size_t)r * d * 4, cudaMemcpyHostToDevice, st));
+  // X travels in token chunks on a copy stream; the Hessian of each chunk is
+  // accumulated on `stream` as soon as the chunk has landed, so the tensor-core
+  // work hides behind the host-to-device copy of the next chunk.
+  const int64_t chunk = x_chunk_tokens(n);
+  const int64_t nch = n > 0 ? (n + chunk - 1) / chunk : 0;
+  CopyStream *cs = nullptr;
+  GPTQ_TRY(copy_stream((size_t)nch + 2, &cs));
+  GPTQ_CUDA_TRY(cudaEventRecord(cs->ev[0], st));   // the workspace is free on `stream`
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(cs->s, cs->ev[0], 0));
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(W, W_host, (size_t)r * d * 4, cudaMemcpyHostToDevice, cs->s));
   GPTQ_CUDA_TRY(cudaMemsetAsync(H, 0, (size_t)d * d * 4, st));
-  GPTQ_TRY(gptq_hessian_accumulate(X, n, d, d, H, stream));
+  for (int64_t c = 0; c < nch; ++c) {
+    const int64_t t0 = c * chunk, tn = (n - t0) < chunk ? (n - t0) : chunk;
+    GPTQ_CUDA_TRY(cudaMemcpyAsync(X + t0 * d, X_host + t0 * d, (size_t)tn * d * 2,
+                                  cudaMemcpyHostToDevice, cs->s));
+    GPTQ_CUDA_TRY(cudaEventRecord(cs->ev[c + 1], cs->s));
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(st, cs->ev[c + 1], 0));
+    GPTQ_TRY(gptq_hessian_accumulate(X + t0 * d, tn, d, d, H, stream));
+  }
+  GPTQ_CUDA_TRY(cudaEventRecord(cs->ev[nch + 1], cs->s));   // W (copied first) and all of X
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(st, cs->ev[nch + 1], 0));
   GPTQ_TRY(gptq_quantize_layer(W, r, d, H, bits, group, block, damp, act_order, nullptr, qw, sc,
                                zr, gi, nullptr, loss, ws + L.qws, L.total - L.qws, stream));
   GPTQ_CUDA_TRY(cudaMemcpyAsync(qweight_host, qw, (size_t)r * (d * bits / 32) * 4,

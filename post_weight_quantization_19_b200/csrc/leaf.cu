@@ -23,9 +23,9 @@ namespace {
 typedef float real;                // leaf arithmetic
 constexpr int LB = 128;            // largest block
 constexpr int LLD = LB + 4;        // shared-memory leading dimension (16-byte rows)
-constexpr int LT = 256;            // threads
+constexpr int LT = 512;            // threads (the products; more loads in flight)
 constexpr int GC = 16;             // column-factor thread grid: (CF_THREADS / GC) x GC tiles
-constexpr int CF_THREADS = LT;     // threads of the column factor
+constexpr int CF_THREADS = 256;    // threads of the column factor (a named barrier)
 constexpr int BASE = 32;           // blocks up to this size go to the column factor
 constexpr size_t LEAF_SMEM = ((size_t)LB * LLD + 64 * 68) * sizeof(real);
 
