@@ -94,22 +94,6 @@ __global__ void permute_sym_kernel(const float *H, int64_t ld, int d, const int 
   Hp[(size_t)a * d + b] = v;
 }
 
-// dst[i][j] = src[i][j] for a rows x cols block (cols a multiple of 4, rows
-// 16-byte aligned).
-__global__ void copy_block_kernel(float *dst, int64_t ldd, const float *src, int64_t lds, int rows,
-                                  int cols, const int *status) {
-  pdl_wait_then_release();
-  if (*(volatile const int *)status) return;
-  const int q = cols / 4;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)rows * q;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = i / q;
-    const int c = (int)(i - r * q) * 4;
-    *reinterpret_cast<float4 *>(dst + r * ldd + c) =
-        *reinterpret_cast<const float4 *>(src + r * lds + c);
-  }
-}
-
 }  // namespace
 
 // ---------------------------------------------------------------- host drivers
@@ -141,7 +125,7 @@ int launch_priority(bool background) {
 
 namespace {
 
-// Node sizes of the recursion: a node of n columns (nblk = ceil(n/128)
+// Node sizes of the merge tree: a node of n columns (nblk = ceil(n/128)
 // blocks) splits into h = 128 * floor(nblk/2) leading and m = n - h trailing
 // columns.  The largest node of each depth is the trailing child of the
 // largest node of the depth above.
@@ -166,25 +150,28 @@ size_t factor_scratch_floats(int64_t d) {
 
 namespace {
 
-// Per-device stream for the background products, and events to fork and
-// join it (two per recursion node).
-struct SideStream {
-  cudaStream_t s = nullptr;
+// Per-device streams for the work taken off the critical path -- the trailing
+// rank-128 updates and the merges that assemble U -- and events to order them.
+struct SideStreams {
+  cudaStream_t trail = nullptr, merge = nullptr;
   std::vector<cudaEvent_t> ev;
 };
 
-int side_stream(int64_t d, SideStream **out) {
-  static SideStream side[64];
+int side_streams(size_t events, SideStreams **out) {
+  static SideStreams side[64];
   static std::mutex mu;
   int dev = 0;
   GPTQ_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return GPTQ_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(mu);
-  SideStream &ss = side[dev];
-  if (!ss.s) GPTQ_CUDA_TRY(cudaStreamCreateWithPriority(&ss.s, cudaStreamNonBlocking,
-                                                        launch_priority(true)));
-  const size_t need = 2 * (size_t)((d + kLeaf - 1) / kLeaf);
-  while (ss.ev.size() < need) {
+  SideStreams &ss = side[dev];
+  if (!ss.trail) {
+    GPTQ_CUDA_TRY(cudaStreamCreateWithPriority(&ss.trail, cudaStreamNonBlocking,
+                                               launch_priority(true)));
+    GPTQ_CUDA_TRY(cudaStreamCreateWithPriority(&ss.merge, cudaStreamNonBlocking,
+                                               launch_priority(true)));
+  }
+  while (ss.ev.size() < events) {
     cudaEvent_t e;
     GPTQ_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
     ss.ev.push_back(e);
@@ -193,96 +180,169 @@ int side_stream(int64_t d, SideStream **out) {
   return GPTQ_OK;
 }
 
-struct FactorRun {
-  float *A;
-  int64_t ld;
-  float *scratch;                  // factor_scratch_floats(d) floats
-  std::vector<size_t> depth_off;   // offset of each depth's product in scratch
-  int *status;
-  cudaStream_t stream;
-  SideStream *side;
-  size_t next_ev;
+// A node of the merge tree: columns [off, off + h + m), split at off + h.
+struct MergeNode {
+  int64_t off, h, m;
+  int depth;
 };
 
-// Node [off, off+n) of A -> U in place.
-//   A22 -> U22 (recursively);  T = A12 U22^T;  A11 -= T T^T;  P = T U22;
-//   A11 -> U11 (recursively);  A12 = -U11 P.
-// P does not depend on U11, so when the node is square (h == m) it is formed
-// on the side stream, at the least priority, while A11 is factored, and it is
-// stored in the node's strictly lower block A21 (h x m there, scratch), so
-// the last product writes A12 directly.  T lives in its depth's scratch,
-// which the A11 subtree (one depth down) does not touch.
-int potrf_inv(FactorRun &fr, int64_t off, int64_t n, int depth) {
-  const int64_t nblk = (n + kLeaf - 1) / kLeaf;
-  float *A = fr.A;
-  const int64_t ld = fr.ld;
-  if (nblk <= 1) return launch_leaf(A + off * ld + off, ld, (int)n, fr.status, fr.stream);
+void merge_nodes(int64_t off, int64_t n, int depth, std::vector<MergeNode> &out) {
+  if ((n + kLeaf - 1) / kLeaf <= 1) return;
   int64_t h, m;
   split(n, &h, &m);
+  merge_nodes(off + h, m, depth + 1, out);
+  merge_nodes(off, h, depth + 1, out);
+  out.push_back(MergeNode{off, h, m, depth});   // after both children
+}
+
+// U12 = -U11 R12 U22 for one node, once U11 and U22 are in place:
+//   P = R12 U22  (into the node's strictly lower block when square, else
+//   its depth's scratch);  A12 = -U11 P.
+int merge(float *A, int64_t ld, const MergeNode &nd, float *scratch,
+          const std::vector<size_t> &depth_off, int *status, bool background,
+          cudaStream_t st) {
+  const int64_t off = nd.off, h = nd.h, m = nd.m;
   float *A11 = A + off * ld + off;
   float *A12 = A + off * ld + (off + h);
-  float *A21 = A + (off + h) * ld + off;
   float *A22 = A + (off + h) * ld + (off + h);
-  float *T = fr.scratch + fr.depth_off[depth];
-  int *status = fr.status;
-  cudaStream_t st = fr.stream;
-  int rc;
-  if ((rc = potrf_inv(fr, off + h, m, depth + 1)) != GPTQ_OK) return rc;
-  // T = A12 U22^T   (U22^T is lower: k >= n)
-  GemmArgs g{(int)h, (int)m, (int)m, A12, ld, A22, ld, T, m, 1.f, 0.f, GEMM_KMIN_COL, status};
-  if ((rc = launch_gemm(g, true, st)) != GPTQ_OK) return rc;
-  // A11 -= T T^T  (upper tiles)
-  g = GemmArgs{(int)h, (int)h, (int)m, T, m, T, m, A11, ld, -1.f, 1.f, GEMM_UPPER_C, status};
-  if ((rc = launch_gemm(g, true, st)) != GPTQ_OK) return rc;
-  if (h == m && fr.side) {
-    cudaEvent_t fork = fr.side->ev[fr.next_ev++], join = fr.side->ev[fr.next_ev++];
-    GPTQ_CUDA_TRY(cudaEventRecord(fork, st));
-    GPTQ_CUDA_TRY(cudaStreamWaitEvent(fr.side->s, fork, 0));
-    // P = T U22 into A21   (U22 upper: k <= n)
-    g = GemmArgs{(int)h, (int)m, (int)m, T, m, A22, ld, A21, ld, 1.f, 0.f, GEMM_KMAX_COL, status,
-                 true};
-    if ((rc = launch_gemm(g, false, fr.side->s)) != GPTQ_OK) return rc;
-    GPTQ_CUDA_TRY(cudaEventRecord(join, fr.side->s));
-    if ((rc = potrf_inv(fr, off, h, depth + 1)) != GPTQ_OK) return rc;
-    GPTQ_CUDA_TRY(cudaStreamWaitEvent(st, join, 0));
-    // A12 = -U11 P   (U11 upper: k >= m)
-    g = GemmArgs{(int)h, (int)m, (int)h, A11, ld, A21, ld, A12, ld, -1.f, 0.f, GEMM_KMIN_ROW,
-                 status};
-    return launch_gemm(g, false, st);
+  float *P;
+  int64_t ldp;
+  if (h == m) {
+    P = A + (off + h) * ld + off;
+    ldp = ld;
+  } else {
+    P = scratch + depth_off[nd.depth];
+    ldp = m;
   }
-  // A12 <- T U22
-  g = GemmArgs{(int)h, (int)m, (int)m, T, m, A22, ld, A12, ld, 1.f, 0.f, GEMM_KMAX_COL, status};
+  int rc;
+  // P = R12 U22   (U22 upper: k <= n)
+  GemmArgs g{(int)h, (int)m, (int)m, A12, ld, A22, ld, P, ldp, 1.f, 0.f, GEMM_KMAX_COL, status,
+             background};
   if ((rc = launch_gemm(g, false, st)) != GPTQ_OK) return rc;
-  if ((rc = potrf_inv(fr, off, h, depth + 1)) != GPTQ_OK) return rc;
-  // T = -U11 A12, then A12 <- T
-  g = GemmArgs{(int)h, (int)m, (int)h, A11, ld, A12, ld, T, m, -1.f, 0.f, GEMM_KMIN_ROW, status};
-  if ((rc = launch_gemm(g, false, st)) != GPTQ_OK) return rc;
-  const int64_t pieces = h * (m / 4);
-  const int64_t cap = (int64_t)num_sms() * 8;
-  const int blocks = (int)((pieces + 255) / 256 < cap ? (pieces + 255) / 256 : cap);
-  GPTQ_LAUNCH_PDL(copy_block_kernel, dim3(blocks), dim3(256), 0, st, A12, ld, (const float *)T, m,
-                  (int)h, (int)m, (const int *)status);
-  return GPTQ_OK;
+  // A12 = -U11 P   (U11 upper: k >= m)
+  g = GemmArgs{(int)h, (int)m, (int)h, A11, ld, P, ldp, A12, ld, -1.f, 0.f, GEMM_KMIN_ROW, status,
+               background};
+  return launch_gemm(g, false, st);
 }
 
 }  // namespace
 
+// H_d = R R^T with R upper (the Cholesky taken from the bottom-right corner),
+// then U = R^-1, in place: U in the upper triangle of A.
+//
+// Cholesky, right-looking by 128-column blocks from the last one (block k =
+// columns [c0, c0 + ck)):
+//   leaf:      A_kk -> U_kk = R_kk^-1                       (one CTA)
+//   panel:     R[0:c0, k] = A[0:c0, k] U_kk^T                (k tiles)
+//   next:      A[0:c0, k-1] -= R[0:c0, k] R[c0-128:c0, k]^T  (the next block column)
+//   trailing:  A[0:c0-128, 0:c0-128] -= R[.., k] R[.., k]^T  (upper tiles)
+// Only leaf -> panel -> next is on the critical path; the trailing update of
+// step k runs on a least-priority side stream and must finish before step
+// k-1's "next" (which writes a block column it also writes).
+//
+// Inverse: the diagonal blocks already hold U_kk; each node of the merge tree
+// forms U12 = -U11 R12 U22 once both halves are inverted.  A node's merge
+// reads only R and U in its own columns, which are final as soon as the leaf
+// of its first block has run, and nothing the later Cholesky steps touch
+// (rows above the node), so merges run on a third stream alongside the
+// Cholesky.
 int launch_factor(float *A, int64_t d, float *T1, int *status, cudaStream_t stream,
                   bool use_side) {
-  FactorRun fr{A, d, T1, {}, status, stream, nullptr, 0};
-  size_t off = 0;
-  for (int64_t n = d; (n + kLeaf - 1) / kLeaf > 1;) {
-    int64_t h, m;
-    split(n, &h, &m);
-    fr.depth_off.push_back(off);
-    off += (size_t)h * (size_t)m;
-    n = m;
+  const int64_t ld = d;
+  const int64_t nb = (d + kLeaf - 1) / kLeaf;
+  if (nb <= 1) return launch_leaf(A, ld, (int)d, status, stream);
+  std::vector<size_t> depth_off;
+  {
+    size_t off = 0;
+    for (int64_t n = d; (n + kLeaf - 1) / kLeaf > 1;) {
+      int64_t h, m;
+      split(n, &h, &m);
+      depth_off.push_back(off);
+      off += (size_t)h * (size_t)m;
+      n = m;
+    }
   }
-  if (use_side && !fr.depth_off.empty()) {
-    const int rc = side_stream(d, &fr.side);
+  std::vector<MergeNode> nodes;
+  merge_nodes(0, d, 0, nodes);
+  // Nodes by the block of their first column, children before parents.
+  std::vector<std::vector<MergeNode>> at(nb);
+  for (const MergeNode &nd : nodes) at[nd.off / kLeaf].push_back(nd);
+
+  SideStreams *ss = nullptr;
+  if (use_side) {
+    const int rc = side_streams((size_t)(3 * nb + 2), &ss);
     if (rc != GPTQ_OK) return rc;
   }
-  return potrf_inv(fr, 0, d, 0);
+  size_t nev = 0;
+  auto event = [&]() { return ss->ev[nev++]; };
+  cudaStream_t st = stream;
+  cudaEvent_t trail_done = nullptr;   // trailing update of the step before
+  int rc;
+  if (ss) {
+    // The side streams start after everything already on `stream`.
+    cudaEvent_t start = event();
+    GPTQ_CUDA_TRY(cudaEventRecord(start, st));
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(ss->trail, start, 0));
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(ss->merge, start, 0));
+  }
+  for (int64_t k = nb - 1; k >= 0; --k) {
+    const int64_t c0 = k * kLeaf;
+    const int64_t ck = (d - c0) < kLeaf ? (d - c0) : kLeaf;
+    if ((rc = launch_leaf(A + c0 * ld + c0, ld, (int)ck, status, st)) != GPTQ_OK) return rc;
+    // Merges whose first block is k: their halves are inverted now.
+    if (!at[k].empty()) {
+      cudaStream_t ms = st;
+      if (ss) {
+        cudaEvent_t e = event();
+        GPTQ_CUDA_TRY(cudaEventRecord(e, st));
+        GPTQ_CUDA_TRY(cudaStreamWaitEvent(ss->merge, e, 0));
+        ms = ss->merge;
+      }
+      for (const MergeNode &nd : at[k])
+        if ((rc = merge(A, ld, nd, T1, depth_off, status, ss != nullptr, ms)) != GPTQ_OK)
+          return rc;
+    }
+    if (k == 0) break;
+    float *colk = A + c0;   // block column k, rows 0 .. c0
+    // panel: R[0:c0, k] = A[0:c0, k] U_kk^T, in place (each tile reads only its own rows)
+    GemmArgs g{(int)c0, (int)ck, (int)ck, colk, ld, A + c0 * ld + c0, ld, colk, ld, 1.f, 0.f,
+               GEMM_KMIN_COL, status};
+    if ((rc = launch_gemm(g, true, st)) != GPTQ_OK) return rc;
+    // trailing: A[0:c0-128, 0:c0-128] -= R R^T over the rows above the next block
+    cudaEvent_t this_trail = nullptr;
+    if (k >= 2) {
+      const int64_t mt = c0 - kLeaf;
+      g = GemmArgs{(int)mt, (int)mt, (int)ck, colk, ld, colk, ld, A, ld, -1.f, 1.f, GEMM_UPPER_C,
+                   status, ss != nullptr};
+      if (ss) {
+        cudaEvent_t fork = event();
+        this_trail = event();
+        GPTQ_CUDA_TRY(cudaEventRecord(fork, st));
+        GPTQ_CUDA_TRY(cudaStreamWaitEvent(ss->trail, fork, 0));
+        if ((rc = launch_gemm(g, true, ss->trail)) != GPTQ_OK) return rc;
+        GPTQ_CUDA_TRY(cudaEventRecord(this_trail, ss->trail));
+      } else if ((rc = launch_gemm(g, true, st)) != GPTQ_OK) {
+        return rc;
+      }
+    }
+    // next: A[0:c0, k-1] -= R[0:c0, k] R[c0-128:c0, k]^T, after the previous
+    // step's trailing update (it wrote block column k-1 too)
+    if (trail_done) GPTQ_CUDA_TRY(cudaStreamWaitEvent(st, trail_done, 0));
+    g = GemmArgs{(int)c0, (int)kLeaf, (int)ck, colk, ld, colk + (c0 - kLeaf) * ld, ld,
+                 A + (c0 - kLeaf), ld, -1.f, 1.f, 0, status};
+    if ((rc = launch_gemm(g, true, st)) != GPTQ_OK) return rc;
+    trail_done = this_trail;
+  }
+  if (ss) {
+    // Join: the last merges (the root's) and any trailing update still running.
+    cudaEvent_t e = event();
+    GPTQ_CUDA_TRY(cudaEventRecord(e, ss->merge));
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(st, e, 0));
+    e = event();
+    GPTQ_CUDA_TRY(cudaEventRecord(e, ss->trail));
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(st, e, 0));
+  }
+  return GPTQ_OK;
 }
 
 }  // namespace gptq
