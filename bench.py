@@ -229,6 +229,25 @@ def run_reference(args, wl, rank: int, world: int):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ multi-rank timing
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest per-rank value over the process group (a job takes as long as its
+    slowest rank); ``dist`` is None for a single process."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_ms_per_layer(elapsed_ms: float, steps: int, world: int) -> float:
+    """Whole-job metric: the slowest rank's time over all layers the ranks processed
+    (each rank solves one layer per step)."""
+    return elapsed_ms / (steps * world)
+
+
 # ------------------------------------------------------------------ GPU leg
 
 def run_ours(args, wl, rank: int, world: int, dist):
@@ -311,13 +330,9 @@ def run_ours(args, wl, rank: int, world: int, dist):
     torch.cuda.synchronize(dev)
     launches = g.gptq_launch_count() - launches0
     clocks = sampler.stop()
-    elapsed = t_start.elapsed_time(t_end)
-    if dist is not None:
-        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
     ms_per_step = elapsed / args.steps
-    value = elapsed / (args.steps * world)
+    value = job_ms_per_layer(elapsed, args.steps, world)
 
     # end to end through the host-buffer entry point
     e2e = None
@@ -343,13 +358,10 @@ def run_ours(args, wl, rank: int, world: int, dist):
                                     outputs=host_out, stream=stream)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
         out_bytes = sum(v.numel() * v.element_size() for v in host_out.values()) + 8
-        e2e = {"value": round(e_ms / (args.e2e_steps * world), 3), "unit": "ms per layer",
+        e2e = {"value": round(job_ms_per_layer(e_ms, args.e2e_steps, world), 3),
+               "unit": "ms per layer",
                "h2d_bytes_per_step": int(X.nbytes + W.nbytes), "d2h_bytes_per_step": int(out_bytes)}
 
     if rank != 0:

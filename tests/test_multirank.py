@@ -1,0 +1,69 @@
+"""bench.py's multi-rank path on CPU: two gloo ranks in separate processes.
+
+One process per GPU solves its own layer each step (weak scaling, no collective on the
+data path); the job's time is the slowest rank's, and the metric counts every rank's
+layers.  The GPU-free parts of that contract run here with the gloo backend.
+"""
+
+import os
+import socket
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        slowest = bench.max_over_ranks(10.0 + 5.0 * rank, dist, "cpu")
+        q.put((rank, slowest, bench.job_ms_per_layer(slowest, 3, world)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_report_the_slowest_rank_over_all_layers():
+    mp = pytest.importorskip("torch.multiprocessing")
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # rank 0 ran for 10 ms, rank 1 for 15 ms: both see 15 ms, and the job solved
+    # 3 steps x 2 ranks = 6 layers in it
+    assert results == [(0, 15.0, 2.5), (1, 15.0, 2.5)]
+
+
+def test_single_process_needs_no_group():
+    import bench
+    assert bench.max_over_ranks(7.0, None, "cpu") == 7.0
+    assert bench.job_ms_per_layer(12.0, 4, 1) == 3.0
+
+
+def test_reference_arm_runs_on_rank_zero_only(capsys):
+    import bench
+    from synth import workload
+
+    class Args:
+        steps, warmup, gpus = 1, 0, 2
+
+    bench.run_reference(Args(), workload("tiny_128x256"), rank=1, world=2)
+    assert capsys.readouterr().out == ""
