@@ -200,6 +200,30 @@ def test_each_step_is_the_obs_optimum():
         np.testing.assert_allclose(pre[:, j], (W64[:, F] - corr)[:, 0], rtol=1e-9, atol=1e-12)
 
 
+def test_group_parameters_come_from_the_compensated_weights():
+    # [Tutorial] §分组方案 with §误差补偿: a group's (scale, zero) are the min-max of its
+    # columns as they stand when the sweep reaches the group's first column, i.e. the
+    # OBS optimum given the columns already quantised -- computed here from H_d
+    # directly, with no Cholesky factor.
+    X, W = make_problem(6, 16, 300, seed=14)
+    H = oracle.hessian(X)
+    Hd, _ = oracle.dampen(H, 0.01)
+    g, bits = 4, 3
+    out = oracle.gptq_quantize_layer(W, H, bits=bits, group=g, block=8)
+    What, W64 = out["What"], W.astype(np.float64)
+    for j in range(0, 16, g):
+        Q, F = np.arange(j), np.arange(j, 16)
+        cur = W64[:, F].copy()
+        if j:
+            cur -= np.linalg.solve(Hd[np.ix_(F, F)],
+                                   Hd[np.ix_(F, Q)] @ (What[:, Q] - W64[:, Q]).T).T
+        lo = np.minimum(cur[:, :g].min(axis=1), 0.0)
+        hi = np.maximum(cur[:, :g].max(axis=1), 0.0)
+        s = (hi - lo) / (2 ** bits - 1)
+        np.testing.assert_allclose(out["scales"][:, j // g], s, rtol=1e-9)
+        np.testing.assert_array_equal(out["zeros"][:, j // g], np.rint(-lo / s))
+
+
 def test_single_column_update_matches_paper_form():
     # delta_F = (q - w_q)/[H^-1]_qq * [H^-1]_{F,q} for the first column.
     X, W = make_problem(5, 6, 100, seed=12)
