@@ -8,13 +8,12 @@
 //
 // Route: H_d = R R^T with R upper (a Cholesky taken from the bottom-right
 // corner), then U = R^-1, which is upper and satisfies U^T U = H_d^-1, i.e. U
-// is exactly the upper Cholesky factor of H_d^-1 that GPTQ needs.  Both are
-// computed together by a recursion on 2 x 2 block partitions
-//     [A11 A12; . A22]:  A22 -> U22;  R12 = A12 U22^T;  A11 -= R12 R12^T;
-//                        A11 -> U11;  U12 = -U11 R12 U22
-// whose work is dense GEMMs with triangular operands (tensor cores, 3xTF32,
-// gemm_tc.cu), down to 128 x 128 leaves that one CTA factors and inverts in
-// registers (fp64).
+// is exactly the upper Cholesky factor of H_d^-1 that GPTQ needs.  R comes
+// from a blocked right-looking Cholesky over 128-column blocks whose diagonal
+// blocks one CTA factors and inverts (leaf.cu, fp32); U is assembled from R and
+// those inverted blocks over a binary merge tree, U12 = -U11 R12 U22.  All the
+// remaining work is dense GEMMs with triangular operands on the tensor cores
+// (3xTF32, gemm_tc.cu); see launch_factor for the order and the streams.
 #include <mutex>
 #include <vector>
 

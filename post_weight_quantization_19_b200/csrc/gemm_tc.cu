@@ -3,7 +3,7 @@
 //   C = alpha * A * op(B) + beta * C     (row-major fp32; op(B) = B or B^T)
 //
 // Used by the trailing (lazy-batch) updates of the column sweep and by the
-// block recursion that forms U -- the dense contractions of the layer solve
+// blocked factorisation that forms U -- the dense contractions of the layer solve
 // (GPTQ reading card, 方法适配: the deferred global update is a matrix product).
 //
 // Each fp32 operand x is split as hi = tf32(x) and lo = tf32(x - hi), both

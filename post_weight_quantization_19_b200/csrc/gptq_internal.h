@@ -97,12 +97,13 @@ int launch_damp(float *H, int64_t ld, int d, float damp, bool add_in_place, floa
                 cudaStream_t stream);
 int launch_act_order(const float *H, int64_t ld, int d, int *perm, int *inv, const float *lambda,
                      float *Hp, cudaStream_t stream);
-// Scratch of the factorisation: one h x m product per recursion depth.
+// Scratch of the factorisation: one h x m product per depth of the merge tree.
 size_t factor_scratch_floats(int64_t d);
 // One diagonal block (nb <= 128, nb % 32 == 0) of H_d -> U in place (full block, zeros below).
 int launch_leaf(float *A, int64_t ld, int nb, int *status, cudaStream_t stream);
-// use_side: form the background products on a second stream (created once
-// per device, with its events); false keeps everything on `stream`.
+// use_side: run the trailing updates and the merge products on two side streams
+// (created once per device, with their events); false keeps everything on
+// `stream`.
 int launch_factor(float *A, int64_t d, float *T1, int *status, cudaStream_t stream,
                   bool use_side);
 

@@ -7,7 +7,7 @@
 // come from a Cholesky kernel; the "LLM 量化技术" blog §2.3 item 3.
 //
 // The block lives in shared memory (fp32, like the rest of the solve) and is
-// processed by the same 2 x 2 block recursion as the full matrix,
+// processed by a 2 x 2 block recursion,
 //     A22 -> U22;  T = A12 U22^T;  A11 -= T T^T;  A12 = T U22;
 //     A11 -> U11;  A12 = -U11 A12,
 // with register-tiled shared-memory products run by all LT threads, down to

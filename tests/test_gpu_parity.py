@@ -207,6 +207,34 @@ def test_host_buffer_entry_point_matches_device_path():
     assert loss == dev["loss"]
 
 
+def test_host_entry_point_accumulates_the_hessian_per_uploaded_chunk():
+    # X travels in chunks of max(32768, ceil(n/64)) tokens and H is accumulated as
+    # each chunk lands: bit for bit the H of one gptq_hessian_accumulate per chunk.
+    import post_weight_quantization_19_b200 as g
+    X, W = make_problem(48, 256, 70000, seed=42)
+    r, d = W.shape
+    n = X.shape[0]
+    chunk = max(32768, (n + 63) // 64)
+    Xd = torch.from_numpy(X).cuda()
+    H = torch.zeros((d, d), device="cuda")
+    for t0 in range(0, n, chunk):
+        g.gptq_hessian_accumulate(Xd[t0:t0 + chunk], H)
+    dev = g.gptq_quantize_layer(torch.from_numpy(W).cuda(), H, bits=4, group=64)
+    torch.cuda.synchronize()
+    ws = torch.empty(g.gptq_layer_host_workspace_bytes(r, d, n, 4, 64), dtype=torch.uint8,
+                     device="cuda")
+    out = {"qweight": torch.empty((r, d // 8), dtype=torch.int32).pin_memory(),
+           "scales": torch.empty((r, d // 64), dtype=torch.float32).pin_memory(),
+           "zeros": torch.empty((r, d // 64), dtype=torch.int32).pin_memory()}
+    loss = g.gptq_solve_layer_host(torch.from_numpy(X).pin_memory(),
+                                   torch.from_numpy(W).pin_memory(), bits=4, group=64,
+                                   dev_workspace=ws, outputs=out)
+    np.testing.assert_array_equal(out["qweight"].numpy(), dev["qweight"].cpu().numpy())
+    np.testing.assert_array_equal(out["scales"].numpy(), dev["scales"].cpu().numpy())
+    np.testing.assert_array_equal(out["zeros"].numpy(), dev["zeros"].cpu().numpy())
+    assert loss == dev["loss"]
+
+
 def test_workspace_too_small_is_reported():
     import post_weight_quantization_19_b200 as g
     W = torch.zeros((8, 64), device="cuda")
