@@ -229,6 +229,42 @@ def run_reference(args, wl, rank: int, world: int):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ per-phase rooflines
+
+def phase_rooflines(wl, phases_ms: dict, peaks: dict) -> dict:
+    """Each phase of one layer against the roofline of its algorithmic work.
+
+    hessian: n*d*(d+1) flop vs the sustained fp16 (bf16) tensor peak; factor_U:
+    2 d^3 / 3 flop (Cholesky and triangular inverse) and sweep: r*d*(d-B) flop of
+    the trailing updates that dominate it, both fp32-equivalent against a third of
+    the TF32 peak (three TF32 products per fp32 product; TF32 is half the bf16 rate);
+    damp_perm and finalize_pack: the bytes they must move vs the measured HBM copy
+    rate.  The two latency-chain phases (factor_U, the in-block part of sweep) are
+    not expected to approach their bound.
+    """
+    r, d, n, B = wl.r, wl.d, wl.n, wl.block
+    tc = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    tf32x3 = tc / 2.0 / 3.0
+    G = 1 if wl.group == -1 else d // wl.group
+    work = {
+        "hessian": ("TFLOP/s", float(n) * d * (d + 1) / 1e12, tc),
+        "damp_perm": ("GB/s", 8.0 * d * (d if wl.act_order else 1) / 1e9, hbm),
+        "factor_U": ("TFLOP/s", 2.0 * d ** 3 / 3.0 / 1e12, tf32x3),
+        "sweep": ("TFLOP/s", 2.0 * r * d * max(d - B, 0) / 1e12, tf32x3),
+        "finalize_pack": ("GB/s", (r * d * (4 + 4 + 1 + wl.bits / 8.0) + 8.0 * r * G) / 1e9, hbm),
+    }
+    out = {}
+    for name, (unit, amount, peak) in work.items():
+        ms = phases_ms.get(name)
+        if not ms or ms <= 0:
+            continue
+        achieved = amount / (ms * 1e-3)
+        out[name] = {"achieved": round(achieved, 2), "peak": round(peak, 1), "unit": unit,
+                     "frac": round(achieved / peak, 4)}
+    return out
+
+
 # ------------------------------------------------------------------ multi-rank timing
 
 def max_over_ranks(x: float, dist, device) -> float:
@@ -374,6 +410,9 @@ def run_ours(args, wl, rank: int, world: int, dist):
         peak, peak_src = float(peaks["bf16_tflops_sustained"]), "measured (sustained)"
     else:
         peak, peak_src = 1400.0, "fallback (sustained)"
+    phases_ms = {"hessian": round(phase_h, 4), "damp_perm": round(phases[0], 4),
+                 "factor_U": round(phases[1], 4), "sweep": round(phases[2], 4),
+                 "finalize_pack": round(phases[3], 4)}
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": "ms per layer", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -385,9 +424,8 @@ def run_ours(args, wl, rank: int, world: int, dist):
                      "frac": round(achieved / peak, 4), "traffic": _traffic(wl),
                      "peak_source": peak_src + " bf16 cuBLAS peak; fp16 runs at the same rate",
                      "flops_per_launch": flops, "avg_launch_ms": round(h_avg, 4)},
-        "phases_ms": {"hessian": round(phase_h, 4), "damp_perm": round(phases[0], 4),
-                      "factor_U": round(phases[1], 4), "sweep": round(phases[2], 4),
-                      "finalize_pack": round(phases[3], 4)},
+        "phases_ms": phases_ms,
+        "phase_roofline": phase_rooflines(wl, phases_ms, peaks),
         "loss": loss,
         "gpu_launches": int(launches),
         "clocks": clocks,

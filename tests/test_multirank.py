@@ -67,3 +67,25 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
 
     bench.run_reference(Args(), workload("tiny_128x256"), rank=1, world=2)
     assert capsys.readouterr().out == ""
+
+
+def test_phase_rooflines_from_measured_phase_times():
+    # The per-phase rooflines of the bench line: algorithmic work over the phase
+    # time, against the measured peaks (checked here on the 4096-wide layer).
+    import bench
+    from synth import workload
+    wl = workload("llama7b_q_proj_4096x4096")
+    peaks = {"bf16_tflops_sustained": 1367.3, "hbm_gbs": 6539.5}
+    phases = {"hessian": 3.62, "damp_perm": 0.017, "factor_U": 2.18, "sweep": 1.18,
+              "finalize_pack": 0.05}
+    roof = bench.phase_rooflines(wl, phases, peaks)
+    assert set(roof) == set(phases)
+    h = roof["hessian"]
+    assert h["unit"] == "TFLOP/s" and h["peak"] == 1367.3
+    assert h["achieved"] == pytest.approx(262144 * 4096 * 4097 / 3.62e-3 / 1e12, rel=1e-3)
+    u = roof["factor_U"]
+    assert u["peak"] == pytest.approx(1367.3 / 6, rel=1e-3)
+    assert u["achieved"] == pytest.approx(2 * 4096 ** 3 / 3 / 2.18e-3 / 1e12, rel=1e-3)
+    f = roof["finalize_pack"]
+    assert f["unit"] == "GB/s" and 0 < f["frac"] < 1
+    assert bench.phase_rooflines(wl, {"hessian": 0.0}, peaks) == {}
