@@ -151,6 +151,32 @@ int gptq_pack(const uint8_t *codes, int64_t r, int64_t d, int bits, int32_t *qwe
               gptq_stream_t stream);
 
 /*
+ * gptq_dequant_gemv -- y = x W^^T straight from a packed layer
+ *   ([Card] §计算设置: the quantised layers run through a dequantising
+ *   matrix-vector kernel at inference; [Explainer] §三: int32 packing,
+ *   group_size and desc_act)
+ *
+ *   W^[row, c] = scales[row, gi(c)] * (q[row, c] - zeros[row, gi(c)]), with q the
+ *   bits-bit code of column c unpacked from qweight (the layout gptq_quantize_layer
+ *   and gptq_pack write) and gi(c) = g_idx[c] if g_idx is given, else c / group
+ *   (0 for group = -1).
+ *
+ *   qweight device int32 [r x d*bits/32];  scales device fp32 [r x G];
+ *   zeros   device int32 [r x G], G = 1 (group = -1) or d / group;
+ *   g_idx   device int32 [d] or NULL (entries outside [0, G) are clamped to it);
+ *   x       device fp32 [m x d] row-major, 16-byte aligned;
+ *   y       device fp32 [m x r] row-major, written.
+ *   d % 32 == 0; bits 2, 3, 4 or 8; group -1 or a multiple of 32 dividing d;
+ *   0 <= m <= GPTQ_GEMV_MAX_M.  r == 0 or m == 0: nothing to do.  Invalid
+ *   arguments return GPTQ_ERR_INVALID_ARG before anything is launched.
+ *   Accumulation in fp32.  Asynchronous.
+ */
+#define GPTQ_GEMV_MAX_M 8
+int gptq_dequant_gemv(const int32_t *qweight, const float *scales, const int32_t *zeros,
+                      const int32_t *g_idx, int64_t r, int64_t d, int bits, int group,
+                      const float *x, int64_t m, float *y, gptq_stream_t stream);
+
+/*
  * gptq_quantize_layer_noalloc -- gptq_quantize_layer for callers that cannot
  * allocate device memory.  (The GPTQ pages have no counterpart: this is a
  * deployment convenience of this library, not a step of the method.)

@@ -9,6 +9,7 @@ from .gptq_ref import (  # noqa: F401
     act_order_perm,
     brute_force_min_loss,
     dampen,
+    dequant_gemv,
     dequantize,
     gptq_quantize_layer,
     gptq_sweep,

@@ -338,3 +338,29 @@ def unpack_rows(words: np.ndarray, bits: int, d: int) -> np.ndarray:
             v |= w[:, wi + 1] << np.uint64(32 - off)
         out[:, c] = (v & mask).astype(np.int64)
     return out
+
+
+# ---------------------------------------------------------------------------
+# Using the packed layer: y = W^ x  ([Card] §计算设置 -- the quantised layers
+# are consumed by a dequantising matrix-vector kernel at inference; the
+# packing of [Explainer] §三)
+# ---------------------------------------------------------------------------
+
+def dequant_gemv(qweight: np.ndarray, scales: np.ndarray, zeros: np.ndarray, bits: int,
+                 group: int, x: np.ndarray, g_idx: np.ndarray | None = None) -> np.ndarray:
+    """y [m x r] = x [m x d] @ W^^T with W^[row, c] = s[row, gi(c)] (q[row, c] - z[row, gi(c)]).
+
+    q comes from unpacking ``qweight`` (LSB-first stream per row); gi(c) = g_idx[c]
+    when given (act-order), else c // group (0 for group = -1).  float64 throughout.
+    """
+    x = np.atleast_2d(np.asarray(x, dtype=F64))
+    d = x.shape[1]
+    q = unpack_rows(qweight, bits, d).astype(F64)
+    if g_idx is not None:
+        gi = np.asarray(g_idx, dtype=np.int64)
+    else:
+        gi = np.zeros(d, dtype=np.int64) if group == -1 else np.arange(d) // group
+    s = np.asarray(scales, dtype=F64)[:, gi]
+    z = np.asarray(zeros, dtype=F64)[:, gi]
+    return x @ (s * (q - z)).T
+

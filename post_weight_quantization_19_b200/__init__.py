@@ -14,6 +14,7 @@ from .gptq import (  # noqa: F401
     gptq_last_phase_ms,
     gptq_launch_count,
     gptq_layer_host_workspace_bytes,
+    gptq_dequant_gemv,
     gptq_pack,
     gptq_quantize_layer,
     gptq_quantize_workspace_bytes,

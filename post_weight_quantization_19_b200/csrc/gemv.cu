@@ -1,0 +1,136 @@
+// Dequantising matrix-vector product over a packed layer: y = x W^^T.
+//
+// Sources: the GPTQ reading card ("GPTQ: Accurate Post-Training Quantization
+// for Generative Pre-trained Transformers", 计算设置) -- the quantised layers
+// run through a dequantising matrix-vector kernel at inference, which is
+// bound by reading the packed weights; "一文读懂GPTQ" §三 -- 3/4-bit codes in
+// 32-bit integer arrays, group_size and desc_act (the group index g_idx).
+//
+// W^[row, c] = s[row, gi(c)] (q[row, c] - z[row, gi(c)]), with q the b-bit code
+// of column c in the row's LSB-first stream (the layout gptq_quantize_layer and
+// gptq_pack write) and gi(c) = g_idx[c] when given (act-order), else c / group
+// (0 for group = -1).  One warp per row: lane l takes the 32-code chunks l,
+// l + 32, ... of the row (b consecutive words each), unpacks them with static
+// shifts, and accumulates up to GEMV_MAX_M dot products in fp32; a shuffle
+// reduction ends the row.  Bandwidth bound at small m: r*d*b/8 bytes of codes,
+// 8*r*G bytes of scales and zeros, 4*m*(d + r) bytes of x and y.
+#include "gptq_internal.h"
+
+namespace gptq {
+namespace {
+
+constexpr int GEMV_WARPS = 8;
+constexpr int GEMV_MAX_M = GPTQ_GEMV_MAX_M;
+
+struct GemvArgs {
+  const uint32_t *qweight;
+  const float *scales;
+  const int32_t *zeros;
+  const int32_t *g_idx;   // may be NULL
+  int64_t r;
+  int d, group, G, m;
+  const float *x;         // [m x d], 16-byte aligned rows
+  float *y;               // [m x r]
+};
+
+template <int BITS>
+__global__ void __launch_bounds__(32 * GEMV_WARPS) gemv_kernel(GemvArgs a) {
+  constexpr uint32_t mask = (1u << BITS) - 1u;
+  const int lane = threadIdx.x & 31;
+  const int nchunk = a.d / 32;
+  const int64_t wpr = (int64_t)nchunk * BITS;   // words per row
+  for (int64_t row = (int64_t)blockIdx.x * GEMV_WARPS + (threadIdx.x >> 5); row < a.r;
+       row += (int64_t)gridDim.x * GEMV_WARPS) {
+    float acc[GEMV_MAX_M];
+#pragma unroll
+    for (int i = 0; i < GEMV_MAX_M; ++i) acc[i] = 0.f;
+    const uint32_t *qrow = a.qweight + row * wpr;
+    const float *srow = a.scales + row * a.G;
+    const int32_t *zrow = a.zeros + row * a.G;
+    for (int k = lane; k < nchunk; k += 32) {
+      uint32_t w[BITS];
+#pragma unroll
+      for (int t = 0; t < BITS; ++t) w[t] = __ldg(qrow + (int64_t)k * BITS + t);
+      float s = 0.f, z = 0.f;
+      if (!a.g_idx) {   // groups are multiples of 32 columns: one group per chunk
+        const int gi = a.group > 0 ? (k * 32) / a.group : 0;
+        s = __ldg(srow + gi);
+        z = (float)__ldg(zrow + gi);
+      }
+#pragma unroll
+      for (int j4 = 0; j4 < 32; j4 += 4) {
+        float4 xv[GEMV_MAX_M];
+#pragma unroll
+        for (int i = 0; i < GEMV_MAX_M; ++i)
+          if (i < a.m)
+            xv[i] = __ldg(reinterpret_cast<const float4 *>(a.x + (int64_t)i * a.d + k * 32 + j4));
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int j = j4 + jj;
+          const int pos = j * BITS, wi = pos >> 5, off = pos & 31;
+          uint32_t v = w[wi] >> off;
+          if (off + BITS > 32) v |= w[wi + 1] << (32 - off);
+          const float q = (float)(v & mask);
+          if (a.g_idx) {
+            int gi = __ldg(a.g_idx + k * 32 + j);
+            gi = gi < 0 ? 0 : (gi >= a.G ? a.G - 1 : gi);   // out-of-range entries clamp
+            s = __ldg(srow + gi);
+            z = (float)__ldg(zrow + gi);
+          }
+          const float wv = s * (q - z);
+#pragma unroll
+          for (int i = 0; i < GEMV_MAX_M; ++i) {
+            if (i < a.m) {
+              const float xj = jj == 0 ? xv[i].x : jj == 1 ? xv[i].y : jj == 2 ? xv[i].z : xv[i].w;
+              acc[i] = fmaf(wv, xj, acc[i]);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < GEMV_MAX_M; ++i) {
+      float v = acc[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0 && i < a.m) a.y[(int64_t)i * a.r + row] = v;
+    }
+  }
+}
+
+}  // namespace
+}  // namespace gptq
+
+using namespace gptq;
+
+extern "C" int gptq_dequant_gemv(const int32_t *qweight, const float *scales,
+                                 const int32_t *zeros, const int32_t *g_idx, int64_t r,
+                                 int64_t d, int bits, int group, const float *x, int64_t m,
+                                 float *y, gptq_stream_t stream) {
+  if (r < 0 || r > (int64_t)INT32_MAX) return GPTQ_ERR_INVALID_ARG;
+  if (d <= 0 || d % 32 != 0 || d > 65536) return GPTQ_ERR_INVALID_ARG;
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_INVALID_ARG;
+  if (group != -1 && (group < 32 || group % 32 != 0 || d % group != 0))
+    return GPTQ_ERR_INVALID_ARG;
+  if (m < 0 || m > GEMV_MAX_M) return GPTQ_ERR_INVALID_ARG;
+  if (r == 0 || m == 0) return GPTQ_OK;
+  if (!qweight || !scales || !zeros || !x || !y) return GPTQ_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(qweight) % 4 ||
+      reinterpret_cast<uintptr_t>(scales) % 4 || reinterpret_cast<uintptr_t>(zeros) % 4 ||
+      reinterpret_cast<uintptr_t>(y) % 4 || (g_idx && reinterpret_cast<uintptr_t>(g_idx) % 4))
+    return GPTQ_ERR_INVALID_ARG;
+  GemvArgs a{reinterpret_cast<const uint32_t *>(qweight), scales, zeros, g_idx, r, (int)d,
+             group, group < 0 ? 1 : (int)(d / group), (int)m, x, y};
+  const int64_t want = (r + GEMV_WARPS - 1) / GEMV_WARPS;
+  const int64_t cap = (int64_t)num_sms() * 16;
+  const dim3 grid((unsigned)(want < cap ? want : cap));
+  cudaStream_t st = (cudaStream_t)stream;
+  switch (bits) {
+    case 2: gemv_kernel<2><<<grid, 32 * GEMV_WARPS, 0, st>>>(a); break;
+    case 3: gemv_kernel<3><<<grid, 32 * GEMV_WARPS, 0, st>>>(a); break;
+    case 4: gemv_kernel<4><<<grid, 32 * GEMV_WARPS, 0, st>>>(a); break;
+    default: gemv_kernel<8><<<grid, 32 * GEMV_WARPS, 0, st>>>(a); break;
+  }
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}

@@ -110,6 +110,25 @@ def gptq_quantize_layer(W: torch.Tensor, H: torch.Tensor, *, bits: int, group: i
     return res
 
 
+def gptq_dequant_gemv(qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                      x: torch.Tensor, bits: int, group: int, g_idx: torch.Tensor | None = None,
+                      y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y [m, r] = x [m, d] W^^T from the packed layer (x fp32, m <= GPTQ_GEMV_MAX_M)."""
+    lib = _abi.load()
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    m, d = x.shape
+    r = qweight.shape[0]
+    if y is None:
+        y = torch.empty((m, r), dtype=torch.float32, device=x.device)
+    _check(lib.gptq_dequant_gemv(
+        _ptr(qweight, torch.int32, "qweight"), _ptr(scales, torch.float32, "scales"),
+        _ptr(zeros, torch.int32, "zeros"), _ptr(g_idx, torch.int32, "g_idx"), r, d, bits, group,
+        _ptr(x, torch.float32, "x"), m, _ptr(y, torch.float32, "y"), _stream(stream)),
+        "gptq_dequant_gemv")
+    return y
+
+
 def gptq_pack(codes: torch.Tensor, bits: int, qweight: torch.Tensor | None = None,
               stream=None) -> torch.Tensor:
     lib = _abi.load()

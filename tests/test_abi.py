@@ -86,6 +86,15 @@ def test_validation_returns_before_cuda(lib):
     assert h(p, 0, 128, 128, p, None) == 0           # no tokens: nothing to do
     assert lib.gptq_pack(p, 4, 100, 4, p, None) == 1
     assert lib.gptq_pack(p, 4, 128, 6, p, None) == 1
+    gv = lib.gptq_dequant_gemv
+    assert gv(p, p, p, None, 8, 100, 4, -1, p, 1, p, None) == 1     # d % 32
+    assert gv(p, p, p, None, 8, 128, 5, -1, p, 1, p, None) == 1     # bits
+    assert gv(p, p, p, None, 8, 128, 4, 48, p, 1, p, None) == 1     # group not a multiple of 32
+    assert gv(p, p, p, None, 8, 128, 4, -1, p, 9, p, None) == 1     # m > GPTQ_GEMV_MAX_M
+    assert gv(p, p, p, None, 8, 128, 4, -1, ctypes.c_void_p(4100), 1, p, None) == 1  # x alignment
+    assert gv(p, p, p, None, 8, 128, 4, -1, None, 1, p, None) == 1  # missing x
+    assert gv(p, p, p, None, 0, 128, 4, -1, p, 1, p, None) == 0     # no rows: nothing to do
+    assert gv(p, p, p, None, 8, 128, 4, -1, p, 0, p, None) == 0     # no vectors
 
 
 def test_no_kernels_launched_on_cpu(lib):

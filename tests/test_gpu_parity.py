@@ -278,3 +278,61 @@ def test_graph_replay_matches_direct_launch():
     for loss, q in results[1:]:
         assert loss == results[0][0]
         np.testing.assert_array_equal(q, results[0][1])
+
+
+# ------------------------------------------------------------------ using the packed layer
+
+@pytest.mark.parametrize("case", [(4, 128, False, 1), (3, -1, False, 3), (4, 32, True, 2),
+                                  (2, 64, False, 8), (8, 128, True, 1), (3, 128, False, 5)],
+                         ids=lambda c: "b{}_g{}_a{}_m{}".format(*(int(v) for v in c)))
+def test_dequant_gemv_matches_oracle(case):
+    # y = x W^^T from the GPU's own packed output, against the float64 oracle on the
+    # same words, scales, zeros and g_idx.  fp32 accumulation over d terms.
+    import post_weight_quantization_19_b200 as g
+    bits, group, act, m = case
+    X, W = make_problem(200, 512, 3000, seed=50 + bits)
+    got = gpu_layer(X, W, bits=bits, group=group, act_order=act)
+    x = np.random.default_rng(m).standard_normal((m, 512)).astype(np.float32)
+    y = g.gptq_dequant_gemv(torch.from_numpy(got["qweight"]).cuda(),
+                            torch.from_numpy(got["scales"]).cuda(),
+                            torch.from_numpy(got["zeros"]).cuda(), torch.from_numpy(x).cuda(),
+                            bits, group,
+                            g_idx=torch.from_numpy(got["g_idx"]).cuda() if act else None)
+    torch.cuda.synchronize()
+    ref = oracle.dequant_gemv(got["qweight"], got["scales"], got["zeros"], bits, group, x,
+                              g_idx=got["g_idx"] if act else None)
+    err = np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max()
+    assert err <= 1e-5, err
+    # and it is the product with the dequantised weights the layer reported
+    np.testing.assert_allclose(ref, x.astype(np.float64) @ got["W_hat"].astype(np.float64).T,
+                               rtol=1e-6, atol=1e-6 * np.abs(ref).max())
+
+
+def test_dequant_gemv_full_layer_bandwidth():
+    # The 4096 x 4096 4-bit group-128 layer at batch 1: parity on all rows and the
+    # achieved read bandwidth (packed codes + scales + zeros + x) printed.
+    import post_weight_quantization_19_b200 as g
+    r = d = 4096
+    rng = np.random.default_rng(7)
+    codes = rng.integers(0, 16, size=(r, d), dtype=np.uint8)
+    qweight = oracle.pack_rows(codes, 4)
+    scales = (rng.random((r, d // 128)) * 0.01 + 1e-3).astype(np.float32)
+    zeros = rng.integers(0, 16, size=(r, d // 128)).astype(np.int32)
+    x = rng.standard_normal((1, d)).astype(np.float32)
+    qd, sd, zd, xd = (torch.from_numpy(a).cuda() for a in (qweight, scales, zeros, x))
+    y = g.gptq_dequant_gemv(qd, sd, zd, xd, 4, 128)
+    ref = oracle.dequant_gemv(qweight, scales, zeros, 4, 128, x)
+    torch.cuda.synchronize()
+    assert np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max() <= 1e-5
+    for _ in range(3):
+        g.gptq_dequant_gemv(qd, sd, zd, xd, 4, 128, y=y)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(50):
+        g.gptq_dequant_gemv(qd, sd, zd, xd, 4, 128, y=y)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / 50
+    nbytes = qweight.nbytes + scales.nbytes + zeros.nbytes + x.nbytes + r * 4
+    print(f"dequant_gemv 4096x4096 4-bit g128 m=1: {ms * 1e3:.2f} us, {nbytes / ms / 1e6:.0f} GB/s")
+

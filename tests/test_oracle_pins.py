@@ -356,3 +356,21 @@ def test_pack_matches_big_integer_stream(bits):
 def test_pack_rejects_partial_words():
     with pytest.raises(ValueError):
         oracle.pack_rows(np.zeros((1, 5), dtype=np.int64), 3)
+
+
+# ---------------------------------------------------------------- using the packed layer
+
+@pytest.mark.parametrize("bits,group,act", [(4, 32, False), (3, -1, False), (4, 32, True),
+                                            (2, 64, False), (8, 32, True)])
+def test_dequant_gemv_equals_the_dequantised_layer(bits, group, act):
+    # y = W^ x computed from the packed words, the scales, the zeros and g_idx alone
+    # equals the product with the layer's dequantised weights -- which pins the
+    # unpacking, the group lookup (including act-order's g_idx) and the product.
+    X, W = make_problem(9, 128, 600, seed=30 + bits)
+    out = oracle.gptq_quantize_layer(W, oracle.hessian(X), bits=bits, group=group,
+                                     act_order=act)
+    qw = oracle.pack_rows(out["codes"], bits)
+    x = np.random.default_rng(bits).standard_normal((3, 128))
+    y = oracle.dequant_gemv(qw, out["scales"], out["zeros"], bits, group, x,
+                            g_idx=out["g_idx"] if act else None)
+    np.testing.assert_allclose(y, x @ out["What"].T, rtol=1e-12, atol=1e-12)
