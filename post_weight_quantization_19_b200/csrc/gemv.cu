@@ -10,9 +10,9 @@
 // of column c in the row's LSB-first stream (the layout gptq_quantize_layer and
 // gptq_pack write) and gi(c) = g_idx[c] when given (act-order), else c / group
 // (0 for group = -1).  One warp per row: lane l takes the 32-code chunks l,
-// l + 32, ... of the row (b consecutive words each), unpacks them with static
-// shifts, and accumulates up to GEMV_MAX_M dot products in fp32; a shuffle
-// reduction ends the row.  Bandwidth bound at small m: r*d*b/8 bytes of codes,
+// l + 32, ... of the row (b consecutive words each, fetched 4 chunks ahead),
+// unpacks them with static shifts, and accumulates the m dot products in fp32
+// (m rounded up to 1, 2, 4 or 8 accumulators); a shuffle reduction ends the row.  Bandwidth bound at small m: r*d*b/8 bytes of codes,
 // 8*r*G bytes of scales and zeros, 4*m*(d + r) bytes of x and y.
 #include "gptq_internal.h"
 
@@ -33,69 +33,99 @@ struct GemvArgs {
   float *y;               // [m x r]
 };
 
-template <int BITS>
-__global__ void __launch_bounds__(32 * GEMV_WARPS) gemv_kernel(GemvArgs a) {
+// One 32-code chunk: unpack with static shifts and accumulate MB dot products.
+template <int BITS, int MB>
+__device__ __forceinline__ void gemv_chunk(const uint32_t (&w)[BITS], const GemvArgs &a,
+                                           const float *srow, const int32_t *zrow, int k,
+                                           float (&acc)[MB]) {
   constexpr uint32_t mask = (1u << BITS) - 1u;
+  float s = 0.f, z = 0.f;
+  if (!a.g_idx) {   // groups are multiples of 32 columns: one group per chunk
+    const int gi = a.group > 0 ? (k * 32) / a.group : 0;
+    s = __ldg(srow + gi);
+    z = (float)__ldg(zrow + gi);
+  }
+#pragma unroll
+  for (int j4 = 0; j4 < 32; j4 += 4) {
+    float4 xv[MB];
+#pragma unroll
+    for (int i = 0; i < MB; ++i)
+      xv[i] = i < a.m ? __ldg(reinterpret_cast<const float4 *>(a.x + (int64_t)i * a.d + k * 32 + j4))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = j4 + jj;
+      const int pos = j * BITS, wi = pos >> 5, off = pos & 31;
+      uint32_t v = w[wi] >> off;
+      if (off + BITS > 32) v |= w[wi + 1] << (32 - off);
+      const float q = (float)(v & mask);
+      if (a.g_idx) {
+        int gi = __ldg(a.g_idx + k * 32 + j);
+        gi = gi < 0 ? 0 : (gi >= a.G ? a.G - 1 : gi);   // out-of-range entries clamp
+        s = __ldg(srow + gi);
+        z = (float)__ldg(zrow + gi);
+      }
+      const float wv = s * (q - z);
+#pragma unroll
+      for (int i = 0; i < MB; ++i) {
+        const float xj = jj == 0 ? xv[i].x : jj == 1 ? xv[i].y : jj == 2 ? xv[i].z : xv[i].w;
+        acc[i] = fmaf(wv, xj, acc[i]);
+      }
+    }
+  }
+}
+
+// MB accumulators (the batch rounded up to 1, 2, 4 or 8); a lane fetches the
+// words of up to PF of its chunks before any arithmetic, so each row waits on
+// memory about once.
+template <int BITS, int MB>
+__global__ void __launch_bounds__(32 * GEMV_WARPS) gemv_kernel(GemvArgs a) {
+  constexpr int PF = 4;
   const int lane = threadIdx.x & 31;
   const int nchunk = a.d / 32;
   const int64_t wpr = (int64_t)nchunk * BITS;   // words per row
   for (int64_t row = (int64_t)blockIdx.x * GEMV_WARPS + (threadIdx.x >> 5); row < a.r;
        row += (int64_t)gridDim.x * GEMV_WARPS) {
-    float acc[GEMV_MAX_M];
+    float acc[MB];
 #pragma unroll
-    for (int i = 0; i < GEMV_MAX_M; ++i) acc[i] = 0.f;
+    for (int i = 0; i < MB; ++i) acc[i] = 0.f;
     const uint32_t *qrow = a.qweight + row * wpr;
     const float *srow = a.scales + row * a.G;
     const int32_t *zrow = a.zeros + row * a.G;
-    for (int k = lane; k < nchunk; k += 32) {
-      uint32_t w[BITS];
+    for (int k0 = lane; k0 < nchunk; k0 += 32 * PF) {
+      uint32_t w[PF][BITS];
 #pragma unroll
-      for (int t = 0; t < BITS; ++t) w[t] = __ldg(qrow + (int64_t)k * BITS + t);
-      float s = 0.f, z = 0.f;
-      if (!a.g_idx) {   // groups are multiples of 32 columns: one group per chunk
-        const int gi = a.group > 0 ? (k * 32) / a.group : 0;
-        s = __ldg(srow + gi);
-        z = (float)__ldg(zrow + gi);
+      for (int p = 0; p < PF; ++p) {
+        const int k = k0 + 32 * p;
+#pragma unroll
+        for (int t = 0; t < BITS; ++t) w[p][t] = k < nchunk ? __ldg(qrow + (int64_t)k * BITS + t) : 0u;
       }
 #pragma unroll
-      for (int j4 = 0; j4 < 32; j4 += 4) {
-        float4 xv[GEMV_MAX_M];
-#pragma unroll
-        for (int i = 0; i < GEMV_MAX_M; ++i)
-          if (i < a.m)
-            xv[i] = __ldg(reinterpret_cast<const float4 *>(a.x + (int64_t)i * a.d + k * 32 + j4));
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int j = j4 + jj;
-          const int pos = j * BITS, wi = pos >> 5, off = pos & 31;
-          uint32_t v = w[wi] >> off;
-          if (off + BITS > 32) v |= w[wi + 1] << (32 - off);
-          const float q = (float)(v & mask);
-          if (a.g_idx) {
-            int gi = __ldg(a.g_idx + k * 32 + j);
-            gi = gi < 0 ? 0 : (gi >= a.G ? a.G - 1 : gi);   // out-of-range entries clamp
-            s = __ldg(srow + gi);
-            z = (float)__ldg(zrow + gi);
-          }
-          const float wv = s * (q - z);
-#pragma unroll
-          for (int i = 0; i < GEMV_MAX_M; ++i) {
-            if (i < a.m) {
-              const float xj = jj == 0 ? xv[i].x : jj == 1 ? xv[i].y : jj == 2 ? xv[i].z : xv[i].w;
-              acc[i] = fmaf(wv, xj, acc[i]);
-            }
-          }
-        }
-      }
+      for (int p = 0; p < PF; ++p)
+        if (k0 + 32 * p < nchunk) gemv_chunk<BITS, MB>(w[p], a, srow, zrow, k0 + 32 * p, acc);
     }
 #pragma unroll
-    for (int i = 0; i < GEMV_MAX_M; ++i) {
+    for (int i = 0; i < MB; ++i) {
       float v = acc[i];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       if (lane == 0 && i < a.m) a.y[(int64_t)i * a.r + row] = v;
     }
   }
+}
+
+template <int BITS>
+int gemv_launch(const GemvArgs &a, dim3 grid, cudaStream_t st) {
+  if (a.m <= 1)
+    gemv_kernel<BITS, 1><<<grid, 32 * GEMV_WARPS, 0, st>>>(a);
+  else if (a.m <= 2)
+    gemv_kernel<BITS, 2><<<grid, 32 * GEMV_WARPS, 0, st>>>(a);
+  else if (a.m <= 4)
+    gemv_kernel<BITS, 4><<<grid, 32 * GEMV_WARPS, 0, st>>>(a);
+  else
+    gemv_kernel<BITS, GEMV_MAX_M><<<grid, 32 * GEMV_WARPS, 0, st>>>(a);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
 }
 
 }  // namespace
@@ -126,11 +156,9 @@ extern "C" int gptq_dequant_gemv(const int32_t *qweight, const float *scales,
   const dim3 grid((unsigned)(want < cap ? want : cap));
   cudaStream_t st = (cudaStream_t)stream;
   switch (bits) {
-    case 2: gemv_kernel<2><<<grid, 32 * GEMV_WARPS, 0, st>>>(a); break;
-    case 3: gemv_kernel<3><<<grid, 32 * GEMV_WARPS, 0, st>>>(a); break;
-    case 4: gemv_kernel<4><<<grid, 32 * GEMV_WARPS, 0, st>>>(a); break;
-    default: gemv_kernel<8><<<grid, 32 * GEMV_WARPS, 0, st>>>(a); break;
+    case 2: return gemv_launch<2>(a, grid, st);
+    case 3: return gemv_launch<3>(a, grid, st);
+    case 4: return gemv_launch<4>(a, grid, st);
+    default: return gemv_launch<8>(a, grid, st);
   }
-  GPTQ_LAUNCH_CHECK();
-  return GPTQ_OK;
 }

@@ -324,15 +324,26 @@ def test_dequant_gemv_full_layer_bandwidth():
     ref = oracle.dequant_gemv(qweight, scales, zeros, 4, 128, x)
     torch.cuda.synchronize()
     assert np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max() <= 1e-5
-    for _ in range(3):
-        g.gptq_dequant_gemv(qd, sd, zd, xd, 4, 128, y=y)
+    # 50 launches replayed as one CUDA graph: the kernel's time, not the binding's
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            g.gptq_dequant_gemv(qd, sd, zd, xd, 4, 128, y=y)
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(50):
+            g.gptq_dequant_gemv(qd, sd, zd, xd, 4, 128, y=y)
+    graph.replay()
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(50):
-        g.gptq_dequant_gemv(qd, sd, zd, xd, 4, 128, y=y)
+    graph.replay()
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / 50
+    assert np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max() <= 1e-5
     nbytes = qweight.nbytes + scales.nbytes + zeros.nbytes + x.nbytes + r * 4
     print(f"dequant_gemv 4096x4096 4-bit g128 m=1: {ms * 1e3:.2f} us, {nbytes / ms / 1e6:.0f} GB/s")
 
