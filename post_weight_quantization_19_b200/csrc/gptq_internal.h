@@ -51,6 +51,21 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return launch_pdl_prio(false, kernel, grid, block, smem, stream, std::forward<Args>(args)...);
 }
 
+// The dynamic shared-memory limit of a kernel, raised once per device (the
+// attribute belongs to the kernel in the current device's context).
+template <typename K>
+int ensure_smem_attr(K kernel, size_t bytes, bool (&done)[64]) {
+  int dev = 0;
+  GPTQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return GPTQ_ERR_INVALID_ARG;
+  if (!done[dev]) {
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bytes));
+    done[dev] = true;
+  }
+  return GPTQ_OK;
+}
+
 // launch_pdl with the library's launch accounting and error reporting; a
 // template kernel name goes in parentheses.
 #define GPTQ_LAUNCH_PDL(kernel, grid, block, smem, stream, ...)                          \

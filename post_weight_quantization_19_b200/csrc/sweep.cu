@@ -432,12 +432,8 @@ template <int CW, int L>
 static int sweep_launch(const SweepArgs &a, cudaStream_t stream) {
   constexpr int B = CW * L;
   const size_t smem = (size_t)B * (CW + 4) * L * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(sweep_block_kernel<CW, L>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    attr = true;
-  }
+  static bool attr[64] = {};
+  if (const int rc = ensure_smem_attr(sweep_block_kernel<CW, L>, smem, attr)) return rc;
   // Every row gets its lanes in one wave when the SMs can hold them (two CTAs
   // per SM: about 180 registers per thread).
   const int rows_per_cta = SWEEP_WARPS * (32 / L);
