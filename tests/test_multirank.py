@@ -89,3 +89,29 @@ def test_phase_rooflines_from_measured_phase_times():
     f = roof["finalize_pack"]
     assert f["unit"] == "GB/s" and 0 < f["frac"] < 1
     assert bench.phase_rooflines(wl, {"hessian": 0.0}, peaks) == {}
+
+
+def test_reference_arm_prints_one_complete_json_line():
+    # `bench.py --impl reference` times the float64 oracle on the host cores and
+    # prints the same JSON line as the GPU arm plus "impl": "reference".
+    import json
+    import subprocess
+    out = subprocess.run(
+        [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+         "tiny_128x256", "--steps", "1", "--warmup", "0"],
+        capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    lines = [ln for ln in out.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["higher_is_better"] is False
+    assert line["value"] > 0 and line["unit"] == "ms per layer"
+    assert line["config"]["workload"] == "tiny_128x256"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["h2d_bytes_per_step"] == 0
