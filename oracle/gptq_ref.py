@@ -41,6 +41,13 @@ design notes):
   row.
 * Act-order: stable argsort of -diag(H) (ties keep the lower index); groups
   are formed over permuted positions and g_idx maps original columns to them.
+* Symmetric variant ([Survey] §1.2, whose formula is garbled): zero point 0,
+  s = max|x| / (2^(b-1) - 1) (s = 1 for an all-zero row), signed codes
+  clamped to [-2^(b-1), 2^(b-1) - 1] and stored as unsigned codes with
+  z = 2^(b-1).
+* Static groups (not on the pages; the plainest reading of parameters fixed
+  before the sweep): every group's parameters come from the original W over
+  the layer's own column groups, so under act-order g_idx[c] = c // group.
 * Packing: per row, codes form an LSB-first bit stream along the input
   dimension, 32 bits per int32 word; 3-bit codes straddle words.
 
@@ -121,9 +128,20 @@ def inverse_upper_cholesky(Hd: np.ndarray) -> np.ndarray:
 # Asymmetric min-max quantiser  ([Tutorial] §分组方案; [Survey] §1.2)
 # ---------------------------------------------------------------------------
 
-def quant_params(x: np.ndarray, bits: int) -> tuple[np.ndarray, np.ndarray]:
-    """Per-row (scale, zero) of x [rows x cols] (float64 in, float64 out)."""
+def quant_params(x: np.ndarray, bits: int, sym: bool = False) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row (scale, zero) of x [rows x cols] (float64 in, float64 out).
+
+    ``sym``: the symmetric quantiser of [Survey] §1.2 (zero point 0, scale
+    max|x| / (2^(b-1) - 1), signed codes clamped to [-2^(b-1), 2^(b-1) - 1]).
+    The signed code is stored as the unsigned b-bit code code + 2^(b-1), so the
+    same quantize/dequantize pair serves it with z = 2^(b-1).
+    """
     x = np.asarray(x, dtype=F64)
+    if sym:
+        amax = np.abs(x).max(axis=1)
+        half = 1 << (bits - 1)
+        s = np.where(amax == 0.0, 1.0, amax / (half - 1))
+        return s, np.full_like(s, float(half))
     maxq = (1 << bits) - 1
     xmin = np.minimum(x.min(axis=1), 0.0)
     xmax = np.maximum(x.max(axis=1), 0.0)
@@ -144,7 +162,8 @@ def dequantize(q: np.ndarray, s: np.ndarray, z: np.ndarray) -> np.ndarray:
     return s * (q - z)
 
 
-def rtn(W: np.ndarray, bits: int, group: int) -> tuple[np.ndarray, np.ndarray]:
+def rtn(W: np.ndarray, bits: int, group: int,
+        sym: bool = False) -> tuple[np.ndarray, np.ndarray]:
     """Round-to-nearest baseline: same quantiser, parameters from W, no compensation.
 
     Returns (codes int64 [r x d], W^ float64 [r x d]).
@@ -156,7 +175,7 @@ def rtn(W: np.ndarray, bits: int, group: int) -> tuple[np.ndarray, np.ndarray]:
     What = np.zeros((r, d), dtype=F64)
     for c0 in range(0, d, g):
         blk = W[:, c0:c0 + g]
-        s, z = quant_params(blk, bits)
+        s, z = quant_params(blk, bits, sym)
         q = quantize(blk, s[:, None], z[:, None], bits)
         codes[:, c0:c0 + g] = q.astype(np.int64)
         What[:, c0:c0 + g] = dequantize(q, s[:, None], z[:, None])
@@ -179,7 +198,8 @@ def _check_groups(d: int, group: int, block: int) -> None:
         raise ValueError("lazy batches need block % group == 0 or group % block == 0")
 
 
-def gptq_sweep(W: np.ndarray, U: np.ndarray, bits: int, group: int, block: int):
+def gptq_sweep(W: np.ndarray, U: np.ndarray, bits: int, group: int, block: int,
+               sym: bool = False, fixed=None):
     """Quantise W [r x d] column by column in fixed order.
 
     At column j: q = quantize(w_j), e_j = (w_j - w^_j)/U_jj, and the columns
@@ -188,26 +208,37 @@ def gptq_sweep(W: np.ndarray, U: np.ndarray, bits: int, group: int, block: int):
     deferred to the block's end as one product E_blk @ U[blk, end:] (the lazy
     batch).  ``block >= d`` is the plain unblocked loop.
 
+    ``fixed`` = (scales [r x G], zeros [r x G], col_group [d]) gives static
+    group parameters chosen before the sweep: column j uses group col_group[j]
+    and no parameters are taken from the compensated weights.
+
     Returns (codes int64, scales, zeros (float64 holding integers), W^ float64,
     E float64 [r x d] with E[:, j] = e_j).
     """
     W = np.array(W, dtype=F64, copy=True)
     U = np.asarray(U, dtype=F64)
     r, d = W.shape
-    _check_groups(d, group, block)
     G = 1 if group == -1 else d // group
     codes = np.zeros((r, d), dtype=np.int64)
-    scales = np.zeros((r, G), dtype=F64)
-    zeros = np.zeros((r, G), dtype=F64)
     E = np.zeros((r, d), dtype=F64)
-    if group == -1:
-        s, z = quant_params(W, bits)
-        scales[:, 0], zeros[:, 0] = s, z
+    if fixed is not None:
+        scales = np.asarray(fixed[0], dtype=F64)
+        zeros = np.asarray(fixed[1], dtype=F64)
+        col_group = np.asarray(fixed[2], dtype=np.int64)
+    else:
+        _check_groups(d, group, block)
+        scales = np.zeros((r, G), dtype=F64)
+        zeros = np.zeros((r, G), dtype=F64)
+        if group == -1:
+            s, z = quant_params(W, bits, sym)
+            scales[:, 0], zeros[:, 0] = s, z
     for b0 in range(0, d, block):
         b1 = min(d, b0 + block)
         for j in range(b0, b1):
-            if group != -1 and j % group == 0:
-                s, z = quant_params(W[:, j:j + group], bits)
+            if fixed is not None:
+                s, z = scales[:, col_group[j]], zeros[:, col_group[j]]
+            elif group != -1 and j % group == 0:
+                s, z = quant_params(W[:, j:j + group], bits, sym)
                 scales[:, j // group], zeros[:, j // group] = s, z
             w = W[:, j]
             q = quantize(w, s, z, bits)
@@ -246,11 +277,19 @@ def layer_loss_direct(W: np.ndarray, What: np.ndarray, X: np.ndarray) -> float:
 
 def gptq_quantize_layer(W: np.ndarray, H: np.ndarray, *, bits: int, group: int,
                         block: int = 128, damp: float = 0.01,
-                        act_order: bool = False, rows: np.ndarray | None = None) -> dict:
+                        act_order: bool = False, rows: np.ndarray | None = None,
+                        sym: bool = False, static_groups: bool = False) -> dict:
     """Damp, order, factor, sweep, score and unpermute one layer.
 
     ``rows`` restricts the sweep to a subset of output rows (rows are
     independent once U is fixed), for checks at full layer width.
+
+    ``sym`` selects the symmetric quantiser (see ``quant_params``).
+    ``static_groups`` takes every group's parameters from the original W over
+    the layer's own column groups (columns c with c // group = k) before the
+    sweep, instead of from the compensated W when the sweep reaches a group;
+    under act-order the groups then stay contiguous in the original column
+    order, so g_idx[c] = c // group.  With group = -1 both rules coincide.
     """
     W = np.asarray(W, dtype=F64)
     H = np.asarray(H, dtype=F64)
@@ -261,10 +300,21 @@ def gptq_quantize_layer(W: np.ndarray, H: np.ndarray, *, bits: int, group: int,
     perm = act_order_perm(H) if act_order else np.arange(d)
     inv = np.argsort(perm)
     U = inverse_upper_cholesky(Hd[np.ix_(perm, perm)])
-    codes_p, scales, zeros, What_p, E = gptq_sweep(W[:, perm], U, bits, group, block)
+    fixed = None
+    g_idx = (inv // group) if group != -1 else np.zeros(d, dtype=np.int64)
+    if static_groups and group != -1:
+        G = d // group
+        fs = np.zeros((r, G), dtype=F64)
+        fz = np.zeros((r, G), dtype=F64)
+        for k in range(G):
+            fs[:, k], fz[:, k] = quant_params(W[:, k * group:(k + 1) * group], bits, sym)
+        # sweep position j holds original column perm[j]
+        fixed = (fs, fz, perm // group)
+        g_idx = np.arange(d) // group
+    codes_p, scales, zeros, What_p, E = gptq_sweep(W[:, perm], U, bits, group, block,
+                                                   sym=sym, fixed=fixed)
     codes = codes_p[:, inv]
     What = What_p[:, inv]
-    g_idx = (inv // group) if group != -1 else np.zeros(d, dtype=np.int64)
     return {
         "codes": codes,
         "scales": scales,
@@ -284,7 +334,7 @@ def gptq_quantize_layer(W: np.ndarray, H: np.ndarray, *, bits: int, group: int,
 # Brute force for tiny rows (the grid is fixed by the row's own min/max)
 # ---------------------------------------------------------------------------
 
-def brute_force_min_loss(w: np.ndarray, H: np.ndarray, bits: int) -> float:
+def brute_force_min_loss(w: np.ndarray, H: np.ndarray, bits: int, sym: bool = False) -> float:
     """min over every code vector of 1/2 (w - w^) H (w - w^)^T for one row.
 
     The row's (s, z) come from its original values (group = -1), as in the
@@ -292,7 +342,7 @@ def brute_force_min_loss(w: np.ndarray, H: np.ndarray, bits: int) -> float:
     """
     w = np.asarray(w, dtype=F64).reshape(1, -1)
     d = w.shape[1]
-    s, z = quant_params(w, bits)
+    s, z = quant_params(w, bits, sym)
     levels = np.arange(1 << bits, dtype=F64)
     cand = np.array(list(itertools.product(levels, repeat=d)), dtype=F64)
     D = w - dequantize(cand, s[0], z[0])

@@ -50,8 +50,19 @@ MUTANTS = [
     ("deferred update dropped", "            W[:, b1:] -= E[:, b0:b1] @ U[b0:b1, b1:]\n",
      "            pass\n"),
     ("group parameters from the original weights",
-     "                s, z = quant_params(W[:, j:j + group], bits)\n",
-     "                s, z = quant_params(W0[:, j:j + group], bits)\n"),
+     "                s, z = quant_params(W[:, j:j + group], bits, sym)\n",
+     "                s, z = quant_params(W0[:, j:j + group], bits, sym)\n"),
+    ("symmetric scale over 2^b - 1", "amax / (half - 1))", "amax / (2 * half - 1))"),
+    ("symmetric zero point stored as 0", "return s, np.full_like(s, float(half))",
+     "return s, np.zeros_like(s)"),
+    ("symmetric range from the signed maximum", "amax = np.abs(x).max(axis=1)",
+     "amax = x.max(axis=1)"),
+    ("static groups ignored", "    if static_groups and group != -1:\n", "    if False:\n"),
+    ("static groups indexed by sweep position", "fixed = (fs, fz, perm // group)",
+     "fixed = (fs, fz, np.arange(d) // group)"),
+    ("static parameters from the permuted weights",
+     "quant_params(W[:, k * group:(k + 1) * group], bits, sym)",
+     "quant_params(W[:, perm][:, k * group:(k + 1) * group], bits, sym)"),
     ("bit stream most-significant first", "        v = codes[:, c].astype(np.uint64) << np.uint64(off)\n",
      "        v = codes[:, c].astype(np.uint64) << np.uint64(32 - bits - off if off + bits <= 32 else off)\n"),
 ]

@@ -107,9 +107,9 @@ def test_inverse_upper_cholesky_diagonal_and_residual():
 
 # -------------------------------------------------------------- quantiser ---
 
-def _golden_quantizer():
+def _golden_quantizer(fname="quantizer_cases.txt"):
     cases = []
-    with open(os.path.join(GOLDEN, "quantizer_cases.txt")) as f:
+    with open(os.path.join(GOLDEN, fname)) as f:
         for line in f:
             line = line.strip()
             if not line or line.startswith("#"):
@@ -149,15 +149,19 @@ def test_quantizer_error_bound():
 
 # ------------------------------------------------------------ column sweep ---
 
+@pytest.mark.parametrize("static", [False, True])
+@pytest.mark.parametrize("sym", [False, True])
 @pytest.mark.parametrize("group", [-1, 32])
 @pytest.mark.parametrize("bits", [3, 4])
-def test_identity_hessian_reduces_to_rtn(bits, group):
+def test_identity_hessian_reduces_to_rtn(bits, group, sym, static):
     # With H proportional to I the factor U is diagonal: no column compensates
-    # another, so GPTQ is round-to-nearest exactly (for any damping).
+    # another, so GPTQ is round-to-nearest exactly (for any damping), with either
+    # quantiser and either group rule.
     _, W = make_problem(16, 128, 1, seed=8)
     for scale in (1.0, 37.5):
-        out = oracle.gptq_quantize_layer(W, scale * np.eye(128), bits=bits, group=group)
-        codes, What = oracle.rtn(W, bits, group)
+        out = oracle.gptq_quantize_layer(W, scale * np.eye(128), bits=bits, group=group,
+                                         sym=sym, static_groups=static)
+        codes, What = oracle.rtn(W, bits, group, sym=sym)
         np.testing.assert_array_equal(out["codes"], codes)
         np.testing.assert_allclose(out["What"], What, rtol=0, atol=0)
 
@@ -314,6 +318,108 @@ def test_brute_force_bounds_tiny_rows():
         r_total += rl
     assert wins >= 0.90 * len(seeds)
     assert g_total < r_total
+
+
+# ------------------------------------------------------- quantiser variants ---
+
+@pytest.mark.parametrize("case", _golden_quantizer("sym_quantizer_cases.txt"))
+def test_sym_quantizer_golden(case):
+    bits, x, s_exp, z_exp, q_exp, wq_exp = case
+    s, z = oracle.quant_params(x[None, :], bits, sym=True)
+    assert s[0] == s_exp and z[0] == z_exp
+    q = oracle.quantize(x, s[0], z[0], bits)
+    np.testing.assert_array_equal(q, q_exp)
+    np.testing.assert_array_equal(oracle.dequantize(q, s[0], z[0]), wq_exp)
+
+
+def test_sym_codes_clamp_to_the_signed_range():
+    # [Survey] §1.2: signed codes clamp to [-2^(b-1), 2^(b-1) - 1].  At 4 bits with
+    # s = 0.25, -2.125 and 2.125 are -8.5 and 8.5 steps; ties go to even, giving -8
+    # (stored 0, the one code a group's own values never reach) and 8, which
+    # clamps to 7 (stored 15).
+    q = oracle.quantize(np.array([-2.125, 2.125]), 0.25, 8.0, 4)
+    np.testing.assert_array_equal(q, [0, 15])
+    np.testing.assert_array_equal(oracle.dequantize(q, 0.25, 8.0), [-2.0, 1.75])
+
+
+def test_sym_grid_is_odd_and_never_clips_its_own_group():
+    # Zero point 0 makes the grid symmetric about 0: -x lands on minus x's value
+    # (rint is odd).  Every |x| <= max|x| = s (2^(b-1) - 1), so no value of the
+    # group is clipped and every error is at most s/2; the absolute maximum is
+    # itself a grid point.
+    rng = _rng(21)
+    rows = np.arange(40)
+    for bits in (2, 3, 4, 8):
+        x = rng.standard_normal((40, 64))
+        s, z = oracle.quant_params(x, bits, sym=True)
+        s_neg, _ = oracle.quant_params(-x, bits, sym=True)
+        np.testing.assert_array_equal(s_neg, s)
+        s2, z2 = s[:, None], z[:, None]
+        wq = oracle.dequantize(oracle.quantize(x, s2, z2, bits), s2, z2)
+        wq_neg = oracle.dequantize(oracle.quantize(-x, s2, z2, bits), s2, z2)
+        np.testing.assert_array_equal(wq_neg, -wq)
+        assert np.all(np.abs(wq - x) <= s2 * (0.5 + 1e-12))
+        i = np.argmax(np.abs(x), axis=1)
+        np.testing.assert_allclose(np.abs(wq[rows, i]), np.abs(x[rows, i]), rtol=1e-15)
+
+
+@pytest.mark.parametrize("act", [False, True])
+def test_static_group_parameters_ignore_the_compensation(act):
+    # Static groups fix every group's (scale, zero) from the original W over the
+    # layer's own column groups before the sweep: the parameters of the
+    # identity-Hessian run (round-to-nearest, nothing compensated) whatever H is.
+    # Under act-order the groups stay contiguous in the original columns, and
+    # every output column lies on its own group's grid.
+    X, W = make_problem(12, 128, 900, seed=22)
+    H = oracle.hessian(X)
+    ref = oracle.gptq_quantize_layer(W, np.eye(128), bits=4, group=32)
+    out = oracle.gptq_quantize_layer(W, H, bits=4, group=32, act_order=act,
+                                     static_groups=True)
+    np.testing.assert_array_equal(out["scales"], ref["scales"])
+    np.testing.assert_array_equal(out["zeros"], ref["zeros"])
+    np.testing.assert_array_equal(out["g_idx"], np.arange(128) // 32)
+    s = np.repeat(out["scales"], 32, axis=1)
+    z = np.repeat(out["zeros"], 32, axis=1)
+    np.testing.assert_array_equal(out["What"], s * (out["codes"] - z))
+    # the default rule reads the compensated weights, so it differs here
+    lazy = oracle.gptq_quantize_layer(W, H, bits=4, group=32, act_order=act)
+    assert not np.array_equal(lazy["scales"], out["scales"])
+
+
+def test_variants_keep_the_obs_steps():
+    # The quantiser variants change only the grid: before each column is rounded,
+    # the remaining columns still sit at the OBS optimum given the quantised ones
+    # (as in the default pin above), here with the symmetric quantiser, static
+    # groups and act-order together, in the permuted order.
+    X, W = make_problem(6, 12, 200, seed=23)
+    H = oracle.hessian(X)
+    Hd, _ = oracle.dampen(H, 0.01)
+    out = oracle.gptq_quantize_layer(W, H, bits=3, group=4, block=8, act_order=True,
+                                     sym=True, static_groups=True)
+    p = out["perm"]
+    U, E = out["U"], out["E"]
+    What, W64, Hp = out["What"][:, p], W.astype(np.float64)[:, p], Hd[np.ix_(p, p)]
+    pre = What + E * np.diag(U)[None, :]
+    for j in range(1, 12):
+        Q, F = np.arange(j), np.arange(j, 12)
+        corr = np.linalg.solve(Hp[np.ix_(F, F)], Hp[np.ix_(F, Q)] @ (What[:, Q] - W64[:, Q]).T).T
+        np.testing.assert_allclose(pre[:, j], (W64[:, F] - corr)[:, 0], rtol=1e-9, atol=1e-12)
+    assert np.all(out["zeros"] == 4)
+
+
+def test_sym_brute_force_bounds_tiny_rows():
+    # The symmetric grid is fixed by each row's own max|w| (group = -1), so GPTQ's
+    # damped objective can never go below the exhaustive minimum over that grid.
+    for seed in range(200):
+        rng = _rng(20_000 + seed)
+        X = (rng.standard_normal((16, 6)) * rng.lognormal(0, 1, 6)).astype(np.float16)
+        W = rng.standard_normal((2, 6)) * 0.02
+        H = oracle.hessian(X)
+        Hd, _ = oracle.dampen(H, 0.01)
+        out = oracle.gptq_quantize_layer(W, H, bits=2, group=-1, sym=True)
+        for i in range(2):
+            D = W[i] - out["What"][i]
+            assert 0.5 * D @ Hd @ D >= oracle.brute_force_min_loss(W[i], Hd, 2, sym=True) * (1 - 1e-9)
 
 
 # ------------------------------------------------------------------ pack ---
