@@ -21,6 +21,7 @@ from .gptq_ref import (  # noqa: F401
     pack_rows,
     quant_params,
     quantize,
+    quantize_chain,
     rtn,
     unpack_rows,
 )

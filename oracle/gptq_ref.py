@@ -414,3 +414,36 @@ def dequant_gemv(qweight: np.ndarray, scales: np.ndarray, zeros: np.ndarray, bit
     z = np.asarray(zeros, dtype=F64)[:, gi]
     return x @ (s * (q - z)).T
 
+
+
+# ---------------------------------------------------------------------------
+# Sequential layers  ([Card] §计算设置: quantise one block, then run the
+# quantised block to produce the next block's calibration inputs; [Concept]
+# §3 技術原理: at inference the codes are dequantised to FP16 and multiplied in
+# floating point)
+# ---------------------------------------------------------------------------
+
+def quantize_chain(X0: np.ndarray, Ws: list, *, bits: int, group: int, block: int = 128,
+                   damp: float = 0.01, act_order: bool = False, sym: bool = False,
+                   static_groups: bool = False) -> list[dict]:
+    """Quantise a chain of linear layers in order, each on its true inputs.
+
+    Layer k (W_k [r_k x d_k], d_{k+1} = r_k) is solved with H_k = hessian(X_k);
+    the next inputs are the quantised layer's outputs X_{k+1} = fp16(X_k
+    fp16(W^_k)^T), accumulated in float64 over the fp16 values and rounded once
+    to fp16 (an output beyond the fp16 range is an error).  Each entry is
+    ``gptq_quantize_layer``'s result plus ``inputs`` = X_k (fp16).
+    """
+    X = np.asarray(X0, dtype=np.float16)
+    outs = []
+    for W in Ws:
+        out = gptq_quantize_layer(W, hessian(X), bits=bits, group=group, block=block,
+                                  damp=damp, act_order=act_order, sym=sym,
+                                  static_groups=static_groups)
+        out["inputs"] = X
+        outs.append(out)
+        Wh16 = out["What"].astype(np.float16).astype(F64)
+        X = (X.astype(F64) @ Wh16.T).astype(np.float16)
+        if not np.all(np.isfinite(X)):
+            raise ValueError("layer outputs overflow fp16")
+    return outs

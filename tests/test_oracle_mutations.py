@@ -63,6 +63,14 @@ MUTANTS = [
     ("static parameters from the permuted weights",
      "quant_params(W[:, k * group:(k + 1) * group], bits, sym)",
      "quant_params(W[:, perm][:, k * group:(k + 1) * group], bits, sym)"),
+    ("chain inputs not propagated", "        X = (X.astype(F64) @ Wh16.T).astype(np.float16)\n",
+     "        pass\n"),
+    ("chain run on the original weights", "        Wh16 = out[\"What\"].astype(np.float16).astype(F64)\n",
+     "        Wh16 = np.asarray(W, dtype=F64).astype(np.float16).astype(F64)\n"),
+    ("chain outputs kept in float64", "        X = (X.astype(F64) @ Wh16.T).astype(np.float16)\n",
+     "        X = X.astype(F64) @ Wh16.T\n"),
+    ("chain weights not rounded to fp16", "        Wh16 = out[\"What\"].astype(np.float16).astype(F64)\n",
+     "        Wh16 = out[\"What\"]\n"),
     ("bit stream most-significant first", "        v = codes[:, c].astype(np.uint64) << np.uint64(off)\n",
      "        v = codes[:, c].astype(np.uint64) << np.uint64(32 - bits - off if off + bits <= 32 else off)\n"),
 ]

@@ -422,6 +422,68 @@ def test_sym_brute_force_bounds_tiny_rows():
             assert 0.5 * D @ Hd @ D >= oracle.brute_force_min_loss(W[i], Hd, 2, sym=True) * (1 - 1e-9)
 
 
+# ------------------------------------------------------- sequential layers ---
+
+def test_chain_of_one_layer_is_the_layer():
+    X, W = make_problem(24, 64, 500, seed=24)
+    out = oracle.quantize_chain(X, [W], bits=4, group=32)
+    ref = oracle.gptq_quantize_layer(W, oracle.hessian(X), bits=4, group=32)
+    assert len(out) == 1
+    np.testing.assert_array_equal(out[0]["codes"], ref["codes"])
+    np.testing.assert_array_equal(out[0]["inputs"], X)
+    assert out[0]["loss"] == ref["loss"]
+
+
+def _on_grid_weights(rng, r, d, bits):
+    # W = s (q - z) with s a power of two and every row holding the codes 0 and
+    # 2^b - 1: the row's min-max gives back exactly this (s, z), every column
+    # rounds to itself (e_j = 0), and the values are exact in fp16.
+    maxq = (1 << bits) - 1
+    q = rng.integers(0, maxq + 1, size=(r, d))
+    q[:, 0], q[:, 1] = 0, maxq
+    z = rng.integers(0, maxq + 1, size=(r, 1))
+    return (2.0 ** -6) * (q - z), q
+
+
+def test_on_grid_chain_is_the_plain_forward():
+    # [Card] §计算设置: each layer is calibrated on what the quantised layers
+    # before it output.  Weights already on their own grid quantise to themselves,
+    # so every loss is 0 and the inputs follow the unquantised fp16 forward pass,
+    # written here as the recurrence X_{k+1} = fp16(X_k W_k^T).
+    rng = _rng(25)
+    X0, _ = make_problem(1, 32, 300, seed=25)
+    shapes = [(48, 32), (16, 48), (40, 16)]
+    Ws, Qs = zip(*[_on_grid_weights(rng, r, d, 4) for r, d in shapes])
+    out = oracle.quantize_chain(X0, list(Ws), bits=4, group=-1)
+    X = X0
+    for k, (W, Q) in enumerate(zip(Ws, Qs)):
+        np.testing.assert_array_equal(out[k]["inputs"], X)
+        assert out[k]["inputs"].dtype == np.float16
+        np.testing.assert_array_equal(out[k]["What"], W)
+        np.testing.assert_array_equal(out[k]["codes"], Q)
+        assert out[k]["loss"] == 0.0
+        X = (X.astype(np.float64) @ W.T).astype(np.float16)
+
+
+def test_chain_after_an_rtn_layer_sees_the_quantised_outputs():
+    # Orthogonal calibration tokens (X_0 = c [I; I]) make H_0 proportional to I,
+    # so layer 0 is round-to-nearest exactly (pinned above); the next layer's
+    # inputs are then the fp16 outputs of the dequantised RTN weights, and the
+    # next loss is measured directly on those inputs.
+    d0, r0, r1 = 32, 48, 16
+    c = 0.75
+    X0 = np.vstack([c * np.eye(d0), c * np.eye(d0)]).astype(np.float16)
+    _, W0 = make_problem(r0, d0, 1, seed=26)
+    _, W1 = make_problem(r1, r0, 1, seed=27)
+    out = oracle.quantize_chain(X0, [W0, W1], bits=3, group=16)
+    _, What0 = oracle.rtn(W0, 3, 16)
+    np.testing.assert_array_equal(out[0]["What"], What0)
+    X1 = (X0.astype(np.float64) @ What0.astype(np.float16).astype(np.float64).T).astype(np.float16)
+    np.testing.assert_array_equal(out[1]["inputs"], X1)
+    assert out[1]["loss"] == pytest.approx(oracle.layer_loss_direct(W1, out[1]["What"], X1),
+                                           rel=1e-10)
+
+
 # ------------------------------------------------------------------ pack ---
 
 def _golden_pack():
