@@ -21,3 +21,4 @@ from .gptq import (  # noqa: F401
     gptq_set_phase_timing,
     gptq_solve_layer_host,
 )
+from .sharded import row_shard, shard_range, solve_layer_sharded, token_shard  # noqa: F401

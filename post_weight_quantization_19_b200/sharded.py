@@ -1,0 +1,94 @@
+"""One layer solved across the ranks of a process group (one process per GPU).
+
+Token-sharded Hessian: H is a sum over calibration tokens ("GPTQ：一键量化大模型
+压缩", §二阶信息), so rank i accumulates H_i = 2 X_i^T X_i over its own tokens with
+``gptq_hessian_accumulate`` and one all-reduce (sum) leaves H = 2 X^T X on every
+rank.  Row-sharded solve: every row of W is quantised in the same column order
+with the same inverse-Hessian factor (GPTQ reading card, §方法适配), so once H is
+known the rows are independent problems; rank i solves the rows
+``row_shard(r, i, N)`` with ``gptq_quantize_layer`` on its own copy of H (the
+factor is recomputed on each rank instead of broadcast: the library's entry
+point factors and sweeps in one call).  The packed rows, scales and zeros are
+then all-gathered, so every rank returns the whole layer, and the per-rank
+losses (sums over rows) are all-reduced.
+
+The exchange is two collectives per layer (d^2 fp32 words for H, the packed
+layer for the gather), issued through ``torch.distributed`` (NCCL on GPUs).
+"""
+
+from __future__ import annotations
+
+import torch
+
+from .gptq import gptq_hessian_accumulate, gptq_quantize_layer
+
+
+def shard_range(count: int, rank: int, world: int) -> tuple[int, int]:
+    """Contiguous slice [a, b) of ``count`` items for ``rank`` of ``world``.
+
+    Every rank but the last few gets ceil(count / world) items; ranks past the
+    end get an empty slice.
+    """
+    if world < 1 or not 0 <= rank < world or count < 0:
+        raise ValueError("need 0 <= rank < world and count >= 0")
+    per = -(-count // world)
+    a = min(count, rank * per)
+    return a, min(count, a + per)
+
+
+def token_shard(X: torch.Tensor, rank: int, world: int) -> torch.Tensor:
+    """This rank's calibration tokens (rows of X), as a contiguous view."""
+    a, b = shard_range(X.shape[0], rank, world)
+    return X[a:b]
+
+
+def row_shard(r: int, rank: int, world: int) -> tuple[int, int]:
+    """The output rows of W that ``rank`` solves."""
+    return shard_range(r, rank, world)
+
+
+def _gather_rows(local: torch.Tensor, r: int, world: int, dist, group) -> torch.Tensor:
+    # all_gather needs equal shapes: pad each rank's rows to ceil(r / world)
+    per = -(-r // world)
+    buf = local.new_zeros((per,) + tuple(local.shape[1:]))
+    buf[:local.shape[0]] = local
+    parts = [torch.empty_like(buf) for _ in range(world)]
+    dist.all_gather(parts, buf, group=group)
+    return torch.cat(parts)[:r]
+
+
+def solve_layer_sharded(X_local: torch.Tensor, W: torch.Tensor, *, bits: int, group: int,
+                        block: int = 128, damp: float = 0.01, act_order: bool = False,
+                        process_group=None) -> dict:
+    """GPTQ solve of one layer W [r, d] spread over the ranks of ``process_group``.
+
+    ``X_local`` holds this rank's calibration tokens (fp16 [n_i, d]); every rank
+    passes the whole W (fp32).  Every rank must call this with the same W,
+    shapes and options.  Returns the whole layer on every rank: ``qweight``,
+    ``scales``, ``zeros``, ``g_idx`` (act-order only) and ``loss``.
+    """
+    import torch.distributed as dist
+
+    world = dist.get_world_size(process_group)
+    rank = dist.get_rank(process_group)
+    r, d = W.shape
+    if r < world:
+        raise ValueError("need at least one row of W per rank")
+    if X_local.shape[1] != d:
+        raise ValueError("X_local must have d columns")
+    H = torch.zeros((d, d), dtype=torch.float32, device=W.device)
+    if X_local.shape[0] > 0:
+        gptq_hessian_accumulate(X_local, H)
+    dist.all_reduce(H, group=process_group)
+    a, b = row_shard(r, rank, world)
+    g_idx = torch.empty(d, dtype=torch.int32, device=W.device) if act_order else None
+    res = gptq_quantize_layer(W[a:b].contiguous(), H, bits=bits, group=group, block=block,
+                              damp=damp, act_order=act_order, g_idx=g_idx)
+    loss = torch.tensor([res["loss"]], dtype=torch.float64, device=W.device)
+    dist.all_reduce(loss, group=process_group)
+    out = {key: _gather_rows(res[key], r, world, dist, process_group)
+           for key in ("qweight", "scales", "zeros")}
+    out["loss"] = float(loss.item())
+    if act_order:
+        out["g_idx"] = res["g_idx"]
+    return out

@@ -115,3 +115,94 @@ def test_reference_arm_prints_one_complete_json_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["h2d_bytes_per_step"] == 0
+
+
+# ------------------------------------------------- one layer over two ranks ---
+
+def test_shard_ranges_cover_every_item_once():
+    from post_weight_quantization_19_b200.sharded import shard_range
+    for count in (0, 1, 5, 11, 64, 4097):
+        for world in (1, 2, 3, 8):
+            spans = [shard_range(count, k, world) for k in range(world)]
+            covered = [i for a, b in spans for i in range(a, b)]
+            assert covered == list(range(count))
+            assert max(b - a for a, b in spans) == -(-count // world)
+    with pytest.raises(ValueError):
+        shard_range(4, 2, 2)
+
+
+def _integer_layer():
+    # Small integer activations: every partial Hessian and their all-reduced sum
+    # are exact integers in fp32, so the sharded H equals the single-process H
+    # bit for bit and so must every code.
+    import numpy as np
+    import torch
+    rng = np.random.default_rng(5)
+    X = rng.integers(-8, 9, size=(130, 64)).astype(np.float16)
+    W = (0.02 * rng.standard_normal((11, 64))).astype(np.float32)
+    return torch.from_numpy(X), torch.from_numpy(W)
+
+
+def _sharded_worker(rank, world, port, q, act_order):
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from post_weight_quantization_19_b200 import sharded
+
+    # The two GPU entry points, played on the CPU by the oracle (same arguments
+    # and outputs as the binding's, H exact in fp32).
+    def hessian(X, H):
+        H += torch.from_numpy(oracle.hessian(X.numpy())).to(H.dtype)
+
+    def quantize_layer(W, H, *, bits, group, block, damp, act_order, g_idx=None):
+        o = oracle.gptq_quantize_layer(W.numpy(), H.double().numpy(), bits=bits, group=group,
+                                       block=block, damp=damp, act_order=act_order)
+        if g_idx is not None:
+            g_idx.copy_(torch.from_numpy(o["g_idx"]))
+        return {"qweight": torch.from_numpy(oracle.pack_rows(o["codes"], bits)),
+                "scales": torch.from_numpy(o["scales"]).float(),
+                "zeros": torch.from_numpy(o["zeros"]).int(), "loss": o["loss"],
+                "g_idx": g_idx}
+
+    sharded.gptq_hessian_accumulate = hessian
+    sharded.gptq_quantize_layer = quantize_layer
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        X, W = _integer_layer()
+        res = sharded.solve_layer_sharded(sharded.token_shard(X, rank, world), W, bits=4,
+                                          group=16, act_order=act_order)
+        q.put((rank, {k: v.numpy() if torch.is_tensor(v) else v for k, v in res.items()}))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("act_order", [False, True])
+def test_two_ranks_solve_one_layer_like_one_process(act_order):
+    import numpy as np
+
+    import oracle
+    mp = pytest.importorskip("torch.multiprocessing")
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sharded_worker, args=(r, 2, port, q, act_order))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    results = dict(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    X, W = _integer_layer()
+    ref = oracle.gptq_quantize_layer(W.numpy(), oracle.hessian(X.numpy()), bits=4, group=16,
+                                     act_order=act_order)
+    for rank in (0, 1):
+        got = results[rank]
+        np.testing.assert_array_equal(got["qweight"], oracle.pack_rows(ref["codes"], 4))
+        np.testing.assert_array_equal(got["scales"], ref["scales"].astype(np.float32))
+        np.testing.assert_array_equal(got["zeros"], ref["zeros"])
+        assert got["loss"] == pytest.approx(ref["loss"], rel=1e-12)
+        if act_order:
+            np.testing.assert_array_equal(got["g_idx"], ref["g_idx"])
