@@ -33,6 +33,10 @@ constexpr int kSuperblock = 1024;  // columns per global (deferred) trailing upd
 
 bool valid_bits(int b) { return b == 2 || b == 3 || b == 4 || b == 8; }
 
+bool valid_options(int options) {
+  return (options & ~(GPTQ_ACT_ORDER | GPTQ_SYMMETRIC | GPTQ_STATIC_GROUPS)) == 0;
+}
+
 bool valid_layer(int64_t r, int64_t d, int bits, int group, int block) {
   if (r < 0 || r > (int64_t)INT32_MAX / 2) return false;
   if (d <= 0 || d % 32 != 0 || d > 65536) return false;
@@ -60,7 +64,7 @@ struct Layout {
   size_t Wk, ErrS, codes_p, perm, inv, Hp, T1, loss_rows, dsq_rows, out, lambda, status, total;
 };
 
-Layout layout(int64_t r, int64_t d, int group, int block, int act_order) {
+Layout layout(int64_t r, int64_t d, int group, int block, int options) {
   Layout L{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -74,7 +78,7 @@ Layout layout(int64_t r, int64_t d, int group, int block, int act_order) {
   L.codes_p = take((size_t)r * d);
   L.perm = take((size_t)d * 4);
   L.inv = take((size_t)d * 4);
-  L.Hp = take(act_order ? (size_t)d * d * 4 : 0);
+  L.Hp = take((options & GPTQ_ACT_ORDER) ? (size_t)d * d * 4 : 0);
   L.T1 = take(factor_scratch_floats(d) * 4);
   L.loss_rows = take((size_t)r * 8);
   L.dsq_rows = take((size_t)r * 8);
@@ -106,14 +110,14 @@ struct GraphKey {
   int64_t r, d;
   int bits, group, block;
   float damp;
-  int act_order;
+  int options;
   int device = -1;
   bool operator==(const GraphKey &o) const {
     return W == o.W && H == o.H && W_hat == o.W_hat && qweight == o.qweight &&
            scales == o.scales && zeros == o.zeros && g_idx == o.g_idx && codes == o.codes &&
            ws == o.ws && ws_bytes == o.ws_bytes && stream == o.stream && r == o.r &&
            d == o.d && bits == o.bits && group == o.group && block == o.block &&
-           memcmp(&damp, &o.damp, sizeof(float)) == 0 && act_order == o.act_order &&
+           memcmp(&damp, &o.damp, sizeof(float)) == 0 && options == o.options &&
            device == o.device;
   }
 };
@@ -235,20 +239,24 @@ extern "C" int gptq_check_device_status(gptq_stream_t stream) {
 }
 
 extern "C" size_t gptq_quantize_workspace_bytes(int64_t r, int64_t d, int bits, int group,
-                                                int block, int act_order) {
-  if (!valid_layer(r, d, bits, group, block)) return 0;
-  return layout(r, d, group, block, act_order).total;
+                                                int block, int options) {
+  if (!valid_layer(r, d, bits, group, block) || !valid_options(options)) return 0;
+  return layout(r, d, group, block, options).total;
 }
 
 namespace gptq {
 
 int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int group, int block,
-                   float damp, int act_order, float *W_hat, int32_t *qweight, float *scales,
+                   float damp, int options, float *W_hat, int32_t *qweight, float *scales,
                    int32_t *zeros, int32_t *g_idx, uint8_t *codes, double *loss, void *workspace,
                    size_t workspace_bytes, gptq_stream_t stream, bool plain) {
   if (!valid_layer(r, d, bits, group, block)) return GPTQ_ERR_INVALID_ARG;
   if (!(damp >= 0.f) || damp > 1e30f) return GPTQ_ERR_INVALID_ARG;
-  if (act_order != 0 && act_order != 1) return GPTQ_ERR_INVALID_ARG;
+  if (!valid_options(options)) return GPTQ_ERR_INVALID_ARG;
+  const bool act_order = (options & GPTQ_ACT_ORDER) != 0;
+  const int sym = (options & GPTQ_SYMMETRIC) ? 1 : 0;
+  // with one group per row both rules take the parameters from the original row
+  const int static_groups = (options & GPTQ_STATIC_GROUPS) && group > 0 ? 1 : 0;
   if (r == 0) {
     if (loss) *loss = 0.0;
     return GPTQ_OK;
@@ -261,7 +269,7 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
       reinterpret_cast<uintptr_t>(zeros) % 4 || (g_idx && reinterpret_cast<uintptr_t>(g_idx) % 16) ||
       (codes && reinterpret_cast<uintptr_t>(codes) % 4))
     return GPTQ_ERR_INVALID_ARG;
-  const Layout L = layout(r, d, group, block, act_order);
+  const Layout L = layout(r, d, group, block, options);
   if (workspace_bytes < L.total) return GPTQ_ERR_NO_MEMORY;
 
   cudaStream_t st = (cudaStream_t)stream;
@@ -307,7 +315,9 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
     // predecessor, so the kernel just before each of them must not write U:
     // the copy of W separates the factorisation from the first block.
     GPTQ_TRY(launch_gather_w(W, ri, di, act_order ? perm : nullptr, Wk, status, st));
-    if (group < 0) GPTQ_TRY(launch_row_params(Wk, ri, di, bits, scales, zeros, status, st));
+    if (group < 0) GPTQ_TRY(launch_row_params(Wk, ri, di, di, bits, sym, scales, zeros, status, st));
+    if (static_groups)
+      GPTQ_TRY(launch_row_params(W, ri, di, group, bits, sym, scales, zeros, status, st));
     for (int s0 = 0; s0 < di; s0 += S) {
       const int sEnd = s0 + S < di ? s0 + S : di;
       for (int j0 = s0; j0 < sEnd; j0 += block) {
@@ -325,8 +335,9 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
         a.scales = scales;
         a.zeros = zeros;
         a.G = G;
+        a.flags = (sym ? SWEEP_SYM : 0) | (static_groups ? SWEEP_STATIC : 0);
         a.codes = codes_p;
-        a.ldc = d;
+        a.perm = static_groups && act_order ? perm : nullptr;
         a.err = ErrS + (j0 - s0);
         a.lde = S;
         a.loss_rows = loss_rows;
@@ -358,6 +369,7 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
     f.d = di;
     f.bits = bits;
     f.group = group;
+    f.static_groups = static_groups;
     f.W_hat = W_hat;
     f.codes = codes;
     f.qweight = qweight;
@@ -376,7 +388,7 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
   // first call of a configuration runs directly, the second is captured, later
   // ones replay.  Streams that cannot be captured run directly.
   const GraphKey key{W, H, W_hat, qweight, scales, zeros, g_idx, codes, workspace,
-                     workspace_bytes, st, r, d, bits, group, block, damp, act_order};
+                     workspace_bytes, st, r, d, bits, group, block, damp, options};
   int rc = GPTQ_OK;
   if (g_timing || plain) {
     rc = enqueue();
@@ -400,11 +412,11 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
 }  // namespace gptq
 
 extern "C" int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits,
-                                   int group, int block, float damp, int act_order, float *W_hat,
+                                   int group, int block, float damp, int options, float *W_hat,
                                    int32_t *qweight, float *scales, int32_t *zeros,
                                    int32_t *g_idx, uint8_t *codes, double *loss, void *workspace,
                                    size_t workspace_bytes, gptq_stream_t stream) {
-  return gptq::quantize_layer(W, r, d, H, bits, group, block, damp, act_order, W_hat, qweight,
+  return gptq::quantize_layer(W, r, d, H, bits, group, block, damp, options, W_hat, qweight,
                               scales, zeros, g_idx, codes, loss, workspace, workspace_bytes,
                               stream, false);
 }
@@ -447,7 +459,7 @@ int64_t x_chunk_tokens(int64_t n) {
 }
 
 HostLayout host_layout(int64_t r, int64_t d, int64_t n, int bits, int group, int block,
-                       int act_order) {
+                       int options) {
   HostLayout L{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -463,7 +475,7 @@ HostLayout host_layout(int64_t r, int64_t d, int64_t n, int bits, int group, int
   L.sc = take((size_t)r * G * 4);
   L.zr = take((size_t)r * G * 4);
   L.gi = take((size_t)d * 4);
-  L.qws = take(layout(r, d, group, block, act_order).total);
+  L.qws = take(layout(r, d, group, block, options).total);
   L.total = off;
   return L;
 }
@@ -471,18 +483,21 @@ HostLayout host_layout(int64_t r, int64_t d, int64_t n, int bits, int group, int
 }  // namespace
 
 extern "C" size_t gptq_layer_host_workspace_bytes(int64_t r, int64_t d, int64_t n, int bits,
-                                                  int group, int block, int act_order) {
-  if (!valid_layer(r, d, bits, group, block) || n < 0 || n > (int64_t)INT32_MAX) return 0;
-  return host_layout(r, d, n, bits, group, block, act_order).total;
+                                                  int group, int block, int options) {
+  if (!valid_layer(r, d, bits, group, block) || !valid_options(options) || n < 0 ||
+      n > (int64_t)INT32_MAX)
+    return 0;
+  return host_layout(r, d, n, bits, group, block, options).total;
 }
 
 extern "C" int gptq_solve_layer_host(const uint16_t *X_host, int64_t n, const float *W_host,
                                      int64_t r, int64_t d, int bits, int group, int block,
-                                     float damp, int act_order, int32_t *qweight_host,
+                                     float damp, int options, int32_t *qweight_host,
                                      float *scales_host, int32_t *zeros_host,
                                      int32_t *g_idx_host, double *loss, void *dev_workspace,
                                      size_t dev_workspace_bytes, gptq_stream_t stream) {
-  if (!valid_layer(r, d, bits, group, block) || n < 0 || n > (int64_t)INT32_MAX)
+  if (!valid_layer(r, d, bits, group, block) || !valid_options(options) || n < 0 ||
+      n > (int64_t)INT32_MAX)
     return GPTQ_ERR_INVALID_ARG;
   if ((n > 0 && !X_host) || !W_host || !qweight_host || !scales_host || !zeros_host ||
       !dev_workspace || reinterpret_cast<uintptr_t>(dev_workspace) % 256)
@@ -491,7 +506,7 @@ extern "C" int gptq_solve_layer_host(const uint16_t *X_host, int64_t n, const fl
     if (loss) *loss = 0.0;
     return GPTQ_OK;
   }
-  const HostLayout L = host_layout(r, d, n, bits, group, block, act_order);
+  const HostLayout L = host_layout(r, d, n, bits, group, block, options);
   if (dev_workspace_bytes < L.total) return GPTQ_ERR_NO_MEMORY;
   cudaStream_t st = (cudaStream_t)stream;
   char *ws = static_cast<char *>(dev_workspace);
@@ -525,7 +540,7 @@ extern "C" int gptq_solve_layer_host(const uint16_t *X_host, int64_t n, const fl
   }
   GPTQ_CUDA_TRY(cudaEventRecord(cs->ev[nch + 1], cs->s));   // W (copied first) and all of X
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(st, cs->ev[nch + 1], 0));
-  GPTQ_TRY(gptq_quantize_layer(W, r, d, H, bits, group, block, damp, act_order, nullptr, qw, sc,
+  GPTQ_TRY(gptq_quantize_layer(W, r, d, H, bits, group, block, damp, options, nullptr, qw, sc,
                                zr, gi, nullptr, loss, ws + L.qws, L.total - L.qws, stream));
   GPTQ_CUDA_TRY(cudaMemcpyAsync(qweight_host, qw, (size_t)r * (d * bits / 32) * 4,
                                 cudaMemcpyDeviceToHost, st));

@@ -35,6 +35,15 @@ def _stream(stream) -> int:
     return stream.cuda_stream
 
 
+# Option bits of the layer solve (include/gptq.h).
+ACT_ORDER, SYMMETRIC, STATIC_GROUPS = 1, 2, 4
+
+
+def _options(act_order: bool, sym: bool, static_groups: bool) -> int:
+    return ((ACT_ORDER if act_order else 0) | (SYMMETRIC if sym else 0)
+            | (STATIC_GROUPS if static_groups else 0))
+
+
 def _ptr(t: torch.Tensor | None, dtype: torch.dtype | None = None, name: str = "") -> int | None:
     if t is None:
         return None
@@ -59,20 +68,26 @@ def gptq_hessian_accumulate(X: torch.Tensor, H: torch.Tensor, stream=None) -> No
 
 
 def gptq_quantize_workspace_bytes(r: int, d: int, bits: int, group: int, block: int = 128,
-                                  act_order: bool = False) -> int:
-    return int(_abi.load().gptq_quantize_workspace_bytes(r, d, bits, group, block,
-                                                         int(act_order)))
+                                  act_order: bool = False, sym: bool = False,
+                                  static_groups: bool = False) -> int:
+    return int(_abi.load().gptq_quantize_workspace_bytes(
+        r, d, bits, group, block, _options(act_order, sym, static_groups)))
 
 
 def gptq_quantize_layer(W: torch.Tensor, H: torch.Tensor, *, bits: int, group: int,
                         block: int = 128, damp: float = 0.01, act_order: bool = False,
+                        sym: bool = False, static_groups: bool = False,
                         W_hat: torch.Tensor | None = None, codes: torch.Tensor | None = None,
                         g_idx: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                         outputs: dict | None = None, stream=None) -> dict:
     """GPTQ solve of one layer.  H is consumed.  Returns qweight/scales/zeros/loss (+ optional).
 
-    ``outputs`` may hold preallocated ``qweight``, ``scales`` and ``zeros`` tensors.
+    ``sym`` selects the symmetric quantiser and ``static_groups`` fixes every
+    group's parameters from the original W before the sweep (GPTQ_SYMMETRIC and
+    GPTQ_STATIC_GROUPS of the C header).  ``outputs`` may hold preallocated
+    ``qweight``, ``scales`` and ``zeros`` tensors.
     """
+    options = _options(act_order, sym, static_groups)
     lib = _abi.load()
     r, d = W.shape
     G = 1 if group == -1 else d // max(group, 1)
@@ -87,7 +102,7 @@ def gptq_quantize_layer(W: torch.Tensor, H: torch.Tensor, *, bits: int, group: i
     zeros = out.get("zeros")
     if zeros is None:
         zeros = torch.empty((r, G), dtype=torch.int32, device=dev)
-    need = lib.gptq_quantize_workspace_bytes(r, d, bits, group, block, int(act_order))
+    need = lib.gptq_quantize_workspace_bytes(r, d, bits, group, block, options)
     if need == 0 and r > 0:
         raise GPTQError(1, "gptq_quantize_workspace_bytes")
     if workspace is None:
@@ -95,7 +110,7 @@ def gptq_quantize_layer(W: torch.Tensor, H: torch.Tensor, *, bits: int, group: i
     loss = ctypes.c_double(0.0)
     _check(lib.gptq_quantize_layer(
         _ptr(W, torch.float32, "W"), r, d, _ptr(H, torch.float32, "H"), bits, group, block,
-        float(damp), int(act_order), _ptr(W_hat, torch.float32, "W_hat"),
+        float(damp), options, _ptr(W_hat, torch.float32, "W_hat"),
         _ptr(qweight, torch.int32, "qweight"), _ptr(scales, torch.float32, "scales"),
         _ptr(zeros, torch.int32, "zeros"), _ptr(g_idx, torch.int32, "g_idx"),
         _ptr(codes, torch.uint8, "codes"), ctypes.byref(loss), _ptr(workspace, None, "workspace"),
@@ -141,13 +156,15 @@ def gptq_pack(codes: torch.Tensor, bits: int, qweight: torch.Tensor | None = Non
 
 
 def gptq_layer_host_workspace_bytes(r: int, d: int, n: int, bits: int, group: int,
-                                    block: int = 128, act_order: bool = False) -> int:
-    return int(_abi.load().gptq_layer_host_workspace_bytes(r, d, n, bits, group, block,
-                                                           int(act_order)))
+                                    block: int = 128, act_order: bool = False,
+                                    sym: bool = False, static_groups: bool = False) -> int:
+    return int(_abi.load().gptq_layer_host_workspace_bytes(
+        r, d, n, bits, group, block, _options(act_order, sym, static_groups)))
 
 
 def gptq_solve_layer_host(X: torch.Tensor, W: torch.Tensor, *, bits: int, group: int,
                           block: int = 128, damp: float = 0.01, act_order: bool = False,
+                          sym: bool = False, static_groups: bool = False,
                           dev_workspace: torch.Tensor, outputs: dict, stream=None) -> float:
     """Whole layer from host (CPU, ideally pinned) tensors; fills ``outputs`` host tensors."""
     lib = _abi.load()
@@ -161,7 +178,8 @@ def gptq_solve_layer_host(X: torch.Tensor, W: torch.Tensor, *, bits: int, group:
     loss = ctypes.c_double(0.0)
     gi = outputs.get("g_idx")
     _check(lib.gptq_solve_layer_host(
-        X.data_ptr(), n, W.data_ptr(), r, d, bits, group, block, float(damp), int(act_order),
+        X.data_ptr(), n, W.data_ptr(), r, d, bits, group, block, float(damp),
+        _options(act_order, sym, static_groups),
         outputs["qweight"].data_ptr(), outputs["scales"].data_ptr(), outputs["zeros"].data_ptr(),
         gi.data_ptr() if gi is not None else None, ctypes.byref(loss),
         _ptr(dev_workspace, None, "dev_workspace"),

@@ -49,8 +49,11 @@ def test_workspace_query(lib):
                 (16, 256, 4, 48, 128, 0),      # group not a divisor of the block
                 (16, 256, 4, 96, 128, 0),
                 (16, 256, 4, -1, 96, 0),       # block
-                (-1, 256, 4, -1, 128, 0)]:
+                (-1, 256, 4, -1, 128, 0),
+                (16, 256, 4, -1, 128, 8)]:     # unknown option bit
         assert ws(*bad) == 0, bad
+    # the option bits GPTQ_SYMMETRIC and GPTQ_STATIC_GROUPS need no extra workspace
+    assert ws(4096, 4096, 4, 128, 128, 2 | 4) == base
     hw = lib.gptq_layer_host_workspace_bytes(128, 256, 2048, 4, -1, 128, 0)
     assert hw >= 2048 * 256 * 2 + 256 * 256 * 4 + 128 * 256 * 4
 
@@ -66,6 +69,9 @@ def test_validation_returns_before_cuda(lib):
     assert q(p, 8, 256, p, 4, -1, 128, -1.0, 0, None, p, p, p, None, None,
              ctypes.byref(loss), p, 1 << 30, None) == 1
     assert q(p, 8, 256, p, 4, -1, 128, float("nan"), 0, None, p, p, p, None, None,
+             ctypes.byref(loss), p, 1 << 30, None) == 1
+    # unknown option bit
+    assert q(p, 8, 256, p, 4, -1, 128, 0.01, 8, None, p, p, p, None, None,
              ctypes.byref(loss), p, 1 << 30, None) == 1
     # missing output pointer
     assert q(p, 8, 256, p, 4, -1, 128, 0.01, 0, None, None, p, p, None, None,

@@ -119,6 +119,42 @@ def test_full_path_matches_oracle(case):
     check_against_oracle(got, ref, W, bits=bits, group=group)
 
 
+VARIANT_CASES = [
+    # r, d, n, bits, group, block, act_order, sym, static_groups
+    (64, 512, 4096, 4, -1, 128, False, True, False),
+    (48, 384, 3000, 4, 128, 128, True, True, False),
+    (50, 256, 2048, 3, 32, 128, False, True, False),
+    (40, 512, 4096, 4, 64, 128, False, False, True),
+    (48, 384, 3000, 4, 128, 128, True, False, True),
+    (37, 512, 4096, 3, 32, 128, True, True, True),
+    (33, 512, 4096, 4, 256, 128, True, False, True),    # groups longer than the block
+    (64, 256, 2048, 2, 64, 64, True, True, True),
+]
+
+
+@pytest.mark.parametrize("case", VARIANT_CASES, ids=lambda c: "r{}_d{}_b{}_g{}_a{}_s{}_t{}".format(
+    c[0], c[1], c[3], c[4], int(c[6]), int(c[7]), int(c[8])))
+def test_quantiser_variants_match_oracle(case):
+    # Symmetric quantiser and static groups, alone and with act-order, from the
+    # same fp32 Hessian on both sides.
+    r, d, n, bits, group, block, act, sym, static = case
+    X, W = make_problem(r, d, n, seed=r * 13 + d)
+    H32 = oracle.hessian(X).astype(np.float32)
+    got = gpu_layer(None, W, bits=bits, group=group, block=block, act_order=act, H32=H32,
+                    sym=sym, static_groups=static)
+    ref = oracle.gptq_quantize_layer(W, H32.astype(np.float64), bits=bits, group=group,
+                                     block=block, act_order=act, sym=sym, static_groups=static)
+    check_against_oracle(got, ref, W, bits=bits, group=group)
+    if sym:
+        assert np.all(got["zeros"] == 1 << (bits - 1))
+    if static:
+        np.testing.assert_array_equal(got["g_idx"], np.arange(d) // group)
+        # fixed from the original W before the sweep: the same on both sides up
+        # to the fp32 division
+        np.testing.assert_allclose(got["scales"], ref["scales"], rtol=1e-6)
+        assert float(np.mean(got["zeros"] == ref["zeros"])) >= 0.999
+
+
 def test_tiny_workload_end_to_end():
     wl = workload("tiny_128x256")
     X, W = workload_inputs(wl)
