@@ -344,6 +344,27 @@ def test_dequant_gemv_matches_oracle(case):
                                rtol=1e-6, atol=1e-6 * np.abs(ref).max())
 
 
+@pytest.mark.parametrize("d,m,bits", [(4096, 8, 4), (16384, 2, 3), (8192, 8, 4), (65536, 1, 2),
+                                      (2048, 5, 8)])
+def test_dequant_gemv_staged_and_direct_x(d, m, bits):
+    # x is staged in shared memory when m * d * 4.5 bytes fit in 200 KB and read
+    # from global memory otherwise ((8192, 8) and (65536, 1)); both give the
+    # float64 oracle's product on random packed rows.
+    import post_weight_quantization_19_b200 as g
+    r, group = 67, 128
+    rng = np.random.default_rng(d + m)
+    codes = rng.integers(0, 1 << bits, size=(r, d), dtype=np.uint8)
+    qweight = oracle.pack_rows(codes, bits)
+    scales = (rng.random((r, d // group)) * 0.01 + 1e-3).astype(np.float32)
+    zeros = rng.integers(0, 1 << bits, size=(r, d // group)).astype(np.int32)
+    x = rng.standard_normal((m, d)).astype(np.float32)
+    y = g.gptq_dequant_gemv(*(torch.from_numpy(a).cuda() for a in (qweight, scales, zeros, x)),
+                            bits, group)
+    torch.cuda.synchronize()
+    ref = oracle.dequant_gemv(qweight, scales, zeros, bits, group, x)
+    assert np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max() <= 1e-5
+
+
 def test_dequant_gemv_full_layer_bandwidth():
     # The 4096 x 4096 4-bit group-128 layer at batch 1: parity on all rows and the
     # achieved read bandwidth (packed codes + scales + zeros + x) printed.
