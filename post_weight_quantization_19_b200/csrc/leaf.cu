@@ -124,7 +124,7 @@ __device__ __forceinline__ void cf_barrier() {
 // Column factor of an N x N block at S (leading dimension LLD, N = 32 or 64)
 // by CF_THREADS threads: H_d = R R^T with R upper, overwritten by U = R^-1.
 // Thread (gr, gc) of a (CF_THREADS / GC) x GC grid keeps the TR x TC tile at rows
-// gr * TR, columns gc * TC in registers.  Step k = N-1 .. 0 reads a vector v
+// gr * TR, columns gc * TC in registers.  Step k = N-1 .. 0 uses a vector v
 // that holds column k above the diagonal (v_j = S[j][k], j < k), the pivot
 // p = S[k][k] at index k and row k right of the diagonal (v_j = S[k][j],
 // j > k).  With v_k taken as 1,
@@ -133,12 +133,19 @@ __device__ __forceinline__ void cf_barrier() {
 // i.e. the Cholesky update of the leading block together with the
 // substitution that turns the finished rows into rows of R^-1.  Rows below k
 // are final; entries below the diagonal may pick up junk on the way and are
-// zeroed when the tile is written back.  The owners of column k-1 and row k-1
-// publish the next vector into the other half of a double buffer, so a step
-// costs one CTA barrier.  Returns false (in every thread) on a non-positive
-// pivot.
+// zeroed when the tile is written back.
+//
+// Steps go in pairs (k, k-1) with one barrier per pair: before it, the owners
+// publish the vector of step k and the vector of step k-1 as it stands before
+// step k; after it, every thread applies step k to the second vector's entries
+// that it needs (its rows, its columns, the pivot) with the same fused
+// multiply-adds the owners apply to their tiles, so the second step sees
+// exactly the values a barrier between the two steps would have published.
+// The published pairs alternate between two halves of vbuf (4 N floats).
+// Returns false (in every thread) on a non-positive pivot.
 template <int N>
 __device__ __forceinline__ bool col_factor(real *S, real *vbuf) {
+  static_assert(N % 2 == 0, "pairs of steps");
   __shared__ int cf_ok;
   if (threadIdx.x >= CF_THREADS) {   // the other warps wait at the closing barrier
     __syncthreads();
@@ -155,50 +162,92 @@ __device__ __forceinline__ bool col_factor(real *S, real *vbuf) {
   for (int r = 0; r < TR; ++r)
 #pragma unroll
     for (int q = 0; q < TC; ++q) t[r][q] = owner ? S[(i0 + r) * LLD + j0 + q] : 0.f;
-  if (owner && j0 + TC == N) {
+
+  // The owners' entries of the vectors of steps kk (into A) and kk - 1 (into B):
+  // column kk up to the diagonal and row kk right of it, likewise for kk - 1.
+  auto publish = [&](int kk, real *A) {
+    real *B = A + N;
 #pragma unroll
-    for (int r = 0; r < TR; ++r) vbuf[((N - 1) & 1) * N + i0 + r] = t[r][TC - 1];
-  }
-  cf_barrier();
+    for (int r = 0; r < TR; ++r)
+#pragma unroll
+      for (int q = 0; q < TC; ++q) {
+        const int i = i0 + r, j = j0 + q;
+        if (j == kk && i <= kk) A[i] = t[r][q];
+        if (i == kk && j > kk) A[j] = t[r][q];
+        if (j == kk - 1 && i <= kk - 1) B[i] = t[r][q];
+        if (i == kk - 1 && j > kk - 1) B[j] = t[r][q];
+      }
+  };
+  // One step k on the tile, from the vector entries of its rows (vr) and
+  // columns (vc); mip = -1/p, ri = 1/sqrt(p).
+  auto step = [&](int k, const real (&vr)[TR], const real (&vc)[TC], real mip, real ri) {
+    if (!(owner && i0 <= k)) return;
+    real c[TR], v[TC];
+#pragma unroll
+    for (int r = 0; r < TR; ++r) c[r] = i0 + r < k ? vr[r] * mip : 0.f;
+#pragma unroll
+    for (int q = 0; q < TC; ++q) v[q] = j0 + q == k ? 1.f : vc[q];
+#pragma unroll
+    for (int r = 0; r < TR; ++r)
+#pragma unroll
+      for (int q = 0; q < TC; ++q) t[r][q] = fmaf(c[r], v[q], j0 + q == k ? 0.f : t[r][q]);
+#pragma unroll
+    for (int r = 0; r < TR; ++r)
+      if (i0 + r == k) {
+#pragma unroll
+        for (int q = 0; q < TC; ++q) t[r][q] = v[q] * ri;
+      }
+  };
   bool bad = false;
-  // Fully unrolled: every comparison with k below becomes static.
-#pragma unroll
-  for (int k = N - 1; k >= 0; --k) {
-    const real *vb = vbuf + (k & 1) * N;
-    real p = vb[k];
+  auto pivot = [&](real p, real &mip, real &ri) {
     bad |= !(p > 0.f);
     p = bad ? 1.f : p;
-    real ri = rsqrtf(p);
+    ri = rsqrtf(p);
     ri = ri * fmaf(-0.5f * p * ri, ri, 1.5f);   // one Newton step
-    if (owner && i0 <= k) {
-      const real mip = -ri * ri;
-      real c[TR], v[TC];
+    mip = -ri * ri;
+  };
+
+  constexpr int NP = N / 2;   // pairs; pair P holds steps 2P+1 and 2P
+  if (owner) publish(N - 1, vbuf + ((NP - 1) & 1) * 2 * N);
+  cf_barrier();
+  // Fully unrolled: every comparison with k below becomes static.
 #pragma unroll
-      for (int r = 0; r < TR; ++r) c[r] = i0 + r < k ? vb[i0 + r] * mip : 0.f;
+  for (int P = NP - 1; P >= 0; --P) {
+    const int k = 2 * P + 1;
+    const real *A = vbuf + (P & 1) * 2 * N;
+    const real *B = A + N;
+    real mipa, ria;
+    pivot(A[k], mipa, ria);
+    real ar[TR], ac[TC];
 #pragma unroll
-      for (int q = 0; q < TC; ++q) v[q] = j0 + q == k ? 1.f : vb[j0 + q];
+    for (int r = 0; r < TR; ++r) ar[r] = A[i0 + r];
 #pragma unroll
-      for (int r = 0; r < TR; ++r)
+    for (int q = 0; q < TC; ++q) ac[q] = A[j0 + q];
+    // Step k's effect on the entries of step k-1's vector, written as the
+    // owners compute it: c = S[x][k] * mip times v = S[k-1][k] for the column
+    // part (x < k-1), c = S[k-1][k] * mip times v_x (v_k = 1, and 0 replaces
+    // the old entry at x = k) for the pivot and the row part (x >= k-1).
+    const real akm = A[k - 1];
+    const real ckm = akm * mipa;
+    real br[TR], bc[TC];
 #pragma unroll
-        for (int q = 0; q < TC; ++q) t[r][q] = fmaf(c[r], v[q], j0 + q == k ? 0.f : t[r][q]);
-#pragma unroll
-      for (int r = 0; r < TR; ++r)
-        if (i0 + r == k) {
-#pragma unroll
-          for (int q = 0; q < TC; ++q) t[r][q] = v[q] * ri;
-        }
-      const int kn = k - 1;
-      if (kn >= 0) {
-        real *nb = vbuf + (kn & 1) * N;
-#pragma unroll
-        for (int r = 0; r < TR; ++r)
-#pragma unroll
-          for (int q = 0; q < TC; ++q) {
-            if (j0 + q == kn && i0 + r <= kn) nb[i0 + r] = t[r][q];
-            if (i0 + r == kn && j0 + q > kn) nb[j0 + q] = t[r][q];
-          }
-      }
+    for (int r = 0; r < TR; ++r) {
+      const int x = i0 + r;
+      br[r] = x < k - 1 ? fmaf(ar[r] * mipa, akm, B[x])
+                        : fmaf(ckm, x == k ? 1.f : ar[r], x == k ? 0.f : B[x]);
     }
+#pragma unroll
+    for (int q = 0; q < TC; ++q) {
+      const int x = j0 + q;
+      bc[q] = x < k - 1 ? fmaf(ac[q] * mipa, akm, B[x])
+                        : fmaf(ckm, x == k ? 1.f : ac[q], x == k ? 0.f : B[x]);
+    }
+    const real pb = fmaf(ckm, akm, B[k - 1]);
+    step(k, ar, ac, mipa, ria);
+    real mipb, rib;
+    pivot(pb, mipb, rib);
+    step(k - 1, br, bc, mipb, rib);
+    if (P > 0 && owner) publish(k - 2, vbuf + ((P - 1) & 1) * 2 * N);
     cf_barrier();
   }
   if (owner) {
@@ -245,7 +294,7 @@ __device__ __forceinline__ bool node_factor(real *S, real *T, real *vbuf, int of
 
 __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb, int *status) {
   extern __shared__ real lsm[];
-  __shared__ real vbuf[2 * BASE];
+  __shared__ real vbuf[4 * BASE];   // two published pairs of vectors
   pdl_wait_then_release();
   if (*(volatile int *)status) return;
   real *S = lsm;
