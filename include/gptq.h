@@ -201,6 +201,32 @@ int gptq_dequant_gemv(const int32_t *qweight, const float *scales, const int32_t
                       const float *x, int64_t m, float *y, gptq_stream_t stream);
 
 /*
+ * gptq_dequant_fp16 / gptq_linear_fp16 -- run a quantised layer forward on
+ * calibration tokens, to calibrate the next layer on what this one outputs
+ *   ([Card] §计算设置: each block is quantised, then run to produce the next
+ *   block's inputs; [Concept] §3 技術原理: the codes are dequantised to FP16
+ *   and multiplied in floating point)
+ *
+ * gptq_dequant_fp16: W16[row, c] = fp16(scales[row, gi(c)] * (q[row, c] -
+ *   zeros[row, gi(c)])) from the packed layer (arguments as gptq_dequant_gemv;
+ *   W16 device fp16 [r x d], 16-byte aligned, written).  Asynchronous.
+ * gptq_linear_fp16: Y = fp16(X W16^T) -- X device fp16 [n x d] (tokens x
+ *   features), W16 device fp16 [r x d], Y device fp16 [n x r], all row-major and
+ *   16-byte aligned; d % 32 == 0, r % 32 == 0.  fp32 accumulation on the tensor
+ *   cores, folded every 512 features, one rounding to fp16 per output (values
+ *   beyond the fp16 range become +-inf).  n == 0 or r == 0: nothing to do.
+ *   Asynchronous; a bounded in-kernel wait that runs out is reported by
+ *   gptq_check_device_status.
+ * Both return GPTQ_ERR_INVALID_ARG before launching anything when an argument
+ * is out of range.
+ */
+int gptq_dequant_fp16(const int32_t *qweight, const float *scales, const int32_t *zeros,
+                      const int32_t *g_idx, int64_t r, int64_t d, int bits, int group, void *W16,
+                      gptq_stream_t stream);
+int gptq_linear_fp16(const void *X, int64_t n, int64_t d, const void *W16, int64_t r, void *Y,
+                     gptq_stream_t stream);
+
+/*
  * gptq_quantize_layer_noalloc -- gptq_quantize_layer for callers that cannot
  * allocate device memory.  (The GPTQ pages have no counterpart: this is a
  * deployment convenience of this library, not a step of the method.)

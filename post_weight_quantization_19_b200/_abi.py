@@ -32,6 +32,9 @@ SIGNATURES = {
     "gptq_pack": (c_int, [c_void_p, c_int64, c_int64, c_int, c_void_p, c_void_p]),
     "gptq_dequant_gemv": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int,
                                   c_int, c_void_p, c_int64, c_void_p, c_void_p]),
+    "gptq_dequant_fp16": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int,
+                                  c_int, c_void_p, c_void_p]),
+    "gptq_linear_fp16": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int64, c_void_p, c_void_p]),
     "gptq_quantize_layer_noalloc": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int, c_int,
                                             c_int, c_float, c_int, c_void_p, c_void_p, c_void_p,
                                             c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),

@@ -144,6 +144,37 @@ def gptq_dequant_gemv(qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.
     return y
 
 
+def gptq_dequant_fp16(qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, d: int,
+                      bits: int, group: int, g_idx: torch.Tensor | None = None,
+                      W16: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """W16 [r, d] fp16 = s (q - z) from the packed layer."""
+    lib = _abi.load()
+    r = qweight.shape[0]
+    if W16 is None:
+        W16 = torch.empty((r, d), dtype=torch.float16, device=qweight.device)
+    _check(lib.gptq_dequant_fp16(
+        _ptr(qweight, torch.int32, "qweight"), _ptr(scales, torch.float32, "scales"),
+        _ptr(zeros, torch.int32, "zeros"), _ptr(g_idx, torch.int32, "g_idx"), r, d, bits, group,
+        _ptr(W16, torch.float16, "W16"), _stream(stream)), "gptq_dequant_fp16")
+    return W16
+
+
+def gptq_linear_fp16(X: torch.Tensor, W16: torch.Tensor, Y: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Y [n, r] = fp16(X [n, d] W16 [r, d]^T), fp32 accumulation on the tensor cores."""
+    lib = _abi.load()
+    n, d = X.shape
+    r = W16.shape[0]
+    if W16.shape[1] != d:
+        raise ValueError("W16 must be [r, d]")
+    if Y is None:
+        Y = torch.empty((n, r), dtype=torch.float16, device=X.device)
+    _check(lib.gptq_linear_fp16(_ptr(X, torch.float16, "X"), n, d, _ptr(W16, torch.float16, "W16"),
+                                r, _ptr(Y, torch.float16, "Y"), _stream(stream)),
+           "gptq_linear_fp16")
+    return Y
+
+
 def gptq_pack(codes: torch.Tensor, bits: int, qweight: torch.Tensor | None = None,
               stream=None) -> torch.Tensor:
     lib = _abi.load()

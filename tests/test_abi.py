@@ -101,6 +101,17 @@ def test_validation_returns_before_cuda(lib):
     assert gv(p, p, p, None, 8, 128, 4, -1, None, 1, p, None) == 1  # missing x
     assert gv(p, p, p, None, 0, 128, 4, -1, p, 1, p, None) == 0     # no rows: nothing to do
     assert gv(p, p, p, None, 8, 128, 4, -1, p, 0, p, None) == 0     # no vectors
+    df = lib.gptq_dequant_fp16
+    assert df(p, p, p, None, 8, 100, 4, -1, p, None) == 1           # d % 32
+    assert df(p, p, p, None, 8, 128, 6, -1, p, None) == 1           # bits
+    assert df(p, p, p, None, 8, 128, 4, -1, ctypes.c_void_p(4104), None) == 1   # W16 alignment
+    assert df(p, p, p, None, 0, 128, 4, -1, p, None) == 0           # no rows
+    lf = lib.gptq_linear_fp16
+    assert lf(p, 16, 100, p, 64, p, None) == 1                      # d % 32
+    assert lf(p, 16, 128, p, 40, p, None) == 1                      # r % 32
+    assert lf(ctypes.c_void_p(4104), 16, 128, p, 64, p, None) == 1  # X alignment
+    assert lf(p, 0, 128, p, 64, p, None) == 0                       # no tokens
+    assert lf(p, 16, 128, p, 0, p, None) == 0                       # no outputs
 
 
 def test_no_kernels_launched_on_cpu(lib):

@@ -365,6 +365,84 @@ def test_dequant_gemv_staged_and_direct_x(d, m, bits):
     assert np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max() <= 1e-5
 
 
+# ------------------------------------------------------------------ the layer run forward
+
+def _fp16_ulps(a, b):
+    # distance in units in the last place between fp16 arrays of finite values
+    ia = a.view(np.int16).astype(np.int32)
+    ib = b.view(np.int16).astype(np.int32)
+    ia = np.where(ia < 0, -32768 - ia, ia)
+    ib = np.where(ib < 0, -32768 - ib, ib)
+    return np.abs(ia - ib)
+
+
+@pytest.mark.parametrize("bits,group,act", [(4, 128, False), (3, -1, False), (4, 32, True)])
+def test_dequant_fp16_matches_oracle(bits, group, act):
+    # fp16(s (q - z)) from the GPU's own packed layer; the oracle forms s (q - z)
+    # exactly and rounds once, the kernel rounds the fp32 product: equal except
+    # where the fp32 product lands on an fp16 tie (at most one fp16 step).
+    import post_weight_quantization_19_b200 as g
+    X, W = make_problem(70, 512, 3000, seed=60 + bits)
+    got = gpu_layer(X, W, bits=bits, group=group, act_order=act)
+    q = torch.from_numpy(got["qweight"]).cuda()
+    W16 = g.gptq_dequant_fp16(q, torch.from_numpy(got["scales"]).cuda(),
+                              torch.from_numpy(got["zeros"]).cuda(), 512, bits, group,
+                              g_idx=torch.from_numpy(got["g_idx"]).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.dequant_gemv(got["qweight"], got["scales"], got["zeros"], bits, group,
+                              np.eye(512), g_idx=got["g_idx"]).T.astype(np.float16)
+    ulps = _fp16_ulps(W16.cpu().numpy(), ref)
+    assert ulps.max() <= 1 and float(np.mean(ulps == 0)) >= 0.9999
+
+
+@pytest.mark.parametrize("n,d,r", [(1000, 2080, 288), (256, 64, 32), (4096, 512, 768)])
+def test_linear_fp16_matches_oracle(n, d, r):
+    # Y = fp16(X W16^T): float64 sum of the fp16 products rounded once, against the
+    # tensor cores' fp32 accumulation (folded every 512 features) rounded once --
+    # equal except within fp32 rounding of an fp16 rounding boundary.  The shapes
+    # have ragged token tiles, a half-empty last feature stage and a ragged
+    # output tile.
+    import post_weight_quantization_19_b200 as g
+    rng = np.random.default_rng(n + d + r)
+    X = make_activations(n, d, seed=n + d)
+    W16 = (0.02 * rng.standard_normal((r, d))).astype(np.float16)
+    Y = g.gptq_linear_fp16(torch.from_numpy(X).cuda(), torch.from_numpy(W16).cuda())
+    torch.cuda.synchronize()
+    ref = (X.astype(np.float64) @ W16.astype(np.float64).T).astype(np.float16)
+    got = Y.cpu().numpy()
+    assert np.all(np.isfinite(got))
+    ulps = _fp16_ulps(got, ref)
+    assert ulps.max() <= 1 and float(np.mean(ulps == 0)) >= 0.999
+
+
+def test_chain_of_layers_matches_oracle():
+    # Three layers (256 -> 384 -> 128 -> 256), each calibrated on the quantised
+    # outputs of the previous ones.  Layer 0 has the single-layer tolerance.  The
+    # later layers see inputs that differ from the oracle's wherever layer 0 took
+    # a rounding tie the other way or an fp16 output rounded the other way, so
+    # their bar is looser: codes 99 % identical and within one step, loss within 1 %.
+    import post_weight_quantization_19_b200 as g
+    X0 = make_activations(4096, 256, seed=71)
+    shapes = [(384, 256), (128, 384), (256, 128)]
+    Ws = [make_weights(rr, dd, seed=72 + i) for i, (rr, dd) in enumerate(shapes)]
+    codes_gpu = []
+    outs = g.quantize_chain(torch.from_numpy(X0).cuda(),
+                            [torch.from_numpy(np.ascontiguousarray(W, dtype=np.float32)).cuda()
+                             for W in Ws], bits=4, group=128, keep_inputs=True)
+    torch.cuda.synchronize()
+    ref = oracle.quantize_chain(X0, Ws, bits=4, group=128)
+    for k, (o, rf) in enumerate(zip(outs, ref)):
+        d = Ws[k].shape[1]
+        codes = oracle.unpack_rows(o["qweight"].cpu().numpy(), 4, d)
+        codes_gpu.append(codes)
+        assert_codes_close(codes, rf["codes"], 0.999 if k == 0 else 0.99)
+        rel = abs(o["loss"] - rf["loss"]) / rf["loss"]
+        assert rel <= (5e-3 if k == 0 else 1e-2), (k, rel)
+        xin = o["inputs"].cpu().numpy()
+        same = float(np.mean(xin == rf["inputs"]))
+        assert same >= (1.0 if k == 0 else 0.99), (k, same)
+
+
 def test_dequant_gemv_full_layer_bandwidth():
     # The 4096 x 4096 4-bit group-128 layer at batch 1: parity on all rows and the
     # achieved read bandwidth (packed codes + scales + zeros + x) printed.
