@@ -164,6 +164,48 @@ int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits
                         gptq_stream_t stream);
 
 /*
+ * gptq_factor / gptq_quantize_with_factor -- the solve in two halves, so that
+ * one factor serves several sweeps: rows of one layer spread over several
+ * GPUs, or several layers that read the same inputs and so share H.  The
+ * inverse-Hessian information does not depend on W ([Card] 方法适配: every row
+ * is quantised in the same order with the same factor).
+ *
+ * gptq_factor: steps 1-3 of gptq_quantize_layer.
+ *   H        device fp32 [d x d], full symmetric, 16-byte aligned.  On return
+ *            its upper triangle holds U in sweep order (the factor of the
+ *            permuted H_d under GPTQ_ACT_ORDER); the strictly lower triangle is
+ *            scratch.
+ *   options  GPTQ_ACT_ORDER is used; the other bits are accepted and ignored.
+ *   perm     device int32 [d] (GPTQ_ACT_ORDER; may be NULL otherwise): column
+ *            perm[j] of W is quantised j-th.
+ *   lambda   device fp32 [1]: the damping added to the diagonal (the loss
+ *            needs it).
+ *   workspace  gptq_factor_workspace_bytes(d, options) bytes, 256-byte aligned.
+ *   Synchronises `stream` once, at the end; returns GPTQ_ERR_NOT_PD if H_d is
+ *   not positive definite.
+ *
+ * gptq_quantize_with_factor: steps 4-6 of gptq_quantize_layer from a factor
+ *   made by gptq_factor with the same d and GPTQ_ACT_ORDER bit (U, perm and
+ *   lambda are read only, so they can serve any number of calls).  Other
+ *   arguments as gptq_quantize_layer; the workspace is
+ *   gptq_quantize_with_factor_workspace_bytes(r, d, bits, group, block) bytes.
+ *   A perm that is not a permutation of 0..d-1 is found on the device before
+ *   anything uses it and returns GPTQ_ERR_INVALID_ARG (outputs unspecified).
+ *   Synchronises `stream` once, at the end, to read the status and the loss.
+ */
+size_t gptq_factor_workspace_bytes(int64_t d, int options);
+int gptq_factor(float *H, int64_t d, float damp, int options, int32_t *perm, float *lambda,
+                void *workspace, size_t workspace_bytes, gptq_stream_t stream);
+size_t gptq_quantize_with_factor_workspace_bytes(int64_t r, int64_t d, int bits, int group,
+                                                 int block);
+int gptq_quantize_with_factor(const float *W, int64_t r, int64_t d, const float *U,
+                              const int32_t *perm, const float *lambda, int bits, int group,
+                              int block, int options, float *W_hat, int32_t *qweight,
+                              float *scales, int32_t *zeros, int32_t *g_idx, uint8_t *codes,
+                              double *loss, void *workspace, size_t workspace_bytes,
+                              gptq_stream_t stream);
+
+/*
  * gptq_pack -- pack codes into int32 words   ([Explainer] §三, int32 storage of 3/4-bit codes)
  *
  *   codes   device uint8 [r x d], values < 2^bits (higher bits are masked off).

@@ -16,9 +16,11 @@ from .gptq import (  # noqa: F401
     gptq_layer_host_workspace_bytes,
     gptq_dequant_fp16,
     gptq_dequant_gemv,
+    gptq_factor,
     gptq_linear_fp16,
     gptq_pack,
     gptq_quantize_layer,
+    gptq_quantize_with_factor,
     gptq_quantize_workspace_bytes,
     gptq_set_phase_timing,
     gptq_solve_layer_host,

@@ -112,6 +112,8 @@ int launch_damp(float *H, int64_t ld, int d, float damp, bool add_in_place, floa
                 cudaStream_t stream);
 int launch_act_order(const float *H, int64_t ld, int d, int *perm, int *inv, const float *lambda,
                      float *Hp, cudaStream_t stream);
+// inv[perm[p]] = p after checking that perm is a permutation (status set otherwise).
+int launch_check_perm(const int *perm, int d, int *inv, int *status, cudaStream_t stream);
 // Scratch of the factorisation: one h x m product per depth of the merge tree.
 size_t factor_scratch_floats(int64_t d);
 // One diagonal block (nb <= 128, nb % 32 == 0) of H_d -> U in place (full block, zeros below).

@@ -144,6 +144,78 @@ def gptq_dequant_gemv(qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.
     return y
 
 
+def gptq_factor(H: torch.Tensor, *, damp: float = 0.01, act_order: bool = False,
+                workspace: torch.Tensor | None = None, stream=None) -> dict:
+    """Damp, order and factor H in place: returns {"U": H, "perm", "lambda"} for
+    ``gptq_quantize_with_factor`` (perm is None without act-order)."""
+    lib = _abi.load()
+    d = H.shape[0]
+    if H.shape != (d, d):
+        raise ValueError("H must be [d, d]")
+    options = ACT_ORDER if act_order else 0
+    need = lib.gptq_factor_workspace_bytes(d, options)
+    if need == 0:
+        raise GPTQError(1, "gptq_factor_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=H.device)
+    perm = torch.empty(d, dtype=torch.int32, device=H.device) if act_order else None
+    lam = torch.empty(1, dtype=torch.float32, device=H.device)
+    _check(lib.gptq_factor(_ptr(H, torch.float32, "H"), d, float(damp), options,
+                           _ptr(perm, torch.int32, "perm"), _ptr(lam, torch.float32, "lambda"),
+                           _ptr(workspace, None, "workspace"),
+                           workspace.numel() * workspace.element_size(), _stream(stream)),
+           "gptq_factor")
+    return {"U": H, "perm": perm, "lambda": lam}
+
+
+def gptq_quantize_with_factor(W: torch.Tensor, factor: dict, *, bits: int, group: int,
+                              block: int = 128, sym: bool = False, static_groups: bool = False,
+                              W_hat: torch.Tensor | None = None, codes: torch.Tensor | None = None,
+                              g_idx: torch.Tensor | None = None,
+                              workspace: torch.Tensor | None = None, outputs: dict | None = None,
+                              stream=None) -> dict:
+    """The sweep half of the solve from ``gptq_factor``'s result (U, perm, lambda are
+    only read).  Returns qweight/scales/zeros/loss like ``gptq_quantize_layer``."""
+    lib = _abi.load()
+    r, d = W.shape
+    U, perm, lam = factor["U"], factor["perm"], factor["lambda"]
+    options = _options(perm is not None, sym, static_groups)
+    G = 1 if group == -1 else d // max(group, 1)
+    dev = W.device
+    out = dict(outputs or {})
+    qweight = out.get("qweight")
+    if qweight is None:
+        qweight = torch.empty((r, d * bits // 32), dtype=torch.int32, device=dev)
+    scales = out.get("scales")
+    if scales is None:
+        scales = torch.empty((r, G), dtype=torch.float32, device=dev)
+    zeros = out.get("zeros")
+    if zeros is None:
+        zeros = torch.empty((r, G), dtype=torch.int32, device=dev)
+    need = lib.gptq_quantize_with_factor_workspace_bytes(r, d, bits, group, block)
+    if need == 0 and r > 0:
+        raise GPTQError(1, "gptq_quantize_with_factor_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    loss = ctypes.c_double(0.0)
+    _check(lib.gptq_quantize_with_factor(
+        _ptr(W, torch.float32, "W"), r, d, _ptr(U, torch.float32, "U"),
+        _ptr(perm, torch.int32, "perm"), _ptr(lam, torch.float32, "lambda"), bits, group, block,
+        options, _ptr(W_hat, torch.float32, "W_hat"), _ptr(qweight, torch.int32, "qweight"),
+        _ptr(scales, torch.float32, "scales"), _ptr(zeros, torch.int32, "zeros"),
+        _ptr(g_idx, torch.int32, "g_idx"), _ptr(codes, torch.uint8, "codes"), ctypes.byref(loss),
+        _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "gptq_quantize_with_factor")
+    res = {"qweight": qweight, "scales": scales, "zeros": zeros, "loss": loss.value}
+    if W_hat is not None:
+        res["W_hat"] = W_hat
+    if codes is not None:
+        res["codes"] = codes
+    if g_idx is not None:
+        res["g_idx"] = g_idx
+    return res
+
+
 def gptq_dequant_fp16(qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, d: int,
                       bits: int, group: int, g_idx: torch.Tensor | None = None,
                       W16: torch.Tensor | None = None, stream=None) -> torch.Tensor:

@@ -101,6 +101,21 @@ def test_validation_returns_before_cuda(lib):
     assert gv(p, p, p, None, 8, 128, 4, -1, None, 1, p, None) == 1  # missing x
     assert gv(p, p, p, None, 0, 128, 4, -1, p, 1, p, None) == 0     # no rows: nothing to do
     assert gv(p, p, p, None, 8, 128, 4, -1, p, 0, p, None) == 0     # no vectors
+    fw = lib.gptq_factor_workspace_bytes
+    assert fw(100, 0) == 0 and fw(256, 8) == 0 and fw(256, 1) > fw(256, 0) > 0
+    f = lib.gptq_factor
+    assert f(p, 100, 0.01, 0, None, p, p, 1 << 30, None) == 1     # d % 32
+    assert f(p, 256, 0.01, 1, None, p, p, 1 << 30, None) == 1     # act-order without perm
+    assert f(p, 256, -1.0, 0, None, p, p, 1 << 30, None) == 1     # damp
+    assert f(p, 256, 0.01, 0, None, p, ctypes.c_void_p(1 << 20), 64, None) == 4   # workspace
+    qf = lib.gptq_quantize_with_factor
+    assert lib.gptq_quantize_with_factor_workspace_bytes(8, 256, 4, 128, 128) > 0
+    assert qf(p, 8, 256, p, None, p, 4, 128, 128, 1, None, p, p, p, None, None,
+              ctypes.byref(loss), p, 1 << 30, None) == 1             # act-order without perm
+    assert qf(p, 8, 256, p, None, p, 5, 128, 128, 0, None, p, p, p, None, None,
+              ctypes.byref(loss), p, 1 << 30, None) == 1             # bits
+    assert qf(p, 0, 256, p, None, p, 4, 128, 128, 0, None, p, p, p, None, None,
+              ctypes.byref(loss), p, 0, None) == 0                   # no rows
     df = lib.gptq_dequant_fp16
     assert df(p, p, p, None, 8, 100, 4, -1, p, None) == 1           # d % 32
     assert df(p, p, p, None, 8, 128, 6, -1, p, None) == 1           # bits

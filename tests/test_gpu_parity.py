@@ -155,6 +155,52 @@ def test_quantiser_variants_match_oracle(case):
         assert float(np.mean(got["zeros"] == ref["zeros"])) >= 0.999
 
 
+@pytest.mark.parametrize("act,sym,static", [(False, False, False), (True, False, False),
+                                             (True, True, True)])
+def test_factor_then_sweep_equals_one_call(act, sym, static):
+    # The two halves run the same kernels in the same order as the one call,
+    # so the outputs are the same bits; one factor then serves three layers
+    # that share the inputs (and so H), each equal to its own one-call solve.
+    import post_weight_quantization_19_b200 as g
+    X, _ = make_problem(1, 512, 4096, seed=91)
+    Ws = [make_weights(rr, 512, seed=92 + i) for i, rr in enumerate((96, 64, 160))]
+    H32 = oracle.hessian(X).astype(np.float32)
+    fac = g.gptq_factor(torch.from_numpy(H32.copy()).cuda(), act_order=act)
+    for W in Ws:
+        Wd = torch.from_numpy(W).cuda()
+        gi1 = torch.empty(512, dtype=torch.int32, device="cuda")
+        one = g.gptq_quantize_layer(Wd, torch.from_numpy(H32.copy()).cuda(), bits=4, group=128,
+                                    act_order=act, sym=sym, static_groups=static, g_idx=gi1)
+        gi2 = torch.empty(512, dtype=torch.int32, device="cuda")
+        two = g.gptq_quantize_with_factor(Wd, fac, bits=4, group=128, sym=sym,
+                                          static_groups=static, g_idx=gi2)
+        torch.cuda.synchronize()
+        for key in ("qweight", "scales", "zeros"):
+            np.testing.assert_array_equal(two[key].cpu().numpy(), one[key].cpu().numpy())
+        np.testing.assert_array_equal(gi2.cpu().numpy(), gi1.cpu().numpy())
+        assert two["loss"] == one["loss"]
+
+
+def test_sweep_rejects_a_perm_that_is_not_a_permutation():
+    # Checked on the device before anything indexes W with it.
+    import post_weight_quantization_19_b200 as g
+    X, W = make_problem(32, 256, 2048, seed=93)
+    fac = g.gptq_factor(torch.from_numpy(oracle.hessian(X).astype(np.float32)).cuda(),
+                        act_order=True)
+    bad = dict(fac)
+    bad["perm"] = fac["perm"].clone()
+    bad["perm"][7] = bad["perm"][3]          # a repeated entry
+    with pytest.raises(g.GPTQError) as e:
+        g.gptq_quantize_with_factor(torch.from_numpy(W).cuda(), bad, bits=4, group=128)
+    assert e.value.status == 1
+    bad["perm"][7] = 1 << 20                 # out of range
+    with pytest.raises(g.GPTQError):
+        g.gptq_quantize_with_factor(torch.from_numpy(W).cuda(), bad, bits=4, group=128)
+    # and the good one still works afterwards
+    res = g.gptq_quantize_with_factor(torch.from_numpy(W).cuda(), fac, bits=4, group=128)
+    assert res["loss"] > 0
+
+
 def test_tiny_workload_end_to_end():
     wl = workload("tiny_128x256")
     X, W = workload_inputs(wl)
