@@ -147,7 +147,7 @@ int gemv_launch_mb(const GemvArgs &a, cudaStream_t st) {
   size_t smem = 0;
   int64_t cap = (int64_t)num_sms() * 16;
   if constexpr (SX) {
-    static bool attr[64] = {};
+    static std::atomic<bool> attr[64] = {};
     smem = (size_t)a.m * (a.d / 32) * XPAD * sizeof(float);
     if (const int rc = ensure_smem_attr(gemv_kernel<BITS, MB, true>, GEMV_SMEM_MAX, attr))
       return rc;

@@ -53,15 +53,16 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // The dynamic shared-memory limit of a kernel, raised once per device (the
 // attribute belongs to the kernel in the current device's context).
+// (Two threads may both set it the first time; setting it twice is harmless.)
 template <typename K>
-int ensure_smem_attr(K kernel, size_t bytes, bool (&done)[64]) {
+int ensure_smem_attr(K kernel, size_t bytes, std::atomic<bool> (&done)[64]) {
   int dev = 0;
   GPTQ_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return GPTQ_ERR_INVALID_ARG;
-  if (!done[dev]) {
+  if (!done[dev].load(std::memory_order_acquire)) {
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bytes));
-    done[dev] = true;
+    done[dev].store(true, std::memory_order_release);
   }
   return GPTQ_OK;
 }

@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb,
 
 int launch_leaf(float *A, int64_t ld, int nb, int *status, cudaStream_t stream) {
   if (nb <= 0 || nb > LB || nb % 32 != 0) return GPTQ_ERR_INVALID_ARG;
-  static bool attr[64] = {};
+  static std::atomic<bool> attr[64] = {};
   if (const int rc = ensure_smem_attr(leaf_kernel, LEAF_SMEM, attr)) return rc;
   GPTQ_LAUNCH_PDL(leaf_kernel, dim3(1), dim3(LT), LEAF_SMEM, stream, A, ld, nb, status);
   return GPTQ_OK;

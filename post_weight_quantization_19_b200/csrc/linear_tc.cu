@@ -364,7 +364,7 @@ extern "C" int gptq_linear_fp16(const void *X, int64_t n, int64_t d, const void 
   }
   int *status = device_status_word();
   if (!status) return GPTQ_ERR_CUDA;
-  static bool attr[64] = {};
+  static std::atomic<bool> attr[64] = {};
   if (const int rc = ensure_smem_attr(linear_tc_kernel, LSMEM_BYTES, attr)) return rc;
   const int64_t T = ((n + LM - 1) / LM) * ((r + LN - 1) / LN);
   const int grid = (int)(T < num_sms() ? T : num_sms());

@@ -484,7 +484,7 @@ template <int CW, int L, bool VAR>
 static int sweep_launch(const SweepArgs &a, cudaStream_t stream) {
   constexpr int B = CW * L;
   const size_t smem = (size_t)B * (CW + 4) * L * sizeof(float);
-  static bool attr[64] = {};
+  static std::atomic<bool> attr[64] = {};
   if (const int rc = ensure_smem_attr(sweep_block_kernel<CW, L, VAR>, smem, attr)) return rc;
   // Every row gets its lanes in one wave when the SMs can hold them (two CTAs
   // per SM: about 180 registers per thread).

@@ -528,3 +528,36 @@ def test_dequant_gemv_full_layer_bandwidth():
     nbytes = qweight.nbytes + scales.nbytes + zeros.nbytes + x.nbytes + r * 4
     print(f"dequant_gemv 4096x4096 4-bit g128 m=1: {ms * 1e3:.2f} us, {nbytes / ms / 1e6:.0f} GB/s")
 
+
+
+@pytest.mark.parametrize("factor_once", [True, False])
+def test_sharded_solve_at_world_size_one(factor_once):
+    # The multi-rank path on one GPU (NCCL, one rank): the real entry points in
+    # the sharded layout give the single-call solve.
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    import post_weight_quantization_19_b200 as g
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        X, W = make_problem(80, 512, 4096, seed=95)
+        Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda()
+        res = g.solve_layer_sharded(Xd, Wd, bits=4, group=128, act_order=True,
+                                    factor_once=factor_once)
+        H = torch.zeros((512, 512), device="cuda")
+        g.gptq_hessian_accumulate(Xd, H)
+        gi = torch.empty(512, dtype=torch.int32, device="cuda")
+        one = g.gptq_quantize_layer(Wd, H, bits=4, group=128, act_order=True, g_idx=gi)
+        torch.cuda.synchronize()
+        for key in ("qweight", "scales", "zeros"):
+            np.testing.assert_array_equal(res[key].cpu().numpy(), one[key].cpu().numpy())
+        np.testing.assert_array_equal(res["g_idx"].cpu().numpy(), gi.cpu().numpy())
+        assert res["loss"] == pytest.approx(one["loss"], rel=1e-12)
+    finally:
+        dist.destroy_process_group()
