@@ -10,10 +10,10 @@
 // processed by a 2 x 2 block recursion,
 //     A22 -> U22;  T = A12 U22^T;  A11 -= T T^T;  A12 = T U22;
 //     A11 -> U11;  A12 = -U11 A12,
-// with register-tiled shared-memory products run by all LT threads, down to
-// blocks of at most BASE columns that CF_THREADS threads factor and invert one
-// column at a time (each thread keeps a small tile in registers; one barrier
-// per column).  The lower triangle is kept at zero between steps, so the
+// with shared-memory products on the tensor cores (warp-level 3xTF32 mma.sync,
+// all LT / 32 warps), down to blocks of at most BASE columns that CF_THREADS
+// threads factor and invert two columns per barrier (each thread keeps a small
+// tile in registers).  The lower triangle is kept at zero between steps, so the
 // triangular operands can be used as dense ones.
 #include "gptq_internal.h"
 
@@ -30,85 +30,75 @@ constexpr int BASE = 32;           // blocks up to this size go to the column fa
 constexpr size_t LEAF_SMEM = ((size_t)LB * LLD + 64 * 68) * sizeof(real);
 
 // C[M x N] = alpha * A[M x K] * op(B) + beta * C in shared memory, all shapes
-// and strides known at compile time; op(B) = B (K x N) or B^T (B stored N x K).
-// The M x N outputs are spread over all threads in RM x RN register tiles; A
-// (and B^T) are read 4 k values at a time with 16-byte loads.  A thread's
-// columns are interleaved (jt + TN c) when B is read transposed, so the B rows
-// of neighbouring threads fall in different banks, and contiguous otherwise,
-// for 16-byte loads of a B row.  UPPER: only entries with column >= row are
-// written (C is a diagonal block).  Ends with a CTA barrier.
+// and strides known at compile time; op(B) = B (K x N) or B^T (B stored N x K);
+// UPPER: only entries with column >= row are written (C is a diagonal block).
+// On the tensor cores: warp-level mma.sync m16n8k8 in TF32 with the error-compensated split
+// x = hi + lo (hi = tf32(x), lo = tf32(x - hi)) and three products per K step
+// (lo*hi and hi*lo first, then hi*hi), which keeps about 21 bits of each operand
+// -- the precision of the 3xTF32 products elsewhere in the factorisation.
+// Each warp takes 16 x 8 output tiles; fragment layout of m16n8k8 (lane = 4 g + t):
+// A[i0 + g (+8)][k + t (+4)], B[k + t (+4)][j0 + g], C[i0 + g (+8)][j0 + 2 t (+1)].
+// The padded leading dimensions (LLD = 132, m + 4) put the 32 lanes of every
+// fragment load in 32 different banks.  Ends with a CTA barrier.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+  hi = to_tf32(x);
+  lo = to_tf32(x - __uint_as_float(hi));
+}
+
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
+                                         const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 template <int M, int N, int K, int LDA, int LDB, int LDC, bool TB, bool UPPER>
-__device__ __forceinline__ void smem_gemm(real *C, const real *A, const real *B, real alpha,
-                                          real beta) {
-  static_assert(K % 4 == 0 && LDA % 4 == 0 && LDB % 4 == 0 && LDC % 4 == 0, "16-byte rows");
-  constexpr int RM = (M * N >= 16 * LT) ? 4 : 2;
-  constexpr int RN = (M * N >= 8 * LT) ? 4 : 2;
-  constexpr int TN = N / RN;
-  constexpr int NT = (M / RM) * TN;
-  for (int tile = threadIdx.x; tile < NT; tile += LT) {
-    const int i0 = (tile / TN) * RM, jt = tile % TN;
-    auto col = [&](int c) { return TB ? jt + TN * c : jt * RN + c; };
-    if (UPPER && col(RN - 1) < i0) continue;
-    real acc[RM][RN];
-#pragma unroll
-    for (int r = 0; r < RM; ++r)
-#pragma unroll
-      for (int c = 0; c < RN; ++c) acc[r][c] = 0.f;
+__device__ __forceinline__ void smem_gemm_tc(real *C, const real *A, const real *B, real alpha,
+                                             real beta) {
+  static_assert(M % 16 == 0 && N % 8 == 0 && K % 8 == 0, "m16n8k8 tiles");
+  constexpr int TN = N / 8, NT = (M / 16) * TN;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  for (int tile = warp; tile < NT; tile += LT / 32) {
+    const int i0 = (tile / TN) * 16, j0 = (tile % TN) * 8;
+    if (UPPER && j0 + 7 < i0) continue;   // wholly below the diagonal
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
-    for (int k = 0; k < K; k += 4) {
-      float4 a4[RM];
-#pragma unroll
-      for (int r = 0; r < RM; ++r) a4[r] = *reinterpret_cast<const float4 *>(A + (i0 + r) * LDA + k);
-      real a[RM][4];
-#pragma unroll
-      for (int r = 0; r < RM; ++r) {
-        a[r][0] = a4[r].x;
-        a[r][1] = a4[r].y;
-        a[r][2] = a4[r].z;
-        a[r][3] = a4[r].w;
-      }
-      real b[4][RN];
-      if (TB) {
-#pragma unroll
-        for (int c = 0; c < RN; ++c) {
-          const float4 v = *reinterpret_cast<const float4 *>(B + col(c) * LDB + k);
-          b[0][c] = v.x;
-          b[1][c] = v.y;
-          b[2][c] = v.z;
-          b[3][c] = v.w;
-        }
+    for (int k = 0; k < K; k += 8) {
+      const float a[4] = {A[(i0 + g) * LDA + k + t], A[(i0 + g + 8) * LDA + k + t],
+                          A[(i0 + g) * LDA + k + t + 4], A[(i0 + g + 8) * LDA + k + t + 4]};
+      float b[2];
+      if constexpr (TB) {
+        b[0] = B[(j0 + g) * LDB + k + t];
+        b[1] = B[(j0 + g) * LDB + k + t + 4];
       } else {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const real *br = B + (k + kk) * LDB + jt * RN;
-          if constexpr (RN == 4) {
-            const float4 v = *reinterpret_cast<const float4 *>(br);
-            b[kk][0] = v.x;
-            b[kk][1] = v.y;
-            b[kk][2] = v.z;
-            b[kk][3] = v.w;
-          } else {
-            const float2 v = *reinterpret_cast<const float2 *>(br);
-            b[kk][0] = v.x;
-            b[kk][1] = v.y;
-          }
-        }
+        b[0] = B[(k + t) * LDB + j0 + g];
+        b[1] = B[(k + t + 4) * LDB + j0 + g];
       }
+      uint32_t ah[4], al[4], bh[2], bl[2];
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
+      for (int q = 0; q < 4; ++q) split_tf32(a[q], ah[q], al[q]);
 #pragma unroll
-        for (int r = 0; r < RM; ++r)
-#pragma unroll
-          for (int c = 0; c < RN; ++c) acc[r][c] = fmaf(a[r][kk], b[kk][c], acc[r][c]);
+      for (int q = 0; q < 2; ++q) split_tf32(b[q], bh[q], bl[q]);
+      mma_tf32(acc, al, bh);
+      mma_tf32(acc, ah, bl);
+      mma_tf32(acc, ah, bh);
     }
 #pragma unroll
-    for (int r = 0; r < RM; ++r)
-#pragma unroll
-      for (int c = 0; c < RN; ++c) {
-        if (UPPER && col(c) < i0 + r) continue;
-        real *p = C + (i0 + r) * LDC + col(c);
-        *p = alpha * acc[r][c] + (beta != 0.f ? beta * *p : 0.f);
-      }
+    for (int q = 0; q < 4; ++q) {
+      const int row = i0 + g + (q >= 2 ? 8 : 0), col = j0 + 2 * t + (q & 1);
+      if (UPPER && col < row) continue;
+      real *p = C + row * LDC + col;
+      *p = alpha * acc[q] + (beta != 0.f ? beta * *p : 0.f);
+    }
   }
   __syncthreads();
 }
@@ -278,11 +268,11 @@ __device__ __forceinline__ bool node_factor(real *S, real *T, real *vbuf, int of
     // T (h x m): leading dimension m + 4, so rows stay 16-byte aligned and
     // the rows that neighbouring threads read transposed fall in different banks.
     constexpr int LT_ = m + 4;
-    smem_gemm<h, m, m, LLD, LLD, LT_, true, false>(T, A12, U22, 1.f, 0.f);    // R12 = A12 U22^T
-    smem_gemm<h, h, m, LT_, LT_, LLD, true, true>(A11, T, T, -1.f, 1.f);      // A11 -= R12 R12^T
-    smem_gemm<h, m, m, LT_, LLD, LLD, false, false>(A12, T, U22, 1.f, 0.f);   // A12 = R12 U22
+    smem_gemm_tc<h, m, m, LLD, LLD, LT_, true, false>(T, A12, U22, 1.f, 0.f);    // R12 = A12 U22^T
+    smem_gemm_tc<h, h, m, LT_, LT_, LLD, true, true>(A11, T, T, -1.f, 1.f);      // A11 -= R12 R12^T
+    smem_gemm_tc<h, m, m, LT_, LLD, LLD, false, false>(A12, T, U22, 1.f, 0.f);   // A12 = R12 U22
     if (!node_factor<h>(S, T, vbuf, off)) return false;
-    smem_gemm<h, m, h, LLD, LLD, LT_, false, false>(T, A11, A12, -1.f, 0.f);  // T = -U11 A12
+    smem_gemm_tc<h, m, h, LLD, LLD, LT_, false, false>(T, A11, A12, -1.f, 0.f);  // T = -U11 A12
     for (int idx = threadIdx.x; idx < h * m; idx += LT) {
       const int r = idx / m, c = idx - r * m;
       A12[r * LLD + c] = T[r * LT_ + c];
