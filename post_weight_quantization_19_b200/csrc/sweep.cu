@@ -18,6 +18,7 @@
 // it (the same value, so no divergence) and updates its 32 columns with
 // fused multiply-adds.  No inter-warp synchronisation at all.
 #include <float.h>
+#include <stdlib.h>
 
 #include "gptq_internal.h"
 #include "pack_bits.cuh"
@@ -25,9 +26,8 @@
 namespace gptq {
 namespace {
 
-constexpr int SWEEP_WARPS = 4;
-constexpr int SWEEP_THREADS = 32 * SWEEP_WARPS;
-constexpr int SWEEP_CW = 16;    // columns of a 128-column block held by one lane
+constexpr int SWEEP_WARPS = 4;   // warps per CTA (8 for the 16-lane form of the 128-column block)
+constexpr int SWEEP_CW = 16;     // columns of a 128-column block held by one lane
 
 __device__ __forceinline__ float warp_min(float v) {
 #pragma unroll
@@ -146,8 +146,9 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // With static groups under act-order (perm given) every column reads its own
 // group's fixed parameters: the groups of the original columns are scattered
 // over the sweep order.
-template <int CW, int L, bool VAR>
-__global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a) {
+template <int CW, int L, bool VAR, int WARPS>
+__global__ void __launch_bounds__(32 * WARPS) sweep_block_kernel(SweepArgs a) {
+  constexpr int SWEEP_THREADS = 32 * WARPS;
   constexpr int B = CW * L;
   constexpr int CHUNK = CW + 4;        // stride of one lane's part of a U row in shared
                                        // memory: the L parts start in different banks
@@ -205,8 +206,8 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
   const int nsub = nc / CW;       // 32-column parts present in this block
   const bool mine = ql < nsub;
 
-  for (int row0 = (blockIdx.x * SWEEP_WARPS + warp) * RPW; row0 < a.r;
-       row0 += gridDim.x * SWEEP_WARPS * RPW) {
+  for (int row0 = (blockIdx.x * WARPS + warp) * RPW; row0 < a.r;
+       row0 += gridDim.x * WARPS * RPW) {
     // Lanes of rows past the end keep going (zeros) so the shuffles stay whole.
     const int row = row0 + lane / L;
     const bool valid = row < a.r;
@@ -336,15 +337,21 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
         *reinterpret_cast<float4 *>(wp + c) = make_float4(w[c], w[c + 1], w[c + 2], w[c + 3]);
         *reinterpret_cast<float4 *>(ep + c) = make_float4(eo[c], eo[c + 1], eo[c + 2], eo[c + 3]);
       }
+      // 16 codes per 16-byte store (8 per 8-byte store when a lane holds 8 columns)
+      constexpr int CS = CW % 16 == 0 ? 16 : 8;
+      static_assert(CW % CS == 0, "codes per store");
 #pragma unroll
-      for (int c = 0; c < CW; c += 16) {
-        uint32_t wd[4];
+      for (int c = 0; c < CW; c += CS) {
+        uint32_t wd[CS / 4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
+        for (int k = 0; k < CS / 4; ++k)
           wd[k] = (uint32_t)(int)code[c + 4 * k] | ((uint32_t)(int)code[c + 4 * k + 1] << 8) |
                   ((uint32_t)(int)code[c + 4 * k + 2] << 16) |
                   ((uint32_t)(int)code[c + 4 * k + 3] << 24);
-        *reinterpret_cast<uint4 *>(cp + c) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        if constexpr (CS == 16)
+          *reinterpret_cast<uint4 *>(cp + c) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        else
+          *reinterpret_cast<uint2 *>(cp + c) = make_uint2(wd[0], wd[1]);
       }
     }
     if (ql == 0 && valid) a.loss_rows[row] = loss0 + 0.5 * (double)esq;
@@ -480,21 +487,31 @@ int launch_row_params(const float *Wsrc, int r, int d, int g, int bits, int sym,
   return GPTQ_OK;
 }
 
-template <int CW, int L, bool VAR>
+template <int CW, int L, bool VAR, int WARPS = SWEEP_WARPS>
 static int sweep_launch(const SweepArgs &a, cudaStream_t stream) {
   constexpr int B = CW * L;
   const size_t smem = (size_t)B * (CW + 4) * L * sizeof(float);
   static std::atomic<bool> attr[64] = {};
-  if (const int rc = ensure_smem_attr(sweep_block_kernel<CW, L, VAR>, smem, attr)) return rc;
+  if (const int rc = ensure_smem_attr(sweep_block_kernel<CW, L, VAR, WARPS>, smem, attr))
+    return rc;
   // Every row gets its lanes in one wave when the SMs can hold them (two CTAs
   // per SM: about 180 registers per thread).
-  const int rows_per_cta = SWEEP_WARPS * (32 / L);
+  const int rows_per_cta = WARPS * (32 / L);
   const int want = (a.r + rows_per_cta - 1) / rows_per_cta;
   const int cap = num_sms() * 2;
   const int grid = want < cap ? want : cap;
-  GPTQ_LAUNCH_PDL((sweep_block_kernel<CW, L, VAR>), dim3(grid), dim3(SWEEP_THREADS), smem,
+  GPTQ_LAUNCH_PDL((sweep_block_kernel<CW, L, VAR, WARPS>), dim3(grid), dim3(32 * WARPS), smem,
                   stream, a);
   return GPTQ_OK;
+}
+
+// GPTQ_SWEEP_LANES=16 selects the 16-lane form of the 128-column block (read once).
+static bool sweep_lanes16() {
+  static const bool on = [] {
+    const char *v = getenv("GPTQ_SWEEP_LANES");
+    return v && v[0] == '1' && v[1] == '6' && v[2] == 0;
+  }();
+  return on;
 }
 
 template <bool VAR>
@@ -502,7 +519,12 @@ static int sweep_launch_block(const SweepArgs &a, int block, cudaStream_t stream
   switch (block) {
     case 32: return sweep_launch<32, 1, VAR>(a, stream);
     case 64: return sweep_launch<32, 2, VAR>(a, stream);
-    case 128: return sweep_launch<SWEEP_CW, 128 / SWEEP_CW, VAR>(a, stream);
+    case 128:
+      // Experimental form under measurement: 16 lanes of 8 columns per row in
+      // CTAs of 8 warps (twice the warps per SM for the same rows).
+      if (sweep_lanes16())
+        return sweep_launch<8, 16, VAR, 8>(a, stream);
+      return sweep_launch<SWEEP_CW, 128 / SWEEP_CW, VAR>(a, stream);
     default: return GPTQ_ERR_INVALID_ARG;
   }
 }
