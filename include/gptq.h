@@ -72,12 +72,33 @@ int gptq_hessian_accumulate(const void *X, int64_t n, int64_t d, int64_t ldx, fl
                             gptq_stream_t stream);
 
 /*
+ * Options of the layer solve: a bit field, 0 for the plain solve.  Unknown bits
+ * are invalid arguments.
+ *   GPTQ_ACT_ORDER      quantise columns in order of descending diag(H)
+ *                       ([Explainer] §三, desc_act).
+ *   GPTQ_SYMMETRIC      the symmetric quantiser ("LLM 量化技术" §1.2): zero point 0,
+ *                       s = max|x| / (2^(bits-1) - 1) over the group (1 for an
+ *                       all-zero group), signed codes in [-2^(bits-1),
+ *                       2^(bits-1) - 1] stored as code + 2^(bits-1) (so every
+ *                       zero point is 2^(bits-1)).
+ *   GPTQ_STATIC_GROUPS  each group's parameters come from the original W over
+ *                       the layer's own column groups [k*group, (k+1)*group),
+ *                       fixed before the sweep, instead of from the compensated
+ *                       W when the sweep reaches the group; under act-order the
+ *                       groups stay contiguous, g_idx[c] = c / group.  No effect
+ *                       with group = -1.
+ */
+#define GPTQ_ACT_ORDER 1
+#define GPTQ_SYMMETRIC 2
+#define GPTQ_STATIC_GROUPS 4
+
+/*
  * gptq_quantize_workspace_bytes -- device workspace needed by gptq_quantize_layer
  * for these arguments (0 if the arguments are invalid).  The workspace must be
  * 256-byte aligned.
  */
 size_t gptq_quantize_workspace_bytes(int64_t r, int64_t d, int bits, int group, int block,
-                                     int act_order);
+                                     int options);
 
 /*
  * gptq_quantize_layer -- GPTQ solve of one linear layer
@@ -85,14 +106,15 @@ size_t gptq_quantize_workspace_bytes(int64_t r, int64_t d, int bits, int group, 
  *
  * Steps, all on the GPU in stream order:
  *   1. lambda = damp * mean(diag H); H_d = H + lambda I.
- *   2. act_order != 0: perm = stable argsort of -diag(H) (ties keep the lower
+ *   2. GPTQ_ACT_ORDER: perm = stable argsort of -diag(H) (ties keep the lower
  *      index); columns of W and rows/columns of H_d are taken in that order.
  *   3. U = upper Cholesky factor of H_d^-1 (U^T U = H_d^-1), computed as the
  *      "reverse" Cholesky H_d = R R^T (R upper) and U = R^-1.
  *   4. For j = 0..d-1 in blocks of `block` columns: at a group start, per-row
  *      s = (xmax - xmin)/(2^bits - 1) and z = rint(-xmin/s) over the current
  *      group columns (xmin <= 0 <= xmax; s = 1 if the range is empty); for
- *      group = -1 once per row from the original W.  q = clamp(rint(w_j/s) + z,
+ *      group = -1 once per row from the original W (GPTQ_SYMMETRIC and
+ *      GPTQ_STATIC_GROUPS change these parameters, see above).  q = clamp(rint(w_j/s) + z,
  *      0, 2^bits - 1), w^_j = s (q - z), e_j = (w_j - w^_j)/U_jj, and the
  *      later columns of the block move by -e_j U[j, j+1:].  Later blocks are
  *      moved once per block (lazy batch) or once per 1024 columns, an exact
@@ -107,14 +129,15 @@ size_t gptq_quantize_workspace_bytes(int64_t r, int64_t d, int bits, int group, 
  *             d > 0, d % 32 == 0.
  *   H         device fp32 [d x d], full symmetric (as written by
  *             gptq_hessian_accumulate).  CONSUMED: overwritten with the
- *             factorisation (U in the upper triangle when act_order == 0; the
- *             contents are unspecified when act_order != 0).
+ *             factorisation (U in the upper triangle without GPTQ_ACT_ORDER;
+ *             the contents are unspecified with it).
  *   bits      2, 3, 4 or 8.
  *   group     -1 (one scale/zero per row) or a multiple of 32 that divides d
  *             with block % group == 0 or group % block == 0.
  *   block     32, 64 or 128 (the lazy-batch width B; the pages use 128).
  *   damp      relative damping >= 0 (the pages' "mild damping"; 0.01 typical).
- *   act_order 0 or 1.
+ *   options   0 or a combination of GPTQ_ACT_ORDER, GPTQ_SYMMETRIC and
+ *             GPTQ_STATIC_GROUPS.
  *   W_hat     device fp32 [r x d] or NULL: dequantised weights s(q - z) in the
  *             original column order.  May alias W.
  *   qweight   device int32 [r x d*bits/32]: per row, the codes of columns
@@ -122,7 +145,8 @@ size_t gptq_quantize_workspace_bytes(int64_t r, int64_t d, int bits, int group, 
  *             [c*bits, (c+1)*bits), stream bit k = bit k%32 of word k/32).
  *   scales    device fp32 [r x G], G = d/group (G = 1 for group = -1).
  *             Column k belongs to quantisation group k (permuted positions
- *             [k*group, (k+1)*group) under act-order).
+ *             [k*group, (k+1)*group) under act-order; original columns
+ *             [k*group, (k+1)*group) with GPTQ_STATIC_GROUPS).
  *   zeros     device int32 [r x G], integer zero points in [0, 2^bits - 1].
  *   g_idx     device int32 [d] or NULL: group of each original column.
  *   codes     device uint8 [r x d] or NULL: unpacked codes, original order.
@@ -134,10 +158,52 @@ size_t gptq_quantize_workspace_bytes(int64_t r, int64_t d, int bits, int group, 
  *   are then unspecified), GPTQ_ERR_NO_MEMORY if workspace_bytes is too small.
  */
 int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int group,
-                        int block, float damp, int act_order, float *W_hat, int32_t *qweight,
+                        int block, float damp, int options, float *W_hat, int32_t *qweight,
                         float *scales, int32_t *zeros, int32_t *g_idx, uint8_t *codes,
                         double *loss, void *workspace, size_t workspace_bytes,
                         gptq_stream_t stream);
+
+/*
+ * gptq_factor / gptq_quantize_with_factor -- the solve in two halves, so that
+ * one factor serves several sweeps: rows of one layer spread over several
+ * GPUs, or several layers that read the same inputs and so share H.  The
+ * inverse-Hessian information does not depend on W ([Card] 方法适配: every row
+ * is quantised in the same order with the same factor).
+ *
+ * gptq_factor: steps 1-3 of gptq_quantize_layer.
+ *   H        device fp32 [d x d], full symmetric, 16-byte aligned.  On return
+ *            its upper triangle holds U in sweep order (the factor of the
+ *            permuted H_d under GPTQ_ACT_ORDER); the strictly lower triangle is
+ *            scratch.
+ *   options  GPTQ_ACT_ORDER is used; the other bits are accepted and ignored.
+ *   perm     device int32 [d] (GPTQ_ACT_ORDER; may be NULL otherwise): column
+ *            perm[j] of W is quantised j-th.
+ *   lambda   device fp32 [1]: the damping added to the diagonal (the loss
+ *            needs it).
+ *   workspace  gptq_factor_workspace_bytes(d, options) bytes, 256-byte aligned.
+ *   Synchronises `stream` once, at the end; returns GPTQ_ERR_NOT_PD if H_d is
+ *   not positive definite.
+ *
+ * gptq_quantize_with_factor: steps 4-6 of gptq_quantize_layer from a factor
+ *   made by gptq_factor with the same d and GPTQ_ACT_ORDER bit (U, perm and
+ *   lambda are read only, so they can serve any number of calls).  Other
+ *   arguments as gptq_quantize_layer; the workspace is
+ *   gptq_quantize_with_factor_workspace_bytes(r, d, bits, group, block) bytes.
+ *   A perm that is not a permutation of 0..d-1 is found on the device before
+ *   anything uses it and returns GPTQ_ERR_INVALID_ARG (outputs unspecified).
+ *   Synchronises `stream` once, at the end, to read the status and the loss.
+ */
+size_t gptq_factor_workspace_bytes(int64_t d, int options);
+int gptq_factor(float *H, int64_t d, float damp, int options, int32_t *perm, float *lambda,
+                void *workspace, size_t workspace_bytes, gptq_stream_t stream);
+size_t gptq_quantize_with_factor_workspace_bytes(int64_t r, int64_t d, int bits, int group,
+                                                 int block);
+int gptq_quantize_with_factor(const float *W, int64_t r, int64_t d, const float *U,
+                              const int32_t *perm, const float *lambda, int bits, int group,
+                              int block, int options, float *W_hat, int32_t *qweight,
+                              float *scales, int32_t *zeros, int32_t *g_idx, uint8_t *codes,
+                              double *loss, void *workspace, size_t workspace_bytes,
+                              gptq_stream_t stream);
 
 /*
  * gptq_pack -- pack codes into int32 words   ([Explainer] §三, int32 storage of 3/4-bit codes)
@@ -177,6 +243,32 @@ int gptq_dequant_gemv(const int32_t *qweight, const float *scales, const int32_t
                       const float *x, int64_t m, float *y, gptq_stream_t stream);
 
 /*
+ * gptq_dequant_fp16 / gptq_linear_fp16 -- run a quantised layer forward on
+ * calibration tokens, to calibrate the next layer on what this one outputs
+ *   ([Card] §计算设置: each block is quantised, then run to produce the next
+ *   block's inputs; [Concept] §3 技術原理: the codes are dequantised to FP16
+ *   and multiplied in floating point)
+ *
+ * gptq_dequant_fp16: W16[row, c] = fp16(scales[row, gi(c)] * (q[row, c] -
+ *   zeros[row, gi(c)])) from the packed layer (arguments as gptq_dequant_gemv;
+ *   W16 device fp16 [r x d], 16-byte aligned, written).  Asynchronous.
+ * gptq_linear_fp16: Y = fp16(X W16^T) -- X device fp16 [n x d] (tokens x
+ *   features), W16 device fp16 [r x d], Y device fp16 [n x r], all row-major and
+ *   16-byte aligned; d % 32 == 0, r % 32 == 0.  fp32 accumulation on the tensor
+ *   cores, folded every 512 features, one rounding to fp16 per output (values
+ *   beyond the fp16 range become +-inf).  n == 0 or r == 0: nothing to do.
+ *   Asynchronous; a bounded in-kernel wait that runs out is reported by
+ *   gptq_check_device_status.
+ * Both return GPTQ_ERR_INVALID_ARG before launching anything when an argument
+ * is out of range.
+ */
+int gptq_dequant_fp16(const int32_t *qweight, const float *scales, const int32_t *zeros,
+                      const int32_t *g_idx, int64_t r, int64_t d, int bits, int group, void *W16,
+                      gptq_stream_t stream);
+int gptq_linear_fp16(const void *X, int64_t n, int64_t d, const void *W16, int64_t r, void *Y,
+                     gptq_stream_t stream);
+
+/*
  * gptq_quantize_layer_noalloc -- gptq_quantize_layer for callers that cannot
  * allocate device memory.  (The GPTQ pages have no counterpart: this is a
  * deployment convenience of this library, not a step of the method.)
@@ -192,7 +284,7 @@ int gptq_dequant_gemv(const int32_t *qweight, const float *scales, const int32_t
  *   Arguments, results and synchronisation are those of gptq_quantize_layer
  *   without the workspace pair.
  *   Limit: returns GPTQ_ERR_NO_MEMORY (nothing enqueued) when
- *   gptq_quantize_workspace_bytes(r, d, bits, group, block, act_order) exceeds
+ *   gptq_quantize_workspace_bytes(r, d, bits, group, block, options) exceeds
  *   GPTQ_NOALLOC_SCRATCH_BYTES -- e.g. r = d = 2048 fits, r = d = 4096 does not.
  *   The first call on a device looks up the array's device address (once per
  *   device, with that device current); make that first call before any stream
@@ -203,7 +295,7 @@ int gptq_dequant_gemv(const int32_t *qweight, const float *scales, const int32_t
  */
 #define GPTQ_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 int gptq_quantize_layer_noalloc(const float *W, int64_t r, int64_t d, float *H, int bits,
-                                int group, int block, float damp, int act_order, float *W_hat,
+                                int group, int block, float damp, int options, float *W_hat,
                                 int32_t *qweight, float *scales, int32_t *zeros, int32_t *g_idx,
                                 uint8_t *codes, double *loss, gptq_stream_t stream);
 
@@ -226,9 +318,9 @@ int gptq_quantize_layer_noalloc(const float *W, int64_t r, int64_t d, float *H, 
  *   Synchronous: returns when the outputs are in the host buffers.
  */
 size_t gptq_layer_host_workspace_bytes(int64_t r, int64_t d, int64_t n, int bits, int group,
-                                       int block, int act_order);
+                                       int block, int options);
 int gptq_solve_layer_host(const uint16_t *X_host, int64_t n, const float *W_host, int64_t r,
-                          int64_t d, int bits, int group, int block, float damp, int act_order,
+                          int64_t d, int bits, int group, int block, float damp, int options,
                           int32_t *qweight_host, float *scales_host, int32_t *zeros_host,
                           int32_t *g_idx_host, double *loss, void *dev_workspace,
                           size_t dev_workspace_bytes, gptq_stream_t stream);

@@ -14,11 +14,16 @@ from .gptq import (  # noqa: F401
     gptq_last_phase_ms,
     gptq_launch_count,
     gptq_layer_host_workspace_bytes,
+    gptq_dequant_fp16,
     gptq_dequant_gemv,
+    gptq_factor,
+    gptq_linear_fp16,
     gptq_pack,
     gptq_quantize_layer,
+    gptq_quantize_with_factor,
     gptq_quantize_workspace_bytes,
     gptq_set_phase_timing,
     gptq_solve_layer_host,
 )
 from .sharded import row_shard, shard_range, solve_layer_sharded, token_shard  # noqa: F401
+from .chain import quantize_chain  # noqa: F401

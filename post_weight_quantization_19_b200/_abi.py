@@ -29,9 +29,21 @@ SIGNATURES = {
     "gptq_quantize_layer": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int, c_int, c_int,
                                     c_float, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "gptq_factor_workspace_bytes": (c_size_t, [c_int64, c_int]),
+    "gptq_factor": (c_int, [c_void_p, c_int64, c_float, c_int, c_void_p, c_void_p, c_void_p,
+                            c_size_t, c_void_p]),
+    "gptq_quantize_with_factor_workspace_bytes": (c_size_t, [c_int64, c_int64, c_int, c_int,
+                                                             c_int]),
+    "gptq_quantize_with_factor": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_void_p,
+                                          c_void_p, c_int, c_int, c_int, c_int, c_void_p,
+                                          c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                          c_void_p, c_void_p, c_size_t, c_void_p]),
     "gptq_pack": (c_int, [c_void_p, c_int64, c_int64, c_int, c_void_p, c_void_p]),
     "gptq_dequant_gemv": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int,
                                   c_int, c_void_p, c_int64, c_void_p, c_void_p]),
+    "gptq_dequant_fp16": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int,
+                                  c_int, c_void_p, c_void_p]),
+    "gptq_linear_fp16": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int64, c_void_p, c_void_p]),
     "gptq_quantize_layer_noalloc": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int, c_int,
                                             c_int, c_float, c_int, c_void_p, c_void_p, c_void_p,
                                             c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),

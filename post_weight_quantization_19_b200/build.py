@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgptq_b200.so")
 SOURCES = ["hessian_tc.cu", "gemm_tc.cu", "factor.cu", "leaf.cu", "sweep.cu", "pack.cu", "api.cu",
-           "noalloc.cu", "gemv.cu"]
+           "noalloc.cu", "gemv.cu", "linear_tc.cu"]
 
 
 def nvcc() -> str:

@@ -33,6 +33,10 @@ constexpr int kSuperblock = 1024;  // columns per global (deferred) trailing upd
 
 bool valid_bits(int b) { return b == 2 || b == 3 || b == 4 || b == 8; }
 
+bool valid_options(int options) {
+  return (options & ~(GPTQ_ACT_ORDER | GPTQ_SYMMETRIC | GPTQ_STATIC_GROUPS)) == 0;
+}
+
 bool valid_layer(int64_t r, int64_t d, int bits, int group, int block) {
   if (r < 0 || r > (int64_t)INT32_MAX / 2) return false;
   if (d <= 0 || d % 32 != 0 || d > 65536) return false;
@@ -60,7 +64,7 @@ struct Layout {
   size_t Wk, ErrS, codes_p, perm, inv, Hp, T1, loss_rows, dsq_rows, out, lambda, status, total;
 };
 
-Layout layout(int64_t r, int64_t d, int group, int block, int act_order) {
+Layout layout(int64_t r, int64_t d, int group, int block, int options) {
   Layout L{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -74,7 +78,7 @@ Layout layout(int64_t r, int64_t d, int group, int block, int act_order) {
   L.codes_p = take((size_t)r * d);
   L.perm = take((size_t)d * 4);
   L.inv = take((size_t)d * 4);
-  L.Hp = take(act_order ? (size_t)d * d * 4 : 0);
+  L.Hp = take((options & GPTQ_ACT_ORDER) ? (size_t)d * d * 4 : 0);
   L.T1 = take(factor_scratch_floats(d) * 4);
   L.loss_rows = take((size_t)r * 8);
   L.dsq_rows = take((size_t)r * 8);
@@ -106,14 +110,14 @@ struct GraphKey {
   int64_t r, d;
   int bits, group, block;
   float damp;
-  int act_order;
+  int options;
   int device = -1;
   bool operator==(const GraphKey &o) const {
     return W == o.W && H == o.H && W_hat == o.W_hat && qweight == o.qweight &&
            scales == o.scales && zeros == o.zeros && g_idx == o.g_idx && codes == o.codes &&
            ws == o.ws && ws_bytes == o.ws_bytes && stream == o.stream && r == o.r &&
            d == o.d && bits == o.bits && group == o.group && block == o.block &&
-           memcmp(&damp, &o.damp, sizeof(float)) == 0 && act_order == o.act_order &&
+           memcmp(&damp, &o.damp, sizeof(float)) == 0 && options == o.options &&
            device == o.device;
   }
 };
@@ -235,20 +239,145 @@ extern "C" int gptq_check_device_status(gptq_stream_t stream) {
 }
 
 extern "C" size_t gptq_quantize_workspace_bytes(int64_t r, int64_t d, int bits, int group,
-                                                int block, int act_order) {
-  if (!valid_layer(r, d, bits, group, block)) return 0;
-  return layout(r, d, group, block, act_order).total;
+                                                int block, int options) {
+  if (!valid_layer(r, d, bits, group, block) || !valid_options(options)) return 0;
+  return layout(r, d, group, block, options).total;
 }
 
 namespace gptq {
+namespace {
+
+// Phases 0-1 on `st`: lambda = damp * mean(diag H), the act-order permutation
+// (perm, inv and the permuted H_d in Hp), then U in place of H_d.  *U is set to
+// the matrix that holds U (H, or Hp under act-order).
+int enqueue_factor(float *H, int64_t d, float damp, bool act_order, int *perm, int *inv,
+                   float *lambda, float *Hp, float *T1, int *status, cudaStream_t st,
+                   bool use_side, float **U) {
+  const int di = (int)d;
+  float *Hf = H;
+  if (act_order) {
+    GPTQ_TRY(launch_damp(H, d, di, damp, false, lambda, st));
+    GPTQ_TRY(launch_act_order(H, d, di, perm, inv, lambda, Hp, st));
+    Hf = Hp;
+  } else {
+    GPTQ_TRY(launch_damp(H, d, di, damp, true, lambda, st));
+  }
+  GPTQ_TRY(record(1, st));
+  GPTQ_TRY(launch_factor(Hf, d, T1, status, st, use_side));
+  GPTQ_TRY(record(2, st));
+  *U = Hf;
+  return GPTQ_OK;
+}
+
+// Everything the sweep half needs: inputs, outputs and its part of the workspace.
+struct SweepPlan {
+  const float *W;
+  int r, d, bits, group, block, sym, static_groups;
+  const float *U;
+  const int *perm, *inv;   // act-order only (NULL otherwise)
+  const float *lambda;
+  float *W_hat;
+  int32_t *qweight;
+  float *scales;
+  int32_t *zeros;
+  int32_t *g_idx;
+  uint8_t *codes;
+  float *Wk, *ErrS;
+  uint8_t *codes_p;
+  double *loss_rows, *dsq_rows, *out;
+  int *status;
+};
+
+// Phases 2-3 on `st`: working copy of W, column sweep in blocks with lazy
+// trailing updates, then unpermute, loss and packing.  The sweep kernels read
+// their U block before waiting for their predecessor, so the kernel just
+// before each of them must not write U: the copy of W separates the
+// factorisation from the first block.
+int enqueue_sweep(const SweepPlan &p, cudaStream_t st) {
+  const int ri = p.r, di = p.d, group = p.group, block = p.block;
+  const int G = group < 0 ? 1 : di / group;
+  const int S = superblock(p.d, group, block);
+  GPTQ_TRY(launch_gather_w(p.W, ri, di, p.perm, p.Wk, p.status, st));
+  if (group < 0)
+    GPTQ_TRY(launch_row_params(p.Wk, ri, di, di, p.bits, p.sym, p.scales, p.zeros, p.status, st));
+  if (p.static_groups)
+    GPTQ_TRY(launch_row_params(p.W, ri, di, group, p.bits, p.sym, p.scales, p.zeros, p.status, st));
+  for (int s0 = 0; s0 < di; s0 += S) {
+    const int sEnd = s0 + S < di ? s0 + S : di;
+    for (int j0 = s0; j0 < sEnd; j0 += block) {
+      const int j1 = j0 + block < sEnd ? j0 + block : sEnd;
+      SweepArgs a{};
+      a.Wk = p.Wk;
+      a.ldw = di;
+      a.U = p.U;
+      a.ldu = di;
+      a.r = ri;
+      a.j0 = j0;
+      a.ncols = j1 - j0;
+      a.bits = p.bits;
+      a.group = group;
+      a.scales = p.scales;
+      a.zeros = p.zeros;
+      a.G = G;
+      a.flags = (p.sym ? SWEEP_SYM : 0) | (p.static_groups ? SWEEP_STATIC : 0);
+      a.codes = p.codes_p;
+      a.perm = p.static_groups && p.perm ? p.perm : nullptr;
+      a.err = p.ErrS + (j0 - s0);
+      a.lde = S;
+      a.loss_rows = p.loss_rows;
+      a.status = p.status;
+      GPTQ_TRY(launch_sweep_block(a, block, st));
+      if (j1 < sEnd) {
+        // Rest of this superblock: W[:, j1:sEnd] -= E_blk U[j0:j1, j1:sEnd]
+        GemmArgs g{ri, sEnd - j1, j1 - j0, p.ErrS + (j0 - s0), S, p.U + (size_t)j0 * di + j1, di,
+                   p.Wk + j1, di, -1.f, 1.f, 0, p.status};
+        GPTQ_TRY(launch_gemm(g, false, st));
+      }
+    }
+    if (sEnd < di) {
+      // Deferred global update: W[:, sEnd:] -= E_S U[s0:sEnd, sEnd:]
+      GemmArgs g{ri, di - sEnd, sEnd - s0, p.ErrS, S, p.U + (size_t)s0 * di + sEnd, di,
+                 p.Wk + sEnd, di, -1.f, 1.f, 0, p.status};
+      GPTQ_TRY(launch_gemm(g, false, st));
+    }
+  }
+  GPTQ_TRY(record(3, st));
+
+  FinalizeArgs f{};
+  f.W = p.W;
+  f.Wk = p.Wk;
+  f.codes_p = p.codes_p;
+  f.inv = p.inv;
+  f.r = ri;
+  f.d = di;
+  f.bits = p.bits;
+  f.group = group;
+  f.static_groups = p.static_groups;
+  f.W_hat = p.W_hat;
+  f.codes = p.codes;
+  f.qweight = p.qweight;
+  f.g_idx = p.g_idx;
+  f.dsq_rows = p.dsq_rows;
+  f.status = p.status;
+  GPTQ_TRY(launch_finalize(f, st));
+  GPTQ_TRY(launch_loss_reduce(p.loss_rows, p.dsq_rows, ri, p.lambda, p.out, p.status, st));
+  GPTQ_TRY(record(4, st));
+  return GPTQ_OK;
+}
+
+}  // namespace
 
 int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int group, int block,
-                   float damp, int act_order, float *W_hat, int32_t *qweight, float *scales,
+                   float damp, int options, float *W_hat, int32_t *qweight, float *scales,
                    int32_t *zeros, int32_t *g_idx, uint8_t *codes, double *loss, void *workspace,
                    size_t workspace_bytes, gptq_stream_t stream, bool plain) {
   if (!valid_layer(r, d, bits, group, block)) return GPTQ_ERR_INVALID_ARG;
   if (!(damp >= 0.f) || damp > 1e30f) return GPTQ_ERR_INVALID_ARG;
-  if (act_order != 0 && act_order != 1) return GPTQ_ERR_INVALID_ARG;
+  if (!valid_options(options)) return GPTQ_ERR_INVALID_ARG;
+  const bool act_order = (options & GPTQ_ACT_ORDER) != 0;
+  const int sym = (options & GPTQ_SYMMETRIC) ? 1 : 0;
+  // with one group per row both rules take the parameters from the original row
+  const int static_groups = (options & GPTQ_STATIC_GROUPS) && group > 0 ? 1 : 0;
   if (r == 0) {
     if (loss) *loss = 0.0;
     return GPTQ_OK;
@@ -261,7 +390,7 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
       reinterpret_cast<uintptr_t>(zeros) % 4 || (g_idx && reinterpret_cast<uintptr_t>(g_idx) % 16) ||
       (codes && reinterpret_cast<uintptr_t>(codes) % 4))
     return GPTQ_ERR_INVALID_ARG;
-  const Layout L = layout(r, d, group, block, act_order);
+  const Layout L = layout(r, d, group, block, options);
   if (workspace_bytes < L.total) return GPTQ_ERR_NO_MEMORY;
 
   cudaStream_t st = (cudaStream_t)stream;
@@ -279,95 +408,20 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
   float *lambda = reinterpret_cast<float *>(ws + L.lambda);
   int *status = reinterpret_cast<int *>(ws + L.status);
   const int ri = (int)r, di = (int)d;
-  const int G = group < 0 ? 1 : di / group;
-  const int S = superblock(d, group, block);
 
   auto enqueue = [&]() -> int {
     GPTQ_TRY(record(0, st));
     GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 16, st));
     GPTQ_CUDA_TRY(cudaMemsetAsync(loss_rows, 0, (size_t)r * 8, st));
 
-    // Phase 0: damping and act-order.
-    float *Hf = H;
-    if (act_order) {
-      GPTQ_TRY(launch_damp(H, d, di, damp, false, lambda, st));
-      GPTQ_TRY(launch_act_order(H, d, di, perm, inv, lambda, Hp, st));
-      Hf = Hp;
-    } else {
-      GPTQ_TRY(launch_damp(H, d, di, damp, true, lambda, st));
-    }
-    GPTQ_TRY(record(1, st));
-
-    // Phase 1: U = upper Cholesky factor of H_d^-1, in place.
-    GPTQ_TRY(launch_factor(Hf, d, T1, status, st, !plain));
-    GPTQ_TRY(record(2, st));
-
-    // Phase 2: working copy of W, column sweep in blocks, lazy trailing
-    // updates.  The sweep kernels read their U block before waiting for their
-    // predecessor, so the kernel just before each of them must not write U:
-    // the copy of W separates the factorisation from the first block.
-    GPTQ_TRY(launch_gather_w(W, ri, di, act_order ? perm : nullptr, Wk, status, st));
-    if (group < 0) GPTQ_TRY(launch_row_params(Wk, ri, di, bits, scales, zeros, status, st));
-    for (int s0 = 0; s0 < di; s0 += S) {
-      const int sEnd = s0 + S < di ? s0 + S : di;
-      for (int j0 = s0; j0 < sEnd; j0 += block) {
-        const int j1 = j0 + block < sEnd ? j0 + block : sEnd;
-        SweepArgs a{};
-        a.Wk = Wk;
-        a.ldw = d;
-        a.U = Hf;
-        a.ldu = d;
-        a.r = ri;
-        a.j0 = j0;
-        a.ncols = j1 - j0;
-        a.bits = bits;
-        a.group = group;
-        a.scales = scales;
-        a.zeros = zeros;
-        a.G = G;
-        a.codes = codes_p;
-        a.ldc = d;
-        a.err = ErrS + (j0 - s0);
-        a.lde = S;
-        a.loss_rows = loss_rows;
-        a.status = status;
-        GPTQ_TRY(launch_sweep_block(a, block, st));
-        if (j1 < sEnd) {
-          // Rest of this superblock: W[:, j1:sEnd] -= E_blk U[j0:j1, j1:sEnd]
-          GemmArgs g{ri, sEnd - j1, j1 - j0, ErrS + (j0 - s0), S, Hf + (size_t)j0 * d + j1, d,
-                     Wk + j1, d, -1.f, 1.f, 0, status};
-          GPTQ_TRY(launch_gemm(g, false, st));
-        }
-      }
-      if (sEnd < di) {
-        // Deferred global update: W[:, sEnd:] -= E_S U[s0:sEnd, sEnd:]
-        GemmArgs g{ri, di - sEnd, sEnd - s0, ErrS, S, Hf + (size_t)s0 * d + sEnd, d, Wk + sEnd, d,
-                   -1.f, 1.f, 0, status};
-        GPTQ_TRY(launch_gemm(g, false, st));
-      }
-    }
-    GPTQ_TRY(record(3, st));
-
-    // Phase 3: unpermute, loss, packing.
-    FinalizeArgs f{};
-    f.W = W;
-    f.Wk = Wk;
-    f.codes_p = codes_p;
-    f.inv = act_order ? inv : nullptr;
-    f.r = ri;
-    f.d = di;
-    f.bits = bits;
-    f.group = group;
-    f.W_hat = W_hat;
-    f.codes = codes;
-    f.qweight = qweight;
-    f.g_idx = g_idx;
-    f.dsq_rows = dsq_rows;
-    f.status = status;
-    GPTQ_TRY(launch_finalize(f, st));
-    GPTQ_TRY(launch_loss_reduce(loss_rows, dsq_rows, ri, lambda, out, status, st));
-    GPTQ_TRY(record(4, st));
-    return GPTQ_OK;
+    float *U = nullptr;
+    GPTQ_TRY(enqueue_factor(H, d, damp, act_order, perm, inv, lambda, Hp, T1, status, st, !plain,
+                            &U));
+    const SweepPlan sp{W, ri, di, bits, group, block, sym, static_groups, U,
+                       act_order ? perm : nullptr, act_order ? inv : nullptr, lambda, W_hat,
+                       qweight, scales, zeros, g_idx, codes, Wk, ErrS, codes_p, loss_rows,
+                       dsq_rows, out, status};
+    return enqueue_sweep(sp, st);
   };
 
   // Replay the whole kernel sequence as a CUDA graph when the same call
@@ -376,7 +430,7 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
   // first call of a configuration runs directly, the second is captured, later
   // ones replay.  Streams that cannot be captured run directly.
   const GraphKey key{W, H, W_hat, qweight, scales, zeros, g_idx, codes, workspace,
-                     workspace_bytes, st, r, d, bits, group, block, damp, act_order};
+                     workspace_bytes, st, r, d, bits, group, block, damp, options};
   int rc = GPTQ_OK;
   if (g_timing || plain) {
     rc = enqueue();
@@ -400,13 +454,164 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
 }  // namespace gptq
 
 extern "C" int gptq_quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits,
-                                   int group, int block, float damp, int act_order, float *W_hat,
+                                   int group, int block, float damp, int options, float *W_hat,
                                    int32_t *qweight, float *scales, int32_t *zeros,
                                    int32_t *g_idx, uint8_t *codes, double *loss, void *workspace,
                                    size_t workspace_bytes, gptq_stream_t stream) {
-  return gptq::quantize_layer(W, r, d, H, bits, group, block, damp, act_order, W_hat, qweight,
+  return gptq::quantize_layer(W, r, d, H, bits, group, block, damp, options, W_hat, qweight,
                               scales, zeros, g_idx, codes, loss, workspace, workspace_bytes,
                               stream, false);
+}
+
+// ------------------------------------------------------- factor once, sweep many
+
+namespace {
+
+struct FactorLayout {
+  size_t inv, Hp, T1, status, total;
+};
+
+FactorLayout factor_layout(int64_t d, int options) {
+  FactorLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  L.inv = take((size_t)d * 4);
+  L.Hp = take((options & GPTQ_ACT_ORDER) ? (size_t)d * d * 4 : 0);
+  L.T1 = take(factor_scratch_floats(d) * 4);
+  L.status = take(16);
+  L.total = off;
+  return L;
+}
+
+struct SweepLayout {
+  size_t Wk, ErrS, codes_p, inv, loss_rows, dsq_rows, out, status, total;
+};
+
+SweepLayout sweep_layout(int64_t r, int64_t d, int group, int block) {
+  SweepLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  const int S = superblock(d, group, block);
+  L.Wk = take((size_t)r * d * 4);
+  L.ErrS = take((size_t)r * S * 4);
+  L.codes_p = take((size_t)r * d);
+  L.inv = take((size_t)d * 4);
+  L.loss_rows = take((size_t)r * 8);
+  L.dsq_rows = take((size_t)r * 8);
+  L.out = take(4 * 8);
+  L.status = take(16);
+  L.total = off;
+  return L;
+}
+
+bool valid_d(int64_t d) { return d > 0 && d % 32 == 0 && d <= 65536; }
+
+}  // namespace
+
+extern "C" size_t gptq_factor_workspace_bytes(int64_t d, int options) {
+  if (!valid_d(d) || !valid_options(options)) return 0;
+  return factor_layout(d, options).total;
+}
+
+extern "C" int gptq_factor(float *H, int64_t d, float damp, int options, int32_t *perm,
+                           float *lambda, void *workspace, size_t workspace_bytes,
+                           gptq_stream_t stream) {
+  if (!valid_d(d) || !valid_options(options)) return GPTQ_ERR_INVALID_ARG;
+  if (!(damp >= 0.f) || damp > 1e30f) return GPTQ_ERR_INVALID_ARG;
+  const bool act_order = (options & GPTQ_ACT_ORDER) != 0;
+  if (!H || !lambda || !workspace || (act_order && !perm)) return GPTQ_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(H) % 16 || reinterpret_cast<uintptr_t>(lambda) % 4 ||
+      reinterpret_cast<uintptr_t>(workspace) % 256 ||
+      (perm && reinterpret_cast<uintptr_t>(perm) % 4))
+    return GPTQ_ERR_INVALID_ARG;
+  const FactorLayout L = factor_layout(d, options);
+  if (workspace_bytes < L.total) return GPTQ_ERR_NO_MEMORY;
+  cudaStream_t st = (cudaStream_t)stream;
+  char *ws = static_cast<char *>(workspace);
+  int *inv = reinterpret_cast<int *>(ws + L.inv);
+  float *Hp = reinterpret_cast<float *>(ws + L.Hp);
+  float *T1 = reinterpret_cast<float *>(ws + L.T1);
+  int *status = reinterpret_cast<int *>(ws + L.status);
+  GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 16, st));
+  float *U = nullptr;
+  GPTQ_TRY(enqueue_factor(H, d, damp, act_order, perm, inv, lambda, Hp, T1, status, st, true, &U));
+  if (U != H)   // act-order: the factor of the permuted H_d goes back into H
+    GPTQ_CUDA_TRY(cudaMemcpyAsync(H, U, (size_t)d * d * 4, cudaMemcpyDeviceToDevice, st));
+  int host_status = 0;
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(&host_status, status, sizeof(int), cudaMemcpyDeviceToHost, st));
+  GPTQ_CUDA_TRY(cudaStreamSynchronize(st));
+  return host_status;
+}
+
+extern "C" size_t gptq_quantize_with_factor_workspace_bytes(int64_t r, int64_t d, int bits,
+                                                            int group, int block) {
+  if (!valid_layer(r, d, bits, group, block)) return 0;
+  return sweep_layout(r, d, group, block).total;
+}
+
+extern "C" int gptq_quantize_with_factor(const float *W, int64_t r, int64_t d, const float *U,
+                                         const int32_t *perm, const float *lambda, int bits,
+                                         int group, int block, int options, float *W_hat,
+                                         int32_t *qweight, float *scales, int32_t *zeros,
+                                         int32_t *g_idx, uint8_t *codes, double *loss,
+                                         void *workspace, size_t workspace_bytes,
+                                         gptq_stream_t stream) {
+  if (!valid_layer(r, d, bits, group, block) || !valid_options(options))
+    return GPTQ_ERR_INVALID_ARG;
+  const bool act_order = (options & GPTQ_ACT_ORDER) != 0;
+  const int sym = (options & GPTQ_SYMMETRIC) ? 1 : 0;
+  const int static_groups = (options & GPTQ_STATIC_GROUPS) && group > 0 ? 1 : 0;
+  if (r == 0) {
+    if (loss) *loss = 0.0;
+    return GPTQ_OK;
+  }
+  if (!W || !U || !lambda || !qweight || !scales || !zeros || !workspace || (act_order && !perm))
+    return GPTQ_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(W) % 16 || reinterpret_cast<uintptr_t>(U) % 16 ||
+      reinterpret_cast<uintptr_t>(workspace) % 256 || reinterpret_cast<uintptr_t>(lambda) % 4 ||
+      (W_hat && reinterpret_cast<uintptr_t>(W_hat) % 16) ||
+      reinterpret_cast<uintptr_t>(qweight) % 4 || reinterpret_cast<uintptr_t>(scales) % 4 ||
+      reinterpret_cast<uintptr_t>(zeros) % 4 ||
+      (g_idx && reinterpret_cast<uintptr_t>(g_idx) % 16) ||
+      (codes && reinterpret_cast<uintptr_t>(codes) % 4) ||
+      (perm && reinterpret_cast<uintptr_t>(perm) % 4))
+    return GPTQ_ERR_INVALID_ARG;
+  const SweepLayout L = sweep_layout(r, d, group, block);
+  if (workspace_bytes < L.total) return GPTQ_ERR_NO_MEMORY;
+  cudaStream_t st = (cudaStream_t)stream;
+  char *ws = static_cast<char *>(workspace);
+  int *inv = reinterpret_cast<int *>(ws + L.inv);
+  double *loss_rows = reinterpret_cast<double *>(ws + L.loss_rows);
+  double *out = reinterpret_cast<double *>(ws + L.out);
+  int *status = reinterpret_cast<int *>(ws + L.status);
+  GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 16, st));
+  GPTQ_CUDA_TRY(cudaMemsetAsync(loss_rows, 0, (size_t)r * 8, st));
+  // The caller's permutation indexes W: checked on the device before any
+  // kernel uses it (a bad one sets the status word and the sweep is skipped).
+  if (act_order) GPTQ_TRY(launch_check_perm(perm, (int)d, inv, status, st));
+  const SweepPlan sp{W, (int)r, (int)d, bits, group, block, sym, static_groups, U,
+                     act_order ? perm : nullptr, act_order ? inv : nullptr, lambda, W_hat,
+                     qweight, scales, zeros, g_idx, codes,
+                     reinterpret_cast<float *>(ws + L.Wk), reinterpret_cast<float *>(ws + L.ErrS),
+                     reinterpret_cast<uint8_t *>(ws + L.codes_p), loss_rows,
+                     reinterpret_cast<double *>(ws + L.dsq_rows), out, status};
+  GPTQ_TRY(enqueue_sweep(sp, st));
+  double host_out[3] = {0, 0, 0};
+  int host_status = 0;
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(host_out, out, sizeof(host_out), cudaMemcpyDeviceToHost, st));
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(&host_status, status, sizeof(int), cudaMemcpyDeviceToHost, st));
+  GPTQ_CUDA_TRY(cudaStreamSynchronize(st));
+  if (host_status != 0) return host_status;
+  if (loss) *loss = host_out[0];
+  return GPTQ_OK;
 }
 
 namespace {
@@ -447,7 +652,7 @@ int64_t x_chunk_tokens(int64_t n) {
 }
 
 HostLayout host_layout(int64_t r, int64_t d, int64_t n, int bits, int group, int block,
-                       int act_order) {
+                       int options) {
   HostLayout L{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -463,7 +668,7 @@ HostLayout host_layout(int64_t r, int64_t d, int64_t n, int bits, int group, int
   L.sc = take((size_t)r * G * 4);
   L.zr = take((size_t)r * G * 4);
   L.gi = take((size_t)d * 4);
-  L.qws = take(layout(r, d, group, block, act_order).total);
+  L.qws = take(layout(r, d, group, block, options).total);
   L.total = off;
   return L;
 }
@@ -471,18 +676,21 @@ HostLayout host_layout(int64_t r, int64_t d, int64_t n, int bits, int group, int
 }  // namespace
 
 extern "C" size_t gptq_layer_host_workspace_bytes(int64_t r, int64_t d, int64_t n, int bits,
-                                                  int group, int block, int act_order) {
-  if (!valid_layer(r, d, bits, group, block) || n < 0 || n > (int64_t)INT32_MAX) return 0;
-  return host_layout(r, d, n, bits, group, block, act_order).total;
+                                                  int group, int block, int options) {
+  if (!valid_layer(r, d, bits, group, block) || !valid_options(options) || n < 0 ||
+      n > (int64_t)INT32_MAX)
+    return 0;
+  return host_layout(r, d, n, bits, group, block, options).total;
 }
 
 extern "C" int gptq_solve_layer_host(const uint16_t *X_host, int64_t n, const float *W_host,
                                      int64_t r, int64_t d, int bits, int group, int block,
-                                     float damp, int act_order, int32_t *qweight_host,
+                                     float damp, int options, int32_t *qweight_host,
                                      float *scales_host, int32_t *zeros_host,
                                      int32_t *g_idx_host, double *loss, void *dev_workspace,
                                      size_t dev_workspace_bytes, gptq_stream_t stream) {
-  if (!valid_layer(r, d, bits, group, block) || n < 0 || n > (int64_t)INT32_MAX)
+  if (!valid_layer(r, d, bits, group, block) || !valid_options(options) || n < 0 ||
+      n > (int64_t)INT32_MAX)
     return GPTQ_ERR_INVALID_ARG;
   if ((n > 0 && !X_host) || !W_host || !qweight_host || !scales_host || !zeros_host ||
       !dev_workspace || reinterpret_cast<uintptr_t>(dev_workspace) % 256)
@@ -491,7 +699,7 @@ extern "C" int gptq_solve_layer_host(const uint16_t *X_host, int64_t n, const fl
     if (loss) *loss = 0.0;
     return GPTQ_OK;
   }
-  const HostLayout L = host_layout(r, d, n, bits, group, block, act_order);
+  const HostLayout L = host_layout(r, d, n, bits, group, block, options);
   if (dev_workspace_bytes < L.total) return GPTQ_ERR_NO_MEMORY;
   cudaStream_t st = (cudaStream_t)stream;
   char *ws = static_cast<char *>(dev_workspace);
@@ -525,7 +733,7 @@ extern "C" int gptq_solve_layer_host(const uint16_t *X_host, int64_t n, const fl
   }
   GPTQ_CUDA_TRY(cudaEventRecord(cs->ev[nch + 1], cs->s));   // W (copied first) and all of X
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(st, cs->ev[nch + 1], 0));
-  GPTQ_TRY(gptq_quantize_layer(W, r, d, H, bits, group, block, damp, act_order, nullptr, qw, sc,
+  GPTQ_TRY(gptq_quantize_layer(W, r, d, H, bits, group, block, damp, options, nullptr, qw, sc,
                                zr, gi, nullptr, loss, ws + L.qws, L.total - L.qws, stream));
   GPTQ_CUDA_TRY(cudaMemcpyAsync(qweight_host, qw, (size_t)r * (d * bits / 32) * 4,
                                 cudaMemcpyDeviceToHost, st));

@@ -80,17 +80,45 @@ __global__ void __launch_bounds__(256) rank_kernel(const float *H, int64_t ld, i
   }
 }
 
-// Hp[a][b] = H[perm[a]][perm[b]] (+ lambda on the diagonal).
+// Hp[a][b] = H[perm[a]][perm[b]] (+ lambda on the diagonal); rows a step by
+// the grid's height (at most 65535).
 __global__ void permute_sym_kernel(const float *H, int64_t ld, int d, const int *perm,
                                    const float *lambda, float *Hp) {
   pdl_wait_then_release();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  const int a = blockIdx.y;
   if (b >= d) return;
-  const int pa = perm[a], pb = perm[b];
-  float v = H[(size_t)pa * ld + pb];
-  if (a == b) v += *lambda;
-  Hp[(size_t)a * d + b] = v;
+  const int pb = perm[b];
+  for (int a = blockIdx.y; a < d; a += gridDim.y) {
+    float v = H[(size_t)perm[a] * ld + pb];
+    if (a == b) v += *lambda;
+    Hp[(size_t)a * d + b] = v;
+  }
+}
+
+// inv[perm[p]] = p after checking that perm is a permutation of 0 .. d-1
+// (d <= 65536); otherwise the status word is set and the later kernels skip.
+__global__ void __launch_bounds__(1024) check_perm_kernel(const int *perm, int d, int *inv,
+                                                          int *status) {
+  __shared__ unsigned seen[65536 / 32];
+  __shared__ int bad;
+  pdl_wait_then_release();
+  for (int i = threadIdx.x; i < 65536 / 32; i += blockDim.x) seen[i] = 0u;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  for (int p = threadIdx.x; p < d; p += blockDim.x) {
+    const int c = perm[p];
+    if (c < 0 || c >= d) {
+      bad = 1;
+      continue;
+    }
+    const unsigned bit = 1u << (c & 31);
+    if (atomicOr(&seen[c >> 5], bit) & bit)
+      bad = 1;   // a repeated entry (so another is missing)
+    else
+      inv[c] = p;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && bad) atomicCAS(status, 0, (int)GPTQ_ERR_INVALID_ARG);
 }
 
 }  // namespace
@@ -107,9 +135,15 @@ int launch_damp(float *H, int64_t ld, int d, float damp, bool add_in_place, floa
 int launch_act_order(const float *H, int64_t ld, int d, int *perm, int *inv, const float *lambda,
                      float *Hp, cudaStream_t stream) {
   GPTQ_LAUNCH_PDL(rank_kernel, dim3((d + 255) / 256), dim3(256), 0, stream, H, ld, d, perm, inv);
-  dim3 grid((d + 255) / 256, d);
+  dim3 grid((d + 255) / 256, d < 65535 ? d : 65535);
   GPTQ_LAUNCH_PDL(permute_sym_kernel, grid, dim3(256), 0, stream, H, ld, d, (const int *)perm,
                   lambda, Hp);
+  return GPTQ_OK;
+}
+
+int launch_check_perm(const int *perm, int d, int *inv, int *status, cudaStream_t stream) {
+  if (d <= 0 || d > 65536) return GPTQ_ERR_INVALID_ARG;
+  GPTQ_LAUNCH_PDL(check_perm_kernel, dim3(1), dim3(1024), 0, stream, perm, d, inv, status);
   return GPTQ_OK;
 }
 

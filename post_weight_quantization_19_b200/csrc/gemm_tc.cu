@@ -456,7 +456,7 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
     set_last_error_msg(__FILE__, __LINE__, "cuTensorMapEncodeTiled rejected a GEMM operand");
     return GPTQ_ERR_CUDA;
   }
-  static bool attr[64] = {};
+  static std::atomic<bool> attr[64] = {};
   if (const int rc = ensure_smem_attr(gemm_tc_kernel, SMEM_BYTES, attr)) return rc;
   TcArgs a{g.M, g.N, g.K, g.C, g.ldc, g.alpha, g.beta, g.flags, trans_b ? 1 : 0, g.status,
            device_status_word()};

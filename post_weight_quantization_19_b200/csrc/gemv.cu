@@ -12,8 +12,16 @@
 // (0 for group = -1).  One warp per row: lane l takes the 32-code chunks l,
 // l + 32, ... of the row (b consecutive words each, fetched 4 chunks ahead),
 // unpacks them with static shifts, and accumulates the m dot products in fp32
-// (m rounded up to 1, 2, 4 or 8 accumulators); a shuffle reduction ends the row.  Bandwidth bound at small m: r*d*b/8 bytes of codes,
-// 8*r*G bytes of scales and zeros, 4*m*(d + r) bytes of x and y.
+// (m rounded up to 1, 2, 4 or 8 accumulators); a shuffle reduction ends the
+// row.  Bandwidth bound at small m: r*d*b/8 bytes of codes, 8*r*G bytes of
+// scales and zeros, 4*m*(d + r) bytes of x and y.
+//
+// x is read by every row.  Neighbouring lanes need x 128 bytes apart (one
+// chunk each), so a warp's 16-byte load of x straight from global memory
+// touches 32 cache lines; each CTA therefore first copies x into shared memory
+// with 4 floats of padding after every 32, where the same warp-wide read hits
+// every bank exactly four times (the minimum for 512 bytes).  Shapes whose x
+// does not fit read it from global memory instead.
 #include "gptq_internal.h"
 
 namespace gptq {
@@ -21,6 +29,9 @@ namespace {
 
 constexpr int GEMV_WARPS = 8;
 constexpr int GEMV_MAX_M = GPTQ_GEMV_MAX_M;
+
+constexpr int XPAD = 36;                         // floats per staged 32-float chunk of x
+constexpr size_t GEMV_SMEM_MAX = 200u << 10;     // staged x, bytes
 
 struct GemvArgs {
   const uint32_t *qweight;
@@ -34,10 +45,11 @@ struct GemvArgs {
 };
 
 // One 32-code chunk: unpack with static shifts and accumulate MB dot products.
-template <int BITS, int MB>
+// SX: x staged in shared memory (sx, XPAD floats per chunk), else read from a.x.
+template <int BITS, int MB, bool SX>
 __device__ __forceinline__ void gemv_chunk(const uint32_t (&w)[BITS], const GemvArgs &a,
                                            const float *srow, const int32_t *zrow, int k,
-                                           float (&acc)[MB]) {
+                                           const float *sx, float (&acc)[MB]) {
   constexpr uint32_t mask = (1u << BITS) - 1u;
   float s = 0.f, z = 0.f;
   if (!a.g_idx) {   // groups are multiples of 32 columns: one group per chunk
@@ -49,9 +61,14 @@ __device__ __forceinline__ void gemv_chunk(const uint32_t (&w)[BITS], const Gemv
   for (int j4 = 0; j4 < 32; j4 += 4) {
     float4 xv[MB];
 #pragma unroll
-    for (int i = 0; i < MB; ++i)
-      xv[i] = i < a.m ? __ldg(reinterpret_cast<const float4 *>(a.x + (int64_t)i * a.d + k * 32 + j4))
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < MB; ++i) {
+      if (i >= a.m)
+        xv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      else if constexpr (SX)
+        xv[i] = *reinterpret_cast<const float4 *>(sx + ((size_t)i * (a.d / 32) + k) * XPAD + j4);
+      else
+        xv[i] = __ldg(reinterpret_cast<const float4 *>(a.x + (int64_t)i * a.d + k * 32 + j4));
+    }
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
       const int j = j4 + jj;
@@ -78,11 +95,21 @@ __device__ __forceinline__ void gemv_chunk(const uint32_t (&w)[BITS], const Gemv
 // MB accumulators (the batch rounded up to 1, 2, 4 or 8); a lane fetches the
 // words of up to PF of its chunks before any arithmetic, so each row waits on
 // memory about once.
-template <int BITS, int MB>
+template <int BITS, int MB, bool SX>
 __global__ void __launch_bounds__(32 * GEMV_WARPS) gemv_kernel(GemvArgs a) {
   constexpr int PF = 4;
+  extern __shared__ __align__(16) float sx[];   // SX: [m][d/32][XPAD]
   const int lane = threadIdx.x & 31;
   const int nchunk = a.d / 32;
+  if constexpr (SX) {
+    const int per = nchunk * 8;                  // 16-byte pieces of one vector
+    for (int idx = threadIdx.x; idx < a.m * per; idx += blockDim.x) {
+      const int i = idx / per, rem = idx - i * per, k = rem >> 3, q = rem & 7;
+      *reinterpret_cast<float4 *>(sx + ((size_t)i * nchunk + k) * XPAD + q * 4) =
+          __ldg(reinterpret_cast<const float4 *>(a.x + (int64_t)i * a.d + k * 32 + q * 4));
+    }
+    __syncthreads();
+  }
   const int64_t wpr = (int64_t)nchunk * BITS;   // words per row
   for (int64_t row = (int64_t)blockIdx.x * GEMV_WARPS + (threadIdx.x >> 5); row < a.r;
        row += (int64_t)gridDim.x * GEMV_WARPS) {
@@ -102,7 +129,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS) gemv_kernel(GemvArgs a) {
       }
 #pragma unroll
       for (int p = 0; p < PF; ++p)
-        if (k0 + 32 * p < nchunk) gemv_chunk<BITS, MB>(w[p], a, srow, zrow, k0 + 32 * p, acc);
+        if (k0 + 32 * p < nchunk) gemv_chunk<BITS, MB, SX>(w[p], a, srow, zrow, k0 + 32 * p, sx, acc);
     }
 #pragma unroll
     for (int i = 0; i < MB; ++i) {
@@ -114,18 +141,39 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS) gemv_kernel(GemvArgs a) {
   }
 }
 
-template <int BITS>
-int gemv_launch(const GemvArgs &a, dim3 grid, cudaStream_t st) {
-  if (a.m <= 1)
-    gemv_kernel<BITS, 1><<<grid, 32 * GEMV_WARPS, 0, st>>>(a);
-  else if (a.m <= 2)
-    gemv_kernel<BITS, 2><<<grid, 32 * GEMV_WARPS, 0, st>>>(a);
-  else if (a.m <= 4)
-    gemv_kernel<BITS, 4><<<grid, 32 * GEMV_WARPS, 0, st>>>(a);
-  else
-    gemv_kernel<BITS, GEMV_MAX_M><<<grid, 32 * GEMV_WARPS, 0, st>>>(a);
+template <int BITS, int MB, bool SX>
+int gemv_launch_mb(const GemvArgs &a, cudaStream_t st) {
+  const int64_t want = (a.r + GEMV_WARPS - 1) / GEMV_WARPS;
+  size_t smem = 0;
+  int64_t cap = (int64_t)num_sms() * 16;
+  if constexpr (SX) {
+    static std::atomic<bool> attr[64] = {};
+    smem = (size_t)a.m * (a.d / 32) * XPAD * sizeof(float);
+    if (const int rc = ensure_smem_attr(gemv_kernel<BITS, MB, true>, GEMV_SMEM_MAX, attr))
+      return rc;
+    // every CTA stages x once: a few CTAs per SM, each looping over rows
+    const int64_t per_sm = (int64_t)(GEMV_SMEM_MAX / smem);
+    cap = (int64_t)num_sms() * (per_sm < 1 ? 1 : per_sm > 4 ? 4 : per_sm);
+  }
+  const dim3 grid((unsigned)(want < cap ? want : cap));
+  gemv_kernel<BITS, MB, SX><<<grid, 32 * GEMV_WARPS, smem, st>>>(a);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
+}
+
+template <int BITS, bool SX>
+int gemv_launch_sx(const GemvArgs &a, cudaStream_t st) {
+  if (a.m <= 1) return gemv_launch_mb<BITS, 1, SX>(a, st);
+  if (a.m <= 2) return gemv_launch_mb<BITS, 2, SX>(a, st);
+  if (a.m <= 4) return gemv_launch_mb<BITS, 4, SX>(a, st);
+  return gemv_launch_mb<BITS, GEMV_MAX_M, SX>(a, st);
+}
+
+template <int BITS>
+int gemv_launch(const GemvArgs &a, cudaStream_t st) {
+  const size_t staged = (size_t)a.m * (a.d / 32) * XPAD * sizeof(float);
+  return staged <= GEMV_SMEM_MAX ? gemv_launch_sx<BITS, true>(a, st)
+                                 : gemv_launch_sx<BITS, false>(a, st);
 }
 
 }  // namespace
@@ -151,14 +199,11 @@ extern "C" int gptq_dequant_gemv(const int32_t *qweight, const float *scales,
     return GPTQ_ERR_INVALID_ARG;
   GemvArgs a{reinterpret_cast<const uint32_t *>(qweight), scales, zeros, g_idx, r, (int)d,
              group, group < 0 ? 1 : (int)(d / group), (int)m, x, y};
-  const int64_t want = (r + GEMV_WARPS - 1) / GEMV_WARPS;
-  const int64_t cap = (int64_t)num_sms() * 16;
-  const dim3 grid((unsigned)(want < cap ? want : cap));
   cudaStream_t st = (cudaStream_t)stream;
   switch (bits) {
-    case 2: return gemv_launch<2>(a, grid, st);
-    case 3: return gemv_launch<3>(a, grid, st);
-    case 4: return gemv_launch<4>(a, grid, st);
-    default: return gemv_launch<8>(a, grid, st);
+    case 2: return gemv_launch<2>(a, st);
+    case 3: return gemv_launch<3>(a, st);
+    case 4: return gemv_launch<4>(a, st);
+    default: return gemv_launch<8>(a, st);
   }
 }

@@ -53,15 +53,16 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // The dynamic shared-memory limit of a kernel, raised once per device (the
 // attribute belongs to the kernel in the current device's context).
+// (Two threads may both set it the first time; setting it twice is harmless.)
 template <typename K>
-int ensure_smem_attr(K kernel, size_t bytes, bool (&done)[64]) {
+int ensure_smem_attr(K kernel, size_t bytes, std::atomic<bool> (&done)[64]) {
   int dev = 0;
   GPTQ_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return GPTQ_ERR_INVALID_ARG;
-  if (!done[dev]) {
+  if (!done[dev].load(std::memory_order_acquire)) {
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bytes));
-    done[dev] = true;
+    done[dev].store(true, std::memory_order_release);
   }
   return GPTQ_OK;
 }
@@ -112,6 +113,8 @@ int launch_damp(float *H, int64_t ld, int d, float damp, bool add_in_place, floa
                 cudaStream_t stream);
 int launch_act_order(const float *H, int64_t ld, int d, int *perm, int *inv, const float *lambda,
                      float *Hp, cudaStream_t stream);
+// inv[perm[p]] = p after checking that perm is a permutation (status set otherwise).
+int launch_check_perm(const int *perm, int d, int *inv, int *status, cudaStream_t stream);
 // Scratch of the factorisation: one h x m product per depth of the merge tree.
 size_t factor_scratch_floats(int64_t d);
 // One diagonal block (nb <= 128, nb % 32 == 0) of H_d -> U in place (full block, zeros below).
@@ -125,9 +128,16 @@ int launch_factor(float *A, int64_t d, float *T1, int *status, cudaStream_t stre
 // gptq_quantize_layer; plain = true creates nothing (no CUDA graph, no second
 // stream or events) and launches every kernel directly on `stream`.
 int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int group, int block,
-                   float damp, int act_order, float *W_hat, int32_t *qweight, float *scales,
+                   float damp, int options, float *W_hat, int32_t *qweight, float *scales,
                    int32_t *zeros, int32_t *g_idx, uint8_t *codes, double *loss, void *workspace,
                    size_t workspace_bytes, gptq_stream_t stream, bool plain);
+
+// SweepArgs::flags.  (The struct stays at 128 bytes: a larger kernel parameter
+// block costs the sweep kernel about 35 registers.)
+enum SweepFlags {
+  SWEEP_SYM = 1,     // symmetric quantiser
+  SWEEP_STATIC = 2   // parameters fixed before the sweep: read, never computed
+};
 
 struct SweepArgs {
   float *Wk;          // working weights r x d (sweep order), row stride ldw
@@ -139,8 +149,10 @@ struct SweepArgs {
   float *scales;      // r x G
   int32_t *zeros;     // r x G
   int G;
-  uint8_t *codes;     // r x d codes in sweep order
-  int64_t ldc;
+  int flags;          // SWEEP_SYM | SWEEP_STATIC
+  uint8_t *codes;     // r x d codes in sweep order, row stride ldw
+  const int *perm;    // static groups under act-order: column j of the sweep is
+                      // original column perm[j], of group perm[j] / group
   float *err;         // r x lde; column 0 is the block's first column
   int64_t lde;
   double *loss_rows;  // per-row running sum of e^2 / 2
@@ -149,8 +161,10 @@ struct SweepArgs {
 
 int launch_gather_w(const float *W, int r, int d, const int *perm, float *Wk, const int *status,
                     cudaStream_t stream);
-int launch_row_params(const float *Wk, int r, int d, int bits, float *scales, int32_t *zeros,
-                      const int *status, cudaStream_t stream);
+// Per-row parameters of groups of g consecutive columns of Wsrc [r x d] (g = d:
+// one group per row), G = d / g per row.
+int launch_row_params(const float *Wsrc, int r, int d, int g, int bits, int sym, float *scales,
+                      int32_t *zeros, const int *status, cudaStream_t stream);
 int launch_sweep_block(const SweepArgs &a, int block, cudaStream_t stream);
 
 struct FinalizeArgs {
@@ -159,6 +173,7 @@ struct FinalizeArgs {
   const uint8_t *codes_p;
   const int *inv;       // inv[c] = sweep position of column c (NULL: identity)
   int r, d, bits, group;
+  int static_groups;    // g_idx[c] = c / group even under act-order
   float *W_hat;         // may be NULL
   uint8_t *codes;       // may be NULL
   int32_t *qweight;

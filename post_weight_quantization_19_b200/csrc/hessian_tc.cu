@@ -38,29 +38,33 @@ __device__ int g_device_status;
 
 // Per-device lookups are cached so that no runtime query runs inside a
 // stream capture of the solve.
+// (Atomic slots: host threads driving different devices may fill them at once.)
 int *device_status_word() {
-  static int *cache[64] = {};
+  static std::atomic<int *> cache[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!cache[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-    cache[dev] = static_cast<int *>(p);
+  int *p = cache[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void *q = nullptr;
+    if (cudaGetSymbolAddress(&q, g_device_status) != cudaSuccess) return nullptr;
+    p = static_cast<int *>(q);
+    cache[dev].store(p, std::memory_order_release);
   }
-  return cache[dev];
+  return p;
 }
 
 int num_sms() {
-  static int cache[64] = {};
+  static std::atomic<int> cache[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return 1;
-  if (!cache[dev]) {
-    int v = 0;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (!v) {
     cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = v > 0 ? v : 1;
+    v = v > 0 ? v : 1;
+    cache[dev].store(v, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return v;
 }
 
 namespace {

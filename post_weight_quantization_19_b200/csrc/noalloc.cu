@@ -53,10 +53,10 @@ int scratch_address(void **out) {
 
 extern "C" int gptq_quantize_layer_noalloc(const float *W, int64_t r, int64_t d, float *H,
                                            int bits, int group, int block, float damp,
-                                           int act_order, float *W_hat, int32_t *qweight,
+                                           int options, float *W_hat, int32_t *qweight,
                                            float *scales, int32_t *zeros, int32_t *g_idx,
                                            uint8_t *codes, double *loss, gptq_stream_t stream) {
-  const size_t need = gptq_quantize_workspace_bytes(r, d, bits, group, block, act_order);
+  const size_t need = gptq_quantize_workspace_bytes(r, d, bits, group, block, options);
   if (need == 0) return GPTQ_ERR_INVALID_ARG;
   if (need > gptq::kScratchBytes) {
     gptq::set_last_error_msg(__FILE__, __LINE__,
@@ -74,7 +74,7 @@ extern "C" int gptq_quantize_layer_noalloc(const float *W, int64_t r, int64_t d,
   // whatever an earlier call left in the array does not leak into this one.
   // The plain form launches the kernels directly: no CUDA graph and no second
   // stream are created on this path.
-  return gptq::quantize_layer(W, r, d, H, bits, group, block, damp, act_order, W_hat, qweight,
+  return gptq::quantize_layer(W, r, d, H, bits, group, block, damp, options, W_hat, qweight,
                               scales, zeros, g_idx, codes, loss, scratch, gptq::kScratchBytes,
                               stream, true);
 }

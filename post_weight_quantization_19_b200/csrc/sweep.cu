@@ -18,6 +18,7 @@
 // it (the same value, so no divergence) and updates its 32 columns with
 // fused multiply-adds.  No inter-warp synchronisation at all.
 #include <float.h>
+#include <stdlib.h>
 
 #include "gptq_internal.h"
 #include "pack_bits.cuh"
@@ -25,9 +26,8 @@
 namespace gptq {
 namespace {
 
-constexpr int SWEEP_WARPS = 4;
-constexpr int SWEEP_THREADS = 32 * SWEEP_WARPS;
-constexpr int SWEEP_CW = 16;    // columns of a 128-column block held by one lane
+constexpr int SWEEP_WARPS = 4;   // warps per CTA (8 for the 16-lane form of the 128-column block)
+constexpr int SWEEP_CW = 16;     // columns of a 128-column block held by one lane
 
 __device__ __forceinline__ float warp_min(float v) {
 #pragma unroll
@@ -53,9 +53,21 @@ __device__ __forceinline__ float row_max(float v) {
   return v;
 }
 
-// Asymmetric min-max parameters over a range [lo, hi] widened to include 0:
-// s = (xmax - xmin)/(2^b - 1) (1 for an empty range), z = rint(-xmin/s).
-__device__ __forceinline__ void minmax_params(float lo, float hi, float maxq, float &s, float &z) {
+// Parameters of a group whose values span [lo, hi].
+// Asymmetric min-max: the range widened to include 0, s = (xmax - xmin)/(2^b - 1)
+// (1 for an empty range), z = rint(-xmin/s).
+// Symmetric ("LLM 量化技术" §1.2): zero point 0 in the signed code, s = max|x| /
+// (2^(b-1) - 1) (1 for an all-zero group); the signed code is stored as code +
+// 2^(b-1), i.e. z = 2^(b-1), and the clamp [-z, maxq - z] is then the signed range.
+__device__ __forceinline__ void quant_params(float lo, float hi, float maxq, bool sym, float &s,
+                                             float &z) {
+  if (sym) {
+    const float amax = fmaxf(fabsf(lo), fabsf(hi));
+    const float half = 0.5f * (maxq + 1.f);
+    s = amax == 0.f ? 1.f : __fdiv_rn(amax, half - 1.f);
+    z = half;
+    return;
+  }
   const float xmin = fminf(lo, 0.f), xmax = fmaxf(hi, 0.f);
   s = (xmax == xmin) ? 1.f : __fdiv_rn(xmax - xmin, maxq);
   z = rintf(__fdiv_rn(-xmin, s));
@@ -79,29 +91,36 @@ __global__ void gather_w_kernel(const float *__restrict__ W, int64_t total, int 
   }
 }
 
-// group = -1: one (s, z) per row from the row's original values.
-__global__ void row_params_kernel(const float *__restrict__ Wk, int r, int d, int bits,
-                                  float *__restrict__ scales, int32_t *__restrict__ zeros,
-                                  const int *status) {
+// Parameters fixed before the sweep, one warp per row, over groups of g
+// consecutive columns of Wsrc: g = d for group = -1 (one (s, z) per row, from
+// the sweep-order copy: a permutation leaves the minimum and maximum alone),
+// g = group for static groups (from the original W, in its own column order).
+__global__ void row_params_kernel(const float *__restrict__ Wsrc, int r, int d, int g, int bits,
+                                  int sym, float *__restrict__ scales,
+                                  int32_t *__restrict__ zeros, const int *status) {
   pdl_wait_then_release();
   if (*(volatile const int *)status) return;
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= r) return;
-  const float *w = Wk + (size_t)row * d;
-  float lo = FLT_MAX, hi = -FLT_MAX;
-  for (int c = lane; c < d; c += 32) {
-    const float x = w[c];
-    lo = fminf(lo, x);
-    hi = fmaxf(hi, x);
-  }
-  lo = warp_min(lo);
-  hi = warp_max(hi);
-  float s, z;
-  minmax_params(lo, hi, (float)((1 << bits) - 1), s, z);
-  if (lane == 0) {
-    scales[row] = s;
-    zeros[row] = (int32_t)z;
+  const float *w = Wsrc + (size_t)row * d;
+  const int G = d / g;
+  const float maxq = (float)((1 << bits) - 1);
+  for (int k = 0; k < G; ++k) {
+    float lo = FLT_MAX, hi = -FLT_MAX;
+    for (int c = k * g + lane; c < (k + 1) * g; c += 32) {
+      const float x = w[c];
+      lo = fminf(lo, x);
+      hi = fmaxf(hi, x);
+    }
+    lo = warp_min(lo);
+    hi = warp_max(hi);
+    float s, z;
+    quant_params(lo, hi, maxq, sym != 0, s, z);
+    if (lane == 0) {
+      scales[(size_t)row * G + k] = s;
+      zeros[(size_t)row * G + k] = (int32_t)z;
+    }
   }
 }
 
@@ -122,8 +141,14 @@ __device__ __forceinline__ void cp_async_wait_all() {
 }
 
 // B = CW * L columns per block: each row is held by L lanes with CW columns each.
-template <int CW, int L>
-__global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a) {
+// VAR: the quantiser variants of SweepArgs::flags are honoured (the plain
+// instantiation compiles them out, leaving its registers and schedule alone).
+// With static groups under act-order (perm given) every column reads its own
+// group's fixed parameters: the groups of the original columns are scattered
+// over the sweep order.
+template <int CW, int L, bool VAR, int WARPS>
+__global__ void __launch_bounds__(32 * WARPS) sweep_block_kernel(SweepArgs a) {
+  constexpr int SWEEP_THREADS = 32 * WARPS;
   constexpr int B = CW * L;
   constexpr int CHUNK = CW + 4;        // stride of one lane's part of a U row in shared
                                        // memory: the L parts start in different banks
@@ -132,6 +157,7 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
   // U[j0+j][j0+c] for c > j, else 0; element (j, c) at j * RSTRIDE + (c / CW) * CHUNK + c % CW
   extern __shared__ __align__(16) float sU[];
   __shared__ float sDinv[B];
+  __shared__ int sGrp[VAR ? B : 1];   // group of each column of the block (per-column mode)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nc = a.ncols;
@@ -165,6 +191,12 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
 
   const float maxq = (float)((1 << a.bits) - 1);
   const int g = a.group;   // -1 or a multiple of 32
+  const int flags = VAR ? a.flags : 0;
+  const bool percol = VAR && a.perm != nullptr;   // uniform over the grid
+  if (percol) {
+    for (int j = tid; j < B; j += SWEEP_THREADS) sGrp[j] = j < nc ? a.perm[a.j0 + j] / g : 0;
+    __syncthreads();
+  }
   const int gmask = (g > 0 && g <= B) ? g - 1 : -1;         // groups start inside the block
   const bool start_here = g > B && (a.j0 % g) == 0;         // a long group starts at column 0
   const bool inherit = g < 0 || (g > B && !start_here);     // parameters set before this block
@@ -174,8 +206,8 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
   const int nsub = nc / CW;       // 32-column parts present in this block
   const bool mine = ql < nsub;
 
-  for (int row0 = (blockIdx.x * SWEEP_WARPS + warp) * RPW; row0 < a.r;
-       row0 += gridDim.x * SWEEP_WARPS * RPW) {
+  for (int row0 = (blockIdx.x * WARPS + warp) * RPW; row0 < a.r;
+       row0 += gridDim.x * WARPS * RPW) {
     // Lanes of rows past the end keep going (zeros) so the shuffles stay whole.
     const int row = row0 + lane / L;
     const bool valid = row < a.r;
@@ -208,7 +240,16 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
     for (int sb = 0; sb < nsub; ++sb) {
       const int jb = sb * CW;
       // Groups are multiples of 32 columns, so they start only at a part's first column.
-      if ((gmask >= 0 && (jb & gmask) == 0) || (jb == 0 && start_here)) {
+      if (percol) {
+        // parameters are read per column below
+      } else if ((flags & SWEEP_STATIC) &&
+                 ((gmask >= 0 && (jb & gmask) == 0) || (jb == 0 && start_here))) {
+        // fixed before the sweep: read, not computed
+        const int gi = (a.j0 + jb) / g;
+        s = valid ? a.scales[(size_t)row * a.G + gi] : 1.f;
+        z = valid ? (float)a.zeros[(size_t)row * a.G + gi] : 0.f;
+        si = recip(s);
+      } else if ((gmask >= 0 && (jb & gmask) == 0) || (jb == 0 && start_here)) {
         float lo = FLT_MAX, hi = -FLT_MAX;
         const int jend = gmask >= 0 ? jb + g : B;
         if (mine && ql >= sb && ql * CW < jend) {
@@ -230,7 +271,7 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
         }
         lo = row_min<L>(lo);
         hi = row_max<L>(hi);
-        minmax_params(lo, hi, maxq, s, z);
+        quant_params(lo, hi, maxq, (flags & SWEEP_SYM) != 0, s, z);
         si = recip(s);
         if (ql == 0 && valid) {
           const int gi = (a.j0 + jb) / g;
@@ -245,10 +286,19 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
       // rint(x) is taken as (x + 1.5 * 2^23) - 1.5 * 2^23 in round-to-nearest-
       // even: exact for |x| < 2^22, and for larger |x| both forms clamp to the
       // same end of [-z, maxq - z].
-      const float tlo = -z, thi = maxq - z;
+      float tlo = -z, thi = maxq - z;
       float wj = __shfl_sync(0xffffffffu, w[0], base + sb);
 #pragma unroll
       for (int i = 0; i < CW; ++i) {
+        if (percol) {
+          // the same column for every row: one broadcast read of its group
+          const size_t at = (size_t)(valid ? row : 0) * a.G + sGrp[jb + i];
+          s = __ldg(a.scales + at);
+          z = (float)__ldg(a.zeros + at);
+          si = recip(s);
+          tlo = -z;
+          thi = maxq - z;
+        }
         const float t = fminf(fmaxf(round_even(wj * si), tlo), thi);
         const float wq = s * t;
         const float e = (wj - wq) * dv[i];
@@ -281,21 +331,27 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(SweepArgs a)
     if (valid && mine) {
       float *wp = wrow + ql * CW;
       float *ep = a.err + (size_t)row * a.lde + ql * CW;
-      uint8_t *cp = a.codes + (size_t)row * a.ldc + a.j0 + ql * CW;
+      uint8_t *cp = a.codes + (size_t)row * a.ldw + a.j0 + ql * CW;
 #pragma unroll
       for (int c = 0; c < CW; c += 4) {
         *reinterpret_cast<float4 *>(wp + c) = make_float4(w[c], w[c + 1], w[c + 2], w[c + 3]);
         *reinterpret_cast<float4 *>(ep + c) = make_float4(eo[c], eo[c + 1], eo[c + 2], eo[c + 3]);
       }
+      // 16 codes per 16-byte store (8 per 8-byte store when a lane holds 8 columns)
+      constexpr int CS = CW % 16 == 0 ? 16 : 8;
+      static_assert(CW % CS == 0, "codes per store");
 #pragma unroll
-      for (int c = 0; c < CW; c += 16) {
-        uint32_t wd[4];
+      for (int c = 0; c < CW; c += CS) {
+        uint32_t wd[CS / 4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
+        for (int k = 0; k < CS / 4; ++k)
           wd[k] = (uint32_t)(int)code[c + 4 * k] | ((uint32_t)(int)code[c + 4 * k + 1] << 8) |
                   ((uint32_t)(int)code[c + 4 * k + 2] << 16) |
                   ((uint32_t)(int)code[c + 4 * k + 3] << 24);
-        *reinterpret_cast<uint4 *>(cp + c) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        if constexpr (CS == 16)
+          *reinterpret_cast<uint4 *>(cp + c) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        else
+          *reinterpret_cast<uint2 *>(cp + c) = make_uint2(wd[0], wd[1]);
       }
     }
     if (ql == 0 && valid) a.loss_rows[row] = loss0 + 0.5 * (double)esq;
@@ -334,7 +390,9 @@ __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
         if (row == 0 && a.g_idx) {
           const int g = a.group;
           *reinterpret_cast<int4 *>(a.g_idx + c) =
-              g < 0 ? make_int4(0, 0, 0, 0) : make_int4(p.x / g, p.y / g, p.z / g, p.w / g);
+              g < 0              ? make_int4(0, 0, 0, 0)
+              : a.static_groups  ? make_int4(c / g, (c + 1) / g, (c + 2) / g, (c + 3) / g)
+                                 : make_int4(p.x / g, p.y / g, p.z / g, p.w / g);
         }
       } else {
         wq = *reinterpret_cast<const float4 *>(wk + c);
@@ -421,36 +479,60 @@ int launch_gather_w(const float *W, int r, int d, const int *perm, float *Wk, co
   return GPTQ_OK;
 }
 
-int launch_row_params(const float *Wk, int r, int d, int bits, float *scales, int32_t *zeros,
-                      const int *status, cudaStream_t stream) {
-  GPTQ_LAUNCH_PDL(row_params_kernel, dim3((r + 7) / 8), dim3(256), 0, stream, Wk, r, d, bits, scales,
-                  zeros, status);
+int launch_row_params(const float *Wsrc, int r, int d, int g, int bits, int sym, float *scales,
+                      int32_t *zeros, const int *status, cudaStream_t stream) {
+  if (g <= 0 || g % 32 != 0 || d % g != 0) return GPTQ_ERR_INVALID_ARG;
+  GPTQ_LAUNCH_PDL(row_params_kernel, dim3((r + 7) / 8), dim3(256), 0, stream, Wsrc, r, d, g, bits,
+                  sym, scales, zeros, status);
   return GPTQ_OK;
 }
 
-template <int CW, int L>
+template <int CW, int L, bool VAR, int WARPS = SWEEP_WARPS>
 static int sweep_launch(const SweepArgs &a, cudaStream_t stream) {
   constexpr int B = CW * L;
   const size_t smem = (size_t)B * (CW + 4) * L * sizeof(float);
-  static bool attr[64] = {};
-  if (const int rc = ensure_smem_attr(sweep_block_kernel<CW, L>, smem, attr)) return rc;
+  static std::atomic<bool> attr[64] = {};
+  if (const int rc = ensure_smem_attr(sweep_block_kernel<CW, L, VAR, WARPS>, smem, attr))
+    return rc;
   // Every row gets its lanes in one wave when the SMs can hold them (two CTAs
   // per SM: about 180 registers per thread).
-  const int rows_per_cta = SWEEP_WARPS * (32 / L);
+  const int rows_per_cta = WARPS * (32 / L);
   const int want = (a.r + rows_per_cta - 1) / rows_per_cta;
   const int cap = num_sms() * 2;
   const int grid = want < cap ? want : cap;
-  GPTQ_LAUNCH_PDL((sweep_block_kernel<CW, L>), dim3(grid), dim3(SWEEP_THREADS), smem, stream, a);
+  GPTQ_LAUNCH_PDL((sweep_block_kernel<CW, L, VAR, WARPS>), dim3(grid), dim3(32 * WARPS), smem,
+                  stream, a);
   return GPTQ_OK;
 }
 
-int launch_sweep_block(const SweepArgs &a, int block, cudaStream_t stream) {
+// GPTQ_SWEEP_LANES=16 selects the 16-lane form of the 128-column block (read once).
+static bool sweep_lanes16() {
+  static const bool on = [] {
+    const char *v = getenv("GPTQ_SWEEP_LANES");
+    return v && v[0] == '1' && v[1] == '6' && v[2] == 0;
+  }();
+  return on;
+}
+
+template <bool VAR>
+static int sweep_launch_block(const SweepArgs &a, int block, cudaStream_t stream) {
   switch (block) {
-    case 32: return sweep_launch<32, 1>(a, stream);
-    case 64: return sweep_launch<32, 2>(a, stream);
-    case 128: return sweep_launch<SWEEP_CW, 128 / SWEEP_CW>(a, stream);
+    case 32: return sweep_launch<32, 1, VAR>(a, stream);
+    case 64: return sweep_launch<32, 2, VAR>(a, stream);
+    case 128:
+      // Experimental form under measurement: 16 lanes of 8 columns per row in
+      // CTAs of 8 warps (twice the warps per SM for the same rows).
+      if (sweep_lanes16())
+        return sweep_launch<8, 16, VAR, 8>(a, stream);
+      return sweep_launch<SWEEP_CW, 128 / SWEEP_CW, VAR>(a, stream);
     default: return GPTQ_ERR_INVALID_ARG;
   }
+}
+
+int launch_sweep_block(const SweepArgs &a, int block, cudaStream_t stream) {
+  if (a.perm && !((a.flags & SWEEP_STATIC) && a.group > 0)) return GPTQ_ERR_INVALID_ARG;
+  return (a.flags || a.perm) ? sweep_launch_block<true>(a, block, stream)
+                             : sweep_launch_block<false>(a, block, stream);
 }
 
 int launch_finalize(const FinalizeArgs &a, cudaStream_t stream) {

@@ -32,7 +32,8 @@ def assert_codes_close(got: np.ndarray, ref: np.ndarray, frac: float = CODE_MATC
 
 
 def gpu_layer(X: np.ndarray | None, W: np.ndarray, *, bits: int, group: int, block: int = 128,
-              damp: float = 0.01, act_order: bool = False, H32: np.ndarray | None = None) -> dict:
+              damp: float = 0.01, act_order: bool = False, H32: np.ndarray | None = None,
+              sym: bool = False, static_groups: bool = False) -> dict:
     """Run the CUDA path: H from X on the GPU (or a given fp32 H), then the solve."""
     import torch
 
@@ -52,7 +53,8 @@ def gpu_layer(X: np.ndarray | None, W: np.ndarray, *, bits: int, group: int, blo
     codes = torch.empty((r, d), dtype=torch.uint8, device=dev)
     g_idx = torch.empty((d,), dtype=torch.int32, device=dev)
     res = g.gptq_quantize_layer(Wd, H, bits=bits, group=group, block=block, damp=damp,
-                                act_order=act_order, W_hat=W_hat, codes=codes, g_idx=g_idx)
+                                act_order=act_order, sym=sym, static_groups=static_groups,
+                                W_hat=W_hat, codes=codes, g_idx=g_idx)
     torch.cuda.synchronize()
     return {
         "H": H_used,

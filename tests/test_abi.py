@@ -49,8 +49,11 @@ def test_workspace_query(lib):
                 (16, 256, 4, 48, 128, 0),      # group not a divisor of the block
                 (16, 256, 4, 96, 128, 0),
                 (16, 256, 4, -1, 96, 0),       # block
-                (-1, 256, 4, -1, 128, 0)]:
+                (-1, 256, 4, -1, 128, 0),
+                (16, 256, 4, -1, 128, 8)]:     # unknown option bit
         assert ws(*bad) == 0, bad
+    # the option bits GPTQ_SYMMETRIC and GPTQ_STATIC_GROUPS need no extra workspace
+    assert ws(4096, 4096, 4, 128, 128, 2 | 4) == base
     hw = lib.gptq_layer_host_workspace_bytes(128, 256, 2048, 4, -1, 128, 0)
     assert hw >= 2048 * 256 * 2 + 256 * 256 * 4 + 128 * 256 * 4
 
@@ -66,6 +69,9 @@ def test_validation_returns_before_cuda(lib):
     assert q(p, 8, 256, p, 4, -1, 128, -1.0, 0, None, p, p, p, None, None,
              ctypes.byref(loss), p, 1 << 30, None) == 1
     assert q(p, 8, 256, p, 4, -1, 128, float("nan"), 0, None, p, p, p, None, None,
+             ctypes.byref(loss), p, 1 << 30, None) == 1
+    # unknown option bit
+    assert q(p, 8, 256, p, 4, -1, 128, 0.01, 8, None, p, p, p, None, None,
              ctypes.byref(loss), p, 1 << 30, None) == 1
     # missing output pointer
     assert q(p, 8, 256, p, 4, -1, 128, 0.01, 0, None, None, p, p, None, None,
@@ -95,6 +101,32 @@ def test_validation_returns_before_cuda(lib):
     assert gv(p, p, p, None, 8, 128, 4, -1, None, 1, p, None) == 1  # missing x
     assert gv(p, p, p, None, 0, 128, 4, -1, p, 1, p, None) == 0     # no rows: nothing to do
     assert gv(p, p, p, None, 8, 128, 4, -1, p, 0, p, None) == 0     # no vectors
+    fw = lib.gptq_factor_workspace_bytes
+    assert fw(100, 0) == 0 and fw(256, 8) == 0 and fw(256, 1) > fw(256, 0) > 0
+    f = lib.gptq_factor
+    assert f(p, 100, 0.01, 0, None, p, p, 1 << 30, None) == 1     # d % 32
+    assert f(p, 256, 0.01, 1, None, p, p, 1 << 30, None) == 1     # act-order without perm
+    assert f(p, 256, -1.0, 0, None, p, p, 1 << 30, None) == 1     # damp
+    assert f(p, 256, 0.01, 0, None, p, ctypes.c_void_p(1 << 20), 64, None) == 4   # workspace
+    qf = lib.gptq_quantize_with_factor
+    assert lib.gptq_quantize_with_factor_workspace_bytes(8, 256, 4, 128, 128) > 0
+    assert qf(p, 8, 256, p, None, p, 4, 128, 128, 1, None, p, p, p, None, None,
+              ctypes.byref(loss), p, 1 << 30, None) == 1             # act-order without perm
+    assert qf(p, 8, 256, p, None, p, 5, 128, 128, 0, None, p, p, p, None, None,
+              ctypes.byref(loss), p, 1 << 30, None) == 1             # bits
+    assert qf(p, 0, 256, p, None, p, 4, 128, 128, 0, None, p, p, p, None, None,
+              ctypes.byref(loss), p, 0, None) == 0                   # no rows
+    df = lib.gptq_dequant_fp16
+    assert df(p, p, p, None, 8, 100, 4, -1, p, None) == 1           # d % 32
+    assert df(p, p, p, None, 8, 128, 6, -1, p, None) == 1           # bits
+    assert df(p, p, p, None, 8, 128, 4, -1, ctypes.c_void_p(4104), None) == 1   # W16 alignment
+    assert df(p, p, p, None, 0, 128, 4, -1, p, None) == 0           # no rows
+    lf = lib.gptq_linear_fp16
+    assert lf(p, 16, 100, p, 64, p, None) == 1                      # d % 32
+    assert lf(p, 16, 128, p, 40, p, None) == 1                      # r % 32
+    assert lf(ctypes.c_void_p(4104), 16, 128, p, 64, p, None) == 1  # X alignment
+    assert lf(p, 0, 128, p, 64, p, None) == 0                       # no tokens
+    assert lf(p, 16, 128, p, 0, p, None) == 0                       # no outputs
 
 
 def test_no_kernels_launched_on_cpu(lib):

@@ -119,6 +119,136 @@ def test_full_path_matches_oracle(case):
     check_against_oracle(got, ref, W, bits=bits, group=group)
 
 
+VARIANT_CASES = [
+    # r, d, n, bits, group, block, act_order, sym, static_groups
+    (64, 512, 4096, 4, -1, 128, False, True, False),
+    (48, 384, 3000, 4, 128, 128, True, True, False),
+    (50, 256, 2048, 3, 32, 128, False, True, False),
+    (40, 512, 4096, 4, 64, 128, False, False, True),
+    (48, 384, 3000, 4, 128, 128, True, False, True),
+    (37, 512, 4096, 3, 32, 128, True, True, True),
+    (33, 512, 4096, 4, 256, 128, True, False, True),    # groups longer than the block
+    (64, 256, 2048, 2, 64, 64, True, True, True),
+]
+
+
+@pytest.mark.parametrize("case", VARIANT_CASES, ids=lambda c: "r{}_d{}_b{}_g{}_a{}_s{}_t{}".format(
+    c[0], c[1], c[3], c[4], int(c[6]), int(c[7]), int(c[8])))
+def test_quantiser_variants_match_oracle(case):
+    # Symmetric quantiser and static groups, alone and with act-order, from the
+    # same fp32 Hessian on both sides.
+    r, d, n, bits, group, block, act, sym, static = case
+    X, W = make_problem(r, d, n, seed=r * 13 + d)
+    H32 = oracle.hessian(X).astype(np.float32)
+    got = gpu_layer(None, W, bits=bits, group=group, block=block, act_order=act, H32=H32,
+                    sym=sym, static_groups=static)
+    ref = oracle.gptq_quantize_layer(W, H32.astype(np.float64), bits=bits, group=group,
+                                     block=block, act_order=act, sym=sym, static_groups=static)
+    check_against_oracle(got, ref, W, bits=bits, group=group)
+    if sym:
+        assert np.all(got["zeros"] == 1 << (bits - 1))
+    if static:
+        np.testing.assert_array_equal(got["g_idx"], np.arange(d) // group)
+        # fixed from the original W before the sweep: the same on both sides up
+        # to the fp32 division
+        np.testing.assert_allclose(got["scales"], ref["scales"], rtol=1e-6)
+        assert float(np.mean(got["zeros"] == ref["zeros"])) >= 0.999
+
+
+@pytest.mark.parametrize("act,sym,static", [(False, False, False), (True, False, False),
+                                             (True, True, True)])
+def test_factor_then_sweep_equals_one_call(act, sym, static):
+    # The two halves run the same kernels in the same order as the one call,
+    # so the outputs are the same bits; one factor then serves three layers
+    # that share the inputs (and so H), each equal to its own one-call solve.
+    import post_weight_quantization_19_b200 as g
+    X, _ = make_problem(1, 512, 4096, seed=91)
+    Ws = [make_weights(rr, 512, seed=92 + i) for i, rr in enumerate((96, 64, 160))]
+    H32 = oracle.hessian(X).astype(np.float32)
+    fac = g.gptq_factor(torch.from_numpy(H32.copy()).cuda(), act_order=act)
+    for W in Ws:
+        Wd = torch.from_numpy(W).cuda()
+        gi1 = torch.empty(512, dtype=torch.int32, device="cuda")
+        one = g.gptq_quantize_layer(Wd, torch.from_numpy(H32.copy()).cuda(), bits=4, group=128,
+                                    act_order=act, sym=sym, static_groups=static, g_idx=gi1)
+        gi2 = torch.empty(512, dtype=torch.int32, device="cuda")
+        two = g.gptq_quantize_with_factor(Wd, fac, bits=4, group=128, sym=sym,
+                                          static_groups=static, g_idx=gi2)
+        torch.cuda.synchronize()
+        for key in ("qweight", "scales", "zeros"):
+            np.testing.assert_array_equal(two[key].cpu().numpy(), one[key].cpu().numpy())
+        np.testing.assert_array_equal(gi2.cpu().numpy(), gi1.cpu().numpy())
+        assert two["loss"] == one["loss"]
+
+
+def test_sweep_rejects_a_perm_that_is_not_a_permutation():
+    # Checked on the device before anything indexes W with it.
+    import post_weight_quantization_19_b200 as g
+    X, W = make_problem(32, 256, 2048, seed=93)
+    fac = g.gptq_factor(torch.from_numpy(oracle.hessian(X).astype(np.float32)).cuda(),
+                        act_order=True)
+    bad = dict(fac)
+    bad["perm"] = fac["perm"].clone()
+    bad["perm"][7] = bad["perm"][3]          # a repeated entry
+    with pytest.raises(g.GPTQError) as e:
+        g.gptq_quantize_with_factor(torch.from_numpy(W).cuda(), bad, bits=4, group=128)
+    assert e.value.status == 1
+    bad["perm"][7] = 1 << 20                 # out of range
+    with pytest.raises(g.GPTQError):
+        g.gptq_quantize_with_factor(torch.from_numpy(W).cuda(), bad, bits=4, group=128)
+    # and the good one still works afterwards
+    res = g.gptq_quantize_with_factor(torch.from_numpy(W).cuda(), fac, bits=4, group=128)
+    assert res["loss"] > 0
+
+
+def test_sixteen_lane_sweep_gives_the_same_layer():
+    # The 16-lane form of the 128-column block (selected by GPTQ_SWEEP_LANES=16,
+    # read once per process) runs in a child process and must give the same
+    # codes as the default form here.
+    import os
+    import subprocess
+    import sys
+    r, d, n = 77, 640, 4096
+    X, W = make_problem(r, d, n, seed=97)
+    H32 = oracle.hessian(X).astype(np.float32)
+    got = gpu_layer(None, W, bits=4, group=128, act_order=True, H32=H32)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import sys, numpy as np; sys.path[:0] = [%r, %r]\n"
+        "from synth import make_problem\nimport oracle\nfrom parity_util import gpu_layer\n"
+        "X, W = make_problem(%d, %d, %d, seed=97)\n"
+        "got = gpu_layer(None, W, bits=4, group=128, act_order=True,"
+        " H32=oracle.hessian(X).astype(np.float32))\n"
+        "np.save(sys.argv[1], got['codes'])\n" % (root, os.path.join(root, "tests"), r, d, n))
+    out = os.path.join(os.environ.get("TMPDIR", "/tmp"), "codes16_%d.npy" % os.getpid())
+    env = dict(os.environ, GPTQ_SWEEP_LANES="16")
+    subprocess.run([sys.executable, "-c", code, out], check=True, env=env, timeout=600)
+    np.testing.assert_array_equal(np.load(out), got["codes"])
+
+
+def test_earlier_leaf_gives_the_same_layer():
+    # GPTQ_LEAF=1 (read once per process) runs the earlier leaf (FFMA products,
+    # one column per barrier); its U differs only by rounding, so the codes agree
+    # with the default leaf's up to the usual tie decisions.
+    import os
+    import subprocess
+    import sys
+    r, d, n = 64, 512, 4096
+    X, W = make_problem(r, d, n, seed=98)
+    got = gpu_layer(None, W, bits=4, group=128, H32=oracle.hessian(X).astype(np.float32))
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import sys, numpy as np; sys.path[:0] = [%r, %r]\n"
+        "from synth import make_problem\nimport oracle\nfrom parity_util import gpu_layer\n"
+        "X, W = make_problem(%d, %d, %d, seed=98)\n"
+        "got = gpu_layer(None, W, bits=4, group=128, H32=oracle.hessian(X).astype(np.float32))\n"
+        "np.save(sys.argv[1], got['codes'])\n" % (root, os.path.join(root, "tests"), r, d, n))
+    out = os.path.join(os.environ.get("TMPDIR", "/tmp"), "codes_leaf1_%d.npy" % os.getpid())
+    env = dict(os.environ, GPTQ_LEAF="1")
+    subprocess.run([sys.executable, "-c", code, out], check=True, env=env, timeout=600)
+    assert_codes_close(np.load(out), got["codes"])
+
+
 def test_tiny_workload_end_to_end():
     wl = workload("tiny_128x256")
     X, W = workload_inputs(wl)
@@ -308,6 +438,115 @@ def test_dequant_gemv_matches_oracle(case):
                                rtol=1e-6, atol=1e-6 * np.abs(ref).max())
 
 
+@pytest.mark.parametrize("d,m,bits", [(4096, 8, 4), (16384, 2, 3), (8192, 8, 4), (65536, 1, 2),
+                                      (2048, 5, 8)])
+def test_dequant_gemv_staged_and_direct_x(d, m, bits):
+    # x is staged in shared memory when m * d * 4.5 bytes fit in 200 KB and read
+    # from global memory otherwise ((8192, 8) and (65536, 1)); both give the
+    # float64 oracle's product on random packed rows.
+    import post_weight_quantization_19_b200 as g
+    r, group = 67, 128
+    rng = np.random.default_rng(d + m)
+    codes = rng.integers(0, 1 << bits, size=(r, d), dtype=np.uint8)
+    qweight = oracle.pack_rows(codes, bits)
+    scales = (rng.random((r, d // group)) * 0.01 + 1e-3).astype(np.float32)
+    zeros = rng.integers(0, 1 << bits, size=(r, d // group)).astype(np.int32)
+    x = rng.standard_normal((m, d)).astype(np.float32)
+    y = g.gptq_dequant_gemv(*(torch.from_numpy(a).cuda() for a in (qweight, scales, zeros, x)),
+                            bits, group)
+    torch.cuda.synchronize()
+    ref = oracle.dequant_gemv(qweight, scales, zeros, bits, group, x)
+    assert np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max() <= 1e-5
+
+
+# ------------------------------------------------------------------ the layer run forward
+
+def _fp16_ulps(a, b):
+    # distance in units in the last place between fp16 arrays of finite values
+    ia = a.view(np.int16).astype(np.int32)
+    ib = b.view(np.int16).astype(np.int32)
+    ia = np.where(ia < 0, -32768 - ia, ia)
+    ib = np.where(ib < 0, -32768 - ib, ib)
+    return np.abs(ia - ib)
+
+
+@pytest.mark.parametrize("bits,group,act", [(4, 128, False), (3, -1, False), (4, 32, True)])
+def test_dequant_fp16_matches_oracle(bits, group, act):
+    # fp16(s (q - z)) from the GPU's own packed layer; the oracle forms s (q - z)
+    # exactly and rounds once, the kernel rounds the fp32 product: equal except
+    # where the fp32 product lands on an fp16 tie (at most one fp16 step).
+    import post_weight_quantization_19_b200 as g
+    X, W = make_problem(70, 512, 3000, seed=60 + bits)
+    got = gpu_layer(X, W, bits=bits, group=group, act_order=act)
+    q = torch.from_numpy(got["qweight"]).cuda()
+    W16 = g.gptq_dequant_fp16(q, torch.from_numpy(got["scales"]).cuda(),
+                              torch.from_numpy(got["zeros"]).cuda(), 512, bits, group,
+                              g_idx=torch.from_numpy(got["g_idx"]).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.dequant_gemv(got["qweight"], got["scales"], got["zeros"], bits, group,
+                              np.eye(512), g_idx=got["g_idx"]).T.astype(np.float16)
+    # a double rounding differs from the single one with probability about 2^-13
+    ulps = _fp16_ulps(W16.cpu().numpy(), ref)
+    assert ulps.max() <= 1 and float(np.mean(ulps == 0)) >= 0.999
+
+
+@pytest.mark.parametrize("n,d,r", [(1000, 2080, 288), (256, 64, 32), (4096, 512, 768)])
+def test_linear_fp16_matches_oracle(n, d, r):
+    # Y = fp16(X W16^T) against the exact sum of the fp16 products.  The error
+    # allowed is half an fp16 step (the final rounding) plus the tensor cores'
+    # fp32 accumulation: chains of 32 MMAs of K = 16, each within a few fp32
+    # ulps of its running sum (not necessarily rounded to nearest), folded into
+    # fp32 registers every 512 features -- well inside 2^-14 of sum |x w|.  The
+    # shapes have ragged token tiles, a half-empty last feature stage and a
+    # ragged output tile.
+    import post_weight_quantization_19_b200 as g
+    rng = np.random.default_rng(n + d + r)
+    X = make_activations(n, d, seed=n + d)
+    W16 = (0.02 * rng.standard_normal((r, d))).astype(np.float16)
+    Y = g.gptq_linear_fp16(torch.from_numpy(X).cuda(), torch.from_numpy(W16).cuda())
+    torch.cuda.synchronize()
+    X64, W64 = X.astype(np.float64), W16.astype(np.float64)
+    exact = X64 @ W64.T
+    absum = np.abs(X64) @ np.abs(W64).T
+    got = Y.cpu().numpy()
+    assert np.all(np.isfinite(got))
+    half_step = 0.5 * np.spacing(np.abs(exact).astype(np.float16)).astype(np.float64)
+    err = np.abs(got.astype(np.float64) - exact)
+    assert np.all(err <= half_step + 2.0 ** -14 * absum)
+    # and most outputs are the correctly rounded value itself
+    assert float(np.mean(got == exact.astype(np.float16))) >= 0.95
+
+
+def test_chain_of_layers_matches_oracle():
+    # Three layers (256 -> 384 -> 128 -> 256), each calibrated on the quantised
+    # outputs of the previous ones.  Layer 0 has the single-layer tolerance.  The
+    # later layers see inputs that differ from the oracle's wherever layer 0 took
+    # a rounding tie the other way or an fp16 output rounded the other way, so
+    # their bar is looser: codes 99 % identical and within one step, loss within 1 %.
+    import post_weight_quantization_19_b200 as g
+    X0 = make_activations(4096, 256, seed=71)
+    shapes = [(384, 256), (128, 384), (256, 128)]
+    Ws = [make_weights(rr, dd, seed=72 + i) for i, (rr, dd) in enumerate(shapes)]
+    codes_gpu = []
+    outs = g.quantize_chain(torch.from_numpy(X0).cuda(),
+                            [torch.from_numpy(np.ascontiguousarray(W, dtype=np.float32)).cuda()
+                             for W in Ws], bits=4, group=128, keep_inputs=True)
+    torch.cuda.synchronize()
+    ref = oracle.quantize_chain(X0, Ws, bits=4, group=128)
+    for k, (o, rf) in enumerate(zip(outs, ref)):
+        d = Ws[k].shape[1]
+        codes = oracle.unpack_rows(o["qweight"].cpu().numpy(), 4, d)
+        codes_gpu.append(codes)
+        assert_codes_close(codes, rf["codes"], 0.999 if k == 0 else 0.99)
+        rel = abs(o["loss"] - rf["loss"]) / rf["loss"]
+        assert rel <= (5e-3 if k == 0 else 1e-2), (k, rel)
+        xin = o["inputs"].cpu().numpy()
+        if k == 0:
+            np.testing.assert_array_equal(xin, rf["inputs"])
+        else:
+            assert rel_fro(xin, rf["inputs"]) <= 2e-3, k
+
+
 def test_dequant_gemv_full_layer_bandwidth():
     # The 4096 x 4096 4-bit group-128 layer at batch 1: parity on all rows and the
     # achieved read bandwidth (packed codes + scales + zeros + x) printed.
@@ -347,3 +586,36 @@ def test_dequant_gemv_full_layer_bandwidth():
     nbytes = qweight.nbytes + scales.nbytes + zeros.nbytes + x.nbytes + r * 4
     print(f"dequant_gemv 4096x4096 4-bit g128 m=1: {ms * 1e3:.2f} us, {nbytes / ms / 1e6:.0f} GB/s")
 
+
+
+@pytest.mark.parametrize("factor_once", [True, False])
+def test_sharded_solve_at_world_size_one(factor_once):
+    # The multi-rank path on one GPU (NCCL, one rank): the real entry points in
+    # the sharded layout give the single-call solve.
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    import post_weight_quantization_19_b200 as g
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        X, W = make_problem(80, 512, 4096, seed=95)
+        Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda()
+        res = g.solve_layer_sharded(Xd, Wd, bits=4, group=128, act_order=True,
+                                    factor_once=factor_once)
+        H = torch.zeros((512, 512), device="cuda")
+        g.gptq_hessian_accumulate(Xd, H)
+        gi = torch.empty(512, dtype=torch.int32, device="cuda")
+        one = g.gptq_quantize_layer(Wd, H, bits=4, group=128, act_order=True, g_idx=gi)
+        torch.cuda.synchronize()
+        for key in ("qweight", "scales", "zeros"):
+            np.testing.assert_array_equal(res[key].cpu().numpy(), one[key].cpu().numpy())
+        np.testing.assert_array_equal(res["g_idx"].cpu().numpy(), gi.cpu().numpy())
+        assert res["loss"] == pytest.approx(one["loss"], rel=1e-12)
+    finally:
+        dist.destroy_process_group()
