@@ -4,8 +4,9 @@
 One step = one layer: H = 0, H += 2 X^T X (tensor cores), then the solve
 (damping, Cholesky factor and inverse, column sweep with lazy trailing updates,
 unpermute, loss, int32 packing).  Inputs are resident in HBM before the timed
-region; X (2.1 GB for the default workload) is larger than L2, so nothing is
-reused between steps through the cache.
+region; X (6.4 GB for the default OPT-175B fc2 layer, 12288 x 49152 with 65536
+tokens) is larger than L2, so nothing is reused between steps through the
+cache.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -37,13 +38,14 @@ if ROOT not in sys.path:
 from synth import WORKLOADS, workload, workload_inputs  # noqa: E402
 
 METRIC = "ms per layer (Hessian+Cholesky+solve+pack) and % of tensor/HBM roofline"
-DEFAULT_WORKLOAD = "llama7b_q_proj_4096x4096"
+DEFAULT_WORKLOAD = "opt175b_fc2_12288x49152"
 
 
 def _args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=60)
+    p.add_argument("--steps", type=int, default=None,
+                   help="timed steps (default: about half a minute of layers)")
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -63,9 +65,9 @@ def _config(wl) -> dict:
     }
 
 
-# DRAM bytes (read + write) of one full-size launch of the dominant kernel, from a one-pass
-# ncu capture (profiles/hessian_tc_kernel_traffic.md).  Valid only for the kernel source it
-# was taken on: reported as null as soon as the sources hash differently.
+# DRAM bytes (read + write) of one full-size launch of the Hessian kernel, from a one-pass
+# ncu capture of the same workload.  Valid only for the kernel source it was taken on:
+# reported as null as soon as the sources hash differently.
 KERNEL_TRAFFIC = {
     "llama7b_q_proj_4096x4096": {
         "kernel": "hessian_tc_kernel",
@@ -163,27 +165,6 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle leg
 
-def _oracle_sample(wl, X, W, n_s: int, r_s: int) -> dict:
-    """Time the float64 oracle on a bounded sample and scale each phase to the layer."""
-    import oracle
-
-    t0 = time.perf_counter()
-    H = oracle.hessian(X[:n_s])
-    t1 = time.perf_counter()
-    Hd, _ = oracle.dampen(H, wl.damp)
-    perm = oracle.act_order_perm(H) if wl.act_order else np.arange(wl.d)
-    U = oracle.inverse_upper_cholesky(Hd[np.ix_(perm, perm)])
-    t2 = time.perf_counter()
-    codes, *_ = oracle.gptq_sweep(W[:r_s][:, perm], U, wl.bits, wl.group, wl.block)
-    t3 = time.perf_counter()
-    oracle.pack_rows(codes, wl.bits)
-    t4 = time.perf_counter()
-    ms = 1e3 * ((t1 - t0) * wl.n / n_s + (t2 - t1) + (t3 - t2) * wl.r / r_s
-                + (t4 - t3) * wl.r / r_s)
-    return {"ms_per_layer": ms, "measured_s": t4 - t0,
-            "phases_s": [t1 - t0, t2 - t1, t3 - t2, t4 - t3]}
-
-
 def _cores() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -191,77 +172,154 @@ def _cores() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(wl, X, W, n_s: int, r_s: int) -> dict:
-    res = _oracle_sample(wl, X, W, n_s, r_s)
+def sample_sizes(wl, big: bool) -> tuple[int, int, int]:
+    """(tokens, features, rows) of the bounded CPU sample: a leading block of the layer."""
+    if big:
+        return min(wl.n, 16384), min(wl.d, 8192), min(wl.r, 256)
+    return min(wl.n, 8192), min(wl.d, 4096), min(wl.r, 128)
+
+
+def _oracle_sample(wl, X, W, n_s: int, d_s: int, r_s: int) -> dict:
+    """Time the float64 oracle on the leading n_s x d_s block of X and r_s x d_s of W,
+    then extrapolate each phase to the whole layer by its cost model:
+    Hessian n*d*(d+1); factor d^3; sweep a*d + b*d^2 per row (fitted from the
+    sample at d_s and d_s/2: the column loop and the deferred updates), times
+    r/r_s; packing r*d."""
+    import oracle
+
+    Xs = np.ascontiguousarray(X[:n_s, :d_s])
+    Ws = np.ascontiguousarray(W[:r_s, :d_s])
+    t0 = time.perf_counter()
+    H = oracle.hessian(Xs)
+    t1 = time.perf_counter()
+    Hd, _ = oracle.dampen(H, wl.damp)
+    perm = oracle.act_order_perm(H) if wl.act_order else np.arange(d_s)
+    U = oracle.inverse_upper_cholesky(Hd[np.ix_(perm, perm)])
+    t2 = time.perf_counter()
+    g = wl.group if wl.group == -1 or d_s % wl.group == 0 else -1
+    codes, *_ = oracle.gptq_sweep(Ws[:, perm], U, wl.bits, g, wl.block)
+    t3 = time.perf_counter()
+    h2 = d_s // 2
+    oracle.gptq_sweep(Ws[:, perm][:, :h2], U[:h2, :h2], wl.bits, g if g == -1 or h2 % g == 0
+                      else -1, wl.block)
+    t4 = time.perf_counter()
+    oracle.pack_rows(codes, wl.bits)
+    t5 = time.perf_counter()
+    th, tf, ts, ts2, tp = t1 - t0, t2 - t1, t3 - t2, t4 - t3, t5 - t4
+    # sweep(d) = a d + b d^2 through (d_s/2, ts2) and (d_s, ts)
+    b = max((ts - 2.0 * ts2) / (d_s * d_s / 2.0), 0.0)
+    a = max((ts - b * d_s * d_s) / d_s, 0.0)
+    d, n, r = wl.d, wl.n, wl.r
+    phases = {
+        "hessian": th * (n / n_s) * (d * (d + 1.0)) / (d_s * (d_s + 1.0)),
+        "factor": tf * (d / d_s) ** 3,
+        "sweep": (a * d + b * d * d) * (r / r_s),
+        "pack": tp * (r / r_s) * (d / d_s),
+    }
+    return {"ms_per_layer": 1e3 * sum(phases.values()), "measured_s": t5 - t0,
+            "phases_s": phases,
+            "sample": (f"float64 numpy oracle on a leading block: Hessian of {n_s} tokens x {d_s} "
+                       f"features (x{n / n_s:g} tokens, x{(d * (d + 1.0)) / (d_s * (d_s + 1.0)):.4g} "
+                       f"features^2), damping+inverse+Cholesky at {d_s} (x{(d / d_s) ** 3:.4g}, "
+                       f"d^3), sweep of {r_s} rows at {d_s} and {h2} columns fitted to a*d+b*d^2 "
+                       f"and scaled to {d} columns x {r / r_s:g} rows, packing x{r / r_s * d / d_s:.4g}"
+                       f"; {t5 - t0:.1f} s measured, the rest extrapolated")}
+
+
+def cpu_baseline(wl, X, W) -> dict:
+    n_s, d_s, r_s = sample_sizes(wl, big=True)
+    res = _oracle_sample(wl, X, W, n_s, d_s, r_s)
     return {"value": round(res["ms_per_layer"], 3), "unit": "ms per layer", "cores": _cores(),
-            "kind": "oracle",
-            "sample": f"float64 numpy oracle: Hessian on {n_s} of {wl.n} tokens (x{wl.n / n_s:g}),"
-                      f" full {wl.d}x{wl.d} damping+inverse+Cholesky, sweep+pack on {r_s} of "
-                      f"{wl.r} rows (x{wl.r / r_s:g}); {res['measured_s']:.1f} s measured"}
+            "kind": "oracle", "extrapolated": True, "sample": res["sample"],
+            "phases_s": {k: round(v, 3) for k, v in res["phases_s"].items()}}
 
 
 def run_reference(args, wl, rank: int, world: int):
     if rank != 0:
         return
-    n_s, r_s = min(wl.n, 8192), min(wl.r, 32)
+    n_s, d_s, r_s = sample_sizes(wl, big=False)
     X, W = workload_inputs(wl, n=n_s)
+    steps = args.steps if args.steps is not None else 10
     for _ in range(args.warmup):
-        _oracle_sample(wl, X, W, n_s, r_s)
-    vals, wall = [], 0.0
-    for _ in range(args.steps):
-        res = _oracle_sample(wl, X, W, n_s, r_s)
+        _oracle_sample(wl, X, W, n_s, d_s, r_s)
+    vals, wall, res = [], 0.0, None
+    for _ in range(steps):
+        res = _oracle_sample(wl, X, W, n_s, d_s, r_s)
         vals.append(res["ms_per_layer"])
         wall += res["measured_s"]
     value = float(np.mean(vals))
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "ms per layer",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
         "ms_per_step": round(value, 3), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": _config(wl),
+        "extrapolated": True,
         "cpu_baseline": {"value": round(value, 3), "unit": "ms per layer", "cores": _cores(),
-                         "kind": "oracle",
-                         "sample": f"each step: Hessian on {n_s} tokens (scaled x{wl.n / n_s:g}), "
-                                   f"full d={wl.d} factor, sweep+pack on {r_s} rows (scaled "
-                                   f"x{wl.r / r_s:g})"},
+                         "kind": "oracle", "extrapolated": True,
+                         "sample": "each step: " + res["sample"],
+                         "measured_s_per_step": round(wall / steps, 3)},
         "e2e": {"value": round(value, 3), "unit": "ms per layer", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-# ------------------------------------------------------------------ per-phase rooflines
+# ------------------------------------------------------------------ rooflines
 
-def phase_rooflines(wl, phases_ms: dict, peaks: dict) -> dict:
-    """Each phase of one layer against the roofline of its algorithmic work.
+# Nominal dense tensor rates (PFLOP/s) used to carry the measured bf16 peak over
+# to another operand type: tf32 is 1.1 against 2.25 for fp16/bf16.
+TF32_OVER_BF16 = 1.1 / 2.25
 
-    hessian: n*d*(d+1) flop vs the sustained fp16 (bf16) tensor peak; factor_U:
-    2 d^3 / 3 flop (Cholesky and triangular inverse) and sweep: r*d*(d-B) flop of
-    the trailing updates that dominate it, both fp32-equivalent against a third of
-    the TF32 peak (three TF32 products per fp32 product; TF32 is half the bf16 rate);
-    damp_perm and finalize_pack: the bytes they must move vs the measured HBM copy
-    rate.  The two latency-chain phases (factor_U, the in-block part of sweep) are
-    not expected to approach their bound.
-    """
+
+def tensor_peak(peaks: dict, clocks: dict | None) -> tuple[float, str]:
+    """Measured bf16 tensor peak: the burst figure while the sampled SM clock held
+    its maximum during the timed region, else the sustained (power-capped) one."""
+    burst = peaks.get("bf16_tflops")
+    sust = peaks.get("bf16_tflops_sustained")
+    if burst is None or sust is None:
+        return 1590.0, "fallback burst (no MEASURED_PEAKS.json)"
+    sm, smax = (clocks or {}).get("sm_mhz"), (clocks or {}).get("sm_max_mhz")
+    if sm and smax and sm >= 0.97 * smax:
+        return float(burst), f"measured burst: the SM clock held {sm:.0f} of {smax:.0f} MHz"
+    return float(sust), (f"measured sustained: the SM clock median was {sm} of {smax} MHz"
+                         if sm else "measured sustained: no clock samples")
+
+
+def phase_work(wl) -> dict:
+    """Algorithmic work of each phase of one layer: (unit, amount, kind).
+
+    hessian: n*d*(d+1) flop (the symmetric product, upper triangle credited);
+    factor_U: 2 d^3 / 3 flop (Cholesky and triangular inverse); sweep: r*d*(d-B)
+    flop of the deferred trailing updates that dominate it (the sum over blocks
+    of 2 r B (d - end of block)); damp_perm and finalize_pack: the bytes they must
+    move.  Flops of the fp32 phases are fp32-equivalent."""
     r, d, n, B = wl.r, wl.d, wl.n, wl.block
-    tc = float(peaks.get("bf16_tflops_sustained", 1400.0))
-    hbm = float(peaks.get("hbm_gbs", 6650.0))
-    tf32x3 = tc / 2.0 / 3.0
     G = 1 if wl.group == -1 else d // wl.group
-    work = {
-        "hessian": ("TFLOP/s", float(n) * d * (d + 1) / 1e12, tc),
-        "damp_perm": ("GB/s", 8.0 * d * (d if wl.act_order else 1) / 1e9, hbm),
-        "factor_U": ("TFLOP/s", 2.0 * d ** 3 / 3.0 / 1e12, tf32x3),
-        "sweep": ("TFLOP/s", 2.0 * r * d * max(d - B, 0) / 1e12, tf32x3),
-        "finalize_pack": ("GB/s", (r * d * (4 + 4 + 1 + wl.bits / 8.0) + 8.0 * r * G) / 1e9, hbm),
+    return {
+        "hessian": ("TFLOP/s", float(n) * d * (d + 1) / 1e12, "fp16"),
+        "damp_perm": ("GB/s", 8.0 * d * (d if wl.act_order else 1) / 1e9, "hbm"),
+        "factor_U": ("TFLOP/s", 2.0 * d ** 3 / 3.0 / 1e12, "3xtf32"),
+        "sweep": ("TFLOP/s", float(r) * d * max(d - B, 0) / 1e12, "3xtf32"),
+        "finalize_pack": ("GB/s", (r * d * (4 + 4 + 1 + wl.bits / 8.0) + 8.0 * r * G) / 1e9, "hbm"),
     }
+
+
+def phase_rooflines(wl, phases_ms: dict, peaks: dict, tc_peak: float) -> dict:
+    """Each phase of one layer against the roofline of its algorithmic work:
+    fp16 contractions against the bf16 tensor peak; the fp32 products (three
+    TF32 products per fp32 product on the tensor cores) against a third of the
+    TF32 peak; byte-bound phases against the measured HBM copy rate."""
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    peak_of = {"fp16": tc_peak, "3xtf32": tc_peak * TF32_OVER_BF16 / 3.0, "hbm": hbm}
     out = {}
-    for name, (unit, amount, peak) in work.items():
+    for name, (unit, amount, kind) in phase_work(wl).items():
         ms = phases_ms.get(name)
         if not ms or ms <= 0:
             continue
         achieved = amount / (ms * 1e-3)
-        out[name] = {"achieved": round(achieved, 2), "peak": round(peak, 1), "unit": unit,
-                     "frac": round(achieved / peak, 4)}
+        out[name] = {"achieved": round(achieved, 2), "peak": round(peak_of[kind], 1), "unit": unit,
+                     "frac": round(achieved / peak_of[kind], 4), "work": amount,
+                     "ms": round(ms, 4)}
     return out
 
 
@@ -286,6 +344,12 @@ def job_ms_per_layer(elapsed_ms: float, steps: int, world: int) -> float:
 
 # ------------------------------------------------------------------ GPU leg
 
+def default_steps(wl) -> int:
+    """About half a minute of timed layers: 60 steps of the 4096-wide layers, fewer of
+    the wider ones."""
+    return 10 if wl.d >= 16384 else (30 if wl.d >= 8192 else 60)
+
+
 def run_ours(args, wl, rank: int, world: int, dist):
     import torch
 
@@ -294,6 +358,7 @@ def run_ours(args, wl, rank: int, world: int, dist):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    steps = args.steps if args.steps is not None else default_steps(wl)
     X, W = workload_inputs(wl)
     r, d, n = wl.r, wl.d, wl.n
     G = 1 if wl.group == -1 else d // wl.group
@@ -311,33 +376,25 @@ def run_ours(args, wl, rank: int, world: int, dist):
     torch.cuda.set_stream(stream)
     h_start = torch.cuda.Event(enable_timing=True)
     h_end = torch.cuda.Event(enable_timing=True)
+    names = ["damp_perm", "factor_U", "sweep", "finalize_pack"]
 
-    def step(time_h: bool):
+    def step():
+        """One layer; returns (loss, Hessian ms, phase ms) -- every time on the device,
+        with CUDA events on the launching stream (the solve's phase events are
+        nodes of its replayed graph)."""
         H.zero_()
-        if time_h:
-            h_start.record(stream)
+        h_start.record(stream)
         g.gptq_hessian_accumulate(Xd, H, stream=stream)
-        if time_h:
-            h_end.record(stream)
+        h_end.record(stream)
         res = g.gptq_quantize_layer(Wd, H, bits=wl.bits, group=wl.group, block=wl.block,
                                     damp=wl.damp, act_order=wl.act_order, g_idx=g_idx,
                                     workspace=ws, outputs=outs, stream=stream)
-        return res["loss"]
+        # quantize_layer returns after synchronising its stream
+        return res["loss"], h_start.elapsed_time(h_end), g.gptq_last_phase_ms()
 
-    for _ in range(max(args.warmup, 1)):
-        step(False)
-    # per-phase times (one extra untimed step with phase events on)
     g.gptq_set_phase_timing(True)
-    h_start.record(stream)
-    H.zero_()
-    g.gptq_hessian_accumulate(Xd, H, stream=stream)
-    h_end.record(stream)
-    loss = g.gptq_quantize_layer(Wd, H, bits=wl.bits, group=wl.group, block=wl.block,
-                                 damp=wl.damp, act_order=wl.act_order, g_idx=g_idx,
-                                 workspace=ws, outputs=outs, stream=stream)["loss"]
-    phases = g.gptq_last_phase_ms()
-    phase_h = h_start.elapsed_time(h_end)
-    g.gptq_set_phase_timing(False)
+    for _ in range(max(args.warmup, 1)):
+        step()
 
     bus = None
     try:
@@ -354,11 +411,12 @@ def run_ours(args, wl, rank: int, world: int, dist):
     launches0 = g.gptq_launch_count()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    h_ms = []
+    h_ms, ph_ms, loss = [], [], None
     t_start.record(stream)
-    for _ in range(args.steps):
-        step(True)
-        h_ms.append(h_start.elapsed_time(h_end))
+    for _ in range(steps):
+        loss, hm, ph = step()
+        h_ms.append(hm)
+        ph_ms.append(ph)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     if dist is not None:
@@ -366,15 +424,17 @@ def run_ours(args, wl, rank: int, world: int, dist):
     torch.cuda.synchronize(dev)
     launches = g.gptq_launch_count() - launches0
     clocks = sampler.stop()
+    g.gptq_set_phase_timing(False)
     elapsed = max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
-    ms_per_step = elapsed / args.steps
-    value = job_ms_per_layer(elapsed, args.steps, world)
+    ms_per_step = elapsed / steps
+    value = job_ms_per_layer(elapsed, steps, world)
 
     # end to end through the host-buffer entry point
     e2e = None
     if args.e2e_steps > 0:
         Xh = torch.from_numpy(X).pin_memory()
         Wh = torch.from_numpy(W).pin_memory()
+        del Xd
         hws = torch.empty(g.gptq_layer_host_workspace_bytes(r, d, n, wl.bits, wl.group,
                                                             wl.block, wl.act_order),
                           dtype=torch.uint8, device=dev)
@@ -403,36 +463,44 @@ def run_ours(args, wl, rank: int, world: int, dist):
     if rank != 0:
         return
     peaks = _peaks()
-    h_avg = float(np.mean(h_ms))
-    flops = float(n) * d * (d + 1)       # symmetric Hessian, upper triangle credited
-    achieved = flops / (h_avg * 1e-3) / 1e12
-    if "bf16_tflops_sustained" in peaks:
-        peak, peak_src = float(peaks["bf16_tflops_sustained"]), "measured (sustained)"
-    else:
-        peak, peak_src = 1400.0, "fallback (sustained)"
-    phases_ms = {"hessian": round(phase_h, 4), "damp_perm": round(phases[0], 4),
-                 "factor_U": round(phases[1], 4), "sweep": round(phases[2], 4),
-                 "finalize_pack": round(phases[3], 4)}
+    tc_peak, peak_src = tensor_peak(peaks, clocks)
+    phases_ms = {"hessian": round(float(np.mean(h_ms)), 4)}
+    for i, nm in enumerate(names):
+        vals = [p[i] for p in ph_ms if len(p) > i and p[i] > 0]
+        if vals:
+            phases_ms[nm] = round(float(np.mean(vals)), 4)
+    pr = phase_rooflines(wl, phases_ms, peaks, tc_peak)
+    # The dominant kernel: the Hessian is one launch per step; the factorisation and
+    # the sweep are phases whose tensor work is the 3xTF32 GEMM (with the leaves /
+    # in-block sweep kernels on their critical path), timed by the phase events.
+    kernel_of = {"hessian": "hessian_tc_kernel",
+                 "factor_U": "gemm_tc_kernel (factorisation phase: leaf_kernel chain + 3xTF32 GEMMs)",
+                 "sweep": "gemm_tc_kernel (sweep phase: trailing-update GEMMs + sweep_block_kernel)"}
+    dom = max((k for k in kernel_of if k in pr), key=lambda k: pr[k]["ms"])
+    dp = pr[dom]
+    roofline = {"bound": "tensor", "kernel": kernel_of[dom], "phase": dom,
+                "achieved": dp["achieved"], "peak": dp["peak"], "unit": "TFLOP/s",
+                "frac": dp["frac"], "traffic": _traffic(wl) if dom == "hessian" else None,
+                "peak_source": peak_src + ("; fp16 runs at the bf16 rate" if dom == "hessian" else
+                                           "; TF32 = bf16 x 1.1/2.25 (nominal ratio), three TF32 "
+                                           "products per fp32-equivalent product"),
+                "work_per_step": dp["work"] * 1e12, "avg_ms": dp["ms"]}
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": "ms per layer", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f16 in / f32 accumulate (Hessian); f32 solve", "data": "synthetic",
-        "config": _config(wl),
-        "roofline": {"bound": "tensor", "kernel": "hessian_tc_kernel",
-                     "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": _traffic(wl),
-                     "peak_source": peak_src + " bf16 cuBLAS peak; fp16 runs at the same rate",
-                     "flops_per_launch": flops, "avg_launch_ms": round(h_avg, 4)},
+        "dtype": "f16 in / f32 accumulate (Hessian); f32 solve (3xTF32 tensor-core products)",
+        "data": "synthetic", "config": _config(wl),
+        "roofline": roofline,
         "phases_ms": phases_ms,
-        "phase_roofline": phase_rooflines(wl, phases_ms, peaks),
+        "phase_roofline": pr,
         "loss": loss,
         "gpu_launches": int(launches),
         "clocks": clocks,
         "e2e": e2e,
     }
     if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, X, W, min(n, 8192), min(r, 32))
+        line["cpu_baseline"] = cpu_baseline(wl, X, W)
     print(json.dumps(line), flush=True)
 
 

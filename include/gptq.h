@@ -279,11 +279,13 @@ int gptq_linear_fp16(const void *X, int64_t n, int64_t d, const void *W16, int64
  * takes its scratch from a fixed array of GPTQ_NOALLOC_SCRATCH_BYTES bytes in
  * the library's own device memory instead of a workspace argument; every GPU
  * that loads the library holds that array until the process exits.  It calls
- * no allocator of any kind.
+ * no allocator of any kind and creates no stream, event or graph (phase timing,
+ * gptq_set_phase_timing, does not apply to this path).
  *
  *   Arguments, results and synchronisation are those of gptq_quantize_layer
  *   without the workspace pair.
- *   Limit: returns GPTQ_ERR_NO_MEMORY (nothing enqueued) when
+ *   Arguments are checked first (GPTQ_ERR_INVALID_ARG as for
+ *   gptq_quantize_layer); then the limit: returns GPTQ_ERR_NO_MEMORY (nothing enqueued) when
  *   gptq_quantize_workspace_bytes(r, d, bits, group, block, options) exceeds
  *   GPTQ_NOALLOC_SCRATCH_BYTES -- e.g. r = d = 2048 fits, r = d = 4096 does not.
  *   The first call on a device looks up the array's device address (once per
@@ -355,6 +357,59 @@ uint64_t gptq_launch_count(void);
  */
 int gptq_set_phase_timing(int enable);
 int gptq_last_phase_ms(float *ms, int n);
+
+/*
+ * gptq_selftest_timeout -- exercises the failure path of the kernels' bounded
+ * waits (no page counterpart: a check of this library's error handling).
+ * Launches one tensor-core GEMM of 128 x 128 x 256 on `stream` whose operand
+ * loads stop after two of its eight K steps, so its waits for the missing
+ * stages run out after about one second; the kernel then records
+ * GPTQ_ERR_TIMEOUT in the library's device status word, waits (bounded) for its
+ * own tensor-core work, frees its tensor memory and returns.  Nothing faults
+ * and the context stays usable; gptq_check_device_status(stream) afterwards
+ * returns GPTQ_ERR_TIMEOUT once (and clears it).
+ *
+ *   buf   device scratch of 81920 floats (320 KB), 16-byte aligned; its
+ *         contents are read and partly overwritten.
+ * Returns GPTQ_OK once launched, GPTQ_ERR_INVALID_ARG for a bad buffer.
+ */
+int gptq_selftest_timeout(float *buf, gptq_stream_t stream);
+
+/*
+ * gptq_factor_plan -- a host-only diagnostic of the factorisation's schedule
+ * (the Cholesky and inverse steps of gptq_quantize_layer): writes, without
+ * touching a GPU, one text line per kernel the factorisation of a d x d H_d
+ * would launch and per stream event it would record or wait on, in program
+ * order.  The schedule is a blocked right-looking Cholesky taken from the
+ * bottom-right corner with U assembled over a merge tree (the "LLM 量化技术"
+ * blog §2.3 item 3 and the GPTQ reading card, 方法适配, call for a Cholesky in
+ * place of an explicit inverse); the plan lets a test replay it in any order
+ * its streams and events allow.
+ *
+ *   d             matrix size (a multiple of 32, at most 65536).
+ *   outer_cols    outer block width S (a multiple of 128, or d); 0 = the width
+ *                 gptq_quantize_layer uses for this d.
+ *   side_streams  nonzero: the schedule with side streams (as in
+ *                 gptq_quantize_layer); 0: everything on one stream.
+ *   buf, buf_bytes  output text (NUL-terminated; may be NULL to query the size).
+ *
+ * Line formats (pointers as a buffer name and a float offset: A = the d x d
+ * matrix, row stride d; T = the factorisation scratch):
+ *   P d=<d> S=<S> T=<scratch floats> side=<0|1>
+ *   L s=<stream> A=<ptr> ld=<ld> nb=<nb>                  leaf: block -> its U
+ *   G s=<stream> M= N= K= A= lda= B= ldb= C= ldc= alpha= beta= flags= tb= prio=
+ *                                                         C = alpha A op(B) + beta C
+ *   C s=<stream> dst= ldd= src= lds= rows= cols=          2-D copy
+ *   E s=<stream> e=<id>                                   record event id on a stream
+ *   W s=<stream> e=<id>                                   the stream waits for the event
+ * GEMM flags: 1 = A upper (k from the row tile), 2 = op(B) lower (k from the
+ * column tile), 4 = B upper (k to the column tile), 8 = output tiles on or
+ * above the diagonal only; tiles are 128 x 128.
+ * Returns the bytes the full text needs (including the NUL), or 0 for invalid
+ * arguments.
+ */
+size_t gptq_factor_plan(int64_t d, int64_t outer_cols, int side_streams, char *buf,
+                        size_t buf_bytes);
 
 #ifdef __cplusplus
 }

@@ -12,10 +12,12 @@ from .gptq_ref import (  # noqa: F401
     dequant_gemv,
     dequantize,
     gptq_quantize_layer,
+    gptq_quantize_rows_lowmem,
     gptq_sweep,
     hessian,
     hessian_rows,
     inverse_upper_cholesky,
+    inverse_upper_cholesky_inplace,
     layer_loss,
     layer_loss_direct,
     pack_rows,

@@ -124,6 +124,127 @@ def inverse_upper_cholesky(Hd: np.ndarray) -> np.ndarray:
     return np.ascontiguousarray(L.T)
 
 
+def _lapack64():
+    """dsyrk, dpotrf and dpotri of the OpenBLAS bundled with numpy, which takes
+    64-bit integers (matrices of 2^31 elements and more), or None if absent.
+
+    Reference BLAS/LAPACK calling convention: every argument by reference,
+    column-major arrays, hidden lengths of the character arguments last.
+    """
+    import ctypes
+    import glob
+    import os
+
+    site = os.path.dirname(os.path.dirname(np.__file__))
+    found = glob.glob(os.path.join(site, "numpy.libs", "libscipy_openblas64_*.so"))
+    if not found:
+        return None
+    lib = ctypes.CDLL(found[0])
+    try:
+        fns = {k: getattr(lib, f"scipy_{k}_64_") for k in ("dsyrk", "dpotrf", "dpotri")}
+    except AttributeError:
+        return None
+    for f in fns.values():
+        f.restype = None
+    return fns
+
+
+_L64 = None
+
+
+def _l64():
+    global _L64
+    if _L64 is None:
+        _L64 = _lapack64() or {}
+    return _L64
+
+
+def _ref_args(*vals):
+    import ctypes
+    out = []
+    for v in vals:
+        if isinstance(v, bytes):
+            out.append(ctypes.c_char_p(v))
+        elif isinstance(v, float):
+            out.append(ctypes.byref(ctypes.c_double(v)))
+        else:
+            out.append(ctypes.byref(ctypes.c_int64(v)))
+    return out
+
+
+def syrk_upper_inplace(C: np.ndarray, A: np.ndarray, alpha: float) -> None:
+    """C += alpha A A^T on the upper triangle (library dsyrk), in place.
+
+    C: Fortran-ordered float64 d x d; A: Fortran-ordered float64 d x k."""
+    import ctypes
+
+    if not (C.flags.f_contiguous and A.flags.f_contiguous and C.dtype == F64 and A.dtype == F64):
+        raise ValueError("syrk needs Fortran-ordered float64 operands")
+    d, k = A.shape
+    L = _l64()
+    if L:
+        n_, k_, al, be, lda, ldc = _ref_args(d, k, float(alpha), 1.0, d, d)
+        L["dsyrk"](b"U", b"N", n_, k_, al, A.ctypes.data_as(ctypes.c_void_p), lda, be,
+                   C.ctypes.data_as(ctypes.c_void_p), ldc, ctypes.c_size_t(1), ctypes.c_size_t(1))
+        return
+    if d * d >= 2 ** 31:
+        raise RuntimeError("no 64-bit-index BLAS for a matrix this large")
+    from scipy.linalg import blas
+    out = blas.dsyrk(alpha, A, beta=1.0, c=C, trans=0, lower=0, overwrite_c=1)
+    if not np.shares_memory(out, C):
+        raise RuntimeError("dsyrk did not work in place")
+
+
+def _potr(name: str, A: np.ndarray) -> int:
+    import ctypes
+
+    d = A.shape[0]
+    L = _l64()
+    if L:
+        info = ctypes.c_int64(0)
+        n_, lda = _ref_args(d, d)
+        L[name](b"U", n_, A.ctypes.data_as(ctypes.c_void_p), lda, ctypes.byref(info),
+                ctypes.c_size_t(1))
+        return int(info.value)
+    if d * d >= 2 ** 31:
+        raise RuntimeError("no 64-bit-index LAPACK for a matrix this large")
+    from scipy.linalg import lapack
+    if name == "dpotrf":
+        c, info = lapack.dpotrf(A, lower=0, clean=0, overwrite_a=1)
+    else:
+        c, info = lapack.dpotri(A, lower=0, overwrite_c=1)
+    if not np.shares_memory(c, A):
+        raise RuntimeError(f"{name} did not work in place")
+    return int(info)
+
+
+def inverse_upper_cholesky_inplace(Hd: np.ndarray) -> np.ndarray:
+    """``inverse_upper_cholesky`` in the storage of Hd, for H too large to copy.
+
+    Hd must be float64 in Fortran order with its upper triangle filled (the
+    strictly lower triangle is ignored).  The same definition -- invert, then
+    take the Cholesky factor of the inverse -- with each step a LAPACK routine
+    working in place: the Cholesky factor of Hd (potrf), the inverse from that
+    factor (potri), and the upper Cholesky factor of the inverse (potrf, which
+    returns U with Hd^-1 = U^T U).  Returns U (the same storage) with the
+    strictly lower triangle zeroed.
+    """
+    if Hd.dtype != F64 or not Hd.flags.f_contiguous:
+        raise ValueError("Hd must be a Fortran-ordered float64 array")
+    for step, name in (("potrf of H_d", "dpotrf"), ("potri", "dpotri"),
+                       ("potrf of H_d^-1", "dpotrf")):
+        info = _potr(name, Hd)
+        if info != 0:
+            raise np.linalg.LinAlgError(f"{step}: info {info}")
+    d = Hd.shape[0]
+    for j0 in range(0, d, 4096):   # zero the strictly lower triangle, a band of columns at a time
+        blk = Hd[:, j0:j0 + 4096]
+        r = np.arange(d)[:, None]
+        c = np.arange(j0, min(d, j0 + 4096))[None, :]
+        blk[r > c] = 0.0
+    return Hd
+
+
 # ---------------------------------------------------------------------------
 # Asymmetric min-max quantiser  ([Tutorial] §分组方案; [Survey] §1.2)
 # ---------------------------------------------------------------------------
@@ -327,6 +448,56 @@ def gptq_quantize_layer(W: np.ndarray, H: np.ndarray, *, bits: int, group: int,
         "perm": perm,
         "U": U,
         "E": E,
+    }
+
+
+def gptq_quantize_rows_lowmem(X: np.ndarray, W: np.ndarray, rows: np.ndarray, *, bits: int,
+                              group: int, block: int = 128, damp: float = 0.01,
+                              chunk: int = 8192) -> dict:
+    """``gptq_quantize_layer(W, hessian(X), rows=rows)`` holding one d x d array.
+
+    For layers whose float64 H fits in host memory once but not the three or
+    four times the plain path needs (the OPT-175B fc2 layer: d = 49152, one
+    float64 H is 19.3 GB).  The steps are the same -- H = 2 sum x x^T
+    ([Tutorial] §二阶信息), damping by damp * mean(diag H) and the upper
+    Cholesky factor of H_d^-1 ([Card] 方法适配), the column sweep of the sampled
+    rows -- with H accumulated into one triangle of a Fortran-ordered array by
+    a symmetric rank-k library product per token chunk and factored in place
+    (``inverse_upper_cholesky_inplace``).  H no longer exists after the
+    factorisation, so each row's objective ||(w - w^) X^T||^2 is taken from X
+    directly.  Natural column order only (no act-order).
+
+    Returns codes/scales/zeros/What of the rows, ``row_loss`` [rows] and
+    ``loss`` (their sum), ``lambda``.
+    """
+    X = np.asarray(X)
+    n, d = X.shape
+    rows = np.asarray(rows, dtype=np.int64)
+    Wr = np.asarray(W, dtype=F64)[rows]
+    H = np.zeros((d, d), dtype=F64, order="F")
+    for t0 in range(0, n, chunk):
+        Xc = X[t0:t0 + chunk].astype(F64)
+        # Xc.T is a Fortran-ordered d x t view: H += 2 Xc^T Xc, upper triangle
+        syrk_upper_inplace(H, Xc.T, 2.0)
+    idx = np.arange(d)
+    lam = float(damp) * float(np.mean(H[idx, idx]))
+    H[idx, idx] += lam
+    U = inverse_upper_cholesky_inplace(H)
+    codes, scales, zeros, What, _ = gptq_sweep(Wr, U, bits, group, block)
+    del U, H
+    D = Wr - What
+    row_loss = np.zeros(rows.size, dtype=F64)
+    for t0 in range(0, n, chunk):
+        Y = D @ X[t0:t0 + chunk].astype(F64).T
+        row_loss += np.sum(Y * Y, axis=1)
+    return {
+        "codes": codes,
+        "scales": scales,
+        "zeros": zeros.astype(np.int64),
+        "What": What,
+        "row_loss": row_loss,
+        "loss": float(np.sum(row_loss)),
+        "lambda": lam,
     }
 
 

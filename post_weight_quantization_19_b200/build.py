@@ -5,6 +5,7 @@ Usage: python -m post_weight_quantization_19_b200.build [--verbose]
 
 from __future__ import annotations
 
+import concurrent.futures
 import os
 import shutil
 import subprocess
@@ -50,12 +51,13 @@ def build(force: bool = False, verbose: bool = False) -> str:
     ]
     if verbose:
         flags += ["-Xptxas", "-v"]
-    objs = []
-    for src in SOURCES:
-        obj = os.path.join(build_dir, src.replace(".cu", ".o"))
-        cmd = [nvcc(), *flags, "-c", os.path.join(CSRC, src), "-o", obj]
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+    objs = [os.path.join(build_dir, src.replace(".cu", ".o")) for src in SOURCES]
+    cmds = [[nvcc(), *flags, "-c", os.path.join(CSRC, src), "-o", obj]
+            for src, obj in zip(SOURCES, objs)]
+    # the translation units are independent: compile them side by side
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 1)) as ex:
+        for fut in [ex.submit(subprocess.run, c, check=True) for c in cmds]:
+            fut.result()
     tmp = LIB + ".tmp"
     subprocess.run([nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
                     *objs, "-o", tmp], check=True)

@@ -89,14 +89,31 @@ Layout layout(int64_t r, int64_t d, int group, int block, int options) {
   return L;
 }
 
-// Phase timing (optional).
+// Phase timing (optional).  The phase events are recorded on the solve's
+// stream -- as event-record nodes when the sequence replays as a CUDA graph --
+// and read after the call's final synchronisation.  t_timing is set only
+// around the enqueue of a gptq_quantize_layer call that times its phases (not
+// the no-alloc path, which creates nothing).
 bool g_timing = false;
 float g_phase_ms[4] = {0, 0, 0, 0};
 cudaEvent_t g_ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+int g_ev_device = -1;
+thread_local bool t_timing = false;
+
+int ensure_phase_events() {
+  int dev = 0;
+  GPTQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (g_ev_device != dev) {
+    for (auto &e : g_ev) e = nullptr;   // events of another device's context are not reused
+    g_ev_device = dev;
+  }
+  for (auto &e : g_ev)
+    if (!e) GPTQ_CUDA_TRY(cudaEventCreate(&e));
+  return GPTQ_OK;
+}
 
 int record(int i, cudaStream_t s) {
-  if (!g_timing) return GPTQ_OK;
-  if (!g_ev[i]) GPTQ_CUDA_TRY(cudaEventCreate(&g_ev[i]));
+  if (!t_timing) return GPTQ_OK;
   GPTQ_CUDA_TRY(cudaEventRecord(g_ev[i], s));
   return GPTQ_OK;
 }
@@ -111,6 +128,7 @@ struct GraphKey {
   int bits, group, block;
   float damp;
   int options;
+  bool timing;
   int device = -1;
   bool operator==(const GraphKey &o) const {
     return W == o.W && H == o.H && W_hat == o.W_hat && qweight == o.qweight &&
@@ -118,7 +136,7 @@ struct GraphKey {
            ws == o.ws && ws_bytes == o.ws_bytes && stream == o.stream && r == o.r &&
            d == o.d && bits == o.bits && group == o.group && block == o.block &&
            memcmp(&damp, &o.damp, sizeof(float)) == 0 && options == o.options &&
-           device == o.device;
+           timing == o.timing && device == o.device;
   }
 };
 
@@ -367,13 +385,30 @@ int enqueue_sweep(const SweepPlan &p, cudaStream_t st) {
 
 }  // namespace
 
+int check_layer_args(const float *W, int64_t r, int64_t d, const float *H, int bits, int group,
+                     int block, float damp, int options, const float *W_hat,
+                     const int32_t *qweight, const float *scales, const int32_t *zeros,
+                     const int32_t *g_idx, const uint8_t *codes) {
+  if (!valid_layer(r, d, bits, group, block)) return GPTQ_ERR_INVALID_ARG;
+  if (!(damp >= 0.f) || damp > 1e30f) return GPTQ_ERR_INVALID_ARG;
+  if (!valid_options(options)) return GPTQ_ERR_INVALID_ARG;
+  if (r == 0) return GPTQ_OK;   // nothing is read or written
+  if (!W || !H || !qweight || !scales || !zeros) return GPTQ_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(W) % 16 || reinterpret_cast<uintptr_t>(H) % 16 ||
+      (W_hat && reinterpret_cast<uintptr_t>(W_hat) % 16) ||
+      reinterpret_cast<uintptr_t>(qweight) % 4 || reinterpret_cast<uintptr_t>(scales) % 4 ||
+      reinterpret_cast<uintptr_t>(zeros) % 4 || (g_idx && reinterpret_cast<uintptr_t>(g_idx) % 16) ||
+      (codes && reinterpret_cast<uintptr_t>(codes) % 4))
+    return GPTQ_ERR_INVALID_ARG;
+  return GPTQ_OK;
+}
+
 int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int group, int block,
                    float damp, int options, float *W_hat, int32_t *qweight, float *scales,
                    int32_t *zeros, int32_t *g_idx, uint8_t *codes, double *loss, void *workspace,
                    size_t workspace_bytes, gptq_stream_t stream, bool plain) {
-  if (!valid_layer(r, d, bits, group, block)) return GPTQ_ERR_INVALID_ARG;
-  if (!(damp >= 0.f) || damp > 1e30f) return GPTQ_ERR_INVALID_ARG;
-  if (!valid_options(options)) return GPTQ_ERR_INVALID_ARG;
+  GPTQ_TRY(check_layer_args(W, r, d, H, bits, group, block, damp, options, W_hat, qweight, scales,
+                            zeros, g_idx, codes));
   const bool act_order = (options & GPTQ_ACT_ORDER) != 0;
   const int sym = (options & GPTQ_SYMMETRIC) ? 1 : 0;
   // with one group per row both rules take the parameters from the original row
@@ -382,14 +417,7 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
     if (loss) *loss = 0.0;
     return GPTQ_OK;
   }
-  if (!W || !H || !qweight || !scales || !zeros || !workspace) return GPTQ_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(W) % 16 || reinterpret_cast<uintptr_t>(H) % 16 ||
-      reinterpret_cast<uintptr_t>(workspace) % 256 ||
-      (W_hat && reinterpret_cast<uintptr_t>(W_hat) % 16) ||
-      reinterpret_cast<uintptr_t>(qweight) % 4 || reinterpret_cast<uintptr_t>(scales) % 4 ||
-      reinterpret_cast<uintptr_t>(zeros) % 4 || (g_idx && reinterpret_cast<uintptr_t>(g_idx) % 16) ||
-      (codes && reinterpret_cast<uintptr_t>(codes) % 4))
-    return GPTQ_ERR_INVALID_ARG;
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256) return GPTQ_ERR_INVALID_ARG;
   const Layout L = layout(r, d, group, block, options);
   if (workspace_bytes < L.total) return GPTQ_ERR_NO_MEMORY;
 
@@ -429,14 +457,13 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
   // hundred short kernels whose launch cost would otherwise pace the GPU.  The
   // first call of a configuration runs directly, the second is captured, later
   // ones replay.  Streams that cannot be captured run directly.
+  const bool timing = g_timing && !plain;
+  if (timing) GPTQ_TRY(ensure_phase_events());
   const GraphKey key{W, H, W_hat, qweight, scales, zeros, g_idx, codes, workspace,
-                     workspace_bytes, st, r, d, bits, group, block, damp, options};
-  int rc = GPTQ_OK;
-  if (g_timing || plain) {
-    rc = enqueue();
-  } else {
-    rc = run_graph_cached(key, st, enqueue);
-  }
+                     workspace_bytes, st, r, d, bits, group, block, damp, options, timing};
+  t_timing = timing;
+  const int rc = plain ? enqueue() : run_graph_cached(key, st, enqueue);
+  t_timing = false;
   if (rc != GPTQ_OK) return rc;
 
   double host_out[3] = {0, 0, 0};
@@ -444,8 +471,10 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
   GPTQ_CUDA_TRY(cudaMemcpyAsync(host_out, out, sizeof(host_out), cudaMemcpyDeviceToHost, st));
   GPTQ_CUDA_TRY(cudaMemcpyAsync(&host_status, status, sizeof(int), cudaMemcpyDeviceToHost, st));
   GPTQ_CUDA_TRY(cudaStreamSynchronize(st));
-  if (g_timing)
-    for (int i = 0; i < 4; ++i) cudaEventElapsedTime(&g_phase_ms[i], g_ev[i], g_ev[i + 1]);
+  if (timing)
+    for (int i = 0; i < 4; ++i)
+      if (cudaEventElapsedTime(&g_phase_ms[i], g_ev[i], g_ev[i + 1]) != cudaSuccess)
+        g_phase_ms[i] = -1.f;
   if (host_status != 0) return host_status;
   if (loss) *loss = host_out[0];
   return GPTQ_OK;

@@ -71,6 +71,7 @@ struct TcArgs {
   int trans_b;
   const int *status;
   int *dev_status;
+  int stall_after;   // self-test only: the producer stops after this many K steps (-1: never)
 };
 
 // The tensor core reads an fp32 operand in kind::tf32 as its top 19 bits
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int kb = 0; kb < nk; ++kb) {
         const int s = kb % RS;
         const uint32_t ph = (kb / RS) & 1;
-        if (*(volatile int *)&sh.abort) break;
+        if (*(volatile int *)&sh.abort || kb == g.stall_after) break;
         if (!mbar_wait_bounded(&sh.empty[s], ph ^ 1)) {
           fail_timeout(sh, g.dev_status);
           break;
@@ -446,6 +447,18 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
     set_last_error_msg(__FILE__, __LINE__, "GEMM operands not 16-byte aligned / K % 32 != 0");
     return GPTQ_ERR_INVALID_ARG;
   }
+  if (PlanRecorder *rec = plan_recorder()) {
+    char a[64], b[64], c[64];
+    rec->ref(g.A, a, sizeof a);
+    rec->ref(g.B, b, sizeof b);
+    rec->ref(g.C, c, sizeof c);
+    rec->line("G s=%d M=%d N=%d K=%d A=%s lda=%lld B=%s ldb=%lld C=%s ldc=%lld alpha=%g beta=%g "
+              "flags=%d tb=%d prio=%d\n",
+              plan_stream_index(stream), g.M, g.N, g.K, a, (long long)g.lda, b, (long long)g.ldb,
+              c, (long long)g.ldc, (double)g.alpha, (double)g.beta, g.flags, trans_b ? 1 : 0,
+              g.prio);
+    return GPTQ_OK;
+  }
   CUtensorMap ta, tb, tc;
   const CUtensorMapSwizzle kmaj = CU_TENSOR_MAP_SWIZZLE_128B;
   const CUtensorMapSwizzle mnmaj = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
@@ -459,11 +472,11 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
   static std::atomic<bool> attr[64] = {};
   if (const int rc = ensure_smem_attr(gemm_tc_kernel, SMEM_BYTES, attr)) return rc;
   TcArgs a{g.M, g.N, g.K, g.C, g.ldc, g.alpha, g.beta, g.flags, trans_b ? 1 : 0, g.status,
-           device_status_word()};
+           device_status_word(), g.stall_after};
   dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM);
   if (grid.y > 65535) return GPTQ_ERR_INVALID_ARG;
   count_launch();
-  const cudaError_t e = launch_pdl_prio(g.background, gemm_tc_kernel, grid, dim3(THREADS),
+  const cudaError_t e = launch_pdl_prio(g.prio, gemm_tc_kernel, grid, dim3(THREADS),
                                         SMEM_BYTES, stream, ta, tb, tc, a);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
@@ -474,3 +487,19 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
 }
 
 }  // namespace gptq
+
+// ---------------------------------------------------------------- self-test
+
+using namespace gptq;
+
+// A 128 x 128 x 256 product whose operand loads stop after two of its eight K
+// steps: the converter warps' and the MMA warp's bounded waits run out, the
+// kernel records GPTQ_ERR_TIMEOUT in the status word, frees its tensor memory
+// and returns.
+extern "C" int gptq_selftest_timeout(float *buf, gptq_stream_t stream) {
+  if (!buf || reinterpret_cast<uintptr_t>(buf) % 16) return GPTQ_ERR_INVALID_ARG;
+  float *A = buf, *B = buf + 128 * 256, *C = buf + 2 * 128 * 256;
+  GemmArgs g{128, 128, 256, A, 256, B, 128, C, 128, 1.f, 0.f, 0, nullptr};
+  g.stall_after = 2;
+  return launch_gemm(g, false, (cudaStream_t)stream);
+}

@@ -21,20 +21,22 @@ __device__ __forceinline__ void pdl_wait_then_release() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Scheduling priority of a launch: the layer sequence runs at the device's
-// greatest priority; work taken off its critical path (the background
-// products of the factorisation) at the least, so the SMs it frees go to the
-// critical path first.
-int launch_priority(bool background);
+// Scheduling priority of a launch, by level: 0 = the layer sequence's critical
+// path (the device's greatest priority), 1 = work the critical path will wait
+// for soon (the factorisation's trailing updates; the middle of the range), 2 =
+// work only the end of the factorisation waits for (the merge products that
+// assemble U; the least priority).  SMs that free up go to the higher level
+// first.
+int launch_priority(int level);
 
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl_prio(bool background, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+cudaError_t launch_pdl_prio(int level, void (*kernel)(KArgs...), dim3 grid, dim3 block,
                             size_t smem, cudaStream_t stream, Args &&...args) {
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   attr[1].id = cudaLaunchAttributePriority;
-  attr[1].val.priority = launch_priority(background);
+  attr[1].val.priority = launch_priority(level);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -48,7 +50,7 @@ cudaError_t launch_pdl_prio(bool background, void (*kernel)(KArgs...), dim3 grid
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t stream, Args &&...args) {
-  return launch_pdl_prio(false, kernel, grid, block, smem, stream, std::forward<Args>(args)...);
+  return launch_pdl_prio(0, kernel, grid, block, smem, stream, std::forward<Args>(args)...);
 }
 
 // The dynamic shared-memory limit of a kernel, raised once per device (the
@@ -104,7 +106,8 @@ struct GemmArgs {
   float alpha, beta;
   int flags;
   const int *status;  // skip the launch's work if *status != 0 (may be NULL)
-  bool background = false;   // off the critical path: least launch priority
+  int prio = 0;              // launch priority level (see launch_priority)
+  int stall_after = -1;      // self-test of the timeout path only (see gptq_selftest_timeout)
 };
 
 int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream);
@@ -115,16 +118,49 @@ int launch_act_order(const float *H, int64_t ld, int d, int *perm, int *inv, con
                      float *Hp, cudaStream_t stream);
 // inv[perm[p]] = p after checking that perm is a permutation (status set otherwise).
 int launch_check_perm(const int *perm, int d, int *inv, int *status, cudaStream_t stream);
-// Scratch of the factorisation: one h x m product per depth of the merge tree.
+// Scratch floats of the factorisation of a d x d matrix: the merge products of
+// non-square merge-tree nodes and, for wide layers, a copy of the outer panel.
 size_t factor_scratch_floats(int64_t d);
 // One diagonal block (nb <= 128, nb % 32 == 0) of H_d -> U in place (full block, zeros below).
 int launch_leaf(float *A, int64_t ld, int nb, int *status, cudaStream_t stream);
-// use_side: run the trailing updates and the merge products on two side streams
-// (created once per device, with their events); false keeps everything on
-// `stream`.
+// dst[rows x cols] = src[rows x cols] (fp32, row strides ldd / lds; all multiples of 4 floats).
+int launch_copy2d(float *dst, int64_t ldd, const float *src, int64_t lds, int64_t rows,
+                  int64_t cols, const int *status, cudaStream_t stream);
+// use_side: run the work off the critical path (trailing updates, merge
+// products) on side streams (created once per device, with their events);
+// false keeps everything on `stream`.
 int launch_factor(float *A, int64_t d, float *T1, int *status, cudaStream_t stream,
                   bool use_side);
 
+// ---- factorisation plan recording (a host-only diagnostic) ----
+// While a PlanRecorder is installed on the calling thread, launch_leaf,
+// launch_gemm and launch_copy2d validate their arguments and append one line
+// to it instead of launching, and launch_factor records its stream events
+// instead of creating them.  Pointers are written as a buffer name and an
+// element offset into one of the registered buffers.
+struct PlanRecorder {
+  char *out = nullptr;     // caller's text buffer (may be NULL: count only)
+  size_t cap = 0, used = 0;
+  const char *name[4] = {nullptr, nullptr, nullptr, nullptr};
+  const float *base[4] = {nullptr, nullptr, nullptr, nullptr};
+  size_t len[4] = {0, 0, 0, 0};   // floats
+  int nevents = 0;
+  void line(const char *fmt, ...);
+  // "name+offset" of p (or "?") into buf
+  void ref(const float *p, char *buf, size_t n) const;
+};
+PlanRecorder *plan_recorder();
+// stream handle -> index recorded in the plan (fake handles in recording mode)
+int plan_stream_index(cudaStream_t s);
+// outer block width of the factorisation of a d-wide layer (d: one block)
+int64_t factor_outer_cols(int64_t d);
+int launch_factor_plan(float *A, int64_t d, int64_t S, float *T1, bool use_side);
+
+// The argument checks of gptq_quantize_layer other than the workspace's.
+int check_layer_args(const float *W, int64_t r, int64_t d, const float *H, int bits, int group,
+                     int block, float damp, int options, const float *W_hat,
+                     const int32_t *qweight, const float *scales, const int32_t *zeros,
+                     const int32_t *g_idx, const uint8_t *codes);
 // gptq_quantize_layer; plain = true creates nothing (no CUDA graph, no second
 // stream or events) and launches every kernel directly on `stream`.
 int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int group, int block,

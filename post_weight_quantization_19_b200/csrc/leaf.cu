@@ -435,23 +435,23 @@ __device__ __forceinline__ bool col_factor_v1(real *S, real *vbuf) {
 // Node [off, off + N) of the shared-memory block.  N is a compile-time size
 // (32, 64, 96 or 128), so the recursion unfolds at compile time and uses no
 // call stack.
-template <int N, bool V2>
+template <int N, int V>
 __device__ __forceinline__ bool node_factor(real *S, real *T, real *vbuf, int off) {
   if constexpr (N <= BASE) {
-    if constexpr (V2)
+    if constexpr (V & 1)
       return col_factor<N>(S + off * LLD + off, vbuf);
     else
       return col_factor_v1<N>(S + off * LLD + off, vbuf);
   } else {
     constexpr int h = 32 * ((N / 32) / 2), m = N - h;
-    if (!node_factor<m, V2>(S, T, vbuf, off + h)) return false;
+    if (!node_factor<m, V>(S, T, vbuf, off + h)) return false;
     real *A11 = S + off * LLD + off;
     real *A12 = S + off * LLD + off + h;
     const real *U22 = S + (off + h) * LLD + off + h;
     // T (h x m): leading dimension m + 4, so rows stay 16-byte aligned and
     // the rows that neighbouring threads read transposed fall in different banks.
     constexpr int LT_ = m + 4;
-    if constexpr (V2) {
+    if constexpr ((V & 2) != 0) {
       smem_gemm_tc<h, m, m, LLD, LLD, LT_, true, false>(T, A12, U22, 1.f, 0.f);    // R12 = A12 U22^T
       smem_gemm_tc<h, h, m, LT_, LT_, LLD, true, true>(A11, T, T, -1.f, 1.f);      // A11 -= R12 R12^T
       smem_gemm_tc<h, m, m, LT_, LLD, LLD, false, false>(A12, T, U22, 1.f, 0.f);   // A12 = R12 U22
@@ -460,8 +460,8 @@ __device__ __forceinline__ bool node_factor(real *S, real *T, real *vbuf, int of
       smem_gemm_v1<h, h, m, LT_, LT_, LLD, true, true>(A11, T, T, -1.f, 1.f);
       smem_gemm_v1<h, m, m, LT_, LLD, LLD, false, false>(A12, T, U22, 1.f, 0.f);
     }
-    if (!node_factor<h, V2>(S, T, vbuf, off)) return false;
-    if constexpr (V2)
+    if (!node_factor<h, V>(S, T, vbuf, off)) return false;
+    if constexpr ((V & 2) != 0)
       smem_gemm_tc<h, m, h, LLD, LLD, LT_, false, false>(T, A11, A12, -1.f, 0.f);  // T = -U11 A12
     else
       smem_gemm_v1<h, m, h, LLD, LLD, LT_, false, false>(T, A11, A12, -1.f, 0.f);
@@ -474,7 +474,7 @@ __device__ __forceinline__ bool node_factor(real *S, real *T, real *vbuf, int of
   }
 }
 
-template <bool V2>
+template <int V>
 __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb, int *status) {
   extern __shared__ real lsm[];
   __shared__ real vbuf[4 * BASE];   // two published pairs of vectors
@@ -496,10 +496,10 @@ __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb,
   __syncthreads();
   bool ok;
   switch (nb) {
-    case 32: ok = node_factor<32, V2>(S, T, vbuf, 0); break;
-    case 64: ok = node_factor<64, V2>(S, T, vbuf, 0); break;
-    case 96: ok = node_factor<96, V2>(S, T, vbuf, 0); break;
-    default: ok = node_factor<128, V2>(S, T, vbuf, 0); break;
+    case 32: ok = node_factor<32, V>(S, T, vbuf, 0); break;
+    case 64: ok = node_factor<64, V>(S, T, vbuf, 0); break;
+    case 96: ok = node_factor<96, V>(S, T, vbuf, 0); break;
+    default: ok = node_factor<128, V>(S, T, vbuf, 0); break;
   }
   if (!ok) {
     if (threadIdx.x == 0) atomicCAS(status, 0, (int)GPTQ_ERR_NOT_PD);
@@ -516,28 +516,38 @@ __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb,
 
 }  // namespace
 
-// GPTQ_LEAF=1 selects the earlier leaf (FFMA products, one column per barrier)
-// for A/B timing (read once).
-static bool leaf_v1() {
-  static const bool on = [] {
-    const char *v = getenv("GPTQ_LEAF");
-    return v && v[0] == '1' && v[1] == 0;
+// Leaf form: bit 0 = two column steps per barrier, bit 1 = tensor-core
+// products (GPTQ_LEAF=0..3 while the forms are compared; default 3).
+static int leaf_form() {
+  static const int v = [] {
+    const char *e = getenv("GPTQ_LEAF");
+    return (e && e[0] >= '0' && e[0] <= '3' && e[1] == 0) ? e[0] - '0' : 3;
   }();
-  return on;
+  return v;
+}
+
+template <int V>
+static int launch_leaf_form(float *A, int64_t ld, int nb, int *status, cudaStream_t stream) {
+  static std::atomic<bool> attr[64] = {};
+  if (const int rc = ensure_smem_attr(leaf_kernel<V>, LEAF_SMEM, attr)) return rc;
+  GPTQ_LAUNCH_PDL(leaf_kernel<V>, dim3(1), dim3(LT), LEAF_SMEM, stream, A, ld, nb, status);
+  return GPTQ_OK;
 }
 
 int launch_leaf(float *A, int64_t ld, int nb, int *status, cudaStream_t stream) {
   if (nb <= 0 || nb > LB || nb % 32 != 0) return GPTQ_ERR_INVALID_ARG;
-  if (leaf_v1()) {
-    static std::atomic<bool> attr1[64] = {};
-    if (const int rc = ensure_smem_attr(leaf_kernel<false>, LEAF_SMEM, attr1)) return rc;
-    GPTQ_LAUNCH_PDL(leaf_kernel<false>, dim3(1), dim3(LT), LEAF_SMEM, stream, A, ld, nb, status);
+  if (PlanRecorder *rec = plan_recorder()) {
+    char a[64];
+    rec->ref(A, a, sizeof a);
+    rec->line("L s=%d A=%s ld=%lld nb=%d\n", plan_stream_index(stream), a, (long long)ld, nb);
     return GPTQ_OK;
   }
-  static std::atomic<bool> attr[64] = {};
-  if (const int rc = ensure_smem_attr(leaf_kernel<true>, LEAF_SMEM, attr)) return rc;
-  GPTQ_LAUNCH_PDL(leaf_kernel<true>, dim3(1), dim3(LT), LEAF_SMEM, stream, A, ld, nb, status);
-  return GPTQ_OK;
+  switch (leaf_form()) {
+    case 0: return launch_leaf_form<0>(A, ld, nb, status, stream);
+    case 1: return launch_leaf_form<1>(A, ld, nb, status, stream);
+    case 2: return launch_leaf_form<2>(A, ld, nb, status, stream);
+    default: return launch_leaf_form<3>(A, ld, nb, status, stream);
+  }
 }
 
 }  // namespace gptq

@@ -56,6 +56,11 @@ extern "C" int gptq_quantize_layer_noalloc(const float *W, int64_t r, int64_t d,
                                            int options, float *W_hat, int32_t *qweight,
                                            float *scales, int32_t *zeros, int32_t *g_idx,
                                            uint8_t *codes, double *loss, gptq_stream_t stream) {
+  // Every argument is checked before the size, so a bad argument reports
+  // GPTQ_ERR_INVALID_ARG whatever the layer's size.
+  const int bad = gptq::check_layer_args(W, r, d, H, bits, group, block, damp, options, W_hat,
+                                         qweight, scales, zeros, g_idx, codes);
+  if (bad != GPTQ_OK) return bad;
   const size_t need = gptq_quantize_workspace_bytes(r, d, bits, group, block, options);
   if (need == 0) return GPTQ_ERR_INVALID_ARG;
   if (need > gptq::kScratchBytes) {
@@ -72,8 +77,8 @@ extern "C" int gptq_quantize_layer_noalloc(const float *W, int64_t r, int64_t d,
   if (rc != GPTQ_OK) return rc;
   // The solve clears every part of its workspace that must start at zero, so
   // whatever an earlier call left in the array does not leak into this one.
-  // The plain form launches the kernels directly: no CUDA graph and no second
-  // stream are created on this path.
+  // The plain form launches the kernels directly: no CUDA graph, stream or
+  // event is created on this path (phase timing does not apply to it).
   return gptq::quantize_layer(W, r, d, H, bits, group, block, damp, options, W_hat, qweight,
                               scales, zeros, g_idx, codes, loss, scratch, gptq::kScratchBytes,
                               stream, true);

@@ -11,12 +11,13 @@
 // With U the upper Cholesky factor of H_d^-1, column j of every row does
 //   q = clamp(rint(w_j / s) + z, 0, 2^b - 1),  w^_j = s (q - z),
 //   e_j = (w_j - w^_j) / U_jj,  w_{j+1..} -= e_j U[j, j+1..].
-// Rows are independent.  One row of the current block belongs to L = B/32
-// neighbouring lanes of a warp, each holding 32 consecutive columns in
-// registers; the block of U sits in shared memory.  Column j is broadcast
-// from its lane by one shuffle, every lane of the row runs the quantiser on
-// it (the same value, so no divergence) and updates its 32 columns with
-// fused multiply-adds.  No inter-warp synchronisation at all.
+// Rows are independent.  One row of the current block belongs to L = B/CW
+// neighbouring lanes of a warp, each holding CW consecutive columns in
+// registers (CW = 16 for 128-column blocks: 8 lanes per row; 32 for narrower
+// blocks); the block of U sits in shared memory.  Column j is broadcast from
+// its lane by one shuffle, every lane of the row runs the quantiser on it
+// (the same value, so no divergence) and updates its CW columns with fused
+// multiply-adds.  No inter-warp synchronisation at all.
 #include <float.h>
 #include <stdlib.h>
 
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(32 * WARPS) sweep_block_kernel(SweepArgs a) {
   const bool start_here = g > B && (a.j0 % g) == 0;         // a long group starts at column 0
   const bool inherit = g < 0 || (g > B && !start_here);     // parameters set before this block
   const int gi0 = g < 0 ? 0 : a.j0 / (g > 0 ? g : 1);
-  const int ql = lane % L;        // this lane holds columns ql*32 .. ql*32+31 of the block
+  const int ql = lane % L;        // this lane holds columns ql*CW .. ql*CW+CW-1 of the block
   const int base = lane - ql;     // first lane of the row
   const int nsub = nc / CW;       // 32-column parts present in this block
   const bool mine = ql < nsub;
@@ -505,26 +506,12 @@ static int sweep_launch(const SweepArgs &a, cudaStream_t stream) {
   return GPTQ_OK;
 }
 
-// GPTQ_SWEEP_LANES=16 selects the 16-lane form of the 128-column block (read once).
-static bool sweep_lanes16() {
-  static const bool on = [] {
-    const char *v = getenv("GPTQ_SWEEP_LANES");
-    return v && v[0] == '1' && v[1] == '6' && v[2] == 0;
-  }();
-  return on;
-}
-
 template <bool VAR>
 static int sweep_launch_block(const SweepArgs &a, int block, cudaStream_t stream) {
   switch (block) {
     case 32: return sweep_launch<32, 1, VAR>(a, stream);
     case 64: return sweep_launch<32, 2, VAR>(a, stream);
-    case 128:
-      // Experimental form under measurement: 16 lanes of 8 columns per row in
-      // CTAs of 8 warps (twice the warps per SM for the same rows).
-      if (sweep_lanes16())
-        return sweep_launch<8, 16, VAR, 8>(a, stream);
-      return sweep_launch<SWEEP_CW, 128 / SWEEP_CW, VAR>(a, stream);
+    case 128: return sweep_launch<SWEEP_CW, 128 / SWEEP_CW, VAR>(a, stream);
     default: return GPTQ_ERR_INVALID_ARG;
   }
 }

@@ -307,3 +307,14 @@ def gptq_last_phase_ms() -> list[float]:
     buf = (ctypes.c_float * 4)()
     n = _abi.load().gptq_last_phase_ms(buf, 4)
     return [float(buf[i]) for i in range(n)]
+
+
+def gptq_factor_plan(d: int, outer_cols: int = 0, side_streams: bool = True) -> str:
+    """The factorisation's launches and stream events for a d x d H_d (no GPU used)."""
+    lib = _abi.load()
+    n = lib.gptq_factor_plan(d, outer_cols, int(side_streams), None, 0)
+    if n == 0:
+        raise GPTQError(1, "gptq_factor_plan: invalid arguments")
+    buf = ctypes.create_string_buffer(n)
+    lib.gptq_factor_plan(d, outer_cols, int(side_streams), buf, n)
+    return buf.value.decode()

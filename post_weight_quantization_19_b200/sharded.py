@@ -29,14 +29,14 @@ from .gptq import (GPTQError, gptq_factor, gptq_hessian_accumulate, gptq_quantiz
 def shard_range(count: int, rank: int, world: int) -> tuple[int, int]:
     """Contiguous slice [a, b) of ``count`` items for ``rank`` of ``world``.
 
-    Every rank but the last few gets ceil(count / world) items; ranks past the
-    end get an empty slice.
+    Balanced: the first ``count % world`` ranks get one item more than the
+    others, so every rank has at least one item whenever count >= world.
     """
     if world < 1 or not 0 <= rank < world or count < 0:
         raise ValueError("need 0 <= rank < world and count >= 0")
-    per = -(-count // world)
-    a = min(count, rank * per)
-    return a, min(count, a + per)
+    base, extra = divmod(count, world)
+    a = rank * base + min(rank, extra)
+    return a, a + base + (1 if rank < extra else 0)
 
 
 def token_shard(X: torch.Tensor, rank: int, world: int) -> torch.Tensor:
@@ -51,13 +51,15 @@ def row_shard(r: int, rank: int, world: int) -> tuple[int, int]:
 
 
 def _gather_rows(local: torch.Tensor, r: int, world: int, dist, group) -> torch.Tensor:
-    # all_gather needs equal shapes: pad each rank's rows to ceil(r / world)
+    # all_gather needs equal shapes: every rank pads its rows to ceil(r / world),
+    # and the padding is dropped rank by rank.
     per = -(-r // world)
     buf = local.new_zeros((per,) + tuple(local.shape[1:]))
     buf[:local.shape[0]] = local
     parts = [torch.empty_like(buf) for _ in range(world)]
     dist.all_gather(parts, buf, group=group)
-    return torch.cat(parts)[:r]
+    sizes = [b - a for a, b in (shard_range(r, k, world) for k in range(world))]
+    return torch.cat([p[:n] for p, n in zip(parts, sizes)])
 
 
 def _factor_on_root(H: torch.Tensor, rank: int, root: int, damp: float, act_order: bool,

@@ -40,8 +40,11 @@ def test_status_strings(lib):
 def test_workspace_query(lib):
     ws = lib.gptq_quantize_workspace_bytes
     base = ws(4096, 4096, 4, 128, 128, 0)
-    # working copy of W, superblock errors, codes, and the recursion scratch
-    assert base >= 4096 * 4096 * 4 + 4096 * 1024 * 4 + 4096 * 4096 + 2048 * 2048 * 4
+    # working copy of W, superblock errors and codes (every merge-tree node of a
+    # 4096-wide factor is square, so the factorisation needs no extra scratch)
+    assert base >= 4096 * 4096 * 4 + 4096 * 1024 * 4 + 4096 * 4096
+    # wide layers also hold a copy of the outer panel (d x 1024 floats)
+    assert ws(64, 49152, 3, 128, 128, 0) >= 64 * 49152 * 5 + 49152 * 1024 * 4
     assert ws(4096, 4096, 4, 128, 128, 1) >= base + 4096 * 4096 * 4   # permuted H
     assert base % 256 == 0
     for bad in [(16, 100, 4, -1, 128, 0),      # d % 32
@@ -127,6 +130,16 @@ def test_validation_returns_before_cuda(lib):
     assert lf(ctypes.c_void_p(4104), 16, 128, p, 64, p, None) == 1  # X alignment
     assert lf(p, 0, 128, p, 64, p, None) == 0                       # no tokens
     assert lf(p, 16, 128, p, 0, p, None) == 0                       # no outputs
+    st = lib.gptq_selftest_timeout
+    assert st(None, None) == 1 and st(ctypes.c_void_p(4100), None) == 1
+    na = lib.gptq_quantize_layer_noalloc
+    # a bad argument is reported as such even for a layer beyond the fixed scratch
+    assert na(p, 4096, 4096, p, 4, 128, 128, -1.0, 0, None, p, p, p, None, None,
+              ctypes.byref(loss), None) == 1
+    assert na(p, 4096, 4096, p, 4, 128, 128, 0.01, 0, None, None, p, p, None, None,
+              ctypes.byref(loss), None) == 1
+    assert na(p, 4096, 4096, p, 4, 128, 128, 0.01, 0, None, p, p, p, None, None,
+              ctypes.byref(loss), None) == 4
 
 
 def test_no_kernels_launched_on_cpu(lib):

@@ -105,6 +105,50 @@ def test_inverse_upper_cholesky_diagonal_and_residual():
     assert np.abs(res).max() < 1e-10
 
 
+def test_inplace_factor_closed_forms_and_residual():
+    # the 2x2 closed form and the diagonal case of the previous pins, now through
+    # the in-place LAPACK route; then the residual U^T U H_d = I on a layer.
+    a, b, c = 5.0, 2.0, 3.0
+    det = a * c - b * b
+    A = np.asfortranarray(np.array([[a, b], [-99.0, c]]))   # lower entry must be ignored
+    U = oracle.inverse_upper_cholesky_inplace(A)
+    expect = np.array([[np.sqrt(c / det), -b / np.sqrt(c * det)], [0.0, 1.0 / np.sqrt(c)]])
+    np.testing.assert_allclose(U, expect, rtol=1e-14)
+    assert np.shares_memory(U, A)
+    h = np.array([4.0, 9.0, 0.25, 16.0])
+    np.testing.assert_allclose(oracle.inverse_upper_cholesky_inplace(np.asfortranarray(np.diag(h))),
+                               np.diag(1.0 / np.sqrt(h)), rtol=1e-15)
+    X, _ = make_problem(4, 96, 2000, seed=6)
+    Hd, _ = oracle.dampen(oracle.hessian(X), 0.01)
+    U = oracle.inverse_upper_cholesky_inplace(np.asfortranarray(np.triu(Hd)))
+    assert np.all(np.tril(U, -1) == 0) and np.all(np.diag(U) > 0)
+    assert np.abs(U.T @ U @ Hd - np.eye(96)).max() < 1e-10
+    with pytest.raises(ValueError):
+        oracle.inverse_upper_cholesky_inplace(np.ascontiguousarray(Hd))
+
+
+@pytest.mark.parametrize("group", [-1, 32])
+def test_lowmem_rows_equal_the_plain_layer(group):
+    # The one-array route for very wide layers must give the plain route's codes
+    # and parameters; its per-row objective, taken from X, must equal
+    # 1/2 tr(D H D^T) of the plain route row by row.
+    X, W = make_problem(24, 160, 3000, seed=17)
+    rows = np.array([1, 5, 6, 19, 23])
+    H = oracle.hessian(X)
+    ref = oracle.gptq_quantize_layer(W, H, bits=3, group=group, block=32, damp=0.01, rows=rows)
+    got = oracle.gptq_quantize_rows_lowmem(X, W, rows, bits=3, group=group, block=32, damp=0.01,
+                                           chunk=1024)
+    np.testing.assert_array_equal(got["codes"], ref["codes"])
+    np.testing.assert_array_equal(got["zeros"], ref["zeros"])
+    np.testing.assert_allclose(got["scales"], ref["scales"], rtol=1e-12)
+    np.testing.assert_allclose(got["What"], ref["What"], rtol=1e-12, atol=1e-15)
+    assert abs(got["lambda"] - ref["lambda"]) <= 1e-12 * ref["lambda"]
+    D = np.asarray(W, float)[rows] - ref["What"]
+    per_row = 0.5 * np.einsum("ij,jk,ik->i", D, H, D)
+    np.testing.assert_allclose(got["row_loss"], per_row, rtol=1e-9)
+    assert abs(got["loss"] - ref["loss"]) <= 1e-9 * ref["loss"]
+
+
 # -------------------------------------------------------------- quantiser ---
 
 def _golden_quantizer(fname="quantizer_cases.txt"):
