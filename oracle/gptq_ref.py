@@ -125,7 +125,7 @@ def inverse_upper_cholesky(Hd: np.ndarray) -> np.ndarray:
 
 
 def _lapack64():
-    """dsyrk, dpotrf and dpotri of the OpenBLAS bundled with numpy, which takes
+    """dgemm, dpotrf and dpotri of the OpenBLAS bundled with numpy, which takes
     64-bit integers (matrices of 2^31 elements and more), or None if absent.
 
     Reference BLAS/LAPACK calling convention: every argument by reference,
@@ -141,7 +141,7 @@ def _lapack64():
         return None
     lib = ctypes.CDLL(found[0])
     try:
-        fns = {k: getattr(lib, f"scipy_{k}_64_") for k in ("dsyrk", "dpotrf", "dpotri")}
+        fns = {k: getattr(lib, f"scipy_{k}_64_") for k in ("dgemm", "dpotrf", "dpotri")}
     except AttributeError:
         return None
     for f in fns.values():
@@ -172,27 +172,27 @@ def _ref_args(*vals):
     return out
 
 
-def syrk_upper_inplace(C: np.ndarray, A: np.ndarray, alpha: float) -> None:
-    """C += alpha A A^T on the upper triangle (library dsyrk), in place.
+def gemm_acc_inplace(H: np.ndarray, j0: int, j1: int, Xc: np.ndarray, alpha: float) -> None:
+    """H[:j1, j0:j1] += alpha Xc[:, :j1]^T Xc[:, j0:j1] (library dgemm, in place).
 
-    C: Fortran-ordered float64 d x d; A: Fortran-ordered float64 d x k."""
+    H: Fortran-ordered float64 d x d; Xc: C-ordered float64 t x d."""
     import ctypes
 
-    if not (C.flags.f_contiguous and A.flags.f_contiguous and C.dtype == F64 and A.dtype == F64):
-        raise ValueError("syrk needs Fortran-ordered float64 operands")
-    d, k = A.shape
+    if not (H.flags.f_contiguous and Xc.flags.c_contiguous and H.dtype == F64
+            and Xc.dtype == F64):
+        raise ValueError("gemm needs a Fortran-ordered H and a C-ordered Xc (float64)")
+    t, d = Xc.shape
     L = _l64()
-    if L:
-        n_, k_, al, be, lda, ldc = _ref_args(d, k, float(alpha), 1.0, d, d)
-        L["dsyrk"](b"U", b"N", n_, k_, al, A.ctypes.data_as(ctypes.c_void_p), lda, be,
-                   C.ctypes.data_as(ctypes.c_void_p), ldc, ctypes.c_size_t(1), ctypes.c_size_t(1))
+    if not L:
+        H[:j1, j0:j1] += alpha * (Xc[:, :j1].T @ Xc[:, j0:j1])
         return
-    if d * d >= 2 ** 31:
-        raise RuntimeError("no 64-bit-index BLAS for a matrix this large")
-    from scipy.linalg import blas
-    out = blas.dsyrk(alpha, A, beta=1.0, c=C, trans=0, lower=0, overwrite_c=1)
-    if not np.shares_memory(out, C):
-        raise RuntimeError("dsyrk did not work in place")
+    # column-major view: Y = Xc^T is d x t with leading dimension d; the block is
+    # Y[:j1, :] Y[j0:j1, :]^T
+    m_, n_, k_, al, be, lda, ldb, ldc = _ref_args(j1, j1 - j0, t, float(alpha), 1.0, d, d, d)
+    base = Xc.ctypes.data
+    L["dgemm"](b"N", b"T", m_, n_, k_, al, ctypes.c_void_p(base), lda,
+               ctypes.c_void_p(base + 8 * j0), ldb, be, ctypes.c_void_p(H.ctypes.data + 8 * d * j0),
+               ldc, ctypes.c_size_t(1), ctypes.c_size_t(1))
 
 
 def _potr(name: str, A: np.ndarray) -> int:
@@ -461,9 +461,10 @@ def gptq_quantize_rows_lowmem(X: np.ndarray, W: np.ndarray, rows: np.ndarray, *,
     float64 H is 19.3 GB).  The steps are the same -- H = 2 sum x x^T
     ([Tutorial] §二阶信息), damping by damp * mean(diag H) and the upper
     Cholesky factor of H_d^-1 ([Card] 方法适配), the column sweep of the sampled
-    rows -- with H accumulated into one triangle of a Fortran-ordered array by
-    a symmetric rank-k library product per token chunk and factored in place
-    (``inverse_upper_cholesky_inplace``).  H no longer exists after the
+    rows -- with the upper triangle of H accumulated into a Fortran-ordered
+    array by float64 matrix products (a band of columns at a time per token
+    chunk; its diagonal checked against the column norms of X) and factored in
+    place (``inverse_upper_cholesky_inplace``).  H no longer exists after the
     factorisation, so each row's objective ||(w - w^) X^T||^2 is taken from X
     directly.  Natural column order only (no act-order).
 
@@ -475,14 +476,34 @@ def gptq_quantize_rows_lowmem(X: np.ndarray, W: np.ndarray, rows: np.ndarray, *,
     rows = np.asarray(rows, dtype=np.int64)
     Wr = np.asarray(W, dtype=F64)[rows]
     H = np.zeros((d, d), dtype=F64, order="F")
+    diag = np.zeros(d, dtype=F64)
+    band = 4096
     for t0 in range(0, n, chunk):
         Xc = X[t0:t0 + chunk].astype(F64)
-        # Xc.T is a Fortran-ordered d x t view: H += 2 Xc^T Xc, upper triangle
-        syrk_upper_inplace(H, Xc.T, 2.0)
+        diag += np.einsum("ij,ij->j", Xc, Xc)
+        # the upper triangle, a band of columns at a time: H[:j1, j0:j1] +=
+        # 2 Xc[:, :j1]^T Xc[:, j0:j1] (a float64 matrix product accumulated in place)
+        for j0 in range(0, d, band):
+            j1 = min(d, j0 + band)
+            gemm_acc_inplace(H, j0, j1, Xc, 2.0)
+    diag *= 2.0
     idx = np.arange(d)
+    if not np.allclose(H[idx, idx], diag, rtol=1e-12, atol=0.0):
+        raise RuntimeError("Hessian diagonal disagrees with the column norms")
     lam = float(damp) * float(np.mean(H[idx, idx]))
     H[idx, idx] += lam
     U = inverse_upper_cholesky_inplace(H)
+    # U^T U H_d e_j = e_j on a few columns, with H_d e_j = 2 X^T (X e_j) + lambda e_j
+    for j in (0, d // 3, d - 1):
+        v = np.zeros(d)
+        for t0 in range(0, n, chunk):
+            Xc = X[t0:t0 + chunk]
+            v += 2.0 * (Xc.T.astype(F64) @ Xc[:, j].astype(F64))
+        v[j] += lam
+        res = U.T @ (U @ v)
+        res[j] -= 1.0
+        if np.abs(res).max() > 1e-6:
+            raise np.linalg.LinAlgError(f"U^T U H_d e_{j} is off the unit vector by {np.abs(res).max():.2e}")
     codes, scales, zeros, What, _ = gptq_sweep(Wr, U, bits, group, block)
     del U, H
     D = Wr - What

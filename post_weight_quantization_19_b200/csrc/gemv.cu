@@ -141,6 +141,181 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS) gemv_kernel(GemvArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- the fold form
+// (no g_idx, x staged): per 32-code chunk (one group), with x_j the inputs,
+//   sum_j s (q_j - z) x_j = s (sum_j q_j x_j - z sum_j x_j),
+// so each code costs one bit operation that places it in the mantissa of
+// 2^23 (LOP3: (w & mask << off) | 0x4B000000 is the float 2^23 + q 2^off,
+// exact while q 2^off < 2^23), one subtraction of 2^23 and one fused
+// multiply-add with x_j 2^-off -- the staged copy of x carries that power of
+// two, so the product is exactly q_j x_j.  Codes whose offset is too high for
+// the exponent trick are read from the word shifted right once by FSH bits;
+// the two 3-bit codes that straddle words come from a funnel shift.  The sums
+// of x per chunk are staged too.  One warp per row; the grid holds one CTA per
+// SM with just enough warps that every warp takes the same number of rows.
+
+template <int BITS>
+struct CodeAt {
+  static constexpr int FSH = BITS == 8 ? 16 : 12;   // shift of the high codes
+  static constexpr int TOP = 23 - BITS;              // highest offset the trick takes
+  __host__ __device__ static constexpr int pos(int j) { return j * BITS; }
+  __host__ __device__ static constexpr int word(int j) { return pos(j) >> 5; }
+  __host__ __device__ static constexpr int off(int j) { return pos(j) & 31; }
+  __host__ __device__ static constexpr bool straddle(int j) { return off(j) + BITS > 32; }
+  // offset of the code in the value it is extracted from
+  __host__ __device__ static constexpr int eff(int j) {
+    return straddle(j) ? 0 : (off(j) <= TOP ? off(j) : off(j) - FSH);
+  }
+};
+
+__device__ __forceinline__ int xs_index(int k, int j) {   // swizzled float4 slots of a chunk
+  return k * 32 + ((((j >> 2) ^ (k & 7)) << 2) | (j & 3));
+}
+
+template <int BITS, int MB>
+__device__ __forceinline__ void fold_chunk(const uint32_t (&w)[BITS], const float *xs, int nchunk,
+                                           int k, float (&part)[MB], int m) {
+  using C = CodeAt<BITS>;
+  constexpr uint32_t mask = (1u << BITS) - 1u;
+  uint32_t wsh[BITS];
+#pragma unroll
+  for (int t = 0; t < BITS; ++t) wsh[t] = w[t] >> C::FSH;
+#pragma unroll
+  for (int i = 0; i < MB; ++i) part[i] = 0.f;
+#pragma unroll
+  for (int j4 = 0; j4 < 32; j4 += 4) {
+    float4 xv[MB];
+#pragma unroll
+    for (int i = 0; i < MB; ++i)
+      xv[i] = i < m ? *reinterpret_cast<const float4 *>(xs + (size_t)i * nchunk * 32 + xs_index(k, j4))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = j4 + jj;
+      uint32_t bits;
+      if (C::straddle(j))
+        bits = (__funnelshift_r(w[C::word(j)], w[C::word(j) + 1], C::off(j)) & mask) | 0x4B000000u;
+      else if (C::off(j) <= C::TOP)
+        bits = (w[C::word(j)] & (mask << C::off(j))) | 0x4B000000u;
+      else
+        bits = (wsh[C::word(j)] & (mask << C::eff(j))) | 0x4B000000u;
+      const float q = __uint_as_float(bits) - 8388608.f;   // q_j 2^eff, exact
+#pragma unroll
+      for (int i = 0; i < MB; ++i) {
+        const float xj = jj == 0 ? xv[i].x : jj == 1 ? xv[i].y : jj == 2 ? xv[i].z : xv[i].w;
+        part[i] = fmaf(q, xj, part[i]);
+      }
+    }
+  }
+}
+
+// Threads per CTA of the fold form: fewer for more vectors (registers).
+__host__ __device__ constexpr int fold_threads(int mb) { return mb <= 2 ? 1024 : (mb == 4 ? 512 : 256); }
+
+template <int BITS, int MB>
+__global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a) {
+  using C = CodeAt<BITS>;
+  constexpr int PF = 4;
+  extern __shared__ __align__(16) float fsm[];
+  const int nchunk = a.d / 32;
+  float *xs = fsm;                                   // [m][nchunk][32], swizzled, scaled
+  float *xsum = fsm + (size_t)a.m * nchunk * 32;     // [m][nchunk]
+  // stage x: thread per (vector, chunk)
+  for (int idx = threadIdx.x; idx < a.m * nchunk; idx += blockDim.x) {
+    const int i = idx / nchunk, k = idx - i * nchunk;
+    const float *src = a.x + (int64_t)i * a.d + k * 32;
+    float sum = 0.f;
+#pragma unroll
+    for (int j4 = 0; j4 < 32; j4 += 4) {
+      const float4 v = __ldg(reinterpret_cast<const float4 *>(src + j4));
+      sum += (v.x + v.y) + (v.z + v.w);
+      float4 o;
+      o.x = ldexpf(v.x, -C::eff(j4 + 0));
+      o.y = ldexpf(v.y, -C::eff(j4 + 1));
+      o.z = ldexpf(v.z, -C::eff(j4 + 2));
+      o.w = ldexpf(v.w, -C::eff(j4 + 3));
+      *reinterpret_cast<float4 *>(xs + (size_t)i * nchunk * 32 + xs_index(k, j4)) = o;
+    }
+    xsum[idx] = sum;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int64_t row0 = (int64_t)blockIdx.x * a.r / gridDim.x;
+  const int64_t row1 = (int64_t)(blockIdx.x + 1) * a.r / gridDim.x;
+  const int64_t wpr = (int64_t)nchunk * BITS;
+  for (int64_t row = row0 + warp; row < row1; row += nwarps) {
+    float acc[MB];
+#pragma unroll
+    for (int i = 0; i < MB; ++i) acc[i] = 0.f;
+    const uint32_t *qrow = a.qweight + row * wpr;
+    const float *srow = a.scales + row * a.G;
+    const int32_t *zrow = a.zeros + row * a.G;
+    for (int k0 = lane; k0 < nchunk; k0 += 32 * PF) {
+      uint32_t w[PF][BITS];
+#pragma unroll
+      for (int p = 0; p < PF; ++p) {
+        const int k = k0 + 32 * p;
+#pragma unroll
+        for (int t = 0; t < BITS; ++t) w[p][t] = k < nchunk ? __ldg(qrow + (int64_t)k * BITS + t) : 0u;
+      }
+#pragma unroll
+      for (int p = 0; p < PF; ++p) {
+        const int k = k0 + 32 * p;
+        if (k < nchunk) {
+          float part[MB];
+          fold_chunk<BITS, MB>(w[p], xs, nchunk, k, part, a.m);
+          const int gi = a.group > 0 ? (k * 32) / a.group : 0;
+          const float s = __ldg(srow + gi), z = (float)__ldg(zrow + gi);
+#pragma unroll
+          for (int i = 0; i < MB; ++i)
+            if (i < a.m) acc[i] = fmaf(s, fmaf(-z, xsum[i * nchunk + k], part[i]), acc[i]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < MB; ++i) {
+      float v = acc[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0 && i < a.m) a.y[(int64_t)i * a.r + row] = v;
+    }
+  }
+}
+
+// Shared memory of the fold form: staged x and its chunk sums.
+size_t fold_smem(const GemvArgs &a) { return (size_t)a.m * (a.d / 32) * 33 * sizeof(float); }
+constexpr size_t FOLD_SMEM_MAX = 220u << 10;
+
+template <int BITS, int MB>
+int gemv_launch_fold(const GemvArgs &a, cudaStream_t st) {
+  static std::atomic<bool> attr[64] = {};
+  if (const int rc = ensure_smem_attr(gemv_fold_kernel<BITS, MB>, FOLD_SMEM_MAX, attr)) return rc;
+  const size_t smem = fold_smem(a);
+  const int sms = num_sms();
+  // CTAs per SM: as many as the staged x allows, up to 2048 threads
+  int per_sm = (int)(FOLD_SMEM_MAX / (smem > 0 ? smem : 1));
+  const int by_threads = 2048 / fold_threads(MB);
+  per_sm = per_sm < 1 ? 1 : (per_sm > by_threads ? by_threads : per_sm);
+  int64_t ctas = (int64_t)sms * per_sm;
+  if (ctas > a.r) ctas = a.r;
+  // warps per CTA: the fewest that take every CTA's rows in whole rounds
+  const int64_t rows = (a.r + ctas - 1) / ctas;
+  const int max_w = fold_threads(MB) / 32;
+  const int64_t rounds = (rows + max_w - 1) / max_w;
+  const int warps = (int)((rows + rounds - 1) / rounds);
+  gemv_fold_kernel<BITS, MB><<<(unsigned)ctas, 32 * warps, smem, st>>>(a);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+template <int BITS>
+int gemv_launch_fold_m(const GemvArgs &a, cudaStream_t st) {
+  if (a.m <= 1) return gemv_launch_fold<BITS, 1>(a, st);
+  if (a.m <= 2) return gemv_launch_fold<BITS, 2>(a, st);
+  if (a.m <= 4) return gemv_launch_fold<BITS, 4>(a, st);
+  return gemv_launch_fold<BITS, GEMV_MAX_M>(a, st);
+}
+
 template <int BITS, int MB, bool SX>
 int gemv_launch_mb(const GemvArgs &a, cudaStream_t st) {
   const int64_t want = (a.r + GEMV_WARPS - 1) / GEMV_WARPS;
@@ -171,6 +346,7 @@ int gemv_launch_sx(const GemvArgs &a, cudaStream_t st) {
 
 template <int BITS>
 int gemv_launch(const GemvArgs &a, cudaStream_t st) {
+  if (!a.g_idx && fold_smem(a) <= FOLD_SMEM_MAX) return gemv_launch_fold_m<BITS>(a, st);
   const size_t staged = (size_t)a.m * (a.d / 32) * XPAD * sizeof(float);
   return staged <= GEMV_SMEM_MAX ? gemv_launch_sx<BITS, true>(a, st)
                                  : gemv_launch_sx<BITS, false>(a, st);

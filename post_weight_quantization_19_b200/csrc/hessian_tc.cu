@@ -25,9 +25,10 @@
 //    to nearest, so each TMEM accumulation chain is limited to 512 tokens and
 //    then folded into fp32 registers of the epilogue warps (double-buffered
 //    TMEM, so the tensor core keeps running while a chain is folded).
-//  * Persistent grid of one cluster per SM pair walking the tile list; all
-//    clusters sweep the tokens at the same pace, so the current X slab is
-//    shared through L2.
+//  * Persistent grid of one cluster per SM pair walking the tile list (in
+//    bands of 8 tile rows, column by column; see tile_coords); all clusters
+//    sweep the tokens at the same pace, so the current X slab is shared
+//    through L2.
 #include <mutex>
 
 #include "gptq_common.cuh"
@@ -176,12 +177,36 @@ __device__ __forceinline__ void umma_commit_pair_local(uint64_t *bar) {
 }
 
 // Pair tile t -> (P, J): the 256 x 256 output block with rows 256 P .. and
-// columns 256 J .., J >= P.
+// columns 256 J .., J >= P.  Tiles are ordered in bands of BAND tile rows;
+// inside a band column by column (J from the band's first row on), each
+// column's rows top to bottom.  The pairs walk the list in lockstep (tile t,
+// t + pairs, ...), so the tiles in flight at one time are about pairs / BAND
+// consecutive columns of one band: they read about BAND + pairs / BAND
+// distinct 256-feature panels of the current token slab between them instead
+// of one panel per tile, which keeps the traffic from HBM well below the
+// operand stream of the tensor cores on wide layers.
+constexpr int BAND = 8;
+
 __device__ __forceinline__ void tile_coords(int t, int nP, int nJ, int &P, int &J) {
-  for (P = 0; P < nP; ++P) {
-    const int cnt = nJ - P;
+  for (int P0 = 0; P0 < nP; P0 += BAND) {
+    const int hb = min(BAND, nP - P0);
+    // columns P0 .. P0 + hb - 1 hold 1 .. hb tiles, later columns hb each
+    const int tri = hb * (hb + 1) / 2;
+    const int cnt = tri + hb * (nJ - P0 - hb);
     if (t < cnt) {
-      J = P + t;
+      if (t < tri) {
+        int c = 0;
+        while (t >= c + 1) {
+          t -= c + 1;
+          ++c;
+        }
+        J = P0 + c;
+        P = P0 + t;
+      } else {
+        t -= tri;
+        J = P0 + hb + t / hb;
+        P = P0 + t % hb;
+      }
       return;
     }
     t -= cnt;

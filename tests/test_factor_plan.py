@@ -321,7 +321,7 @@ def _check(d, S, side, seeds=(0,), check_races=True):
 @pytest.mark.parametrize("d,S", [(512, 0), (608, 0), (1024, 256), (1152, 384), (1184, 512),
                                  (1280, 128)])
 def test_plan_with_side_streams_gives_U_in_any_allowed_order(d, S):
-    _check(d, S, True, seeds=(0, 1, 2))
+    _check(d, S, True, seeds=(0, 1))
 
 
 @pytest.mark.parametrize("d,S", [(608, 0), (1184, 512)])

@@ -101,17 +101,29 @@ def test_code_mismatches_sit_on_rounding_ties():
     # float64.  Where they differ, the value being rounded must have been within
     # a hair of a half-integer step on the oracle's side (after the first
     # mismatch a row's later columns see different compensation, so only each
-    # row's first mismatch is tested).  The first column of every row is put
-    # exactly on a tie (w = s (k + 1/2 - z)), which both sides must round the
-    # same way (to even).
+    # row's first mismatch is tested).  Column 0 of every row is put exactly on
+    # a tie that both precisions see: columns 1 and 2 pin the first group's
+    # range to [-z s, (7 - z) s] with s a power of two (the rest of the group
+    # lies inside it), so s and z come out exactly, and w_0 = s (k + 1/2 - z)
+    # is exact in fp32; both sides must round it to even.
     r, d, bits, group = 256, 1024, 3, 128
     X, W = make_problem(r, d, 8 * d, seed=306)
     H32 = oracle.hessian(X).astype(np.float32)
-    s0, z0 = oracle.quant_params(W[:, :group].astype(np.float64), bits)
-    k = np.clip(np.rint(W[:, 0] / s0 + z0), 0, (1 << bits) - 2)
-    W[:, 0] = (s0 * (k + 0.5 - z0)).astype(np.float32)
+    rng = np.random.default_rng(309)
+    s0 = np.float32(2.0 ** -5)
+    z0 = rng.integers(2, 6, size=r).astype(np.float32)
+    k = rng.integers(0, 7, size=r).astype(np.float32)
+    lo, hi = -z0 * s0, (7 - z0) * s0
+    W[:, 3:group] = np.clip(W[:, 3:group], 0.9 * lo[:, None], 0.9 * hi[:, None])
+    W[:, 1], W[:, 2] = lo, hi
+    W[:, 0] = s0 * (k + np.float32(0.5) - z0)
     got = gpu_layer(None, W, bits=bits, group=group, H32=H32)
     ref = oracle.gptq_quantize_layer(W, H32.astype(np.float64), bits=bits, group=group)
+    np.testing.assert_array_equal(ref["scales"][:, 0], s0)
+    np.testing.assert_array_equal(got["scales"][:, 0], s0)
+    # rint(k - z + 1/2) is the even one of k - z and k - z + 1
+    np.testing.assert_array_equal(ref["codes"][:, 0], np.where((k - z0) % 2 == 0, k, k + 1))
+    np.testing.assert_array_equal(got["codes"][:, 0], ref["codes"][:, 0])
     assert_codes_close(got["codes"], ref["codes"])
     # the value rounded at column j, in code units: t = w_j / s + z, with
     # w_j = w^_j + e_j U_jj (e_j = (w_j - w^_j) / U_jj)
@@ -128,7 +140,6 @@ def test_code_mismatches_sit_on_rounding_ties():
     print(f"exact ties {exact_ties}, rows with a mismatch {rows.size}/{r}, "
           f"largest distance of a first mismatch from a tie {worst:.2e} (code units)")
     assert exact_ties >= r   # the planted first-column ties (at least)
-    np.testing.assert_array_equal(got["codes"][:, 0], ref["codes"][:, 0])
     assert worst <= 1e-3, worst
 
 

@@ -3,10 +3,11 @@
 The GPU runs the whole layer in the launch configuration the benchmark times.
 Where the float64 Hessian fits on the host, the oracle computes H and U in
 full (rows are independent once U is fixed) and sweeps a seeded sample of rows.
-The OPT-175B fc2 layer (d = 49152: a float64 H alone is 19 GB) is checked
-through properties that hold at any size: sampled rows of H, the
-dequantisation and packing identities, and GPTQ's layer objective against
-round-to-nearest on sampled rows, both evaluated from X directly.
+The OPT-175B fc2 layer (d = 49152: a float64 H alone is 19 GB and the oracle
+needs minutes of host time for it) is compared with the oracle's result for 16
+seeded rows, stored by tests/golden/make_opt175b_fc2_rows.py from the same
+seeded inputs (checked by a fingerprint), plus sampled rows of H and the
+dequantisation and packing identities.
 """
 
 import numpy as np
@@ -72,12 +73,39 @@ def test_w3_8192(name):
     _check_sampled(name, nrows=32)
 
 
-def test_opt175b_fc2_properties():
-    wl = workload("opt175b_fc2_12288x49152")
-    X, W = workload_inputs(wl)
-    r, d = W.shape
-    import post_weight_quantization_19_b200 as g
+def _row_losses(W, What, X, chunk=4096):
+    # ||(w - w^) X^T||^2 per row, summed over token chunks in float64
+    D = np.asarray(W, np.float64) - np.asarray(What, np.float64)
+    out = np.zeros(D.shape[0])
+    for t in range(0, X.shape[0], chunk):
+        Y = D @ X[t:t + chunk].astype(np.float64).T
+        out += np.sum(Y * Y, axis=1)
+    return out
 
+
+def test_opt175b_fc2_matches_stored_oracle_rows():
+    # The OPT-175B fc2 layer (d = 49152) in the launch configuration the bench
+    # times, against the float64 oracle's result for 16 seeded rows, written by
+    # tests/golden/make_opt175b_fc2_rows.py from the same seeded inputs (the
+    # oracle's float64 H alone is 19 GB and its factorisation takes minutes).
+    import os
+
+    import post_weight_quantization_19_b200 as g
+    golden = os.path.join(os.path.dirname(__file__), "golden", "opt175b_fc2_rows.npz")
+    if not os.path.exists(golden):
+        pytest.skip("stored oracle rows not written yet")
+    ref = np.load(golden)
+    wl = workload("opt175b_fc2_12288x49152")
+    assert list(ref["config"]) == [wl.r, wl.d, wl.n, wl.bits, wl.group, wl.block, wl.seed]
+    X, W = workload_inputs(wl)
+    rows = ref["rows"]
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "make_rows", os.path.join(os.path.dirname(golden), "make_opt175b_fc2_rows.py"))
+    mk = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mk)
+    np.testing.assert_array_equal(mk.fingerprint(X, W, rows), ref["fingerprint"])
+    r, d = W.shape
     dev = torch.device("cuda")
     Xd = torch.from_numpy(X).to(dev)
     H = torch.zeros((d, d), dtype=torch.float32, device=dev)
@@ -85,8 +113,7 @@ def test_opt175b_fc2_properties():
     del Xd
     hrows = np.array([0, 777, d // 2, d - 1])
     Hs = H[torch.from_numpy(hrows).to(dev)].cpu().numpy()
-    Href = oracle.hessian_rows(X, hrows)
-    assert rel_fro(Hs, Href) <= H_REL_FRO
+    assert rel_fro(Hs, oracle.hessian_rows(X, hrows)) <= H_REL_FRO
     Wd = torch.from_numpy(W).to(dev)
     W_hat = torch.empty_like(Wd)
     codes = torch.empty((r, d), dtype=torch.uint8, device=dev)
@@ -95,7 +122,6 @@ def test_opt175b_fc2_properties():
                                 damp=wl.damp, W_hat=W_hat, codes=codes, g_idx=g_idx)
     torch.cuda.synchronize()
     del H
-    rows = np.sort(np.random.default_rng(wl.seed).choice(r, 8, replace=False))
     rt = torch.from_numpy(rows).to(dev)
     c = codes[rt].cpu().numpy()
     wh = W_hat[rt].cpu().numpy()
@@ -104,15 +130,20 @@ def test_opt175b_fc2_properties():
     q = res["qweight"][rt].cpu().numpy()
     gi = np.arange(d) // wl.group
     np.testing.assert_array_equal(g_idx.cpu().numpy(), gi)
-    assert c.max() <= (1 << wl.bits) - 1 and zr.min() >= 0 and zr.max() <= (1 << wl.bits) - 1
+    match = assert_codes_close(c, ref["codes"])
     np.testing.assert_array_equal(wh, sc[:, gi] * (c.astype(np.float32) - zr[:, gi].astype(np.float32)))
     np.testing.assert_array_equal(q, oracle.pack_rows(c, wl.bits))
-    # GPTQ's objective on the sampled rows against round-to-nearest, both from X
-    _, rtn_hat = oracle.rtn(W[rows], wl.bits, wl.group)
-    # ||D X^T||^2 is a sum over tokens, so it is taken over 4096-token chunks
-    lg = sum(oracle.layer_loss_direct(W[rows], wh, X[t:t + 4096]) for t in range(0, wl.n, 4096))
-    lr = sum(oracle.layer_loss_direct(W[rows], rtn_hat, X[t:t + 4096])
-             for t in range(0, wl.n, 4096))
-    assert lg < lr, (lg, lr)
+    # scales and zeros where every earlier code of the row agrees
+    mism = c != ref["codes"]
+    first_bad = np.where(mism.any(axis=1), mism.argmax(axis=1), d)
+    ok = (np.arange(d // wl.group) * wl.group)[None, :] <= first_bad[:, None]
+    assert np.all(np.abs(sc[ok] - ref["scales"][ok]) <= 1e-4 * np.abs(ref["scales"][ok]))
+    assert float(np.mean(zr[ok] == ref["zeros"][ok])) >= 0.999
+    # the objective of each sampled row, from X, against the oracle's
+    lg = _row_losses(W[rows], wh, X)
+    rel = np.abs(lg - ref["row_loss"]) / ref["row_loss"]
+    assert rel.max() <= LOSS_REL, rel
+    assert abs(lg.sum() - ref["row_loss"].sum()) <= LOSS_REL * ref["row_loss"].sum()
     assert np.isfinite(res["loss"]) and res["loss"] > 0
-    print(f"opt175b fc2: sampled-row objective GPTQ {lg:.4g} vs RTN {lr:.4g}")
+    print(f"opt175b fc2: codes {match:.6f} identical on {len(rows)} rows, row objective "
+          f"within {rel.max():.2e} of the oracle")

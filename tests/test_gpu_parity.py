@@ -418,9 +418,11 @@ def test_dequant_gemv_matches_oracle(case):
 @pytest.mark.parametrize("d,m,bits", [(4096, 8, 4), (16384, 2, 3), (8192, 8, 4), (65536, 1, 2),
                                       (2048, 5, 8)])
 def test_dequant_gemv_staged_and_direct_x(d, m, bits):
-    # x is staged in shared memory when m * d * 4.5 bytes fit in 200 KB and read
-    # from global memory otherwise ((8192, 8) and (65536, 1)); both give the
-    # float64 oracle's product on random packed rows.
+    # Without g_idx the kernel folds the zero point out of each 32-code chunk
+    # and stages x (scaled per code position) with its chunk sums when
+    # m * d * 33/8 floats fit in 220 KB; otherwise x is read from global memory
+    # ((8192, 8) and (65536, 1)).  Both give the float64 oracle's product on
+    # random packed rows.
     import post_weight_quantization_19_b200 as g
     r, group = 67, 128
     rng = np.random.default_rng(d + m)
@@ -524,33 +526,19 @@ def test_chain_of_layers_matches_oracle():
             assert rel_fro(xin, rf["inputs"]) <= 2e-3, k
 
 
-def test_dequant_gemv_full_layer_bandwidth():
-    # The 4096 x 4096 4-bit group-128 layer at batch 1: parity on all rows and the
-    # achieved read bandwidth (packed codes + scales + zeros + x) printed.
+def _time_gemv(args, reps=20):
+    # reps launches replayed as one CUDA graph: the kernel's time, not the binding's
     import post_weight_quantization_19_b200 as g
-    r = d = 4096
-    rng = np.random.default_rng(7)
-    codes = rng.integers(0, 16, size=(r, d), dtype=np.uint8)
-    qweight = oracle.pack_rows(codes, 4)
-    scales = (rng.random((r, d // 128)) * 0.01 + 1e-3).astype(np.float32)
-    zeros = rng.integers(0, 16, size=(r, d // 128)).astype(np.int32)
-    x = rng.standard_normal((1, d)).astype(np.float32)
-    qd, sd, zd, xd = (torch.from_numpy(a).cuda() for a in (qweight, scales, zeros, x))
-    y = g.gptq_dequant_gemv(qd, sd, zd, xd, 4, 128)
-    ref = oracle.dequant_gemv(qweight, scales, zeros, 4, 128, x)
-    torch.cuda.synchronize()
-    assert np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max() <= 1e-5
-    # 50 launches replayed as one CUDA graph: the kernel's time, not the binding's
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         for _ in range(3):
-            g.gptq_dequant_gemv(qd, sd, zd, xd, 4, 128, y=y)
+            g.gptq_dequant_gemv(*args)
     torch.cuda.current_stream().wait_stream(s)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        for _ in range(50):
-            g.gptq_dequant_gemv(qd, sd, zd, xd, 4, 128, y=y)
+        for _ in range(reps):
+            g.gptq_dequant_gemv(*args)
     graph.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -558,11 +546,46 @@ def test_dequant_gemv_full_layer_bandwidth():
     graph.replay()
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / 50
-    assert np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max() <= 1e-5
-    nbytes = qweight.nbytes + scales.nbytes + zeros.nbytes + x.nbytes + r * 4
-    print(f"dequant_gemv 4096x4096 4-bit g128 m=1: {ms * 1e3:.2f} us, {nbytes / ms / 1e6:.0f} GB/s")
+    return e0.elapsed_time(e1) / reps
 
+
+@pytest.mark.parametrize("r,d,bits", [(4096, 4096, 4), (12288, 49152, 3)])
+def test_dequant_gemv_full_layer_bandwidth(r, d, bits):
+    # A whole layer at batch 1 (the 4096 x 4096 4-bit layer, and the OPT-175B
+    # fc2 shape at 3 bits: 226 MB of codes, larger than L2): parity on sampled
+    # rows, and the achieved read bandwidth (codes + scales + zeros + x + y)
+    # printed against the measured HBM copy rate.
+    import json
+    import os
+
+    import post_weight_quantization_19_b200 as g
+    group = 128
+    rng = np.random.default_rng(r + d)
+    codes = rng.integers(0, 1 << bits, size=(r, d), dtype=np.uint8)
+    qweight = oracle.pack_rows(codes, bits)
+    del codes
+    scales = (rng.random((r, d // group)) * 0.01 + 1e-3).astype(np.float32)
+    zeros = rng.integers(0, 1 << bits, size=(r, d // group)).astype(np.int32)
+    x = rng.standard_normal((1, d)).astype(np.float32)
+    qd, sd, zd, xd = (torch.from_numpy(a).cuda() for a in (qweight, scales, zeros, x))
+    y = g.gptq_dequant_gemv(qd, sd, zd, xd, bits, group)
+    torch.cuda.synchronize()
+    rows = np.sort(rng.choice(r, 64, replace=False))
+    ref = oracle.dequant_gemv(qweight[rows], scales[rows], zeros[rows], bits, group, x)
+    assert np.abs(y.cpu().numpy()[:, rows] - ref).max() / np.abs(ref).max() <= 1e-5
+    ms = _time_gemv((qd, sd, zd, xd, bits, group, None, y))
+    assert np.abs(y.cpu().numpy()[:, rows] - ref).max() / np.abs(ref).max() <= 1e-5
+    nbytes = qweight.nbytes + scales.nbytes + zeros.nbytes + x.nbytes + r * 4
+    peak = 6539.5
+    try:
+        with open(os.path.join(os.path.dirname(os.path.dirname(__file__)),
+                               "MEASURED_PEAKS.json")) as f:
+            peak = float(json.load(f)["hbm_gbs"])
+    except (OSError, KeyError, ValueError):
+        pass
+    gbs = nbytes / ms / 1e6
+    print(f"dequant_gemv {r}x{d} {bits}-bit g{group} m=1: {ms * 1e3:.2f} us, {gbs:.0f} GB/s "
+          f"= {gbs / peak:.3f} of {peak:.0f} GB/s")
 
 
 @pytest.mark.parametrize("factor_once", [True, False])
