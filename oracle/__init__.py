@@ -17,7 +17,7 @@ from .gptq_ref import (  # noqa: F401
     hessian,
     hessian_rows,
     inverse_upper_cholesky,
-    inverse_upper_cholesky_inplace,
+    inverse_upper_cholesky_lowmem,
     layer_loss,
     layer_loss_direct,
     pack_rows,

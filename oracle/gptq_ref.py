@@ -125,7 +125,7 @@ def inverse_upper_cholesky(Hd: np.ndarray) -> np.ndarray:
 
 
 def _lapack64():
-    """dgemm, dpotrf and dpotri of the OpenBLAS bundled with numpy, which takes
+    """dgemm of the OpenBLAS bundled with numpy, which takes
     64-bit integers (matrices of 2^31 elements and more), or None if absent.
 
     Reference BLAS/LAPACK calling convention: every argument by reference,
@@ -141,7 +141,7 @@ def _lapack64():
         return None
     lib = ctypes.CDLL(found[0])
     try:
-        fns = {k: getattr(lib, f"scipy_{k}_64_") for k in ("dgemm", "dpotrf", "dpotri")}
+        fns = {k: getattr(lib, f"scipy_{k}_64_") for k in ("dgemm",)}
     except AttributeError:
         return None
     for f in fns.values():
@@ -195,54 +195,30 @@ def gemm_acc_inplace(H: np.ndarray, j0: int, j1: int, Xc: np.ndarray, alpha: flo
                ldc, ctypes.c_size_t(1), ctypes.c_size_t(1))
 
 
-def _potr(name: str, A: np.ndarray) -> int:
-    import ctypes
+def inverse_upper_cholesky_lowmem(box: list) -> np.ndarray:
+    """``inverse_upper_cholesky`` of a d x d H_d held once, for very large d.
 
-    d = A.shape[0]
-    L = _l64()
-    if L:
-        info = ctypes.c_int64(0)
-        n_, lda = _ref_args(d, d)
-        L[name](b"U", n_, A.ctypes.data_as(ctypes.c_void_p), lda, ctypes.byref(info),
-                ctypes.c_size_t(1))
-        return int(info.value)
-    if d * d >= 2 ** 31:
-        raise RuntimeError("no 64-bit-index LAPACK for a matrix this large")
-    from scipy.linalg import lapack
-    if name == "dpotrf":
-        c, info = lapack.dpotrf(A, lower=0, clean=0, overwrite_a=1)
-    else:
-        c, info = lapack.dpotri(A, lower=0, overwrite_c=1)
-    if not np.shares_memory(c, A):
-        raise RuntimeError(f"{name} did not work in place")
-    return int(info)
-
-
-def inverse_upper_cholesky_inplace(Hd: np.ndarray) -> np.ndarray:
-    """``inverse_upper_cholesky`` in the storage of Hd, for H too large to copy.
-
-    Hd must be float64 in Fortran order with its upper triangle filled (the
-    strictly lower triangle is ignored).  The same definition -- invert, then
-    take the Cholesky factor of the inverse -- with each step a LAPACK routine
-    working in place: the Cholesky factor of Hd (potrf), the inverse from that
-    factor (potri), and the upper Cholesky factor of the inverse (potrf, which
-    returns U with Hd^-1 = U^T U).  Returns U (the same storage) with the
-    strictly lower triangle zeroed.
+    ``box`` = [Hd]: Hd float64 in Fortran order with its upper triangle filled
+    (the strictly lower triangle is ignored); the box is emptied so that Hd can
+    be released as soon as it is no longer needed.  The same definition --
+    invert, then take the Cholesky factor of the inverse -- with each step a
+    LAPACK routine of PyTorch's CPU build: the Cholesky factor of Hd, the
+    inverse from that factor (cholesky_inverse), and the upper Cholesky factor
+    of the inverse.  At most two d x d arrays are alive at any time.
     """
+    import torch
+
+    Hd = box.pop()
     if Hd.dtype != F64 or not Hd.flags.f_contiguous:
         raise ValueError("Hd must be a Fortran-ordered float64 array")
-    for step, name in (("potrf of H_d", "dpotrf"), ("potri", "dpotri"),
-                       ("potrf of H_d^-1", "dpotrf")):
-        info = _potr(name, Hd)
-        if info != 0:
-            raise np.linalg.LinAlgError(f"{step}: info {info}")
-    d = Hd.shape[0]
-    for j0 in range(0, d, 4096):   # zero the strictly lower triangle, a band of columns at a time
-        blk = Hd[:, j0:j0 + 4096]
-        r = np.arange(d)[:, None]
-        c = np.arange(j0, min(d, j0 + 4096))[None, :]
-        blk[r > c] = 0.0
-    return Hd
+    # Hd.T is C-ordered with the lower triangle filled
+    L = torch.linalg.cholesky(torch.from_numpy(Hd.T), upper=False)
+    del Hd
+    Hinv = torch.cholesky_inverse(L, upper=False)
+    del L
+    U = torch.linalg.cholesky(Hinv, upper=True)
+    del Hinv
+    return U.numpy()
 
 
 # ---------------------------------------------------------------------------
@@ -463,8 +439,9 @@ def gptq_quantize_rows_lowmem(X: np.ndarray, W: np.ndarray, rows: np.ndarray, *,
     Cholesky factor of H_d^-1 ([Card] 方法适配), the column sweep of the sampled
     rows -- with the upper triangle of H accumulated into a Fortran-ordered
     array by float64 matrix products (a band of columns at a time per token
-    chunk; its diagonal checked against the column norms of X) and factored in
-    place (``inverse_upper_cholesky_inplace``).  H no longer exists after the
+    chunk; its diagonal checked against the column norms of X) and factored
+    with at most two d x d arrays alive (``inverse_upper_cholesky_lowmem``);
+    U^T U H_d e_j = e_j is checked on three columns.  H no longer exists after the
     factorisation, so each row's objective ||(w - w^) X^T||^2 is taken from X
     directly.  Natural column order only (no act-order).
 
@@ -492,7 +469,9 @@ def gptq_quantize_rows_lowmem(X: np.ndarray, W: np.ndarray, rows: np.ndarray, *,
         raise RuntimeError("Hessian diagonal disagrees with the column norms")
     lam = float(damp) * float(np.mean(H[idx, idx]))
     H[idx, idx] += lam
-    U = inverse_upper_cholesky_inplace(H)
+    box = [H]
+    del H
+    U = inverse_upper_cholesky_lowmem(box)
     # U^T U H_d e_j = e_j on a few columns, with H_d e_j = 2 X^T (X e_j) + lambda e_j
     for j in (0, d // 3, d - 1):
         v = np.zeros(d)
@@ -505,7 +484,7 @@ def gptq_quantize_rows_lowmem(X: np.ndarray, W: np.ndarray, rows: np.ndarray, *,
         if np.abs(res).max() > 1e-6:
             raise np.linalg.LinAlgError(f"U^T U H_d e_{j} is off the unit vector by {np.abs(res).max():.2e}")
     codes, scales, zeros, What, _ = gptq_sweep(Wr, U, bits, group, block)
-    del U, H
+    del U
     D = Wr - What
     row_loss = np.zeros(rows.size, dtype=F64)
     for t0 in range(0, n, chunk):

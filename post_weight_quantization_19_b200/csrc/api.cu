@@ -114,7 +114,9 @@ int ensure_phase_events() {
 
 int record(int i, cudaStream_t s) {
   if (!t_timing) return GPTQ_OK;
-  GPTQ_CUDA_TRY(cudaEventRecord(g_ev[i], s));
+  // "external": under stream capture this becomes an event-record node of the
+  // graph (a plain record would only become a dependency edge)
+  GPTQ_CUDA_TRY(cudaEventRecordWithFlags(g_ev[i], s, cudaEventRecordExternal));
   return GPTQ_OK;
 }
 

@@ -521,7 +521,7 @@ __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb,
 static int leaf_form() {
   static const int v = [] {
     const char *e = getenv("GPTQ_LEAF");
-    return (e && e[0] >= '0' && e[0] <= '3' && e[1] == 0) ? e[0] - '0' : 3;
+    return (e && e[0] >= '0' && e[0] <= '3' && e[1] == 0) ? e[0] - '0' : 0;
   }();
   return v;
 }

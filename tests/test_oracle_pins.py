@@ -105,26 +105,26 @@ def test_inverse_upper_cholesky_diagonal_and_residual():
     assert np.abs(res).max() < 1e-10
 
 
-def test_inplace_factor_closed_forms_and_residual():
+def test_lowmem_factor_closed_forms_and_residual():
     # the 2x2 closed form and the diagonal case of the previous pins, now through
-    # the in-place LAPACK route; then the residual U^T U H_d = I on a layer.
+    # the low-memory route; then the residual U^T U H_d = I on a layer.
     a, b, c = 5.0, 2.0, 3.0
     det = a * c - b * b
-    A = np.asfortranarray(np.array([[a, b], [-99.0, c]]))   # lower entry must be ignored
-    U = oracle.inverse_upper_cholesky_inplace(A)
+    box = [np.asfortranarray(np.array([[a, b], [-99.0, c]]))]   # lower entry must be ignored
+    U = oracle.inverse_upper_cholesky_lowmem(box)
+    assert box == []
     expect = np.array([[np.sqrt(c / det), -b / np.sqrt(c * det)], [0.0, 1.0 / np.sqrt(c)]])
     np.testing.assert_allclose(U, expect, rtol=1e-14)
-    assert np.shares_memory(U, A)
     h = np.array([4.0, 9.0, 0.25, 16.0])
-    np.testing.assert_allclose(oracle.inverse_upper_cholesky_inplace(np.asfortranarray(np.diag(h))),
+    np.testing.assert_allclose(oracle.inverse_upper_cholesky_lowmem([np.asfortranarray(np.diag(h))]),
                                np.diag(1.0 / np.sqrt(h)), rtol=1e-15)
     X, _ = make_problem(4, 96, 2000, seed=6)
     Hd, _ = oracle.dampen(oracle.hessian(X), 0.01)
-    U = oracle.inverse_upper_cholesky_inplace(np.asfortranarray(np.triu(Hd)))
+    U = oracle.inverse_upper_cholesky_lowmem([np.asfortranarray(np.triu(Hd))])
     assert np.all(np.tril(U, -1) == 0) and np.all(np.diag(U) > 0)
     assert np.abs(U.T @ U @ Hd - np.eye(96)).max() < 1e-10
     with pytest.raises(ValueError):
-        oracle.inverse_upper_cholesky_inplace(np.ascontiguousarray(Hd))
+        oracle.inverse_upper_cholesky_lowmem([np.ascontiguousarray(Hd)])
 
 
 @pytest.mark.parametrize("group", [-1, 32])
