@@ -89,11 +89,11 @@ Layout layout(int64_t r, int64_t d, int group, int block, int options) {
   return L;
 }
 
-// Phase timing (optional).  The phase events are recorded on the solve's
-// stream -- as event-record nodes when the sequence replays as a CUDA graph --
-// and read after the call's final synchronisation.  t_timing is set only
-// around the enqueue of a gptq_quantize_layer call that times its phases (not
-// the no-alloc path, which creates nothing).
+// Phase timing (optional).  The solve replays as four CUDA graphs, one per
+// phase, and the phase events are recorded on the solve's stream between them
+// (never inside a capture), then read after the call's final synchronisation.
+// t_timing is set only around a gptq_quantize_layer call that times its phases
+// (not the no-alloc path, which creates nothing).
 bool g_timing = false;
 float g_phase_ms[4] = {0, 0, 0, 0};
 cudaEvent_t g_ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
@@ -114,9 +114,7 @@ int ensure_phase_events() {
 
 int record(int i, cudaStream_t s) {
   if (!t_timing) return GPTQ_OK;
-  // "external": under stream capture this becomes an event-record node of the
-  // graph (a plain record would only become a dependency edge)
-  GPTQ_CUDA_TRY(cudaEventRecordWithFlags(g_ev[i], s, cudaEventRecordExternal));
+  GPTQ_CUDA_TRY(cudaEventRecord(g_ev[i], s));
   return GPTQ_OK;
 }
 
@@ -130,7 +128,7 @@ struct GraphKey {
   int bits, group, block;
   float damp;
   int options;
-  bool timing;
+  int segment;   // phase of the solve this graph replays
   int device = -1;
   bool operator==(const GraphKey &o) const {
     return W == o.W && H == o.H && W_hat == o.W_hat && qweight == o.qweight &&
@@ -138,7 +136,7 @@ struct GraphKey {
            ws == o.ws && ws_bytes == o.ws_bytes && stream == o.stream && r == o.r &&
            d == o.d && bits == o.bits && group == o.group && block == o.block &&
            memcmp(&damp, &o.damp, sizeof(float)) == 0 && options == o.options &&
-           timing == o.timing && device == o.device;
+           segment == o.segment && device == o.device;
   }
 };
 
@@ -153,7 +151,7 @@ struct GraphEntry {
 std::mutex g_graph_mu;
 std::vector<GraphEntry> g_graphs;
 uint64_t g_graph_clock = 0;
-constexpr size_t kMaxGraphs = 16;
+constexpr size_t kMaxGraphs = 32;
 
 template <class F>
 int run_graph_cached(GraphKey key, cudaStream_t st, F &&enqueue) {
@@ -270,21 +268,30 @@ namespace {
 // Phases 0-1 on `st`: lambda = damp * mean(diag H), the act-order permutation
 // (perm, inv and the permuted H_d in Hp), then U in place of H_d.  *U is set to
 // the matrix that holds U (H, or Hp under act-order).
+// Phase 0: lambda = damp * mean(diag H) and, under act-order, the permutation
+// (perm, inv) and the permuted H_d in Hp.  Returns the matrix to factor (H, or
+// Hp under act-order).
+float *enqueue_damp(float *H, int64_t d, float damp, bool act_order, int *perm, int *inv,
+                    float *lambda, float *Hp, cudaStream_t st, int *rc) {
+  const int di = (int)d;
+  if (act_order) {
+    *rc = launch_damp(H, d, di, damp, false, lambda, st);
+    if (*rc == GPTQ_OK) *rc = launch_act_order(H, d, di, perm, inv, lambda, Hp, st);
+    return Hp;
+  }
+  *rc = launch_damp(H, d, di, damp, true, lambda, st);
+  return H;
+}
+
+// Phases 0-1 on `st`: damping / act-order, then U in place of H_d.  *U is set
+// to the matrix that holds U (H, or Hp under act-order).
 int enqueue_factor(float *H, int64_t d, float damp, bool act_order, int *perm, int *inv,
                    float *lambda, float *Hp, float *T1, int *status, cudaStream_t st,
                    bool use_side, float **U) {
-  const int di = (int)d;
-  float *Hf = H;
-  if (act_order) {
-    GPTQ_TRY(launch_damp(H, d, di, damp, false, lambda, st));
-    GPTQ_TRY(launch_act_order(H, d, di, perm, inv, lambda, Hp, st));
-    Hf = Hp;
-  } else {
-    GPTQ_TRY(launch_damp(H, d, di, damp, true, lambda, st));
-  }
-  GPTQ_TRY(record(1, st));
+  int rc = GPTQ_OK;
+  float *Hf = enqueue_damp(H, d, damp, act_order, perm, inv, lambda, Hp, st, &rc);
+  GPTQ_TRY(rc);
   GPTQ_TRY(launch_factor(Hf, d, T1, status, st, use_side));
-  GPTQ_TRY(record(2, st));
   *U = Hf;
   return GPTQ_OK;
 }
@@ -361,8 +368,12 @@ int enqueue_sweep(const SweepPlan &p, cudaStream_t st) {
       GPTQ_TRY(launch_gemm(g, false, st));
     }
   }
-  GPTQ_TRY(record(3, st));
+  return GPTQ_OK;
+}
 
+// Phase 3 on `st`: unpermute, loss and packing.
+int enqueue_finalize(const SweepPlan &p, cudaStream_t st) {
+  const int ri = p.r, di = p.d, group = p.group;
   FinalizeArgs f{};
   f.W = p.W;
   f.Wk = p.Wk;
@@ -381,7 +392,6 @@ int enqueue_sweep(const SweepPlan &p, cudaStream_t st) {
   f.status = p.status;
   GPTQ_TRY(launch_finalize(f, st));
   GPTQ_TRY(launch_loss_reduce(p.loss_rows, p.dsq_rows, ri, p.lambda, p.out, p.status, st));
-  GPTQ_TRY(record(4, st));
   return GPTQ_OK;
 }
 
@@ -439,32 +449,59 @@ int quantize_layer(const float *W, int64_t r, int64_t d, float *H, int bits, int
   int *status = reinterpret_cast<int *>(ws + L.status);
   const int ri = (int)r, di = (int)d;
 
-  auto enqueue = [&]() -> int {
-    GPTQ_TRY(record(0, st));
+  // The four phases of the solve: damping (and the act-order permutation),
+  // the factor U, the sweep, and finalize (unpermute, loss, packing).
+  float *U = nullptr;
+  auto seg_damp = [&]() -> int {
     GPTQ_CUDA_TRY(cudaMemsetAsync(status, 0, 16, st));
     GPTQ_CUDA_TRY(cudaMemsetAsync(loss_rows, 0, (size_t)r * 8, st));
-
-    float *U = nullptr;
-    GPTQ_TRY(enqueue_factor(H, d, damp, act_order, perm, inv, lambda, Hp, T1, status, st, !plain,
-                            &U));
-    const SweepPlan sp{W, ri, di, bits, group, block, sym, static_groups, U,
-                       act_order ? perm : nullptr, act_order ? inv : nullptr, lambda, W_hat,
-                       qweight, scales, zeros, g_idx, codes, Wk, ErrS, codes_p, loss_rows,
-                       dsq_rows, out, status};
-    return enqueue_sweep(sp, st);
+    int rc = GPTQ_OK;
+    U = enqueue_damp(H, d, damp, act_order, perm, inv, lambda, Hp, st, &rc);
+    return rc;
   };
+  auto seg_factor = [&]() -> int { return launch_factor(U, d, T1, status, st, !plain); };
+  auto sweep_plan = [&]() {
+    return SweepPlan{W, ri, di, bits, group, block, sym, static_groups, U,
+                     act_order ? perm : nullptr, act_order ? inv : nullptr, lambda, W_hat,
+                     qweight, scales, zeros, g_idx, codes, Wk, ErrS, codes_p, loss_rows,
+                     dsq_rows, out, status};
+  };
+  auto seg_sweep = [&]() -> int { return enqueue_sweep(sweep_plan(), st); };
+  auto seg_final = [&]() -> int { return enqueue_finalize(sweep_plan(), st); };
 
-  // Replay the whole kernel sequence as a CUDA graph when the same call
-  // (pointers, sizes, settings, stream) repeats: the sequence holds a few
-  // hundred short kernels whose launch cost would otherwise pace the GPU.  The
-  // first call of a configuration runs directly, the second is captured, later
-  // ones replay.  Streams that cannot be captured run directly.
+  // Each phase replays as a CUDA graph when the same call (pointers, sizes,
+  // settings, stream) repeats: the phases hold a few hundred short kernels
+  // whose launch cost would otherwise pace the GPU.  The first call of a
+  // configuration runs directly, the second is captured, later ones replay.
+  // Streams that cannot be captured run directly.  The phase events (when
+  // timing) are recorded between the phases, outside any capture.
   const bool timing = g_timing && !plain;
   if (timing) GPTQ_TRY(ensure_phase_events());
-  const GraphKey key{W, H, W_hat, qweight, scales, zeros, g_idx, codes, workspace,
-                     workspace_bytes, st, r, d, bits, group, block, damp, options, timing};
   t_timing = timing;
-  const int rc = plain ? enqueue() : run_graph_cached(key, st, enqueue);
+  GraphKey key{W, H, W_hat, qweight, scales, zeros, g_idx, codes, workspace,
+               workspace_bytes, st, r, d, bits, group, block, damp, options, 0};
+  int rc = GPTQ_OK;
+  if (plain) {
+    rc = seg_damp();
+    if (rc == GPTQ_OK) rc = seg_factor();
+    if (rc == GPTQ_OK) rc = seg_sweep();
+    if (rc == GPTQ_OK) rc = seg_final();
+  } else {
+    // the matrix to factor is known without running the damping phase
+    U = act_order ? Hp : H;
+    rc = record(0, st);
+    if (rc == GPTQ_OK) rc = run_graph_cached(key, st, seg_damp);
+    if (rc == GPTQ_OK) rc = record(1, st);
+    key.segment = 1;
+    if (rc == GPTQ_OK) rc = run_graph_cached(key, st, seg_factor);
+    if (rc == GPTQ_OK) rc = record(2, st);
+    key.segment = 2;
+    if (rc == GPTQ_OK) rc = run_graph_cached(key, st, seg_sweep);
+    if (rc == GPTQ_OK) rc = record(3, st);
+    key.segment = 3;
+    if (rc == GPTQ_OK) rc = run_graph_cached(key, st, seg_final);
+    if (rc == GPTQ_OK) rc = record(4, st);
+  }
   t_timing = false;
   if (rc != GPTQ_OK) return rc;
 
@@ -635,6 +672,7 @@ extern "C" int gptq_quantize_with_factor(const float *W, int64_t r, int64_t d, c
                      reinterpret_cast<uint8_t *>(ws + L.codes_p), loss_rows,
                      reinterpret_cast<double *>(ws + L.dsq_rows), out, status};
   GPTQ_TRY(enqueue_sweep(sp, st));
+  GPTQ_TRY(enqueue_finalize(sp, st));
   double host_out[3] = {0, 0, 0};
   int host_status = 0;
   GPTQ_CUDA_TRY(cudaMemcpyAsync(host_out, out, sizeof(host_out), cudaMemcpyDeviceToHost, st));

@@ -6,11 +6,20 @@
 // blocked factorisation that forms U -- the dense contractions of the layer solve
 // (GPTQ reading card, 方法适配: the deferred global update is a matrix product).
 //
-// Each fp32 operand x is split as hi = tf32(x) and lo = tf32(x - hi), both
-// truncations; hi is the raw operand as the tensor core reads it.  The product
-// is hi*hi + hi*lo + lo*hi: three tcgen05.mma.kind::tf32 per K step
-// accumulating in TMEM, which keeps about 20 bits of each operand (the
-// dropped lo*lo term is ~2^-20 relative).
+// Each fp32 operand is split into two TF32 parts and the product is
+// hi*hi + hi*lo + lo*hi: three tcgen05.mma.kind::tf32 per K step.  A's parts are
+// rounded to nearest (hi = rna(a), lo = rna(a - hi)); B's hi part is the raw
+// tile, which the tensor core reads as its top 19 bits (truncation), and its lo
+// part is rna(b - trunc(b)).  So the dropped lo*lo term has a random sign (A's
+// lo is rounded to nearest) and every split residual is unbiased: the product
+// is good to about 2^-21 relative with no systematic drift.  The tensor core's
+// fp32 accumulation is not rounded to nearest, so each K step (12 MMAs) goes
+// into one of two TMEM accumulators and is folded into fp32 registers of the
+// converter warps one step later, while the next step accumulates in the other
+// buffer: the long sums of the trailing updates (K up to 1024) are rounded to
+// nearest like plain fp32 sums.  These GEMMs feed the Cholesky updates and the
+// sweep's compensation, whose errors the ill-conditioned Hessians of
+// calibration sets with few tokens per feature amplify.
 //
 // Tile 128 x 128 x 32 per stage: a 3-deep TMA ring of raw A/B tiles and a
 // 3-deep ring of converted operands.  A (and B^T) are K-major with a 128-byte
@@ -20,11 +29,12 @@
 // TMEM) and B's lo part into shared memory (B's hi part is the raw tile), so
 // the three MMAs of a K step read only B from shared memory -- shared-memory
 // bandwidth is what bounds this three-pass product.  Warp 0 issues TMA, warp 1
-// issues UMMA, warps 2..9 convert each landed stage and afterwards drain the
-// TMEM accumulator (two warps per TMEM lane quarter, 64 columns each).  The C tile travels by TMA both ways: it is
-// loaded into shared memory while the main loop runs (when beta != 0), updated
-// there in place by the epilogue warps, and stored with four bulk tensor
-// stores, so every global access of the epilogue is a full 128-byte line.
+// issues UMMA, warps 2..9 convert each landed stage, fold the previous step's
+// accumulator (two warps per TMEM lane quarter, 64 columns each) and end with
+// the epilogue.  The C tile travels by TMA both ways: it is loaded into shared
+// memory while the main loop runs (when beta != 0), updated there in place by
+// the epilogue warps, and stored with four bulk tensor stores, so every global
+// access of the epilogue is a full 128-byte line.
 #include <mutex>
 
 #include "gptq_internal.h"
@@ -42,10 +52,11 @@ constexpr int CONV_THREADS = 256;
 constexpr int C_BOX_BYTES = 128 * 32 * 4;  // one 32-column box of the C tile
 constexpr int C_BYTES = 4 * C_BOX_BYTES;    // 64 KB: the 128 x 128 C tile
 constexpr size_t SMEM_BYTES = (size_t)RS * PAIR_BYTES + (size_t)LS * TILE_BYTES + C_BYTES + 1024;
-// TMEM columns: the 128 x 128 accumulator, then per converted stage t the A
-// hi part (32 columns, one K value each) and the A lo part (32 columns).
+// TMEM columns: two 128 x 128 accumulators (K steps alternate), then per
+// converted stage t the A hi part (32 columns, one K value each) and the A lo
+// part (32 columns).
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_A0 = TN;
+constexpr uint32_t TMEM_A0 = 2 * TN;
 __host__ __device__ constexpr uint32_t tmem_a_hi(int t) { return TMEM_A0 + (uint32_t)t * 2 * TK; }
 __host__ __device__ constexpr uint32_t tmem_a_lo(int t) { return tmem_a_hi(t) + TK; }
 static_assert(TMEM_A0 + LS * 2 * TK <= TMEM_COLS, "TMEM budget");
@@ -55,7 +66,8 @@ struct TcShared {
   uint64_t empty[RS];
   uint64_t conv[LS];
   uint64_t lofree[LS];
-  uint64_t accf;
+  uint64_t accf[2];   // a K step's products are in accumulator b
+  uint64_t acce[2];   // accumulator b has been folded (8 converter warps)
   uint64_t drain;
   uint64_t cfull;
   uint32_t tmem_base;
@@ -80,6 +92,13 @@ struct TcArgs {
 // (full ALU rate): |x - hi - lo| <= 2^-20 |x|.
 __device__ __forceinline__ float tf32_trunc(float x) {
   return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+}
+
+// Round to the nearest TF32 value, ties away from zero, with integer ops (full
+// ALU rate): add half a TF32 ulp to the magnitude bits and clear the low 13
+// (a carry into the exponent is the correct rounding up).
+__device__ __forceinline__ float tf32_rna(float x) {
+  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -138,7 +157,7 @@ __device__ __forceinline__ void fail_timeout(TcShared &sh, int *dev_status) {
   *(volatile int *)&sh.abort = 1;
 }
 
-// lo part of one 16 KB tile: lo = trunc(x - trunc(x)), same (swizzled) layout.
+// lo part of one 16 KB B tile: lo = rna(x - trunc(x)), same (swizzled) layout.
 __device__ __forceinline__ void split_tile(const uint8_t *tile, uint8_t *lo, int t) {
   const float4 *p = reinterpret_cast<const float4 *>(tile);
   float4 *q = reinterpret_cast<float4 *>(lo);
@@ -146,10 +165,10 @@ __device__ __forceinline__ void split_tile(const uint8_t *tile, uint8_t *lo, int
   for (int i = t; i < TILE_BYTES / 16; i += CONV_THREADS) {
     const float4 v = p[i];
     float4 l;
-    l.x = tf32_trunc(v.x - tf32_trunc(v.x));
-    l.y = tf32_trunc(v.y - tf32_trunc(v.y));
-    l.z = tf32_trunc(v.z - tf32_trunc(v.z));
-    l.w = tf32_trunc(v.w - tf32_trunc(v.w));
+    l.x = tf32_rna(v.x - tf32_trunc(v.x));
+    l.y = tf32_rna(v.y - tf32_trunc(v.y));
+    l.z = tf32_rna(v.z - tf32_trunc(v.z));
+    l.w = tf32_rna(v.w - tf32_trunc(v.w));
     q[i] = l;
   }
 }
@@ -181,7 +200,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&sh.conv[t], CONV_THREADS / 32);
       mbar_init(&sh.lofree[t], 1);
     }
-    mbar_init(&sh.accf, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh.accf[b], 1);
+      mbar_init(&sh.acce[b], CONV_THREADS / 32);
+    }
     mbar_init(&sh.drain, 1);
     mbar_init(&sh.cfull, 1);
     sh.abort = 0;
@@ -254,12 +276,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       const uint32_t idesc = instr_desc(2, 2, 0, g.trans_b ? 0u : 1u, TM, TN);
       for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % RS, t = kb % LS;
-        if (!mbar_wait_bounded(&sh.conv[t], (kb / LS) & 1)) {
+        const int s = kb % RS, t = kb % LS, ab = kb & 1;
+        // accumulator ab is free once the step two before has been folded
+        if ((kb >= 2 && !mbar_wait_bounded(&sh.acce[ab], ((kb >> 1) - 1) & 1)) ||
+            !mbar_wait_bounded(&sh.conv[t], (kb / LS) & 1)) {
           fail_timeout(sh, g.dev_status);
           break;
         }
         tc_fence_after();
+        const uint32_t dacc = tmem + (uint32_t)ab * TN;
         const uint32_t b = smem_u32(smem + (size_t)s * PAIR_BYTES) + TILE_BYTES;
         const uint32_t bl = smem_u32(loring + (size_t)t * TILE_BYTES);
 #pragma unroll
@@ -279,22 +304,47 @@ __global__ void __launch_bounds__(THREADS, 1)
             bd = smem_desc(b + kk * 1024, TK * 128, 512, 1);
             bld = smem_desc(bl + kk * 1024, TK * 128, 512, 1);
           }
-          const uint32_t acc0 = (kb > 0 || kk > 0) ? 1u : 0u;
-          umma_tf32_ts(tmem, ah, bd, idesc, acc0);
-          umma_tf32_ts(tmem, ah, bld, idesc, 1u);
-          umma_tf32_ts(tmem, al, bd, idesc, 1u);
+          const uint32_t acc0 = kk > 0 ? 1u : 0u;   // each K step starts its accumulator
+          umma_tf32_ts(dacc, ah, bd, idesc, acc0);
+          umma_tf32_ts(dacc, ah, bld, idesc, 1u);
+          umma_tf32_ts(dacc, al, bd, idesc, 1u);
         }
         umma_commit(&sh.empty[s]);
         umma_commit(&sh.lofree[t]);
+        umma_commit(&sh.accf[ab]);
       }
-      umma_commit(&sh.accf);
       umma_commit(&sh.drain);
       (void)mbar_wait_bounded(&sh.drain, 0);
     }
   } else {
     // ---------------------------------------------------------------- split + epilogue
     const int tt = threadIdx.x - 64;
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;   // which 64 of the 128 columns
+    const int row = quarter * 32 + lane;  // row of the tile = TMEM lane
     bool ok = true;
+    float acc[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+    // fold K step c (accumulator c & 1) into acc once its MMAs are complete
+    auto fold = [&](int c) -> bool {
+      const int ab = c & 1;
+      if (!mbar_wait_bounded(&sh.accf[ab], (c >> 1) & 1)) return false;
+      tc_fence_after();
+      const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)ab * TN + half * 64;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float v[32];
+        tmem_ld_32x32b_x32(base + 32 * j, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[32 * j + i] += v[i];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.acce[ab]);
+      return true;
+    };
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % RS, t = kb % LS;
       if (!mbar_wait_bounded(&sh.full[s], (kb / RS) & 1) ||
@@ -323,7 +373,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           hi[4 * c + 3] = v.w;
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) lo[i] = tf32_trunc(hi[i] - tf32_trunc(hi[i]));
+        for (int i = 0; i < 16; ++i) {
+          const float x = hi[i];
+          hi[i] = tf32_rna(x);
+          lo[i] = tf32_rna(x - hi[i]);
+        }
         const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + hf * 16;
         tmem_st_32x32b_x16(lane_base + tmem_a_hi(t), hi);
         tmem_st_32x32b_x16(lane_base + tmem_a_lo(t), lo);
@@ -333,16 +387,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.conv[t]);
-    }
-    const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;   // which 64 of the 128 columns
-    const int row = quarter * 32 + lane;  // row of the tile = TMEM lane
-    if (ok && nk > 0) {
-      if (!mbar_wait_bounded(&sh.accf, 0)) {
+      // the previous step's products are (about) done by now
+      if (kb >= 1 && !fold(kb - 1)) {
         if (lane == 0) fail_timeout(sh, g.dev_status);
         ok = false;
+        break;
       }
-      tc_fence_after();
+    }
+    if (ok && nk > 0 && !fold(nk - 1)) {
+      if (lane == 0) fail_timeout(sh, g.dev_status);
+      ok = false;
     }
     if (ok && load_c && !mbar_wait_bounded(&sh.cfull, 0)) {
       if (lane == 0) fail_timeout(sh, g.dev_status);
@@ -353,17 +407,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       // 128 rows x 32 columns: 16-byte chunk c of a row is stored at chunk
       // position c ^ (row & 7), so the 8 rows of each quarter-warp phase hit
       // distinct banks.
-#pragma unroll 1
+#pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int box = 2 * half + j;
-        float v[32];
-        if (nk > 0) {
-          tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + box * 32, v);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0.f;
-        }
+        const float *v = acc + 32 * j;   // compile-time offsets (unrolled): acc stays in registers
         uint8_t *rp = ctile + box * C_BOX_BYTES + row * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
