@@ -21,10 +21,20 @@
 //    loads complete on the leader CTA's barrier), warp 1 of the leader issues
 //    the pair's UMMAs into one of two 256-column TMEM accumulators and
 //    commits to barriers in both CTAs, warps 2..9 of each CTA drain its TMEM.
-//  * Accuracy: the tensor core's fp32 accumulation is not guaranteed to round
-//    to nearest, so each TMEM accumulation chain is limited to 512 tokens and
-//    then folded into fp32 registers of the epilogue warps (double-buffered
-//    TMEM, so the tensor core keeps running while a chain is folded).
+//  * Accuracy: the tensor core's fp32 accumulation is not rounded to nearest,
+//    so each TMEM accumulation chain is limited to 128 tokens and then folded
+//    into fp32 registers of the epilogue warps (double-buffered TMEM, so the
+//    tensor core keeps running while a chain is folded).  Longer chains bias
+//    H by about 2e-6, which the ill-conditioned Hessians of calibration sets
+//    with few tokens per feature turn into different codes.
+//  * Pacing: X is read once from HBM only while the pairs working on tiles
+//    that share panels read the same token slab at about the same time.
+//    Every PACE_EVERY stages each pair's leader publishes how many stages it
+//    has issued (per device, tagged with the launch) and, if it is more than
+//    PACE_LAG stages ahead of the slowest pair still working, waits for it --
+//    a bounded wait after which it goes on anyway, so pacing can only cost
+//    time, never stall the kernel (pairs not yet resident just are not waited
+//    for beyond the bound).
 //  * Persistent grid of one cluster per SM pair walking the tile list (in
 //    bands of 8 tile rows, column by column; see tile_coords); all clusters
 //    sweep the tokens at the same pace, so the current X slab is shared
@@ -36,6 +46,10 @@
 namespace gptq {
 
 __device__ int g_device_status;
+
+// Progress of the Hessian's CTA pairs: (launch tag << 32) | stages issued;
+// the low word 0xFFFFFFFF marks a pair that has finished its tiles.
+__device__ unsigned long long g_hess_progress[256];
 
 // Per-device lookups are cached so that no runtime query runs inside a
 // stream capture of the solve.
@@ -74,7 +88,10 @@ constexpr int HM = 128;                          // tile rows per CTA (UMMA M = 
 constexpr int HN = 256;                          // tile cols  (UMMA N)
 constexpr int HK = 64;                           // tokens per pipeline stage
 constexpr int STAGES = 6;
-constexpr int FOLD = 8;                          // stages per TMEM chain (512 tokens)
+constexpr int FOLD = 2;                          // stages per TMEM chain (128 tokens)
+constexpr int PACE_EVERY = 32;                   // stages between progress reports
+constexpr int PACE_LAG = 96;                     // stages a pair may run ahead of the slowest
+constexpr int PACE_SPINS = 500;                  // bounded wait: about 1 ms, then go on
 constexpr int BOXF = 64;                         // features per TMA box (128 bytes)
 constexpr int BOX_BYTES = BOXF * HK * 2;         // 8 KB
 constexpr int A_BYTES = HM * HK * 2;             // 16 KB: this CTA's 128 rows
@@ -222,7 +239,7 @@ __device__ __forceinline__ void record_timeout(int *status, HessShared &sh) {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, int64_t n, int d,
-                      float *__restrict__ H, int *__restrict__ status) {
+                      float *__restrict__ H, int *__restrict__ status, uint32_t tag) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ HessShared sh;
   uint8_t *smem =
@@ -267,51 +284,74 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
-      const uint32_t full0 = cluster_addr(&sh.full[0], 0);   // the leader's barriers
-      uint32_t stage = 0, phase = 0;
-      uint32_t issued = 0, issued_par = 0;  // leader: bit s = stage s armed / its parity
-      bool ok = true;
-      for (int t = pair; t < T && ok; t += npairs) {
-        int P, J;
-        tile_coords(t, nP, nJ, P, J);
-        const int i0 = P * 2 * HM + (int)rank * HM;      // this CTA's rows
-        const int j0 = J * HN + (int)rank * (HN / 2);    // this CTA's half of the columns
-        for (int ks = 0; ks < nsteps; ++ks) {
+    // Lane 0 issues the loads; in the leader the whole warp reads the other
+    // pairs' progress for pacing.
+    const uint32_t full0 = cluster_addr(&sh.full[0], 0);   // the leader's barriers
+    uint32_t stage = 0, phase = 0;
+    uint32_t issued = 0, issued_par = 0;  // leader: bit s = stage s armed / its parity
+    bool ok = true;
+    uint32_t done = 0;                    // stages this pair has issued
+    bool pacing = true;                   // off once a wait has run out
+    const unsigned long long mine = (unsigned long long)tag << 32;
+    for (int t = pair; t < T && ok; t += npairs) {
+      int P, J;
+      tile_coords(t, nP, nJ, P, J);
+      const int i0 = P * 2 * HM + (int)rank * HM;      // this CTA's rows
+      const int j0 = J * HN + (int)rank * (HN / 2);    // this CTA's half of the columns
+      for (int ks = 0; ks < nsteps; ++ks, ++done) {
+        if (leader && pacing && done % PACE_EVERY == 0) {
+          if (lane == 0) atomicExch(&g_hess_progress[pair], mine | done);
+          int spin = 0;
+          for (; spin < PACE_SPINS; ++spin) {
+            uint32_t slowest = 0xFFFFFFFFu;
+            for (int q = lane; q < npairs; q += 32) {
+              const unsigned long long v = *(volatile unsigned long long *)&g_hess_progress[q];
+              const uint32_t got = (v >> 32) == tag ? (uint32_t)v : 0u;   // not started: 0
+              slowest = min(slowest, got);
+            }
+            for (int o = 16; o > 0; o >>= 1) slowest = min(slowest, __shfl_xor_sync(0xffffffffu, slowest, o));
+            if (slowest == 0xFFFFFFFFu || done <= slowest + PACE_LAG) break;
+            __nanosleep(2000);
+          }
+          if (spin == PACE_SPINS) pacing = false;   // a pair is not coming: stop waiting
+        }
+        if (lane == 0) {
           // A failure in the other CTA surfaces here as a bounded wait running out.
           if (*(volatile int *)&sh.abort) {
             ok = false;
-            break;
-          }
-          if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1)) {
+          } else if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1)) {
             record_timeout(status, sh);
             ok = false;
-            break;
-          }
-          uint8_t *sA = smem + (size_t)stage * STAGE_BYTES;
-          uint8_t *sB = sA + A_BYTES;
-          const int y = ks * HK;
-          const uint32_t fb = full0 + stage * (uint32_t)sizeof(uint64_t);
-          if (leader) {
-            mbar_arrive_expect_tx(&sh.full[stage], 2 * STAGE_BYTES);
-            issued |= 1u << stage;
-            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          }
-          tma_load_2d_pair(sA, &tmap, i0, y, fb);
-          tma_load_2d_pair(sA + BOX_BYTES, &tmap, i0 + BOXF, y, fb);
-          tma_load_2d_pair(sB, &tmap, j0, y, fb);
-          tma_load_2d_pair(sB + BOX_BYTES, &tmap, j0 + BOXF, y, fb);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
+          } else {
+            uint8_t *sA = smem + (size_t)stage * STAGE_BYTES;
+            uint8_t *sB = sA + A_BYTES;
+            const int y = ks * HK;
+            const uint32_t fb = full0 + stage * (uint32_t)sizeof(uint64_t);
+            if (leader) {
+              mbar_arrive_expect_tx(&sh.full[stage], 2 * STAGE_BYTES);
+              issued |= 1u << stage;
+              issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+            }
+            tma_load_2d_pair(sA, &tmap, i0, y, fb);
+            tma_load_2d_pair(sA + BOX_BYTES, &tmap, i0 + BOXF, y, fb);
+            tma_load_2d_pair(sB, &tmap, j0, y, fb);
+            tma_load_2d_pair(sB + BOX_BYTES, &tmap, j0 + BOXF, y, fb);
           }
         }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
       }
-      // Let every armed stage land (both CTAs' loads) before the pair can exit.
-      if (leader)
-        for (int s = 0; s < STAGES; ++s)
-          if (issued & (1u << s)) (void)mbar_wait_bounded(&sh.full[s], (issued_par >> s) & 1u);
     }
+    // This pair is done: the others no longer wait for it.
+    if (leader && lane == 0) atomicExch(&g_hess_progress[pair], mine | 0xFFFFFFFFull);
+    // Let every armed stage land (both CTAs' loads) before the pair can exit.
+    if (leader && lane == 0)
+      for (int s = 0; s < STAGES; ++s)
+        if (issued & (1u << s)) (void)mbar_wait_bounded(&sh.full[s], (issued_par >> s) & 1u);
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer (leader)
     if (leader && lane == 0) {
@@ -488,8 +528,11 @@ extern "C" int gptq_hessian_accumulate(const void *X, int64_t n, int64_t d, int6
   for (int P = 0; P < nJ; ++P) T += nJ - P;
   const int max_pairs = num_sms() / 2 > 0 ? num_sms() / 2 : 1;
   const int pairs = T < max_pairs ? T : max_pairs;
+  // a tag per launch, so that progress left by an earlier launch is not read as this one's
+  static std::atomic<uint32_t> launches{1};
+  const uint32_t tag = launches.fetch_add(1, std::memory_order_relaxed);
   hessian_tc_kernel<<<2 * pairs, THREADS, SMEM_BYTES, (cudaStream_t)stream>>>(tmap, n, (int)d, H,
-                                                                              status);
+                                                                              status, tag);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }
