@@ -251,12 +251,18 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
     const float *srow = a.scales + row * a.G;
     const int32_t *zrow = a.zeros + row * a.G;
     for (int k0 = lane; k0 < nchunk; k0 += 32 * PF) {
+      // every load of the PF chunks (codes, scale, zero) before any arithmetic
       uint32_t w[PF][BITS];
+      float sc[PF], zr[PF];
 #pragma unroll
       for (int p = 0; p < PF; ++p) {
         const int k = k0 + 32 * p;
+        const bool in = k < nchunk;
 #pragma unroll
-        for (int t = 0; t < BITS; ++t) w[p][t] = k < nchunk ? __ldg(qrow + (int64_t)k * BITS + t) : 0u;
+        for (int t = 0; t < BITS; ++t) w[p][t] = in ? __ldg(qrow + (int64_t)k * BITS + t) : 0u;
+        const int gi = a.group > 0 ? (k * 32) / a.group : 0;
+        sc[p] = in ? __ldg(srow + gi) : 0.f;
+        zr[p] = in ? (float)__ldg(zrow + gi) : 0.f;
       }
 #pragma unroll
       for (int p = 0; p < PF; ++p) {
@@ -264,11 +270,9 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
         if (k < nchunk) {
           float part[MB];
           fold_chunk<BITS, MB>(w[p], xs, nchunk, k, part, a.m);
-          const int gi = a.group > 0 ? (k * 32) / a.group : 0;
-          const float s = __ldg(srow + gi), z = (float)__ldg(zrow + gi);
 #pragma unroll
           for (int i = 0; i < MB; ++i)
-            if (i < a.m) acc[i] = fmaf(s, fmaf(-z, xsum[i * nchunk + k], part[i]), acc[i]);
+            if (i < a.m) acc[i] = fmaf(sc[p], fmaf(-zr[p], xsum[i * nchunk + k], part[i]), acc[i]);
         }
       }
     }

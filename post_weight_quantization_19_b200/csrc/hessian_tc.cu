@@ -89,8 +89,8 @@ constexpr int HN = 256;                          // tile cols  (UMMA N)
 constexpr int HK = 64;                           // tokens per pipeline stage
 constexpr int STAGES = 6;
 constexpr int FOLD = 2;                          // stages per TMEM chain (128 tokens)
-constexpr int PACE_EVERY = 32;                   // stages between progress reports
-constexpr int PACE_LAG = 96;                     // stages a pair may run ahead of the slowest
+constexpr int PACE_EVERY = 64;                   // stages between progress reports
+constexpr int PACE_LAG = 160;                    // stages a pair may run ahead of the slowest
 constexpr int PACE_SPINS = 500;                  // bounded wait: about 1 ms, then go on
 constexpr int BOXF = 64;                         // features per TMA box (128 bytes)
 constexpr int BOX_BYTES = BOXF * HK * 2;         // 8 KB
@@ -423,13 +423,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         tc_fence_after();
         const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + abuf * HN + half * 128;
+        // 32 columns per load, one wait per load (the chain of a stage pair
+        // gives the fold about 1000 cycles)
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
-          float v[16];
-          tmem_ld_32x32b_x16(base + p * 16, v);
+        for (int p = 0; p < 4; ++p) {
+          float v[32];
+          tmem_ld_32x32b_x32(base + p * 32, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) acc[p * 16 + i] += v[i];
+          for (int i = 0; i < 32; ++i) acc[p * 32 + i] += v[i];
         }
         tc_fence_before();
         __syncwarp();

@@ -10,12 +10,12 @@
 // processed by a 2 x 2 block recursion,
 //     A22 -> U22;  T = A12 U22^T;  A11 -= T T^T;  A12 = T U22;
 //     A11 -> U11;  A12 = -U11 A12,
-// with shared-memory products on the tensor cores (warp-level 3xTF32 mma.sync,
-// all LT / 32 warps), down to blocks of at most BASE columns that CF_THREADS
-// threads factor and invert two columns per barrier (each thread keeps a small
-// tile in registers).  The lower triangle is kept at zero between steps, so the
-// triangular operands can be used as dense ones.
-#include <stdlib.h>
+// with register-tiled fp32 shared-memory products (all LT threads), down to
+// blocks of at most BASE columns that CF_THREADS threads factor and invert one
+// column per barrier (each thread keeps a small tile in registers).  The lower
+// triangle is kept at zero between steps, so the triangular operands can be
+// used as dense ones.  (Tensor-core products and two column steps per barrier
+// were measured slower on the 4096-wide layer, by 0.03 ms and 0.25 ms.)
 
 #include "gptq_internal.h"
 
@@ -31,80 +31,6 @@ constexpr int CF_THREADS = 256;    // threads of the column factor (a named barr
 constexpr int BASE = 32;           // blocks up to this size go to the column factor
 constexpr size_t LEAF_SMEM = ((size_t)LB * LLD + 64 * 68) * sizeof(real);
 
-// C[M x N] = alpha * A[M x K] * op(B) + beta * C in shared memory, all shapes
-// and strides known at compile time; op(B) = B (K x N) or B^T (B stored N x K);
-// UPPER: only entries with column >= row are written (C is a diagonal block).
-// On the tensor cores: warp-level mma.sync m16n8k8 in TF32 with the error-compensated split
-// x = hi + lo (hi = tf32(x), lo = tf32(x - hi)) and three products per K step
-// (lo*hi and hi*lo first, then hi*hi), which keeps about 21 bits of each operand
-// -- the precision of the 3xTF32 products elsewhere in the factorisation.
-// Each warp takes 16 x 8 output tiles; fragment layout of m16n8k8 (lane = 4 g + t):
-// A[i0 + g (+8)][k + t (+4)], B[k + t (+4)][j0 + g], C[i0 + g (+8)][j0 + 2 t (+1)].
-// The padded leading dimensions (LLD = 132, m + 4) put the 32 lanes of every
-// fragment load in 32 different banks.  Ends with a CTA barrier.
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
-
-__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
-  hi = to_tf32(x);
-  lo = to_tf32(x - __uint_as_float(hi));
-}
-
-__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
-                                         const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-template <int M, int N, int K, int LDA, int LDB, int LDC, bool TB, bool UPPER>
-__device__ __forceinline__ void smem_gemm_tc(real *C, const real *A, const real *B, real alpha,
-                                             real beta) {
-  static_assert(M % 16 == 0 && N % 8 == 0 && K % 8 == 0, "m16n8k8 tiles");
-  constexpr int TN = N / 8, NT = (M / 16) * TN;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  for (int tile = warp; tile < NT; tile += LT / 32) {
-    const int i0 = (tile / TN) * 16, j0 = (tile % TN) * 8;
-    if (UPPER && j0 + 7 < i0) continue;   // wholly below the diagonal
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int k = 0; k < K; k += 8) {
-      const float a[4] = {A[(i0 + g) * LDA + k + t], A[(i0 + g + 8) * LDA + k + t],
-                          A[(i0 + g) * LDA + k + t + 4], A[(i0 + g + 8) * LDA + k + t + 4]};
-      float b[2];
-      if constexpr (TB) {
-        b[0] = B[(j0 + g) * LDB + k + t];
-        b[1] = B[(j0 + g) * LDB + k + t + 4];
-      } else {
-        b[0] = B[(k + t) * LDB + j0 + g];
-        b[1] = B[(k + t + 4) * LDB + j0 + g];
-      }
-      uint32_t ah[4], al[4], bh[2], bl[2];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) split_tf32(a[q], ah[q], al[q]);
-#pragma unroll
-      for (int q = 0; q < 2; ++q) split_tf32(b[q], bh[q], bl[q]);
-      mma_tf32(acc, al, bh);
-      mma_tf32(acc, ah, bl);
-      mma_tf32(acc, ah, bh);
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int row = i0 + g + (q >= 2 ? 8 : 0), col = j0 + 2 * t + (q & 1);
-      if (UPPER && col < row) continue;
-      real *p = C + row * LDC + col;
-      *p = alpha * acc[q] + (beta != 0.f ? beta * *p : 0.f);
-    }
-  }
-  __syncthreads();
-}
-
 // Barrier of the column factor's threads only (warps 0 .. CF_THREADS/32 - 1).
 __device__ __forceinline__ void cf_barrier() {
   if constexpr (CF_THREADS == LT)
@@ -113,148 +39,6 @@ __device__ __forceinline__ void cf_barrier() {
     asm volatile("bar.sync 1, %0;" ::"n"(CF_THREADS) : "memory");
 }
 
-// Column factor of an N x N block at S (leading dimension LLD, N = 32 or 64)
-// by CF_THREADS threads: H_d = R R^T with R upper, overwritten by U = R^-1.
-// Thread (gr, gc) of a (CF_THREADS / GC) x GC grid keeps the TR x TC tile at rows
-// gr * TR, columns gc * TC in registers.  Step k = N-1 .. 0 uses a vector v
-// that holds column k above the diagonal (v_j = S[j][k], j < k), the pivot
-// p = S[k][k] at index k and row k right of the diagonal (v_j = S[k][j],
-// j > k).  With v_k taken as 1,
-//   rows i < k:  S[i][j] <- (j == k ? 0 : S[i][j]) - S[i][k] v_j / p
-//   row  k:      S[k][j] <- v_j / sqrt(p)
-// i.e. the Cholesky update of the leading block together with the
-// substitution that turns the finished rows into rows of R^-1.  Rows below k
-// are final; entries below the diagonal may pick up junk on the way and are
-// zeroed when the tile is written back.
-//
-// Steps go in pairs (k, k-1) with one barrier per pair: before it, the owners
-// publish the vector of step k and the vector of step k-1 as it stands before
-// step k; after it, every thread applies step k to the second vector's entries
-// that it needs (its rows, its columns, the pivot) with the same fused
-// multiply-adds the owners apply to their tiles, so the second step sees
-// exactly the values a barrier between the two steps would have published.
-// The published pairs alternate between two halves of vbuf (4 N floats).
-// Returns false (in every thread) on a non-positive pivot.
-template <int N>
-__device__ __forceinline__ bool col_factor(real *S, real *vbuf) {
-  static_assert(N % 2 == 0, "pairs of steps");
-  __shared__ int cf_ok;
-  if (threadIdx.x >= CF_THREADS) {   // the other warps wait at the closing barrier
-    __syncthreads();
-    return cf_ok != 0;
-  }
-  constexpr int GR = CF_THREADS / GC;
-  constexpr int TR = N / GR, TC = N / GC;
-  static_assert(TR >= 1 && TC >= 1 && TR * GR == N && TC * GC == N, "tile grid");
-  const int gr = threadIdx.x / GC, gc = threadIdx.x % GC;
-  const int i0 = gr * TR, j0 = gc * TC;
-  const bool owner = j0 + TC - 1 >= i0;   // the tile reaches the upper triangle
-  real t[TR][TC];
-#pragma unroll
-  for (int r = 0; r < TR; ++r)
-#pragma unroll
-    for (int q = 0; q < TC; ++q) t[r][q] = owner ? S[(i0 + r) * LLD + j0 + q] : 0.f;
-
-  // The owners' entries of the vectors of steps kk (into A) and kk - 1 (into B):
-  // column kk up to the diagonal and row kk right of it, likewise for kk - 1.
-  auto publish = [&](int kk, real *A) {
-    real *B = A + N;
-#pragma unroll
-    for (int r = 0; r < TR; ++r)
-#pragma unroll
-      for (int q = 0; q < TC; ++q) {
-        const int i = i0 + r, j = j0 + q;
-        if (j == kk && i <= kk) A[i] = t[r][q];
-        if (i == kk && j > kk) A[j] = t[r][q];
-        if (j == kk - 1 && i <= kk - 1) B[i] = t[r][q];
-        if (i == kk - 1 && j > kk - 1) B[j] = t[r][q];
-      }
-  };
-  // One step k on the tile, from the vector entries of its rows (vr) and
-  // columns (vc); mip = -1/p, ri = 1/sqrt(p).
-  auto step = [&](int k, const real (&vr)[TR], const real (&vc)[TC], real mip, real ri) {
-    if (!(owner && i0 <= k)) return;
-    real c[TR], v[TC];
-#pragma unroll
-    for (int r = 0; r < TR; ++r) c[r] = i0 + r < k ? vr[r] * mip : 0.f;
-#pragma unroll
-    for (int q = 0; q < TC; ++q) v[q] = j0 + q == k ? 1.f : vc[q];
-#pragma unroll
-    for (int r = 0; r < TR; ++r)
-#pragma unroll
-      for (int q = 0; q < TC; ++q) t[r][q] = fmaf(c[r], v[q], j0 + q == k ? 0.f : t[r][q]);
-#pragma unroll
-    for (int r = 0; r < TR; ++r)
-      if (i0 + r == k) {
-#pragma unroll
-        for (int q = 0; q < TC; ++q) t[r][q] = v[q] * ri;
-      }
-  };
-  bool bad = false;
-  auto pivot = [&](real p, real &mip, real &ri) {
-    bad |= !(p > 0.f);
-    p = bad ? 1.f : p;
-    ri = rsqrtf(p);
-    ri = ri * fmaf(-0.5f * p * ri, ri, 1.5f);   // one Newton step
-    mip = -ri * ri;
-  };
-
-  constexpr int NP = N / 2;   // pairs; pair P holds steps 2P+1 and 2P
-  if (owner) publish(N - 1, vbuf + ((NP - 1) & 1) * 2 * N);
-  cf_barrier();
-  // Fully unrolled: every comparison with k below becomes static.
-#pragma unroll
-  for (int P = NP - 1; P >= 0; --P) {
-    const int k = 2 * P + 1;
-    const real *A = vbuf + (P & 1) * 2 * N;
-    const real *B = A + N;
-    real mipa, ria;
-    pivot(A[k], mipa, ria);
-    real ar[TR], ac[TC];
-#pragma unroll
-    for (int r = 0; r < TR; ++r) ar[r] = A[i0 + r];
-#pragma unroll
-    for (int q = 0; q < TC; ++q) ac[q] = A[j0 + q];
-    // Step k's effect on the entries of step k-1's vector, written as the
-    // owners compute it: c = S[x][k] * mip times v = S[k-1][k] for the column
-    // part (x < k-1), c = S[k-1][k] * mip times v_x (v_k = 1, and 0 replaces
-    // the old entry at x = k) for the pivot and the row part (x >= k-1).
-    const real akm = A[k - 1];
-    const real ckm = akm * mipa;
-    real br[TR], bc[TC];
-#pragma unroll
-    for (int r = 0; r < TR; ++r) {
-      const int x = i0 + r;
-      br[r] = x < k - 1 ? fmaf(ar[r] * mipa, akm, B[x])
-                        : fmaf(ckm, x == k ? 1.f : ar[r], x == k ? 0.f : B[x]);
-    }
-#pragma unroll
-    for (int q = 0; q < TC; ++q) {
-      const int x = j0 + q;
-      bc[q] = x < k - 1 ? fmaf(ac[q] * mipa, akm, B[x])
-                        : fmaf(ckm, x == k ? 1.f : ac[q], x == k ? 0.f : B[x]);
-    }
-    const real pb = fmaf(ckm, akm, B[k - 1]);
-    step(k, ar, ac, mipa, ria);
-    real mipb, rib;
-    pivot(pb, mipb, rib);
-    step(k - 1, br, bc, mipb, rib);
-    if (P > 0 && owner) publish(k - 2, vbuf + ((P - 1) & 1) * 2 * N);
-    cf_barrier();
-  }
-  if (owner) {
-#pragma unroll
-    for (int r = 0; r < TR; ++r)
-#pragma unroll
-      for (int q = 0; q < TC; ++q)
-        S[(i0 + r) * LLD + j0 + q] = j0 + q >= i0 + r ? t[r][q] : 0.f;
-  }
-  if (threadIdx.x == 0) cf_ok = !bad;
-  __syncthreads();
-  return !bad;
-}
-
-// ---- The earlier forms (FFMA products, one column per barrier), kept for A/B timing ----
 
 // C[M x N] = alpha * A[M x K] * op(B) + beta * C in shared memory, all shapes
 // and strides known at compile time; op(B) = B (K x N) or B^T (B stored N x K).
@@ -265,7 +49,7 @@ __device__ __forceinline__ bool col_factor(real *S, real *vbuf) {
 // for 16-byte loads of a B row.  UPPER: only entries with column >= row are
 // written (C is a diagonal block).  Ends with a CTA barrier.
 template <int M, int N, int K, int LDA, int LDB, int LDC, bool TB, bool UPPER>
-__device__ __forceinline__ void smem_gemm_v1(real *C, const real *A, const real *B, real alpha,
+__device__ __forceinline__ void smem_gemm(real *C, const real *A, const real *B, real alpha,
                                           real beta) {
   static_assert(K % 4 == 0 && LDA % 4 == 0 && LDB % 4 == 0 && LDC % 4 == 0, "16-byte rows");
   constexpr int RM = (M * N >= 16 * LT) ? 4 : 2;
@@ -357,7 +141,7 @@ __device__ __forceinline__ void smem_gemm_v1(real *C, const real *A, const real 
 // costs one CTA barrier.  Returns false (in every thread) on a non-positive
 // pivot.
 template <int N>
-__device__ __forceinline__ bool col_factor_v1(real *S, real *vbuf) {
+__device__ __forceinline__ bool col_factor(real *S, real *vbuf) {
   __shared__ int cf_ok;
   if (threadIdx.x >= CF_THREADS) {   // the other warps wait at the closing barrier
     __syncthreads();
@@ -435,36 +219,24 @@ __device__ __forceinline__ bool col_factor_v1(real *S, real *vbuf) {
 // Node [off, off + N) of the shared-memory block.  N is a compile-time size
 // (32, 64, 96 or 128), so the recursion unfolds at compile time and uses no
 // call stack.
-template <int N, int V>
+template <int N>
 __device__ __forceinline__ bool node_factor(real *S, real *T, real *vbuf, int off) {
   if constexpr (N <= BASE) {
-    if constexpr (V & 1)
-      return col_factor<N>(S + off * LLD + off, vbuf);
-    else
-      return col_factor_v1<N>(S + off * LLD + off, vbuf);
+    return col_factor<N>(S + off * LLD + off, vbuf);
   } else {
     constexpr int h = 32 * ((N / 32) / 2), m = N - h;
-    if (!node_factor<m, V>(S, T, vbuf, off + h)) return false;
+    if (!node_factor<m>(S, T, vbuf, off + h)) return false;
     real *A11 = S + off * LLD + off;
     real *A12 = S + off * LLD + off + h;
     const real *U22 = S + (off + h) * LLD + off + h;
     // T (h x m): leading dimension m + 4, so rows stay 16-byte aligned and
     // the rows that neighbouring threads read transposed fall in different banks.
     constexpr int LT_ = m + 4;
-    if constexpr ((V & 2) != 0) {
-      smem_gemm_tc<h, m, m, LLD, LLD, LT_, true, false>(T, A12, U22, 1.f, 0.f);    // R12 = A12 U22^T
-      smem_gemm_tc<h, h, m, LT_, LT_, LLD, true, true>(A11, T, T, -1.f, 1.f);      // A11 -= R12 R12^T
-      smem_gemm_tc<h, m, m, LT_, LLD, LLD, false, false>(A12, T, U22, 1.f, 0.f);   // A12 = R12 U22
-    } else {
-      smem_gemm_v1<h, m, m, LLD, LLD, LT_, true, false>(T, A12, U22, 1.f, 0.f);
-      smem_gemm_v1<h, h, m, LT_, LT_, LLD, true, true>(A11, T, T, -1.f, 1.f);
-      smem_gemm_v1<h, m, m, LT_, LLD, LLD, false, false>(A12, T, U22, 1.f, 0.f);
-    }
-    if (!node_factor<h, V>(S, T, vbuf, off)) return false;
-    if constexpr ((V & 2) != 0)
-      smem_gemm_tc<h, m, h, LLD, LLD, LT_, false, false>(T, A11, A12, -1.f, 0.f);  // T = -U11 A12
-    else
-      smem_gemm_v1<h, m, h, LLD, LLD, LT_, false, false>(T, A11, A12, -1.f, 0.f);
+      smem_gemm<h, m, m, LLD, LLD, LT_, true, false>(T, A12, U22, 1.f, 0.f);
+      smem_gemm<h, h, m, LT_, LT_, LLD, true, true>(A11, T, T, -1.f, 1.f);
+      smem_gemm<h, m, m, LT_, LLD, LLD, false, false>(A12, T, U22, 1.f, 0.f);
+    if (!node_factor<h>(S, T, vbuf, off)) return false;
+      smem_gemm<h, m, h, LLD, LLD, LT_, false, false>(T, A11, A12, -1.f, 0.f);
     for (int idx = threadIdx.x; idx < h * m; idx += LT) {
       const int r = idx / m, c = idx - r * m;
       A12[r * LLD + c] = T[r * LT_ + c];
@@ -474,7 +246,6 @@ __device__ __forceinline__ bool node_factor(real *S, real *T, real *vbuf, int of
   }
 }
 
-template <int V>
 __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb, int *status) {
   extern __shared__ real lsm[];
   __shared__ real vbuf[4 * BASE];   // two published pairs of vectors
@@ -496,10 +267,10 @@ __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb,
   __syncthreads();
   bool ok;
   switch (nb) {
-    case 32: ok = node_factor<32, V>(S, T, vbuf, 0); break;
-    case 64: ok = node_factor<64, V>(S, T, vbuf, 0); break;
-    case 96: ok = node_factor<96, V>(S, T, vbuf, 0); break;
-    default: ok = node_factor<128, V>(S, T, vbuf, 0); break;
+    case 32: ok = node_factor<32>(S, T, vbuf, 0); break;
+    case 64: ok = node_factor<64>(S, T, vbuf, 0); break;
+    case 96: ok = node_factor<96>(S, T, vbuf, 0); break;
+    default: ok = node_factor<128>(S, T, vbuf, 0); break;
   }
   if (!ok) {
     if (threadIdx.x == 0) atomicCAS(status, 0, (int)GPTQ_ERR_NOT_PD);
@@ -516,24 +287,6 @@ __global__ void __launch_bounds__(LT) leaf_kernel(float *A, int64_t lda, int nb,
 
 }  // namespace
 
-// Leaf form: bit 0 = two column steps per barrier, bit 1 = tensor-core
-// products (GPTQ_LEAF=0..3 while the forms are compared; default 3).
-static int leaf_form() {
-  static const int v = [] {
-    const char *e = getenv("GPTQ_LEAF");
-    return (e && e[0] >= '0' && e[0] <= '3' && e[1] == 0) ? e[0] - '0' : 0;
-  }();
-  return v;
-}
-
-template <int V>
-static int launch_leaf_form(float *A, int64_t ld, int nb, int *status, cudaStream_t stream) {
-  static std::atomic<bool> attr[64] = {};
-  if (const int rc = ensure_smem_attr(leaf_kernel<V>, LEAF_SMEM, attr)) return rc;
-  GPTQ_LAUNCH_PDL(leaf_kernel<V>, dim3(1), dim3(LT), LEAF_SMEM, stream, A, ld, nb, status);
-  return GPTQ_OK;
-}
-
 int launch_leaf(float *A, int64_t ld, int nb, int *status, cudaStream_t stream) {
   if (nb <= 0 || nb > LB || nb % 32 != 0) return GPTQ_ERR_INVALID_ARG;
   if (PlanRecorder *rec = plan_recorder()) {
@@ -542,12 +295,10 @@ int launch_leaf(float *A, int64_t ld, int nb, int *status, cudaStream_t stream) 
     rec->line("L s=%d A=%s ld=%lld nb=%d\n", plan_stream_index(stream), a, (long long)ld, nb);
     return GPTQ_OK;
   }
-  switch (leaf_form()) {
-    case 0: return launch_leaf_form<0>(A, ld, nb, status, stream);
-    case 1: return launch_leaf_form<1>(A, ld, nb, status, stream);
-    case 2: return launch_leaf_form<2>(A, ld, nb, status, stream);
-    default: return launch_leaf_form<3>(A, ld, nb, status, stream);
-  }
+  static std::atomic<bool> attr[64] = {};
+  if (const int rc = ensure_smem_attr(leaf_kernel, LEAF_SMEM, attr)) return rc;
+  GPTQ_LAUNCH_PDL(leaf_kernel, dim3(1), dim3(LT), LEAF_SMEM, stream, A, ld, nb, status);
+  return GPTQ_OK;
 }
 
 }  // namespace gptq

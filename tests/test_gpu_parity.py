@@ -203,29 +203,6 @@ def test_sweep_rejects_a_perm_that_is_not_a_permutation():
     assert res["loss"] > 0
 
 
-def test_earlier_leaf_gives_the_same_layer():
-    # GPTQ_LEAF=1 (read once per process) runs the earlier leaf (FFMA products,
-    # one column per barrier); its U differs only by rounding, so the codes agree
-    # with the default leaf's up to the usual tie decisions.
-    import os
-    import subprocess
-    import sys
-    r, d, n = 64, 512, 4096
-    X, W = make_problem(r, d, n, seed=98)
-    got = gpu_layer(None, W, bits=4, group=128, H32=oracle.hessian(X).astype(np.float32))
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    code = (
-        "import sys, numpy as np; sys.path[:0] = [%r, %r]\n"
-        "from synth import make_problem\nimport oracle\nfrom parity_util import gpu_layer\n"
-        "X, W = make_problem(%d, %d, %d, seed=98)\n"
-        "got = gpu_layer(None, W, bits=4, group=128, H32=oracle.hessian(X).astype(np.float32))\n"
-        "np.save(sys.argv[1], got['codes'])\n" % (root, os.path.join(root, "tests"), r, d, n))
-    out = os.path.join(os.environ.get("TMPDIR", "/tmp"), "codes_leaf1_%d.npy" % os.getpid())
-    env = dict(os.environ, GPTQ_LEAF="1")
-    subprocess.run([sys.executable, "-c", code, out], check=True, env=env, timeout=600)
-    assert_codes_close(np.load(out), got["codes"])
-
-
 def test_tiny_workload_end_to_end():
     wl = workload("tiny_128x256")
     X, W = workload_inputs(wl)
