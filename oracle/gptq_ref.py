@@ -375,11 +375,18 @@ def layer_loss_direct(W: np.ndarray, What: np.ndarray, X: np.ndarray) -> float:
 def gptq_quantize_layer(W: np.ndarray, H: np.ndarray, *, bits: int, group: int,
                         block: int = 128, damp: float = 0.01,
                         act_order: bool = False, rows: np.ndarray | None = None,
-                        sym: bool = False, static_groups: bool = False) -> dict:
+                        sym: bool = False, static_groups: bool = False,
+                        perm: np.ndarray | None = None) -> dict:
     """Damp, order, factor, sweep, score and unpermute one layer.
 
     ``rows`` restricts the sweep to a subset of output rows (rows are
     independent once U is fixed), for checks at full layer width.
+
+    ``perm`` (act-order only) gives the column order instead of computing it
+    from diag(H): for checking a result whose order differs from the oracle's
+    only among columns whose diagonal entries are equal to within the
+    precision of the H it was computed from (either order is then a stable
+    descending order of the same values).
 
     ``sym`` selects the symmetric quantiser (see ``quant_params``).
     ``static_groups`` takes every group's parameters from the original W over
@@ -394,7 +401,14 @@ def gptq_quantize_layer(W: np.ndarray, H: np.ndarray, *, bits: int, group: int,
         W = W[np.asarray(rows)]
     r, d = W.shape
     Hd, lam = dampen(H, damp)
-    perm = act_order_perm(H) if act_order else np.arange(d)
+    if perm is not None:
+        if not act_order:
+            raise ValueError("a column order is given only with act-order")
+        perm = np.asarray(perm, dtype=np.int64)
+        if not np.array_equal(np.sort(perm), np.arange(d)):
+            raise ValueError("perm is not a permutation")
+    else:
+        perm = act_order_perm(H) if act_order else np.arange(d)
     inv = np.argsort(perm)
     U = inverse_upper_cholesky(Hd[np.ix_(perm, perm)])
     fixed = None

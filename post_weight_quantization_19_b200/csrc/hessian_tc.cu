@@ -22,11 +22,13 @@
 //    the pair's UMMAs into one of two 256-column TMEM accumulators and
 //    commits to barriers in both CTAs, warps 2..9 of each CTA drain its TMEM.
 //  * Accuracy: the tensor core's fp32 accumulation is not rounded to nearest,
-//    so each TMEM accumulation chain is limited to 128 tokens and then folded
+//    so each TMEM accumulation chain is limited to 256 tokens and then folded
 //    into fp32 registers of the epilogue warps (double-buffered TMEM, so the
-//    tensor core keeps running while a chain is folded).  Longer chains bias
-//    H by about 2e-6, which the ill-conditioned Hessians of calibration sets
-//    with few tokens per feature turn into different codes.
+//    tensor core keeps running while a chain is folded).  512-token chains
+//    bias H by about 2e-6, which the ill-conditioned Hessians of calibration
+//    sets with few tokens per feature turn into different codes; 128-token
+//    chains leave the fold (a TMEM read of the whole accumulator) too little
+//    time.
 //  * Pacing: X is read once from HBM only while the pairs working on tiles
 //    that share panels read the same token slab at about the same time.
 //    Every PACE_EVERY stages each pair's leader publishes how many stages it
@@ -88,7 +90,7 @@ constexpr int HM = 128;                          // tile rows per CTA (UMMA M = 
 constexpr int HN = 256;                          // tile cols  (UMMA N)
 constexpr int HK = 64;                           // tokens per pipeline stage
 constexpr int STAGES = 6;
-constexpr int FOLD = 2;                          // stages per TMEM chain (128 tokens)
+constexpr int FOLD = 4;                          // stages per TMEM chain (256 tokens)
 constexpr int PACE_EVERY = 64;                   // stages between progress reports
 constexpr int PACE_LAG = 160;                    // stages a pair may run ahead of the slowest
 constexpr int PACE_SPINS = 500;                  // bounded wait: about 1 ms, then go on
@@ -423,8 +425,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         tc_fence_after();
         const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + abuf * HN + half * 128;
-        // 32 columns per load, one wait per load (the chain of a stage pair
-        // gives the fold about 1000 cycles)
+        // 32 columns per load, one wait per load
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
           float v[32];

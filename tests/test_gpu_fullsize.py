@@ -37,8 +37,22 @@ def _check_sampled(name: str, nrows: int = 64):
     err = rel_fro(got["H"], H)
     assert err <= H_REL_FRO, err
     rows = np.sort(np.random.default_rng(wl.seed).choice(wl.r, nrows, replace=False))
+    perm = None
+    if wl.act_order:
+        # The order is a stable descending sort of diag(H).  The GPU sorts its
+        # fp32 H, whose entries differ from the float64 ones by up to the H
+        # tolerance, so columns whose diagonals agree to within it may come in
+        # either order (both are valid).  Check that the GPU's order is
+        # descending in the float64 diagonal up to that tolerance, then compare
+        # with the oracle run in that order.
+        perm = np.argsort(-np.diag(got["H"]).astype(np.float64), kind="stable")
+        dg = np.diag(H)[perm]
+        assert np.all(dg[1:] <= dg[:-1] * (1 + H_REL_FRO))
+        swapped = int(np.sum(perm != oracle.act_order_perm(H)))
+        print(f"{name}: {swapped} columns ordered differently from the float64 order "
+              f"(near-equal diagonals)")
     ref = oracle.gptq_quantize_layer(W, H, bits=wl.bits, group=wl.group, block=wl.block,
-                                     damp=wl.damp, act_order=wl.act_order, rows=rows)
+                                     damp=wl.damp, act_order=wl.act_order, rows=rows, perm=perm)
     match = assert_codes_close(got["codes"][rows], ref["codes"])
     gl = oracle.layer_loss(W[rows], got["W_hat"][rows], H)
     assert abs(gl - ref["loss"]) <= LOSS_REL * ref["loss"], (gl, ref["loss"])

@@ -324,6 +324,23 @@ def test_act_order_is_permutation_equivariant():
     assert out["loss"] == pytest.approx(ref["loss"], rel=1e-12)
 
 
+def test_given_order_equals_the_computed_one_and_is_checked():
+    # The act-order run with its own order passed back in is the same run;
+    # another order gives the permutation-equivariant result of that order.
+    X, W = make_problem(9, 96, 1500, seed=41)
+    H = oracle.hessian(X)
+    a = oracle.gptq_quantize_layer(W, H, bits=3, group=32, block=32, act_order=True)
+    b = oracle.gptq_quantize_layer(W, H, bits=3, group=32, block=32, act_order=True,
+                                   perm=a["perm"])
+    np.testing.assert_array_equal(a["codes"], b["codes"])
+    assert a["loss"] == b["loss"]
+    with pytest.raises(ValueError):
+        oracle.gptq_quantize_layer(W, H, bits=3, group=32, act_order=True,
+                                   perm=np.zeros(96, dtype=int))
+    with pytest.raises(ValueError):
+        oracle.gptq_quantize_layer(W, H, bits=3, group=32, perm=a["perm"])
+
+
 def test_dequantised_output_is_on_the_grid():
     X, W = make_problem(8, 128, 600, seed=16)
     out = oracle.gptq_quantize_layer(W, oracle.hessian(X), bits=3, group=32)
