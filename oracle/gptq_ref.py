@@ -296,7 +296,7 @@ def _check_groups(d: int, group: int, block: int) -> None:
 
 
 def gptq_sweep(W: np.ndarray, U: np.ndarray, bits: int, group: int, block: int,
-               sym: bool = False, fixed=None):
+               sym: bool = False, fixed=None, forced=None):
     """Quantise W [r x d] column by column in fixed order.
 
     At column j: q = quantize(w_j), e_j = (w_j - w^_j)/U_jj, and the columns
@@ -308,6 +308,10 @@ def gptq_sweep(W: np.ndarray, U: np.ndarray, bits: int, group: int, block: int,
     ``fixed`` = (scales [r x G], zeros [r x G], col_group [d]) gives static
     group parameters chosen before the sweep: column j uses group col_group[j]
     and no parameters are taken from the compensated weights.
+
+    ``forced`` = {j: codes [r]} replaces the rounding decision at column j by
+    the given codes (then compensated as usual): for following another
+    result's choice at a rounding tie, where both choices are correct.
 
     Returns (codes int64, scales, zeros (float64 holding integers), W^ float64,
     E float64 [r x d] with E[:, j] = e_j).
@@ -339,6 +343,8 @@ def gptq_sweep(W: np.ndarray, U: np.ndarray, bits: int, group: int, block: int,
                 scales[:, j // group], zeros[:, j // group] = s, z
             w = W[:, j]
             q = quantize(w, s, z, bits)
+            if forced is not None and j in forced:
+                q = np.asarray(forced[j], dtype=F64).copy()
             wq = dequantize(q, s, z)
             e = (w - wq) / U[j, j]
             codes[:, j] = q.astype(np.int64)

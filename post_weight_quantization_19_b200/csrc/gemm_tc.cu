@@ -451,6 +451,311 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------- CTA pairs
+// The same product on pairs of CTAs (a cluster of two along M): one
+// tcgen05.mma.cta_group::2 of M = 256, N = 128, K = 8 takes A from both CTAs'
+// tensor memory (128 rows each) and B from both CTAs' shared memory (64 of the
+// 128 columns each).  Each CTA loads, converts and holds only half of B, so
+// the shared-memory traffic per K step and CTA falls from about 128 KB to
+// about 80 KB -- below what the tensor core needs the step to take -- for the
+// same 128 x 128 of output per CTA.  Each CTA's loads complete on its own
+// barrier (its converters read them); the converters of both CTAs arrive on
+// the leader's barrier, which the leader's MMA thread waits on; the MMA
+// commits reach both CTAs.  A K range bounded by the row tile (GEMM_KMIN_ROW)
+// is the leader's; the second CTA zeroes the A values of its rows below its
+// own bound.  With GEMM_UPPER_C the second CTA of a pair on the diagonal
+// computes a tile below it and does not store it.
+
+constexpr int PN = 128;                              // pair tile columns (UMMA N)
+constexpr int PB_BYTES = (PN / 2) * TK * 4;          // 8 KB: this CTA's half of B
+constexpr int PSTAGE_BYTES = TILE_BYTES + PB_BYTES;  // 24 KB: A rows + B half
+constexpr size_t PSMEM_BYTES = (size_t)RS * PSTAGE_BYTES + (size_t)LS * PB_BYTES + C_BYTES + 1024;
+
+__device__ __forceinline__ void split_half(const uint8_t *tile, uint8_t *lo, int t) {
+  const float4 *p = reinterpret_cast<const float4 *>(tile);
+  float4 *q = reinterpret_cast<float4 *>(lo);
+#pragma unroll
+  for (int i = t; i < PB_BYTES / 16; i += CONV_THREADS) {
+    const float4 v = p[i];
+    float4 l;
+    l.x = tf32_rna(v.x - tf32_trunc(v.x));
+    l.y = tf32_rna(v.y - tf32_trunc(v.y));
+    l.z = tf32_rna(v.z - tf32_trunc(v.z));
+    l.w = tf32_rna(v.w - tf32_trunc(v.w));
+    q[i] = l;
+  }
+}
+
+__global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, TcArgs g) {
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ TcShared sh;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int bn = blockIdx.x, bm = blockIdx.y;       // bm = 2 * pair + rank
+  const int bm0 = bm - (int)rank;                   // the leader's row tile
+  if ((g.flags & GEMM_UPPER_C) && bn < bm0) return; // both tiles below the diagonal
+  const bool store = !((g.flags & GEMM_UPPER_C) && bn < bm);
+  const int m0 = bm * TM, n0 = bn * PN;
+  int klo = 0, khi = g.K;
+  if (g.flags & GEMM_KMIN_ROW) klo = max(klo, bm0 * TM);
+  if (g.flags & GEMM_KMIN_COL) klo = max(klo, n0);
+  if (g.flags & GEMM_KMAX_COL) khi = min(khi, n0 + PN);
+  const int nk = khi > klo ? (khi - klo) / TK : 0;
+  const int a_klo = (g.flags & GEMM_KMIN_ROW) ? m0 : 0;   // this CTA's rows are zero below it
+
+  uint8_t *smem =
+      reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < RS; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.empty[s], 1);
+    }
+    for (int t = 0; t < LS; ++t) {
+      mbar_init(&sh.conv[t], 2 * CONV_THREADS / 32);   // leader: both CTAs' converter warps
+      mbar_init(&sh.lofree[t], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh.accf[b], 1);
+      mbar_init(&sh.acce[b], 2 * CONV_THREADS / 32);   // leader: both CTAs have folded
+    }
+    mbar_init(&sh.drain, 1);
+    mbar_init(&sh.cfull, 1);
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmC);
+  }
+  pdl_wait_then_release();
+  if (threadIdx.x == 0) sh.abort = g.status ? *(volatile const int *)g.status : 0;
+  __syncthreads();
+  if (sh.abort) return;   // an earlier step failed: the same value in both CTAs
+  uint8_t *loring = smem + (size_t)RS * PSTAGE_BYTES;   // B lo halves
+  uint8_t *ctile = loring + (size_t)LS * PB_BYTES;
+  const bool load_c = g.beta != 0.f;
+  if (warp == 1) {
+    tmem_alloc_pair(&sh.tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  // Both CTAs' barriers are initialised and the pair's TMEM is allocated
+  // before either CTA signals the other.
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t issued = 0, issued_par = 0;
+      const int c_after = min(nk, RS) - 1;
+      bool c_issued = false;
+      auto issue_c = [&]() {
+        mbar_arrive_expect_tx(&sh.cfull, C_BYTES);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_load_2d(ctile + b * C_BOX_BYTES, &tmC, n0 + 32 * b, m0, &sh.cfull);
+        c_issued = true;
+      };
+      if (load_c && c_after < 0) issue_c();
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % RS;
+        const uint32_t ph = (kb / RS) & 1;
+        if (*(volatile int *)&sh.abort) break;
+        if (!mbar_wait_bounded(&sh.empty[s], ph ^ 1)) {
+          fail_timeout(sh, g.dev_status);
+          break;
+        }
+        uint8_t *st = smem + (size_t)s * PSTAGE_BYTES;
+        const int k0 = klo + kb * TK;
+        const int nh = n0 + (int)rank * (PN / 2);   // this CTA's half of the columns
+        mbar_arrive_expect_tx(&sh.full[s], PSTAGE_BYTES);
+        tma_load_2d(st, &tmA, k0, m0, &sh.full[s]);
+        if (g.trans_b) {
+          tma_load_2d(st + TILE_BYTES, &tmB, k0, nh, &sh.full[s]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < PN / 2 / 32; ++c)
+            tma_load_2d(st + TILE_BYTES + c * (TK * 128), &tmB, nh + 32 * c, k0, &sh.full[s]);
+        }
+        issued |= 1u << s;
+        issued_par = (issued_par & ~(1u << s)) | (ph << s);
+        if (load_c && kb == c_after) issue_c();
+      }
+      for (int s = 0; s < RS; ++s)
+        if (issued & (1u << s)) (void)mbar_wait_bounded(&sh.full[s], (issued_par >> s) & 1u);
+      if (c_issued) (void)mbar_wait_bounded(&sh.cfull, 0);
+    }
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      const uint32_t idesc = instr_desc(2, 2, 0, g.trans_b ? 0u : 1u, 2 * TM, PN);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % RS, t = kb % LS, ab = kb & 1;
+        if ((kb >= 2 && !mbar_wait_bounded(&sh.acce[ab], ((kb >> 1) - 1) & 1)) ||
+            !mbar_wait_bounded(&sh.conv[t], (kb / LS) & 1)) {
+          fail_timeout(sh, g.dev_status);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dacc = tmem + (uint32_t)ab * TN;
+        const uint32_t b = smem_u32(smem + (size_t)s * PSTAGE_BYTES) + TILE_BYTES;
+        const uint32_t bl = smem_u32(loring + (size_t)t * PB_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < TK / 8; ++kk) {
+          const uint32_t ah = tmem + tmem_a_hi(t) + kk * 8;
+          const uint32_t al = tmem + tmem_a_lo(t) + kk * 8;
+          uint64_t bd, bld;
+          if (g.trans_b) {
+            bd = smem_desc(b + kk * 32, 16, 1024, 2);
+            bld = smem_desc(bl + kk * 32, 16, 1024, 2);
+          } else {
+            bd = smem_desc(b + kk * 1024, TK * 128, 512, 1);
+            bld = smem_desc(bl + kk * 1024, TK * 128, 512, 1);
+          }
+          const uint32_t acc0 = kk > 0 ? 1u : 0u;
+          umma_tf32_pair_ts(dacc, ah, bd, idesc, acc0);
+          umma_tf32_pair_ts(dacc, ah, bld, idesc, 1u);
+          umma_tf32_pair_ts(dacc, al, bd, idesc, 1u);
+        }
+        umma_commit_both(&sh.empty[s]);
+        umma_commit_both(&sh.lofree[t]);
+        umma_commit_both(&sh.accf[ab]);
+      }
+      umma_commit_pair_local(&sh.drain);
+      (void)mbar_wait_bounded(&sh.drain, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- split + fold + epilogue
+    const int tt = threadIdx.x - 64;
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = quarter * 32 + lane;
+    const uint32_t conv0 = cluster_addr(&sh.conv[0], 0);   // the leader's barriers
+    const uint32_t acce0 = cluster_addr(&sh.acce[0], 0);
+    bool ok = true;
+    float acc[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+    auto fold = [&](int c) -> bool {
+      const int ab = c & 1;
+      if (!mbar_wait_bounded(&sh.accf[ab], (c >> 1) & 1)) return false;
+      tc_fence_after();
+      const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)ab * TN + half * 64;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float v[32];
+        tmem_ld_32x32b_x32(base + 32 * j, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[32 * j + i] += v[i];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acce0 + ab * (uint32_t)sizeof(uint64_t));
+      return true;
+    };
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % RS, t = kb % LS;
+      if (!mbar_wait_bounded(&sh.full[s], (kb / RS) & 1) ||
+          !mbar_wait_bounded(&sh.lofree[t], ((kb / LS) & 1) ^ 1)) {
+        if (lane == 0) fail_timeout(sh, g.dev_status);
+        ok = false;
+        break;
+      }
+      uint8_t *st = smem + (size_t)s * PSTAGE_BYTES;
+      split_half(st + TILE_BYTES, loring + (size_t)t * PB_BYTES, tt);
+      {
+        const int q = warp & 3, hf = (warp - 2) >> 2;
+        const int r = q * 32 + lane;
+        const uint8_t *rowp = st + r * 128;
+        const int kbase = klo + kb * TK + hf * 16;   // K index of this thread's first value
+        float hi[16], lo[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float4 v =
+              *reinterpret_cast<const float4 *>(rowp + (((hf * 4 + c) ^ (r & 7)) << 4));
+          hi[4 * c + 0] = v.x;
+          hi[4 * c + 1] = v.y;
+          hi[4 * c + 2] = v.z;
+          hi[4 * c + 3] = v.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float x = kbase + i < a_klo ? 0.f : hi[i];
+          hi[i] = tf32_rna(x);
+          lo[i] = tf32_rna(x - hi[i]);
+        }
+        const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + hf * 16;
+        tmem_st_32x32b_x16(lane_base + tmem_a_hi(t), hi);
+        tmem_st_32x32b_x16(lane_base + tmem_a_lo(t), lo);
+        tmem_wait_st();
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(conv0 + t * (uint32_t)sizeof(uint64_t));
+      if (kb >= 1 && !fold(kb - 1)) {
+        if (lane == 0) fail_timeout(sh, g.dev_status);
+        ok = false;
+        break;
+      }
+    }
+    if (ok && nk > 0 && !fold(nk - 1)) {
+      if (lane == 0) fail_timeout(sh, g.dev_status);
+      ok = false;
+    }
+    if (ok && load_c && !mbar_wait_bounded(&sh.cfull, 0)) {
+      if (lane == 0) fail_timeout(sh, g.dev_status);
+      ok = false;
+    }
+    if (ok && store) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int box = 2 * half + j;
+        const float *v = acc + 32 * j;
+        uint8_t *rp = ctile + box * C_BOX_BYTES + row * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float4 *q = reinterpret_cast<float4 *>(rp + ((c ^ (row & 7)) << 4));
+          float4 o;
+          if (load_c) {
+            const float4 cv = *q;
+            o.x = fmaf(g.alpha, v[4 * c + 0], g.beta * cv.x);
+            o.y = fmaf(g.alpha, v[4 * c + 1], g.beta * cv.y);
+            o.z = fmaf(g.alpha, v[4 * c + 2], g.beta * cv.z);
+            o.w = fmaf(g.alpha, v[4 * c + 3], g.beta * cv.w);
+          } else {
+            o = make_float4(g.alpha * v[4 * c], g.alpha * v[4 * c + 1], g.alpha * v[4 * c + 2],
+                            g.alpha * v[4 * c + 3]);
+          }
+          *q = o;
+        }
+      }
+      fence_async_smem();
+    }
+    epilogue_bar();
+    if (ok && store && tt == 0 && !*(volatile int *)&sh.abort) {
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        if (n0 + 32 * b < g.N) tma_store_2d(&tmC, ctile + b * C_BOX_BYTES, n0 + 32 * b, m0);
+      bulk_commit_and_wait_read();
+    }
+  }
+
+  // Neither CTA frees the pair's TMEM (or leaves) while the other may still
+  // use its barriers, shared memory or tensor memory.
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -506,25 +811,40 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
               g.prio);
     return GPTQ_OK;
   }
+  // Two or more row tiles: CTA pairs (the self-test keeps the single-CTA form).
+  const int mt = (g.M + TM - 1) / TM;
+  const bool pair = mt >= 2 && g.stall_after < 0;
   CUtensorMap ta, tb, tc;
   const CUtensorMapSwizzle kmaj = CU_TENSOR_MAP_SWIZZLE_128B;
   const CUtensorMapSwizzle mnmaj = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
+  const int bt_rows = pair ? PN / 2 : TN;   // rows of a B^T box (this CTA's columns)
   if (!make_map(&ta, g.A, g.M, g.K, g.lda, TM, kmaj) ||
-      !(trans_b ? make_map(&tb, g.B, g.N, g.K, g.ldb, TN, kmaj)
+      !(trans_b ? make_map(&tb, g.B, g.N, g.K, g.ldb, bt_rows, kmaj)
                 : make_map(&tb, g.B, g.K, g.N, g.ldb, TK, mnmaj)) ||
       !make_map(&tc, g.C, g.M, g.N, g.ldc, TM, kmaj)) {
     set_last_error_msg(__FILE__, __LINE__, "cuTensorMapEncodeTiled rejected a GEMM operand");
     return GPTQ_ERR_CUDA;
   }
-  static std::atomic<bool> attr[64] = {};
-  if (const int rc = ensure_smem_attr(gemm_tc_kernel, SMEM_BYTES, attr)) return rc;
   TcArgs a{g.M, g.N, g.K, g.C, g.ldc, g.alpha, g.beta, g.flags, trans_b ? 1 : 0, g.status,
            device_status_word(), g.stall_after};
-  dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM);
-  if (grid.y > 65535) return GPTQ_ERR_INVALID_ARG;
-  count_launch();
-  const cudaError_t e = launch_pdl_prio(g.prio, gemm_tc_kernel, grid, dim3(THREADS),
-                                        SMEM_BYTES, stream, ta, tb, tc, a);
+  cudaError_t e;
+  if (pair) {
+    static std::atomic<bool> attr[64] = {};
+    if (const int rc = ensure_smem_attr(gemm_pair_kernel, PSMEM_BYTES, attr)) return rc;
+    dim3 grid((g.N + PN - 1) / PN, 2 * ((mt + 1) / 2));
+    if (grid.y > 65535) return GPTQ_ERR_INVALID_ARG;
+    count_launch();
+    e = launch_pdl_prio(g.prio, gemm_pair_kernel, grid, dim3(THREADS), PSMEM_BYTES, stream, ta,
+                        tb, tc, a);
+  } else {
+    static std::atomic<bool> attr[64] = {};
+    if (const int rc = ensure_smem_attr(gemm_tc_kernel, SMEM_BYTES, attr)) return rc;
+    dim3 grid((g.N + TN - 1) / TN, mt);
+    if (grid.y > 65535) return GPTQ_ERR_INVALID_ARG;
+    count_launch();
+    e = launch_pdl_prio(g.prio, gemm_tc_kernel, grid, dim3(THREADS), SMEM_BYTES, stream, ta, tb,
+                        tc, a);
+  }
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     set_last_error(__FILE__, __LINE__, "kernel launch", e);

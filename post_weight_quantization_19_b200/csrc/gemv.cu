@@ -249,13 +249,15 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
   // start together otherwise alternate between all waiting and all
   // computing).
   const int per_row = (nchunk + 32 * PF - 1) / (32 * PF);
-  const int64_t my_rows = row1 - row0 > warp ? (row1 - row0 - warp + nwarps - 1) / nwarps : 0;
-  const int64_t steps = my_rows * per_row;
+  const int my_rows = row1 - row0 > warp ? (int)((row1 - row0 - warp + nwarps - 1) / nwarps) : 0;
+  const int steps = my_rows * per_row;
   uint32_t w[2][PF][BITS];
   float sc[2][PF], zr[2][PF];
-  auto fetch = [&](int64_t i, int buf) {
-    const int64_t row = row0 + warp + (i / per_row) * nwarps;
-    const int k0 = lane + (int)(i % per_row) * 32 * PF;
+  // (row, group) of the next step to fetch and of the step being computed
+  int fr = 0, fg = 0, cr = 0, cg = 0;
+  auto fetch = [&](int buf) {
+    const int64_t row = row0 + warp + (int64_t)fr * nwarps;
+    const int k0 = lane + fg * 32 * PF;
     const uint32_t *qrow = a.qweight + row * wpr;
 #pragma unroll
     for (int p = 0; p < PF; ++p) {
@@ -267,19 +269,22 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
       sc[buf][p] = in ? __ldg(a.scales + row * a.G + gi) : 0.f;
       zr[buf][p] = in ? (float)__ldg(a.zeros + row * a.G + gi) : 0.f;
     }
+    if (++fg == per_row) {
+      fg = 0;
+      ++fr;
+    }
   };
   float acc[MB];
 #pragma unroll
   for (int i = 0; i < MB; ++i) acc[i] = 0.f;
-  if (steps > 0) fetch(0, 0);
-  for (int64_t i = 0; i < steps; i += 2) {
+  if (steps > 0) fetch(0);
+  for (int i = 0; i < steps; i += 2) {
     // two steps per trip, so the double buffer is indexed by constants
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
-      const int64_t st = i + b;
-      if (st < steps) {
-        if (st + 1 < steps) fetch(st + 1, b ^ 1);
-        const int k0 = lane + (int)(st % per_row) * 32 * PF;
+      if (i + b < steps) {
+        if (i + b + 1 < steps) fetch(b ^ 1);
+        const int k0 = lane + cg * 32 * PF;
 #pragma unroll
         for (int p = 0; p < PF; ++p) {
           const int k = k0 + 32 * p;
@@ -292,8 +297,8 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
                 acc[q] = fmaf(sc[b][p], fmaf(-zr[b][p], xsum[q * nchunk + k], part[q]), acc[q]);
           }
         }
-        if (st % per_row == per_row - 1) {   // the row is complete
-          const int64_t row = row0 + warp + (st / per_row) * nwarps;
+        if (++cg == per_row) {   // the row is complete
+          const int64_t row = row0 + warp + (int64_t)cr * nwarps;
 #pragma unroll
           for (int q = 0; q < MB; ++q) {
             float v = acc[q];
@@ -302,6 +307,8 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
             if (lane == 0 && q < a.m) a.y[(int64_t)q * a.r + row] = v;
             acc[q] = 0.f;
           }
+          cg = 0;
+          ++cr;
         }
       }
     }

@@ -20,15 +20,15 @@
 //  * Warp roles: warp 0 issues TMA into a 6-stage ring (both CTAs; the
 //    loads complete on the leader CTA's barrier), warp 1 of the leader issues
 //    the pair's UMMAs into one of two 256-column TMEM accumulators and
-//    commits to barriers in both CTAs, warps 2..9 of each CTA drain its TMEM.
+//    commits to barriers in both CTAs, warps 2..17 of each CTA drain its TMEM.
 //  * Accuracy: the tensor core's fp32 accumulation is not rounded to nearest,
-//    so each TMEM accumulation chain is limited to 256 tokens and then folded
+//    so each TMEM accumulation chain is limited to 128 tokens and then folded
 //    into fp32 registers of the epilogue warps (double-buffered TMEM, so the
-//    tensor core keeps running while a chain is folded).  512-token chains
-//    bias H by about 2e-6, which the ill-conditioned Hessians of calibration
-//    sets with few tokens per feature turn into different codes; 128-token
-//    chains leave the fold (a TMEM read of the whole accumulator) too little
-//    time.
+//    tensor core keeps running while a chain is folded).  Longer chains bias
+//    H (about 2e-6 for 512 tokens, 1e-6 for 256), which the ill-conditioned
+//    Hessians of calibration sets with few tokens per feature turn into
+//    different codes.  Sixteen epilogue warps (four per TMEM lane quarter, 64
+//    columns each) fold a chain within the next chain's MMA time.
 //  * Pacing: X is read once from HBM only while the pairs working on tiles
 //    that share panels read the same token slab at about the same time.
 //    Every PACE_EVERY stages each pair's leader publishes how many stages it
@@ -90,7 +90,7 @@ constexpr int HM = 128;                          // tile rows per CTA (UMMA M = 
 constexpr int HN = 256;                          // tile cols  (UMMA N)
 constexpr int HK = 64;                           // tokens per pipeline stage
 constexpr int STAGES = 6;
-constexpr int FOLD = 4;                          // stages per TMEM chain (256 tokens)
+constexpr int FOLD = 2;                          // stages per TMEM chain (128 tokens)
 constexpr int PACE_EVERY = 64;                   // stages between progress reports
 constexpr int PACE_LAG = 160;                    // stages a pair may run ahead of the slowest
 constexpr int PACE_SPINS = 500;                  // bounded wait: about 1 ms, then go on
@@ -99,7 +99,8 @@ constexpr int BOX_BYTES = BOXF * HK * 2;         // 8 KB
 constexpr int A_BYTES = HM * HK * 2;             // 16 KB: this CTA's 128 rows
 constexpr int B_BYTES = (HN / 2) * HK * 2;       // 16 KB: this CTA's half of the columns
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 32 KB
-constexpr int NUM_EPI_WARPS = 8;
+constexpr int NUM_EPI_WARPS = 16;                // 4 per TMEM lane quarter, 64 columns each
+constexpr int EPI_COLS = HN / (NUM_EPI_WARPS / 4);   // accumulator columns per epilogue thread
 constexpr int THREADS = 32 * (2 + NUM_EPI_WARPS);
 constexpr uint32_t TMEM_COLS = 512;              // two 256-column accumulators
 constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024;
@@ -113,87 +114,6 @@ struct HessShared {
   uint32_t tmem_base;
   int abort;
 };
-
-// ---- CTA-pair primitives (cluster of two CTAs) ----
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Address of this CTA's shared variable `p` as seen in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-  return r;
-}
-
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr)
-               : "memory");
-}
-
-// 2-D TMA load into this CTA's shared memory whose completion is counted on an
-// mbarrier that may live in the other CTA of the pair.
-__device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorMap *tmap, int x,
-                                                 int y, uint32_t bar_addr) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar_addr)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(dst_smem)),
-               "r"(ncols)
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-
-// The pair's MMA: D (both CTAs' TMEM) (+)= A (both CTAs) * B (both halves).
-__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                              uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive once on the barrier at this offset in both CTAs when the pair's
-// earlier MMAs have completed.
-__device__ __forceinline__ void umma_commit_both(uint64_t *bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(smem_u32(bar)),
-      "h"((uint16_t)3)
-      : "memory");
-}
-
-// Arrive on this CTA's barrier only.
-__device__ __forceinline__ void umma_commit_pair_local(uint64_t *bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
 
 // Pair tile t -> (P, J): the 256 x 256 output block with rows 256 P .. and
 // columns 256 J .., J >= P.  Tiles are ordered in bands of BAND tile rows;
@@ -407,16 +327,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int ew = warp - 2;
     const int quarter = warp & 3;       // TMEM lanes this warp may access
-    const int half = ew >> 2;           // which 128 of the 256 tile columns
+    const int half = ew >> 2;           // which EPI_COLS of the 256 tile columns
     uint32_t abuf = 0, aphase = 0;
     bool ok = true;
     for (int t = pair; t < T && ok; t += npairs) {
       int P, J;
       tile_coords(t, nP, nJ, P, J);
       const int i0 = P * 2 * HM + (int)rank * HM, j0 = J * HN;
-      float acc[128];
+      float acc[EPI_COLS];
 #pragma unroll
-      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      for (int i = 0; i < EPI_COLS; ++i) acc[i] = 0.f;
       for (int c = 0; c < nchunks; ++c) {
         if (!mbar_wait_bounded(&sh.accf[abuf], aphase)) {
           if (lane == 0) record_timeout(status, sh);
@@ -424,10 +344,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + abuf * HN + half * 128;
+        const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + abuf * HN + half * EPI_COLS;
         // 32 columns per load, one wait per load
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
+        for (int p = 0; p < EPI_COLS / 32; ++p) {
           float v[32];
           tmem_ld_32x32b_x32(base + p * 32, v);
           tmem_wait_ld();
@@ -442,10 +362,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
       if (!ok) break;
       const int row = i0 + quarter * 32 + lane;
-      const int cb = j0 + half * 128;
+      const int cb = j0 + half * EPI_COLS;
       if (row < d) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
+        for (int i = 0; i < EPI_COLS; ++i) {
           const int col = cb + i;
           if (col < d && col >= row) {
             const float v = 2.f * acc[i];

@@ -101,3 +101,53 @@ def check_against_oracle(got: dict, ref: dict, W: np.ndarray, *, bits: int, grou
     assert zmatch >= CODE_MATCH
     stats["zero_match"] = zmatch
     return stats
+
+
+def reconcile_at_ties(got_codes: np.ndarray, W: np.ndarray, ref: dict, *, bits: int, group: int,
+                      block: int, max_ties: int = 16, delta: float = 1e-3) -> dict:
+    """Rows whose codes differ from the oracle's: the first difference must sit at
+    a rounding tie on the oracle's side (its value within ``delta`` code steps of a
+    half-integer), where either choice is correct; the row is then re-swept by the
+    oracle with the GPU's choice there, and so on until the row matches.
+
+    After one tie is decided differently, the compensation of every later column
+    of the row differs, so the rest of the row is another correct result, not a
+    rounding error.  ``ref`` is ``oracle.gptq_quantize_layer``'s result for the
+    rows of ``W`` (with "U", "perm", "scales", "zeros", "E", "What").  Returns
+    the number of rows followed and of ties followed."""
+    import oracle
+
+    perm = np.asarray(ref["perm"])
+    inv = np.argsort(perm)
+    U = ref["U"]
+    d = W.shape[1]
+    gi = np.zeros(d, dtype=np.int64) if group == -1 else np.arange(d) // group
+    rows_followed, ties = 0, 0
+    for i in range(W.shape[0]):
+        if np.array_equal(got_codes[i], ref["codes"][i]):
+            continue
+        rows_followed += 1
+        want = np.asarray(got_codes[i], dtype=np.int64)[perm]    # sweep order
+        forced = {}
+        Wi = np.asarray(W[i:i + 1], dtype=np.float64)[:, perm]
+        codes_p = ref["codes"][i][perm]
+        E = ref["E"][i:i + 1]
+        What_p = ref["What"][i:i + 1][:, perm]
+        sc, zr = ref["scales"][i:i + 1], ref["zeros"][i:i + 1]
+        for _ in range(max_ties + 1):
+            diff = np.where(codes_p != want)[0]
+            if diff.size == 0:
+                break
+            j = int(diff[0])
+            t = (What_p[0, j] + E[0, j] * U[j, j]) / sc[0, gi[j]] + zr[0, gi[j]]
+            off = abs(t - np.floor(t) - 0.5)
+            assert off <= delta, f"row {i}: column {perm[j]} differs {off:.2e} code steps from a tie"
+            assert abs(int(want[j]) - int(codes_p[j])) == 1, f"row {i}: not a neighbouring code"
+            forced[j] = np.array([want[j]])
+            ties += 1
+            c, sc, zr, What_p, E = oracle.gptq_sweep(Wi, U, bits, group, block, forced=forced)
+            codes_p = c[0]
+        else:
+            raise AssertionError(f"row {i}: more than {max_ties} ties to follow")
+        assert np.array_equal(codes_p, want), f"row {i} does not reconcile"
+    return {"rows": rows_followed, "ties": ties}

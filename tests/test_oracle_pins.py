@@ -341,6 +341,21 @@ def test_given_order_equals_the_computed_one_and_is_checked():
         oracle.gptq_quantize_layer(W, H, bits=3, group=32, perm=a["perm"])
 
 
+def test_forced_decisions_follow_the_given_codes():
+    # Forcing the sweep's own decisions reproduces it; forcing another code at
+    # one column changes that code and, through the compensation, only later
+    # columns.
+    X, W = make_problem(6, 64, 800, seed=43)
+    U = oracle.inverse_upper_cholesky(oracle.dampen(oracle.hessian(X), 0.01)[0])
+    c0, *_ = oracle.gptq_sweep(W, U, 3, -1, 32)
+    c1, *_ = oracle.gptq_sweep(W, U, 3, -1, 32, forced={10: c0[:, 10]})
+    np.testing.assert_array_equal(c0, c1)
+    alt = np.where(c0[:, 10] > 0, c0[:, 10] - 1, 1)
+    c2, *_ = oracle.gptq_sweep(W, U, 3, -1, 32, forced={10: alt})
+    np.testing.assert_array_equal(c2[:, :10], c0[:, :10])
+    np.testing.assert_array_equal(c2[:, 10], alt)
+
+
 def test_dequantised_output_is_on_the_grid():
     X, W = make_problem(8, 128, 600, seed=16)
     out = oracle.gptq_quantize_layer(W, oracle.hessian(X), bits=3, group=32)
