@@ -486,7 +486,7 @@ __device__ __forceinline__ void split_half(const uint8_t *tile, uint8_t *lo, int
   }
 }
 
-__global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, TcArgs g) {
   extern __shared__ uint8_t dyn_smem[];
@@ -791,6 +791,58 @@ bool make_map(CUtensorMap *m, const float *base, int64_t rows, int64_t cols, int
 
 }  // namespace
 
+// A pair launch: the cluster shape (two CTAs along y) is a launch attribute,
+// the kernel carries no compile-time cluster size. Programmatic serialisation
+// and the stream priority are asked for as well; where the driver refuses that
+// combination outside a capture, the launch is retried with fewer attributes
+// and the accepted set is kept for the process (mode 0: cluster, priority and
+// programmatic serialisation; 1: cluster and priority; 2: cluster only).
+static std::atomic<int> g_pair_mode{0};
+
+static cudaError_t launch_pair(int level, dim3 grid, cudaStream_t stream, const CUtensorMap &ta,
+                               const CUtensorMap &tb, const CUtensorMap &tc, const TcArgs &a) {
+  cudaError_t e = cudaErrorInvalidConfiguration;
+  for (int mode = g_pair_mode.load(std::memory_order_relaxed); mode < 3; ++mode) {
+    cudaLaunchAttribute attr[3];
+    unsigned n = 0;
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 1;
+    attr[n].val.clusterDim.y = 2;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+    if (mode < 2) {
+      attr[n].id = cudaLaunchAttributePriority;
+      attr[n].val.priority = launch_priority(level);
+      ++n;
+    }
+    if (mode < 1) {
+      attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[n].val.programmaticStreamSerializationAllowed = 1;
+      ++n;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = PSMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, ta, tb, tc, a);
+    if (e == cudaSuccess) {
+      g_pair_mode.store(mode, std::memory_order_relaxed);
+      return e;
+    }
+    if (e != cudaErrorInvalidClusterSize && e != cudaErrorNotSupported &&
+        e != cudaErrorInvalidValue)
+      return e;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+      return e;   // a refused launch inside a capture is not retried
+    (void)cudaGetLastError();
+  }
+  return e;
+}
+
 int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return GPTQ_OK;
   if (g.K % TK != 0 || g.lda % 4 || g.ldb % 4 || g.ldc % 4 ||
@@ -834,8 +886,7 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
     dim3 grid((g.N + PN - 1) / PN, 2 * ((mt + 1) / 2));
     if (grid.y > 65535) return GPTQ_ERR_INVALID_ARG;
     count_launch();
-    e = launch_pdl_prio(g.prio, gemm_pair_kernel, grid, dim3(THREADS), PSMEM_BYTES, stream, ta,
-                        tb, tc, a);
+    e = launch_pair(g.prio, grid, stream, ta, tb, tc, a);
   } else {
     static std::atomic<bool> attr[64] = {};
     if (const int rc = ensure_smem_attr(gemm_tc_kernel, SMEM_BYTES, attr)) return rc;

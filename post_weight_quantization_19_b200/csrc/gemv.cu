@@ -210,12 +210,12 @@ __device__ __forceinline__ void fold_chunk(const uint32_t (&w)[BITS], const floa
 }
 
 // Threads per CTA of the fold form: fewer for more vectors (registers).
-__host__ __device__ constexpr int fold_threads(int mb) { return mb <= 2 ? 768 : (mb == 4 ? 512 : 256); }
+__host__ __device__ constexpr int fold_threads(int mb) { return mb <= 2 ? 1024 : (mb == 4 ? 512 : 256); }
 
 template <int BITS, int MB>
 __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a) {
   using C = CodeAt<BITS>;
-  constexpr int PF = BITS == 8 ? 2 : 4;   // chunks per step (registers: 2 x PF x BITS words)
+  constexpr int PF = 4;
   extern __shared__ __align__(16) float fsm[];
   const int nchunk = a.d / 32;
   float *xs = fsm;                                   // [m][nchunk][32], swizzled, scaled
@@ -243,74 +243,45 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
   const int64_t row0 = (int64_t)blockIdx.x * a.r / gridDim.x;
   const int64_t row1 = (int64_t)(blockIdx.x + 1) * a.r / gridDim.x;
   const int64_t wpr = (int64_t)nchunk * BITS;
-  // This warp's work is a flat sequence of (row, PF-chunk group) steps; the
-  // loads of step i + 1 are issued before the arithmetic of step i, so each
-  // warp keeps a group of code words in flight while it computes (warps that
-  // start together otherwise alternate between all waiting and all
-  // computing).
-  const int per_row = (nchunk + 32 * PF - 1) / (32 * PF);
-  const int my_rows = row1 - row0 > warp ? (int)((row1 - row0 - warp + nwarps - 1) / nwarps) : 0;
-  const int steps = my_rows * per_row;
-  uint32_t w[2][PF][BITS];
-  float sc[2][PF], zr[2][PF];
-  // (row, group) of the next step to fetch and of the step being computed
-  int fr = 0, fg = 0, cr = 0, cg = 0;
-  auto fetch = [&](int buf) {
-    const int64_t row = row0 + warp + (int64_t)fr * nwarps;
-    const int k0 = lane + fg * 32 * PF;
+  for (int64_t row = row0 + warp; row < row1; row += nwarps) {
+    float acc[MB];
+#pragma unroll
+    for (int i = 0; i < MB; ++i) acc[i] = 0.f;
     const uint32_t *qrow = a.qweight + row * wpr;
+    const float *srow = a.scales + row * a.G;
+    const int32_t *zrow = a.zeros + row * a.G;
+    for (int k0 = lane; k0 < nchunk; k0 += 32 * PF) {
+      // every load of the PF chunks (codes, scale, zero) before any arithmetic
+      uint32_t w[PF][BITS];
+      float sc[PF], zr[PF];
 #pragma unroll
-    for (int p = 0; p < PF; ++p) {
-      const int k = k0 + 32 * p;
-      const bool in = k < nchunk;
+      for (int p = 0; p < PF; ++p) {
+        const int k = k0 + 32 * p;
+        const bool in = k < nchunk;
 #pragma unroll
-      for (int t = 0; t < BITS; ++t) w[buf][p][t] = in ? __ldg(qrow + (int64_t)k * BITS + t) : 0u;
-      const int gi = a.group > 0 ? (k * 32) / a.group : 0;
-      sc[buf][p] = in ? __ldg(a.scales + row * a.G + gi) : 0.f;
-      zr[buf][p] = in ? (float)__ldg(a.zeros + row * a.G + gi) : 0.f;
-    }
-    if (++fg == per_row) {
-      fg = 0;
-      ++fr;
-    }
-  };
-  float acc[MB];
+        for (int t = 0; t < BITS; ++t) w[p][t] = in ? __ldg(qrow + (int64_t)k * BITS + t) : 0u;
+        const int gi = a.group > 0 ? (k * 32) / a.group : 0;
+        sc[p] = in ? __ldg(srow + gi) : 0.f;
+        zr[p] = in ? (float)__ldg(zrow + gi) : 0.f;
+      }
 #pragma unroll
-  for (int i = 0; i < MB; ++i) acc[i] = 0.f;
-  if (steps > 0) fetch(0);
-  for (int i = 0; i < steps; i += 2) {
-    // two steps per trip, so the double buffer is indexed by constants
+      for (int p = 0; p < PF; ++p) {
+        const int k = k0 + 32 * p;
+        if (k < nchunk) {
+          float part[MB];
+          fold_chunk<BITS, MB>(w[p], xs, nchunk, k, part, a.m);
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      if (i + b < steps) {
-        if (i + b + 1 < steps) fetch(b ^ 1);
-        const int k0 = lane + cg * 32 * PF;
-#pragma unroll
-        for (int p = 0; p < PF; ++p) {
-          const int k = k0 + 32 * p;
-          if (k < nchunk) {
-            float part[MB];
-            fold_chunk<BITS, MB>(w[b][p], xs, nchunk, k, part, a.m);
-#pragma unroll
-            for (int q = 0; q < MB; ++q)
-              if (q < a.m)
-                acc[q] = fmaf(sc[b][p], fmaf(-zr[b][p], xsum[q * nchunk + k], part[q]), acc[q]);
-          }
-        }
-        if (++cg == per_row) {   // the row is complete
-          const int64_t row = row0 + warp + (int64_t)cr * nwarps;
-#pragma unroll
-          for (int q = 0; q < MB; ++q) {
-            float v = acc[q];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0 && q < a.m) a.y[(int64_t)q * a.r + row] = v;
-            acc[q] = 0.f;
-          }
-          cg = 0;
-          ++cr;
+          for (int i = 0; i < MB; ++i)
+            if (i < a.m) acc[i] = fmaf(sc[p], fmaf(-zr[p], xsum[i * nchunk + k], part[i]), acc[i]);
         }
       }
+    }
+#pragma unroll
+    for (int i = 0; i < MB; ++i) {
+      float v = acc[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0 && i < a.m) a.y[(int64_t)i * a.r + row] = v;
     }
   }
 }
