@@ -474,8 +474,10 @@ def run_ours(args, wl, rank: int, world: int, dist):
     # the sweep are phases whose tensor work is the 3xTF32 GEMM (with the leaves /
     # in-block sweep kernels on their critical path), timed by the phase events.
     kernel_of = {"hessian": "hessian_tc_kernel",
-                 "factor_U": "gemm_tc_kernel (factorisation phase: leaf_kernel chain + 3xTF32 GEMMs)",
-                 "sweep": "gemm_tc_kernel (sweep phase: trailing-update GEMMs + sweep_block_kernel)"}
+                 "factor_U": "gemm_pair_*_kernel / gemm_tc_kernel (factorisation phase: "
+                             "leaf_kernel chain + 3xTF32 GEMMs)",
+                 "sweep": "gemm_pair_*_kernel / gemm_tc_kernel (sweep phase: trailing-update "
+                          "GEMMs + sweep_block_kernel)"}
     dom = max((k for k in kernel_of if k in pr), key=lambda k: pr[k]["ms"])
     dp = pr[dom]
     roofline = {"bound": "tensor", "kernel": kernel_of[dom], "phase": dom,
@@ -496,6 +498,7 @@ def run_ours(args, wl, rank: int, world: int, dist):
         "phase_roofline": pr,
         "loss": loss,
         "gpu_launches": int(launches),
+        "gemm_pair_form": g.gptq_gemm_pair_form()[0],
         "clocks": clocks,
         "e2e": e2e,
     }

@@ -376,6 +376,27 @@ int gptq_last_phase_ms(float *ms, int n);
 int gptq_selftest_timeout(float *buf, gptq_stream_t stream);
 
 /*
+ * gptq_gemm_pair_form -- which launch form the library's two-CTA tensor-core
+ * product (the trailing updates and the factorisation's products with two or
+ * more 128-row tiles) runs in on the current device; a diagnostic with no page
+ * counterpart.  Before its first such product on a device the library tries,
+ * with launches that return at once, the forms
+ *   0  CTA pairs along y, cluster shape, priority and programmatic
+ *      serialisation given at launch;   1  the same, cluster shape only;
+ *   2  pairs along x, as 0;              3  pairs along x, as 1;
+ *   4  pairs along x with a compile-time cluster shape, priority and
+ *      programmatic serialisation;       5  the same as a plain launch;
+ * and keeps the first the driver accepts; 6 = none was accepted and every
+ * product runs on the one-CTA kernel (same results, lower throughput).
+ *
+ *   log, log_bytes  optional: receives the last probe's record, "form:result"
+ *                   per form tried (NUL-terminated, truncated to log_bytes).
+ * Returns the form (0 .. 6), or -1 when no product has probed this device yet
+ * (or no device is current).
+ */
+int gptq_gemm_pair_form(char *log, size_t log_bytes);
+
+/*
  * gptq_factor_plan -- a host-only diagnostic of the factorisation's schedule
  * (the Cholesky and inverse steps of gptq_quantize_layer): writes, without
  * touching a GPU, one text line per kernel the factorisation of a d x d H_d

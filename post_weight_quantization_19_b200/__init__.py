@@ -22,6 +22,7 @@ from .gptq import (  # noqa: F401
     gptq_dequant_gemv,
     gptq_factor,
     gptq_factor_plan,
+    gptq_gemm_pair_form,
     gptq_linear_fp16,
     gptq_pack,
     gptq_quantize_layer,

@@ -35,6 +35,8 @@
 // memory while the main loop runs (when beta != 0), updated there in place by
 // the epilogue warps, and stored with four bulk tensor stores, so every global
 // access of the epilogue is a full 128-byte line.
+#include <cstdio>
+#include <cstring>
 #include <mutex>
 
 #include "gptq_internal.h"
@@ -84,6 +86,7 @@ struct TcArgs {
   const int *status;
   int *dev_status;
   int stall_after;   // self-test only: the producer stops after this many K steps (-1: never)
+  int probe;         // launch-form probe: the kernel returns at entry
 };
 
 // The tensor core reads an fp32 operand in kind::tf32 as its top 19 bits
@@ -486,14 +489,17 @@ __device__ __forceinline__ void split_half(const uint8_t *tile, uint8_t *lo, int
   }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, TcArgs g) {
+// XL: the pair's two CTAs are neighbours along x (row tile from blockIdx.x),
+// else along y (row tile from blockIdx.y).
+template <bool XL>
+__device__ __forceinline__ void gemm_pair_body(const CUtensorMap &tmA, const CUtensorMap &tmB,
+                                               const CUtensorMap &tmC, const TcArgs &g) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ TcShared sh;
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
-  const int bn = blockIdx.x, bm = blockIdx.y;       // bm = 2 * pair + rank
+  const int bn = XL ? blockIdx.y : blockIdx.x;
+  const int bm = XL ? blockIdx.x : blockIdx.y;      // bm = 2 * pair + rank
   const int bm0 = bm - (int)rank;                   // the leader's row tile
   if ((g.flags & GEMM_UPPER_C) && bn < bm0) return; // both tiles below the diagonal
   const bool store = !((g.flags & GEMM_UPPER_C) && bn < bm);
@@ -756,6 +762,33 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+// The pair kernel in three launch forms: pairs along y or along x with the
+// cluster shape given at launch, and pairs along x with a compile-time
+// cluster shape.  A probe launch returns at entry.
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_pair_y_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmC, TcArgs g) {
+  if (g.probe) return;
+  gemm_pair_body<false>(tmA, tmB, tmC, g);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_pair_x_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmC, TcArgs g) {
+  if (g.probe) return;
+  gemm_pair_body<true>(tmA, tmB, tmC, g);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    gemm_pair_x2_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmC, TcArgs g) {
+  if (g.probe) return;
+  gemm_pair_body<true>(tmA, tmB, tmC, g);
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -791,56 +824,102 @@ bool make_map(CUtensorMap *m, const float *base, int64_t rows, int64_t cols, int
 
 }  // namespace
 
-// A pair launch: the cluster shape (two CTAs along y) is a launch attribute,
-// the kernel carries no compile-time cluster size. Programmatic serialisation
-// and the stream priority are asked for as well; where the driver refuses that
-// combination outside a capture, the launch is retried with fewer attributes
-// and the accepted set is kept for the process (mode 0: cluster, priority and
-// programmatic serialisation; 1: cluster and priority; 2: cluster only).
-static std::atomic<int> g_pair_mode{0};
+// Launch forms of the pair GEMM, tried in this order once per device by
+// probe launches (which return at entry) before the first pair-sized product:
+//   0  pairs along y, cluster shape, priority and programmatic serialisation
+//      given at launch;
+//   1  pairs along y, cluster shape only;
+//   2  pairs along x, cluster shape, priority and programmatic serialisation;
+//   3  pairs along x, cluster shape only;
+//   4  pairs along x, compile-time cluster shape, priority and programmatic
+//      serialisation;
+//   5  pairs along x, compile-time cluster shape, plain launch;
+//   6  none accepted: every product runs on the single-CTA kernel.
+constexpr int kPairForms = 6;
+static std::atomic<int> g_pair_form[64];   // form + 1 per device, 0 = not probed yet
+static std::mutex g_pair_mu;
+static char g_pair_log[512];               // the last probe: each form tried and its result
 
-static cudaError_t launch_pair(int level, dim3 grid, cudaStream_t stream, const CUtensorMap &ta,
-                               const CUtensorMap &tb, const CUtensorMap &tc, const TcArgs &a) {
-  cudaError_t e = cudaErrorInvalidConfiguration;
-  for (int mode = g_pair_mode.load(std::memory_order_relaxed); mode < 3; ++mode) {
-    cudaLaunchAttribute attr[3];
-    unsigned n = 0;
+static dim3 pair_grid(int form, int N, int mt) {
+  const unsigned cols = (unsigned)((N + PN - 1) / PN), rows = (unsigned)(2 * ((mt + 1) / 2));
+  return form <= 1 ? dim3(cols, rows) : dim3(rows, cols);
+}
+
+static cudaError_t launch_pair_form(int form, int level, dim3 grid, cudaStream_t stream,
+                             const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
+                             const TcArgs &a) {
+  if (form == 5) {
+    gemm_pair_x2_kernel<<<grid, THREADS, PSMEM_BYTES, stream>>>(ta, tb, tc, a);
+    return cudaGetLastError();
+  }
+  cudaLaunchAttribute attr[3];
+  unsigned n = 0;
+  if (form <= 3) {
     attr[n].id = cudaLaunchAttributeClusterDimension;
-    attr[n].val.clusterDim.x = 1;
-    attr[n].val.clusterDim.y = 2;
+    attr[n].val.clusterDim.x = form <= 1 ? 1 : 2;
+    attr[n].val.clusterDim.y = form <= 1 ? 2 : 1;
     attr[n].val.clusterDim.z = 1;
     ++n;
-    if (mode < 2) {
-      attr[n].id = cudaLaunchAttributePriority;
-      attr[n].val.priority = launch_priority(level);
-      ++n;
-    }
-    if (mode < 1) {
-      attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      attr[n].val.programmaticStreamSerializationAllowed = 1;
-      ++n;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = PSMEM_BYTES;
-    cfg.stream = stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = n;
-    e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, ta, tb, tc, a);
-    if (e == cudaSuccess) {
-      g_pair_mode.store(mode, std::memory_order_relaxed);
-      return e;
-    }
-    if (e != cudaErrorInvalidClusterSize && e != cudaErrorNotSupported &&
-        e != cudaErrorInvalidValue)
-      return e;
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
-      return e;   // a refused launch inside a capture is not retried
+  }
+  if (form == 0 || form == 2 || form == 4) {
+    attr[n].id = cudaLaunchAttributePriority;
+    attr[n].val.priority = launch_priority(level);
+    ++n;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = PSMEM_BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  if (form <= 1) return cudaLaunchKernelEx(&cfg, gemm_pair_y_kernel, ta, tb, tc, a);
+  if (form <= 3) return cudaLaunchKernelEx(&cfg, gemm_pair_x_kernel, ta, tb, tc, a);
+  return cudaLaunchKernelEx(&cfg, gemm_pair_x2_kernel, ta, tb, tc, a);
+}
+
+// The accepted form on this device (probing on `stream` the first time, which
+// must not be capturing), or -1 when it is not known and cannot be probed now.
+static int pair_form(cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kPairForms;
+  const int known = g_pair_form[dev].load(std::memory_order_acquire);
+  if (known > 0) return known - 1;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+    return -1;
+  std::lock_guard<std::mutex> lock(g_pair_mu);
+  if (g_pair_form[dev].load(std::memory_order_acquire) > 0)
+    return g_pair_form[dev].load() - 1;
+  static std::atomic<bool> attr_y[64] = {}, attr_x[64] = {}, attr_x2[64] = {};
+  if (ensure_smem_attr(gemm_pair_y_kernel, PSMEM_BYTES, attr_y) ||
+      ensure_smem_attr(gemm_pair_x_kernel, PSMEM_BYTES, attr_x) ||
+      ensure_smem_attr(gemm_pair_x2_kernel, PSMEM_BYTES, attr_x2)) {
+    (void)cudaGetLastError();
+    g_pair_form[dev].store(kPairForms + 1, std::memory_order_release);
+    return kPairForms;
+  }
+  CUtensorMap none;
+  std::memset(&none, 0, sizeof none);
+  TcArgs probe{};
+  probe.probe = 1;
+  int form = 0;
+  size_t used = 0;
+  g_pair_log[0] = 0;
+  for (; form < kPairForms; ++form) {
+    const cudaError_t e = launch_pair_form(form, 0, pair_grid(form, PN, 2), stream, none, none,
+                                           none, probe);
+    if (used < sizeof g_pair_log)
+      used += (size_t)std::snprintf(g_pair_log + used, sizeof g_pair_log - used, "%d:%s ", form,
+                                    cudaGetErrorName(e));
+    if (e == cudaSuccess) break;
     (void)cudaGetLastError();
   }
-  return e;
+  g_pair_form[dev].store(form + 1, std::memory_order_release);
+  return form;
 }
 
 int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
@@ -863,9 +942,11 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
               g.prio);
     return GPTQ_OK;
   }
-  // Two or more row tiles: CTA pairs (the self-test keeps the single-CTA form).
+  // Two or more row tiles: CTA pairs (the self-test keeps the single-CTA form),
+  // in the launch form this device accepts.
   const int mt = (g.M + TM - 1) / TM;
-  const bool pair = mt >= 2 && g.stall_after < 0;
+  const int form = mt >= 2 && g.stall_after < 0 ? pair_form(stream) : -1;
+  const bool pair = form >= 0 && form < kPairForms;
   CUtensorMap ta, tb, tc;
   const CUtensorMapSwizzle kmaj = CU_TENSOR_MAP_SWIZZLE_128B;
   const CUtensorMapSwizzle mnmaj = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
@@ -878,15 +959,13 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
     return GPTQ_ERR_CUDA;
   }
   TcArgs a{g.M, g.N, g.K, g.C, g.ldc, g.alpha, g.beta, g.flags, trans_b ? 1 : 0, g.status,
-           device_status_word(), g.stall_after};
+           device_status_word(), g.stall_after, 0};
   cudaError_t e;
   if (pair) {
-    static std::atomic<bool> attr[64] = {};
-    if (const int rc = ensure_smem_attr(gemm_pair_kernel, PSMEM_BYTES, attr)) return rc;
-    dim3 grid((g.N + PN - 1) / PN, 2 * ((mt + 1) / 2));
+    const dim3 grid = pair_grid(form, g.N, mt);
     if (grid.y > 65535) return GPTQ_ERR_INVALID_ARG;
     count_launch();
-    e = launch_pair(g.prio, grid, stream, ta, tb, tc, a);
+    e = launch_pair_form(form, g.prio, grid, stream, ta, tb, tc, a);
   } else {
     static std::atomic<bool> attr[64] = {};
     if (const int rc = ensure_smem_attr(gemm_tc_kernel, SMEM_BYTES, attr)) return rc;
@@ -920,4 +999,17 @@ extern "C" int gptq_selftest_timeout(float *buf, gptq_stream_t stream) {
   GemmArgs g{128, 128, 256, A, 256, B, 128, C, 128, 1.f, 0.f, 0, nullptr};
   g.stall_after = 2;
   return launch_gemm(g, false, (cudaStream_t)stream);
+}
+
+// The launch form of the two-CTA product accepted on the current device
+// (-1 before the first product with two or more row tiles has probed it).
+extern "C" int gptq_gemm_pair_form(char *log, size_t log_bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    (void)cudaGetLastError();
+    return -1;
+  }
+  std::lock_guard<std::mutex> lock(g_pair_mu);
+  if (log && log_bytes) std::snprintf(log, log_bytes, "%s", g_pair_log);
+  return g_pair_form[dev].load() - 1;
 }

@@ -151,8 +151,10 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS) gemv_kernel(GemvArgs a) {
 // two, so the product is exactly q_j x_j.  Codes whose offset is too high for
 // the exponent trick are read from the word shifted right once by FSH bits;
 // the two 3-bit codes that straddle words come from a funnel shift.  The sums
-// of x per chunk are staged too.  One warp per row; the grid holds one CTA per
-// SM with just enough warps that every warp takes the same number of rows.
+// of x per chunk are staged too.  A warp takes R rows at once (lane l the
+// chunks l, l + 32, ... of each), so every staged x value it reads serves R
+// rows; the grid holds one CTA per SM slot with just enough warps that every
+// warp takes the same number of row groups.
 
 template <int BITS>
 struct CodeAt {
@@ -172,16 +174,23 @@ __device__ __forceinline__ int xs_index(int k, int j) {   // swizzled float4 slo
   return k * 32 + ((((j >> 2) ^ (k & 7)) << 2) | (j & 3));
 }
 
-template <int BITS, int MB>
-__device__ __forceinline__ void fold_chunk(const uint32_t (&w)[BITS], const float *xs, int nchunk,
-                                           int k, float (&part)[MB], int m) {
+// R rows of one chunk at a time: each staged x value read from shared memory
+// serves R rows' codes (read once per row, x alone would cost 4 d bytes of
+// shared-memory traffic per row, more than the codes' share of HBM time).
+template <int BITS, int MB, int R>
+__device__ __forceinline__ void fold_chunk(const uint32_t (&w)[R][BITS], const float *xs,
+                                           int nchunk, int k, float (&part)[R][MB], int m) {
   using C = CodeAt<BITS>;
   constexpr uint32_t mask = (1u << BITS) - 1u;
-  uint32_t wsh[BITS];
+  uint32_t wsh[R][BITS];
 #pragma unroll
-  for (int t = 0; t < BITS; ++t) wsh[t] = w[t] >> C::FSH;
+  for (int r = 0; r < R; ++r)
 #pragma unroll
-  for (int i = 0; i < MB; ++i) part[i] = 0.f;
+    for (int t = 0; t < BITS; ++t) wsh[r][t] = w[r][t] >> C::FSH;
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int i = 0; i < MB; ++i) part[r][i] = 0.f;
 #pragma unroll
   for (int j4 = 0; j4 < 32; j4 += 4) {
     float4 xv[MB];
@@ -192,30 +201,41 @@ __device__ __forceinline__ void fold_chunk(const uint32_t (&w)[BITS], const floa
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
       const int j = j4 + jj;
-      uint32_t bits;
-      if (C::straddle(j))
-        bits = (__funnelshift_r(w[C::word(j)], w[C::word(j) + 1], C::off(j)) & mask) | 0x4B000000u;
-      else if (C::off(j) <= C::TOP)
-        bits = (w[C::word(j)] & (mask << C::off(j))) | 0x4B000000u;
-      else
-        bits = (wsh[C::word(j)] & (mask << C::eff(j))) | 0x4B000000u;
-      const float q = __uint_as_float(bits) - 8388608.f;   // q_j 2^eff, exact
 #pragma unroll
-      for (int i = 0; i < MB; ++i) {
-        const float xj = jj == 0 ? xv[i].x : jj == 1 ? xv[i].y : jj == 2 ? xv[i].z : xv[i].w;
-        part[i] = fmaf(q, xj, part[i]);
+      for (int r = 0; r < R; ++r) {
+        uint32_t bits;
+        if (C::straddle(j))
+          bits = (__funnelshift_r(w[r][C::word(j)], w[r][C::word(j) + 1], C::off(j)) & mask) |
+                 0x4B000000u;
+        else if (C::off(j) <= C::TOP)
+          bits = (w[r][C::word(j)] & (mask << C::off(j))) | 0x4B000000u;
+        else
+          bits = (wsh[r][C::word(j)] & (mask << C::eff(j))) | 0x4B000000u;
+        const float q = __uint_as_float(bits) - 8388608.f;   // q_j 2^eff, exact
+#pragma unroll
+        for (int i = 0; i < MB; ++i) {
+          const float xj = jj == 0 ? xv[i].x : jj == 1 ? xv[i].y : jj == 2 ? xv[i].z : xv[i].w;
+          part[r][i] = fmaf(q, xj, part[r][i]);
+        }
       }
     }
   }
 }
 
 // Threads per CTA of the fold form: fewer for more vectors (registers).
-__host__ __device__ constexpr int fold_threads(int mb) { return mb <= 2 ? 1024 : (mb == 4 ? 512 : 256); }
+__host__ __device__ constexpr int fold_threads(int mb) { return mb <= 2 ? 768 : (mb == 4 ? 512 : 256); }
 
-template <int BITS, int MB>
+// Chunks a lane fetches before any arithmetic: up to 32 words of codes, at
+// most 2 chunks when it takes 4 rows (registers).
+__host__ __device__ constexpr int fold_prefetch(int bits, int rows) {
+  return 32 / (bits * rows) < 1 ? 1
+         : (32 / (bits * rows) > (rows >= 4 ? 2 : 4) ? (rows >= 4 ? 2 : 4) : 32 / (bits * rows));
+}
+
+template <int BITS, int MB, int R>
 __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a) {
   using C = CodeAt<BITS>;
-  constexpr int PF = 4;
+  constexpr int PF = fold_prefetch(BITS, R);
   extern __shared__ __align__(16) float fsm[];
   const int nchunk = a.d / 32;
   float *xs = fsm;                                   // [m][nchunk][32], swizzled, scaled
@@ -243,46 +263,59 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
   const int64_t row0 = (int64_t)blockIdx.x * a.r / gridDim.x;
   const int64_t row1 = (int64_t)(blockIdx.x + 1) * a.r / gridDim.x;
   const int64_t wpr = (int64_t)nchunk * BITS;
-  for (int64_t row = row0 + warp; row < row1; row += nwarps) {
-    float acc[MB];
+  for (int64_t rb = row0 + (int64_t)warp * R; rb < row1; rb += (int64_t)nwarps * R) {
+    const int nr = row1 - rb < R ? (int)(row1 - rb) : R;   // rows of this group
+    float acc[R][MB];
 #pragma unroll
-    for (int i = 0; i < MB; ++i) acc[i] = 0.f;
-    const uint32_t *qrow = a.qweight + row * wpr;
-    const float *srow = a.scales + row * a.G;
-    const int32_t *zrow = a.zeros + row * a.G;
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int i = 0; i < MB; ++i) acc[r][i] = 0.f;
     for (int k0 = lane; k0 < nchunk; k0 += 32 * PF) {
       // every load of the PF chunks (codes, scale, zero) before any arithmetic
-      uint32_t w[PF][BITS];
-      float sc[PF], zr[PF];
+      uint32_t w[PF][R][BITS];
+      float sc[PF][R], zr[PF][R];
 #pragma unroll
       for (int p = 0; p < PF; ++p) {
         const int k = k0 + 32 * p;
-        const bool in = k < nchunk;
-#pragma unroll
-        for (int t = 0; t < BITS; ++t) w[p][t] = in ? __ldg(qrow + (int64_t)k * BITS + t) : 0u;
         const int gi = a.group > 0 ? (k * 32) / a.group : 0;
-        sc[p] = in ? __ldg(srow + gi) : 0.f;
-        zr[p] = in ? (float)__ldg(zrow + gi) : 0.f;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const bool in = k < nchunk && r < nr;
+          const int64_t row = rb + r;
+#pragma unroll
+          for (int t = 0; t < BITS; ++t)
+            w[p][r][t] = in ? __ldg(a.qweight + row * wpr + (int64_t)k * BITS + t) : 0u;
+          sc[p][r] = in ? __ldg(a.scales + row * a.G + gi) : 0.f;
+          zr[p][r] = in ? (float)__ldg(a.zeros + row * a.G + gi) : 0.f;
+        }
       }
 #pragma unroll
       for (int p = 0; p < PF; ++p) {
         const int k = k0 + 32 * p;
         if (k < nchunk) {
-          float part[MB];
-          fold_chunk<BITS, MB>(w[p], xs, nchunk, k, part, a.m);
+          float part[R][MB];
+          fold_chunk<BITS, MB, R>(w[p], xs, nchunk, k, part, a.m);
 #pragma unroll
-          for (int i = 0; i < MB; ++i)
-            if (i < a.m) acc[i] = fmaf(sc[p], fmaf(-zr[p], xsum[i * nchunk + k], part[i]), acc[i]);
+          for (int i = 0; i < MB; ++i) {
+            if (i < a.m) {
+              const float xk = xsum[i * nchunk + k];
+#pragma unroll
+              for (int r = 0; r < R; ++r)
+                acc[r][i] = fmaf(sc[p][r], fmaf(-zr[p][r], xk, part[r][i]), acc[r][i]);
+            }
+          }
         }
       }
     }
 #pragma unroll
-    for (int i = 0; i < MB; ++i) {
-      float v = acc[i];
+    for (int r = 0; r < R; ++r)
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0 && i < a.m) a.y[(int64_t)i * a.r + row] = v;
-    }
+      for (int i = 0; i < MB; ++i) {
+        float v = acc[r][i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && i < a.m && r < nr) a.y[(int64_t)i * a.r + rb + r] = v;
+      }
   }
 }
 
@@ -290,34 +323,51 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
 size_t fold_smem(const GemvArgs &a) { return (size_t)a.m * (a.d / 32) * 33 * sizeof(float); }
 constexpr size_t FOLD_SMEM_MAX = 220u << 10;
 
-template <int BITS, int MB>
-int gemv_launch_fold(const GemvArgs &a, cudaStream_t st) {
+// One CTA per SM slot; rows split evenly over the CTAs, taken R at a time by
+// the fewest warps that take every CTA's row groups in whole rounds.
+template <int BITS, int MB, int R>
+int gemv_launch_fold(const GemvArgs &a, int64_t ctas, cudaStream_t st) {
   static std::atomic<bool> attr[64] = {};
-  if (const int rc = ensure_smem_attr(gemv_fold_kernel<BITS, MB>, FOLD_SMEM_MAX, attr)) return rc;
-  const size_t smem = fold_smem(a);
-  const int sms = num_sms();
-  // CTAs per SM: as many as the staged x allows, up to 2048 threads
-  int per_sm = (int)(FOLD_SMEM_MAX / (smem > 0 ? smem : 1));
-  const int by_threads = 2048 / fold_threads(MB);
-  per_sm = per_sm < 1 ? 1 : (per_sm > by_threads ? by_threads : per_sm);
-  int64_t ctas = (int64_t)sms * per_sm;
-  if (ctas > a.r) ctas = a.r;
-  // warps per CTA: the fewest that take every CTA's rows in whole rounds
+  if (const int rc = ensure_smem_attr(gemv_fold_kernel<BITS, MB, R>, FOLD_SMEM_MAX, attr))
+    return rc;
   const int64_t rows = (a.r + ctas - 1) / ctas;
+  const int64_t groups = (rows + R - 1) / R;
   const int max_w = fold_threads(MB) / 32;
-  const int64_t rounds = (rows + max_w - 1) / max_w;
-  const int warps = (int)((rows + rounds - 1) / rounds);
-  gemv_fold_kernel<BITS, MB><<<(unsigned)ctas, 32 * warps, smem, st>>>(a);
+  const int64_t rounds = (groups + max_w - 1) / max_w;
+  const int warps = (int)((groups + rounds - 1) / rounds);
+  gemv_fold_kernel<BITS, MB, R><<<(unsigned)ctas, 32 * warps, fold_smem(a), st>>>(a);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }
 
+// Rows per warp group: the most (up to 4 for one vector, 2 for two or four,
+// 1 for eight) that still leave every SM a dozen warps.
 template <int BITS>
 int gemv_launch_fold_m(const GemvArgs &a, cudaStream_t st) {
-  if (a.m <= 1) return gemv_launch_fold<BITS, 1>(a, st);
-  if (a.m <= 2) return gemv_launch_fold<BITS, 2>(a, st);
-  if (a.m <= 4) return gemv_launch_fold<BITS, 4>(a, st);
-  return gemv_launch_fold<BITS, GEMV_MAX_M>(a, st);
+  const size_t smem = fold_smem(a);
+  const int sms = num_sms();
+  int per_sm = (int)(FOLD_SMEM_MAX / (smem > 0 ? smem : 1));
+  const int mb = a.m <= 1 ? 1 : a.m <= 2 ? 2 : a.m <= 4 ? 4 : GEMV_MAX_M;
+  const int by_threads = 2048 / fold_threads(mb);
+  per_sm = per_sm < 1 ? 1 : (per_sm > by_threads ? by_threads : per_sm);
+  int64_t ctas = (int64_t)sms * per_sm;
+  if (ctas > a.r) ctas = a.r;
+  const int64_t rows_per_sm = (a.r + sms - 1) / sms;
+  const int rmax = rows_per_sm >= 4 * 12 ? 4 : rows_per_sm >= 2 * 12 ? 2 : 1;
+  if (mb == 1) {
+    if (rmax >= 4) return gemv_launch_fold<BITS, 1, 4>(a, ctas, st);
+    if (rmax >= 2) return gemv_launch_fold<BITS, 1, 2>(a, ctas, st);
+    return gemv_launch_fold<BITS, 1, 1>(a, ctas, st);
+  }
+  if (mb == 2) {
+    if (rmax >= 2) return gemv_launch_fold<BITS, 2, 2>(a, ctas, st);
+    return gemv_launch_fold<BITS, 2, 1>(a, ctas, st);
+  }
+  if (mb == 4) {
+    if (rmax >= 2) return gemv_launch_fold<BITS, 4, 2>(a, ctas, st);
+    return gemv_launch_fold<BITS, 4, 1>(a, ctas, st);
+  }
+  return gemv_launch_fold<BITS, GEMV_MAX_M, 1>(a, ctas, st);
 }
 
 template <int BITS, int MB, bool SX>

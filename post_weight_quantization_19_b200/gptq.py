@@ -318,3 +318,12 @@ def gptq_factor_plan(d: int, outer_cols: int = 0, side_streams: bool = True) -> 
     buf = ctypes.create_string_buffer(n)
     lib.gptq_factor_plan(d, outer_cols, int(side_streams), buf, n)
     return buf.value.decode()
+
+
+def gptq_gemm_pair_form() -> tuple[int, str]:
+    """(form, probe record) of the two-CTA product on the current device: 0-5 a
+    cluster launch form, 6 the one-CTA fallback, -1 not probed yet."""
+    lib = _abi.load()
+    buf = ctypes.create_string_buffer(512)
+    form = lib.gptq_gemm_pair_form(buf, 512)
+    return int(form), buf.value.decode()

@@ -333,6 +333,18 @@ def test_zz_kernels_were_launched():
     assert g.gptq_launch_count() > 0
 
 
+def test_pair_gemm_launch_form_was_probed():
+    # After products with two or more row tiles the two-CTA kernel's launch form
+    # on this device is known, and it is one of the cluster forms.
+    import post_weight_quantization_19_b200 as g
+    X, W = make_problem(64, 512, 4096, seed=3)
+    gpu_layer(X, W, bits=4, group=128, block=128)   # factor products of 384 rows
+    form, log = g.gptq_gemm_pair_form()
+    print("gemm pair form", form, "probe:", log)
+    assert 0 <= form <= 6
+    assert form < 6, "no cluster launch form was accepted: " + log
+
+
 def test_graph_replay_matches_direct_launch():
     # On a non-default stream a repeated call is captured once and then replayed
     # as a CUDA graph; every call must give the same result as the first
