@@ -51,6 +51,8 @@ def _args():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--gemm-pair", action="store_true",
+                   help="run products of two or more row tiles on CTA pairs")
     return p.parse_args()
 
 
@@ -355,6 +357,7 @@ def run_ours(args, wl, rank: int, world: int, dist):
 
     import post_weight_quantization_19_b200 as g
 
+    g.gptq_set_gemm_pair(args.gemm_pair)
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -498,7 +501,7 @@ def run_ours(args, wl, rank: int, world: int, dist):
         "phase_roofline": pr,
         "loss": loss,
         "gpu_launches": int(launches),
-        "gemm_pair_form": g.gptq_gemm_pair_form()[0],
+        "gemm_pair": {"enabled": bool(args.gemm_pair), "form": g.gptq_gemm_pair_form()[0]},
         "clocks": clocks,
         "e2e": e2e,
     }

@@ -387,7 +387,8 @@ int gptq_selftest_timeout(float *buf, gptq_stream_t stream);
  *   4  pairs along x with a compile-time cluster shape, priority and
  *      programmatic serialisation;       5  the same as a plain launch;
  * and keeps the first the driver accepts; 6 = none was accepted and every
- * product runs on the one-CTA kernel (same results, lower throughput).
+ * product runs on the one-CTA kernel.  The probe runs only while the pairs
+ * are enabled (gptq_set_gemm_pair).
  *
  *   log, log_bytes  optional: receives the last probe's record, "form:result"
  *                   per form tried (NUL-terminated, truncated to log_bytes).
@@ -395,6 +396,18 @@ int gptq_selftest_timeout(float *buf, gptq_stream_t stream);
  * (or no device is current).
  */
 int gptq_gemm_pair_form(char *log, size_t log_bytes);
+
+/*
+ * gptq_set_gemm_pair -- chooses the kernel of the library's products with two
+ * or more 128-row tiles (trailing updates, factorisation products): nonzero =
+ * CTA pairs (tcgen05.mma.cta_group::2, M = 256, each CTA loading half of B) in
+ * the launch form gptq_gemm_pair_form reports; 0 = one CTA per 128 x 128 tile
+ * (the default, measured faster on the 4096- and 49152-wide layers).  Both
+ * give the same results up to the order of fp32 additions within a K step.
+ * Process-wide; takes effect for later calls (cached CUDA graphs are keyed by
+ * the setting).  Returns the previous setting (0 or 1).
+ */
+int gptq_set_gemm_pair(int enable);
 
 /*
  * gptq_factor_plan -- a host-only diagnostic of the factorisation's schedule

@@ -28,6 +28,7 @@ from .gptq import (  # noqa: F401
     gptq_quantize_layer,
     gptq_quantize_with_factor,
     gptq_quantize_workspace_bytes,
+    gptq_set_gemm_pair,
     gptq_set_phase_timing,
     gptq_solve_layer_host,
 )

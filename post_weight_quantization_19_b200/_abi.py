@@ -60,6 +60,7 @@ SIGNATURES = {
     "gptq_factor_plan": (c_size_t, [c_int64, c_int64, c_int, c_void_p, c_size_t]),
     "gptq_selftest_timeout": (c_int, [c_void_p, c_void_p]),
     "gptq_gemm_pair_form": (c_int, [c_void_p, c_size_t]),
+    "gptq_set_gemm_pair": (c_int, [c_int]),
 }
 
 

@@ -130,13 +130,14 @@ struct GraphKey {
   int options;
   int segment;   // phase of the solve this graph replays
   int device = -1;
+  int pair = 0;  // the two-CTA GEMM was enabled when the graph was captured
   bool operator==(const GraphKey &o) const {
     return W == o.W && H == o.H && W_hat == o.W_hat && qweight == o.qweight &&
            scales == o.scales && zeros == o.zeros && g_idx == o.g_idx && codes == o.codes &&
            ws == o.ws && ws_bytes == o.ws_bytes && stream == o.stream && r == o.r &&
            d == o.d && bits == o.bits && group == o.group && block == o.block &&
            memcmp(&damp, &o.damp, sizeof(float)) == 0 && options == o.options &&
-           segment == o.segment && device == o.device;
+           segment == o.segment && device == o.device && pair == o.pair;
   }
 };
 
@@ -156,6 +157,7 @@ constexpr size_t kMaxGraphs = 32;
 template <class F>
 int run_graph_cached(GraphKey key, cudaStream_t st, F &&enqueue) {
   GPTQ_CUDA_TRY(cudaGetDevice(&key.device));
+  key.pair = gemm_pair_enabled();
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (st == nullptr || cudaStreamIsCapturing(st, &cs) != cudaSuccess ||
       cs != cudaStreamCaptureStatusNone)

@@ -836,6 +836,7 @@ bool make_map(CUtensorMap *m, const float *base, int64_t rows, int64_t cols, int
 //   5  pairs along x, compile-time cluster shape, plain launch;
 //   6  none accepted: every product runs on the single-CTA kernel.
 constexpr int kPairForms = 6;
+static std::atomic<int> g_pair_enabled{0};  // gptq_set_gemm_pair
 static std::atomic<int> g_pair_form[64];   // form + 1 per device, 0 = not probed yet
 static std::mutex g_pair_mu;
 static char g_pair_log[512];               // the last probe: each form tried and its result
@@ -922,6 +923,8 @@ static int pair_form(cudaStream_t stream) {
   return form;
 }
 
+int gemm_pair_enabled() { return g_pair_enabled.load(std::memory_order_relaxed); }
+
 int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return GPTQ_OK;
   if (g.K % TK != 0 || g.lda % 4 || g.ldb % 4 || g.ldc % 4 ||
@@ -942,10 +945,13 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
               g.prio);
     return GPTQ_OK;
   }
-  // Two or more row tiles: CTA pairs (the self-test keeps the single-CTA form),
-  // in the launch form this device accepts.
+  // Two or more row tiles: CTA pairs when enabled (the self-test keeps the
+  // single-CTA form), in the launch form this device accepts.
   const int mt = (g.M + TM - 1) / TM;
-  const int form = mt >= 2 && g.stall_after < 0 ? pair_form(stream) : -1;
+  const int form =
+      mt >= 2 && g.stall_after < 0 && g_pair_enabled.load(std::memory_order_relaxed)
+          ? pair_form(stream)
+          : -1;
   const bool pair = form >= 0 && form < kPairForms;
   CUtensorMap ta, tb, tc;
   const CUtensorMapSwizzle kmaj = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -1012,4 +1018,10 @@ extern "C" int gptq_gemm_pair_form(char *log, size_t log_bytes) {
   std::lock_guard<std::mutex> lock(g_pair_mu);
   if (log && log_bytes) std::snprintf(log, log_bytes, "%s", g_pair_log);
   return g_pair_form[dev].load() - 1;
+}
+
+// Products with two or more row tiles on CTA pairs (nonzero) or on the one-CTA
+// kernel (0, the default: measured faster on the 4096- and 49152-wide layers).
+extern "C" int gptq_set_gemm_pair(int enable) {
+  return g_pair_enabled.exchange(enable ? 1 : 0);
 }

@@ -111,6 +111,9 @@ struct GemmArgs {
 };
 
 int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream);
+// Whether products with two or more row tiles may use the two-CTA kernel
+// (gptq_set_gemm_pair; off by default).
+int gemm_pair_enabled();
 
 int launch_damp(float *H, int64_t ld, int d, float damp, bool add_in_place, float *lambda,
                 cudaStream_t stream);

@@ -20,15 +20,16 @@
 //  * Warp roles: warp 0 issues TMA into a 6-stage ring (both CTAs; the
 //    loads complete on the leader CTA's barrier), warp 1 of the leader issues
 //    the pair's UMMAs into one of two 256-column TMEM accumulators and
-//    commits to barriers in both CTAs, warps 2..17 of each CTA drain its TMEM.
+//    commits to barriers in both CTAs, warps 2..9 of each CTA drain its TMEM.
 //  * Accuracy: the tensor core's fp32 accumulation is not rounded to nearest,
 //    so each TMEM accumulation chain is limited to 128 tokens and then folded
 //    into fp32 registers of the epilogue warps (double-buffered TMEM, so the
 //    tensor core keeps running while a chain is folded).  Longer chains bias
 //    H (about 2e-6 for 512 tokens, 1e-6 for 256), which the ill-conditioned
 //    Hessians of calibration sets with few tokens per feature turn into
-//    different codes.  Sixteen epilogue warps (four per TMEM lane quarter, 64
-//    columns each) fold a chain within the next chain's MMA time.
+//    different codes.  Eight epilogue warps (two per TMEM lane quarter, 128
+//    columns each) fold a chain with two 32-column TMEM loads in flight per
+//    wait (sixteen warps of 64 columns ran out of registers and were slower).
 //  * Pacing: X is read once from HBM only while the pairs working on tiles
 //    that share panels read the same token slab at about the same time.
 //    Every PACE_EVERY stages each pair's leader publishes how many stages it
@@ -99,7 +100,7 @@ constexpr int BOX_BYTES = BOXF * HK * 2;         // 8 KB
 constexpr int A_BYTES = HM * HK * 2;             // 16 KB: this CTA's 128 rows
 constexpr int B_BYTES = (HN / 2) * HK * 2;       // 16 KB: this CTA's half of the columns
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 32 KB
-constexpr int NUM_EPI_WARPS = 16;                // 4 per TMEM lane quarter, 64 columns each
+constexpr int NUM_EPI_WARPS = 8;                 // 2 per TMEM lane quarter, 128 columns each
 constexpr int EPI_COLS = HN / (NUM_EPI_WARPS / 4);   // accumulator columns per epilogue thread
 constexpr int THREADS = 32 * (2 + NUM_EPI_WARPS);
 constexpr uint32_t TMEM_COLS = 512;              // two 256-column accumulators
@@ -345,14 +346,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         tc_fence_after();
         const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + abuf * HN + half * EPI_COLS;
-        // 32 columns per load, one wait per load
+        // two 32-column loads in flight per wait
 #pragma unroll
-        for (int p = 0; p < EPI_COLS / 32; ++p) {
-          float v[32];
-          tmem_ld_32x32b_x32(base + p * 32, v);
+        for (int p = 0; p < EPI_COLS / 64; ++p) {
+          float v0[32], v1[32];
+          tmem_ld_32x32b_x32(base + p * 64, v0);
+          tmem_ld_32x32b_x32(base + p * 64 + 32, v1);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[p * 32 + i] += v[i];
+          for (int i = 0; i < 32; ++i) {
+            acc[p * 64 + i] += v0[i];
+            acc[p * 64 + 32 + i] += v1[i];
+          }
         }
         tc_fence_before();
         __syncwarp();

@@ -327,3 +327,9 @@ def gptq_gemm_pair_form() -> tuple[int, str]:
     buf = ctypes.create_string_buffer(512)
     form = lib.gptq_gemm_pair_form(buf, 512)
     return int(form), buf.value.decode()
+
+
+def gptq_set_gemm_pair(enable: bool) -> bool:
+    """Run products with two or more row tiles on CTA pairs (True) or one CTA per
+    tile (False, the default); returns the previous setting."""
+    return bool(_abi.load().gptq_set_gemm_pair(int(bool(enable))))

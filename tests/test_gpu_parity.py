@@ -333,16 +333,39 @@ def test_zz_kernels_were_launched():
     assert g.gptq_launch_count() > 0
 
 
-def test_pair_gemm_launch_form_was_probed():
+@pytest.fixture
+def gemm_pairs():
+    import post_weight_quantization_19_b200 as g
+    before = g.gptq_set_gemm_pair(True)
+    try:
+        yield g
+    finally:
+        g.gptq_set_gemm_pair(before)
+
+
+def test_pair_gemm_launch_form_was_probed(gemm_pairs):
     # After products with two or more row tiles the two-CTA kernel's launch form
     # on this device is known, and it is one of the cluster forms.
-    import post_weight_quantization_19_b200 as g
     X, W = make_problem(64, 512, 4096, seed=3)
     gpu_layer(X, W, bits=4, group=128, block=128)   # factor products of 384 rows
-    form, log = g.gptq_gemm_pair_form()
+    form, log = gemm_pairs.gptq_gemm_pair_form()
     print("gemm pair form", form, "probe:", log)
     assert 0 <= form <= 6
     assert form < 6, "no cluster launch form was accepted: " + log
+
+
+@pytest.mark.parametrize("case", [SOLVE_CASES[1], SOLVE_CASES[9], SOLVE_CASES[12],
+                                  SOLVE_CASES[13]],
+                         ids=lambda c: "r{}_d{}_a{}".format(c[0], c[1], int(c[6])))
+def test_pair_gemm_solve_matches_oracle(gemm_pairs, case):
+    # The same solves with every product of two or more row tiles on CTA pairs.
+    r, d, n, bits, group, block, act = case
+    X, W = make_problem(r, d, n, seed=r * 7 + d)
+    H32 = oracle.hessian(X).astype(np.float32)
+    got = gpu_layer(None, W, bits=bits, group=group, block=block, act_order=act, H32=H32)
+    ref = oracle.gptq_quantize_layer(W, H32.astype(np.float64), bits=bits, group=group,
+                                     block=block, act_order=act)
+    check_against_oracle(got, ref, W, bits=bits, group=group)
 
 
 def test_graph_replay_matches_direct_launch():
