@@ -42,6 +42,7 @@ struct GemvArgs {
   int d, group, G, m;
   const float *x;         // [m x d], 16-byte aligned rows
   float *y;               // [m x r]
+  uint32_t magic;         // 0x4B000000, the bits of 2^23, passed at run time (fold_chunk)
 };
 
 // One 32-code chunk: unpack with static shifts and accumulate MB dot products.
@@ -179,7 +180,8 @@ __device__ __forceinline__ int xs_index(int k, int j) {   // swizzled float4 slo
 // shared-memory traffic per row, more than the codes' share of HBM time).
 template <int BITS, int MB, int R>
 __device__ __forceinline__ void fold_chunk(const uint32_t (&w)[R][BITS], const float *xs,
-                                           int nchunk, int k, float (&part)[R][MB], int m) {
+                                           int nchunk, int k, float (&part)[R][MB], int m,
+                                           uint32_t magic) {
   using C = CodeAt<BITS>;
   constexpr uint32_t mask = (1u << BITS) - 1u;
   uint32_t wsh[R][BITS];
@@ -203,14 +205,16 @@ __device__ __forceinline__ void fold_chunk(const uint32_t (&w)[R][BITS], const f
       const int j = j4 + jj;
 #pragma unroll
       for (int r = 0; r < R; ++r) {
+        // (value & mask) | magic: one LOP3, the mask an immediate and magic a
+        // register (a run-time value, so it is not folded into a second one)
         uint32_t bits;
         if (C::straddle(j))
           bits = (__funnelshift_r(w[r][C::word(j)], w[r][C::word(j) + 1], C::off(j)) & mask) |
-                 0x4B000000u;
+                 magic;
         else if (C::off(j) <= C::TOP)
-          bits = (w[r][C::word(j)] & (mask << C::off(j))) | 0x4B000000u;
+          bits = (w[r][C::word(j)] & (mask << C::off(j))) | magic;
         else
-          bits = (wsh[r][C::word(j)] & (mask << C::eff(j))) | 0x4B000000u;
+          bits = (wsh[r][C::word(j)] & (mask << C::eff(j))) | magic;
         const float q = __uint_as_float(bits) - 8388608.f;   // q_j 2^eff, exact
 #pragma unroll
         for (int i = 0; i < MB; ++i) {
@@ -294,7 +298,7 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
         const int k = k0 + 32 * p;
         if (k < nchunk) {
           float part[R][MB];
-          fold_chunk<BITS, MB, R>(w[p], xs, nchunk, k, part, a.m);
+          fold_chunk<BITS, MB, R>(w[p], xs, nchunk, k, part, a.m, a.magic);
 #pragma unroll
           for (int i = 0; i < MB; ++i) {
             if (i < a.m) {
@@ -428,7 +432,7 @@ extern "C" int gptq_dequant_gemv(const int32_t *qweight, const float *scales,
       reinterpret_cast<uintptr_t>(y) % 4 || (g_idx && reinterpret_cast<uintptr_t>(g_idx) % 4))
     return GPTQ_ERR_INVALID_ARG;
   GemvArgs a{reinterpret_cast<const uint32_t *>(qweight), scales, zeros, g_idx, r, (int)d,
-             group, group < 0 ? 1 : (int)(d / group), (int)m, x, y};
+             group, group < 0 ? 1 : (int)(d / group), (int)m, x, y, 0x4B000000u};
   cudaStream_t st = (cudaStream_t)stream;
   switch (bits) {
     case 2: return gemv_launch<2>(a, st);

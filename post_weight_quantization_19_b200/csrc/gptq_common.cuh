@@ -230,9 +230,14 @@ __device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
   return r;
 }
 
+// Arrive on an mbarrier that may live in the other CTA of the pair (default
+// semantics: release at CTA scope).  The arrivals that use it follow a
+// completed tcgen05.wait and a tcgen05 fence (and a proxy fence for shared
+// memory the tensor core reads), so the data they publish is already complete;
+// release at cluster scope added a memory barrier to every arrival, the
+// largest stall of the Hessian's epilogue.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
 
 // 2-D TMA load into this CTA's shared memory whose completion is counted on an
