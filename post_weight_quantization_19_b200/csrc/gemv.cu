@@ -171,16 +171,14 @@ struct CodeAt {
   }
 };
 
-__device__ __forceinline__ int xs_index(int k, int j) {   // swizzled float4 slots of a chunk
-  return k * 32 + ((((j >> 2) ^ (k & 7)) << 2) | (j & 3));
-}
-
 // R rows of one chunk at a time: each staged x value read from shared memory
 // serves R rows' codes (read once per row, x alone would cost 4 d bytes of
 // shared-memory traffic per row, more than the codes' share of HBM time).
+// xk: the staged chunk of vector 0 (XPAD floats per chunk, vectors vstride
+// floats apart), read at compile-time offsets.
 template <int BITS, int MB, int R>
-__device__ __forceinline__ void fold_chunk(const uint32_t (&w)[R][BITS], const float *xs,
-                                           int nchunk, int k, float (&part)[R][MB], int m,
+__device__ __forceinline__ void fold_chunk(const uint32_t (&w)[R][BITS], const float *xk,
+                                           size_t vstride, float (&part)[R][MB], int m,
                                            uint32_t magic) {
   using C = CodeAt<BITS>;
   constexpr uint32_t mask = (1u << BITS) - 1u;
@@ -198,8 +196,8 @@ __device__ __forceinline__ void fold_chunk(const uint32_t (&w)[R][BITS], const f
     float4 xv[MB];
 #pragma unroll
     for (int i = 0; i < MB; ++i)
-      xv[i] = i < m ? *reinterpret_cast<const float4 *>(xs + (size_t)i * nchunk * 32 + xs_index(k, j4))
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      xv[i] = (i == 0 || i < m) ? *reinterpret_cast<const float4 *>(xk + i * vstride + j4)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
       const int j = j4 + jj;
@@ -242,12 +240,14 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
   constexpr int PF = fold_prefetch(BITS, R);
   extern __shared__ __align__(16) float fsm[];
   const int nchunk = a.d / 32;
-  float *xs = fsm;                                   // [m][nchunk][32], swizzled, scaled
-  float *xsum = fsm + (size_t)a.m * nchunk * 32;     // [m][nchunk]
+  const size_t vstride = (size_t)nchunk * XPAD;      // floats between staged vectors
+  float *xs = fsm;                                   // [m][nchunk][XPAD], scaled
+  float *xsum = fsm + (size_t)a.m * vstride;         // [m][nchunk]
   // stage x: thread per (vector, chunk)
   for (int idx = threadIdx.x; idx < a.m * nchunk; idx += blockDim.x) {
     const int i = idx / nchunk, k = idx - i * nchunk;
     const float *src = a.x + (int64_t)i * a.d + k * 32;
+    float *dst = xs + (size_t)idx * XPAD;
     float sum = 0.f;
 #pragma unroll
     for (int j4 = 0; j4 < 32; j4 += 4) {
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
       o.y = ldexpf(v.y, -C::eff(j4 + 1));
       o.z = ldexpf(v.z, -C::eff(j4 + 2));
       o.w = ldexpf(v.w, -C::eff(j4 + 3));
-      *reinterpret_cast<float4 *>(xs + (size_t)i * nchunk * 32 + xs_index(k, j4)) = o;
+      *reinterpret_cast<float4 *>(dst + j4) = o;
     }
     xsum[idx] = sum;
   }
@@ -267,8 +267,23 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
   const int64_t row0 = (int64_t)blockIdx.x * a.r / gridDim.x;
   const int64_t row1 = (int64_t)(blockIdx.x + 1) * a.r / gridDim.x;
   const int64_t wpr = (int64_t)nchunk * BITS;
+  // chunks per group: a power of two in every layout the library writes, else
+  // a division per chunk
+  const int cpg = a.group > 0 ? a.group / 32 : nchunk;
+  const int gshift = (cpg & (cpg - 1)) == 0 ? __ffs(cpg) - 1 : -1;
   for (int64_t rb = row0 + (int64_t)warp * R; rb < row1; rb += (int64_t)nwarps * R) {
     const int nr = row1 - rb < R ? (int)(row1 - rb) : R;   // rows of this group
+    // rows past the group's last read the last row again (their sums are dropped)
+    const uint32_t *qp[R];
+    const float *sp[R];
+    const int32_t *zp[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t row = rb + (r < nr ? r : nr - 1);
+      qp[r] = a.qweight + row * wpr;
+      sp[r] = a.scales + row * a.G;
+      zp[r] = a.zeros + row * a.G;
+    }
     float acc[R][MB];
 #pragma unroll
     for (int r = 0; r < R; ++r)
@@ -281,16 +296,15 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
 #pragma unroll
       for (int p = 0; p < PF; ++p) {
         const int k = k0 + 32 * p;
-        const int gi = a.group > 0 ? (k * 32) / a.group : 0;
+        const bool in = k < nchunk;
+        const int gi = !in ? 0 : (gshift >= 0 ? k >> gshift : k / cpg);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          const bool in = k < nchunk && r < nr;
-          const int64_t row = rb + r;
 #pragma unroll
           for (int t = 0; t < BITS; ++t)
-            w[p][r][t] = in ? __ldg(a.qweight + row * wpr + (int64_t)k * BITS + t) : 0u;
-          sc[p][r] = in ? __ldg(a.scales + row * a.G + gi) : 0.f;
-          zr[p][r] = in ? (float)__ldg(a.zeros + row * a.G + gi) : 0.f;
+            w[p][r][t] = in ? __ldg(qp[r] + (int64_t)k * BITS + t) : 0u;
+          sc[p][r] = in ? __ldg(sp[r] + gi) : 0.f;
+          zr[p][r] = in ? (float)__ldg(zp[r] + gi) : 0.f;
         }
       }
 #pragma unroll
@@ -298,10 +312,10 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
         const int k = k0 + 32 * p;
         if (k < nchunk) {
           float part[R][MB];
-          fold_chunk<BITS, MB, R>(w[p], xs, nchunk, k, part, a.m, a.magic);
+          fold_chunk<BITS, MB, R>(w[p], xs + (size_t)k * XPAD, vstride, part, a.m, a.magic);
 #pragma unroll
           for (int i = 0; i < MB; ++i) {
-            if (i < a.m) {
+            if (i == 0 || i < a.m) {
               const float xk = xsum[i * nchunk + k];
 #pragma unroll
               for (int r = 0; r < R; ++r)
@@ -324,8 +338,10 @@ __global__ void __launch_bounds__(fold_threads(MB)) gemv_fold_kernel(GemvArgs a)
 }
 
 // Shared memory of the fold form: staged x and its chunk sums.
-size_t fold_smem(const GemvArgs &a) { return (size_t)a.m * (a.d / 32) * 33 * sizeof(float); }
-constexpr size_t FOLD_SMEM_MAX = 220u << 10;
+size_t fold_smem(const GemvArgs &a) {
+  return (size_t)a.m * (a.d / 32) * (XPAD + 1) * sizeof(float);
+}
+constexpr size_t FOLD_SMEM_MAX = 227u << 10;   // the per-CTA limit (no static shared memory)
 
 // One CTA per SM slot; rows split evenly over the CTAs, taken R at a time by
 // the fewest warps that take every CTA's row groups in whole rounds.
@@ -344,8 +360,8 @@ int gemv_launch_fold(const GemvArgs &a, int64_t ctas, cudaStream_t st) {
   return GPTQ_OK;
 }
 
-// Rows per warp group: the most (up to 4 for one vector, 2 for two or four,
-// 1 for eight) that still leave every SM a dozen warps.
+// Rows per warp group: the most (up to 4 for one vector, 2 for two, 1 for
+// four or eight: registers) that still leave every SM a dozen warps.
 template <int BITS>
 int gemv_launch_fold_m(const GemvArgs &a, cudaStream_t st) {
   const size_t smem = fold_smem(a);
@@ -367,10 +383,7 @@ int gemv_launch_fold_m(const GemvArgs &a, cudaStream_t st) {
     if (rmax >= 2) return gemv_launch_fold<BITS, 2, 2>(a, ctas, st);
     return gemv_launch_fold<BITS, 2, 1>(a, ctas, st);
   }
-  if (mb == 4) {
-    if (rmax >= 2) return gemv_launch_fold<BITS, 4, 2>(a, ctas, st);
-    return gemv_launch_fold<BITS, 4, 1>(a, ctas, st);
-  }
+  if (mb == 4) return gemv_launch_fold<BITS, 4, 1>(a, ctas, st);
   return gemv_launch_fold<BITS, GEMV_MAX_M, 1>(a, ctas, st);
 }
 

@@ -432,7 +432,7 @@ def test_dequant_gemv_matches_oracle(case):
 def test_dequant_gemv_staged_and_direct_x(d, m, bits):
     # Without g_idx the kernel folds the zero point out of each 32-code chunk
     # and stages x (scaled per code position) with its chunk sums when
-    # m * d * 33/8 floats fit in 220 KB; otherwise x is read from global memory
+    # m * d * 37/32 floats fit in 227 KB; otherwise x is read from global memory
     # ((8192, 8) and (65536, 1)).  Both give the float64 oracle's product on
     # random packed rows.
     import post_weight_quantization_19_b200 as g
@@ -448,6 +448,30 @@ def test_dequant_gemv_staged_and_direct_x(d, m, bits):
     torch.cuda.synchronize()
     ref = oracle.dequant_gemv(qweight, scales, zeros, bits, group, x)
     assert np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max() <= 1e-5
+
+
+@pytest.mark.parametrize("r,d,m,bits,group", [(7500, 2112, 1, 4, 96), (7500, 2112, 1, 3, -1),
+                                               (7500, 2080, 2, 2, 32), (7403, 2080, 1, 8, 160)])
+def test_dequant_gemv_row_groups(r, d, m, bits, group):
+    # Enough rows that a warp takes 4 (one vector) or 2 (two) rows at once, with
+    # a ragged last group in most CTAs, a chunk count that is not a multiple of
+    # the prefetch depth, and groups of 3 and 5 chunks (not powers of two).
+    import post_weight_quantization_19_b200 as g
+    rng = np.random.default_rng(r + d + bits)
+    G = 1 if group < 0 else d // group
+    codes = rng.integers(0, 1 << bits, size=(r, d), dtype=np.uint8)
+    qweight = oracle.pack_rows(codes, bits)
+    del codes
+    scales = (rng.random((r, G)) * 0.01 + 1e-3).astype(np.float32)
+    zeros = rng.integers(0, 1 << bits, size=(r, G)).astype(np.int32)
+    x = rng.standard_normal((m, d)).astype(np.float32)
+    y = g.gptq_dequant_gemv(*(torch.from_numpy(a).cuda() for a in (qweight, scales, zeros, x)),
+                            bits, group)
+    torch.cuda.synchronize()
+    rows = np.sort(np.concatenate([np.arange(8), np.arange(r - 8, r),
+                                   rng.choice(r, 48, replace=False)]))
+    ref = oracle.dequant_gemv(qweight[rows], scales[rows], zeros[rows], bits, group, x)
+    assert np.abs(y.cpu().numpy()[:, rows] - ref).max() / np.abs(ref).max() <= 1e-5
 
 
 # ------------------------------------------------------------------ the layer run forward
