@@ -29,9 +29,10 @@
 // TMEM) and B's lo part into shared memory (B's hi part is the raw tile), so
 // the three MMAs of a K step read only B from shared memory -- shared-memory
 // bandwidth is what bounds this three-pass product.  Warp 0 issues TMA, warp 1
-// issues UMMA, warps 2..9 convert each landed stage, fold the previous step's
-// accumulator (two warps per TMEM lane quarter, 64 columns each) and end with
-// the epilogue.  The C tile travels by TMA both ways: it is loaded into shared
+// issues UMMA, warps 2..17 convert each landed stage, fold the previous step's
+// accumulator (four warps per TMEM lane quarter, 32 columns each) and end with
+// the epilogue (the CTA-pair kernel below has 8 such warps per CTA; with 8,
+// the conversion and fold of a step took longer than its MMAs).  The C tile travels by TMA both ways: it is loaded into shared
 // memory while the main loop runs (when beta != 0), updated there in place by
 // the epilogue warps, and stored with four bulk tensor stores, so every global
 // access of the epilogue is a full 128-byte line.
@@ -49,8 +50,10 @@ constexpr int RS = 3;                       // TMA ring: raw A, B tiles
 constexpr int LS = 3;                       // converted operands: B_lo (shared), A hi/lo (TMEM)
 constexpr int TILE_BYTES = 128 * TK * 4;    // 16 KB: 128 rows x 32 fp32
 constexpr int PAIR_BYTES = 2 * TILE_BYTES;  // A and B
-constexpr int THREADS = 32 * 10;
+constexpr int THREADS = 32 * 10;             // CTA-pair kernel: producer, MMA, 8 converter warps
 constexpr int CONV_THREADS = 256;
+constexpr int CONV1_THREADS = 512;           // one-CTA kernel: 16 converter/epilogue warps
+constexpr int THREADS1 = 64 + CONV1_THREADS;
 constexpr int C_BOX_BYTES = 128 * 32 * 4;  // one 32-column box of the C tile
 constexpr int C_BYTES = 4 * C_BOX_BYTES;    // 64 KB: the 128 x 128 C tile
 constexpr size_t SMEM_BYTES = (size_t)RS * PAIR_BYTES + (size_t)LS * TILE_BYTES + C_BYTES + 1024;
@@ -69,7 +72,7 @@ struct TcShared {
   uint64_t conv[LS];
   uint64_t lofree[LS];
   uint64_t accf[2];   // a K step's products are in accumulator b
-  uint64_t acce[2];   // accumulator b has been folded (8 converter warps)
+  uint64_t acce[2];   // accumulator b has been folded (by every converter warp)
   uint64_t drain;
   uint64_t cfull;
   uint32_t tmem_base;
@@ -135,6 +138,15 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const float (
       : "memory");
 }
 
+// 32 lanes x 8 columns of 32-bit TMEM <- 8 registers per thread.
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const float (&v)[8]) {
+  const uint32_t *u = reinterpret_cast<const uint32_t *>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -150,9 +162,10 @@ __device__ __forceinline__ void umma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
-// Epilogue warps only (warps 2..9).
+// Epilogue warps only (warps 2 .. 2 + N/32 - 1).
+template <int N = CONV_THREADS>
 __device__ __forceinline__ void epilogue_bar() {
-  asm volatile("bar.sync 1, %0;" ::"n"(CONV_THREADS) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void fail_timeout(TcShared &sh, int *dev_status) {
@@ -161,11 +174,12 @@ __device__ __forceinline__ void fail_timeout(TcShared &sh, int *dev_status) {
 }
 
 // lo part of one 16 KB B tile: lo = rna(x - trunc(x)), same (swizzled) layout.
+template <int N>
 __device__ __forceinline__ void split_tile(const uint8_t *tile, uint8_t *lo, int t) {
   const float4 *p = reinterpret_cast<const float4 *>(tile);
   float4 *q = reinterpret_cast<float4 *>(lo);
 #pragma unroll 4
-  for (int i = t; i < TILE_BYTES / 16; i += CONV_THREADS) {
+  for (int i = t; i < TILE_BYTES / 16; i += N) {
     const float4 v = p[i];
     float4 l;
     l.x = tf32_rna(v.x - tf32_trunc(v.x));
@@ -176,7 +190,7 @@ __device__ __forceinline__ void split_tile(const uint8_t *tile, uint8_t *lo, int
   }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS1, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, TcArgs g) {
   extern __shared__ uint8_t dyn_smem[];
@@ -200,12 +214,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&sh.empty[s], 1);
     }
     for (int t = 0; t < LS; ++t) {
-      mbar_init(&sh.conv[t], CONV_THREADS / 32);
+      mbar_init(&sh.conv[t], CONV1_THREADS / 32);
       mbar_init(&sh.lofree[t], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.accf[b], 1);
-      mbar_init(&sh.acce[b], CONV_THREADS / 32);
+      mbar_init(&sh.acce[b], CONV1_THREADS / 32);
     }
     mbar_init(&sh.drain, 1);
     mbar_init(&sh.cfull, 1);
@@ -321,28 +335,27 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------------- split + epilogue
+    // 16 warps: warp w reaches TMEM lanes 32 (w % 4) .. + 31 (its quarter) and
+    // takes part (w - 2) / 4 of the work: 8 of the 32 K values of A per step,
+    // 32 of the 128 accumulator columns, one 32-column box of C.
     const int tt = threadIdx.x - 64;
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;   // which 64 of the 128 columns
+    const int part = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;  // row of the tile = TMEM lane
     bool ok = true;
-    float acc[64];
+    float acc[32];
 #pragma unroll
-    for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
     // fold K step c (accumulator c & 1) into acc once its MMAs are complete
     auto fold = [&](int c) -> bool {
       const int ab = c & 1;
       if (!mbar_wait_bounded(&sh.accf[ab], (c >> 1) & 1)) return false;
       tc_fence_after();
-      const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)ab * TN + half * 64;
+      float v[32];
+      tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)ab * TN + part * 32, v);
+      tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float v[32];
-        tmem_ld_32x32b_x32(base + 32 * j, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[32 * j + i] += v[i];
-      }
+      for (int i = 0; i < 32; ++i) acc[i] += v[i];
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.acce[ab]);
@@ -357,33 +370,31 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       uint8_t *st = smem + (size_t)s * PAIR_BYTES;
-      split_tile(st + TILE_BYTES, loring + (size_t)t * TILE_BYTES, tt);
+      split_tile<CONV1_THREADS>(st + TILE_BYTES, loring + (size_t)t * TILE_BYTES, tt);
       {
-        // A: this thread's row (TMEM lane) and 16 of the 32 K values; the raw
+        // A: this thread's row (TMEM lane) and 8 of the 32 K values; the raw
         // tile is K-major with the 128-byte swizzle (16-byte chunk c of row r
         // at chunk position c ^ (r & 7)).
-        const int q = warp & 3, hf = (warp - 2) >> 2;
-        const int r = q * 32 + lane;
-        const uint8_t *rowp = st + r * 128;
-        float hi[16], lo[16];
+        const uint8_t *rowp = st + row * 128;
+        float hi[8], lo[8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           const float4 v =
-              *reinterpret_cast<const float4 *>(rowp + (((hf * 4 + c) ^ (r & 7)) << 4));
+              *reinterpret_cast<const float4 *>(rowp + (((part * 2 + c) ^ (row & 7)) << 4));
           hi[4 * c + 0] = v.x;
           hi[4 * c + 1] = v.y;
           hi[4 * c + 2] = v.z;
           hi[4 * c + 3] = v.w;
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 8; ++i) {
           const float x = hi[i];
           hi[i] = tf32_rna(x);
           lo[i] = tf32_rna(x - hi[i]);
         }
-        const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + hf * 16;
-        tmem_st_32x32b_x16(lane_base + tmem_a_hi(t), hi);
-        tmem_st_32x32b_x16(lane_base + tmem_a_lo(t), lo);
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + part * 8;
+        tmem_st_32x32b_x8(lane_base + tmem_a_hi(t), hi);
+        tmem_st_32x32b_x8(lane_base + tmem_a_lo(t), lo);
         tmem_wait_st();
       }
       fence_async_smem();
@@ -407,36 +418,31 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (ok) {
       // The C tile sits in shared memory as four 128-byte-swizzled boxes of
-      // 128 rows x 32 columns: 16-byte chunk c of a row is stored at chunk
-      // position c ^ (row & 7), so the 8 rows of each quarter-warp phase hit
-      // distinct banks.
+      // 128 rows x 32 columns (box = part): 16-byte chunk c of a row is stored
+      // at chunk position c ^ (row & 7), so the 8 rows of each quarter-warp
+      // phase hit distinct banks.
+      uint8_t *rp = ctile + part * C_BOX_BYTES + row * 128;
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int box = 2 * half + j;
-        const float *v = acc + 32 * j;   // compile-time offsets (unrolled): acc stays in registers
-        uint8_t *rp = ctile + box * C_BOX_BYTES + row * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float4 *q = reinterpret_cast<float4 *>(rp + ((c ^ (row & 7)) << 4));
-          float4 o;
-          if (load_c) {
-            const float4 cv = *q;
-            o.x = fmaf(g.alpha, v[4 * c + 0], g.beta * cv.x);
-            o.y = fmaf(g.alpha, v[4 * c + 1], g.beta * cv.y);
-            o.z = fmaf(g.alpha, v[4 * c + 2], g.beta * cv.z);
-            o.w = fmaf(g.alpha, v[4 * c + 3], g.beta * cv.w);
-          } else {
-            o = make_float4(g.alpha * v[4 * c], g.alpha * v[4 * c + 1], g.alpha * v[4 * c + 2],
-                            g.alpha * v[4 * c + 3]);
-          }
-          *q = o;
+      for (int c = 0; c < 8; ++c) {
+        float4 *q = reinterpret_cast<float4 *>(rp + ((c ^ (row & 7)) << 4));
+        float4 o;
+        if (load_c) {
+          const float4 cv = *q;
+          o.x = fmaf(g.alpha, acc[4 * c + 0], g.beta * cv.x);
+          o.y = fmaf(g.alpha, acc[4 * c + 1], g.beta * cv.y);
+          o.z = fmaf(g.alpha, acc[4 * c + 2], g.beta * cv.z);
+          o.w = fmaf(g.alpha, acc[4 * c + 3], g.beta * cv.w);
+        } else {
+          o = make_float4(g.alpha * acc[4 * c], g.alpha * acc[4 * c + 1],
+                          g.alpha * acc[4 * c + 2], g.alpha * acc[4 * c + 3]);
         }
+        *q = o;
       }
       fence_async_smem();
     }
     // ok is the same in every epilogue warp unless a wait timed out; the
     // barrier is passed by all of them either way.
-    epilogue_bar();
+    epilogue_bar<CONV1_THREADS>();
     if (ok && tt == 0 && !*(volatile int *)&sh.abort) {
 #pragma unroll
       for (int b = 0; b < 4; ++b)
@@ -743,7 +749,7 @@ __device__ __forceinline__ void gemm_pair_body(const CUtensorMap &tmA, const CUt
       }
       fence_async_smem();
     }
-    epilogue_bar();
+    epilogue_bar<CONV_THREADS>();
     if (ok && store && tt == 0 && !*(volatile int *)&sh.abort) {
 #pragma unroll
       for (int b = 0; b < 4; ++b)
@@ -978,7 +984,7 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
     dim3 grid((g.N + TN - 1) / TN, mt);
     if (grid.y > 65535) return GPTQ_ERR_INVALID_ARG;
     count_launch();
-    e = launch_pdl_prio(g.prio, gemm_tc_kernel, grid, dim3(THREADS), SMEM_BYTES, stream, ta, tb,
+    e = launch_pdl_prio(g.prio, gemm_tc_kernel, grid, dim3(THREADS1), SMEM_BYTES, stream, ta, tb,
                         tc, a);
   }
   if (e != cudaSuccess) {
