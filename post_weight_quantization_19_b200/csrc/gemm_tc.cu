@@ -52,11 +52,20 @@ constexpr int TILE_BYTES = 128 * TK * 4;    // 16 KB: 128 rows x 32 fp32
 constexpr int PAIR_BYTES = 2 * TILE_BYTES;  // A and B
 constexpr int THREADS = 32 * 10;             // CTA-pair kernel: producer, MMA, 8 converter warps
 constexpr int CONV_THREADS = 256;
-constexpr int CONV1_THREADS = 512;           // one-CTA kernel: 16 converter/epilogue warps
-constexpr int THREADS1 = 64 + CONV1_THREADS;
+// One-CTA kernel: 4 converter warps (one per TMEM lane quarter) run ahead of
+// the MMAs; 8 fold/epilogue warps drain one of three TMEM accumulators while
+// the tensor core fills the other two.
+constexpr int CONV1_THREADS = 128;
+constexpr int FOLD1_THREADS = 256;
+constexpr int THREADS1 = 64 + CONV1_THREADS + FOLD1_THREADS;
+constexpr int LS1 = 2;                       // converted stages of the one-CTA kernel
+constexpr int NACC1 = 3;                     // its accumulators
+
 constexpr int C_BOX_BYTES = 128 * 32 * 4;  // one 32-column box of the C tile
 constexpr int C_BYTES = 4 * C_BOX_BYTES;    // 64 KB: the 128 x 128 C tile
-constexpr size_t SMEM_BYTES = (size_t)RS * PAIR_BYTES + (size_t)LS * TILE_BYTES + C_BYTES + 1024;
+
+constexpr size_t SMEM1_BYTES =
+    (size_t)RS * PAIR_BYTES + (size_t)LS1 * TILE_BYTES + C_BYTES + 1024;
 // TMEM columns: two 128 x 128 accumulators (K steps alternate), then per
 // converted stage t the A hi part (32 columns, one K value each) and the A lo
 // part (32 columns).
@@ -65,14 +74,18 @@ constexpr uint32_t TMEM_A0 = 2 * TN;
 __host__ __device__ constexpr uint32_t tmem_a_hi(int t) { return TMEM_A0 + (uint32_t)t * 2 * TK; }
 __host__ __device__ constexpr uint32_t tmem_a_lo(int t) { return tmem_a_hi(t) + TK; }
 static_assert(TMEM_A0 + LS * 2 * TK <= TMEM_COLS, "TMEM budget");
+constexpr uint32_t TMEM1_A0 = NACC1 * TN;
+__host__ __device__ constexpr uint32_t tmem1_a_hi(int t) { return TMEM1_A0 + (uint32_t)t * 2 * TK; }
+__host__ __device__ constexpr uint32_t tmem1_a_lo(int t) { return tmem1_a_hi(t) + TK; }
+static_assert(TMEM1_A0 + LS1 * 2 * TK <= TMEM_COLS, "TMEM budget (one-CTA kernel)");
 
 struct TcShared {
   uint64_t full[RS];
   uint64_t empty[RS];
   uint64_t conv[LS];
   uint64_t lofree[LS];
-  uint64_t accf[2];   // a K step's products are in accumulator b
-  uint64_t acce[2];   // accumulator b has been folded (by every converter warp)
+  uint64_t accf[NACC1];   // a K step's products are in accumulator b
+  uint64_t acce[NACC1];   // accumulator b has been folded (by every fold warp)
   uint64_t drain;
   uint64_t cfull;
   uint32_t tmem_base;
@@ -213,13 +226,13 @@ __global__ void __launch_bounds__(THREADS1, 1)
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.empty[s], 1);
     }
-    for (int t = 0; t < LS; ++t) {
+    for (int t = 0; t < LS1; ++t) {
       mbar_init(&sh.conv[t], CONV1_THREADS / 32);
       mbar_init(&sh.lofree[t], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NACC1; ++b) {
       mbar_init(&sh.accf[b], 1);
-      mbar_init(&sh.acce[b], CONV1_THREADS / 32);
+      mbar_init(&sh.acce[b], FOLD1_THREADS / 32);
     }
     mbar_init(&sh.drain, 1);
     mbar_init(&sh.cfull, 1);
@@ -237,7 +250,7 @@ __global__ void __launch_bounds__(THREADS1, 1)
   __syncthreads();
   if (sh.abort) return;   // an earlier step failed: the same value in every thread
   uint8_t *loring = smem + (size_t)RS * PAIR_BYTES;       // B lo tiles
-  uint8_t *ctile = loring + (size_t)LS * TILE_BYTES;
+  uint8_t *ctile = loring + (size_t)LS1 * TILE_BYTES;
   const bool load_c = g.beta != 0.f;
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, TMEM_COLS);
@@ -293,10 +306,10 @@ __global__ void __launch_bounds__(THREADS1, 1)
     if (lane == 0) {
       const uint32_t idesc = instr_desc(2, 2, 0, g.trans_b ? 0u : 1u, TM, TN);
       for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % RS, t = kb % LS, ab = kb & 1;
-        // accumulator ab is free once the step two before has been folded
-        if ((kb >= 2 && !mbar_wait_bounded(&sh.acce[ab], ((kb >> 1) - 1) & 1)) ||
-            !mbar_wait_bounded(&sh.conv[t], (kb / LS) & 1)) {
+        const int s = kb % RS, t = kb % LS1, ab = kb % NACC1;
+        // accumulator ab is free once the step NACC1 before has been folded
+        if ((kb >= NACC1 && !mbar_wait_bounded(&sh.acce[ab], (kb / NACC1 - 1) & 1)) ||
+            !mbar_wait_bounded(&sh.conv[t], (kb / LS1) & 1)) {
           fail_timeout(sh, g.dev_status);
           break;
         }
@@ -309,8 +322,8 @@ __global__ void __launch_bounds__(THREADS1, 1)
           // A from TMEM: 8 K values = 8 columns per K step.
           // B^T: K-major, 8 tf32 = 32 bytes per K step inside the swizzle atom.
           // B row-major: MN-major, 8 K rows (1024 bytes) per K step.
-          const uint32_t ah = tmem + tmem_a_hi(t) + kk * 8;
-          const uint32_t al = tmem + tmem_a_lo(t) + kk * 8;
+          const uint32_t ah = tmem + tmem1_a_hi(t) + kk * 8;
+          const uint32_t al = tmem + tmem1_a_lo(t) + kk * 8;
           uint64_t bd, bld;
           if (g.trans_b) {
             bd = smem_desc(b + kk * 32, 16, 1024, 2);
@@ -333,84 +346,85 @@ __global__ void __launch_bounds__(THREADS1, 1)
       umma_commit(&sh.drain);
       (void)mbar_wait_bounded(&sh.drain, 0);
     }
-  } else {
-    // ---------------------------------------------------------------- split + epilogue
-    // 16 warps: warp w reaches TMEM lanes 32 (w % 4) .. + 31 (its quarter) and
-    // takes part (w - 2) / 4 of the work: 8 of the 32 K values of A per step,
-    // 32 of the 128 accumulator columns, one 32-column box of C.
+  } else if (warp < 2 + CONV1_THREADS / 32) {
+    // ---------------------------------------------------------------- conversion
+    // Warps 2..5 (one per TMEM lane quarter): each thread converts its A row
+    // (all 32 K values) into TMEM and a quarter of B's lo part, as far ahead
+    // of the MMAs as the converted stages allow.
     const int tt = threadIdx.x - 64;
-    const int quarter = warp & 3;
-    const int part = (warp - 2) >> 2;
-    const int row = quarter * 32 + lane;  // row of the tile = TMEM lane
-    bool ok = true;
-    float acc[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-    // fold K step c (accumulator c & 1) into acc once its MMAs are complete
-    auto fold = [&](int c) -> bool {
-      const int ab = c & 1;
-      if (!mbar_wait_bounded(&sh.accf[ab], (c >> 1) & 1)) return false;
-      tc_fence_after();
-      float v[32];
-      tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)ab * TN + part * 32, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] += v[i];
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.acce[ab]);
-      return true;
-    };
+    const int row = (warp & 3) * 32 + lane;   // row of the tile = TMEM lane
     for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % RS, t = kb % LS;
+      const int s = kb % RS, t = kb % LS1;
       if (!mbar_wait_bounded(&sh.full[s], (kb / RS) & 1) ||
-          !mbar_wait_bounded(&sh.lofree[t], ((kb / LS) & 1) ^ 1)) {
+          !mbar_wait_bounded(&sh.lofree[t], ((kb / LS1) & 1) ^ 1)) {
         if (lane == 0) fail_timeout(sh, g.dev_status);
-        ok = false;
         break;
       }
       uint8_t *st = smem + (size_t)s * PAIR_BYTES;
       split_tile<CONV1_THREADS>(st + TILE_BYTES, loring + (size_t)t * TILE_BYTES, tt);
-      {
-        // A: this thread's row (TMEM lane) and 8 of the 32 K values; the raw
-        // tile is K-major with the 128-byte swizzle (16-byte chunk c of row r
-        // at chunk position c ^ (r & 7)).
-        const uint8_t *rowp = st + row * 128;
-        float hi[8], lo[8];
+      // A: the raw tile is K-major with the 128-byte swizzle (16-byte chunk c
+      // of row r at chunk position c ^ (r & 7)).
+      const uint8_t *rowp = st + row * 128;
+      const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+      for (int h = 0; h < 2; ++h) {
+        float hi[16], lo[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
           const float4 v =
-              *reinterpret_cast<const float4 *>(rowp + (((part * 2 + c) ^ (row & 7)) << 4));
+              *reinterpret_cast<const float4 *>(rowp + (((h * 4 + c) ^ (row & 7)) << 4));
           hi[4 * c + 0] = v.x;
           hi[4 * c + 1] = v.y;
           hi[4 * c + 2] = v.z;
           hi[4 * c + 3] = v.w;
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 16; ++i) {
           const float x = hi[i];
           hi[i] = tf32_rna(x);
           lo[i] = tf32_rna(x - hi[i]);
         }
-        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + part * 8;
-        tmem_st_32x32b_x8(lane_base + tmem_a_hi(t), hi);
-        tmem_st_32x32b_x8(lane_base + tmem_a_lo(t), lo);
-        tmem_wait_st();
+        tmem_st_32x32b_x16(lane_base + tmem1_a_hi(t) + h * 16, hi);
+        tmem_st_32x32b_x16(lane_base + tmem1_a_lo(t) + h * 16, lo);
       }
+      tmem_wait_st();
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.conv[t]);
-      // the previous step's products are (about) done by now
-      if (kb >= 1 && !fold(kb - 1)) {
+    }
+  } else {
+    // ---------------------------------------------------------------- fold + epilogue
+    // Warps 6..13: two per TMEM lane quarter, 64 accumulator columns each.
+    const int ft = threadIdx.x - 64 - CONV1_THREADS;
+    const int quarter = warp & 3;
+    const int half = (warp - 2 - CONV1_THREADS / 32) >> 2;
+    const int row = quarter * 32 + lane;
+    bool ok = true;
+    float acc[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+    for (int c = 0; c < nk; ++c) {
+      const int ab = c % NACC1;
+      if (!mbar_wait_bounded(&sh.accf[ab], (c / NACC1) & 1)) {
         if (lane == 0) fail_timeout(sh, g.dev_status);
         ok = false;
         break;
       }
-    }
-    if (ok && nk > 0 && !fold(nk - 1)) {
-      if (lane == 0) fail_timeout(sh, g.dev_status);
-      ok = false;
+      tc_fence_after();
+      const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)ab * TN + half * 64;
+      float v0[32], v1[32];
+      tmem_ld_32x32b_x32(base, v0);
+      tmem_ld_32x32b_x32(base + 32, v1);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.acce[ab]);   // the registers hold it now
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        acc[i] += v0[i];
+        acc[32 + i] += v1[i];
+      }
     }
     if (ok && load_c && !mbar_wait_bounded(&sh.cfull, 0)) {
       if (lane == 0) fail_timeout(sh, g.dev_status);
@@ -418,32 +432,37 @@ __global__ void __launch_bounds__(THREADS1, 1)
     }
     if (ok) {
       // The C tile sits in shared memory as four 128-byte-swizzled boxes of
-      // 128 rows x 32 columns (box = part): 16-byte chunk c of a row is stored
-      // at chunk position c ^ (row & 7), so the 8 rows of each quarter-warp
-      // phase hit distinct banks.
-      uint8_t *rp = ctile + part * C_BOX_BYTES + row * 128;
+      // 128 rows x 32 columns: 16-byte chunk c of a row is stored at chunk
+      // position c ^ (row & 7), so the 8 rows of each quarter-warp phase hit
+      // distinct banks.
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float4 *q = reinterpret_cast<float4 *>(rp + ((c ^ (row & 7)) << 4));
-        float4 o;
-        if (load_c) {
-          const float4 cv = *q;
-          o.x = fmaf(g.alpha, acc[4 * c + 0], g.beta * cv.x);
-          o.y = fmaf(g.alpha, acc[4 * c + 1], g.beta * cv.y);
-          o.z = fmaf(g.alpha, acc[4 * c + 2], g.beta * cv.z);
-          o.w = fmaf(g.alpha, acc[4 * c + 3], g.beta * cv.w);
-        } else {
-          o = make_float4(g.alpha * acc[4 * c], g.alpha * acc[4 * c + 1],
-                          g.alpha * acc[4 * c + 2], g.alpha * acc[4 * c + 3]);
+      for (int j = 0; j < 2; ++j) {
+        const int box = 2 * half + j;
+        const float *v = acc + 32 * j;   // compile-time offsets (unrolled): acc stays in registers
+        uint8_t *rp = ctile + box * C_BOX_BYTES + row * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float4 *q = reinterpret_cast<float4 *>(rp + ((c ^ (row & 7)) << 4));
+          float4 o;
+          if (load_c) {
+            const float4 cv = *q;
+            o.x = fmaf(g.alpha, v[4 * c + 0], g.beta * cv.x);
+            o.y = fmaf(g.alpha, v[4 * c + 1], g.beta * cv.y);
+            o.z = fmaf(g.alpha, v[4 * c + 2], g.beta * cv.z);
+            o.w = fmaf(g.alpha, v[4 * c + 3], g.beta * cv.w);
+          } else {
+            o = make_float4(g.alpha * v[4 * c], g.alpha * v[4 * c + 1], g.alpha * v[4 * c + 2],
+                            g.alpha * v[4 * c + 3]);
+          }
+          *q = o;
         }
-        *q = o;
       }
       fence_async_smem();
     }
-    // ok is the same in every epilogue warp unless a wait timed out; the
-    // barrier is passed by all of them either way.
-    epilogue_bar<CONV1_THREADS>();
-    if (ok && tt == 0 && !*(volatile int *)&sh.abort) {
+    // ok is the same in every fold warp unless a wait timed out; the barrier
+    // is passed by all of them either way.
+    epilogue_bar<FOLD1_THREADS>();
+    if (ok && ft == 0 && !*(volatile int *)&sh.abort) {
 #pragma unroll
       for (int b = 0; b < 4; ++b)
         if (n0 + 32 * b < g.N) tma_store_2d(&tmC, ctile + b * C_BOX_BYTES, n0 + 32 * b, m0);
@@ -980,11 +999,11 @@ int launch_gemm(const GemmArgs &g, bool trans_b, cudaStream_t stream) {
     e = launch_pair_form(form, g.prio, grid, stream, ta, tb, tc, a);
   } else {
     static std::atomic<bool> attr[64] = {};
-    if (const int rc = ensure_smem_attr(gemm_tc_kernel, SMEM_BYTES, attr)) return rc;
+    if (const int rc = ensure_smem_attr(gemm_tc_kernel, SMEM1_BYTES, attr)) return rc;
     dim3 grid((g.N + TN - 1) / TN, mt);
     if (grid.y > 65535) return GPTQ_ERR_INVALID_ARG;
     count_launch();
-    e = launch_pdl_prio(g.prio, gemm_tc_kernel, grid, dim3(THREADS1), SMEM_BYTES, stream, ta, tb,
+    e = launch_pdl_prio(g.prio, gemm_tc_kernel, grid, dim3(THREADS1), SMEM1_BYTES, stream, ta, tb,
                         tc, a);
   }
   if (e != cudaSuccess) {
