@@ -151,15 +151,6 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const float (
       : "memory");
 }
 
-// 32 lanes x 8 columns of 32-bit TMEM <- 8 registers per thread.
-__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const float (&v)[8]) {
-  const uint32_t *u = reinterpret_cast<const uint32_t *>(v);
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
-      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7])
-      : "memory");
-}
-
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
