@@ -75,8 +75,15 @@ KERNEL_TRAFFIC = {
         "kernel": "hessian_tc_kernel",
         "sources": ["post_weight_quantization_19_b200/csrc/hessian_tc.cu",
                     "post_weight_quantization_19_b200/csrc/gptq_common.cuh"],
-        "sha256": "53c32a78488a3a1be69bbb69f51edb36d0ae8754eef01037ae5f30d86b1c4e17",
-        "bytes": 7386331136 + 51261184,
+        "sha256": "c1316476f1761699e7b737b98978fa5e2f66baf5e0da481d69f9379a7422d40c",
+        "bytes": 4269406976 + 42836480,
+    },
+    "opt175b_fc2_12288x49152": {
+        "kernel": "hessian_tc_kernel",
+        "sources": ["post_weight_quantization_19_b200/csrc/hessian_tc.cu",
+                    "post_weight_quantization_19_b200/csrc/gptq_common.cuh"],
+        "sha256": "c1316476f1761699e7b737b98978fa5e2f66baf5e0da481d69f9379a7422d40c",
+        "bytes": 175541137408 + 9743772160,
     },
 }
 
@@ -473,6 +480,8 @@ def run_ours(args, wl, rank: int, world: int, dist):
         if vals:
             phases_ms[nm] = round(float(np.mean(vals)), 4)
     pr = phase_rooflines(wl, phases_ms, peaks, tc_peak)
+    if "hessian" in pr:   # DRAM bytes of the one-launch phase, when captured on this source
+        pr["hessian"]["traffic"] = _traffic(wl)
     # The dominant kernel: the Hessian is one launch per step; the factorisation and
     # the sweep are phases whose tensor work is the 3xTF32 GEMM (with the leaves /
     # in-block sweep kernels on their critical path), timed by the phase events.
