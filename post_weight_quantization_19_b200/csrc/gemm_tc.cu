@@ -21,8 +21,8 @@
 // sweep's compensation, whose errors the ill-conditioned Hessians of
 // calibration sets with few tokens per feature amplify.
 //
-// Tile 128 x 128 x 32 per stage: a 3-deep TMA ring of raw A/B tiles and a
-// 3-deep ring of converted operands.  A (and B^T) are K-major with a 128-byte
+// Tile 128 x 128 x 32 per stage: a 4-deep TMA ring of raw A/B tiles and a
+// 2-deep ring of converted operands (3-deep in the CTA-pair kernel).  A (and B^T) are K-major with a 128-byte
 // swizzle; a row-major B is consumed MN-major with the 128-byte swizzle of
 // 32-byte atoms (the only MN-major layout for tf32).  The converter warps put
 // A's hi and lo parts into tensor memory (tcgen05.st; the MMAs take A from
@@ -46,7 +46,7 @@ namespace gptq {
 namespace {
 
 constexpr int TM = 128, TN = 128, TK = 32;
-constexpr int RS = 3;                       // TMA ring: raw A, B tiles
+constexpr int RS = 4;                       // TMA ring: raw A, B tiles
 constexpr int LS = 3;                       // converted operands: B_lo (shared), A hi/lo (TMEM)
 constexpr int TILE_BYTES = 128 * TK * 4;    // 16 KB: 128 rows x 32 fp32
 constexpr int PAIR_BYTES = 2 * TILE_BYTES;  // A and B
