@@ -15,7 +15,11 @@
 // column per barrier (each thread keeps a small tile in registers).  The lower
 // triangle is kept at zero between steps, so the triangular operands can be
 // used as dense ones.  (Tensor-core products and two column steps per barrier
-// were measured slower on the 4096-wide layer, by 0.03 ms and 0.25 ms.)
+// were measured slower on the 4096-wide layer, by 0.03 ms and 0.25 ms.)  The
+// recursion levels, the column factor and the products are separate
+// (non-inlined) functions: the fully inlined kernel was four times the code
+// and stalled on instruction fetch; sharing one copy of each took the 4096
+// layer's factorisation from 2.42 to 2.32 ms.
 
 #include "gptq_internal.h"
 
@@ -49,7 +53,7 @@ __device__ __forceinline__ void cf_barrier() {
 // for 16-byte loads of a B row.  UPPER: only entries with column >= row are
 // written (C is a diagonal block).  Ends with a CTA barrier.
 template <int M, int N, int K, int LDA, int LDB, int LDC, bool TB, bool UPPER>
-__device__ __forceinline__ void smem_gemm(real *C, const real *A, const real *B, real alpha,
+__device__ __noinline__ void smem_gemm(real *C, const real *A, const real *B, real alpha,
                                           real beta) {
   static_assert(K % 4 == 0 && LDA % 4 == 0 && LDB % 4 == 0 && LDC % 4 == 0, "16-byte rows");
   constexpr int RM = (M * N >= 16 * LT) ? 4 : 2;
@@ -141,7 +145,7 @@ __device__ __forceinline__ void smem_gemm(real *C, const real *A, const real *B,
 // costs one CTA barrier.  Returns false (in every thread) on a non-positive
 // pivot.
 template <int N>
-__device__ __forceinline__ bool col_factor(real *S, real *vbuf) {
+__device__ __noinline__ bool col_factor(real *S, real *vbuf) {
   __shared__ int cf_ok;
   if (threadIdx.x >= CF_THREADS) {   // the other warps wait at the closing barrier
     __syncthreads();
@@ -220,7 +224,7 @@ __device__ __forceinline__ bool col_factor(real *S, real *vbuf) {
 // (32, 64, 96 or 128), so the recursion unfolds at compile time and uses no
 // call stack.
 template <int N>
-__device__ __forceinline__ bool node_factor(real *S, real *T, real *vbuf, int off) {
+__device__ __noinline__ bool node_factor(real *S, real *T, real *vbuf, int off) {
   if constexpr (N <= BASE) {
     return col_factor<N>(S + off * LLD + off, vbuf);
   } else {
