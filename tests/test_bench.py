@@ -131,6 +131,20 @@ def test_tensor_peak_follows_the_sampled_clock():
     assert "fallback" in why
 
 
+@pytest.mark.parametrize("name", ["llama7b_q_proj_4096x4096", "opt175b_fc2_12288x49152"])
+def test_recorded_hessian_traffic_is_for_the_current_kernel(name):
+    # The DRAM bytes the bench reports for the Hessian come from an ncu capture of
+    # the kernel as it is now: a change to its sources voids them (reported as
+    # null) until they are captured again, and this test says so.
+    import bench
+    from synth import workload
+    wl = workload(name)
+    t = bench._traffic(wl)
+    assert t is not None, "hessian_tc.cu or gptq_common.cuh changed since the capture"
+    algorithmic = wl.x_bytes + 2 * 4 * wl.d * wl.d
+    assert algorithmic <= t <= 10 * algorithmic
+
+
 def test_cpu_sample_extrapolates_each_phase_by_its_cost():
     # The bounded CPU sample of a layer is scaled phase by phase; on the tiny
     # layer the sample is the whole layer, so nothing is scaled up.
